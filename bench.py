@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark: decode step of a tensor-parallel Llama-2-7B-shaped block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one decode step of one decoder block (dim 4096, 32 heads x 128,
+SwiGLU 11008, KV cache 1024, batch 1) partitioned into n = 4 slices with int8
+(Q8) sync buffers, i.e. every step on the hot path: RMSNorm+Q8, q/k/v slice
+products with RoPE and cache write, split-context attention, W_O partials,
+merge, RMSNorm+Q8, W1/W3+SwiGLU, W2 partials, merge. Inputs are seeded
+synthetic tensors of those shapes; the 404.75 MB of weights per step are
+larger than L2, so no flush is needed between steps.
+
+Rank 0 prints one JSON line. With N > 1 (torchrun) every rank runs its own
+replica on its own GPU (the path does not shard across GPUs), the time is the
+max over ranks and the value is the sum of all ranks' tokens.
+
+Also measured (same run, N=1 fields): the PaLM-shaped FFN (E 18432, F 73728,
+B 512) through tp_ffn_forward in its fused, 1D-64 and 2D-8x8 forms, as TFLOP/s.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s & HBM GB/s per TP-sliced block; FFN TFLOP/s at B=512 (1 B200)"
+STAGES = ["rmsnorm_q8", "qkv_rope", "attention", "wo_partials", "merge_norm", "w13_swiglu",
+          "w2_partials", "merge"]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--graph-steps", type=int, default=100, help="steps captured per CUDA graph")
+    ap.add_argument("--e2e-steps", type=int, default=1000)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=150.0)
+    ap.add_argument("--no-ffn", action="store_true", help="skip the PaLM FFN measurement")
+    ap.add_argument("--ffn-iters", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            sel = None
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if sel:
+            cmd += ["-i", sel]
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def allreduce_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def block_bytes(s):
+    qd, kd = s.n_heads * s.head_dim, s.n_kv_heads * s.head_dim
+    weights = (qd * s.dim + 2 * kd * s.dim + s.dim * qd + 3 * s.ffn_dim * s.dim) * 2
+    kv = 2 * s.batch * s.n_kv_heads * (s.pos + 1) * s.head_dim * 2
+    return weights, kv
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def time_oracle(inp, s, seconds: float, max_steps: int | None = None):
+    import oracle
+
+    cores = len(os.sched_getaffinity(0))
+    oracle.block_forward(inp, s.n_slices, s.sync_quant)  # first call (page-in), untimed
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.block_forward(inp, s.n_slices, s.sync_quant)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_steps is not None and n >= max_steps):
+            break
+    return n * s.batch / el, n, el, cores
+
+
+def run_reference(args):
+    """The oracle (float64 NumPy on the host cores) on the same workload."""
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    s = synth.C2
+    inp = synth.block_inputs(synth.CONFIG_SEED["C2"], s)
+    tps, n, el, cores = time_oracle(inp, s, args.ref_seconds, max_steps=args.steps)
+    w, kv = block_bytes(s)
+    sample = (f"{n} of {args.steps} requested steps of the C2 block (batch 1) through the float64 "
+              f"oracle, bounded to {args.ref_seconds:.0f} s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": world,
+        "steps": n, "warmup": 1, "ms_per_step": el / n * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "C2: Llama-2-7B-shaped decoder block decode, dim 4096, 32x128 heads, "
+                               "SwiGLU 11008, KV 1024, batch 1, n=4 slices, Q8 sync buffers",
+                   "batch": 1, "n_slices": 4, "sync_quant": True, "kv_len": 1024},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "hbm_gbs_equiv": (w + kv) * tps / 1e9,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def make_events(torch, n):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:  # force creation so that the raw handle exists
+        e.record()
+    torch.cuda.synchronize()
+    return evs
+
+
+def bench_block(args, world, rank, local):
+    import torch
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+    from synth.device import DeviceBlock
+
+    s = synth.C2
+    B = s.batch
+    inp = synth.block_inputs(synth.CONFIG_SEED["C2"], s)
+    dev = DeviceBlock(inp)
+    dims = tpb.make_dims(s.dim, s.n_heads, s.n_kv_heads, s.head_dim, s.ffn_dim, s.vocab, B,
+                         s.max_seq, s.norm_eps, s.rope_theta)
+    nbytes = tpb.tp_block_workspace_bytes(dims, s.n_slices, tpb.TP_PART_1D, 1)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    h = tpb.tp_block_create(dims, s.n_slices, tpb.TP_PART_1D, 1, tpb.make_weights(*dev.weights()),
+                            ws, nbytes)
+    x0 = dev.x.clone()
+
+    def fwd():
+        tpb.tp_block_forward(h, dev.x, dev.k_cache, dev.v_cache, dev.pos, B)
+
+    # eager warm-up (module load, attribute setup), then capture
+    for _ in range(3):
+        fwd()
+    torch.cuda.synchronize()
+    K = max(1, args.steps)
+    S = max(1, min(args.graph_steps, K))
+    R = (K + S - 1) // S
+    K = R * S
+    nstage = len(STAGES) + 1
+    evs = [make_events(torch, nstage) for _ in range(S)]
+    arrs = [(ctypes.c_void_p * nstage)(*[e.cuda_event for e in ev]) for ev in evs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(S):
+            tpb.tp_block_set_events(h, arrs[i], nstage)
+            fwd()
+    tpb.tp_block_set_events(h, None, 0)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(1, (args.warmup + S - 1) // S)):
+        g.replay()
+    dev.x.copy_(x0)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = ClockSampler(local)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    start.record(stream)
+    for _ in range(R):
+        g.replay()
+    end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    ms_max = allreduce_max(ms, world)
+    # per-stage device time from the events of the last replay (S steps)
+    stage_ms = [0.0] * len(STAGES)
+    for ev in evs:
+        for i in range(len(STAGES)):
+            stage_ms[i] += ev[i].elapsed_time(ev[i + 1]) / S
+    stage_ms_max = [allreduce_max(v, world) for v in stage_ms]
+    del g
+
+    # end to end through the public API: host buffers, copies inside the timed region
+    xh = torch.empty_like(dev.x, device="cpu").pin_memory()
+    xh.copy_(x0.cpu())
+    posh = torch.from_numpy(inp.pos.copy()).pin_memory()
+    outh = torch.empty_like(xh).pin_memory()
+    E = max(1, args.e2e_steps)
+    for _ in range(3):
+        dev.x.copy_(xh, non_blocking=True)
+        dev.pos.copy_(posh, non_blocking=True)
+        fwd()
+        outh.copy_(dev.x, non_blocking=True)
+        stream.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(E):
+        dev.x.copy_(xh, non_blocking=True)
+        dev.pos.copy_(posh, non_blocking=True)
+        fwd()
+        outh.copy_(dev.x, non_blocking=True)
+        stream.synchronize()
+    e2e_s = allreduce_max(time.perf_counter() - t0, world)
+    tpb.tp_block_destroy(h)
+
+    wbytes, kvbytes = block_bytes(s)
+    step_s = ms_max / 1e3 / K
+    hbm, bf16_tf, bf16_sus, peak_kind = peaks()
+    w13_bytes = 2 * s.ffn_dim * s.dim * 2 + B * s.dim * (1 + 4 / 32) + B * s.ffn_dim * 4
+    w13_s = stage_ms_max[STAGES.index("w13_swiglu")] / 1e3
+    launches_per_step = 9 * 1  # batch <= 4: one launch per stage (attention = chunks + combine)
+    res = {
+        "tokens_per_s": world * B * K / (ms_max / 1e3), "ms_per_step": ms_max / K, "K": K,
+        "block_gbs": (wbytes + kvbytes) / step_s / 1e9, "stage_us": {
+            n: v * 1e3 for n, v in zip(STAGES, stage_ms_max)},
+        "roofline": {"bound": "hbm", "achieved": w13_bytes / w13_s / 1e9, "peak": hbm,
+                     "unit": "GB/s", "frac": w13_bytes / w13_s / 1e9 / hbm, "traffic": None,
+                     "kernel": "k_gemv<1,EPI_SWIGLU> (W1/W3 + SwiGLU)",
+                     "algorithmic_bytes": w13_bytes, "peak_kind": peak_kind},
+        "e2e": {"value": world * B * E / e2e_s, "unit": "tokens/s",
+                "h2d_bytes_per_step": B * s.dim * 4 + B * 4, "d2h_bytes_per_step": B * s.dim * 4},
+        "gpu_launches": launches_per_step * K, "clocks": clk, "inp": inp,
+        "block_roofline_frac": (wbytes + kvbytes) / step_s / 1e9 / hbm,
+    }
+    return res
+
+
+def bench_ffn(args):
+    """PaLM FFN (E 18432, F 73728, B 512, ReLU) through tp_ffn_forward; TFLOP/s per form."""
+    import torch
+
+    import tensor_llama_transformer_b200 as tpb
+
+    B, E, F = 512, 18432, 73728
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1004)
+
+    def randn_bf16(shape, std):
+        out = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        rows = max(1, (1 << 26) // shape[1])
+        for r0 in range(0, shape[0], rows):
+            r1 = min(shape[0], r0 + rows)
+            out[r0:r1] = (torch.randn((r1 - r0, shape[1]), generator=gen, device="cuda") * std).to(
+                torch.bfloat16)
+        return out
+
+    X = randn_bf16((B, E), 1.0)
+    W1 = randn_bf16((F, E), 0.01)
+    W2 = randn_bf16((E, F), 0.01)
+    Y = torch.empty((B, E), dtype=torch.float32, device="cuda")
+    flops = 2.0 * B * 2 * E * F
+    out = {}
+    _, bf16_tf, _, peak_kind = peaks()
+    forms = [("fused", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FUSED),
+             ("1d64_faithful", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FAITHFUL),
+             ("2d8x8_faithful", tpb.TP_PART_2D, 64, 8, 8, tpb.TP_MERGE_FAITHFUL)]
+    for name, part, n, gx, gy, merge in forms:
+        desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, part, n, gx, gy, 0, merge)
+        nb = tpb.tp_ffn_workspace_bytes(desc)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        for _ in range(2):
+            tpb.tp_ffn_forward(desc, X, W1, None, W2, Y, ws, nb)
+        torch.cuda.synchronize()
+        t = []
+        for _ in range(max(1, args.ffn_iters)):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            tpb.tp_ffn_forward(desc, X, W1, None, W2, Y, ws, nb)
+            b.record()
+            b.synchronize()
+            t.append(a.elapsed_time(b))
+        err = int(ws[:4].view(torch.int32).item())
+        ms = statistics.median(t)
+        out[name] = {"ms": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                     "frac": flops / (ms / 1e3) / 1e12 / bf16_tf, "pipeline_error": err}
+        del ws
+        torch.cuda.empty_cache()
+    out["peak_tflops"] = bf16_tf
+    out["peak_kind"] = peak_kind
+    out["config"] = "E=18432 F=73728 B=512 ReLU, bf16 weights/activations, fp32 accumulate"
+    return out
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    world, rank, local = dist_setup()
+    res = bench_block(args, world, rank, local)
+    ffn = None if args.no_ffn else bench_ffn(args)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import synth
+
+        tps, n, el, cores = time_oracle(res["inp"], synth.C2, args.cpu_seconds)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} full C2 block decode steps (batch 1) in {el:.1f} s"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": res["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+            "steps": res["K"], "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "dtype_detail": "bf16 weights, fp32 activations and accumulation, int8 Q8 sync buffers",
+            "data": "synthetic",
+            "config": {"workload": "C2: Llama-2-7B-shaped decoder block decode, dim 4096, "
+                                   "32x128 heads, SwiGLU 11008, KV 1024, batch 1, n=4 slices, "
+                                   "Q8 sync buffers",
+                       "batch": 1, "n_slices": 4, "sync_quant": True, "kv_len": 1024,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (404.75 MB of weights per step), no flush"},
+            "hbm_gbs": res["block_gbs"], "block_roofline_frac": res["block_roofline_frac"],
+            "stage_us": res["stage_us"], "roofline": res["roofline"], "cpu_baseline": cpu,
+            "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+            "ffn_b512": ffn,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

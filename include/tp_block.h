@@ -1,0 +1,213 @@
+/*
+ * tp_block.h — C ABI of the tensor-parallel Llama decoder block for B200 (sm_100a).
+ *
+ * One decoder block's decode step, partitioned tensor-parallel into n weight
+ * slices that all run as partitions of the same launches on one GPU, plus the
+ * 1D / 2D partitioned feed-forward layer and the full multi-layer decode step.
+ *
+ * Sources for what is computed (pages on the subject, by title and part):
+ *   - distributed-llama issue #29, "[Feature Suggest] Tensor Parallellism for
+ *     Accelerating LLM": the buildLlama2Arch task list (per-layer order
+ *     RmsAttNorm, QuantizeRmsAtt, SyncRmsAtt, Qkv, MultiheadAtt, AttOutput,
+ *     QuantizeAtt, SyncAtt, DequantizeAtt, MergeAtt, RmfFfn(Norm), QuantizeRmfFfn,
+ *     SyncRmfFfn, Ffn, Ffn2, QuantizeFfn2, SyncFfn2, DequantizeFfn2, MergeFfn2,
+ *     NextBlock; then RmsFinal(Norm), Logits, MergeLogits).
+ *   - aiterms.tw "Tensor Parallelism" glossary: column split, row split, 2D split
+ *     ("core concept") and the FFN procedure with one all-reduce ("how it works").
+ *   - CS349E lecture 4 "03_pope_partitioning.py" (Pope et al.), demo1_1d_vs_2d:
+ *     1D (split F) versus 2D weight-stationary (split E and F) FFN partitions.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named as a tensor is a DEVICE pointer unless stated.
+ *     The caller owns all memory (weights, caches, activations, workspace). The
+ *     library never allocates device memory and never synchronises the device;
+ *     work is enqueued on `stream` (NULL = the legacy default stream).
+ *   - Weights are bf16, stored [out, in] row-major (a PyTorch Linear). A column
+ *     split is a contiguous row range of that storage, a row split a contiguous
+ *     column range; slices are addressed in place, no re-packing is required.
+ *   - Activations and the residual are float32 row-major [B, features].
+ *   - KV caches are bf16 [max_batch, n_kv_heads, max_seq, head_dim].
+ *   - Slice s of n owns query heads [s*H/n, (s+1)*H/n) and kv heads
+ *     [s*Hkv/n, (s+1)*Hkv/n); query head h reads kv head h / (H/Hkv).
+ *   - Pointers must be 16-byte aligned. Return value: TP_OK or a tp_status code;
+ *     nothing is enqueued when an argument check fails. Faults of kernels already
+ *     enqueued surface as CUDA errors at the caller's next synchronisation.
+ */
+#ifndef TP_BLOCK_H_
+#define TP_BLOCK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TP_API __attribute__((visibility("default")))
+#else
+#define TP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tp_stream; /* a cudaStream_t */
+
+enum tp_status {
+  TP_OK = 0,
+  TP_EINVAL = 1,      /* a size or flag is out of range or does not divide */
+  TP_EWORKSPACE = 2,  /* workspace pointer NULL or smaller than required */
+  TP_EARCH = 3,       /* current device is not compute capability 10.0 (B200) */
+  TP_ECUDA = 4,       /* a CUDA runtime call or kernel launch failed */
+  TP_ENOTSUP = 5,     /* a combination this build does not implement */
+  TP_EALIGN = 6       /* a pointer is not 16-byte aligned */
+};
+
+enum { TP_PART_1D = 1, TP_PART_2D = 2 };
+enum { TP_ACT_RELU = 0, TP_ACT_SWIGLU = 1 };
+enum { TP_F32 = 0, TP_BF16 = 1 };
+enum { TP_MERGE_FAITHFUL = 0, TP_MERGE_FUSED = 1 };
+
+/* Model dimensions (the distributed-llama TransformerSpec, reduced to what one
+ * block needs). Requirements checked at create: dim % 32 == 0, head_dim == 128,
+ * n_heads % n_kv_heads == 0, H % n == 0, Hkv % n == 0, ffn_dim % (32*n) == 0,
+ * 1 <= max_batch <= 64, 1 <= max_seq. */
+typedef struct {
+  int32_t dim, n_heads, n_kv_heads, head_dim, ffn_dim, vocab, max_batch, max_seq;
+  float norm_eps, rope_theta;
+} tp_dims;
+
+/* Borrowed device pointers to one block's parameters (the handle keeps them). */
+typedef struct {
+  const float* attn_norm; /* [dim] float32 RMSNorm gain before attention      */
+  const void* wq;         /* bf16 [H*hd, dim]   column split by q-head ranges */
+  const void* wk;         /* bf16 [Hkv*hd, dim] column split by kv-head ranges */
+  const void* wv;         /* bf16 [Hkv*hd, dim]                               */
+  const void* wo;         /* bf16 [dim, H*hd]   row split: slice s reads columns of its heads */
+  const float* ffn_norm;  /* [dim] float32 RMSNorm gain before the FFN        */
+  const void* w1;         /* bf16 [F, dim]      column split (rows F_s)       */
+  const void* w3;         /* bf16 [F, dim]      column split (rows F_s)       */
+  const void* w2;         /* bf16 [dim, F]      row split (columns F_s)       */
+} tp_block_weights;
+
+typedef struct tp_block tp_block;
+
+/* Bytes of device workspace a block needs for dims->max_batch rows.
+ * partition: TP_PART_1D or TP_PART_2D (2D applies to the FFN: a gx x gy grid, gx
+ * the largest divisor of n with gx*gx <= n splits dim, gy = n/gx splits ffn_dim;
+ * attention stays split by heads). sync_quant: 0 = float32 sync buffers,
+ * 1 = int8 blocks of 32 with one float32 scale (d = amax/127, codes = x/d rounded
+ * half away from zero, clamped to +-127; an all-zero block has d = 0). */
+TP_API int tp_block_workspace_bytes(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                             size_t* out_bytes);
+
+/* Validate and build a block handle (host memory only; no device work).
+ * workspace: device buffer of at least tp_block_workspace_bytes, 256-byte
+ * aligned, owned by the caller, used exclusively by this handle's forwards.
+ * Errors: TP_EINVAL, TP_EALIGN, TP_EWORKSPACE, TP_EARCH, TP_ECUDA. */
+TP_API int tp_block_create(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                    const tp_block_weights* w, void* workspace, size_t ws_bytes, tp_block** out);
+
+/* One decode step of the block for `batch` rows (1 <= batch <= max_batch):
+ *   x       float32 [batch, dim], read as the residual input and overwritten with
+ *           the block output x + attn + ffn.
+ *   k_cache, v_cache  bf16 [max_batch, Hkv, max_seq, hd]; positions < pos[b] are
+ *           read, position pos[b] is written with the new rotated k and v.
+ *   pos     device int32 [batch], 0 <= pos[b] < max_seq (not checked on device:
+ *           an out-of-range pos is a caller error).
+ * Steps, in the distributed-llama root order: RMSNorm (+Q8) -> q/k/v slice
+ * products with RoPE and cache write -> attention per head slice (split over
+ * the context, then combined) -> W_O row-split partials [n, batch, dim] ->
+ * merge x += sum_s deq(partial_s) in slice order -> RMSNorm (+Q8) -> W1/W3 slice
+ * products with SwiGLU -> W2 row-split partials -> merge. */
+TP_API int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, const int32_t* pos,
+                     int batch, tp_stream stream);
+
+/* Offsets (bytes from the workspace base) and sizes of intermediate buffers,
+ * for inspection by tests after a forward. which: 0 xnorm int8 codes [B,dim],
+ * 1 xnorm scales float32 [B,dim/32], 2 xnorm float32 [B,dim], 3 q (rotated)
+ * float32 [B,H*hd], 4 attention output float32 [B,H*hd], 5 partials float32
+ * [n,B,dim], 6 SwiGLU output h float32 [B,F]. */
+TP_API int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* bytes);
+
+TP_API void tp_block_destroy(tp_block* blk);
+
+/* Per-stage timing hook. events: host array of n cudaEvent_t handles created by
+ * the caller (timing enabled), or NULL to switch the hook off. While set, each
+ * tp_block_forward records events[i] on `stream` just before stage i and
+ * events[TP_BLOCK_STAGES] after the last stage (n must be TP_BLOCK_STAGES + 1).
+ * Stages: 0 RMSNorm(+Q8), 1 q/k/v products + RoPE + cache write, 2 attention
+ * (chunks + combine), 3 W_O partials, 4 merge + FFN RMSNorm, 5 W1/W3 + SwiGLU
+ * (2D: stage-1 partials + merge), 6 W2 partials, 7 final merge. The handle
+ * borrows the array; recording works inside stream capture. */
+#define TP_BLOCK_STAGES 8
+TP_API int tp_block_set_events(tp_block* blk, void* const* events, int n);
+
+/* ------------------------------------------------------------------------- */
+/* Partitioned feed-forward layer  Y = act(X W1^T [, X W3^T]) W2^T.            */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+  int32_t batch;      /* tokens B */
+  int32_t E, F;       /* model dim and FFN dim */
+  int32_t dtype;      /* TP_F32 (X, W float32) or TP_BF16 (X, W bf16) */
+  int32_t act;        /* TP_ACT_RELU (two matrices) or TP_ACT_SWIGLU (W1, W3, W2) */
+  int32_t partition;  /* TP_PART_1D (n = n_slices over F) or TP_PART_2D (grid_x over E, grid_y over F) */
+  int32_t n_slices, grid_x, grid_y;
+  int32_t sync_quant; /* 1 = Q8 round trip of every partial before its merge */
+  int32_t merge;      /* TP_MERGE_FAITHFUL: partials materialised and summed in slice order;
+                         TP_MERGE_FUSED: partials accumulated in slice order inside the
+                         contraction (bf16 only, sync_quant must be 0) */
+} tp_ffn_desc;
+
+/* Workspace bytes for tp_ffn_forward with this descriptor. */
+TP_API int tp_ffn_workspace_bytes(const tp_ffn_desc* d, size_t* out_bytes);
+
+/* X [B,E], W1 [F,E], W3 [F,E] (NULL unless SwiGLU), W2 [E,F] in d->dtype;
+ * Y float32 [B,E] written. 1D: H_s = act(X W1_s^T) per F-slice (column split),
+ * P_s = H_s W2_s^T (row split), Y = sum_s P_s. 2D: stage 1 sums over the E-slices,
+ * stage 2 over the F-slices. Requirements: E % (32*grid_x) == 0 and F % (32*n)
+ * == 0 (1D) or F % (32*grid_y) == 0 (2D); bf16 needs E % 64 == 0, F % 64 == 0 and
+ * the per-slice contraction length a multiple of 64. */
+TP_API int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const void* W3,
+                   const void* W2, float* Y, void* workspace, size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------------- */
+/* Full decode step: embedding gather, n_layers blocks, final RMSNorm, logits. */
+/* ------------------------------------------------------------------------- */
+typedef struct tp_model tp_model;
+
+TP_API int tp_model_workspace_bytes(const tp_dims* dims, int n_layers, int n_slices, int partition,
+                             int sync_quant, size_t* out_bytes);
+
+/* layers: host array of n_layers tp_block_weights (device pointers inside).
+ * embed bf16 [vocab, dim]; final_norm float32 [dim]; wcls bf16 [vocab, dim]
+ * (the logits are column-split by vocab ranges: each slice writes its own
+ * range of the output, so the merge is a concatenation). */
+TP_API int tp_model_create(const tp_dims* dims, int n_layers, int n_slices, int partition, int sync_quant,
+                    const tp_block_weights* layers, const void* embed, const float* final_norm,
+                    const void* wcls, void* workspace, size_t ws_bytes, tp_model** out);
+
+/* tokens device int32 [batch] in [0, vocab); caches bf16
+ * [n_layers, max_batch, Hkv, max_seq, hd]; logits float32 [batch, vocab] written. */
+TP_API int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
+                     const int32_t* pos, int batch, float* logits, tp_stream stream);
+
+TP_API void tp_model_destroy(tp_model* m);
+
+/* ------------------------------------------------------------------------- */
+/* Standalone Q8 codec of the sync buffers (same arithmetic as inside the block). */
+/* ------------------------------------------------------------------------- */
+/* x float32 [n] -> q int8 [n], d float32 [n/32]; n % 32 == 0. */
+TP_API int tp_quantize_q8(const float* x, int8_t* q, float* d, int64_t n, tp_stream stream);
+/* q int8 [n], d float32 [n/32] -> x float32 [n], x_i = q_i * d_block. */
+TP_API int tp_dequantize_q8(const int8_t* q, const float* d, float* x, int64_t n, tp_stream stream);
+
+/* Human-readable name of a status code (static storage). */
+TP_API const char* tp_status_string(int status);
+
+/* Library build identifier (static storage), e.g. "tp_block sm_100a". */
+TP_API const char* tp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_BLOCK_H_ */

@@ -303,7 +303,8 @@ def ffn_forward(X, W1, W2, act: str = "relu", W3=None, partition: int = 1, n_sli
 # decoder block
 # ---------------------------------------------------------------------------
 
-def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid=None):
+def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid=None,
+                  trace: dict | None = None):
     """One decode step of one decoder block, partitioned into ``n_slices`` slices.
 
     Follows the [DL] root-node task order for one layer:
@@ -320,6 +321,10 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
     With ``partition == 2`` the FFN follows ``ffn_forward``'s 2D grid; attention
     stays split by heads. Slice s owns q heads ``[s H/n, (s+1) H/n)`` and kv heads
     ``[s Hkv/n, (s+1) Hkv/n)``.
+
+    ``trace`` (optional dict) receives the intermediates ``xin``, ``q`` (rotated),
+    ``att`` (all heads), ``x1``, ``xin2`` and, for 1D, ``h``; recording them does
+    not change the arithmetic.
 
     ``inp`` is a ``synth.BlockInputs``. Returns ``(x_out float64 [B, dim],
     k_row uint16 [B, Hkv, hd], v_row uint16 [B, Hkv, hd])``: the new block
@@ -364,16 +369,22 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
 
     # a4-a6
     x1 = x.copy()
+    att_all = np.zeros((B, H * hd))
     for s in range(n):
         heads = range(s * (H // n), (s + 1) * (H // n))
         att_s = attention_decode(q_rot, kc, vc, pos, heads, H, Hkv, hd)
         cols = slice_range(H * hd, n, s)
+        att_all[:, cols] = att_s
         p_s = att_s @ wo[:, cols].T
         x1 = x1 + sync_buffer(p_s, sync_quant)
 
     # a7-a10
     xin2 = sync_buffer(rmsnorm(x1, inp.ffn_norm, s_.norm_eps), sync_quant)
     w1, w3, w2 = bf16_to_f64(inp.w1), bf16_to_f64(inp.w3), bf16_to_f64(inp.w2)
+    if trace is not None:
+        trace.update(xin=xin, q=q_rot, att=att_all, x1=x1, xin2=xin2)
+        if partition == 1:
+            trace["h"] = swiglu(xin2 @ w1.T, xin2 @ w3.T)
     x2 = ffn_forward(xin2, w1, w2, act="swiglu", W3=w3, partition=partition, n_slices=n,
                      grid=grid, quant=sync_quant, residual=x1)
     return x2, k_new, v_new

@@ -25,6 +25,7 @@ the device fill reproduces these bytes exactly.
 """
 from __future__ import annotations
 
+import os
 import zlib
 from dataclasses import dataclass, field
 
@@ -91,7 +92,22 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 # generators
 # ---------------------------------------------------------------------------
 
-_CHUNK = 1 << 24
+_CHUNK = 1 << 22
+
+
+def _parallel_fill(out: np.ndarray, fill, n: int):
+    """Run ``fill(offset, count)`` over chunks of ``out`` on a thread pool."""
+    spans = [(o, min(_CHUNK, n - o)) for o in range(0, n, _CHUNK)]
+    if len(spans) <= 1:
+        for o, c in spans:
+            fill(o, c)
+        return out
+    import concurrent.futures as cf
+
+    workers = min(len(spans), max(1, len(os.sched_getaffinity(0))))
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(lambda oc: fill(*oc), spans))
+    return out
 
 
 def normal_f32(seed: int, name: str, shape, std: float = 1.0, start: int = 0) -> np.ndarray:
@@ -100,20 +116,27 @@ def normal_f32(seed: int, name: str, shape, std: float = 1.0, start: int = 0) ->
     key = stream_key(seed, name)
     out = np.empty(n, dtype=np.float32)
     s = np.float32(std)
-    for o in range(0, n, _CHUNK):
-        c = min(_CHUNK, n - o)
+
+    def fill(o, c):
         h = raw64(key, start + o, c)
         out[o:o + c] = NORMAL_TABLE[(h >> np.uint64(48)).astype(np.int64)] * s
+
+    _parallel_fill(out, fill, n)
     return out.reshape(shape)
 
 
 def normal_bf16(seed: int, name: str, shape, std: float = 1.0, start: int = 0) -> np.ndarray:
     """bf16 bit patterns (uint16) of N(0, std) samples for tensor ``name``."""
     n = int(np.prod(shape))
+    key = stream_key(seed, name)
     out = np.empty(n, dtype=np.uint16)
-    for o in range(0, n, _CHUNK):
-        c = min(_CHUNK, n - o)
-        out[o:o + c] = f32_to_bf16_bits(normal_f32(seed, name, (c,), std, start + o))
+    s = np.float32(std)
+
+    def fill(o, c):
+        h = raw64(key, start + o, c)
+        out[o:o + c] = f32_to_bf16_bits(NORMAL_TABLE[(h >> np.uint64(48)).astype(np.int64)] * s)
+
+    _parallel_fill(out, fill, n)
     return out.reshape(shape)
 
 

@@ -1,0 +1,617 @@
+// Host side of the C ABI declared in include/tp_block.h: argument checks,
+// workspace layout and the launch sequence of a block, a model and an FFN.
+#include <mutex>
+#include <new>
+
+#include "ffn.cuh"
+#include "kernels.cuh"
+
+namespace tp {
+
+// ------------------------------------------------------------------ device info
+namespace {
+constexpr int kMaxDev = 64;
+int g_arch[kMaxDev];  // 0 unknown, 1 sm_100, 2 other
+int g_sms[kMaxDev];
+}  // namespace
+
+int device_check() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return TP_ECUDA;
+  if (g_arch[dev] == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return TP_ECUDA;
+    g_sms[dev] = sms;
+    g_arch[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return g_arch[dev] == 1 ? TP_OK : TP_EARCH;
+}
+
+int set_smem_once(const void* kernel, int bytes) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    int bytes;
+  };
+  static Entry tab[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TP_ECUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (tab[i].fn == kernel && tab[i].dev == dev && tab[i].bytes >= bytes) return TP_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return TP_ECUDA;
+  for (int i = 0; i < used; ++i)
+    if (tab[i].fn == kernel && tab[i].dev == dev) {
+      tab[i].bytes = bytes;
+      return TP_OK;
+    }
+  if (used < 256) tab[used++] = Entry{kernel, dev, bytes};
+  return TP_OK;
+}
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDev || g_sms[dev] == 0) device_check();
+  return (dev >= 0 && dev < kMaxDev && g_sms[dev] > 0) ? g_sms[dev] : 148;
+}
+
+namespace {
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// ------------------------------------------------------------------ block layout
+enum Buf {
+  BUF_XQ = 0, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H, BUF_ERR, BUF_PO, BUF_PML,
+  BUF_PA, BUF_PB, BUF_COUNT
+};
+
+struct Layout {
+  size_t off[BUF_COUNT];
+  size_t size[BUF_COUNT];
+  size_t total;
+};
+
+struct Cfg {
+  tp_dims d;
+  int n, partition, quant, gx, gy, nchunk;
+};
+
+void grid2d(int n, int* gx, int* gy) {
+  int best = 1;
+  for (int v = 1; v * v <= n; ++v)
+    if (n % v == 0) best = v;
+  *gx = best;
+  *gy = n / best;
+}
+
+int check_cfg(const tp_dims* d, int n, int partition, int quant, Cfg* c) {
+  if (!d || !c) return TP_EINVAL;
+  if (n < 1 || (partition != TP_PART_1D && partition != TP_PART_2D) || (quant != 0 && quant != 1))
+    return TP_EINVAL;
+  if (d->dim <= 0 || d->dim % 128 != 0) return TP_EINVAL;
+  if (d->head_dim != kHeadDim) return TP_ENOTSUP;
+  if (d->n_heads <= 0 || d->n_kv_heads <= 0 || d->n_heads % d->n_kv_heads != 0) return TP_EINVAL;
+  const int G = d->n_heads / d->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TP_ENOTSUP;
+  if (d->n_heads % n != 0 || d->n_kv_heads % n != 0) return TP_EINVAL;
+  if (d->ffn_dim <= 0 || d->ffn_dim % (32 * n) != 0) return TP_EINVAL;
+  if (d->max_batch < 1 || d->max_batch > 64 || d->max_seq < 1) return TP_EINVAL;
+  if (!(d->norm_eps >= 0.f) || !(d->rope_theta > 0.f)) return TP_EINVAL;
+  c->d = *d;
+  c->n = n;
+  c->partition = partition;
+  c->quant = quant;
+  if (partition == TP_PART_2D) {
+    grid2d(n, &c->gx, &c->gy);
+    if (d->dim % (32 * c->gx) != 0 || d->ffn_dim % (32 * c->gy) != 0) return TP_EINVAL;
+  } else {
+    c->gx = 1;
+    c->gy = n;
+  }
+  c->nchunk = (d->max_seq + kAttnChunk - 1) / kAttnChunk;
+  return TP_OK;
+}
+
+Layout block_layout(const Cfg& c) {
+  const size_t B = c.d.max_batch, D = c.d.dim, F = c.d.ffn_dim;
+  const size_t QD = (size_t)c.d.n_heads * c.d.head_dim;
+  Layout L{};
+  L.size[BUF_XQ] = B * D;
+  L.size[BUF_XD] = B * (D / 32) * 4;
+  L.size[BUF_XN] = B * D * 4;
+  L.size[BUF_Q] = B * QD * 4;
+  L.size[BUF_ATT] = B * QD * 4;
+  L.size[BUF_PART] = (size_t)c.n * B * D * 4;
+  L.size[BUF_H] = B * F * 4;
+  L.size[BUF_ERR] = 16;
+  L.size[BUF_PO] = B * c.d.n_heads * (size_t)c.nchunk * c.d.head_dim * 4;
+  L.size[BUF_PML] = B * c.d.n_heads * (size_t)c.nchunk * 2 * 4;
+  const size_t pa = c.partition == TP_PART_2D ? (size_t)c.gx * B * F * 4 : 0;
+  L.size[BUF_PA] = pa;
+  L.size[BUF_PB] = pa;
+  size_t o = 0;
+  for (int i = 0; i < BUF_COUNT; ++i) {
+    L.off[i] = o;
+    o += align256(L.size[i]);
+  }
+  L.total = o;
+  return L;
+}
+
+int ctas_for(int nseg, int pairs_per_seg) {
+  int target = num_sms() * 3;
+  int per = target / nseg;
+  if (per < 1) per = 1;
+  if (per > pairs_per_seg) per = pairs_per_seg;
+  return per;
+}
+
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+struct tp_block {
+  Cfg c;
+  Layout L;
+  tp_block_weights w;
+  uint8_t* ws;
+  size_t ws_bytes;
+  void* const* events;  // optional per-stage timing events (borrowed)
+};
+
+struct tp_model {
+  tp_dims d;
+  int n_layers;
+  tp_block* blocks;  // n_layers handles sharing one block workspace
+  const void* embed;
+  const float* final_norm;
+  const void* wcls;
+  float* x;    // residual [max_batch, dim]
+  float* xnf;  // final normed rows [max_batch, dim]
+};
+
+namespace tp_api {
+
+template <typename T>
+T* at(const tp_block* b, int buf) {
+  return reinterpret_cast<T*>(b->ws + b->L.off[buf]);
+}
+
+NormOut norm_out_for(const tp_block* b, const float* gain) {
+  NormOut no{};
+  no.gain = gain;
+  no.eps = b->c.d.norm_eps;
+  no.quant = b->c.quant;
+  if (b->c.quant) {
+    no.xq = at<int8_t>(b, BUF_XQ);
+    no.xd = at<float>(b, BUF_XD);
+  } else {
+    no.xn = at<float>(b, BUF_XN);
+  }
+  return no;
+}
+
+// One block forward. `first` launches the attention RMSNorm (otherwise the
+// caller's previous merge already wrote it); `tail` is the RMSNorm fused
+// after the final merge (gain == nullptr: none).
+int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
+  if (!blk->events) return TP_OK;
+  return cudaEventRecord(static_cast<cudaEvent_t>(blk->events[stage]), s) == cudaSuccess ? TP_OK
+                                                                                        : TP_ECUDA;
+}
+
+int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
+                       cudaStream_t s, bool first, const NormOut& tail) {
+  const Cfg& c = blk->c;
+  const tp_dims& d = c.d;
+  const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
+  const int QD = H * hd;
+  int rc;
+  const bool q = c.quant != 0;
+  const float* xn = at<float>(blk, BUF_XN);
+  const int8_t* xq = at<int8_t>(blk, BUF_XQ);
+  const float* xd = at<float>(blk, BUF_XD);
+  float* part = at<float>(blk, BUF_PART);
+  float* hbuf = at<float>(blk, BUF_H);
+
+  // a1-a2: RMSNorm (+Q8) into the buffer all slices read
+  if ((rc = stage_mark(blk, 0, s))) return rc;
+  if (first) {
+    rc = launch_rmsnorm(x, batch, D, norm_out_for(blk, blk->w.attn_norm), s);
+    if (rc) return rc;
+  }
+  // a3-a4: q/k/v slice products with RoPE and the cache write
+  if ((rc = stage_mark(blk, 1, s))) return rc;
+  {
+    GemvArgs a{};
+    a.w[0] = static_cast<const uint16_t*>(blk->w.wq);
+    a.w[1] = static_cast<const uint16_t*>(blk->w.wk);
+    a.w[2] = static_cast<const uint16_t*>(blk->w.wv);
+    a.rows[0] = QD;
+    a.rows[1] = Hkv * hd;
+    a.rows[2] = Hkv * hd;
+    a.ldw = D;
+    a.Ks = D;
+    a.nseg = 1;
+    a.x = q ? nullptr : xn;
+    a.xq = q ? xq : nullptr;
+    a.xd = q ? xd : nullptr;
+    a.ldx = D;
+    a.b0 = 0;
+    a.nb = batch;
+    a.qout = at<float>(blk, BUF_Q);
+    a.kc = static_cast<uint16_t*>(kc);
+    a.vc = static_cast<uint16_t*>(vc);
+    a.pos = pos;
+    a.n_heads = H;
+    a.n_kv_heads = Hkv;
+    a.max_seq = d.max_seq;
+    a.theta = d.rope_theta;
+    a.ctas_per_seg = ctas_for(1, (QD + 2 * Hkv * hd) / 2);
+    rc = launch_gemv(a, EPI_QKV, s);
+    if (rc) return rc;
+  }
+  // a4: attention per head slice
+  if ((rc = stage_mark(blk, 2, s))) return rc;
+  {
+    AttnArgs a{};
+    a.q = at<float>(blk, BUF_Q);
+    a.kc = static_cast<const uint16_t*>(kc);
+    a.vc = static_cast<const uint16_t*>(vc);
+    a.pos = pos;
+    a.B = batch;
+    a.H = H;
+    a.Hkv = Hkv;
+    a.max_seq = d.max_seq;
+    a.nchunk = c.nchunk;
+    a.part_o = at<float>(blk, BUF_PO);
+    a.part_ml = at<float>(blk, BUF_PML);
+    a.att = at<float>(blk, BUF_ATT);
+    a.err = at<int>(blk, BUF_ERR);
+    rc = launch_attention(a, s);
+    if (rc) return rc;
+  }
+  // a5: W_O row-split partials, one per slice
+  if ((rc = stage_mark(blk, 3, s))) return rc;
+  {
+    GemvArgs a{};
+    a.w[0] = static_cast<const uint16_t*>(blk->w.wo);
+    a.rows[0] = D;
+    a.ldw = QD;
+    a.Ks = QD / c.n;
+    a.nseg = c.n;
+    a.x = at<float>(blk, BUF_ATT);
+    a.ldx = QD;
+    a.nb = batch;
+    a.out = part;
+    a.out_seg = (int64_t)batch * D;
+    a.ldo = D;
+    a.ctas_per_seg = ctas_for(c.n, D / 2);
+    rc = launch_gemv(a, EPI_PLAIN, s);
+    if (rc) return rc;
+  }
+  // a6-a7: merge (dequantise + slice-order sum + residual) and the FFN RMSNorm
+  if ((rc = stage_mark(blk, 4, s))) return rc;
+  rc = launch_merge(x, part, c.n, batch, D, c.quant, norm_out_for(blk, blk->w.ffn_norm), s);
+  if (rc) return rc;
+  // a8: W1/W3 slice products and SwiGLU
+  if ((rc = stage_mark(blk, 5, s))) return rc;
+  if (c.partition == TP_PART_1D) {
+    GemvArgs a{};
+    a.w[0] = static_cast<const uint16_t*>(blk->w.w1);
+    a.w[1] = static_cast<const uint16_t*>(blk->w.w3);
+    a.rows[0] = F;
+    a.ldw = D;
+    a.Ks = D;
+    a.nseg = 1;
+    a.x = q ? nullptr : xn;
+    a.xq = q ? xq : nullptr;
+    a.xd = q ? xd : nullptr;
+    a.ldx = D;
+    a.nb = batch;
+    a.out = hbuf;
+    a.out_seg = 0;
+    a.ldo = F;
+    a.ctas_per_seg = ctas_for(1, F);
+    rc = launch_gemv(a, EPI_SWIGLU, s);
+    if (rc) return rc;
+  } else {
+    // 2D stage 1: partial sums over the gx dim-slices for W1 and W3, merged with SwiGLU
+    float* pa = at<float>(blk, BUF_PA);
+    float* pb = at<float>(blk, BUF_PB);
+    for (int m = 0; m < 2; ++m) {
+      GemvArgs a{};
+      a.w[0] = static_cast<const uint16_t*>(m == 0 ? blk->w.w1 : blk->w.w3);
+      a.rows[0] = F;
+      a.ldw = D;
+      a.Ks = D / c.gx;
+      a.nseg = c.gx;
+      a.x = q ? nullptr : xn;
+      a.xq = q ? xq : nullptr;
+      a.xd = q ? xd : nullptr;
+      a.ldx = D;
+      a.nb = batch;
+      a.out = m == 0 ? pa : pb;
+      a.out_seg = (int64_t)batch * F;
+      a.ldo = F;
+      a.ctas_per_seg = ctas_for(c.gx, F / 2);
+      rc = launch_gemv(a, EPI_PLAIN, s);
+      if (rc) return rc;
+    }
+    FfnMergeArgs m{};
+    m.P1 = pa;
+    m.P3 = pb;
+    m.seg_stride = (int64_t)batch * F;
+    m.nseg = c.gx;
+    m.M = batch;
+    m.N = F;
+    m.quant = c.quant;
+    m.act = ACT_SWIGLU;
+    m.out_f32 = hbuf;
+    rc = launch_ffn_merge(m, s);
+    if (rc) return rc;
+  }
+  // a9: W2 row-split partials
+  if ((rc = stage_mark(blk, 6, s))) return rc;
+  const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
+  {
+    GemvArgs a{};
+    a.w[0] = static_cast<const uint16_t*>(blk->w.w2);
+    a.rows[0] = D;
+    a.ldw = F;
+    a.Ks = F / nseg2;
+    a.nseg = nseg2;
+    a.x = hbuf;
+    a.ldx = F;
+    a.nb = batch;
+    a.out = part;
+    a.out_seg = (int64_t)batch * D;
+    a.ldo = D;
+    a.ctas_per_seg = ctas_for(nseg2, D / 2);
+    rc = launch_gemv(a, EPI_PLAIN, s);
+    if (rc) return rc;
+  }
+  // a10: merge (+ the next sublayer's norm when fused by the caller)
+  if ((rc = stage_mark(blk, 7, s))) return rc;
+  rc = launch_merge(x, part, nseg2, batch, D, c.quant, tail, s);
+  if (rc) return rc;
+  return stage_mark(blk, TP_BLOCK_STAGES, s);
+}
+
+__global__ void k_embed(const uint16_t* __restrict__ emb, const int32_t* __restrict__ tok, int dim,
+                        float* __restrict__ x) {
+  const int b = blockIdx.x;
+  const uint16_t* row = emb + (size_t)tok[b] * dim;
+  for (int i = threadIdx.x; i < dim; i += blockDim.x)
+    x[(size_t)b * dim + i] = __uint_as_float(((uint32_t)row[i]) << 16);
+}
+
+bool weights_aligned(const tp_block_weights* w) {
+  return aligned16(w->attn_norm) && aligned16(w->wq) && aligned16(w->wk) && aligned16(w->wv) &&
+         aligned16(w->wo) && aligned16(w->ffn_norm) && aligned16(w->w1) && aligned16(w->w3) &&
+         aligned16(w->w2);
+}
+
+bool weights_present(const tp_block_weights* w) {
+  return w && w->attn_norm && w->wq && w->wk && w->wv && w->wo && w->ffn_norm && w->w1 && w->w3 &&
+         w->w2;
+}
+
+}  // namespace tp_api
+
+using namespace tp_api;
+
+extern "C" {
+
+const char* tp_status_string(int st) {
+  switch (st) {
+    case TP_OK: return "ok";
+    case TP_EINVAL: return "invalid argument";
+    case TP_EWORKSPACE: return "workspace missing or too small";
+    case TP_EARCH: return "device is not sm_100 (B200)";
+    case TP_ECUDA: return "CUDA runtime error";
+    case TP_ENOTSUP: return "not supported by this build";
+    case TP_EALIGN: return "pointer not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+const char* tp_version(void) { return "tp_block sm_100a 1"; }
+
+int tp_block_workspace_bytes(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                             size_t* out_bytes) {
+  Cfg c;
+  int rc = check_cfg(dims, n_slices, partition, sync_quant, &c);
+  if (rc) return rc;
+  if (!out_bytes) return TP_EINVAL;
+  *out_bytes = block_layout(c).total;
+  return TP_OK;
+}
+
+int tp_block_create(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                    const tp_block_weights* w, void* workspace, size_t ws_bytes, tp_block** out) {
+  if (!out) return TP_EINVAL;
+  *out = nullptr;
+  Cfg c;
+  int rc = check_cfg(dims, n_slices, partition, sync_quant, &c);
+  if (rc) return rc;
+  if (!weights_present(w)) return TP_EINVAL;
+  if (!weights_aligned(w)) return TP_EALIGN;
+  Layout L = block_layout(c);
+  if (!workspace || ws_bytes < L.total) return TP_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return TP_EALIGN;
+  rc = device_check();
+  if (rc) return rc;
+  tp_block* b = new (std::nothrow) tp_block;
+  if (!b) return TP_EINVAL;
+  b->c = c;
+  b->L = L;
+  b->w = *w;
+  b->ws = static_cast<uint8_t*>(workspace);
+  b->ws_bytes = ws_bytes;
+  b->events = nullptr;
+  *out = b;
+  return TP_OK;
+}
+
+int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, const int32_t* pos,
+                     int batch, tp_stream stream) {
+  if (!blk || !x || !k_cache || !v_cache || !pos) return TP_EINVAL;
+  if (batch < 1 || batch > blk->c.d.max_batch) return TP_EINVAL;
+  if (!aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache)) return TP_EALIGN;
+  NormOut none{};
+  return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream, true, none);
+}
+
+int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* bytes) {
+  if (!blk || which < 0 || which >= BUF_COUNT) return TP_EINVAL;
+  if (offset) *offset = blk->L.off[which];
+  if (bytes) *bytes = blk->L.size[which];
+  return TP_OK;
+}
+
+void tp_block_destroy(tp_block* blk) { delete blk; }
+
+int tp_block_set_events(tp_block* blk, void* const* events, int n) {
+  if (!blk) return TP_EINVAL;
+  if (events && n != TP_BLOCK_STAGES + 1) return TP_EINVAL;
+  blk->events = events;
+  return TP_OK;
+}
+
+// ------------------------------------------------------------------ model
+int tp_model_workspace_bytes(const tp_dims* dims, int n_layers, int n_slices, int partition,
+                             int sync_quant, size_t* out_bytes) {
+  if (n_layers < 1 || !out_bytes) return TP_EINVAL;
+  size_t blk = 0;
+  int rc = tp_block_workspace_bytes(dims, n_slices, partition, sync_quant, &blk);
+  if (rc) return rc;
+  const size_t xb = align256((size_t)dims->max_batch * dims->dim * 4);
+  *out_bytes = blk + 2 * xb;
+  return TP_OK;
+}
+
+int tp_model_create(const tp_dims* dims, int n_layers, int n_slices, int partition, int sync_quant,
+                    const tp_block_weights* layers, const void* embed, const float* final_norm,
+                    const void* wcls, void* workspace, size_t ws_bytes, tp_model** out) {
+  if (!out) return TP_EINVAL;
+  *out = nullptr;
+  size_t need = 0;
+  int rc = tp_model_workspace_bytes(dims, n_layers, n_slices, partition, sync_quant, &need);
+  if (rc) return rc;
+  if (!layers || !embed || !final_norm || !wcls) return TP_EINVAL;
+  if (dims->vocab <= 0 || dims->vocab % 2 != 0 || dims->vocab % n_slices != 0) return TP_EINVAL;
+  if (!aligned16(embed) || !aligned16(final_norm) || !aligned16(wcls)) return TP_EALIGN;
+  if (!workspace || ws_bytes < need) return TP_EWORKSPACE;
+  size_t blk_bytes = 0;
+  tp_block_workspace_bytes(dims, n_slices, partition, sync_quant, &blk_bytes);
+  tp_model* m = new (std::nothrow) tp_model;
+  if (!m) return TP_EINVAL;
+  m->blocks = new (std::nothrow) tp_block[n_layers];
+  if (!m->blocks) {
+    delete m;
+    return TP_EINVAL;
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    tp_block* bp = nullptr;
+    rc = tp_block_create(dims, n_slices, partition, sync_quant, &layers[l], workspace, blk_bytes,
+                         &bp);
+    if (rc) {
+      delete[] m->blocks;
+      delete m;
+      return rc;
+    }
+    m->blocks[l] = *bp;
+    delete bp;
+  }
+  m->d = *dims;
+  m->n_layers = n_layers;
+  m->embed = embed;
+  m->final_norm = final_norm;
+  m->wcls = wcls;
+  uint8_t* base = static_cast<uint8_t*>(workspace) + blk_bytes;
+  m->x = reinterpret_cast<float*>(base);
+  m->xnf = reinterpret_cast<float*>(base + align256((size_t)dims->max_batch * dims->dim * 4));
+  *out = m;
+  return TP_OK;
+}
+
+int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
+                     const int32_t* pos, int batch, float* logits, tp_stream stream) {
+  if (!m || !tokens || !k_cache || !v_cache || !pos || !logits) return TP_EINVAL;
+  if (batch < 1 || batch > m->d.max_batch) return TP_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits)) return TP_EALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  const tp_dims& d = m->d;
+  k_embed<<<batch, 256, 0, s>>>(static_cast<const uint16_t*>(m->embed), tokens, d.dim, m->x);
+  TP_LAUNCH_CHECK();
+  const size_t layer_elems =
+      (size_t)d.max_batch * d.n_kv_heads * (size_t)d.max_seq * d.head_dim;
+  for (int l = 0; l < m->n_layers; ++l) {
+    tp_block* b = &m->blocks[l];
+    NormOut tail{};
+    if (l + 1 < m->n_layers) {
+      tail = norm_out_for(&m->blocks[l + 1], m->blocks[l + 1].w.attn_norm);
+    } else {
+      tail.gain = m->final_norm;
+      tail.eps = d.norm_eps;
+      tail.quant = 0;
+      tail.xn = m->xnf;
+    }
+    uint16_t* kc = static_cast<uint16_t*>(k_cache) + (size_t)l * layer_elems;
+    uint16_t* vc = static_cast<uint16_t*>(v_cache) + (size_t)l * layer_elems;
+    int rc = block_forward_impl(b, m->x, kc, vc, pos, batch, s, l == 0, tail);
+    if (rc) return rc;
+  }
+  GemvArgs a{};
+  a.w[0] = static_cast<const uint16_t*>(m->wcls);
+  a.rows[0] = d.vocab;
+  a.ldw = d.dim;
+  a.Ks = d.dim;
+  a.nseg = 1;
+  a.x = m->xnf;
+  a.ldx = d.dim;
+  a.nb = batch;
+  a.out = logits;
+  a.ldo = d.vocab;
+  a.ctas_per_seg = ctas_for(1, d.vocab / 2);
+  return launch_gemv(a, EPI_PLAIN, s);
+}
+
+void tp_model_destroy(tp_model* m) {
+  if (!m) return;
+  delete[] m->blocks;
+  delete m;
+}
+
+// ------------------------------------------------------------------ Q8 codec
+int tp_quantize_q8(const float* x, int8_t* q, float* d, int64_t n, tp_stream stream) {
+  if (n < 0 || n % 32 != 0) return TP_EINVAL;
+  if (n == 0) return TP_OK;
+  if (!x || !q || !d) return TP_EINVAL;
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(d) & 3)) return TP_EALIGN;
+  int rc = device_check();
+  if (rc) return rc;
+  return launch_quantize(x, q, d, n, (cudaStream_t)stream);
+}
+
+int tp_dequantize_q8(const int8_t* q, const float* d, float* x, int64_t n, tp_stream stream) {
+  if (n < 0 || n % 32 != 0) return TP_EINVAL;
+  if (n == 0) return TP_OK;
+  if (!x || !q || !d) return TP_EINVAL;
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(d) & 3)) return TP_EALIGN;
+  int rc = device_check();
+  if (rc) return rc;
+  return launch_dequantize(q, d, x, n, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,143 @@
+// Shared device helpers for the tensor-parallel block kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tp_block.h"
+
+#define TP_DEV __device__ __forceinline__
+
+namespace tp {
+
+constexpr int kQ8Block = 32;
+constexpr int kHeadDim = 128;
+
+// ---------------------------------------------------------------- bf16 unpack
+// A bf16 value is the upper half of a float32, so widening is a shift.
+TP_DEV float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+TP_DEV float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+TP_DEV uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// 16-byte streaming load that bypasses L1 (weights are read once per launch).
+TP_DEV uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------- reductions
+TP_DEV float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+TP_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum; `red` must hold >= 32 floats. All threads get the result.
+TP_DEV float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = lane < nw ? red[lane] : 0.f;
+  return warp_sum(t);
+}
+TP_DEV float block_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = lane < nw ? red[lane] : -INFINITY;
+  return warp_max(t);
+}
+
+// ---------------------------------------------------------------- Q8 codec
+// Int8 block quantisation of a sync buffer, 32 values per block, one float32
+// scale (the Quantize*/Dequantize* tasks of the distributed-llama list; the
+// format is int8 + fp32 scale, d = amax/127, codes = x/d rounded half away
+// from zero). Every step is one IEEE round-to-nearest float32 operation, so
+// the codes are reproducible bit for bit on any IEEE machine.
+TP_DEV float q8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
+
+TP_DEV int q8_code(float x, float d) {
+  if (d == 0.0f) return 0;
+  float v = roundf(__fdiv_rn(x, d));  // roundf: halfway cases away from zero
+  v = fminf(fmaxf(v, -127.0f), 127.0f);
+  return (int)v;
+}
+
+TP_DEV float q8_value(int q, float d) { return __fmul_rn((float)q, d); }
+
+// Quantise-dequantise of 4 consecutive values held by each of 8 consecutive
+// lanes (one 32-value block per 8-lane group). All 32 lanes must call it.
+TP_DEV void q8_roundtrip4(float4& v) {
+  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+  const float d = q8_scale(a);
+  v.x = q8_value(q8_code(v.x, d), d);
+  v.y = q8_value(q8_code(v.y, d), d);
+  v.z = q8_value(q8_code(v.z, d), d);
+  v.w = q8_value(q8_code(v.w, d), d);
+}
+
+// Quantise 4 values per lane (8-lane groups = one block): writes 4 codes; the
+// group's first lane writes the scale. Returns the codes packed little-endian.
+TP_DEV uint32_t q8_quantize4(float4 v, float* scale_out /* nullable */) {
+  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+  const float d = q8_scale(a);
+  if (scale_out && (threadIdx.x & 7) == 0) *scale_out = d;
+  const uint32_t c0 = (uint32_t)(q8_code(v.x, d) & 0xFF), c1 = (uint32_t)(q8_code(v.y, d) & 0xFF);
+  const uint32_t c2 = (uint32_t)(q8_code(v.z, d) & 0xFF), c3 = (uint32_t)(q8_code(v.w, d) & 0xFF);
+  return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+}
+
+TP_DEV float4 q8_unpack4(uint32_t codes, float d) {
+  float4 r;
+  r.x = q8_value((int)(int8_t)(codes & 0xFF), d);
+  r.y = q8_value((int)(int8_t)((codes >> 8) & 0xFF), d);
+  r.z = q8_value((int)(int8_t)((codes >> 16) & 0xFF), d);
+  r.w = q8_value((int)(int8_t)((codes >> 24) & 0xFF), d);
+  return r;
+}
+
+}  // namespace tp
+
+// ---------------------------------------------------------------- host side
+#define TP_CUDA_TRY(expr)                       \
+  do {                                          \
+    cudaError_t err__ = (expr);                 \
+    if (err__ != cudaSuccess) return TP_ECUDA;  \
+  } while (0)
+
+#define TP_LAUNCH_CHECK()                                        \
+  do {                                                           \
+    if (cudaGetLastError() != cudaSuccess) return TP_ECUDA;      \
+  } while (0)
+
+namespace tp {
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+int device_check();   // TP_OK if the current device is sm_100 (cached per device)
+int num_sms();        // SM count of the current device (cached)
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device); later
+// calls are host-only lookups, so launches stay legal inside stream capture.
+int set_smem_once(const void* kernel, int bytes);
+}  // namespace tp

@@ -1,0 +1,210 @@
+// tp_ffn_forward: the partitioned feed-forward layer.
+//
+// aiterms.tw "Tensor Parallelism", how it works: X replicated; Linear1 split by
+// columns (each slice computes its own columns of the hidden layer, no
+// communication); the activation applied locally; Linear2 split by rows (each
+// slice produces a partial of the full output); one all-reduce. Pope et al.
+// (CS349E lecture script, demo1_1d_vs_2d): 1D splits F only, 2D
+// weight-stationary splits E over grid_x and F over grid_y, which adds a
+// partial-sum stage before the activation.
+//
+// On one GPU every slice is a segment of the same launch: a segment is the
+// contraction range one slice owns, and its partial product is written to its
+// own plane of the partial buffer, which the merge kernel sums in slice order
+// (TP_MERGE_FAITHFUL). With TP_MERGE_FUSED the slices' contraction ranges are
+// accumulated in slice order inside the tensor-core accumulator instead, which
+// is the same sum without materialising the partials.
+#include "ffn.cuh"
+#include "gemm_tc.cuh"
+
+namespace tp {
+namespace {
+
+size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct FfnPlan {
+  int nseg1, nseg2, Ks1, Ks2, swiglu, esize;
+  size_t off_err, off_p1a, off_p1b, off_h, off_p2, total;
+};
+
+int plan_ffn(const tp_ffn_desc* d, FfnPlan* p) {
+  if (!d || !p) return TP_EINVAL;
+  if (d->batch < 1 || d->E <= 0 || d->F <= 0) return TP_EINVAL;
+  if (d->dtype != TP_F32 && d->dtype != TP_BF16) return TP_EINVAL;
+  if (d->act != TP_ACT_RELU && d->act != TP_ACT_SWIGLU) return TP_EINVAL;
+  if (d->sync_quant != 0 && d->sync_quant != 1) return TP_EINVAL;
+  if (d->merge != TP_MERGE_FAITHFUL && d->merge != TP_MERGE_FUSED) return TP_EINVAL;
+  if (d->E % 32 != 0 || d->F % 32 != 0) return TP_EINVAL;
+  if (d->partition == TP_PART_1D) {
+    if (d->n_slices < 1 || d->F % (32 * d->n_slices) != 0) return TP_EINVAL;
+    p->nseg1 = 1;
+    p->nseg2 = d->n_slices;
+  } else if (d->partition == TP_PART_2D) {
+    if (d->grid_x < 1 || d->grid_y < 1) return TP_EINVAL;
+    if (d->E % (32 * d->grid_x) != 0 || d->F % (32 * d->grid_y) != 0) return TP_EINVAL;
+    p->nseg1 = d->grid_x;
+    p->nseg2 = d->grid_y;
+  } else {
+    return TP_EINVAL;
+  }
+  p->Ks1 = d->E / p->nseg1;
+  p->Ks2 = d->F / p->nseg2;
+  p->swiglu = d->act == TP_ACT_SWIGLU;
+  p->esize = d->dtype == TP_F32 ? 4 : 2;
+  if (d->dtype == TP_BF16) {
+    // tensor-core operands: 64-element K steps, 128-row M tiles are padded by TMA
+    if (d->E % 64 != 0 || d->F % 64 != 0) return TP_EINVAL;
+    if (d->merge == TP_MERGE_FAITHFUL && (p->Ks1 % 64 != 0 || p->Ks2 % 64 != 0)) return TP_EINVAL;
+  }
+  if (d->merge == TP_MERGE_FUSED && (d->dtype != TP_BF16 || d->sync_quant)) return TP_ENOTSUP;
+  const size_t B = d->batch, E = d->E, F = d->F;
+  const bool fused = d->merge == TP_MERGE_FUSED;
+  size_t o = 0;
+  p->off_err = o;
+  o += 256;
+  p->off_p1a = o;
+  if (!fused) o += a256((size_t)p->nseg1 * B * F * 4);
+  p->off_p1b = o;
+  if (!fused && p->swiglu) o += a256((size_t)p->nseg1 * B * F * 4);
+  p->off_h = o;
+  o += a256(B * F * p->esize);
+  p->off_p2 = o;
+  if (!fused) o += a256((size_t)p->nseg2 * B * E * 4);
+  p->total = o;
+  return TP_OK;
+}
+
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+extern "C" {
+
+int tp_ffn_workspace_bytes(const tp_ffn_desc* d, size_t* out_bytes) {
+  FfnPlan p;
+  int rc = plan_ffn(d, &p);
+  if (rc) return rc;
+  if (!out_bytes) return TP_EINVAL;
+  *out_bytes = p.total;
+  return TP_OK;
+}
+
+int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const void* W3,
+                   const void* W2, float* Y, void* workspace, size_t ws_bytes, tp_stream stream) {
+  FfnPlan p;
+  int rc = plan_ffn(d, &p);
+  if (rc) return rc;
+  if (!X || !W1 || !W2 || !Y || (p.swiglu && !W3)) return TP_EINVAL;
+  if (!aligned16(X) || !aligned16(W1) || !aligned16(W2) || !aligned16(Y) ||
+      (W3 && !aligned16(W3)))
+    return TP_EALIGN;
+  if (p.total > 0 && (!workspace || ws_bytes < p.total)) return TP_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return TP_EALIGN;
+  rc = device_check();
+  if (rc) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int B = d->batch, E = d->E, F = d->F;
+  void* H = ws + p.off_h;
+  int* err = reinterpret_cast<int*>(ws + p.off_err);
+
+  if (d->merge == TP_MERGE_FUSED) {
+    // stage 1: H = act(X W1^T [, X W3^T]) over the full E (slice order = K order)
+    TcGemm g{};
+    g.A = X;
+    g.lda = E;
+    g.B = W1;
+    g.ldb = E;
+    g.B2 = p.swiglu ? W3 : nullptr;
+    g.M = B;
+    g.N = F;
+    g.K = E;
+    g.nseg = 1;
+    g.epi = p.swiglu ? TC_EPI_SWIGLU_BF16 : TC_EPI_RELU_BF16;
+    g.out = H;
+    g.ldo = F;
+    g.err = err;
+    rc = launch_tc_gemm(g, s);
+    if (rc) return rc;
+    // stage 2: Y = H W2^T over the full F
+    TcGemm g2{};
+    g2.A = H;
+    g2.lda = F;
+    g2.B = W2;
+    g2.ldb = F;
+    g2.M = B;
+    g2.N = E;
+    g2.K = F;
+    g2.nseg = 1;
+    g2.epi = TC_EPI_STORE_F32;
+    g2.out = Y;
+    g2.ldo = E;
+    g2.err = err;
+    return launch_tc_gemm(g2, s);
+  }
+
+  float* P1a = reinterpret_cast<float*>(ws + p.off_p1a);
+  float* P1b = reinterpret_cast<float*>(ws + p.off_p1b);
+  float* P2 = reinterpret_cast<float*>(ws + p.off_p2);
+  auto contract = [&](const void* A, int64_t lda, const void* Bm, int64_t ldb, float* P, int M,
+                      int N, int Ks, int nseg) -> int {
+    if (d->dtype == TP_F32) return launch_gemm_simt(TP_F32, A, lda, Bm, ldb, P, M, N, Ks, nseg, s);
+    TcGemm g{};
+    g.A = A;
+    g.lda = lda;
+    g.B = Bm;
+    g.ldb = ldb;
+    g.M = M;
+    g.N = N;
+    g.K = Ks;
+    g.nseg = nseg;
+    g.epi = TC_EPI_STORE_F32;
+    g.out = P;
+    g.ldo = N;
+    g.out_seg = (int64_t)M * N;
+    g.err = err;
+    return launch_tc_gemm(g, s);
+  };
+
+  // stage 1: partials of X W1^T over the E-segments (one segment in 1D)
+  rc = contract(X, E, W1, E, P1a, B, F, p.Ks1, p.nseg1);
+  if (rc) return rc;
+  if (p.swiglu) {
+    rc = contract(X, E, W3, E, P1b, B, F, p.Ks1, p.nseg1);
+    if (rc) return rc;
+  }
+  {
+    FfnMergeArgs m{};
+    m.P1 = P1a;
+    m.P3 = p.swiglu ? P1b : nullptr;
+    m.seg_stride = (int64_t)B * F;
+    m.nseg = p.nseg1;
+    m.M = B;
+    m.N = F;
+    // in 1D the hidden columns stay local to their slice: no sync buffer there
+    m.quant = d->partition == TP_PART_2D ? d->sync_quant : 0;
+    m.act = p.swiglu ? ACT_SWIGLU : ACT_RELU;
+    if (d->dtype == TP_F32)
+      m.out_f32 = static_cast<float*>(H);
+    else
+      m.out_bf16 = static_cast<uint16_t*>(H);
+    rc = launch_ffn_merge(m, s);
+    if (rc) return rc;
+  }
+  // stage 2: partials of H W2^T over the F-segments
+  rc = contract(H, F, W2, F, P2, B, E, p.Ks2, p.nseg2);
+  if (rc) return rc;
+  FfnMergeArgs m{};
+  m.P1 = P2;
+  m.seg_stride = (int64_t)B * E;
+  m.nseg = p.nseg2;
+  m.M = B;
+  m.N = E;
+  m.quant = d->sync_quant;
+  m.act = ACT_NONE;
+  m.out_f32 = Y;
+  return launch_ffn_merge(m, s);
+}
+
+}  // extern "C"

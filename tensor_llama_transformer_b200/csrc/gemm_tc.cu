@@ -1,0 +1,407 @@
+// Persistent tcgen05 GEMM for the batched / prefill FFN (sm_100a).
+//
+//   D[seg, m, n] = sum_{k < K} A[m, seg*K + k] * B[n, seg*K + k]
+//
+// A = activations [M tokens, K] and B = weights [N features, K], both bf16
+// with the contraction dimension contiguous (a PyTorch Linear weight is already
+// in this layout). A segment is the contraction range one tensor-parallel slice
+// owns (a row split); with nseg > 1 each slice's partial product goes to its
+// own plane of the output, to be summed by the merge (aiterms.tw "Tensor
+// Parallelism": Linear2 split by rows, then an all-reduce; Pope et al. demo1:
+// 2D weight-stationary adds a partial-sum stage before the activation).
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0  : TMA producer — 128x64 A tile and 256x64 B tile per stage, 128-byte
+//             swizzle, 4-stage ring of shared memory, completion on mbarriers.
+//   warp 1  : allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
+//             one lane issues tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32);
+//             tcgen05.commit releases each smem stage and publishes each tile.
+//   warps 2-5: epilogue — tcgen05.ld of the accumulator (each warp its 32 TMEM
+//             lanes = 32 output rows), activation, stores to global memory,
+//             overlapped with the next tile's mainloop (double-buffered TMEM).
+// Tiles are visited m-fastest so that the CTAs working at the same time share
+// the weight tile through L2. No TMA multicast is used. Every wait on an
+// mbarrier is bounded by a 2 s timer; on expiry the kernel sets *err and the
+// roles leave their loops, so a fault in the pipeline cannot hang the GPU.
+#include <cuda.h>
+
+#include "gemm_tc.cuh"
+
+namespace tp {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+TP_DEV uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+TP_DEV void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
+}
+TP_DEV void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
+               : "memory");
+}
+TP_DEV void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
+}
+TP_DEV bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(s2u(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of `parity` to complete; gives up after kTimeoutNs.
+TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(b, parity)) return true;
+    if ((i & 255) == 0 && gtimer() - t0 > kTimeoutNs) {
+      if (err) atomicExch(err, 1);
+      return false;
+    }
+  }
+}
+
+TP_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(s2u(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(s2u(bar))
+      : "memory");
+}
+
+TP_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+TP_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+TP_DEV void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                      uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+TP_DEV void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   s2u(bar))
+               : "memory");
+}
+
+TP_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+TP_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart (stride
+// byte offset), descriptor version 1, layout type 2 = SWIZZLE_128B. The leading
+// byte offset is not used by this layout. Advancing K by 16 bf16 elements inside
+// the swizzle atom adds 32 bytes (2 in the >>4 encoding) to the start address.
+TP_DEV uint64_t desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+constexpr uint32_t idesc_bf16(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+TP_DEV uint32_t pack_bf16x2(float a, float b) {
+  return (uint32_t)f32_to_bf16_bits(a) | ((uint32_t)f32_to_bf16_bits(b) << 16);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_tc_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
+              const __grid_constant__ CUtensorMap mB2, TcGemm g, int num_m, int num_n, int ntiles) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&tfull[j], 1);
+      mbar_init(&tempty[j], 4);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     s2u(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = g.K / BK;
+  const int per_seg = num_m * num_n;
+  constexpr int NOUT = EPI == TC_EPI_SWIGLU_BF16 ? BN / 2 : BN;  // output columns per tile
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int seg = tile / per_seg, r = tile - seg * per_seg;
+        const int nb = r / num_m, mb = r - nb * num_m;
+        const int m0 = mb * BM, n0 = nb * NOUT;
+        const int kbase = seg * g.K;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], ph ^ 1, g.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[stage], STAGE_BYTES);
+          const int kx = kbase + kb * BK;
+          tma_load_2d(sA + stage * A_BYTES, &mA, kx, m0, &full[stage]);
+          if (EPI == TC_EPI_SWIGLU_BF16) {
+            tma_load_2d(sB + stage * B_BYTES, &mB, kx, n0, &full[stage]);
+            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, &mB2, kx, n0, &full[stage]);
+          } else {
+            tma_load_2d(sB + stage * B_BYTES, &mB, kx, n0, &full[stage]);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(BM, BN);
+      int stage = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, g.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], ph, g.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc_sw128(s2u(sA + stage * A_BYTES));
+          const uint64_t b0 = desc_sw128(s2u(sB + stage * B_BYTES));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) umma_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lanes 32*(warp%4) .. +31
+    const int q = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(&tfull[acc], aph, g.err)) break;
+      tc_fence_after();
+      const int seg = tile / per_seg, r = tile - seg * per_seg;
+      const int nb = r / num_m, mb = r - nb * num_m;
+      const int row = mb * BM + 32 * q + lane;
+      const int n0 = nb * NOUT;
+      const bool row_ok = row < g.M;
+      const uint32_t taddr = tmem + (uint32_t)(acc * BN) + ((uint32_t)(32 * q) << 16);
+      if (EPI == TC_EPI_STORE_F32) {
+        float* o = static_cast<float*>(g.out) + (size_t)seg * g.out_seg + (size_t)row * g.ldo + n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (row_ok && n0 + c < g.N) {
+            float4* o4 = reinterpret_cast<float4*>(o + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              o4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                  __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          }
+        }
+      } else if (EPI == TC_EPI_RELU_BF16) {
+        uint16_t* o = static_cast<uint16_t*>(g.out) + (size_t)row * g.ldo + n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (row_ok && n0 + c < g.N) {
+            uint4* o4 = reinterpret_cast<uint4*>(o + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = fmaxf(__uint_as_float(v[8 * j + e]), 0.f);
+              o4[j] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+            }
+          }
+        }
+      } else {  // TC_EPI_SWIGLU_BF16: columns [0,128) = X W1^T, [128,256) = X W3^T
+        uint16_t* o = static_cast<uint16_t*>(g.out) + (size_t)row * g.ldo + n0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t a[32], b[32];
+          tmem_ld32(taddr + c, a);
+          tmem_ld32(taddr + BN / 2 + c, b);
+          tmem_wait_ld();
+          if (row_ok && n0 + c < g.N) {
+            uint4* o4 = reinterpret_cast<uint4*>(o + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float z = __uint_as_float(a[8 * j + e]);
+                f[e] = z / (1.0f + expf(-z)) * __uint_as_float(b[8 * j + e]);
+              }
+              o4[j] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D map over a bf16 row-major matrix [rows, inner] with row stride ld elements,
+// box = 64 elements (128 bytes) x box_rows, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t inner, int64_t ld,
+              int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+int launch_epi(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mB2,
+               const TcGemm& g, int num_m, int num_n, int ntiles, cudaStream_t s) {
+  if (set_smem_once((const void*)k_tc_gemm<EPI>, SMEM_BYTES)) return TP_ECUDA;
+  int grid = ntiles < num_sms() ? ntiles : num_sms();
+  k_tc_gemm<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(mA, mB, mB2, g, num_m, num_n, ntiles);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+}  // namespace
+
+int launch_tc_gemm(const TcGemm& g, cudaStream_t s) {
+  if (g.M < 1 || g.N < 1 || g.K < BK || g.K % BK != 0 || g.nseg < 1) return TP_EINVAL;
+  if (g.N % 32 != 0 || g.lda % 8 != 0 || g.ldb % 8 != 0 || g.ldo % 8 != 0) return TP_EINVAL;
+  const bool swiglu = g.epi == TC_EPI_SWIGLU_BF16;
+  if (swiglu && !g.B2) return TP_EINVAL;
+  const int64_t inner = (int64_t)g.nseg * g.K;
+  CUtensorMap mA, mB, mB2;
+  const int brows = swiglu ? BN / 2 : BN;
+  if (!make_map(&mA, g.A, g.M, inner, g.lda, BM) || !make_map(&mB, g.B, g.N, inner, g.ldb, brows) ||
+      !make_map(&mB2, swiglu ? g.B2 : g.B, g.N, inner, g.ldb, brows))
+    return TP_ECUDA;
+  const int nout = swiglu ? BN / 2 : BN;
+  const int num_m = (g.M + BM - 1) / BM;
+  const int num_n = (g.N + nout - 1) / nout;
+  const int64_t nt = (int64_t)num_m * num_n * g.nseg;
+  if (nt > 0x7fffffff) return TP_EINVAL;
+  switch (g.epi) {
+    case TC_EPI_STORE_F32: return launch_epi<TC_EPI_STORE_F32>(mA, mB, mB2, g, num_m, num_n, (int)nt, s);
+    case TC_EPI_RELU_BF16: return launch_epi<TC_EPI_RELU_BF16>(mA, mB, mB2, g, num_m, num_n, (int)nt, s);
+    case TC_EPI_SWIGLU_BF16:
+      return launch_epi<TC_EPI_SWIGLU_BF16>(mA, mB, mB2, g, num_m, num_n, (int)nt, s);
+    default: return TP_EINVAL;
+  }
+}
+
+}  // namespace tp

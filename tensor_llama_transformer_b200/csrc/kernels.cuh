@@ -1,0 +1,84 @@
+// Kernel argument structs and launchers shared by the host API files.
+#pragma once
+
+#include "common.cuh"
+
+namespace tp {
+
+// ------------------------------------------------------------------ RMSNorm (+Q8)
+// x [B, dim] -> normalised rows. Outputs (each nullable):
+//   xn  float32 [B, dim]  (the value the consumers read when quantisation is off)
+//   xq  int8 [B, dim] + xd float32 [B, dim/32]  (Q8 sync buffer)
+//   xb  bf16 [B, dim]     (the consumers' value rounded to bf16, for tensor-core paths)
+struct NormOut {
+  float* xn;
+  int8_t* xq;
+  float* xd;
+  uint16_t* xb;
+  const float* gain;
+  float eps;
+  int quant;
+};
+
+// Merge of n row-split partials [n, B, dim] into the residual x, then an optional
+// RMSNorm of the merged rows for the next sublayer (norm.gain == nullptr: none).
+int launch_rmsnorm(const float* x, int B, int dim, const NormOut& no, cudaStream_t s);
+int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, const NormOut& no,
+                 cudaStream_t s);
+int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s);
+int launch_dequantize(const int8_t* q, const float* d, float* x, int64_t n, cudaStream_t s);
+
+// ------------------------------------------------------------------ slice GEMV
+enum GemvEpi { EPI_PLAIN = 0, EPI_SWIGLU = 1, EPI_QKV = 2 };
+
+struct GemvArgs {
+  // weights: up to three bf16 matrices [rows_i, ldw] stacked in row space (QKV),
+  // or two matrices read row for row together (SwiGLU: W1 row f with W3 row f).
+  const uint16_t* w[3];
+  int rows[3];
+  int64_t ldw;   // row stride in elements (= full input width K)
+  int Ks;        // contraction length of one segment
+  int nseg;      // number of segments: segment s reads columns [s*Ks, (s+1)*Ks)
+  // input: float32 x [B, ldx] or Q8 (xq [B, ldx], xd [B, ldx/32])
+  const float* x;
+  const int8_t* xq;
+  const float* xd;
+  int ldx;
+  int b0, nb;    // batch rows [b0, b0+nb) handled by this launch
+  // EPI_PLAIN / EPI_SWIGLU output: out[seg*out_seg + b*ldo + row]
+  float* out;
+  uint16_t* out_bf16;  // optional bf16 copy, same indexing
+  int64_t out_seg;
+  int ldo;
+  // EPI_QKV
+  float* qout;   // rotated q [B, H*hd]
+  uint16_t* kc;  // caches [maxB, Hkv, max_seq, hd]
+  uint16_t* vc;
+  const int32_t* pos;
+  int n_heads, n_kv_heads, max_seq;
+  float theta;
+  // launch shape
+  int ctas_per_seg;
+};
+
+int launch_gemv(const GemvArgs& a, int epi, cudaStream_t s);
+
+// ------------------------------------------------------------------ attention
+constexpr int kAttnChunk = 128;  // context positions per CTA
+
+struct AttnArgs {
+  const float* q;       // rotated q [B, H*hd]
+  const uint16_t* kc;   // [maxB, Hkv, max_seq, hd] bf16
+  const uint16_t* vc;
+  const int32_t* pos;   // [B]
+  int B, H, Hkv, max_seq, nchunk;
+  float* part_o;        // [B, H, nchunk, hd] unnormalised partial outputs
+  float* part_ml;       // [B, H, nchunk, 2] running max and sum
+  float* att;           // [B, H*hd] combined output
+  uint16_t* att_bf16;   // optional bf16 copy
+  int* err;             // device error flag (bounded waits)
+};
+
+int launch_attention(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace tp

@@ -1,0 +1,119 @@
+"""The C ABI library loads and exports every function include/tp_block.h declares (CPU only).
+
+Only calls that need no GPU are made here: status strings, workspace sizing
+and argument validation that rejects inputs before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp_block.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(tp_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def tpb():
+    import tensor_llama_transformer_b200 as t
+
+    return t
+
+
+def test_every_declared_symbol_is_exported(tpb):
+    names = _declared()
+    assert "tp_block_forward" in names and "tp_ffn_forward" in names and len(names) >= 15
+    lib = ctypes.CDLL(tpb.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) <= set(tpb.EXPORTED)
+
+
+def test_status_strings_and_version(tpb):
+    assert tpb.tp_status_string(0) == "ok"
+    assert "workspace" in tpb.tp_status_string(tpb.TP_EWORKSPACE)
+    assert tpb.tp_status_string(99) == "unknown status"
+    assert "sm_100a" in tpb.tp_version()
+
+
+def _dims(tpb, **kw):
+    base = dict(dim=4096, n_heads=32, n_kv_heads=32, head_dim=128, ffn_dim=11008, vocab=32000,
+                max_batch=1, max_seq=1024)
+    base.update(kw)
+    return tpb.make_dims(**base)
+
+
+def test_workspace_sizes(tpb):
+    d = _dims(tpb)
+    w1 = tpb.tp_block_workspace_bytes(d, 4, tpb.TP_PART_1D, 1)
+    w2 = tpb.tp_block_workspace_bytes(d, 4, tpb.TP_PART_2D, 1)
+    assert 0 < w1 < w2  # the 2D stage-1 partials need room
+    assert w1 % 256 == 0
+    d16 = _dims(tpb, max_batch=16)
+    assert tpb.tp_block_workspace_bytes(d16, 4, tpb.TP_PART_1D, 1) > w1
+    m = tpb.tp_model_workspace_bytes(d, 32, 8, tpb.TP_PART_1D, 0)
+    assert m > tpb.tp_block_workspace_bytes(d, 8, tpb.TP_PART_1D, 0)
+
+
+@pytest.mark.parametrize("kw,n", [
+    (dict(dim=4000), 4),              # dim not a multiple of 128
+    (dict(head_dim=64), 4),           # head_dim other than 128 -> not supported
+    (dict(n_heads=30), 4),            # heads do not divide
+    (dict(n_kv_heads=8), 16),         # kv heads fewer than slices
+    (dict(ffn_dim=11000), 4),         # F % (32 n) != 0
+    (dict(max_batch=0), 4),
+    (dict(max_batch=65), 4),
+    (dict(), 0),
+])
+def test_invalid_dims_rejected(tpb, kw, n):
+    d = _dims(tpb, **kw)
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_block_workspace_bytes(d, n, tpb.TP_PART_1D, 0)
+    assert e.value.status in (tpb.TP_EINVAL, tpb.TP_ENOTSUP)
+
+
+def test_create_rejects_missing_workspace_before_cuda(tpb):
+    d = _dims(tpb)
+    w = tpb.make_weights(*([16] * 9))  # aligned fake addresses; never dereferenced
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_block_create(d, 4, tpb.TP_PART_1D, 1, w, None, 0)
+    assert e.value.status == tpb.TP_EWORKSPACE
+    w_bad = tpb.make_weights(*([16] * 8 + [18]))
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_block_create(d, 4, tpb.TP_PART_1D, 1, w_bad, 256, 1 << 40)
+    assert e.value.status == tpb.TP_EALIGN
+
+
+def test_ffn_plan_validation(tpb):
+    desc = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1, 1,
+                           0, tpb.TP_MERGE_FAITHFUL)
+    ws1d = tpb.tp_ffn_workspace_bytes(desc)
+    assert ws1d >= 64 * 512 * 18432 * 4  # the 64 materialised partials of the row split
+    desc2 = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_2D, 64, 8,
+                            8, 0, tpb.TP_MERGE_FAITHFUL)
+    assert tpb.tp_ffn_workspace_bytes(desc2) < ws1d
+    fused = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1,
+                            1, 0, tpb.TP_MERGE_FUSED)
+    assert tpb.tp_ffn_workspace_bytes(fused) < 512 * 73728 * 2 + 4096
+    bad = tpb.tp_ffn_desc(8, 64, 250, tpb.TP_F32, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 2, 1, 1, 0, 0)
+    with pytest.raises(tpb.TpError):
+        tpb.tp_ffn_workspace_bytes(bad)
+    fused_f32 = tpb.tp_ffn_desc(8, 64, 256, tpb.TP_F32, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 2, 1, 1, 0,
+                                tpb.TP_MERGE_FUSED)
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_ffn_workspace_bytes(fused_f32)
+    assert e.value.status == tpb.TP_ENOTSUP
+
+
+def test_quantize_rejects_bad_sizes(tpb):
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_quantize_q8(16, 16, 16, 33, stream=0)
+    assert e.value.status == tpb.TP_EINVAL
+    tpb.tp_quantize_q8(16, 16, 16, 0, stream=0)  # empty input: nothing to do

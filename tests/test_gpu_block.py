@@ -1,0 +1,139 @@
+"""Decoder block on the GPU through the C ABI versus the float64 oracle.
+
+Bottom-up in the tt-metal thread's manner: the intermediates (normalised input,
+rotated q, attention output, SwiGLU output, the k/v rows written to the cache)
+and the block output are each compared with the oracle, reporting max relative
+error and PCC. The bar is 2e-2 max relative error (bf16 weights, fp32
+accumulation); tighter bounds derived from the arithmetic are asserted as well.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth.device import DeviceBlock, to_bits
+from tests.metrics import BF16_TOL, report
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tpb(cuda_ok):
+    import tensor_llama_transformer_b200 as t
+
+    return t
+
+
+def _dims(tpb, s, max_batch):
+    return tpb.make_dims(s.dim, s.n_heads, s.n_kv_heads, s.head_dim, s.ffn_dim, max(s.vocab, 2),
+                         max_batch, s.max_seq, s.norm_eps, s.rope_theta)
+
+
+def run_block(tpb, inp, n, quant, partition=1, max_batch=None):
+    """Runs one block forward on the GPU; returns (x_out, k_rows, v_rows, buffers, err)."""
+    s = inp.shape
+    B = inp.x.shape[0]
+    mb = max_batch or B
+    dev = DeviceBlock(inp, max_batch=mb)
+    dims = _dims(tpb, s, mb)
+    nbytes = tpb.tp_block_workspace_bytes(dims, n, partition, quant)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    h = tpb.tp_block_create(dims, n, partition, quant, tpb.make_weights(*dev.weights()), ws, nbytes)
+    try:
+        tpb.tp_block_forward(h, dev.x, dev.k_cache, dev.v_cache, dev.pos, B)
+        torch.cuda.synchronize()
+        bufs = {}
+        for name, which, dt in (("att", tpb.BUF_ATT, torch.float32), ("q", tpb.BUF_Q, torch.float32),
+                                ("h", tpb.BUF_H, torch.float32), ("xn", tpb.BUF_XN, torch.float32),
+                                ("xq", tpb.BUF_XQ, torch.int8), ("xd", tpb.BUF_XD, torch.float32)):
+            off, size = tpb.tp_block_buffer(h, which)
+            bufs[name] = ws[off:off + size].view(dt).cpu().numpy()
+        err = int(ws[tpb.tp_block_buffer(h, 7)[0]:][:4].view(torch.int32).item())
+    finally:
+        tpb.tp_block_destroy(h)
+    pos = inp.pos
+    kb = to_bits(dev.k_cache)
+    vb = to_bits(dev.v_cache)
+    k_rows = np.stack([kb[b, :, pos[b], :] for b in range(B)])
+    v_rows = np.stack([vb[b, :, pos[b], :] for b in range(B)])
+    return dev.x.cpu().numpy().astype(np.float64), k_rows, v_rows, bufs, err
+
+
+def check_block(tpb, inp, n, quant, partition=1, tol_out=BF16_TOL, tight=None, name="block"):
+    s = inp.shape
+    B = inp.x.shape[0]
+    tr = {}
+    ref, k_ref, v_ref = oracle.block_forward(inp, n, bool(quant), partition, trace=tr)
+    y, k_rows, v_rows, bufs, err = run_block(tpb, inp, n, quant, partition)
+    assert err == 0, "a bounded wait in a kernel gave up"
+    QD = s.n_heads * s.head_dim
+    r_att, _ = report(f"{name} att", bufs["att"][:B * QD].reshape(B, QD), tr["att"])
+    r_q, _ = report(f"{name} q", bufs["q"][:B * QD].reshape(B, QD), tr["q"])
+    r_k, _ = report(f"{name} k@pos", oracle.bf16_to_f64(k_rows), oracle.bf16_to_f64(k_ref))
+    r_v, _ = report(f"{name} v@pos", oracle.bf16_to_f64(v_rows), oracle.bf16_to_f64(v_ref))
+    r_out, p_out = report(f"{name} out", y, ref)
+    r_dx, _ = report(f"{name} out-x", y - inp.x, ref - inp.x)
+    for r in (r_att, r_q, r_k, r_v, r_out, r_dx):
+        assert r <= tol_out
+    if partition == 1:
+        r_h, _ = report(f"{name} h", bufs["h"][:B * s.ffn_dim].reshape(B, s.ffn_dim), tr["h"])
+        assert r_h <= tol_out
+    if tight is not None:
+        assert max(r_q, r_att, r_out, r_dx) <= tight, "regression against the expected error level"
+    assert p_out > 0.9999
+    return r_out
+
+
+SMALL_MHA = synth.BlockShape(dim=256, n_heads=2, n_kv_heads=2, head_dim=128, ffn_dim=512,
+                             vocab=0, max_seq=300, batch=3, n_slices=2, sync_quant=False, pos=299,
+                             w_std=0.05)
+SMALL_GQA = synth.BlockShape(dim=512, n_heads=8, n_kv_heads=2, head_dim=128, ffn_dim=1024,
+                             vocab=0, max_seq=260, batch=2, n_slices=2, sync_quant=False, pos=259,
+                             w_std=0.04)
+SMALL_GQA8 = synth.BlockShape(dim=1024, n_heads=8, n_kv_heads=1, head_dim=128, ffn_dim=2048,
+                              vocab=0, max_seq=129, batch=5, n_slices=1, sync_quant=False, pos=128,
+                              w_std=0.03)
+
+
+@pytest.mark.parametrize("quant", [0, 1])
+@pytest.mark.parametrize("shape,n,pos", [
+    (SMALL_MHA, 2, [299, 130, 0]),      # ragged context: 3 chunks, 2 chunks, a single position
+    (SMALL_GQA, 2, [259, 127]),         # GQA group of 4 per kv head
+    (SMALL_GQA8, 1, [128, 1, 64, 127, 5]),  # GQA group of 8, batch 5 (two launches of 4 + 1)
+])
+def test_block_small(tpb, shape, n, pos, quant):
+    inp = synth.block_inputs(4242, shape)
+    inp.pos[:] = pos
+    check_block(tpb, inp, n, quant, tight=2e-3 if quant else 2e-4,
+                name=f"d{shape.dim} H{shape.n_heads}/{shape.n_kv_heads} n{n} q{quant}")
+
+
+@pytest.mark.parametrize("quant", [0, 1])
+def test_block_2d_ffn(tpb, quant):
+    shape = synth.BlockShape(dim=512, n_heads=4, n_kv_heads=4, head_dim=128, ffn_dim=1024, vocab=0,
+                             max_seq=64, batch=2, n_slices=4, sync_quant=False, pos=63, w_std=0.04)
+    inp = synth.block_inputs(4343, shape)
+    inp.pos[:] = [63, 10]
+    ref1, _, _ = oracle.block_forward(inp, 4, bool(quant), partition=1)
+    r = check_block(tpb, inp, 4, quant, partition=2, tight=2e-3 if quant else 2e-4, name=f"2d q{quant}")
+    assert r <= BF16_TOL
+    if not quant:  # 2D and 1D agree in exact arithmetic
+        ref2, _, _ = oracle.block_forward(inp, 4, False, partition=2)
+        assert np.max(np.abs(ref2 - ref1)) <= 1e-12 * np.max(np.abs(ref1))
+
+
+def test_block_c2_full_size(tpb):
+    """Llama-2-7B block, n=4, int8 sync, KV 1024, batch 1: the bench's workload."""
+    inp = synth.block_inputs(synth.CONFIG_SEED["C2"], synth.C2)
+    check_block(tpb, inp, synth.C2.n_slices, 1, tight=5e-3, name="C2")
+
+
+def test_block_c2_slices_agree(tpb):
+    """The slice count changes only rounding: n = 1, 2, 4, 8 give the same block (quant off)."""
+    s = synth.BlockShape(dim=4096, n_heads=32, n_kv_heads=32, head_dim=128, ffn_dim=11008, vocab=0,
+                         max_seq=256, batch=1, n_slices=4, sync_quant=False, pos=200)
+    inp = synth.block_inputs(77, s)
+    outs = [run_block(tpb, inp, n, 0)[0] for n in (1, 2, 4, 8)]
+    for o in outs[1:]:
+        assert np.max(np.abs(o - outs[0])) / np.max(np.abs(outs[0])) < 1e-5

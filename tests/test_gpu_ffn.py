@@ -1,0 +1,96 @@
+"""Partitioned FFN on the GPU through the C ABI versus the float64 oracle.
+
+float32 (the ggmlR-shaped two-stage ReLU FFN, 1e-5) on CUDA cores; bf16 on the
+tcgen05 tensor-core contraction (2e-2), in 1D and 2D partitions, with the
+partials materialised (faithful merge) or accumulated in the contraction
+(fused merge), ReLU and SwiGLU, with and without Q8 sync of the partials.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth.device import bf16_tensor, f32_tensor
+from tests.metrics import BF16_TOL, report
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tpb(cuda_ok):
+    import tensor_llama_transformer_b200 as t
+
+    return t
+
+
+def run_ffn(tpb, s: synth.FfnShape, inputs, partition, merge, quant=False):
+    up = f32_tensor if s.dtype == "f32" else bf16_tensor
+    X, W1, W2 = up(inputs["X"]), up(inputs["W1"]), up(inputs["W2"])
+    W3 = up(inputs["W3"]) if "W3" in inputs else None
+    B = inputs["X"].shape[0]
+    gx, gy = (s.grid_x, s.grid_y) if partition == 2 else (1, 1)
+    desc = tpb.tp_ffn_desc(B, s.E, s.F, tpb.TP_F32 if s.dtype == "f32" else tpb.TP_BF16,
+                           tpb.TP_ACT_RELU if s.act == "relu" else tpb.TP_ACT_SWIGLU, partition,
+                           s.n_slices, gx, gy, int(quant), merge)
+    nbytes = tpb.tp_ffn_workspace_bytes(desc)
+    ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+    Y = torch.full((B, s.E), float("nan"), dtype=torch.float32, device="cuda")
+    tpb.tp_ffn_forward(desc, X, W1, W3, W2, Y, ws, nbytes)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "a bounded wait in a kernel gave up"
+    return Y.cpu().numpy().astype(np.float64)
+
+
+def _ref(s, inputs, partition, quant):
+    cv = (lambda a: a.astype(np.float64)) if s.dtype == "f32" else oracle.bf16_to_f64
+    X, W1, W2 = cv(inputs["X"]), cv(inputs["W1"]), cv(inputs["W2"])
+    W3 = cv(inputs["W3"]) if "W3" in inputs else None
+    return oracle.ffn_forward(X, W1, W2, act=s.act, W3=W3, partition=partition,
+                              n_slices=s.n_slices, grid=(s.grid_x, s.grid_y), quant=quant)
+
+
+@pytest.mark.parametrize("partition", [1, 2])
+@pytest.mark.parametrize("quant", [False, True])
+def test_c1_fp32(tpb, partition, quant):
+    s = synth.C1 if partition == 1 else synth.FfnShape(**{**synth.C1.__dict__, "grid_x": 1,
+                                                          "grid_y": 2, "partition": 2})
+    inputs = synth.ffn_inputs(synth.CONFIG_SEED["C1"], s)
+    y = run_ffn(tpb, s, inputs, partition, tpb.TP_MERGE_FAITHFUL, quant)
+    ref = _ref(s, inputs, partition, quant)
+    r, p = report(f"C1 fp32 part{partition} q{int(quant)}", y, ref)
+    # quantised partials: the float32 and float64 partials can straddle a code
+    # boundary, so the quantised case is held to the quantisation step instead
+    assert r <= (1e-5 if not quant else 1e-2)
+    if not quant:
+        unsharded = np.maximum(inputs["X"].astype(np.float64) @ inputs["W1"].T.astype(np.float64), 0) \
+            @ inputs["W2"].T.astype(np.float64)
+        assert np.max(np.abs(y - unsharded)) / np.max(np.abs(unsharded)) <= 1e-5
+
+
+SMALL_BF16 = synth.FfnShape(batch=200, E=512, F=1024, dtype="bf16", act="relu", n_slices=4,
+                            grid_x=2, grid_y=2, x_std=1.0, w_std=0.05)
+
+
+@pytest.mark.parametrize("act", ["relu", "swiglu"])
+@pytest.mark.parametrize("partition,merge,quant", [
+    (1, 0, False), (1, 1, False), (2, 0, False), (1, 0, True), (2, 0, True)])
+def test_bf16_small(tpb, act, partition, merge, quant):
+    s = synth.FfnShape(**{**SMALL_BF16.__dict__, "act": act})
+    inputs = synth.ffn_inputs(5151, s)
+    y = run_ffn(tpb, s, inputs, partition, merge, quant)
+    ref = _ref(s, inputs, partition, quant)
+    r, p = report(f"bf16 {act} part{partition} merge{merge} q{int(quant)}", y, ref)
+    assert r <= BF16_TOL
+    assert p > 0.9999
+
+
+@pytest.mark.parametrize("M", [1, 127, 128, 129, 384])
+def test_bf16_m_tails(tpb, M):
+    s = synth.FfnShape(batch=M, E=256, F=768, dtype="bf16", act="relu", n_slices=3,
+                       x_std=1.0, w_std=0.06)
+    inputs = synth.ffn_inputs(6161 + M, s)
+    for merge in (0, 1):
+        y = run_ffn(tpb, s, inputs, 1, merge)
+        r, _ = report(f"bf16 M={M} merge{merge}", y, _ref(s, inputs, 1, False))
+        assert r <= BF16_TOL
