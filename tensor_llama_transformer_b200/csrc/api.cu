@@ -203,10 +203,18 @@ NormOut norm_out_for(const tp_block* b, const float* gain) {
 // One block forward. `first` launches the attention RMSNorm (otherwise the
 // caller's previous merge already wrote it); `tail` is the RMSNorm fused
 // after the final merge (gain == nullptr: none).
+// Records the caller's timing event before `stage`. Inside stream capture the
+// record must be an external event node (a plain record would only become a
+// dependency edge of the graph and never be timestamped).
 int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
   if (!blk->events) return TP_OK;
-  return cudaEventRecord(static_cast<cudaEvent_t>(blk->events[stage]), s) == cudaSuccess ? TP_OK
-                                                                                        : TP_ECUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return TP_ECUDA;
+  cudaEvent_t ev = static_cast<cudaEvent_t>(blk->events[stage]);
+  const cudaError_t e = cap == cudaStreamCaptureStatusActive
+                            ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                            : cudaEventRecord(ev, s);
+  return e == cudaSuccess ? TP_OK : TP_ECUDA;
 }
 
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
