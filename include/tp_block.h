@@ -58,7 +58,8 @@ enum tp_status {
   TP_EARCH = 3,       /* current device is not compute capability 10.0 (B200) */
   TP_ECUDA = 4,       /* a CUDA runtime call or kernel launch failed */
   TP_ENOTSUP = 5,     /* a combination this build does not implement */
-  TP_EALIGN = 6       /* a pointer is not 16-byte aligned */
+  TP_EALIGN = 6,      /* a pointer is not 16-byte aligned */
+  TP_ESCRATCH = 7     /* the workspace would exceed the no-allocation entry point's fixed scratch */
 };
 
 enum { TP_PART_1D = 1, TP_PART_2D = 2 };
@@ -140,6 +141,35 @@ TP_API void tp_block_destroy(tp_block* blk);
  * borrows the array; recording works inside stream capture. */
 #define TP_BLOCK_STAGES 8
 TP_API int tp_block_set_events(tp_block* blk, void* const* events, int n);
+
+/* One block decode step that allocates nothing (no counterpart in the paper: this
+ * entry point exists for callers, not for the method).
+ *
+ * Some callers cannot hand this library a workspace: a plugin running inside a
+ * host runtime that owns every byte of device memory through its own pool, or a
+ * serving loop that must not call cudaMalloc once it is running (an allocation
+ * there would stall the device or is forbidden by the host's allocator). This
+ * entry point runs the same kernels as tp_block_create + tp_block_forward, with
+ * the same arguments and results, but takes its workspace from one fixed array
+ * of TP_NOALLOC_SCRATCH_BYTES (16 MiB) compiled into the library. Every GPU that
+ * loads the library holds that array until the process exits. Inputs and outputs
+ * are still the caller's: weights, x, the caches and pos as for tp_block_forward.
+ *
+ * - The first call on a device (with that device current) looks up the array's
+ *   device address with cudaGetSymbolAddress; make that first call outside any
+ *   stream capture. The call never allocates memory and frees none.
+ * - Configurations whose tp_block_workspace_bytes exceeds the array are refused
+ *   with TP_ESCRATCH before anything is enqueued (the 7B block at batch 1 needs
+ *   well under 1 MiB; batch 32 of the 70B shape does not fit).
+ * - All calls share the one array, which keeps the previous call's contents; the
+ *   call zeroes the one word that must start at zero (the kernels' error flag)
+ *   on `stream` before its kernels. Calls whose work overlaps on the GPU (other
+ *   streams, other host threads) race on the array: serialise them. */
+#define TP_NOALLOC_SCRATCH_BYTES (16u << 20)
+TP_API int tp_block_forward_noalloc(const tp_dims* dims, int n_slices, int partition,
+                                    int sync_quant, const tp_block_weights* w, float* x,
+                                    void* k_cache, void* v_cache, const int32_t* pos, int batch,
+                                    tp_stream stream);
 
 /* ------------------------------------------------------------------------- */
 /* Partitioned feed-forward layer  Y = act(X W1^T [, X W3^T]) W2^T.            */

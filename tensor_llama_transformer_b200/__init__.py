@@ -20,7 +20,8 @@ if not os.path.exists(LIB_PATH):
         "(there is no fallback implementation)")
 _lib = C.CDLL(LIB_PATH)
 
-TP_OK, TP_EINVAL, TP_EWORKSPACE, TP_EARCH, TP_ECUDA, TP_ENOTSUP, TP_EALIGN = range(7)
+TP_OK, TP_EINVAL, TP_EWORKSPACE, TP_EARCH, TP_ECUDA, TP_ENOTSUP, TP_EALIGN, TP_ESCRATCH = range(8)
+TP_NOALLOC_SCRATCH_BYTES = 16 << 20
 TP_PART_1D, TP_PART_2D = 1, 2
 TP_ACT_RELU, TP_ACT_SWIGLU = 0, 1
 TP_F32, TP_BF16 = 0, 1
@@ -73,6 +74,9 @@ _sig = {
     "tp_model_destroy": (None, [_P]),
     "tp_quantize_q8": (C.c_int, [_P, _P, _P, C.c_int64, _P]),
     "tp_dequantize_q8": (C.c_int, [_P, _P, _P, C.c_int64, _P]),
+    "tp_block_forward_noalloc": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int,
+                                           C.POINTER(tp_block_weights), _P, _P, _P, _P, C.c_int,
+                                           _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -205,3 +209,12 @@ def tp_quantize_q8(x, q, d, n, stream=None):
 def tp_dequantize_q8(q, d, x, n, stream=None):
     _check(_lib.tp_dequantize_q8(_ptr(q), _ptr(d), _ptr(x), n, _stream(stream)),
            "tp_dequantize_q8")
+
+
+def tp_block_forward_noalloc(dims, n_slices, partition, sync_quant, weights, x, k_cache, v_cache,
+                             pos, batch, stream=None):
+    """Block decode step on the library's fixed scratch array (no workspace argument)."""
+    _check(_lib.tp_block_forward_noalloc(C.byref(dims), n_slices, partition, int(sync_quant),
+                                         C.byref(weights), _ptr(x), _ptr(k_cache), _ptr(v_cache),
+                                         _ptr(pos), batch, _stream(stream)),
+           "tp_block_forward_noalloc")

@@ -429,6 +429,7 @@ const char* tp_status_string(int st) {
     case TP_ECUDA: return "CUDA runtime error";
     case TP_ENOTSUP: return "not supported by this build";
     case TP_EALIGN: return "pointer not 16-byte aligned";
+    case TP_ESCRATCH: return "workspace exceeds the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
@@ -495,6 +496,44 @@ int tp_block_set_events(tp_block* blk, void* const* events, int n) {
   blk->events = events;
   return TP_OK;
 }
+
+}  // extern "C"
+
+namespace tp {
+// Forward of one block over a caller-provided workspace using a handle that
+// lives on the stack: no host or device allocation. Same checks as
+// tp_block_create + tp_block_forward; the kernels' error word is zeroed on
+// `stream` first (the workspace may hold an earlier call's contents).
+int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                               const tp_block_weights* w, void* workspace, size_t ws_bytes,
+                               float* x, void* k_cache, void* v_cache, const int32_t* pos,
+                               int batch, cudaStream_t stream) {
+  Cfg c;
+  int rc = check_cfg(dims, n_slices, partition, sync_quant, &c);
+  if (rc) return rc;
+  if (!weights_present(w) || !x || !k_cache || !v_cache || !pos) return TP_EINVAL;
+  if (!weights_aligned(w) || !aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache))
+    return TP_EALIGN;
+  if (batch < 1 || batch > c.d.max_batch) return TP_EINVAL;
+  tp_block blk;
+  blk.c = c;
+  blk.L = block_layout(c);
+  if (!workspace || ws_bytes < blk.L.total) return TP_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return TP_EALIGN;
+  rc = device_check();
+  if (rc) return rc;
+  blk.w = *w;
+  blk.ws = static_cast<uint8_t*>(workspace);
+  blk.ws_bytes = ws_bytes;
+  blk.events = nullptr;
+  if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_ERR], 0, blk.L.size[BUF_ERR], stream) != cudaSuccess)
+    return TP_ECUDA;
+  NormOut none{};
+  return block_forward_impl(&blk, x, k_cache, v_cache, pos, batch, stream, true, none);
+}
+}  // namespace tp
+
+extern "C" {
 
 // ------------------------------------------------------------------ model
 int tp_model_workspace_bytes(const tp_dims* dims, int n_layers, int n_slices, int partition,

@@ -81,4 +81,11 @@ struct AttnArgs {
 
 int launch_attention(const AttnArgs& a, cudaStream_t s);
 
+// One block forward over a caller-provided workspace with a handle on the stack
+// (api.cu); zeroes the kernels' error word in the workspace first.
+int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                               const tp_block_weights* w, void* workspace, size_t ws_bytes,
+                               float* x, void* k_cache, void* v_cache, const int32_t* pos,
+                               int batch, cudaStream_t stream);
+
 }  // namespace tp
