@@ -34,8 +34,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode tokens/s & HBM GB/s per TP-sliced block; FFN TFLOP/s at B=512 (1 B200)"
-STAGES = ["rmsnorm_q8", "qkv_rope", "attention", "wo_partials", "merge_norm", "w13_swiglu",
-          "w2_partials", "merge"]
+STAGES = ["norm_qkv_rope", "attention", "wo_partials", "merge", "norm_w13_swiglu", "w2_partials",
+          "merge2"]
 
 
 def parse_args(argv=None):
@@ -323,15 +323,15 @@ def bench_block(args, world, rank, local):
     step_s = ms_max / 1e3 / K
     hbm, bf16_tf, bf16_sus, peak_kind = peaks()
     w13_bytes = 2 * s.ffn_dim * s.dim * 2 + B * s.dim * (1 + 4 / 32) + B * s.ffn_dim * 4
-    w13_s = stage_ms_max[STAGES.index("w13_swiglu")] / 1e3
-    launches_per_step = 9 * 1  # batch <= 4: one launch per stage (attention = chunks + combine)
+    w13_s = stage_ms_max[STAGES.index("norm_w13_swiglu")] / 1e3
+    launches_per_step = 8  # batch <= 4: one launch per stage, attention = chunks + combine
     res = {
         "tokens_per_s": world * B * K / (ms_max / 1e3), "ms_per_step": ms_max / K, "K": K,
         "block_gbs": (wbytes + kvbytes) / step_s / 1e9, "stage_us": {
             n: v * 1e3 for n, v in zip(STAGES, stage_ms_max)},
         "roofline": {"bound": "hbm", "achieved": w13_bytes / w13_s / 1e9, "peak": hbm,
                      "unit": "GB/s", "frac": w13_bytes / w13_s / 1e9 / hbm, "traffic": None,
-                     "kernel": "k_gemv<1,EPI_SWIGLU> (W1/W3 + SwiGLU)",
+                     "kernel": "k_gemv<1,EPI_SWIGLU,2> (RMSNorm+Q8, W1/W3, SwiGLU)",
                      "algorithmic_bytes": w13_bytes, "peak_kind": peak_kind},
         "e2e": {"value": world * B * E / e2e_s, "unit": "tokens/s",
                 "h2d_bytes_per_step": B * s.dim * 4 + B * 4, "d2h_bytes_per_step": B * s.dim * 4},

@@ -135,11 +135,11 @@ TP_API void tp_block_destroy(tp_block* blk);
  * the caller (timing enabled), or NULL to switch the hook off. While set, each
  * tp_block_forward records events[i] on `stream` just before stage i and
  * events[TP_BLOCK_STAGES] after the last stage (n must be TP_BLOCK_STAGES + 1).
- * Stages: 0 RMSNorm(+Q8), 1 q/k/v products + RoPE + cache write, 2 attention
- * (chunks + combine), 3 W_O partials, 4 merge + FFN RMSNorm, 5 W1/W3 + SwiGLU
- * (2D: stage-1 partials + merge), 6 W2 partials, 7 final merge. The handle
+ * Stages: 0 RMSNorm(+Q8) + q/k/v products + RoPE + cache write, 1 attention
+ * (chunks + combine), 2 W_O partials, 3 merge, 4 RMSNorm(+Q8) + W1/W3 + SwiGLU
+ * (2D: stage-1 partials + their merge), 5 W2 partials, 6 final merge. The handle
  * borrows the array; recording works inside stream capture. */
-#define TP_BLOCK_STAGES 8
+#define TP_BLOCK_STAGES 7
 TP_API int tp_block_set_events(tp_block* blk, void* const* events, int n);
 
 /* One block decode step that allocates nothing (no counterpart in the paper: this

@@ -186,23 +186,22 @@ T* at(const tp_block* b, int buf) {
   return reinterpret_cast<T*>(b->ws + b->L.off[buf]);
 }
 
-NormOut norm_out_for(const tp_block* b, const float* gain) {
-  NormOut no{};
-  no.gain = gain;
-  no.eps = b->c.d.norm_eps;
-  no.quant = b->c.quant;
+// RMSNorm(+Q8) of the residual rows computed in a GEMV's prologue; the first
+// CTA of each segment publishes the shared buffer (Q8 codes + scales, or fp32).
+void set_norm_input(const tp_block* b, GemvArgs& a, const float* x, const float* gain) {
+  a.x = x;
+  a.ldx = b->c.d.dim;
+  a.gain = gain;
+  a.eps = b->c.d.norm_eps;
+  a.quant = b->c.quant;
   if (b->c.quant) {
-    no.xq = at<int8_t>(b, BUF_XQ);
-    no.xd = at<float>(b, BUF_XD);
+    a.xq_out = at<int8_t>(b, BUF_XQ);
+    a.xd_out = at<float>(b, BUF_XD);
   } else {
-    no.xn = at<float>(b, BUF_XN);
+    a.xn_out = at<float>(b, BUF_XN);
   }
-  return no;
 }
 
-// One block forward. `first` launches the attention RMSNorm (otherwise the
-// caller's previous merge already wrote it); `tail` is the RMSNorm fused
-// after the final merge (gain == nullptr: none).
 // Records the caller's timing event before `stage`. Inside stream capture the
 // record must be an external event node (a plain record would only become a
 // dependency edge of the graph and never be timestamped).
@@ -217,28 +216,20 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
   return e == cudaSuccess ? TP_OK : TP_ECUDA;
 }
 
+// One block forward (the distributed-llama root-node order for one layer).
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
-                       cudaStream_t s, bool first, const NormOut& tail) {
+                       cudaStream_t s) {
   const Cfg& c = blk->c;
   const tp_dims& d = c.d;
   const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
   const int QD = H * hd;
   int rc;
-  const bool q = c.quant != 0;
-  const float* xn = at<float>(blk, BUF_XN);
-  const int8_t* xq = at<int8_t>(blk, BUF_XQ);
-  const float* xd = at<float>(blk, BUF_XD);
   float* part = at<float>(blk, BUF_PART);
   float* hbuf = at<float>(blk, BUF_H);
 
-  // a1-a2: RMSNorm (+Q8) into the buffer all slices read
+  // a1-a4: RMSNorm (+Q8, the buffer every slice reads) fused into the q/k/v slice
+  // products, with RoPE and the cache write in the epilogue
   if ((rc = stage_mark(blk, 0, s))) return rc;
-  if (first) {
-    rc = launch_rmsnorm(x, batch, D, norm_out_for(blk, blk->w.attn_norm), s);
-    if (rc) return rc;
-  }
-  // a3-a4: q/k/v slice products with RoPE and the cache write
-  if ((rc = stage_mark(blk, 1, s))) return rc;
   {
     GemvArgs a{};
     a.w[0] = static_cast<const uint16_t*>(blk->w.wq);
@@ -250,11 +241,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.ldw = D;
     a.Ks = D;
     a.nseg = 1;
-    a.x = q ? nullptr : xn;
-    a.xq = q ? xq : nullptr;
-    a.xd = q ? xd : nullptr;
-    a.ldx = D;
-    a.b0 = 0;
+    set_norm_input(blk, a, x, blk->w.attn_norm);
     a.nb = batch;
     a.qout = at<float>(blk, BUF_Q);
     a.kc = static_cast<uint16_t*>(kc);
@@ -265,11 +252,10 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.max_seq = d.max_seq;
     a.theta = d.rope_theta;
     a.ctas_per_seg = ctas_for(1, (QD + 2 * Hkv * hd) / 2);
-    rc = launch_gemv(a, EPI_QKV, s);
-    if (rc) return rc;
+    if ((rc = launch_gemv(a, EPI_QKV, s))) return rc;
   }
-  // a4: attention per head slice
-  if ((rc = stage_mark(blk, 2, s))) return rc;
+  // a4: attention per head slice (context chunks, then their combination)
+  if ((rc = stage_mark(blk, 1, s))) return rc;
   {
     AttnArgs a{};
     a.q = at<float>(blk, BUF_Q);
@@ -285,11 +271,10 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.part_ml = at<float>(blk, BUF_PML);
     a.att = at<float>(blk, BUF_ATT);
     a.err = at<int>(blk, BUF_ERR);
-    rc = launch_attention(a, s);
-    if (rc) return rc;
+    if ((rc = launch_attention(a, s))) return rc;
   }
-  // a5: W_O row-split partials, one per slice
-  if ((rc = stage_mark(blk, 3, s))) return rc;
+  // a5: W_O row-split partials, one plane per slice
+  if ((rc = stage_mark(blk, 2, s))) return rc;
   {
     GemvArgs a{};
     a.w[0] = static_cast<const uint16_t*>(blk->w.wo);
@@ -304,15 +289,13 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.out_seg = (int64_t)batch * D;
     a.ldo = D;
     a.ctas_per_seg = ctas_for(c.n, D / 2);
-    rc = launch_gemv(a, EPI_PLAIN, s);
-    if (rc) return rc;
+    if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
   }
-  // a6-a7: merge (dequantise + slice-order sum + residual) and the FFN RMSNorm
+  // a6: sync + dequantise + merge into the residual
+  if ((rc = stage_mark(blk, 3, s))) return rc;
+  if ((rc = launch_merge(x, part, c.n, batch, D, c.quant, s))) return rc;
+  // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
   if ((rc = stage_mark(blk, 4, s))) return rc;
-  rc = launch_merge(x, part, c.n, batch, D, c.quant, norm_out_for(blk, blk->w.ffn_norm), s);
-  if (rc) return rc;
-  // a8: W1/W3 slice products and SwiGLU
-  if ((rc = stage_mark(blk, 5, s))) return rc;
   if (c.partition == TP_PART_1D) {
     GemvArgs a{};
     a.w[0] = static_cast<const uint16_t*>(blk->w.w1);
@@ -321,19 +304,14 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.ldw = D;
     a.Ks = D;
     a.nseg = 1;
-    a.x = q ? nullptr : xn;
-    a.xq = q ? xq : nullptr;
-    a.xd = q ? xd : nullptr;
-    a.ldx = D;
+    set_norm_input(blk, a, x, blk->w.ffn_norm);
     a.nb = batch;
     a.out = hbuf;
-    a.out_seg = 0;
     a.ldo = F;
     a.ctas_per_seg = ctas_for(1, F);
-    rc = launch_gemv(a, EPI_SWIGLU, s);
-    if (rc) return rc;
+    if ((rc = launch_gemv(a, EPI_SWIGLU, s))) return rc;
   } else {
-    // 2D stage 1: partial sums over the gx dim-slices for W1 and W3, merged with SwiGLU
+    // 2D stage 1: partials over the gx dim-slices for W1 and W3, merged with SwiGLU
     float* pa = at<float>(blk, BUF_PA);
     float* pb = at<float>(blk, BUF_PB);
     for (int m = 0; m < 2; ++m) {
@@ -343,17 +321,13 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.ldw = D;
       a.Ks = D / c.gx;
       a.nseg = c.gx;
-      a.x = q ? nullptr : xn;
-      a.xq = q ? xq : nullptr;
-      a.xd = q ? xd : nullptr;
-      a.ldx = D;
+      set_norm_input(blk, a, x, blk->w.ffn_norm);
       a.nb = batch;
       a.out = m == 0 ? pa : pb;
       a.out_seg = (int64_t)batch * F;
       a.ldo = F;
       a.ctas_per_seg = ctas_for(c.gx, F / 2);
-      rc = launch_gemv(a, EPI_PLAIN, s);
-      if (rc) return rc;
+      if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
     FfnMergeArgs m{};
     m.P1 = pa;
@@ -365,11 +339,10 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     m.quant = c.quant;
     m.act = ACT_SWIGLU;
     m.out_f32 = hbuf;
-    rc = launch_ffn_merge(m, s);
-    if (rc) return rc;
+    if ((rc = launch_ffn_merge(m, s))) return rc;
   }
   // a9: W2 row-split partials
-  if ((rc = stage_mark(blk, 6, s))) return rc;
+  if ((rc = stage_mark(blk, 5, s))) return rc;
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
   {
     GemvArgs a{};
@@ -385,13 +358,11 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.out_seg = (int64_t)batch * D;
     a.ldo = D;
     a.ctas_per_seg = ctas_for(nseg2, D / 2);
-    rc = launch_gemv(a, EPI_PLAIN, s);
-    if (rc) return rc;
+    if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
   }
-  // a10: merge (+ the next sublayer's norm when fused by the caller)
-  if ((rc = stage_mark(blk, 7, s))) return rc;
-  rc = launch_merge(x, part, nseg2, batch, D, c.quant, tail, s);
-  if (rc) return rc;
+  // a10: sync + dequantise + merge
+  if ((rc = stage_mark(blk, 6, s))) return rc;
+  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -477,8 +448,7 @@ int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, cons
   if (!blk || !x || !k_cache || !v_cache || !pos) return TP_EINVAL;
   if (batch < 1 || batch > blk->c.d.max_batch) return TP_EINVAL;
   if (!aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache)) return TP_EALIGN;
-  NormOut none{};
-  return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream, true, none);
+  return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream);
 }
 
 int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* bytes) {
@@ -528,8 +498,7 @@ int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition,
   blk.events = nullptr;
   if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_ERR], 0, blk.L.size[BUF_ERR], stream) != cudaSuccess)
     return TP_ECUDA;
-  NormOut none{};
-  return block_forward_impl(&blk, x, k_cache, v_cache, pos, batch, stream, true, none);
+  return block_forward_impl(&blk, x, k_cache, v_cache, pos, batch, stream);
 }
 }  // namespace tp
 
@@ -604,29 +573,25 @@ int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_
   const size_t layer_elems =
       (size_t)d.max_batch * d.n_kv_heads * (size_t)d.max_seq * d.head_dim;
   for (int l = 0; l < m->n_layers; ++l) {
-    tp_block* b = &m->blocks[l];
-    NormOut tail{};
-    if (l + 1 < m->n_layers) {
-      tail = norm_out_for(&m->blocks[l + 1], m->blocks[l + 1].w.attn_norm);
-    } else {
-      tail.gain = m->final_norm;
-      tail.eps = d.norm_eps;
-      tail.quant = 0;
-      tail.xn = m->xnf;
-    }
     uint16_t* kc = static_cast<uint16_t*>(k_cache) + (size_t)l * layer_elems;
     uint16_t* vc = static_cast<uint16_t*>(v_cache) + (size_t)l * layer_elems;
-    int rc = block_forward_impl(b, m->x, kc, vc, pos, batch, s, l == 0, tail);
+    int rc = block_forward_impl(&m->blocks[l], m->x, kc, vc, pos, batch, s);
     if (rc) return rc;
   }
+  // RmsFinal(Norm) fused into the logits GEMV; the vocab column split writes each
+  // slice's range of the output in place (the MergeLogits concatenation)
   GemvArgs a{};
   a.w[0] = static_cast<const uint16_t*>(m->wcls);
   a.rows[0] = d.vocab;
   a.ldw = d.dim;
   a.Ks = d.dim;
   a.nseg = 1;
-  a.x = m->xnf;
+  a.x = m->x;
   a.ldx = d.dim;
+  a.gain = m->final_norm;
+  a.eps = d.norm_eps;
+  a.quant = 0;
+  a.xn_out = m->xnf;
   a.nb = batch;
   a.out = logits;
   a.ldo = d.vocab;

@@ -5,26 +5,9 @@
 
 namespace tp {
 
-// ------------------------------------------------------------------ RMSNorm (+Q8)
-// x [B, dim] -> normalised rows. Outputs (each nullable):
-//   xn  float32 [B, dim]  (the value the consumers read when quantisation is off)
-//   xq  int8 [B, dim] + xd float32 [B, dim/32]  (Q8 sync buffer)
-//   xb  bf16 [B, dim]     (the consumers' value rounded to bf16, for tensor-core paths)
-struct NormOut {
-  float* xn;
-  int8_t* xq;
-  float* xd;
-  uint16_t* xb;
-  const float* gain;
-  float eps;
-  int quant;
-};
-
-// Merge of n row-split partials [n, B, dim] into the residual x, then an optional
-// RMSNorm of the merged rows for the next sublayer (norm.gain == nullptr: none).
-int launch_rmsnorm(const float* x, int B, int dim, const NormOut& no, cudaStream_t s);
-int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, const NormOut& no,
-                 cudaStream_t s);
+// ------------------------------------------------------------------ merge / codec
+// x[b] += sum_{s<n} sync(part[s][b]) in slice order; part is [n, B, dim].
+int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, cudaStream_t s);
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s);
 int launch_dequantize(const int8_t* q, const float* d, float* x, int64_t n, cudaStream_t s);
 
@@ -39,11 +22,20 @@ struct GemvArgs {
   int64_t ldw;   // row stride in elements (= full input width K)
   int Ks;        // contraction length of one segment
   int nseg;      // number of segments: segment s reads columns [s*Ks, (s+1)*Ks)
-  // input: float32 x [B, ldx] or Q8 (xq [B, ldx], xd [B, ldx/32])
+  // input: float32 x [B, ldx] or Q8 (xq [B, ldx], xd [B, ldx/32]); with `gain`
+  // set, x is a residual and the input is RMSNorm(x) * gain (+Q8 when quant),
+  // computed in the prologue; the first CTA of each segment then writes the
+  // shared buffer (xq_out/xd_out for Q8, xn_out for float32; each nullable).
   const float* x;
   const int8_t* xq;
   const float* xd;
   int ldx;
+  const float* gain;
+  float eps;
+  int quant;
+  int8_t* xq_out;
+  float* xd_out;
+  float* xn_out;
   int b0, nb;    // batch rows [b0, b0+nb) handled by this launch
   // EPI_PLAIN / EPI_SWIGLU output: out[seg*out_seg + b*ldo + row]
   float* out;

@@ -1,0 +1,99 @@
+// The cross-slice merge and the standalone Q8 codec.
+//
+// distributed-llama issue #29: llamaDequantizeAtt + llamaMergeAtt (and the Ffn2
+// twins) sum the slices' partial outputs into the residual. Here one launch
+// does both for every element: each partial passes through the sync buffer's
+// format (the Q8 round trip when quantisation is on), the partials are summed
+// in slice order 0..n-1 in float32, and the sum is added to x. The grid covers
+// the batch rows in 512-element pieces so that the merge of a single token is
+// spread over many SMs instead of waiting on one.
+#include "kernels.cuh"
+
+namespace tp {
+
+namespace {
+
+constexpr int kMergeThreads = 128;  // 4 values per thread: 512 values per CTA
+
+__global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
+                                                         const float* __restrict__ part, int n,
+                                                         int B, int dim, int quant) {
+  const int b = blockIdx.y;
+  const int i4 = blockIdx.x * kMergeThreads + threadIdx.x;  // float4 index within the row
+  const int n4 = dim >> 2;
+  // whole warps stay in the loop so that an 8-lane Q8 group is always complete
+  const bool in = i4 < n4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n; ++s) {
+    float4 p = in ? reinterpret_cast<const float4*>(part + ((size_t)s * B + b) * dim)[i4]
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (quant) q8_roundtrip4(p);
+    acc.x += p.x;
+    acc.y += p.y;
+    acc.z += p.z;
+    acc.w += p.w;
+  }
+  if (in) {
+    float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim);
+    float4 v = xr[i4];
+    v.x += acc.x;
+    v.y += acc.y;
+    v.z += acc.z;
+    v.w += acc.w;
+    xr[i4] = v;
+  }
+}
+
+__global__ void k_quantize(const float* __restrict__ x, int8_t* __restrict__ q,
+                           float* __restrict__ d, int64_t n) {
+  const int64_t n4 = n >> 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t n4r = (n4 + 31) & ~(int64_t)31;
+  for (int64_t i4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4r; i4 += stride) {
+    const bool in = i4 < n4;
+    float4 v = in ? reinterpret_cast<const float4*>(x)[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const uint32_t codes = q8_quantize4(v, in ? d + (i4 >> 3) : nullptr);
+    if (in) reinterpret_cast<uint32_t*>(q)[i4] = codes;
+  }
+}
+
+__global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restrict__ d,
+                             float* __restrict__ x, int64_t n) {
+  const int64_t n4 = n >> 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4; i4 += stride) {
+    const uint32_t c = reinterpret_cast<const uint32_t*>(q)[i4];
+    reinterpret_cast<float4*>(x)[i4] = q8_unpack4(c, d[i4 >> 3]);
+  }
+}
+
+}  // namespace
+
+int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, cudaStream_t s) {
+  const dim3 grid((dim / 4 + kMergeThreads - 1) / kMergeThreads, B);
+  k_merge<<<grid, kMergeThreads, 0, s>>>(x, part, n, B, dim, quant);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s) {
+  if (n == 0) return TP_OK;
+  const int threads = 256;
+  int64_t blocks = ((n >> 2) + threads - 1) / threads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_quantize<<<(unsigned)blocks, threads, 0, s>>>(x, q, d, n);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+int launch_dequantize(const int8_t* q, const float* d, float* x, int64_t n, cudaStream_t s) {
+  if (n == 0) return TP_OK;
+  const int threads = 256;
+  int64_t blocks = ((n >> 2) + threads - 1) / threads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_dequantize<<<(unsigned)blocks, threads, 0, s>>>(q, d, x, n);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+}  // namespace tp
