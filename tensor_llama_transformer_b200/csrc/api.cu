@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/tp_block.h: argument checks,
 // workspace layout and the launch sequence of a block, a model and an FFN.
+#include <cstdlib>
 #include <mutex>
 #include <new>
 
@@ -56,6 +57,14 @@ int set_smem_once(const void* kernel, int bytes) {
   return TP_OK;
 }
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("TP_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 int num_sms() {
   int dev = 0;
   cudaGetDevice(&dev);
@@ -70,7 +79,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // ------------------------------------------------------------------ block layout
 enum Buf {
   BUF_XQ = 0, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H, BUF_ERR, BUF_PO, BUF_PML,
-  BUF_PA, BUF_PB, BUF_COUNT
+  BUF_PA, BUF_PB, BUF_SSQ, BUF_COUNT
 };
 
 struct Layout {
@@ -137,6 +146,7 @@ Layout block_layout(const Cfg& c) {
   const size_t pa = c.partition == TP_PART_2D ? (size_t)c.gx * B * F * 4 : 0;
   L.size[BUF_PA] = pa;
   L.size[BUF_PB] = pa;
+  L.size[BUF_SSQ] = B * (size_t)merge_ssq_parts(c.d.dim) * 4;
   size_t o = 0;
   for (int i = 0; i < BUF_COUNT; ++i) {
     L.off[i] = o;
@@ -217,8 +227,11 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
 }
 
 // One block forward (the distributed-llama root-node order for one layer).
+// chained: x was produced by the previous block's final merge of this same
+// launch sequence, which left the row sums of squares in the workspace (inside
+// a model); the final merge here leaves them for the next block.
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
-                       cudaStream_t s) {
+                       cudaStream_t s, bool chained = false) {
   const Cfg& c = blk->c;
   const tp_dims& d = c.d;
   const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
@@ -242,6 +255,10 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.Ks = D;
     a.nseg = 1;
     set_norm_input(blk, a, x, blk->w.attn_norm);
+    if (chained) {
+      a.ssq = at<float>(blk, BUF_SSQ);
+      a.ssq_parts = merge_ssq_parts(D);
+    }
     a.nb = batch;
     a.qout = at<float>(blk, BUF_Q);
     a.kc = static_cast<uint16_t*>(kc);
@@ -251,7 +268,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.n_kv_heads = Hkv;
     a.max_seq = d.max_seq;
     a.theta = d.rope_theta;
-    a.ctas_per_seg = ctas_for(1, (QD + 2 * Hkv * hd) / 2);
+    a.err = at<int>(blk, BUF_ERR);
     if ((rc = launch_gemv(a, EPI_QKV, s))) return rc;
   }
   // a4: attention per head slice (context chunks, then their combination)
@@ -288,12 +305,12 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.out = part;
     a.out_seg = (int64_t)batch * D;
     a.ldo = D;
-    a.ctas_per_seg = ctas_for(c.n, D / 2);
+    a.err = at<int>(blk, BUF_ERR);
     if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
   }
   // a6: sync + dequantise + merge into the residual
   if ((rc = stage_mark(blk, 3, s))) return rc;
-  if ((rc = launch_merge(x, part, c.n, batch, D, c.quant, s))) return rc;
+  if ((rc = launch_merge(x, part, c.n, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
   // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
   if ((rc = stage_mark(blk, 4, s))) return rc;
   if (c.partition == TP_PART_1D) {
@@ -305,10 +322,12 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.Ks = D;
     a.nseg = 1;
     set_norm_input(blk, a, x, blk->w.ffn_norm);
+    a.ssq = at<float>(blk, BUF_SSQ);  // written by the merge just above
+    a.ssq_parts = merge_ssq_parts(D);
     a.nb = batch;
     a.out = hbuf;
     a.ldo = F;
-    a.ctas_per_seg = ctas_for(1, F);
+    a.err = at<int>(blk, BUF_ERR);
     if ((rc = launch_gemv(a, EPI_SWIGLU, s))) return rc;
   } else {
     // 2D stage 1: partials over the gx dim-slices for W1 and W3, merged with SwiGLU
@@ -322,11 +341,13 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.Ks = D / c.gx;
       a.nseg = c.gx;
       set_norm_input(blk, a, x, blk->w.ffn_norm);
+      a.ssq = at<float>(blk, BUF_SSQ);
+      a.ssq_parts = merge_ssq_parts(D);
       a.nb = batch;
       a.out = m == 0 ? pa : pb;
       a.out_seg = (int64_t)batch * F;
       a.ldo = F;
-      a.ctas_per_seg = ctas_for(c.gx, F / 2);
+      a.err = at<int>(blk, BUF_ERR);
       if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
     FfnMergeArgs m{};
@@ -357,17 +378,19 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.out = part;
     a.out_seg = (int64_t)batch * D;
     a.ldo = D;
-    a.ctas_per_seg = ctas_for(nseg2, D / 2);
+    a.err = at<int>(blk, BUF_ERR);
     if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
   }
   // a10: sync + dequantise + merge
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, s))) return rc;
+  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
 __global__ void k_embed(const uint16_t* __restrict__ emb, const int32_t* __restrict__ tok, int dim,
                         float* __restrict__ x) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.x;
   const uint16_t* row = emb + (size_t)tok[b] * dim;
   for (int i = threadIdx.x; i < dim; i += blockDim.x)
@@ -568,14 +591,15 @@ int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits)) return TP_EALIGN;
   cudaStream_t s = (cudaStream_t)stream;
   const tp_dims& d = m->d;
-  k_embed<<<batch, 256, 0, s>>>(static_cast<const uint16_t*>(m->embed), tokens, d.dim, m->x);
-  TP_LAUNCH_CHECK();
+  int rc0 = launch_pdl(k_embed, dim3(batch), dim3(256), 0, s,
+                       static_cast<const uint16_t*>(m->embed), tokens, (int)d.dim, m->x);
+  if (rc0) return rc0;
   const size_t layer_elems =
       (size_t)d.max_batch * d.n_kv_heads * (size_t)d.max_seq * d.head_dim;
   for (int l = 0; l < m->n_layers; ++l) {
     uint16_t* kc = static_cast<uint16_t*>(k_cache) + (size_t)l * layer_elems;
     uint16_t* vc = static_cast<uint16_t*>(v_cache) + (size_t)l * layer_elems;
-    int rc = block_forward_impl(&m->blocks[l], m->x, kc, vc, pos, batch, s);
+    int rc = block_forward_impl(&m->blocks[l], m->x, kc, vc, pos, batch, s, l > 0);
     if (rc) return rc;
   }
   // RmsFinal(Norm) fused into the logits GEMV; the vocab column split writes each
@@ -595,7 +619,7 @@ int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_
   a.nb = batch;
   a.out = logits;
   a.ldo = d.vocab;
-  a.ctas_per_seg = ctas_for(1, d.vocab / 2);
+  a.err = at<int>(&m->blocks[0], BUF_ERR);
   return launch_gemv(a, EPI_PLAIN, s);
 }
 

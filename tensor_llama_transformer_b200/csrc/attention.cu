@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_chunk(AttnArgs a) {
 
   const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();  // q and the cache row at pos come from the q/k/v kernel
   const int P = a.pos[b] + 1;
   const int t0 = c * kAttnChunk;
   const size_t pbase = ((size_t)b * a.H + (size_t)kvh * G) * a.nchunk + c;
@@ -178,6 +180,8 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_chunk(AttnArgs a) {
 
 // One CTA per (head, batch row); thread d owns output dimension d.
 __global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int P = a.pos[b] + 1;
   const int nc = (P + kAttnChunk - 1) / kAttnChunk;
@@ -201,10 +205,7 @@ int launch_g(const AttnArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)2 * kAttnChunk * kHeadDim * 2 + (size_t)G * kHeadDim * 4 +
                       (size_t)G * kAttnChunk * 4 + (size_t)2 * G * 4 * 4;
   if (set_smem_once((const void*)k_attn_chunk<G>, (int)smem)) return TP_ECUDA;
-  dim3 grid(a.nchunk, a.Hkv, a.B);
-  k_attn_chunk<G><<<grid, kAttnThreads, smem, s>>>(a);
-  TP_LAUNCH_CHECK();
-  return TP_OK;
+  return launch_pdl(k_attn_chunk<G>, dim3(a.nchunk, a.Hkv, a.B), dim3(kAttnThreads), smem, s, a);
 }
 
 }  // namespace
@@ -220,9 +221,7 @@ int launch_attention(const AttnArgs& a, cudaStream_t s) {
     default: return TP_ENOTSUP;
   }
   if (rc != TP_OK) return rc;
-  k_attn_combine<<<dim3(a.H, a.B), kHeadDim, 0, s>>>(a);
-  TP_LAUNCH_CHECK();
-  return TP_OK;
+  return launch_pdl(k_attn_combine, dim3(a.H, a.B), dim3(kHeadDim), 0, s, a);
 }
 
 }  // namespace tp

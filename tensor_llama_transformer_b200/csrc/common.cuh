@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/tp_block.h"
 
 #define TP_DEV __device__ __forceinline__
@@ -119,6 +121,15 @@ TP_DEV float4 q8_unpack4(uint32_t codes, float d) {
   return r;
 }
 
+// ---------------------------------------------------------------- PDL
+// Programmatic dependent launch: a kernel lets the next kernel of the stream be
+// scheduled as soon as all its CTAs have started (launch_dependents), and a
+// kernel waits for its predecessor's completion and memory (wait) only where it
+// first touches data the predecessor produced. Work before the wait may only
+// read inputs no earlier kernel writes (weights, pos, cache rows before pos).
+TP_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+TP_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace tp
 
 // ---------------------------------------------------------------- host side
@@ -135,6 +146,29 @@ TP_DEV float4 q8_unpack4(uint32_t codes, float d) {
 
 namespace tp {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Whether launches carry the programmatic-serialization attribute (default on;
+// the environment variable TP_PDL=0 turns it off, for comparison runs).
+bool pdl_enabled();
+
+// Launches `kernel` on `s`, allowing it to overlap its predecessor's tail
+// (programmatic dependent launch) when pdl_enabled().
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? TP_OK
+                                                                                       : TP_ECUDA;
+}
 int device_check();   // TP_OK if the current device is sm_100 (cached per device)
 int num_sms();        // SM count of the current device (cached)
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device); later

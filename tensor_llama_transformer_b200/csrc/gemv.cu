@@ -1,4 +1,4 @@
-// Weight-streaming slice GEMV for decode (small batch).
+// Weight-streaming slice GEMV for decode (batch 1 or 2 per launch).
 //
 //   out[seg, b, r] = sum_{k < Ks} W[r, seg*Ks + k] * x[b, seg*Ks + k]
 //
@@ -9,265 +9,399 @@
 //     range of every row and writes its own partial [B, rows] of the all-reduce
 //     (aiterms.tw "Tensor Parallelism": Linear2 split by rows needs a reduction).
 //
-// Work split. The kernel is bound by the weight stream, so every SM must stream
-// the same bytes until the end. Rows are handled in pairs (a RoPE pair of q/k,
-// row f of W1 with row f of W3, or two consecutive rows) and each CTA owns a
-// contiguous, equal share of the pairs of one segment. Inside a CTA the 8
-// warps split the contraction of every pair: warp w streams the same column
-// range of each row, 16 bytes per lane per load, with the activations of that
-// range held in registers. Each warp reduces its partial dot products with
-// shuffles and leaves them in shared memory; after the last pair the CTA adds
-// the 8 warps' partials in a fixed order and runs the epilogue.
+// Structure (one persistent CTA per SM). The rows of all segments form one list
+// of row pairs (a RoPE pair of q/k, row f of W1 with row f of W3, or two
+// consecutive rows); every CTA owns a contiguous, equal share of the pairs, so
+// every SM streams the same bytes. A producer warp copies the CTA's rows into a
+// ring of shared-memory stages with bulk asynchronous copies (cp.async.bulk),
+// completion counted on one mbarrier per stage; a stage holds one row pair for
+// each of the NC consumer warps and never crosses a segment boundary, and the
+// ring keeps 100-200 KB per SM in flight. A consumer warp dots its pair with the
+// activations (staged once per segment in shared memory, float32), reduces the
+// two sums across the warp with shuffles, and hands the stage back with an
+// mbarrier arrive. The producer only reads weights, which no kernel writes, so
+// under programmatic dependent launch it starts streaming while the previous
+// kernel finishes; the consumers wait for that kernel before reading the
+// activations. Every mbarrier wait is bounded (2 s) and sets the error flag
+// instead of hanging.
 //
-// Input modes: float32 activations; Q8 codes + scales (dequantised on load);
-// or the RMSNorm of a float32 residual computed in the prologue (each CTA
-// reduces the whole row for the scale, then normalises, and with Q8 quantises,
-// only its warps' column ranges; the first CTA of each segment also writes the
-// normalised / quantised buffer that the slices share).
+// Input modes: float32 activations; Q8 codes + scales (dequantised while
+// staging); or the RMSNorm of a float32 residual computed while staging (each
+// CTA reduces the whole row for the scale; with Q8 the normalised values pass
+// through the int8 block format, and the CTA that owns the first row of a
+// segment also writes the shared int8 (or float32) buffer of that segment).
 //
-// Epilogues: EPI_PLAIN stores (partials, logits); EPI_SWIGLU stores silu(a)*b
-// (llamaFfn); EPI_QKV applies RoPE to q and k row pairs, stores rotated q, and
-// writes k and v into the bf16 cache at pos (llamaMultiheadAtt's "merge kv-cache,
-// add RoPE encoding").
+// Epilogues (after the last stage): EPI_PLAIN stores partials or logits;
+// EPI_SWIGLU stores silu(a)*b (llamaFfn); EPI_QKV applies RoPE to q and k
+// pairs, stores rotated q, and writes k and v into the bf16 cache at pos
+// (llamaMultiheadAtt's "merge kv-cache, add RoPE encoding").
 #include "kernels.cuh"
 
 namespace tp {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kMaxStages = 16;
+constexpr int kSmemBudget = 222 * 1024;
 
-TP_DEV float dot8(const uint4 w, const float* x) {
-  float a = bf16lo(w.x) * x[0];
-  a = fmaf(bf16hi(w.x), x[1], a);
-  a = fmaf(bf16lo(w.y), x[2], a);
-  a = fmaf(bf16hi(w.y), x[3], a);
-  a = fmaf(bf16lo(w.z), x[4], a);
-  a = fmaf(bf16hi(w.z), x[5], a);
-  a = fmaf(bf16lo(w.w), x[6], a);
-  a = fmaf(bf16hi(w.w), x[7], a);
-  return a;
+TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+TP_DEV uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+TP_DEV void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
+}
+TP_DEV void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
+               : "memory");
+}
+TP_DEV void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
+}
+TP_DEV bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(s2u(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(b, parity)) return true;
+    if ((i & 255) == 0 && gtimer() - t0 > kTimeoutNs) {
+      if (err) atomicExch(err, 1);
+      return false;
+    }
+  }
+}
+TP_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          s2u(dst)),
+      "l"(src), "r"(bytes), "r"(s2u(bar))
+      : "memory");
+}
+// Named barrier 1 among the consumer warps only (the producer never joins it).
+TP_DEV void consumers_sync(int nthreads) { asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); }
+
+// acc (two float32 lanes as one 64-bit register pair) += the 8 bf16 weights of
+// w times the 8 activations (lo = elements 0..3, hi = 4..7), two weights per
+// packed fma.rn.f32x2: lane 0 of acc collects the even elements, lane 1 the odd.
+TP_DEV void fma8(uint64_t& acc, const uint4 w, const float4 lo, const float4 hi) {
+  const uint64_t x01 = ((uint64_t)__float_as_uint(lo.y) << 32) | __float_as_uint(lo.x);
+  const uint64_t x23 = ((uint64_t)__float_as_uint(lo.w) << 32) | __float_as_uint(lo.z);
+  const uint64_t x45 = ((uint64_t)__float_as_uint(hi.y) << 32) | __float_as_uint(hi.x);
+  const uint64_t x67 = ((uint64_t)__float_as_uint(hi.w) << 32) | __float_as_uint(hi.z);
+  asm("{\n .reg .b64 w;\n"
+      " mov.b64 w, {%5, %6};  fma.rn.f32x2 %0, w, %1, %0;\n"
+      " mov.b64 w, {%7, %8};  fma.rn.f32x2 %0, w, %2, %0;\n"
+      " mov.b64 w, {%9, %10}; fma.rn.f32x2 %0, w, %3, %0;\n"
+      " mov.b64 w, {%11, %12}; fma.rn.f32x2 %0, w, %4, %0;\n}"
+      : "+l"(acc)
+      : "l"(x01), "l"(x23), "l"(x45), "l"(x67), "r"(w.x << 16), "r"(w.x & 0xFFFF0000u),
+        "r"(w.y << 16), "r"(w.y & 0xFFFF0000u), "r"(w.z << 16), "r"(w.z & 0xFFFF0000u),
+        "r"(w.w << 16), "r"(w.w & 0xFFFF0000u));
 }
 
-// The warp's column range, in 16-byte vectors, aligned to 4-vector groups so
-// that a 32-value quantisation block never straddles two warps.
-TP_DEV void warp_range(int nv, int w, int& vb, int& ve) {
-  const int ng = nv >> 2;
-  vb = ((ng * w) / kWarps) * 4;
-  ve = ((ng * (w + 1)) / kWarps) * 4;
+TP_DEV float hsum2(uint64_t acc) {
+  return __uint_as_float((uint32_t)acc) + __uint_as_float((uint32_t)(acc >> 32));
 }
 
-// Row pointers of pair p of the segment (see GemvArgs): r0 and r1.
 template <int EPI>
-TP_DEV void pair_rows(const GemvArgs& a, int p, size_t col0, const uint16_t*& r0,
-                      const uint16_t*& r1, int& mat, int& lrow) {
+TP_DEV int rows_per_seg(const GemvArgs& a) {
+  if (EPI == EPI_SWIGLU) return 2 * a.rows[0];
+  if (EPI == EPI_QKV) return a.rows[0] + a.rows[1] + a.rows[2];
+  return a.rows[0];
+}
+
+// Global address of virtual row `r` of segment `seg`; mat/lrow name the matrix
+// and its row (SwiGLU interleaves row f of W1 and row f of W3).
+template <int EPI>
+TP_DEV const uint16_t* row_ptr(const GemvArgs& a, int seg, int r, int& mat, int& lrow) {
   mat = 0;
   if (EPI == EPI_SWIGLU) {
-    r0 = a.w[0] + (size_t)p * a.ldw + col0;
-    r1 = a.w[1] + (size_t)p * a.ldw + col0;
-    lrow = p;
+    mat = r & 1;
+    lrow = r >> 1;
   } else {
-    int row = 2 * p;
-    if (EPI == EPI_QKV && row >= a.rows[0]) {
-      row -= a.rows[0];
+    lrow = r;
+    if (EPI == EPI_QKV && lrow >= a.rows[0]) {
+      lrow -= a.rows[0];
       mat = 1;
-      if (row >= a.rows[1]) {
-        row -= a.rows[1];
+      if (lrow >= a.rows[1]) {
+        lrow -= a.rows[1];
         mat = 2;
       }
     }
-    lrow = row;
-    r0 = a.w[mat] + (size_t)row * a.ldw + col0;
-    r1 = r0 + a.ldw;
   }
+  return a.w[mat] + (size_t)lrow * a.ldw + (size_t)seg * a.Ks;
 }
 
-template <int NB, int EPI, int VPL>
-__global__ void __launch_bounds__(kThreads) k_gemv(GemvArgs a) {
-  constexpr int U = VPL == 1 ? 4 : (VPL == 2 ? 2 : 1);  // pairs in flight per warp
-  extern __shared__ float red[];                        // [pairs][kWarps][2][NB]
+// Next stage of a CTA's row range: rows [cur, end) with end - cur <= 2*P (P row
+// pairs per stage) and no segment boundary inside. Producer and consumers walk
+// the same sequence.
+TP_DEV int stage_end(int cur, int nrows, int R0, int rps, int P) {
+  const int g = R0 + cur;
+  const int seg_end = (g / rps + 1) * rps - R0;
+  return min(min(nrows, seg_end), cur + 2 * P);
+}
+
+template <int NB, int EPI>
+__global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_rstd[NB];
-  const int seg = blockIdx.x / a.ctas_per_seg;
-  const int cta = blockIdx.x - seg * a.ctas_per_seg;
+  __shared__ float s_red[8][NB];
+  const int nc = pl.nc, nstage = pl.nstage, P = pl.pairs, Q = pl.split;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nv = a.Ks >> 3;
-  int vb, ve;
-  warp_range(nv, warp, vb, ve);
-  const size_t col0 = (size_t)seg * a.Ks;
+  const int nv = a.Ks >> 3;  // 16-byte vectors per row
+  const uint32_t row_bytes = (uint32_t)a.Ks * 2;
+  uint8_t* ring = smem + pl.ring_off;
+  float4* xs = reinterpret_cast<float4*>(smem + pl.x_off);  // lo[NB][nv] then hi[NB][nv]
+  float* res = reinterpret_cast<float*>(smem + pl.res_off);  // [rows of this CTA][NB]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.bar_off);
+  uint64_t* empty = full + kMaxStages;
 
-  // ---------------------------------------------------------------- activations
-  float xr[NB][VPL][8];
-  if (a.gain) {  // RMSNorm of the residual rows (+Q8)
-    const int D = a.ldx;
-    float ss[NB];
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      ss[b] = 0.f;
-      if (b < a.nb) {
-        const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
-        for (int i = threadIdx.x; i < (D >> 2); i += kThreads) {
-          const float4 v = xrow[i];
-          ss[b] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-        }
-      }
-      ss[b] = warp_sum(ss[b]);
+  const int rps = rows_per_seg<EPI>(a);
+  const int npairs = a.nseg * (rps >> 1);
+  const int P0 = (int)(((int64_t)npairs * blockIdx.x) / gridDim.x);
+  const int P1 = (int)(((int64_t)npairs * (blockIdx.x + 1)) / gridDim.x);
+  const int R0 = 2 * P0, nrows = 2 * (P1 - P0);  // flattened rows [R0, R0 + nrows)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < nstage; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], nc);
     }
-    if (lane == 0)
-#pragma unroll
-      for (int b = 0; b < NB; ++b) red[warp * NB + b] = ss[b];
-    __syncthreads();
-    if (threadIdx.x < NB) {
-      float t = 0.f;
-      for (int w = 0; w < kWarps; ++w) t += red[w * NB + threadIdx.x];
-      s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)D + a.eps);
-    }
-    __syncthreads();
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const bool writer = cta == 0;  // first CTA of the segment publishes the shared buffer
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      const int v = vb + lane + 32 * j;
-      float* xv = xr[b][j];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) xv[e] = 0.f;
-      const bool in = b < a.nb && v < ve;
-      const size_t e0 = (size_t)(a.b0 + b) * a.ldx + col0 + 8 * (size_t)v;
-      if (a.gain) {
-        if (in) {
-          const float rstd = s_rstd[b];
-          const float4 x0 = *reinterpret_cast<const float4*>(a.x + e0);
-          const float4 x1 = *reinterpret_cast<const float4*>(a.x + e0 + 4);
-          const float4 g0 = *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v);
-          const float4 g1 = *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v + 4);
-          xv[0] = __fmul_rn(__fmul_rn(x0.x, rstd), g0.x);
-          xv[1] = __fmul_rn(__fmul_rn(x0.y, rstd), g0.y);
-          xv[2] = __fmul_rn(__fmul_rn(x0.z, rstd), g0.z);
-          xv[3] = __fmul_rn(__fmul_rn(x0.w, rstd), g0.w);
-          xv[4] = __fmul_rn(__fmul_rn(x1.x, rstd), g1.x);
-          xv[5] = __fmul_rn(__fmul_rn(x1.y, rstd), g1.y);
-          xv[6] = __fmul_rn(__fmul_rn(x1.z, rstd), g1.z);
-          xv[7] = __fmul_rn(__fmul_rn(x1.w, rstd), g1.w);
-        }
-        if (a.quant) {  // Q8 of 32-value blocks = 4 consecutive lanes (warp-uniform branch)
-          float am = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
-          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-          const float d = q8_scale(am);
-          uint32_t lo = 0, hi = 0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int c = q8_code(xv[e], d);
-            xv[e] = q8_value(c, d);
-            if (e < 4) lo |= (uint32_t)(c & 0xFF) << (8 * e);
-            else hi |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
+  __syncthreads();
+  pdl_launch_dependents();
+
+  if (warp == nc) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int t = 0;
+      for (int cur = 0; cur < nrows; ++t) {
+        const int end = stage_end(cur, nrows, R0, rps, P);
+        const int s = t % nstage;
+        const uint32_t ph = (uint32_t)(t / nstage) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.err)) break;
+        mbar_expect_tx(&full[s], (uint32_t)(end - cur) * row_bytes);
+        uint8_t* dst = ring + (size_t)s * 2 * P * row_bytes;
+        // one division per stage; rows are then walked with pointer increments
+        const int seg = (R0 + cur) / rps;
+        const int lr0 = R0 + cur - seg * rps;
+        const int n = end - cur;
+        const size_t col0 = (size_t)seg * a.Ks;
+        if (EPI == EPI_SWIGLU) {  // rows alternate W1[f], W3[f]
+          const uint16_t* p1 = a.w[0] + (size_t)(lr0 >> 1) * a.ldw + col0;
+          const uint16_t* p3 = a.w[1] + (size_t)(lr0 >> 1) * a.ldw + col0;
+          for (int i = 0; i < n; i += 2) {
+            bulk_g2s(dst + (size_t)i * row_bytes, p1, row_bytes, &full[s]);
+            bulk_g2s(dst + (size_t)(i + 1) * row_bytes, p3, row_bytes, &full[s]);
+            p1 += a.ldw;
+            p3 += a.ldw;
           }
-          if (writer && in && a.xq_out) {
-            *reinterpret_cast<uint2*>(a.xq_out + e0) = make_uint2(lo, hi);
-            if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = d;
+        } else {  // runs of rows inside one matrix; one copy per run when rows are contiguous
+          int done = 0, r = lr0;
+          while (done < n) {
+            int mat, lrow;
+            const uint16_t* src = row_ptr<EPI>(a, seg, r, mat, lrow);
+            int mat_end = a.rows[0];
+            if (EPI == EPI_QKV) mat_end = mat == 0 ? a.rows[0] : (mat == 1 ? a.rows[0] + a.rows[1] : rps);
+            const int run = min(n - done, mat_end - r);
+            if (a.ldw == a.Ks) {
+              bulk_g2s(dst + (size_t)done * row_bytes, src, (uint32_t)run * row_bytes, &full[s]);
+            } else {
+              for (int i = 0; i < run; ++i, src += a.ldw)
+                bulk_g2s(dst + (size_t)(done + i) * row_bytes, src, row_bytes, &full[s]);
+            }
+            done += run;
+            r += run;
           }
         }
-        if (writer && in && a.xn_out) {
-          *reinterpret_cast<float4*>(a.xn_out + e0) = make_float4(xv[0], xv[1], xv[2], xv[3]);
-          *reinterpret_cast<float4*>(a.xn_out + e0 + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
-        }
-      } else if (in) {
-        if (a.xq) {
-          const uint2 c = *reinterpret_cast<const uint2*>(a.xq + e0);
-          const float d = a.xd[e0 / kQ8Block];
-          const float4 l = q8_unpack4(c.x, d), h = q8_unpack4(c.y, d);
-          xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
-          xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
-        } else {
-          const float4 l = *reinterpret_cast<const float4*>(a.x + e0);
-          const float4 h = *reinterpret_cast<const float4*>(a.x + e0 + 4);
-          xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
-          xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
-        }
+        cur = end;
       }
     }
-  }
-
-  // ---------------------------------------------------------------- weight stream
-  int vrows = a.rows[0];
-  if (EPI == EPI_QKV) vrows += a.rows[1] + a.rows[2];
-  const int npairs = EPI == EPI_SWIGLU ? vrows : vrows >> 1;
-  const int p0 = (int)(((int64_t)npairs * cta) / a.ctas_per_seg);
-  const int p1 = (int)(((int64_t)npairs * (cta + 1)) / a.ctas_per_seg);
-
-  for (int pb = p0; pb < p1; pb += U) {
-    uint4 wv[U][2][VPL];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int p = pb + u;
-      if (p < p1) {
-        const uint16_t *r0, *r1;
-        int mat, lrow;
-        pair_rows<EPI>(a, p, col0, r0, r1, mat, lrow);
-#pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-          const int v = vb + lane + 32 * j;
-          if (v < ve) {
-            wv[u][0][j] = ld_stream16(r0 + 8 * (size_t)v);
-            wv[u][1][j] = ld_stream16(r1 + 8 * (size_t)v);
-          }
-        }
+    pdl_wait();  // the epilogue below writes buffers earlier kernels may read
+  } else {
+    // ---------------------------------------------------------------- consumers
+    pdl_wait();  // activations / residual come from the previous kernel
+    const int ncons = nc * 32;
+    if (a.gain && a.ssq) {  // sums of squares left by the merge that produced x
+      if (threadIdx.x < NB) {
+        float t = 0.f;
+        if ((int)threadIdx.x < a.nb)
+          for (int c = 0; c < a.ssq_parts; ++c) t += a.ssq[(size_t)(a.b0 + threadIdx.x) * a.ssq_parts + c];
+        s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
       }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int p = pb + u;
-      if (p >= p1) break;
-      float acc[2][NB];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) acc[0][b] = acc[1][b] = 0.f;
-#pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        const int v = vb + lane + 32 * j;
-        if (v < ve) {
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            acc[0][b] += dot8(wv[u][0][j], xr[b][j]);
-            acc[1][b] += dot8(wv[u][1][j], xr[b][j]);
-          }
-        }
-      }
+      consumers_sync(ncons);
+    } else if (a.gain) {  // RMSNorm scale of each batch row, over the whole row
+      const int D = a.ldx;
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        acc[0][b] = warp_sum(acc[0][b]);
-        acc[1][b] = warp_sum(acc[1][b]);
+        float ss = 0.f;
+        if (b < a.nb) {
+          const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
+          for (int i = threadIdx.x; i < (D >> 2); i += ncons) {
+            const float4 v = xrow[i];
+            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+          }
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) s_red[warp][b] = ss;
       }
-      if (lane == 0) {
-        float* r = red + ((size_t)(p - p0) * kWarps + warp) * 2 * NB;
+      consumers_sync(ncons);
+      if (threadIdx.x < NB) {
+        float t = 0.f;
+        for (int w = 0; w < nc; ++w) t += s_red[w][threadIdx.x];
+        s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)D + a.eps);
+      }
+      consumers_sync(ncons);
+    }
+
+    int cur_seg = -1;
+    bool ok = true;
+    int t = 0;
+    // this warp's share of a stage: row pair `pw` of the stage, vectors [vb, ve)
+    const int pw = warp / Q, part = warp - pw * Q;
+    const int vb = (nv * part) / Q, ve = (nv * (part + 1)) / Q;
+    for (int cur = 0; cur < nrows; ++t) {
+      const int end = stage_end(cur, nrows, R0, rps, P);
+      const int s = t % nstage;
+      const uint32_t ph = (uint32_t)(t / nstage) & 1u;
+      const int seg = (R0 + cur) / rps;
+      if (seg != cur_seg) {
+        // (re)stage the activations of this segment; whole warps per iteration so
+        // that 4 consecutive lanes always hold one 32-value Q8 block
+        const bool publish = (R0 + cur) == seg * rps;  // this CTA owns the segment's first row
+        const size_t col0 = (size_t)seg * a.Ks;
+        const int nvr = (nv + 31) & ~31;
+        consumers_sync(ncons);
+        for (int b = 0; b < NB; ++b) {
+          for (int v = threadIdx.x; v < nvr; v += ncons) {
+            const bool in = b < a.nb && v < nv;
+            const size_t e0 = (size_t)(a.b0 + b) * a.ldx + col0 + 8 * (size_t)v;
+            float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (in) {
+              if (a.gain) {
+                const float rstd = s_rstd[b];
+                const float4 x0 = *reinterpret_cast<const float4*>(a.x + e0);
+                const float4 x1 = *reinterpret_cast<const float4*>(a.x + e0 + 4);
+                const float4 g0 = *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v);
+                const float4 g1 =
+                    *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v + 4);
+                xv[0] = __fmul_rn(__fmul_rn(x0.x, rstd), g0.x);
+                xv[1] = __fmul_rn(__fmul_rn(x0.y, rstd), g0.y);
+                xv[2] = __fmul_rn(__fmul_rn(x0.z, rstd), g0.z);
+                xv[3] = __fmul_rn(__fmul_rn(x0.w, rstd), g0.w);
+                xv[4] = __fmul_rn(__fmul_rn(x1.x, rstd), g1.x);
+                xv[5] = __fmul_rn(__fmul_rn(x1.y, rstd), g1.y);
+                xv[6] = __fmul_rn(__fmul_rn(x1.z, rstd), g1.z);
+                xv[7] = __fmul_rn(__fmul_rn(x1.w, rstd), g1.w);
+              } else if (a.xq) {
+                const uint2 c = *reinterpret_cast<const uint2*>(a.xq + e0);
+                const float d = a.xd[e0 / kQ8Block];
+                const float4 l = q8_unpack4(c.x, d), h = q8_unpack4(c.y, d);
+                xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
+                xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
+              } else {
+                const float4 l = *reinterpret_cast<const float4*>(a.x + e0);
+                const float4 h = *reinterpret_cast<const float4*>(a.x + e0 + 4);
+                xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
+                xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
+              }
+            }
+            if (a.gain && a.quant) {
+              float am = 0.f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
+              am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+              am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+              const float d = q8_scale(am);
+              uint32_t lo = 0, hi = 0;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int c = q8_code(xv[e], d);
+                xv[e] = q8_value(c, d);
+                if (e < 4) lo |= (uint32_t)(c & 0xFF) << (8 * e);
+                else hi |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
+              }
+              if (publish && in && a.xq_out) {
+                *reinterpret_cast<uint2*>(a.xq_out + e0) = make_uint2(lo, hi);
+                if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = d;
+              }
+            }
+            if (a.gain && publish && in && a.xn_out) {
+              *reinterpret_cast<float4*>(a.xn_out + e0) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+              *reinterpret_cast<float4*>(a.xn_out + e0 + 4) =
+                  make_float4(xv[4], xv[5], xv[6], xv[7]);
+            }
+            if (v < nv) {
+              xs[b * nv + v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+              xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+            }
+          }
+        }
+        consumers_sync(ncons);
+        cur_seg = seg;
+      }
+      // after a wait gives up, keep walking the stages (so that every consumer warp
+      // reaches the same named barriers) but skip the work
+      if (ok && !mbar_wait(&full[s], ph, a.err)) ok = false;
+      const int r = cur + 2 * pw;  // this warp's row pair in the stage
+      if (ok && r < end) {
+        const uint4* w0 = reinterpret_cast<const uint4*>(ring + ((size_t)s * 2 * P + 2 * pw) * row_bytes);
+        const uint4* w1 = w0 + nv;
+        uint64_t acc0[NB], acc1[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc0[b] = acc1[b] = 0ull;
+#pragma unroll 4
+        for (int v = vb + lane; v < ve; v += 32) {
+          const uint4 u0 = w0[v], u1 = w1[v];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const float4 lo = xs[b * nv + v], hi = xs[(NB + b) * nv + v];
+            fma8(acc0[b], u0, lo, hi);
+            fma8(acc1[b], u1, lo, hi);
+          }
+        }
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          r[b] = acc[0][b];
-          r[NB + b] = acc[1][b];
+          const float y0 = warp_sum(hsum2(acc0[b]));
+          const float y1 = warp_sum(hsum2(acc1[b]));
+          if (lane == 0) {
+            res[((size_t)r * NB + b) * Q + part] = y0;
+            res[((size_t)(r + 1) * NB + b) * Q + part] = y1;
+          }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      cur = end;
     }
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- epilogue
-  for (int t = threadIdx.x; t < (p1 - p0) * NB; t += kThreads) {
-    const int pl = t / NB, b = t - pl * NB;
+  for (int t = threadIdx.x; t < (nrows >> 1) * NB; t += blockDim.x) {
+    const int pr = t / NB, b = t - pr * NB;
     if (b >= a.nb) continue;
-    const int p = p0 + pl;
+    const int g = R0 + 2 * pr, seg = g / rps, lr = g - seg * rps;
     float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float* r = red + ((size_t)pl * kWarps + w) * 2 * NB;
-      y0 += r[b];
-      y1 += r[NB + b];
+    for (int q = 0; q < pl.split; ++q) {  // the row's parts, in a fixed order
+      y0 += res[((size_t)(2 * pr) * NB + b) * pl.split + q];
+      y1 += res[((size_t)(2 * pr + 1) * NB + b) * pl.split + q];
     }
-    const uint16_t *r0, *r1;
     int mat, lrow;
-    pair_rows<EPI>(a, p, col0, r0, r1, mat, lrow);
+    row_ptr<EPI>(a, seg, lr, mat, lrow);
     const int gb = a.b0 + b;
     if (EPI == EPI_PLAIN) {
       const size_t o = (size_t)seg * a.out_seg + (size_t)gb * a.ldo + lrow;
@@ -306,71 +440,79 @@ __global__ void __launch_bounds__(kThreads) k_gemv(GemvArgs a) {
   }
 }
 
-template <int NB, int EPI, int VPL>
-int launch_one(const GemvArgs& a, int max_pairs, cudaStream_t s) {
-  const size_t smem = (size_t)max_pairs * kWarps * 2 * NB * sizeof(float);
-  if (smem > 48 * 1024 && set_smem_once((const void*)k_gemv<NB, EPI, VPL>, (int)smem))
-    return TP_ECUDA;
-  k_gemv<NB, EPI, VPL><<<a.ctas_per_seg * a.nseg, kThreads, smem, s>>>(a);
-  TP_LAUNCH_CHECK();
-  return TP_OK;
+size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
+
+// Shared-memory plan: 8 consumer warps; the most row pairs per stage (8, 4, 2,
+// 1) that still leave a ring of at least 3 stages (2 for the longest rows), each
+// pair split over 8 / pairs warps.
+bool make_plan(int NB, int Ks, int cta_rows, GemvPlan* p) {
+  const size_t row_bytes = (size_t)Ks * 2;
+  const size_t x_bytes = a128((size_t)NB * Ks * 4);
+  const size_t bar_bytes = 2 * kMaxStages * 8;
+  for (int min_stages : {3, 2}) {
+    for (int P = 8; P >= 1; P >>= 1) {
+      const int Q = 8 / P;
+      const size_t res_bytes = a128((size_t)cta_rows * NB * Q * 4);
+      const size_t fixed = x_bytes + res_bytes + bar_bytes;
+      if (fixed >= (size_t)kSmemBudget) continue;
+      const size_t stage = 2 * (size_t)P * row_bytes;
+      int ns = (int)(((size_t)kSmemBudget - fixed) / stage);
+      if (ns > kMaxStages) ns = kMaxStages;
+      if (ns >= min_stages) {
+        p->nc = 8;
+        p->pairs = P;
+        p->split = Q;
+        p->nstage = ns;
+        p->cta_rows = cta_rows;
+        p->ring_off = 0;
+        p->x_off = a128((size_t)ns * stage);
+        p->res_off = p->x_off + x_bytes;
+        p->bar_off = p->res_off + res_bytes;
+        p->total = p->bar_off + bar_bytes;
+        return true;
+      }
+    }
+  }
+  return false;
 }
 
 template <int NB, int EPI>
-int launch_vpl(const GemvArgs& a, int max_pairs, cudaStream_t s) {
-  const int nv = a.Ks >> 3;
-  const int per_warp = ((nv >> 2) + kWarps - 1) / kWarps * 4;  // vectors, rounded up
-  if (per_warp <= 32) return launch_one<NB, EPI, 1>(a, max_pairs, s);
-  if (per_warp <= 64) return launch_one<NB, EPI, 2>(a, max_pairs, s);
-  if constexpr (NB <= 2) {
-    if (per_warp <= 128) return launch_one<NB, EPI, 4>(a, max_pairs, s);
-  }
-  if constexpr (NB == 1) {
-    if (per_warp <= 256) return launch_one<NB, EPI, 8>(a, max_pairs, s);
-  }
-  return TP_ENOTSUP;
+int launch_one(const GemvArgs& a, cudaStream_t s) {
+  int rps = a.rows[0];
+  if (EPI == EPI_SWIGLU) rps = 2 * a.rows[0];
+  if (EPI == EPI_QKV) rps = a.rows[0] + a.rows[1] + a.rows[2];
+  const int npairs = a.nseg * (rps >> 1);
+  int grid = num_sms();
+  if (grid > npairs) grid = npairs;
+  const int cta_rows = 2 * ((npairs + grid - 1) / grid);
+  GemvPlan pl;
+  if (!make_plan(NB, a.Ks, cta_rows, &pl)) return TP_ENOTSUP;
+  if (set_smem_once((const void*)k_gemv<NB, EPI>, (int)pl.total)) return TP_ECUDA;
+  return launch_pdl(k_gemv<NB, EPI>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
 }
 
 template <int NB>
 int launch_nb(const GemvArgs& a, int epi, cudaStream_t s) {
-  int vrows = a.rows[0];
-  if (epi == EPI_QKV) vrows += a.rows[1] + a.rows[2];
-  const int npairs = epi == EPI_SWIGLU ? vrows : vrows >> 1;
-  const int max_pairs = (npairs + a.ctas_per_seg - 1) / a.ctas_per_seg;
   switch (epi) {
-    case EPI_PLAIN: return launch_vpl<NB, EPI_PLAIN>(a, max_pairs, s);
-    case EPI_SWIGLU: return launch_vpl<NB, EPI_SWIGLU>(a, max_pairs, s);
-    default: return launch_vpl<NB, EPI_QKV>(a, max_pairs, s);
+    case EPI_PLAIN: return launch_one<NB, EPI_PLAIN>(a, s);
+    case EPI_SWIGLU: return launch_one<NB, EPI_SWIGLU>(a, s);
+    default: return launch_one<NB, EPI_QKV>(a, s);
   }
 }
 
 }  // namespace
 
-// Batch rows are processed in groups of at most 4 per launch (2 when a warp's
-// column range needs more than 64 vectors, 1 above 128); the activations of a
-// group live in registers. Column ranges above 256 vectors per warp (rows longer
-// than 16384 elements per segment) are not supported.
+// Batch rows are handled two at a time (each launch streams the weights once).
 int launch_gemv(const GemvArgs& a0, int epi, cudaStream_t s) {
-  if (a0.Ks % 32 != 0 || a0.ctas_per_seg < 1) return TP_EINVAL;
-  const int nv = a0.Ks >> 3;
-  const int per_warp = ((nv >> 2) + kWarps - 1) / kWarps * 4;
-  if (per_warp > 256) return TP_ENOTSUP;
-  const int maxnb = per_warp <= 64 ? 4 : (per_warp <= 128 ? 2 : 1);
+  if (a0.Ks % 32 != 0 || a0.Ks < 32 || a0.nseg < 1) return TP_EINVAL;
+  if (((a0.rows[0] | a0.rows[1] | a0.rows[2]) & 1) != 0) return TP_EINVAL;
   for (int b = 0; b < a0.nb;) {
     GemvArgs a = a0;
     a.b0 = a0.b0 + b;
-    int nb = a0.nb - b;
-    if (nb > maxnb) nb = maxnb;
-    a.nb = nb;
-    int rc;
-    if (nb == 1)
-      rc = launch_nb<1>(a, epi, s);
-    else if (nb == 2)
-      rc = launch_nb<2>(a, epi, s);
-    else
-      rc = launch_nb<4>(a, epi, s);
+    a.nb = a0.nb - b >= 2 ? 2 : 1;
+    const int rc = a.nb == 2 ? launch_nb<2>(a, epi, s) : launch_nb<1>(a, epi, s);
     if (rc != TP_OK) return rc;
-    b += nb;
+    b += a.nb;
   }
   return TP_OK;
 }

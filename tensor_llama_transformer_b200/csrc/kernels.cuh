@@ -6,8 +6,12 @@
 namespace tp {
 
 // ------------------------------------------------------------------ merge / codec
-// x[b] += sum_{s<n} sync(part[s][b]) in slice order; part is [n, B, dim].
-int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, cudaStream_t s);
+// x[b] += sum_{s<n} sync(part[s][b]) in slice order; part is [n, B, dim]. With
+// ssq != nullptr each CTA also writes the sum of squares of its piece of the new
+// row: ssq[b][piece], piece = 512-element block index (merge_ssq_parts(dim) of them).
+int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
+                 cudaStream_t s);
+inline int merge_ssq_parts(int dim) { return (dim / 4 + 127) / 128; }
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s);
 int launch_dequantize(const int8_t* q, const float* d, float* x, int64_t n, cudaStream_t s);
 
@@ -33,6 +37,8 @@ struct GemvArgs {
   const float* gain;
   float eps;
   int quant;
+  const float* ssq;  // optional per-row partial sums of squares of x [B][ssq_parts] (fixed order)
+  int ssq_parts;
   int8_t* xq_out;
   float* xd_out;
   float* xn_out;
@@ -49,8 +55,21 @@ struct GemvArgs {
   const int32_t* pos;
   int n_heads, n_kv_heads, max_seq;
   float theta;
-  // launch shape
-  int ctas_per_seg;
+  int* err;  // device error flag, set when a bounded wait gives up (nullable)
+  int ctas_per_seg;  // unused by the ring-buffer kernel (one CTA per SM)
+};
+
+// Shared-memory plan of the GEMV (host computes, kernel reads): NC consumer
+// warps, row pairs per stage (each pair split over `split` warps), ring depth,
+// and the offsets of the ring, the staged activations, the per-row partial
+// results and the mbarriers.
+struct GemvPlan {
+  int nc;
+  int pairs;
+  int split;
+  int nstage;
+  int cta_rows;
+  size_t ring_off, x_off, res_off, bar_off, total;
 };
 
 int launch_gemv(const GemvArgs& a, int epi, cudaStream_t s);

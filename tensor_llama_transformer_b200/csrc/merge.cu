@@ -17,7 +17,11 @@ constexpr int kMergeThreads = 128;  // 4 values per thread: 512 values per CTA
 
 __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
                                                          const float* __restrict__ part, int n,
-                                                         int B, int dim, int quant) {
+                                                         int B, int dim, int quant,
+                                                         float* __restrict__ ssq) {
+  __shared__ float red[kMergeThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y;
   const int i4 = blockIdx.x * kMergeThreads + threadIdx.x;  // float4 index within the row
   const int n4 = dim >> 2;
@@ -33,6 +37,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
     acc.z += p.z;
     acc.w += p.w;
   }
+  float sq = 0.f;
   if (in) {
     float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim);
     float4 v = xr[i4];
@@ -41,6 +46,17 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
     v.z += acc.z;
     v.w += acc.w;
     xr[i4] = v;
+    sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (ssq) {  // this piece's sum of squares, for the next RMSNorm (fixed summation order)
+    sq = warp_sum(sq);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.f;
+      for (int w = 0; w < kMergeThreads / 32; ++w) t += red[w];
+      ssq[(size_t)b * gridDim.x + blockIdx.x] = t;
+    }
   }
 }
 
@@ -69,11 +85,10 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 
 }  // namespace
 
-int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, cudaStream_t s) {
-  const dim3 grid((dim / 4 + kMergeThreads - 1) / kMergeThreads, B);
-  k_merge<<<grid, kMergeThreads, 0, s>>>(x, part, n, B, dim, quant);
-  TP_LAUNCH_CHECK();
-  return TP_OK;
+int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
+                 cudaStream_t s) {
+  const dim3 grid(merge_ssq_parts(dim), B);
+  return launch_pdl(k_merge, grid, dim3(kMergeThreads), 0, s, x, part, n, B, dim, quant, ssq);
 }
 
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s) {
