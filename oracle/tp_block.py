@@ -44,7 +44,7 @@ import numpy as np
 __all__ = [
     "bf16_to_f64", "round_to_bf16", "rmsnorm", "q8_quantize", "q8_dequantize", "sync_buffer",
     "rope", "attention_decode", "silu", "swiglu", "relu", "block_forward", "ffn_forward",
-    "model_forward", "grid_2d", "slice_range",
+    "model_forward", "grid_2d", "slice_range", "ffn_unsharded_chunked",
 ]
 
 
@@ -410,3 +410,27 @@ def model_forward(tokens, embed, layers, final_norm, wcls, n_slices: int, sync_q
     V = W.shape[0]
     parts = [xn @ W[slice_range(V, n_slices, s), :].T for s in range(n_slices)]
     return np.concatenate(parts, axis=1)
+
+
+def ffn_unsharded_chunked(X, W1_bits, W2_bits, act: str = "relu", W3_bits=None,
+                          chunk: int = 4096) -> np.ndarray:
+    """``act(X W1^T [, X W3^T]) W2^T`` for a few rows of X, memory-bounded.
+
+    The same unpartitioned FFN as ``ffn_forward`` with one slice ([TP] how it
+    works: the partitioned layer must equal it), for weights too large to hold
+    in float64 at once (the PaLM 540B shapes): the F dimension is walked in
+    ``chunk``-wide pieces, each piece's bf16 weights upcast exactly to float64,
+    and the contributions summed in order. ``X`` is float64 ``[rows, E]``.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    F = W1_bits.shape[0]
+    Y = np.zeros((X.shape[0], W2_bits.shape[0]))
+    for f0 in range(0, F, chunk):
+        fs = slice(f0, min(F, f0 + chunk))
+        a = X @ bf16_to_f64(W1_bits[fs]).T
+        if act == "relu":
+            H = relu(a)
+        else:
+            H = swiglu(a, X @ bf16_to_f64(W3_bits[fs]).T)
+        Y = Y + H @ bf16_to_f64(W2_bits[:, fs]).T
+    return Y

@@ -137,3 +137,10 @@ def test_block_c2_slices_agree(tpb):
     outs = [run_block(tpb, inp, n, 0)[0] for n in (1, 2, 4, 8)]
     for o in outs[1:]:
         assert np.max(np.abs(o - outs[0])) / np.max(np.abs(outs[0])) < 1e-5
+
+
+@pytest.mark.slow
+def test_block_c4_full_size(tpb):
+    """70B-shape GQA block: dim 8192, 64 q heads over 8 kv heads, batch 32, context 4096, n = 8."""
+    inp = synth.block_inputs(synth.CONFIG_SEED["C4"], synth.C4)
+    check_block(tpb, inp, synth.C4.n_slices, 0, tight=2e-3, name="C4")

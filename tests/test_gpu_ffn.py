@@ -94,3 +94,43 @@ def test_bf16_m_tails(tpb, M):
         y = run_ffn(tpb, s, inputs, 1, merge)
         r, _ = report(f"bf16 M={M} merge{merge}", y, _ref(s, inputs, 1, False))
         assert r <= BF16_TOL
+
+
+@pytest.fixture(scope="module")
+def c5_weights(cuda_ok):
+    """PaLM-shaped FFN weights (E 18432, F 73728), generated once for the C5 cases."""
+    s = synth.C5
+    seed = synth.CONFIG_SEED["C5"]
+    W1 = synth.normal_bf16(seed, "W1", (s.F, s.E), s.w_std)
+    W2 = synth.normal_bf16(seed, "W2", (s.E, s.F), s.w_std)
+    return W1, W2, bf16_tensor(W1), bf16_tensor(W2)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("B,forms", [(512, ("fused", "1d", "2d")), (2048, ("fused", "2d")),
+                                     (8192, ("fused",))])
+def test_c5_full_size_sampled_rows(tpb, c5_weights, B, forms):
+    """Full PaLM FFN on the GPU; the oracle checks 8 token rows spread over the M tiles."""
+    W1, W2, W1d, W2d = c5_weights
+    s = synth.FfnShape(**{**synth.C5.__dict__, "batch": B})
+    seed = synth.CONFIG_SEED["C5"]
+    X = synth.normal_bf16(seed, f"X{B}", (B, s.E), s.x_std)
+    Xd = bf16_tensor(X)
+    rows = np.unique(np.array([0, 1, 127, 128, B // 3, B // 2, B - 2, B - 1]))
+    ref = oracle.ffn_unsharded_chunked(oracle.bf16_to_f64(X[rows]), W1, W2, chunk=2048)
+    for form in forms:
+        part, merge = {"fused": (1, 1), "1d": (1, 0), "2d": (2, 0)}[form]
+        gx, gy = (8, 8) if part == 2 else (1, 1)
+        desc = tpb.tp_ffn_desc(B, s.E, s.F, tpb.TP_BF16, tpb.TP_ACT_RELU, part, 64, gx, gy, 0, merge)
+        nb = tpb.tp_ffn_workspace_bytes(desc)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        Y = torch.full((B, s.E), float("nan"), dtype=torch.float32, device="cuda")
+        tpb.tp_ffn_forward(desc, Xd, W1d, None, W2d, Y, ws, nb)
+        torch.cuda.synchronize()
+        assert int(ws[:4].view(torch.int32).item()) == 0
+        y = Y[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64)
+        r, p = report(f"C5 B={B} {form}", y, ref)
+        assert r <= BF16_TOL and p > 0.9999
+        assert torch.isfinite(Y).all()
+        del ws, Y
+        torch.cuda.empty_cache()

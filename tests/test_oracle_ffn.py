@@ -108,3 +108,18 @@ def test_grid_2d_default():
     assert grid_2d(4) == (2, 2)
     assert grid_2d(8) == (2, 4)
     assert grid_2d(1) == (1, 1)
+
+
+@pytest.mark.parametrize("act", ["relu", "swiglu"])
+def test_chunked_unsharded_matches_ffn_forward(act):
+    import synth
+    from oracle import bf16_to_f64, ffn_unsharded_chunked
+
+    s = synth.FfnShape(batch=3, E=64, F=320, dtype="bf16", act=act, n_slices=1, w_std=0.1)
+    inp = synth.ffn_inputs(21, s)
+    X = bf16_to_f64(inp["X"])
+    W3 = inp.get("W3")
+    ref = ffn_forward(X, bf16_to_f64(inp["W1"]), bf16_to_f64(inp["W2"]), act=act,
+                      W3=bf16_to_f64(W3) if W3 is not None else None)
+    got = ffn_unsharded_chunked(X, inp["W1"], inp["W2"], act=act, W3_bits=W3, chunk=96)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
