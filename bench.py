@@ -143,12 +143,14 @@ def dist_setup():
 
 
 def allreduce_max(v: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (device tensor under NCCL, host under gloo)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
