@@ -194,8 +194,7 @@ TP_API int tp_ffn_workspace_bytes(const tp_ffn_desc* d, size_t* out_bytes);
  * Y float32 [B,E] written. 1D: H_s = act(X W1_s^T) per F-slice (column split),
  * P_s = H_s W2_s^T (row split), Y = sum_s P_s. 2D: stage 1 sums over the E-slices,
  * stage 2 over the F-slices. Requirements: E % (32*grid_x) == 0 and F % (32*n)
- * == 0 (1D) or F % (32*grid_y) == 0 (2D); bf16 needs E % 64 == 0, F % 64 == 0 and
- * the per-slice contraction length a multiple of 64. */
+ * == 0 (1D) or F % (32*grid_y) == 0 (2D). */
 TP_API int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const void* W3,
                    const void* W2, float* Y, void* workspace, size_t ws_bytes, tp_stream stream);
 

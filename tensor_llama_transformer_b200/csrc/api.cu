@@ -5,6 +5,7 @@
 #include <new>
 
 #include "ffn.cuh"
+#include "gemm_tc.cuh"
 #include "kernels.cuh"
 
 namespace tp {
@@ -79,7 +80,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // ------------------------------------------------------------------ block layout
 enum Buf {
   BUF_XQ = 0, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H, BUF_ERR, BUF_PO, BUF_PML,
-  BUF_PA, BUF_PB, BUF_SSQ, BUF_COUNT
+  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_COUNT
 };
 
 struct Layout {
@@ -147,6 +148,16 @@ Layout block_layout(const Cfg& c) {
   L.size[BUF_PA] = pa;
   L.size[BUF_PB] = pa;
   L.size[BUF_SSQ] = B * (size_t)merge_ssq_parts(c.d.dim) * 4;
+  // batched decode (tensor-core path): bf16 operands and the float32 product planes
+  if (c.d.max_batch >= kTcMinBatch) {
+    const size_t KD = (size_t)c.d.n_kv_heads * c.d.head_dim;
+    L.size[BUF_XB] = 2 * B * D * 2;  // hi/lo bf16 pairs
+    L.size[BUF_ATTB] = 2 * B * QD * 2;
+    L.size[BUF_HB] = 2 * B * F * 2;
+    const size_t qkv = 2 * B * (QD + 2 * KD) * 4;  // up to 2 contraction parts
+    const size_t w13 = B * 2 * F * 4;
+    L.size[BUF_PLANE] = qkv > w13 ? qkv : w13;
+  }
   size_t o = 0;
   for (int i = 0; i < BUF_COUNT; ++i) {
     L.off[i] = o;
@@ -226,12 +237,161 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
   return e == cudaSuccess ? TP_OK : TP_ECUDA;
 }
 
+int tc_parts_for(int tiles) {
+  // contraction parts so that the q/k/v launch has work for every SM
+  return tiles * 2 <= num_sms() * 3 ? 2 : 1;
+}
+
+// The batched form of the block: the same steps, with the slice products on the
+// tcgen05 GEMM (weights = M operand, batch = N) writing float32 planes, small
+// kernels for the norms and epilogues, and the same attention and merges.
+int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
+                     cudaStream_t s, bool chained) {
+  const Cfg& c = blk->c;
+  const tp_dims& d = c.d;
+  const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
+  const int QD = H * hd, KD = Hkv * hd;
+  int rc;
+  float* part = at<float>(blk, BUF_PART);
+  float* plane = at<float>(blk, BUF_PLANE);
+  uint16_t* xb = at<uint16_t>(blk, BUF_XB);
+  int* err = at<int>(blk, BUF_ERR);
+  auto norm = [&](const float* gain, const float* ssq) -> int {
+    NormRowsArgs n{};
+    n.x = x;
+    n.gain = gain;
+    n.ssq = ssq;
+    n.ssq_parts = merge_ssq_parts(D);
+    n.dim = D;
+    n.eps = d.norm_eps;
+    n.quant = c.quant;
+    n.xq = c.quant ? at<int8_t>(blk, BUF_XQ) : nullptr;
+    n.xd = c.quant ? at<float>(blk, BUF_XD) : nullptr;
+    n.xn = c.quant ? nullptr : at<float>(blk, BUF_XN);
+    n.xb = xb;
+    return launch_norm_rows(n, batch, s);
+  };
+  auto gemm = [&](const void* A0, int m0, const void* A1, int m1, const void* A2, int m2, int nA,
+                  int64_t lda, const uint16_t* Bop, int K, int nseg, float* out, int64_t rows) {
+    TcGemm g{};
+    g.A[0] = A0;
+    g.A[1] = A1;
+    g.A[2] = A2;
+    g.Am[0] = m0;
+    g.Am[1] = m1;
+    g.Am[2] = m2;
+    g.nA = nA;
+    g.lda = lda;
+    g.B = Bop;
+    g.ldb = lda;
+    g.N = 2 * batch;  // hi/lo row pairs of the activations
+    g.K = K;
+    g.nseg = nseg;
+    g.epi = TC_EPI_STORE_T_PAIRS_F32;
+    g.out = out;
+    g.ldo = rows;
+    g.out_seg = (int64_t)batch * rows;
+    g.err = err;
+    return launch_tc_gemm(g, s);
+  };
+
+  // a1-a4
+  if ((rc = stage_mark(blk, 0, s))) return rc;
+  if ((rc = norm(blk->w.attn_norm, chained ? at<float>(blk, BUF_SSQ) : nullptr))) return rc;
+  const int qkv_tiles = (QD + 127) / 128 + 2 * ((KD + 127) / 128);
+  int parts = tc_parts_for(qkv_tiles);
+  if ((D / parts) % 8 != 0) parts = 1;
+  if ((rc = gemm(blk->w.wq, QD, blk->w.wk, KD, blk->w.wv, KD, 3, D, xb, D / parts, parts, plane,
+                 QD + 2 * KD)))
+    return rc;
+  {
+    QkvFinalizeArgs f{};
+    f.plane = plane;
+    f.parts = parts;
+    f.batch = batch;
+    f.qd = QD;
+    f.kd = KD;
+    f.pos = pos;
+    f.theta = d.rope_theta;
+    f.q = at<float>(blk, BUF_Q);
+    f.kc = static_cast<uint16_t*>(kc);
+    f.vc = static_cast<uint16_t*>(vc);
+    f.n_kv_heads = Hkv;
+    f.max_seq = d.max_seq;
+    if ((rc = launch_qkv_finalize(f, s))) return rc;
+  }
+  // a4
+  if ((rc = stage_mark(blk, 1, s))) return rc;
+  {
+    AttnArgs a{};
+    a.q = at<float>(blk, BUF_Q);
+    a.kc = static_cast<const uint16_t*>(kc);
+    a.vc = static_cast<const uint16_t*>(vc);
+    a.pos = pos;
+    a.B = batch;
+    a.H = H;
+    a.Hkv = Hkv;
+    a.max_seq = d.max_seq;
+    a.nchunk = c.nchunk;
+    a.part_o = at<float>(blk, BUF_PO);
+    a.part_ml = at<float>(blk, BUF_PML);
+    a.att = at<float>(blk, BUF_ATT);
+    a.att_bf16 = at<uint16_t>(blk, BUF_ATTB);
+    a.err = err;
+    if ((rc = launch_attention(a, s))) return rc;
+  }
+  // a5: W_O row-split partials (segment s = slice s's head columns)
+  if ((rc = stage_mark(blk, 2, s))) return rc;
+  if ((rc = gemm(blk->w.wo, D, nullptr, 0, nullptr, 0, 1, QD, at<uint16_t>(blk, BUF_ATTB), QD / c.n,
+                 c.n, part, D)))
+    return rc;
+  // a6
+  if ((rc = stage_mark(blk, 3, s))) return rc;
+  if ((rc = launch_merge(x, part, c.n, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
+  // a7-a8
+  if ((rc = stage_mark(blk, 4, s))) return rc;
+  if ((rc = norm(blk->w.ffn_norm, at<float>(blk, BUF_SSQ)))) return rc;
+  float* hbuf = at<float>(blk, BUF_H);
+  uint16_t* hb = at<uint16_t>(blk, BUF_HB);
+  if (c.partition == TP_PART_1D) {
+    if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D, 1, plane, 2 * F))) return rc;
+    if ((rc = launch_swiglu_finalize(plane, F, batch, hbuf, hb, s))) return rc;
+  } else {
+    float* pa = at<float>(blk, BUF_PA);
+    float* pb = at<float>(blk, BUF_PB);
+    if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F))) return rc;
+    if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F))) return rc;
+    FfnMergeArgs m{};
+    m.P1 = pa;
+    m.P3 = pb;
+    m.seg_stride = (int64_t)batch * F;
+    m.nseg = c.gx;
+    m.M = batch;
+    m.N = F;
+    m.quant = c.quant;
+    m.act = ACT_SWIGLU;
+    m.out_f32 = hbuf;
+    m.out_bf16 = hb;
+    m.bf16_split = 1;
+    if ((rc = launch_ffn_merge(m, s))) return rc;
+  }
+  // a9
+  if ((rc = stage_mark(blk, 5, s))) return rc;
+  const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
+  if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2, nseg2, part, D))) return rc;
+  // a10
+  if ((rc = stage_mark(blk, 6, s))) return rc;
+  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
+  return stage_mark(blk, TP_BLOCK_STAGES, s);
+}
+
 // One block forward (the distributed-llama root-node order for one layer).
 // chained: x was produced by the previous block's final merge of this same
 // launch sequence, which left the row sums of squares in the workspace (inside
 // a model); the final merge here leaves them for the next block.
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
                        cudaStream_t s, bool chained = false) {
+  if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained);
   const Cfg& c = blk->c;
   const tp_dims& d = c.d;
   const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;

@@ -197,7 +197,11 @@ __global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a) {
   const float r = o / l;
   const size_t oi = ((size_t)b * a.H + h) * kHeadDim + d;
   a.att[oi] = r;
-  if (a.att_bf16) a.att_bf16[oi] = f32_to_bf16_bits(r);
+  if (a.att_bf16) {  // hi/lo bf16 pair: rows 2b and 2b+1 of [2B, H*hd]
+    const size_t row = (size_t)a.H * kHeadDim;
+    const size_t hi = (size_t)(2 * b) * row + (size_t)h * kHeadDim + d;
+    bf16_split(r, a.att_bf16[hi], a.att_bf16[hi + row]);
+  }
 }
 
 template <int G>

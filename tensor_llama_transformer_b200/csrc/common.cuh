@@ -26,6 +26,14 @@ TP_DEV uint16_t f32_to_bf16_bits(float f) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
+// A float32 value as two bf16 terms, hi = bf16(v) and lo = bf16(v - hi): v - hi
+// is exact in float32, so hi + lo carries about 16 significant bits. Operands of
+// the tensor-core decode path are fed as such pairs (rows 2b and 2b+1).
+TP_DEV void bf16_split(float v, uint16_t& hi, uint16_t& lo) {
+  hi = f32_to_bf16_bits(v);
+  lo = f32_to_bf16_bits(v - __uint_as_float(((uint32_t)hi) << 16));
+}
+
 // 16-byte streaming load that bypasses L1 (weights are read once per launch).
 TP_DEV uint4 ld_stream16(const void* p) {
   uint4 r;

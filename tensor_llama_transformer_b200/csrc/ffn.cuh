@@ -16,7 +16,8 @@ struct FfnMergeArgs {
   int act;              // ACT_NONE / ACT_RELU / ACT_SWIGLU
   const float* residual;  // optional [M, N] added after the activation
   float* out_f32;       // optional [M, N]
-  uint16_t* out_bf16;   // optional [M, N]
+  uint16_t* out_bf16;   // optional [M, N], or hi/lo pairs [2M, N] when bf16_split
+  int bf16_split;
 };
 
 int launch_gemm_simt(int dtype, const void* A, int64_t lda, const void* B, int64_t ldb, float* P,

@@ -51,11 +51,6 @@ int plan_ffn(const tp_ffn_desc* d, FfnPlan* p) {
   p->Ks2 = d->F / p->nseg2;
   p->swiglu = d->act == TP_ACT_SWIGLU;
   p->esize = d->dtype == TP_F32 ? 4 : 2;
-  if (d->dtype == TP_BF16) {
-    // tensor-core operands: 64-element K steps, 128-row M tiles are padded by TMA
-    if (d->E % 64 != 0 || d->F % 64 != 0) return TP_EINVAL;
-    if (d->merge == TP_MERGE_FAITHFUL && (p->Ks1 % 64 != 0 || p->Ks2 % 64 != 0)) return TP_EINVAL;
-  }
   if (d->merge == TP_MERGE_FUSED && (d->dtype != TP_BF16 || d->sync_quant)) return TP_ENOTSUP;
   const size_t B = d->batch, E = d->E, F = d->F;
   const bool fused = d->merge == TP_MERGE_FUSED;
@@ -112,12 +107,13 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
   if (d->merge == TP_MERGE_FUSED) {
     // stage 1: H = act(X W1^T [, X W3^T]) over the full E (slice order = K order)
     TcGemm g{};
-    g.A = X;
+    g.A[0] = X;
+    g.Am[0] = B;
+    g.nA = 1;
     g.lda = E;
     g.B = W1;
     g.ldb = E;
     g.B2 = p.swiglu ? W3 : nullptr;
-    g.M = B;
     g.N = F;
     g.K = E;
     g.nseg = 1;
@@ -129,11 +125,12 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
     if (rc) return rc;
     // stage 2: Y = H W2^T over the full F
     TcGemm g2{};
-    g2.A = H;
+    g2.A[0] = H;
+    g2.Am[0] = B;
+    g2.nA = 1;
     g2.lda = F;
     g2.B = W2;
     g2.ldb = F;
-    g2.M = B;
     g2.N = E;
     g2.K = F;
     g2.nseg = 1;
@@ -151,11 +148,12 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
                       int N, int Ks, int nseg) -> int {
     if (d->dtype == TP_F32) return launch_gemm_simt(TP_F32, A, lda, Bm, ldb, P, M, N, Ks, nseg, s);
     TcGemm g{};
-    g.A = A;
+    g.A[0] = A;
+    g.Am[0] = M;
+    g.nA = 1;
     g.lda = lda;
     g.B = Bm;
     g.ldb = ldb;
-    g.M = M;
     g.N = N;
     g.K = Ks;
     g.nseg = nseg;

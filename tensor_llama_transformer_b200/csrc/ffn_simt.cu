@@ -104,11 +104,20 @@ __global__ void k_ffn_merge(FfnMergeArgs a) {
       r[0] += x.x; r[1] += x.y; r[2] += x.z; r[3] += x.w;
     }
     if (a.out_f32) reinterpret_cast<float4*>(a.out_f32)[i4] = make_float4(r[0], r[1], r[2], r[3]);
-    if (a.out_bf16) {
+    if (a.out_bf16 && !a.bf16_split) {
       uint2 p;
       p.x = (uint32_t)f32_to_bf16_bits(r[0]) | ((uint32_t)f32_to_bf16_bits(r[1]) << 16);
       p.y = (uint32_t)f32_to_bf16_bits(r[2]) | ((uint32_t)f32_to_bf16_bits(r[3]) << 16);
       reinterpret_cast<uint2*>(a.out_bf16)[i4] = p;
+    } else if (a.out_bf16) {
+      const int64_t e = 4 * i4, m = e / a.N, n = e - m * a.N;
+      uint16_t hi[4], lo[4];
+      for (int j = 0; j < 4; ++j) bf16_split(r[j], hi[j], lo[j]);
+      uint16_t* ph = a.out_bf16 + (size_t)(2 * m) * a.N + n;
+      *reinterpret_cast<uint2*>(ph) =
+          make_uint2((uint32_t)hi[0] | ((uint32_t)hi[1] << 16), (uint32_t)hi[2] | ((uint32_t)hi[3] << 16));
+      *reinterpret_cast<uint2*>(ph + a.N) =
+          make_uint2((uint32_t)lo[0] | ((uint32_t)lo[1] << 16), (uint32_t)lo[2] | ((uint32_t)lo[3] << 16));
     }
   }
 }

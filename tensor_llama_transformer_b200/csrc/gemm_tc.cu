@@ -1,20 +1,23 @@
-// Persistent tcgen05 GEMM for the batched / prefill FFN (sm_100a).
+// Persistent tcgen05 GEMM for the batched FFN and the batched decode products (sm_100a).
 //
 //   D[seg, m, n] = sum_{k < K} A[m, seg*K + k] * B[n, seg*K + k]
 //
-// A = activations [M tokens, K] and B = weights [N features, K], both bf16
-// with the contraction dimension contiguous (a PyTorch Linear weight is already
-// in this layout). A segment is the contraction range one tensor-parallel slice
-// owns (a row split); with nseg > 1 each slice's partial product goes to its
-// own plane of the output, to be summed by the merge (aiterms.tw "Tensor
-// Parallelism": Linear2 split by rows, then an all-reduce; Pope et al. demo1:
-// 2D weight-stationary adds a partial-sum stage before the activation).
+// Both operands bf16 with the contraction dimension contiguous (a PyTorch
+// Linear weight is already in this layout). A segment is the contraction range
+// one tensor-parallel slice owns (a row split); with nseg > 1 each slice's
+// partial product goes to its own plane of the output, to be summed by the
+// merge (aiterms.tw "Tensor Parallelism": Linear2 split by rows, then an
+// all-reduce; Pope et al. demo1: 2D weight-stationary adds a partial-sum stage
+// before the activation). The FFN puts tokens on M and features on N (N tile
+// 256); batched decode puts weight rows on M and the batch on N (N tile 32 or
+// 64, transposed store), so the weight stream is the M x K operand.
 //
 // Structure (one CTA per SM, 192 threads):
-//   warp 0  : TMA producer — 128x64 A tile and 256x64 B tile per stage, 128-byte
-//             swizzle, 4-stage ring of shared memory, completion on mbarriers.
-//   warp 1  : allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
-//             one lane issues tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32);
+//   warp 0  : TMA producer — 128x64 A tile and BNx64 B tile per stage, 128-byte
+//             swizzle, a ring of 4 (BN 256) to 10 (BN 32) stages of shared
+//             memory, completion on mbarriers.
+//   warp 1  : allocates TMEM for two 128xBN fp32 accumulators and one lane
+//             issues tcgen05.mma (M=128, N=BN, K=16, bf16 -> fp32);
 //             tcgen05.commit releases each smem stage and publishes each tile.
 //   warps 2-5: epilogue — tcgen05.ld of the accumulator (each warp its 32 TMEM
 //             lanes = 32 output rows), activation, stores to global memory,
@@ -30,13 +33,19 @@
 namespace tp {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, THREADS = 192;
+constexpr int BM = 128, BK = 64, THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+template <int BN>
+struct TcCfg {
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 10 ? 10 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  // two accumulators of BN columns, allocated as a power of two >= 32
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
+};
 
 TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -79,11 +88,12 @@ TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
   }
 }
 
-TP_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+// 3D tile load: coordinates {k within the segment, segment, row}.
+TP_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int seg, int row, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3}], [%4];" ::"r"(s2u(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(s2u(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4}], [%5];" ::"r"(s2u(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(seg), "r"(row), "r"(s2u(bar))
       : "memory");
 }
 
@@ -138,10 +148,21 @@ TP_DEV uint32_t pack_bf16x2(float a, float b) {
   return (uint32_t)f32_to_bf16_bits(a) | ((uint32_t)f32_to_bf16_bits(b) << 16);
 }
 
-template <int EPI>
+// m-tiles of the concatenated A matrices: matrix j owns m-tiles [mt_off[j], mt_off[j+1]).
+struct TcTiles {
+  int mt_off[4];
+  int num_n;
+  int ntiles;
+};
+
+template <int BN, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
-    k_tc_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-              const __grid_constant__ CUtensorMap mB2, TcGemm g, int num_m, int num_n, int ntiles) {
+    k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
+              const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB,
+              const __grid_constant__ CUtensorMap mB2, TcGemm g, TcTiles tt) {
+  using C = TcCfg<BN>;
+  constexpr int STAGES = C::STAGES, B_BYTES = C::B_BYTES, STAGE_BYTES = C::STAGE_BYTES;
+  constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -176,9 +197,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nk = g.K / BK;
-  const int per_seg = num_m * num_n;
+  const int nk = (g.K + BK - 1) / BK;  // a partial last block reads zeros past the segment
+  const int num_m = tt.mt_off[g.nA];
+  const int per_seg = num_m * tt.num_n;
+  const int ntiles = tt.ntiles;
   constexpr int NOUT = EPI == TC_EPI_SWIGLU_BF16 ? BN / 2 : BN;  // output columns per tile
+  // tile -> (segment, n block, matrix, first row in the matrix, first output row)
+  auto decode = [&](int tile, int& seg, int& nb, int& mat, int& m0, int& orow0) {
+    seg = tile / per_seg;
+    const int r = tile - seg * per_seg;
+    nb = r / num_m;
+    const int mt = r - nb * num_m;
+    mat = (mt >= tt.mt_off[1]) + (mt >= tt.mt_off[2]);
+    m0 = (mt - tt.mt_off[mat]) * BM;
+    orow0 = m0;
+    for (int j = 0; j < mat; ++j) orow0 += g.Am[j];
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -186,23 +220,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int seg = tile / per_seg, r = tile - seg * per_seg;
-        const int nb = r / num_m, mb = r - nb * num_m;
-        const int m0 = mb * BM, n0 = nb * NOUT;
-        const int kbase = seg * g.K;
+        int seg, nb, mat, m0, orow0;
+        decode(tile, seg, nb, mat, m0, orow0);
+        const int n0 = nb * NOUT;
+        const CUtensorMap* mA = mat == 0 ? &mA0 : (mat == 1 ? &mA1 : &mA2);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], ph ^ 1, g.err)) {
             ok = false;
             break;
           }
           mbar_expect_tx(&full[stage], STAGE_BYTES);
-          const int kx = kbase + kb * BK;
-          tma_load_2d(sA + stage * A_BYTES, &mA, kx, m0, &full[stage]);
+          const int kx = kb * BK;
+          tma_load_3d(sA + stage * A_BYTES, mA, kx, seg, m0, &full[stage]);
           if (EPI == TC_EPI_SWIGLU_BF16) {
-            tma_load_2d(sB + stage * B_BYTES, &mB, kx, n0, &full[stage]);
-            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, &mB2, kx, n0, &full[stage]);
+            tma_load_3d(sB + stage * B_BYTES, &mB, kx, seg, n0, &full[stage]);
+            tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &mB2, kx, seg, n0, &full[stage]);
           } else {
-            tma_load_2d(sB + stage * B_BYTES, &mB, kx, n0, &full[stage]);
+            tma_load_3d(sB + stage * B_BYTES, &mB, kx, seg, n0, &full[stage]);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -253,13 +287,45 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       if (!mbar_wait(&tfull[acc], aph, g.err)) break;
       tc_fence_after();
-      const int seg = tile / per_seg, r = tile - seg * per_seg;
-      const int nb = r / num_m, mb = r - nb * num_m;
-      const int row = mb * BM + 32 * q + lane;
+      int seg, nb, mat, m0, orow0;
+      decode(tile, seg, nb, mat, m0, orow0);
+      const int row = m0 + 32 * q + lane;  // row within matrix `mat`
       const int n0 = nb * NOUT;
-      const bool row_ok = row < g.M;
+      const bool row_ok = row < g.Am[mat];
       const uint32_t taddr = tmem + (uint32_t)(acc * BN) + ((uint32_t)(32 * q) << 16);
-      if (EPI == TC_EPI_STORE_F32) {
+      if (EPI == TC_EPI_STORE_T_PAIRS_F32) {
+        // columns (2j, 2j+1) hold batch row j's hi and lo terms: fold them
+        float* o = static_cast<float*>(g.out) + (size_t)seg * g.out_seg + orow0 + 32 * q + lane;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int col = n0 + c + 2 * j;
+              if (col < g.N)
+                o[(size_t)(col >> 1) * g.ldo] = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+            }
+          }
+        }
+      } else if (EPI == TC_EPI_STORE_T_F32) {
+        // thread = one output row, 32 consecutive batch columns per TMEM load;
+        // across the warp the stores to one batch column are contiguous
+        float* o = static_cast<float*>(g.out) + (size_t)seg * g.out_seg + orow0 + 32 * q + lane;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + c + j < g.N) o[(size_t)(n0 + c + j) * g.ldo] = __uint_as_float(v[j]);
+          }
+        }
+      } else if (EPI == TC_EPI_STORE_F32) {
         float* o = static_cast<float*>(g.out) + (size_t)seg * g.out_seg + (size_t)row * g.ldo + n0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -352,27 +418,31 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D map over a bf16 row-major matrix [rows, inner] with row stride ld elements,
-// box = 64 elements (128 bytes) x box_rows, 128-byte swizzle, zero fill outside.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t inner, int64_t ld,
+// 3D map over a bf16 row-major matrix whose first nseg*K columns are nseg
+// segments of K: dims {K, nseg, rows}, strides {K*2, ld*2} bytes (the matrix's
+// own memory order), box = 64 elements (128 bytes) x 1 segment x box_rows,
+// 128-byte swizzle, zero fill outside (so a partial last K block of a segment
+// reads zeros, not the next segment).
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int nseg, int64_t K, int64_t ld,
               int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+  cuuint64_t gdim[3] = {(cuuint64_t)K, (cuuint64_t)nseg, (cuuint64_t)rows};
+  cuuint64_t gstride[2] = {(cuuint64_t)K * 2, (cuuint64_t)ld * 2};
+  cuuint32_t box[3] = {(cuuint32_t)BK, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
-int launch_epi(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mB2,
-               const TcGemm& g, int num_m, int num_n, int ntiles, cudaStream_t s) {
-  if (set_smem_once((const void*)k_tc_gemm<EPI>, SMEM_BYTES)) return TP_ECUDA;
-  int grid = ntiles < num_sms() ? ntiles : num_sms();
-  k_tc_gemm<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(mA, mB, mB2, g, num_m, num_n, ntiles);
+template <int BN, int EPI>
+int launch_cfg(const CUtensorMap* mA, const CUtensorMap& mB, const CUtensorMap& mB2,
+               const TcGemm& g, const TcTiles& tt, cudaStream_t s) {
+  constexpr int smem = TcCfg<BN>::SMEM_BYTES;
+  if (set_smem_once((const void*)k_tc_gemm<BN, EPI>, smem)) return TP_ECUDA;
+  int grid = tt.ntiles < num_sms() ? tt.ntiles : num_sms();
+  k_tc_gemm<BN, EPI><<<grid, THREADS, smem, s>>>(mA[0], mA[1], mA[2], mB, mB2, g, tt);
   TP_LAUNCH_CHECK();
   return TP_OK;
 }
@@ -380,26 +450,48 @@ int launch_epi(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& 
 }  // namespace
 
 int launch_tc_gemm(const TcGemm& g, cudaStream_t s) {
-  if (g.M < 1 || g.N < 1 || g.K < BK || g.K % BK != 0 || g.nseg < 1) return TP_EINVAL;
-  if (g.N % 32 != 0 || g.lda % 8 != 0 || g.ldb % 8 != 0 || g.ldo % 8 != 0) return TP_EINVAL;
+  if (g.nA < 1 || g.nA > 3 || g.N < 1 || g.K < 8 || g.K % 8 != 0 || g.nseg < 1) return TP_EINVAL;
+  if (g.lda % 8 != 0 || g.ldb % 8 != 0) return TP_EINVAL;
+  if ((int64_t)g.nseg * g.K > g.lda || (int64_t)g.nseg * g.K > g.ldb) return TP_EINVAL;
   const bool swiglu = g.epi == TC_EPI_SWIGLU_BF16;
+  const bool trans = g.epi == TC_EPI_STORE_T_F32 || g.epi == TC_EPI_STORE_T_PAIRS_F32;
   if (swiglu && !g.B2) return TP_EINVAL;
-  const int64_t inner = (int64_t)g.nseg * g.K;
-  CUtensorMap mA, mB, mB2;
+  if (!trans && (g.N % 32 != 0 || g.ldo % 8 != 0 || g.nA != 1)) return TP_EINVAL;
+  if (trans && g.N > 128) return TP_EINVAL;
+  if (g.epi == TC_EPI_STORE_T_PAIRS_F32 && (g.N & 1)) return TP_EINVAL;
+  const int BN = trans ? (g.N <= 32 ? 32 : (g.N <= 64 ? 64 : 128)) : 256;
+  CUtensorMap mA[3], mB, mB2;
+  TcTiles tt{};
+  tt.mt_off[0] = 0;
+  for (int j = 0; j < 3; ++j) {
+    const int jj = j < g.nA ? j : 0;
+    if (g.Am[jj] < 1) return TP_EINVAL;
+    if (!make_map(&mA[j], g.A[jj], g.Am[jj], g.nseg, g.K, g.lda, BM)) return TP_ECUDA;
+    tt.mt_off[j + 1] = tt.mt_off[j] + (j < g.nA ? (g.Am[j] + BM - 1) / BM : 0);
+  }
   const int brows = swiglu ? BN / 2 : BN;
-  if (!make_map(&mA, g.A, g.M, inner, g.lda, BM) || !make_map(&mB, g.B, g.N, inner, g.ldb, brows) ||
-      !make_map(&mB2, swiglu ? g.B2 : g.B, g.N, inner, g.ldb, brows))
+  if (!make_map(&mB, g.B, g.N, g.nseg, g.K, g.ldb, brows) ||
+      !make_map(&mB2, swiglu ? g.B2 : g.B, g.N, g.nseg, g.K, g.ldb, brows))
     return TP_ECUDA;
   const int nout = swiglu ? BN / 2 : BN;
-  const int num_m = (g.M + BM - 1) / BM;
-  const int num_n = (g.N + nout - 1) / nout;
-  const int64_t nt = (int64_t)num_m * num_n * g.nseg;
+  tt.num_n = (g.N + nout - 1) / nout;
+  const int64_t nt = (int64_t)tt.mt_off[3] * tt.num_n * g.nseg;
   if (nt > 0x7fffffff) return TP_EINVAL;
+  tt.ntiles = (int)nt;
+  if (g.epi == TC_EPI_STORE_T_PAIRS_F32) {
+    if (BN == 32) return launch_cfg<32, TC_EPI_STORE_T_PAIRS_F32>(mA, mB, mB2, g, tt, s);
+    if (BN == 64) return launch_cfg<64, TC_EPI_STORE_T_PAIRS_F32>(mA, mB, mB2, g, tt, s);
+    return launch_cfg<128, TC_EPI_STORE_T_PAIRS_F32>(mA, mB, mB2, g, tt, s);
+  }
+  if (trans) {
+    if (BN == 32) return launch_cfg<32, TC_EPI_STORE_T_F32>(mA, mB, mB2, g, tt, s);
+    if (BN == 64) return launch_cfg<64, TC_EPI_STORE_T_F32>(mA, mB, mB2, g, tt, s);
+    return launch_cfg<128, TC_EPI_STORE_T_F32>(mA, mB, mB2, g, tt, s);
+  }
   switch (g.epi) {
-    case TC_EPI_STORE_F32: return launch_epi<TC_EPI_STORE_F32>(mA, mB, mB2, g, num_m, num_n, (int)nt, s);
-    case TC_EPI_RELU_BF16: return launch_epi<TC_EPI_RELU_BF16>(mA, mB, mB2, g, num_m, num_n, (int)nt, s);
-    case TC_EPI_SWIGLU_BF16:
-      return launch_epi<TC_EPI_SWIGLU_BF16>(mA, mB, mB2, g, num_m, num_n, (int)nt, s);
+    case TC_EPI_STORE_F32: return launch_cfg<256, TC_EPI_STORE_F32>(mA, mB, mB2, g, tt, s);
+    case TC_EPI_RELU_BF16: return launch_cfg<256, TC_EPI_RELU_BF16>(mA, mB, mB2, g, tt, s);
+    case TC_EPI_SWIGLU_BF16: return launch_cfg<256, TC_EPI_SWIGLU_BF16>(mA, mB, mB2, g, tt, s);
     default: return TP_EINVAL;
   }
 }

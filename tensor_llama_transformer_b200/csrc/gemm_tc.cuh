@@ -1,4 +1,5 @@
-// Tensor-core (tcgen05 / TMEM / TMA) contraction for the batched FFN.
+// Tensor-core (tcgen05 / TMEM / TMA) contraction: the batched FFN and the
+// batched decode slice products.
 #pragma once
 
 #include "common.cuh"
@@ -6,25 +7,36 @@
 namespace tp {
 
 enum TcEpi {
-  TC_EPI_STORE_F32 = 0,    // out[seg][m][n] = acc                       (float32)
+  TC_EPI_STORE_F32 = 0,    // out[seg][m][n] = acc                        (float32)
   TC_EPI_RELU_BF16 = 1,    // out[m][n] = bf16(max(acc, 0))
-  TC_EPI_SWIGLU_BF16 = 2,  // out[m][n] = bf16(silu(acc_W1) * acc_W3)   (B = W1, B2 = W3)
+  TC_EPI_SWIGLU_BF16 = 2,  // out[m][n] = bf16(silu(acc_W1) * acc_W3)    (B = W1, B2 = W3)
+  TC_EPI_STORE_T_F32 = 3,  // out[seg][n][row_off(matrix) + m] = acc     (transposed float32)
+  TC_EPI_STORE_T_PAIRS_F32 = 4,  // as 3 with B rows in hi/lo pairs: out[seg][n/2][..] = acc_2j + acc_2j+1
 };
 
 // D[seg, m, n] = sum_{k < K} A[m, seg*K + k] * B[n, seg*K + k]
-// A [M, lda] and B [N, ldb] are bf16 row-major (contraction dimension contiguous).
+// A and B are bf16 row-major with the contraction dimension contiguous. Up to
+// three A matrices (same K and leading dimension) may be given; their rows are
+// concatenated, which TC_EPI_STORE_T_F32 reproduces in its output rows. The FFN
+// uses A = activations [tokens, K], B = weights [features, K]; batched decode
+// uses A = weights [rows, K], B = activations [batch, K] (N <= 128) with the
+// transposed store, so that each partial plane is [batch, rows]; with the
+// activations given as hi/lo bf16 row pairs (N = 2 x batch) the pair-folding
+// store adds the two columns of each batch row.
 struct TcGemm {
-  const void* A;
+  const void* A[3];
+  int Am[3];        // rows of each A matrix
+  int nA;           // 1..3
   int64_t lda;
   const void* B;
   int64_t ldb;
   const void* B2;   // second B operand (SwiGLU gate), same shape as B
-  int M, N, K;      // K = contraction length of one segment
+  int N, K;         // K = contraction length of one segment
   int nseg;
   int epi;
   void* out;
   int64_t ldo;
-  int64_t out_seg;  // elements between segment planes (TC_EPI_STORE_F32)
+  int64_t out_seg;  // elements between segment planes (float32 stores)
   int* err;         // device flag set to 1 when a pipeline wait gives up (nullable: not reported)
 };
 

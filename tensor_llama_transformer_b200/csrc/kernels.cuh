@@ -86,11 +86,45 @@ struct AttnArgs {
   float* part_o;        // [B, H, nchunk, hd] unnormalised partial outputs
   float* part_ml;       // [B, H, nchunk, 2] running max and sum
   float* att;           // [B, H*hd] combined output
-  uint16_t* att_bf16;   // optional bf16 copy
+  uint16_t* att_bf16;   // optional hi/lo bf16 pairs [2B, H*hd] (rows 2b, 2b+1)
   int* err;             // device error flag (bounded waits)
 };
 
 int launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------------ batched decode
+// Batches at least this large run the slice products on the tcgen05 GEMM (the
+// weights as the M operand, the batch as N); smaller ones on the ring GEMV.
+constexpr int kTcMinBatch = 6;
+
+struct NormRowsArgs {
+  const float* x;      // residual [B, dim]
+  const float* gain;   // [dim]
+  const float* ssq;    // optional per-row partial sums of squares [B][ssq_parts]
+  int ssq_parts;
+  int dim;
+  float eps;
+  int quant;
+  int8_t* xq;          // Q8 codes [B, dim] (nullable)
+  float* xd;           // Q8 scales [B, dim/32] (nullable)
+  float* xn;           // float32 value the slices read (nullable)
+  uint16_t* xb;        // that value as hi/lo bf16 pairs [2B, dim] (tensor-core operand)
+};
+int launch_norm_rows(const NormRowsArgs& a, int batch, cudaStream_t s);
+
+struct QkvFinalizeArgs {
+  const float* plane;  // [parts][batch][qd + 2 kd]
+  int parts, batch, qd, kd;
+  const int32_t* pos;
+  float theta;
+  float* q;            // [batch, qd]
+  uint16_t* kc;
+  uint16_t* vc;
+  int n_kv_heads, max_seq;
+};
+int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s);
+int launch_swiglu_finalize(const float* plane, int F, int batch, float* h, uint16_t* hb,
+                           cudaStream_t s);
 
 // One block forward over a caller-provided workspace with a handle on the stack
 // (api.cu); zeroes the kernels' error word in the workspace first.

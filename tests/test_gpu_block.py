@@ -143,4 +143,27 @@ def test_block_c2_slices_agree(tpb):
 def test_block_c4_full_size(tpb):
     """70B-shape GQA block: dim 8192, 64 q heads over 8 kv heads, batch 32, context 4096, n = 8."""
     inp = synth.block_inputs(synth.CONFIG_SEED["C4"], synth.C4)
-    check_block(tpb, inp, synth.C4.n_slices, 0, tight=2e-3, name="C4")
+    # batch 32 runs on the tensor cores with bf16 activations: expected level ~5e-3
+    check_block(tpb, inp, synth.C4.n_slices, 0, tight=1e-2, name="C4")
+
+
+# Batches of 6 or more run the slice products on the tcgen05 GEMM (weights as the M
+# operand, the batch as N) instead of the ring GEMV.
+SMALL_TC_GQA = synth.BlockShape(dim=512, n_heads=8, n_kv_heads=2, head_dim=128, ffn_dim=1024,
+                                vocab=0, max_seq=200, batch=8, n_slices=2, sync_quant=False,
+                                pos=199, w_std=0.04)
+SMALL_TC_MHA = synth.BlockShape(dim=1024, n_heads=8, n_kv_heads=8, head_dim=128, ffn_dim=2816,
+                                vocab=0, max_seq=130, batch=13, n_slices=8, sync_quant=False,
+                                pos=129, w_std=0.03)
+
+
+@pytest.mark.parametrize("quant", [0, 1])
+@pytest.mark.parametrize("shape,n,partition", [
+    (SMALL_TC_GQA, 2, 1), (SMALL_TC_GQA, 2, 2), (SMALL_TC_MHA, 8, 1)])
+def test_block_batched_tensor_path(tpb, shape, n, partition, quant):
+    inp = synth.block_inputs(5252, shape)
+    B = shape.batch
+    inp.pos[:] = [(shape.pos * (i + 1)) // B for i in range(B)]  # ragged contexts
+    # bf16 operands on the tensor cores: 2e-2 bar, ~5e-3 expected level
+    check_block(tpb, inp, n, quant, partition=partition, tight=1e-2,
+                name=f"tc d{shape.dim} B{B} n{n} p{partition} q{quant}")
