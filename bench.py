@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-ffn", action="store_true", help="skip the PaLM FFN measurement")
     ap.add_argument("--ffn-iters", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the C4 block and C3 model measurements")
     return ap.parse_args(argv)
 
 
@@ -354,6 +356,113 @@ def bench_block(args, world, rank, local):
     return res
 
 
+def _randn_bf16(torch, gen, shape, std):
+    out = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    flat = out.view(-1)
+    step = 1 << 26
+    for o in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - o)
+        flat[o:o + n] = (torch.randn(n, generator=gen, device="cuda") * std).to(torch.bfloat16)
+    return out
+
+
+def _time_graph(torch, fn, steps_per_graph, replays, warm=2):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(steps_per_graph):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / (steps_per_graph * replays)
+    del g
+    return ms
+
+
+def bench_c4(args):
+    """70B-shape GQA block (dim 8192, 64/8 heads, F 28672), batch 32, context 4096, n = 8."""
+    import torch
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+
+    s = synth.C4
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1003)
+    B, D, F, H, Hkv, hd = s.batch, s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim
+    w = [torch.ones(D, device="cuda"), _randn_bf16(torch, gen, (H * hd, D), s.w_std),
+         _randn_bf16(torch, gen, (Hkv * hd, D), s.w_std), _randn_bf16(torch, gen, (Hkv * hd, D), s.w_std),
+         _randn_bf16(torch, gen, (D, H * hd), s.w_std), torch.ones(D, device="cuda"),
+         _randn_bf16(torch, gen, (F, D), s.w_std), _randn_bf16(torch, gen, (F, D), s.w_std),
+         _randn_bf16(torch, gen, (D, F), s.w_std)]
+    kc = _randn_bf16(torch, gen, (B, Hkv, s.max_seq, hd), 1.0)
+    vc = _randn_bf16(torch, gen, (B, Hkv, s.max_seq, hd), 1.0)
+    x = torch.randn((B, D), generator=gen, device="cuda")
+    pos = torch.full((B,), s.pos, dtype=torch.int32, device="cuda")
+    dims = tpb.make_dims(D, H, Hkv, hd, F, s.vocab, B, s.max_seq, s.norm_eps, s.rope_theta)
+    nb = tpb.tp_block_workspace_bytes(dims, s.n_slices, 1, 0)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    h = tpb.tp_block_create(dims, s.n_slices, 1, 0, tpb.make_weights(*w), ws, nb)
+    ms = _time_graph(torch, lambda: tpb.tp_block_forward(h, x, kc, vc, pos, B), 10, 5)
+    tpb.tp_block_destroy(h)
+    wb, kvb = block_bytes(s)
+    hbm, _, _, kind = peaks()
+    gbs = (wb + kvb) / (ms / 1e3) / 1e9
+    return {"us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "hbm_gbs": gbs,
+            "frac": gbs / hbm, "bytes_per_step": wb + kvb,
+            "workload": "C4: 70B-shape GQA block, dim 8192, 64/8 heads, SwiGLU 28672, batch 32, "
+                        "context 4096, n=8, float32 sync buffers"}
+
+
+def bench_c3(args, B):
+    """Full 32-layer Llama-2-7B-shaped decode step (embedding -> logits), context 4096, n = 8."""
+    import torch
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+
+    s = synth.C3
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1002)
+    D, F, H, Hkv, hd, L, V = s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim, s.n_layers, s.vocab
+    ones = torch.ones(D, device="cuda")
+    layers, keep = [], []
+    for _ in range(L):
+        t = [_randn_bf16(torch, gen, shp, s.w_std) for shp in
+             ((H * hd, D), (Hkv * hd, D), (Hkv * hd, D), (D, H * hd), (F, D), (F, D), (D, F))]
+        keep.append(t)
+        layers.append(tpb.make_weights(ones, t[0], t[1], t[2], t[3], ones, t[4], t[5], t[6]))
+    emb = _randn_bf16(torch, gen, (V, D), s.w_std)
+    wcls = _randn_bf16(torch, gen, (V, D), s.w_std)
+    kc = _randn_bf16(torch, gen, (L, B, Hkv, s.max_seq, hd), 1.0)
+    vc = _randn_bf16(torch, gen, (L, B, Hkv, s.max_seq, hd), 1.0)
+    toks = torch.randint(0, V, (B,), generator=gen, device="cuda", dtype=torch.int32)
+    pos = torch.full((B,), s.pos, dtype=torch.int32, device="cuda")
+    logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
+    dims = tpb.make_dims(D, H, Hkv, hd, F, V, B, s.max_seq, s.norm_eps, s.rope_theta)
+    nb = tpb.tp_model_workspace_bytes(dims, L, s.n_slices, 1, 0)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    m = tpb.tp_model_create(dims, L, s.n_slices, 1, 0, layers, emb, ones, wcls, ws, nb)
+    ms = _time_graph(torch, lambda: tpb.tp_model_forward(m, toks, kc, vc, pos, B, logits), 3, 5)
+    tpb.tp_model_destroy(m)
+    wb = L * block_bytes(s)[0] + V * D * 2  # every layer's weights + the classifier
+    kvb = L * 2 * B * Hkv * (s.pos + 1) * hd * 2
+    hbm, _, _, kind = peaks()
+    gbs = (wb + kvb) / (ms / 1e3) / 1e9
+    return {"ms_per_step": ms, "tokens_per_s": B / (ms / 1e3), "hbm_gbs": gbs, "frac": gbs / hbm,
+            "bytes_per_step": wb + kvb,
+            "workload": f"C3: 32-layer Llama-2-7B-shaped decode, vocab 32000, context 4096, n=8, "
+                        f"batch {B}"}
+
+
 def bench_ffn(args):
     """PaLM FFN (E 18432, F 73728, B 512, ReLU) through tp_ffn_forward; TFLOP/s per form."""
     import torch
@@ -422,6 +531,16 @@ def main(argv=None):
     world, rank, local = dist_setup()
     res = bench_block(args, world, rank, local)
     ffn = None if args.no_ffn else bench_ffn(args)
+    extra = None
+    if not args.no_extra:
+        import torch
+
+        extra = {"c4_block": bench_c4(args)}
+        torch.cuda.empty_cache()
+        extra["c3_model_b1"] = bench_c3(args, 1)
+        torch.cuda.empty_cache()
+        extra["c3_model_b16"] = bench_c3(args, 16)
+        torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
@@ -451,6 +570,7 @@ def main(argv=None):
             "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
             "ffn_b512": ffn,
+            "extra": extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

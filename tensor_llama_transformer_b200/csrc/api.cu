@@ -126,7 +126,7 @@ int check_cfg(const tp_dims* d, int n, int partition, int quant, Cfg* c) {
     c->gx = 1;
     c->gy = n;
   }
-  c->nchunk = (d->max_seq + kAttnChunk - 1) / kAttnChunk;
+  c->nchunk = attention_max_splits(d->max_seq);
   return TP_OK;
 }
 

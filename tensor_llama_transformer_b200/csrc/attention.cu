@@ -1,196 +1,351 @@
-// Decode attention over the bf16 KV cache, split over the context.
+// Decode attention over the bf16 KV cache: split-context flash decoding on
+// warp-level tensor-core MMAs.
 //
 // distributed-llama issue #29, llamaMultiheadAtt: each slice computes the
 // attention of its own heads locally; tt-metal's Llama-2 thread separates GQA
-// from MHA. One CTA owns (batch row b, kv head, context chunk of 128
-// positions) and all the query heads that share that kv head (1 for MHA, 8 for
-// the 70B shape), so a K/V tile read from HBM serves every head of its group.
-// The chunk's K and V rows are contiguous in the cache and arrive in shared
-// memory by two bulk asynchronous copies (cp.async.bulk, completion counted on
-// an mbarrier). Each CTA writes an unnormalised partial (o, running max m,
-// sum l); a second kernel combines the chunks with the usual rescaling
+// from MHA. A CTA owns (context split, kv head, batch row) and every query head
+// that reads that kv head (1 for MHA, 8 for the 70B shape), so each K/V byte is
+// read from HBM once per step. The split's 64-position K and V tiles stream
+// through a 3-stage shared-memory ring by TMA (128-byte swizzle, so the
+// ldmatrix reads below are conflict-free), issued by a producer warp. Four
+// consumer warps take 16 positions of each tile:
+//   S = Q K^T and O += P V on mma.m16n8k16 (bf16 operands, float32 accumulate),
+//   with an online softmax in registers (running max m, sum l, rescaled O).
+// Q and P enter the MMAs as hi/lo bf16 pairs in the two 8-row halves of the
+// 16-row operand (row g holds bf16(v), row g+8 holds bf16(v - bf16(v)) for head
+// g of the group), so the products keep about 16 significant bits; the halves
+// of S and of O are added in registers. The warps' partials are merged in
+// shared memory and the split writes one unnormalised partial (o, m, l) per
+// head; a second kernel combines the splits with the usual rescaling
 //   M = max_c m_c,  o = sum_c e^{m_c - M} o_c / sum_c e^{m_c - M} l_c.
+// Positions past pos are masked (score -inf, and the V rows zeroed in shared
+// memory), so stale cache contents never reach the output. The MMAs do at most
+// 16 FLOP per KV byte, far below the tensor pipe's rate: the kernel is HBM-bound.
+#include "gemm_tc.cuh"
 #include "kernels.cuh"
 
 namespace tp {
 
 namespace {
 
-constexpr int kAttnThreads = 128;
-constexpr uint32_t kSpinLimit = 1u << 26;  // bounded wait on the copy barrier
+constexpr int kTile = 64;                // positions per tile
+constexpr int kStages = 3;
+constexpr int kCWarps = 4;               // consumer warps, 16 positions of each tile
+constexpr int kAThreads = 32 * (kCWarps + 1);
+constexpr int kBox = kTile * 64 * 2;     // one box: 64 positions x 64 dims of bf16 (8 KB)
+constexpr int kStageBytes = 4 * kBox;    // K (two dim halves) + V (two dim halves)
+constexpr int kQStride = 136;            // staged Q row stride (bf16), padded against conflicts
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 16 * kQStride * 2;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+static_assert(kCWarps * 8 * kHeadDim * 4 <= kStageBytes, "merge staging must fit in stage 0");
 
-TP_DEV uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+TP_DEV uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
 
-TP_DEV void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+TP_DEV void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
 }
 
-TP_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
+TP_DEV void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
                : "memory");
 }
 
-TP_DEV bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+TP_DEV void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
+}
+
+TP_DEV bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(phase)
+      : "r"(s2u(b)), "r"(parity)
       : "memory");
   return ok != 0;
 }
 
-TP_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+// Bounded wait: gives up after kTimeoutNs and raises the error word.
+TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(b, parity)) return true;
+    if ((i & 255) == 0 && gtimer() - t0 > kTimeoutNs) {
+      if (err) atomicExch(err, 1);
+      return false;
+    }
+  }
+}
+
+TP_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(s2u(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(s2u(bar))
       : "memory");
 }
 
-template <int G>
-__global__ void __launch_bounds__(kAttnThreads) k_attn_chunk(AttnArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);                  // [128][128]
-  uint16_t* Vs = Ks + kAttnChunk * kHeadDim;                         // [128][128]
-  float* qs = reinterpret_cast<float*>(Vs + kAttnChunk * kHeadDim);  // [G][128]
-  float* ps = qs + G * kHeadDim;                                     // [G][128]
-  float* red = ps + G * kAttnChunk;                                  // [2][G][4]
-  __shared__ uint64_t bar;
+TP_DEV void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
 
-  const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x;
+TP_DEV void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D (16x8 float32) += A (16x16 bf16, row-major) * B (16x8 bf16, column-major)
+TP_DEV void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3},"
+      " {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+TP_DEV uint32_t pack_bf16x2(uint16_t first, uint16_t second) {
+  return (uint32_t)first | ((uint32_t)second << 16);
+}
+
+// Shared address of 16-byte chunk c (8 dims, 0..15) of row t (0..63) of a K or
+// V tile that TMA wrote as two 64-dim boxes with the 128-byte swizzle.
+TP_DEV uint32_t tile_addr(uint32_t base, int t, int c) {
+  return base + (uint32_t)((c >> 3) * kBox + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
+// Tiles of one split for a context of P positions: the same for both kernels.
+TP_DEV int tiles_per_split(int P, int nsplit) {
+  const int ntiles = (P + kTile - 1) / kTile;
+  return (ntiles + nsplit - 1) / nsplit;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant__ CUtensorMap mK,
+                                                          const __grid_constant__ CUtensorMap mV,
+                                                          AttnArgs a, int nsplit) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint16_t* qs = reinterpret_cast<uint16_t*>(smem + kStages * kStageBytes);  // [16][kQStride]
+  __shared__ uint64_t full[kStages], empty[kStages];
+  __shared__ float s_m[kCWarps][8], s_l[kCWarps][8];
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
-  pdl_wait();  // q and the cache row at pos come from the q/k/v kernel
+  pdl_wait();  // q and the cache rows at pos come from the q/k/v kernel
   const int P = a.pos[b] + 1;
-  const int t0 = c * kAttnChunk;
-  const size_t pbase = ((size_t)b * a.H + (size_t)kvh * G) * a.nchunk + c;
-  if (t0 >= P) {
-    if (tid < G) {
-      a.part_ml[(pbase + (size_t)tid * a.nchunk) * 2 + 0] = -INFINITY;
-      a.part_ml[(pbase + (size_t)tid * a.nchunk) * 2 + 1] = 0.f;
+  const int ntiles = (P + kTile - 1) / kTile;
+  const int tpc = tiles_per_split(P, nsplit);
+  const int i0 = split * tpc, i1 = min(ntiles, i0 + tpc);
+  const size_t pbase = ((size_t)b * a.H + (size_t)kvh * G) * nsplit + split;
+  if (i0 >= i1) {  // nothing left for this split (the combine does not read it)
+    if (threadIdx.x < G) {
+      a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 0] = -INFINITY;
+      a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 1] = 0.f;
     }
     return;
   }
-  const int nt = min(kAttnChunk, P - t0);
-  const uint32_t bytes = (uint32_t)nt * kHeadDim * 2;
-  const size_t row0 = (((size_t)b * a.Hkv + kvh) * a.max_seq + t0) * kHeadDim;
+  const int row_base = (b * a.Hkv + kvh) * a.max_seq;
 
-  if (tid == 0) {
-    mbar_init(&bar, 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCWarps);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    mbar_expect_tx(&bar, 2 * bytes);
-    bulk_g2s(Ks, a.kc + row0, bytes, &bar);
-    bulk_g2s(Vs, a.vc + row0, bytes, &bar);
   }
-  // q of the group's heads, pre-scaled by 1/sqrt(hd)
+  // Q of the group's heads scaled by 1/sqrt(hd): hi in row g, lo in row g + 8
   const float scale = 1.0f / sqrtf((float)kHeadDim);
-  for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
+  for (int i = threadIdx.x; i < 8 * kHeadDim; i += kAThreads) {
     const int g = i / kHeadDim, d = i - g * kHeadDim;
-    qs[i] = a.q[((size_t)b * a.H + (size_t)kvh * G + g) * kHeadDim + d] * scale;
-  }
-  __syncthreads();
-  {
-    uint32_t spins = 0;
-    while (!mbar_try_wait(&bar, 0)) {
-      if (++spins > kSpinLimit) {
-        if (tid == 0) atomicExch(a.err, 1);
-        break;
-      }
-    }
-  }
-
-  // scores: thread t owns position t0+t; reads its K row in 16-byte chunks with a
-  // per-thread rotation so that the 8 threads of a quarter-warp hit 8 different
-  // bank groups.
-  float s[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) s[g] = -INFINITY;
-  if (tid < nt) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) s[g] = 0.f;
-    const uint4* krow = reinterpret_cast<const uint4*>(Ks + tid * kHeadDim);
-#pragma unroll 4
-    for (int j = 0; j < 16; ++j) {
-      const int cch = (j + tid) & 15;
-      const uint4 kv = krow[cch];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float4 q0 = reinterpret_cast<const float4*>(qs + g * kHeadDim)[2 * cch];
-        const float4 q1 = reinterpret_cast<const float4*>(qs + g * kHeadDim)[2 * cch + 1];
-        float acc = s[g];
-        acc = fmaf(bf16lo(kv.x), q0.x, acc);
-        acc = fmaf(bf16hi(kv.x), q0.y, acc);
-        acc = fmaf(bf16lo(kv.y), q0.z, acc);
-        acc = fmaf(bf16hi(kv.y), q0.w, acc);
-        acc = fmaf(bf16lo(kv.z), q1.x, acc);
-        acc = fmaf(bf16hi(kv.z), q1.y, acc);
-        acc = fmaf(bf16lo(kv.w), q1.z, acc);
-        acc = fmaf(bf16hi(kv.w), q1.w, acc);
-        s[g] = acc;
-      }
-    }
-  }
-  // softmax over the chunk (per head of the group)
-  const int lane = tid & 31, wid = tid >> 5;
-  float* rmax = red;
-  float* rsum = red + G * 4;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float m = warp_max(s[g]);
-    if (lane == 0) rmax[g * 4 + wid] = m;
-  }
-  __syncthreads();
-  float mg[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    mg[g] = fmaxf(fmaxf(rmax[g * 4 + 0], rmax[g * 4 + 1]), fmaxf(rmax[g * 4 + 2], rmax[g * 4 + 3]));
-    const float p = tid < nt ? expf(s[g] - mg[g]) : 0.f;
-    ps[g * kAttnChunk + tid] = p;
-    const float l = warp_sum(p);
-    if (lane == 0) rsum[g * 4 + wid] = l;
+    uint16_t hi = 0, lo = 0;
+    if (g < G)
+      bf16_split(a.q[((size_t)b * a.H + (size_t)kvh * G + g) * kHeadDim + d] * scale, hi, lo);
+    qs[g * kQStride + d] = hi;
+    qs[(g + 8) * kQStride + d] = lo;
   }
   __syncthreads();
 
-  // o[g][d] = sum_t p[g][t] v[t][d]; thread tid owns dimension d = tid
-  float o[G];
+  if (warp == kCWarps) {
+    // ------------------------------------------------------------ producer warp
+    if (lane == 0) {
+      for (int i = i0; i < i1; ++i) {
+        const int k = i - i0, s = k % kStages;
+        if (!mbar_wait(&empty[s], ((uint32_t)(k / kStages) & 1u) ^ 1u, a.err)) break;
+        mbar_expect_tx(&full[s], kStageBytes);
+        uint8_t* st = smem + s * kStageBytes;
+        const int y = row_base + i * kTile;
+        tma_load_2d(st, &mK, 0, y, &full[s]);
+        tma_load_2d(st + kBox, &mK, 64, y, &full[s]);
+        tma_load_2d(st + 2 * kBox, &mV, 0, y, &full[s]);
+        tma_load_2d(st + 3 * kBox, &mV, 64, y, &full[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumer warps
+    const int g = lane >> 2;  // the head row whose scores this thread holds
+    uint32_t qa[8][4];        // A fragments of Q, one per 16-dim step
+    {
+      const uint32_t qb = s2u(qs);
+      const int r = (lane & 7) + 8 * ((lane >> 3) & 1), ch = lane >> 4;
 #pragma unroll
-  for (int g = 0; g < G; ++g) o[g] = 0.f;
-  const int d = tid;
-#pragma unroll 4
-  for (int t = 0; t < nt; ++t) {
-    const float v = __uint_as_float(((uint32_t)Vs[t * kHeadDim + d]) << 16);
+      for (int ks = 0; ks < 8; ++ks)
+        ldsm_x4(qb + (uint32_t)((r * kQStride + 16 * ks + 8 * ch) * 2), qa[ks]);
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[16][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) o[g] = fmaf(ps[g * kAttnChunk + t], v, o[g]);
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    bool ok = true;
+    const int w0 = 16 * warp;  // this warp's positions within a tile
+    for (int i = i0; i < i1; ++i) {
+      const int k = i - i0, s = k % kStages;
+      const bool got = ok ? mbar_wait(&full[s], (uint32_t)(k / kStages) & 1u, a.err) : false;
+      ok = __all_sync(0xffffffffu, got);
+      if (ok) {
+        const uint32_t kb = s2u(smem + s * kStageBytes), vb = kb + 2 * kBox;
+        const int t0 = i * kTile;
+        if (t0 + w0 + 16 > P) {  // V rows past pos -> 0 (only the context's last tile)
+          for (int idx = lane; idx < 16 * 16; idx += 32) {
+            const int r = idx >> 4, c = idx & 15;
+            if (t0 + w0 + r >= P)
+              *reinterpret_cast<uint4*>(smem + (tile_addr(vb, w0 + r, c) - s2u(smem))) =
+                  make_uint4(0u, 0u, 0u, 0u);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
+        // S = Q K^T over the warp's two 8-position column tiles
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+          const int t = w0 + (lane & 7) + 8 * (lane >> 4), ch = (lane >> 3) & 1;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            uint32_t bf[4];
+            ldsm_x4(tile_addr(kb, t, 2 * ks + ch), bf);
+            mma_bf16(sc[0], qa[ks], bf[0], bf[1]);
+            mma_bf16(sc[1], qa[ks], bf[2], bf[3]);
+          }
+        }
+        // this thread's scores of head g: positions t0 + w0 + 8 nt + 2 (lane & 3) + j
+        float sv[2][2], tmax = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int tp = t0 + w0 + 8 * nt + 2 * (lane & 3) + j;
+            const float v = sc[nt][j] + sc[nt][2 + j];  // hi row + lo row
+            sv[nt][j] = tp < P ? v : -INFINITY;
+            tmax = fmaxf(tmax, sv[nt][j]);
+          }
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+        const float m_new = fmaxf(m_run, tmax);
+        const float resc = m_new == -INFINITY ? 1.f : expf(m_run - m_new);
+        uint16_t ph[2][2], pl[2][2];
+        float psum = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float p = sv[nt][j] == -INFINITY ? 0.f : expf(sv[nt][j] - m_new);
+            psum += p;
+            bf16_split(p, ph[nt][j], pl[nt][j]);
+          }
+        const uint32_t pa[4] = {pack_bf16x2(ph[0][0], ph[0][1]), pack_bf16x2(pl[0][0], pl[0][1]),
+                                pack_bf16x2(ph[1][0], ph[1][1]), pack_bf16x2(pl[1][0], pl[1][1])};
+        l_run = l_run * resc + psum;
+        m_run = m_new;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          o[nt][0] *= resc;
+          o[nt][1] *= resc;
+          o[nt][2] *= resc;
+          o[nt][3] *= resc;
+        }
+        // O += P V over the warp's 16 positions, 16 dim tiles of 8
+        {
+          const int t = w0 + (lane & 7) + 8 * ((lane >> 3) & 1), ch = lane >> 4;
+#pragma unroll
+          for (int np = 0; np < 8; ++np) {
+            uint32_t bf[4];
+            ldsm_x4_t(tile_addr(vb, t, 2 * np + ch), bf);
+            mma_bf16(o[2 * np], pa, bf[0], bf[1]);
+            mma_bf16(o[2 * np + 1], pa, bf[2], bf[3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // the warp's partial of head g: l summed over the row's 4 lanes
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    if ((lane & 3) == 0) {
+      s_m[warp][g] = m_run;
+      s_l[warp][g] = l_run;
+    }
+    // every tile has been consumed by all consumer warps: stage 0 takes the O partials
+    asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32) : "memory");
+    float* ro = reinterpret_cast<float*>(smem);  // [kCWarps][8][kHeadDim]
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      const int d = 8 * nt + 2 * (lane & 3);
+      ro[(warp * 8 + g) * kHeadDim + d] = o[nt][0] + o[nt][2];
+      ro[(warp * 8 + g) * kHeadDim + d + 1] = o[nt][1] + o[nt][3];
+    }
   }
+  __syncthreads();
+  // merge the consumer warps: thread per (head, dim)
+  const float* ro = reinterpret_cast<const float*>(smem);
+  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kAThreads) {
+    const int gg = idx / kHeadDim, d = idx - gg * kHeadDim;
+    float M = -INFINITY;
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const size_t pi = pbase + (size_t)g * a.nchunk;
-    a.part_o[pi * kHeadDim + d] = o[g];
-    if (tid == 0) {
-      a.part_ml[pi * 2 + 0] = mg[g];
-      a.part_ml[pi * 2 + 1] = rsum[g * 4 + 0] + rsum[g * 4 + 1] + rsum[g * 4 + 2] + rsum[g * 4 + 3];
+    for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, s_m[w][gg]);
+    float os = 0.f, ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w) {
+      const float f = s_m[w][gg] == -INFINITY ? 0.f : expf(s_m[w][gg] - M);
+      os = fmaf(f, ro[(w * 8 + gg) * kHeadDim + d], os);
+      ls = fmaf(f, s_l[w][gg], ls);
+    }
+    const size_t pi = pbase + (size_t)gg * nsplit;
+    a.part_o[pi * kHeadDim + d] = os;
+    if (d == 0) {
+      a.part_ml[pi * 2 + 0] = M;
+      a.part_ml[pi * 2 + 1] = ls;
     }
   }
 }
 
 // One CTA per (head, batch row); thread d owns output dimension d.
-__global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a) {
+__global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a, int nsplit) {
   pdl_launch_dependents();
   pdl_wait();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int P = a.pos[b] + 1;
-  const int nc = (P + kAttnChunk - 1) / kAttnChunk;
-  const size_t base = ((size_t)b * a.H + h) * a.nchunk;
+  const int ntiles = (P + kTile - 1) / kTile;
+  const int tpc = tiles_per_split(P, nsplit);
+  const int nc = (ntiles + tpc - 1) / tpc;  // splits that hold positions
+  const size_t base = ((size_t)b * a.H + h) * nsplit;
   float M = -INFINITY;
   for (int c = 0; c < nc; ++c) M = fmaxf(M, a.part_ml[(base + c) * 2]);
   float l = 0.f, o = 0.f;
   for (int c = 0; c < nc; ++c) {
-    const float w = expf(a.part_ml[(base + c) * 2] - M);
+    const float mc = a.part_ml[(base + c) * 2];
+    const float w = mc == -INFINITY ? 0.f : expf(mc - M);
     l = fmaf(w, a.part_ml[(base + c) * 2 + 1], l);
     o = fmaf(w, a.part_o[(base + c) * kHeadDim + d], o);
   }
@@ -205,27 +360,58 @@ __global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a) {
 }
 
 template <int G>
-int launch_g(const AttnArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)2 * kAttnChunk * kHeadDim * 2 + (size_t)G * kHeadDim * 4 +
-                      (size_t)G * kAttnChunk * 4 + (size_t)2 * G * 4 * 4;
-  if (set_smem_once((const void*)k_attn_chunk<G>, (int)smem)) return TP_ECUDA;
-  return launch_pdl(k_attn_chunk<G>, dim3(a.nchunk, a.Hkv, a.B), dim3(kAttnThreads), smem, s, a);
+int launch_g(const AttnArgs& a, const CUtensorMap& mK, const CUtensorMap& mV, int nsplit,
+             cudaStream_t s) {
+  if (set_smem_once((const void*)k_attn_split<G>, kSmemBytes)) return TP_ECUDA;
+  return launch_pdl(k_attn_split<G>, dim3(nsplit, a.Hkv, a.B), dim3(kAThreads), kSmemBytes, s,
+                    mK, mV, a, nsplit);
 }
 
 }  // namespace
 
+int attention_max_splits(int max_seq) { return (max_seq + kTile - 1) / kTile; }
+
+// Splits per (batch row, kv head): the count that minimises waves x (tiles per
+// CTA + 1), two CTAs resident per SM, over a context of max_seq positions. The
+// kernels divide the actual context (pos + 1) over that many splits.
+int attention_splits(int B, int Hkv, int max_seq) {
+  const int T = attention_max_splits(max_seq);
+  const long slots = 2L * num_sms();
+  int best = 1;
+  long best_cost = -1;
+  for (int sp = 1; sp <= T; ++sp) {
+    const int tpc = (T + sp - 1) / sp;
+    if ((T + tpc - 1) / tpc != sp) continue;  // an equivalent smaller count exists
+    const long ctas = (long)B * Hkv * sp;
+    const long cost = ((ctas + slots - 1) / slots) * (tpc + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  return best;
+}
+
 int launch_attention(const AttnArgs& a, cudaStream_t s) {
   const int G = a.H / a.Hkv;
+  const int nsplit = attention_splits(a.B, a.Hkv, a.max_seq);
+  if (nsplit > a.nchunk) return TP_EINVAL;
+  if (!aligned16(a.kc) || !aligned16(a.vc)) return TP_EALIGN;
+  CUtensorMap mK, mV;
+  const uint64_t rows = (uint64_t)a.B * a.Hkv * a.max_seq;
+  if (!make_tensor_map_2d(&mK, a.kc, rows, kHeadDim, kHeadDim, 64, kTile) ||
+      !make_tensor_map_2d(&mV, a.vc, rows, kHeadDim, kHeadDim, 64, kTile))
+    return TP_ECUDA;
   int rc;
   switch (G) {
-    case 1: rc = launch_g<1>(a, s); break;
-    case 2: rc = launch_g<2>(a, s); break;
-    case 4: rc = launch_g<4>(a, s); break;
-    case 8: rc = launch_g<8>(a, s); break;
+    case 1: rc = launch_g<1>(a, mK, mV, nsplit, s); break;
+    case 2: rc = launch_g<2>(a, mK, mV, nsplit, s); break;
+    case 4: rc = launch_g<4>(a, mK, mV, nsplit, s); break;
+    case 8: rc = launch_g<8>(a, mK, mV, nsplit, s); break;
     default: return TP_ENOTSUP;
   }
   if (rc != TP_OK) return rc;
-  return launch_pdl(k_attn_combine, dim3(a.H, a.B), dim3(kHeadDim), 0, s, a);
+  return launch_pdl(k_attn_combine, dim3(a.H, a.B), dim3(kHeadDim), 0, s, a, nsplit);
 }
 
 }  // namespace tp

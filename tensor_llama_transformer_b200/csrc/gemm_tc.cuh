@@ -2,6 +2,8 @@
 // batched decode slice products.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace tp {
@@ -41,5 +43,10 @@ struct TcGemm {
 };
 
 int launch_tc_gemm(const TcGemm& g, cudaStream_t s);
+
+// 2D TMA map over a bf16 row-major matrix [rows, cols] with row stride `ld`
+// elements: box box_cols x box_rows, 128-byte swizzle, zero fill past the edges.
+bool make_tensor_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint64_t ld, int box_cols, int box_rows);
 
 }  // namespace tp

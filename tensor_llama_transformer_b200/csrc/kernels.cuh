@@ -75,22 +75,23 @@ struct GemvPlan {
 int launch_gemv(const GemvArgs& a, int epi, cudaStream_t s);
 
 // ------------------------------------------------------------------ attention
-constexpr int kAttnChunk = 128;  // context positions per CTA
-
 struct AttnArgs {
   const float* q;       // rotated q [B, H*hd]
   const uint16_t* kc;   // [maxB, Hkv, max_seq, hd] bf16
   const uint16_t* vc;
   const int32_t* pos;   // [B]
-  int B, H, Hkv, max_seq, nchunk;
-  float* part_o;        // [B, H, nchunk, hd] unnormalised partial outputs
-  float* part_ml;       // [B, H, nchunk, 2] running max and sum
+  int B, H, Hkv, max_seq;
+  int nchunk;           // capacity of the partial buffers in context splits
+  float* part_o;        // [B, H, nsplit, hd] unnormalised partial outputs (nsplit <= nchunk)
+  float* part_ml;       // [B, H, nsplit, 2] running max and sum
   float* att;           // [B, H*hd] combined output
   uint16_t* att_bf16;   // optional hi/lo bf16 pairs [2B, H*hd] (rows 2b, 2b+1)
   int* err;             // device error flag (bounded waits)
 };
 
 int launch_attention(const AttnArgs& a, cudaStream_t s);
+// Largest number of context splits any launch over max_seq positions uses.
+int attention_max_splits(int max_seq);
 
 // ------------------------------------------------------------------ batched decode
 // Batches at least this large run the slice products on the tcgen05 GEMM (the
