@@ -142,6 +142,33 @@ TP_API void tp_block_destroy(tp_block* blk);
 #define TP_BLOCK_STAGES 7
 TP_API int tp_block_set_events(tp_block* blk, void* const* events, int n);
 
+/* Persistent block kernel (batch 1-2, 1D partition, GQA group <= 8, n <= 8
+ * slices, shapes whose shared-memory plan fits): the whole block forward as one
+ * cooperative launch of one CTA per SM, the steps separated by grid barriers,
+ * with the weights of the next step streaming into shared memory while the
+ * current one finishes. Same arguments and results as the kernel-per-step path.
+ * enable: 1 use it for this handle's forwards where the shapes allow, 0 never.
+ * The default is 0 unless the environment variable TP_PERSISTENT=1 is set when
+ * the handle is created. Errors: TP_EINVAL. */
+TP_API int tp_block_set_persistent(tp_block* blk, int enable);
+
+/* Phase trace of the persistent block kernel (batch 1-2, 1D partition), which
+ * runs the whole block as one launch and so cannot be split by events. trace:
+ * device buffer owned by the caller, at least (SM count) x TP_BLOCK_TRACE_SLOTS
+ * x 8 bytes, or NULL to switch tracing off. Each forward that runs the persistent
+ * kernel writes, per CTA c, uint64 %globaltimer values (ns) at
+ * trace[c * TP_BLOCK_TRACE_SLOTS + k]: k = 0 kernel start; 2p+1 end of phase p
+ * and 2p+2 end of the grid barrier after it, for the phases p = 0 q/k/v, 1
+ * attention, 2 W_O, 3 W1/W3, 4 W2; 11 end of the final merge; 12 the CTA's last
+ * weight or cache copy issued; 13 end of the grid barrier after the merge of the
+ * W_O partials (which precedes W1/W3), 14 end of the W1/W3 activation staging
+ * (RMSNorm); 15 a duration, not a time: the nanoseconds the CTA's first consumer
+ * thread spent waiting for weight stages during W1/W3. While events are set (tp_block_set_events) the
+ * block runs as separate kernels and the trace is not written.
+ * Errors: TP_EINVAL (NULL handle, buffer too small). */
+#define TP_BLOCK_TRACE_SLOTS 16
+TP_API int tp_block_set_trace(tp_block* blk, void* trace, size_t bytes);
+
 /* One block decode step that allocates nothing (no counterpart in the paper: this
  * entry point exists for callers, not for the method).
  *
@@ -218,6 +245,9 @@ TP_API int tp_model_create(const tp_dims* dims, int n_layers, int n_slices, int 
  * [n_layers, max_batch, Hkv, max_seq, hd]; logits float32 [batch, vocab] written. */
 TP_API int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
                      const int32_t* pos, int batch, float* logits, tp_stream stream);
+
+/* tp_block_set_persistent for every layer of the model. Errors: TP_EINVAL. */
+TP_API int tp_model_set_persistent(tp_model* m, int enable);
 
 TP_API void tp_model_destroy(tp_model* m);
 

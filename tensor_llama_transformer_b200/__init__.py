@@ -63,6 +63,9 @@ _sig = {
     "tp_block_buffer": (C.c_int, [_P, C.c_int, _SZ, _SZ]),
     "tp_block_destroy": (None, [_P]),
     "tp_block_set_events": (C.c_int, [_P, _P, C.c_int]),
+    "tp_block_set_trace": (C.c_int, [_P, _P, C.c_size_t]),
+    "tp_block_set_persistent": (C.c_int, [_P, C.c_int]),
+    "tp_model_set_persistent": (C.c_int, [_P, C.c_int]),
     "tp_ffn_workspace_bytes": (C.c_int, [C.POINTER(tp_ffn_desc), _SZ]),
     "tp_ffn_forward": (C.c_int, [C.POINTER(tp_ffn_desc), _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "tp_model_workspace_bytes": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int, C.c_int,
@@ -163,6 +166,25 @@ TP_BLOCK_STAGES = 8
 def tp_block_set_events(handle, events, n):
     """events: a ctypes array of n cudaEvent_t handles (kept alive by the caller) or None."""
     _check(_lib.tp_block_set_events(handle, events, n), "tp_block_set_events")
+
+
+def tp_block_set_persistent(handle, enable):
+    """1: run this handle's batch 1-2 forwards as the one persistent kernel; 0: never."""
+    _check(_lib.tp_block_set_persistent(handle, int(enable)), "tp_block_set_persistent")
+
+
+def tp_model_set_persistent(handle, enable):
+    """tp_block_set_persistent for every layer of a model handle."""
+    _check(_lib.tp_model_set_persistent(handle, int(enable)), "tp_model_set_persistent")
+
+
+def tp_block_set_trace(handle, buf, nbytes):
+    """buf: device buffer (tensor or pointer) of nbytes for the persistent kernel's
+    per-CTA phase timestamps (TP_BLOCK_TRACE_SLOTS uint64 per CTA), or None."""
+    _check(_lib.tp_block_set_trace(handle, _ptr(buf), nbytes), "tp_block_set_trace")
+
+
+TP_BLOCK_TRACE_SLOTS = 16
 
 
 def tp_ffn_workspace_bytes(desc: tp_ffn_desc) -> int:

@@ -80,8 +80,10 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // ------------------------------------------------------------------ block layout
 enum Buf {
   BUF_XQ = 0, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H, BUF_ERR, BUF_PO, BUF_PML,
-  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_COUNT
+  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_XMID, BUF_CNT, BUF_COUNT
 };
+// BUF_ERR (16 bytes): int error word at byte 0; the persistent kernel's two grid
+// barrier counters at bytes 8 and 12.
 
 struct Layout {
   size_t off[BUF_COUNT];
@@ -147,7 +149,10 @@ Layout block_layout(const Cfg& c) {
   const size_t pa = c.partition == TP_PART_2D ? (size_t)c.gx * B * F * 4 : 0;
   L.size[BUF_PA] = pa;
   L.size[BUF_PB] = pa;
-  L.size[BUF_SSQ] = B * (size_t)merge_ssq_parts(c.d.dim) * 4;
+  // per-row sums of squares: merge pieces of 512 values, or (persistent kernel) 128
+  L.size[BUF_SSQ] = B * (size_t)(c.d.dim / 128) * 4;
+  L.size[BUF_XMID] = B * D * 4;  // x + attention branch (persistent kernel)
+  L.size[BUF_CNT] = B * (size_t)c.d.n_kv_heads * 4;  // finished attention splits (persistent kernel)
   // batched decode (tensor-core path): bf16 operands and the float32 product planes
   if (c.d.max_batch >= kTcMinBatch) {
     const size_t KD = (size_t)c.d.n_kv_heads * c.d.head_dim;
@@ -187,6 +192,9 @@ struct tp_block {
   uint8_t* ws;
   size_t ws_bytes;
   void* const* events;  // optional per-stage timing events (borrowed)
+  bool bar_ready;       // grid barrier counters known to be zero
+  unsigned long long* trace;  // optional phase trace of the persistent kernel
+  int persistent;       // use the persistent kernel where the shapes allow (batch 1-2, 1D)
 };
 
 struct tp_model {
@@ -389,9 +397,71 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
 // chained: x was produced by the previous block's final merge of this same
 // launch sequence, which left the row sums of squares in the workspace (inside
 // a model); the final merge here leaves them for the next block.
+// Batch 1-2, 1D partition: the whole block as one persistent kernel (*used set
+// when it ran; otherwise the caller runs the kernel-per-step path).
+int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos,
+                             int batch, cudaStream_t s, bool* used) {
+  *used = false;
+  const Cfg& c = blk->c;
+  const tp_dims& d = c.d;
+  const int D = d.dim, F = d.ffn_dim, QD = d.n_heads * d.head_dim, KD = d.n_kv_heads * d.head_dim;
+  BpArgs a{};
+  a.D = D;
+  a.F = F;
+  a.H = d.n_heads;
+  a.Hkv = d.n_kv_heads;
+  a.QD = QD;
+  a.n = c.n;
+  a.quant = c.quant;
+  a.max_seq = d.max_seq;
+  a.nb = batch;
+  a.nchunk = c.nchunk;
+  a.eps = d.norm_eps;
+  a.theta = d.rope_theta;
+  a.attn_norm = static_cast<const float*>(blk->w.attn_norm);
+  a.ffn_norm = static_cast<const float*>(blk->w.ffn_norm);
+  const auto wp = [](const void* p) { return static_cast<const uint16_t*>(p); };
+  a.g[0] = BpGemv{{wp(blk->w.wq), wp(blk->w.wk), wp(blk->w.wv)}, {QD, KD, KD}, D, D, 1, QD + 2 * KD, 0, 0};
+  a.g[1] = BpGemv{{wp(blk->w.wo), nullptr, nullptr}, {D, 0, 0}, QD, QD / c.n, c.n, D, 0, 0};
+  a.g[2] = BpGemv{{wp(blk->w.w1), wp(blk->w.w3), nullptr}, {F, 0, 0}, D, D, 1, 2 * F, 0, 0};
+  a.g[3] = BpGemv{{wp(blk->w.w2), nullptr, nullptr}, {D, 0, 0}, F, F / c.n, c.n, D, 0, 0};
+  if (!plan_block_persistent(a, batch)) return TP_OK;
+  a.x = x;
+  a.kc = static_cast<uint16_t*>(kc);
+  a.vc = static_cast<uint16_t*>(vc);
+  a.pos = pos;
+  a.xq = at<int8_t>(blk, BUF_XQ);
+  a.xd = at<float>(blk, BUF_XD);
+  a.xn = at<float>(blk, BUF_XN);
+  a.q = at<float>(blk, BUF_Q);
+  a.part_o = at<float>(blk, BUF_PO);
+  a.part_ml = at<float>(blk, BUF_PML);
+  a.att = at<float>(blk, BUF_ATT);
+  a.part = at<float>(blk, BUF_PART);
+  a.xmid = at<float>(blk, BUF_XMID);
+  a.ssq = at<float>(blk, BUF_SSQ);
+  a.h = at<float>(blk, BUF_H);
+  a.err = at<int>(blk, BUF_ERR);
+  a.bar = reinterpret_cast<unsigned*>(blk->ws + blk->L.off[BUF_ERR] + 8);
+  a.cnt = at<unsigned>(blk, BUF_CNT);
+  a.trace = blk->trace;
+  if (!blk->bar_ready) {  // counters start at zero; each launch leaves them so
+    if (cudaMemsetAsync(a.bar, 0, 8, s) != cudaSuccess) return TP_ECUDA;
+    if (cudaMemsetAsync(a.cnt, 0, blk->L.size[BUF_CNT], s) != cudaSuccess) return TP_ECUDA;
+    blk->bar_ready = true;
+  }
+  *used = true;
+  return launch_block_persistent(a, batch, s);
+}
+
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
                        cudaStream_t s, bool chained = false) {
   if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained);
+  if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent) {
+    bool used = false;
+    const int rc = block_forward_persistent(blk, x, kc, vc, pos, batch, s, &used);
+    if (used || rc) return rc;
+  }
   const Cfg& c = blk->c;
   const tp_dims& d = c.d;
   const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
@@ -622,6 +692,9 @@ int tp_block_create(const tp_dims* dims, int n_slices, int partition, int sync_q
   b->ws = static_cast<uint8_t*>(workspace);
   b->ws_bytes = ws_bytes;
   b->events = nullptr;
+  b->bar_ready = false;
+  b->trace = nullptr;
+  b->persistent = persistent_default() ? 1 : 0;
   *out = b;
   return TP_OK;
 }
@@ -642,6 +715,19 @@ int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* byte
 }
 
 void tp_block_destroy(tp_block* blk) { delete blk; }
+
+int tp_block_set_persistent(tp_block* blk, int enable) {
+  if (!blk || (enable != 0 && enable != 1)) return TP_EINVAL;
+  blk->persistent = enable;
+  return TP_OK;
+}
+
+int tp_block_set_trace(tp_block* blk, void* trace, size_t bytes) {
+  if (!blk) return TP_EINVAL;
+  if (trace && bytes < (size_t)num_sms() * TP_BLOCK_TRACE_SLOTS * 8) return TP_EINVAL;
+  blk->trace = static_cast<unsigned long long*>(trace);
+  return TP_OK;
+}
 
 int tp_block_set_events(tp_block* blk, void* const* events, int n) {
   if (!blk) return TP_EINVAL;
@@ -681,6 +767,11 @@ int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition,
   blk.events = nullptr;
   if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_ERR], 0, blk.L.size[BUF_ERR], stream) != cudaSuccess)
     return TP_ECUDA;
+  if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_CNT], 0, blk.L.size[BUF_CNT], stream) != cudaSuccess)
+    return TP_ECUDA;
+  blk.bar_ready = true;  // the memsets above cover the persistent kernel's counters
+  blk.trace = nullptr;
+  blk.persistent = persistent_default() ? 1 : 0;
   return block_forward_impl(&blk, x, k_cache, v_cache, pos, batch, stream);
 }
 }  // namespace tp
@@ -781,6 +872,12 @@ int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_
   a.ldo = d.vocab;
   a.err = at<int>(&m->blocks[0], BUF_ERR);
   return launch_gemv(a, EPI_PLAIN, s);
+}
+
+int tp_model_set_persistent(tp_model* m, int enable) {
+  if (!m || (enable != 0 && enable != 1)) return TP_EINVAL;
+  for (int l = 0; l < m->n_layers; ++l) m->blocks[l].persistent = enable;
+  return TP_OK;
 }
 
 void tp_model_destroy(tp_model* m) {

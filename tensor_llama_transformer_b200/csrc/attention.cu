@@ -23,6 +23,7 @@
 // 16 FLOP per KV byte, far below the tensor pipe's rate: the kernel is HBM-bound.
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "pipeline.cuh"
 
 namespace tp {
 
@@ -36,92 +37,7 @@ constexpr int kBox = kTile * 64 * 2;     // one box: 64 positions x 64 dims of b
 constexpr int kStageBytes = 4 * kBox;    // K (two dim halves) + V (two dim halves)
 constexpr int kQStride = 136;            // staged Q row stride (bf16), padded against conflicts
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 16 * kQStride * 2;
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 static_assert(kCWarps * 8 * kHeadDim * 4 <= kStageBytes, "merge staging must fit in stage 0");
-
-TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-TP_DEV uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-TP_DEV void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
-}
-
-TP_DEV void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
-               : "memory");
-}
-
-TP_DEV void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
-}
-
-TP_DEV bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(s2u(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait: gives up after kTimeoutNs and raises the error word.
-TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
-  if (mbar_try(b, parity)) return true;
-  const uint64_t t0 = gtimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try(b, parity)) return true;
-    if ((i & 255) == 0 && gtimer() - t0 > kTimeoutNs) {
-      if (err) atomicExch(err, 1);
-      return false;
-    }
-  }
-}
-
-TP_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(s2u(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(s2u(bar))
-      : "memory");
-}
-
-TP_DEV void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-TP_DEV void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-// D (16x8 float32) += A (16x16 bf16, row-major) * B (16x8 bf16, column-major)
-TP_DEV void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3},"
-      " {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-TP_DEV uint32_t pack_bf16x2(uint16_t first, uint16_t second) {
-  return (uint32_t)first | ((uint32_t)second << 16);
-}
-
-// Shared address of 16-byte chunk c (8 dims, 0..15) of row t (0..63) of a K or
-// V tile that TMA wrote as two 64-dim boxes with the 128-byte swizzle.
-TP_DEV uint32_t tile_addr(uint32_t base, int t, int c) {
-  return base + (uint32_t)((c >> 3) * kBox + t * 128 + (((c & 7) ^ (t & 7)) << 4));
-}
 
 // Tiles of one split for a context of P positions: the same for both kernels.
 TP_DEV int tiles_per_split(int P, int nsplit) {
@@ -163,7 +79,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCWarps);
     }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_init_fence();
   }
   // Q of the group's heads scaled by 1/sqrt(hd): hi in row g, lo in row g + 8
   const float scale = 1.0f / sqrtf((float)kHeadDim);
@@ -220,7 +136,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
           for (int idx = lane; idx < 16 * 16; idx += 32) {
             const int r = idx >> 4, c = idx & 15;
             if (t0 + w0 + r >= P)
-              *reinterpret_cast<uint4*>(smem + (tile_addr(vb, w0 + r, c) - s2u(smem))) =
+              *reinterpret_cast<uint4*>(smem + (kv_tile_addr(vb, w0 + r, c) - s2u(smem))) =
                   make_uint4(0u, 0u, 0u, 0u);
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -233,7 +149,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             uint32_t bf[4];
-            ldsm_x4(tile_addr(kb, t, 2 * ks + ch), bf);
+            ldsm_x4(kv_tile_addr(kb, t, 2 * ks + ch), bf);
             mma_bf16(sc[0], qa[ks], bf[0], bf[1]);
             mma_bf16(sc[1], qa[ks], bf[2], bf[3]);
           }
@@ -280,7 +196,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
 #pragma unroll
           for (int np = 0; np < 8; ++np) {
             uint32_t bf[4];
-            ldsm_x4_t(tile_addr(vb, t, 2 * np + ch), bf);
+            ldsm_x4_t(kv_tile_addr(vb, t, 2 * np + ch), bf);
             mma_bf16(o[2 * np], pa, bf[0], bf[1]);
             mma_bf16(o[2 * np + 1], pa, bf[2], bf[3]);
           }
@@ -297,7 +213,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
       s_l[warp][g] = l_run;
     }
     // every tile has been consumed by all consumer warps: stage 0 takes the O partials
-    asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32) : "memory");
+    consumers_sync(kCWarps * 32);
     float* ro = reinterpret_cast<float*>(smem);  // [kCWarps][8][kHeadDim]
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {

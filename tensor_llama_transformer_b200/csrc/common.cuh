@@ -83,9 +83,24 @@ TP_DEV float block_max(float v, float* red) {
 // the codes are reproducible bit for bit on any IEEE machine.
 TP_DEV float q8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
 
+// The code is round(fl(x / d)) with fl the correctly rounded quotient. The
+// quotient is first taken with the fast division __fdividef (at most 2 ulp from
+// x / d for d in the normal range, so at most 2.5 ulp from fl(x / d)); since
+// |x| <= amax gives |x / d| < 128, that is below 2e-5 in absolute terms, and
+// rounding to an integer can only differ from rounding fl(x / d) when the
+// quotient lies that close to a tie k + 1/2. Only then (and for d outside
+// [2^-120, 2^120]) is the correctly rounded division taken.
 TP_DEV int q8_code(float x, float d) {
   if (d == 0.0f) return 0;
-  float v = roundf(__fdiv_rn(x, d));  // roundf: halfway cases away from zero
+  float q;
+  if (d > 0x1p-120f && d < 0x1p120f) {
+    q = __fdividef(x, d);
+    const float a = fabsf(q);
+    if (fabsf(a - truncf(a) - 0.5f) < 4e-5f) q = __fdiv_rn(x, d);
+  } else {
+    q = __fdiv_rn(x, d);
+  }
+  float v = roundf(q);  // roundf: halfway cases away from zero
   v = fminf(fmaxf(v, -127.0f), 127.0f);
   return (int)v;
 }

@@ -36,84 +36,14 @@
 // pairs, stores rotated q, and writes k and v into the bf16 cache at pos
 // (llamaMultiheadAtt's "merge kv-cache, add RoPE encoding").
 #include "kernels.cuh"
+#include "pipeline.cuh"
 
 namespace tp {
 
 namespace {
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kMaxStages = 16;
 constexpr int kSmemBudget = 222 * 1024;
-
-TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-TP_DEV uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-TP_DEV void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
-}
-TP_DEV void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
-               : "memory");
-}
-TP_DEV void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
-}
-TP_DEV bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(s2u(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
-  if (mbar_try(b, parity)) return true;
-  const uint64_t t0 = gtimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try(b, parity)) return true;
-    if ((i & 255) == 0 && gtimer() - t0 > kTimeoutNs) {
-      if (err) atomicExch(err, 1);
-      return false;
-    }
-  }
-}
-TP_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          s2u(dst)),
-      "l"(src), "r"(bytes), "r"(s2u(bar))
-      : "memory");
-}
-// Named barrier 1 among the consumer warps only (the producer never joins it).
-TP_DEV void consumers_sync(int nthreads) { asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); }
-
-// acc (two float32 lanes as one 64-bit register pair) += the 8 bf16 weights of
-// w times the 8 activations (lo = elements 0..3, hi = 4..7), two weights per
-// packed fma.rn.f32x2: lane 0 of acc collects the even elements, lane 1 the odd.
-TP_DEV void fma8(uint64_t& acc, const uint4 w, const float4 lo, const float4 hi) {
-  const uint64_t x01 = ((uint64_t)__float_as_uint(lo.y) << 32) | __float_as_uint(lo.x);
-  const uint64_t x23 = ((uint64_t)__float_as_uint(lo.w) << 32) | __float_as_uint(lo.z);
-  const uint64_t x45 = ((uint64_t)__float_as_uint(hi.y) << 32) | __float_as_uint(hi.x);
-  const uint64_t x67 = ((uint64_t)__float_as_uint(hi.w) << 32) | __float_as_uint(hi.z);
-  asm("{\n .reg .b64 w;\n"
-      " mov.b64 w, {%5, %6};  fma.rn.f32x2 %0, w, %1, %0;\n"
-      " mov.b64 w, {%7, %8};  fma.rn.f32x2 %0, w, %2, %0;\n"
-      " mov.b64 w, {%9, %10}; fma.rn.f32x2 %0, w, %3, %0;\n"
-      " mov.b64 w, {%11, %12}; fma.rn.f32x2 %0, w, %4, %0;\n}"
-      : "+l"(acc)
-      : "l"(x01), "l"(x23), "l"(x45), "l"(x67), "r"(w.x << 16), "r"(w.x & 0xFFFF0000u),
-        "r"(w.y << 16), "r"(w.y & 0xFFFF0000u), "r"(w.z << 16), "r"(w.z & 0xFFFF0000u),
-        "r"(w.w << 16), "r"(w.w & 0xFFFF0000u));
-}
-
-TP_DEV float hsum2(uint64_t acc) {
-  return __uint_as_float((uint32_t)acc) + __uint_as_float((uint32_t)(acc >> 32));
-}
 
 template <int EPI>
 TP_DEV int rows_per_seg(const GemvArgs& a) {

@@ -127,6 +127,60 @@ int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s);
 int launch_swiglu_finalize(const float* plane, int F, int batch, float* h, uint16_t* hb,
                            cudaStream_t s);
 
+// ------------------------------------------------------------------ persistent block
+// One weight-streaming phase of the persistent block kernel: the rows of up to
+// three matrices (q/k/v stacked; W1/W3 interleaved row for row), contracted over
+// nseg segments of Ks columns. pairs/split are filled by the plan.
+struct BpGemv {
+  const uint16_t* w[3];
+  int rows[3];
+  int64_t ldw;
+  int Ks, nseg, rps;  // rps: virtual rows per segment
+  int pairs, split;   // row pairs per ring stage; warps per pair
+};
+
+struct BpArgs {
+  int D, F, H, Hkv, QD, n, quant, max_seq, nb, nchunk;
+  float eps, theta;
+  const float* attn_norm;
+  const float* ffn_norm;
+  BpGemv g[4];          // q/k/v, W_O, W1/W3, W2
+  float* x;             // residual [nb, D], overwritten with the block output
+  uint16_t* kc;         // caches [maxB, Hkv, max_seq, hd]
+  uint16_t* vc;
+  const int32_t* pos;
+  int8_t* xq;           // published sync buffers (Q8 codes, scales, float32 values)
+  float* xd;
+  float* xn;
+  float* q;             // rotated q [nb, QD]
+  float* part_o;        // attention splits [nb, H, nchunk, hd] and [nb, H, nchunk, 2]
+  float* part_ml;
+  float* att;           // attention output [nb, QD]
+  float* part;          // row-split partials [n, nb, D] (W_O, then W2)
+  float* xmid;          // x + attention branch [nb, D]
+  float* ssq;           // sums of squares of x_mid per 128 values [nb][D/128]
+  float* h;             // SwiGLU output [nb, F]
+  int* err;             // error word
+  unsigned* bar;        // grid barrier counters (two words, zero between launches)
+  unsigned* cnt;        // finished context splits per (batch row, kv head), zero between launches
+  unsigned long long* trace;  // optional [grid][kBpTraceSlots] %globaltimer stamps (ns)
+  int grid;
+  uint32_t ring_bytes, xs_off, res_off, smem_total;
+};
+// Trace stamps per CTA: 0 start, then for each phase A..F its end (2k+1) and,
+// for A..E, the end of the grid barrier after it (2k+2); 12 the producer's last
+// issue; 13 the end of the barrier after the W_O-partial merge, 14 the end of
+// the activation staging of phase D; 15 the time (ns) thread 0 waited for ring
+// stages during phase D.
+constexpr int kBpTraceSlots = 16;
+static_assert(kBpTraceSlots == TP_BLOCK_TRACE_SLOTS, "trace layout");
+// Fills the launch plan (grid, shared-memory layout, rows per stage); false when
+// the shapes rule the persistent kernel out.
+bool plan_block_persistent(BpArgs& a, int nb_max);
+// Whether handles use the persistent kernel unless told otherwise (TP_PERSISTENT=1).
+bool persistent_default();
+int launch_block_persistent(const BpArgs& a, int nb_max, cudaStream_t s);
+
 // One block forward over a caller-provided workspace with a handle on the stack
 // (api.cu); zeroes the kernels' error word in the workspace first.
 int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition, int sync_quant,

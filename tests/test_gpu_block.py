@@ -40,8 +40,9 @@ def _dims(tpb, s, max_batch):
                          max_batch, s.max_seq, s.norm_eps, s.rope_theta)
 
 
-def run_block(tpb, inp, n, quant, partition=1, max_batch=None):
-    """Runs one block forward on the GPU; returns (x_out, k_rows, v_rows, buffers, err)."""
+def run_block(tpb, inp, n, quant, partition=1, max_batch=None, persistent=None):
+    """Runs one block forward on the GPU; returns (x_out, k_rows, v_rows, buffers, err).
+    persistent: None keeps the handle's default, 0/1 sets tp_block_set_persistent."""
     s = inp.shape
     B = inp.x.shape[0]
     mb = max_batch or B
@@ -51,6 +52,8 @@ def run_block(tpb, inp, n, quant, partition=1, max_batch=None):
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     h = tpb.tp_block_create(dims, n, partition, quant, tpb.make_weights(*dev.weights()), ws, nbytes)
     try:
+        if persistent is not None:
+            tpb.tp_block_set_persistent(h, persistent)
         tpb.tp_block_forward(h, dev.x, dev.k_cache, dev.v_cache, dev.pos, B)
         torch.cuda.synchronize()
         bufs = {}
@@ -70,12 +73,13 @@ def run_block(tpb, inp, n, quant, partition=1, max_batch=None):
     return dev.x.cpu().numpy().astype(np.float64), k_rows, v_rows, bufs, err
 
 
-def check_block(tpb, inp, n, quant, partition=1, tol_out=BF16_TOL, tight=None, name="block"):
+def check_block(tpb, inp, n, quant, partition=1, tol_out=BF16_TOL, tight=None, name="block",
+                persistent=None):
     s = inp.shape
     B = inp.x.shape[0]
     tr = {}
     ref, k_ref, v_ref = oracle.block_forward(inp, n, bool(quant), partition, trace=tr)
-    y, k_rows, v_rows, bufs, err = run_block(tpb, inp, n, quant, partition)
+    y, k_rows, v_rows, bufs, err = run_block(tpb, inp, n, quant, partition, persistent=persistent)
     assert err == 0, "a bounded wait in a kernel gave up"
     QD = s.n_heads * s.head_dim
     r_att, _ = report(f"{name} att", bufs["att"][:B * QD].reshape(B, QD), tr["att"])

@@ -24,7 +24,7 @@ def tpb(cuda_ok):
 
 
 def run_model(tpb, s: synth.BlockShape, seed: int, pos, quant: int, n_layers: int,
-              sample_rows=None):
+              sample_rows=None, persistent=None):
     """Builds the model layer by layer on the GPU while the oracle runs the same layers.
 
     With ``sample_rows`` the GPU runs every batch row but the oracle only the
@@ -84,6 +84,8 @@ def run_model(tpb, s: synth.BlockShape, seed: int, pos, quant: int, n_layers: in
                             nbytes)
     logits = torch.empty((B, s.vocab), dtype=torch.float32, device="cuda")
     try:
+        if persistent is not None:
+            tpb.tp_model_set_persistent(h, persistent)
         tpb.tp_model_forward(h, i32_tensor(toks), kc, vc, i32_tensor(np.array(pos)), B, logits)
         torch.cuda.synchronize()
     finally:

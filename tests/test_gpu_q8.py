@@ -56,11 +56,26 @@ def _edge_cases():
     return np.concatenate(blocks)
 
 
-@pytest.mark.parametrize("kind", ["edge", "random", "ragged_large"])
+def _near_ties(rng, nblocks=20_000):
+    """Blocks whose quotients x/d sit within a few ulp of k + 1/2 (and exactly on
+    it), where the rounded code depends on the last bit of the quotient."""
+    amax = rng.uniform(1e-3, 1e3, nblocks).astype(np.float32)
+    d = (amax / np.float32(127)).astype(np.float32)
+    k = rng.integers(-127, 127, (nblocks, 31)).astype(np.float32)
+    off = rng.choice(np.array([-2e-4, -5e-5, -4.2e-5, -3e-5, -1e-5, -1e-6, 0.0, 1e-6, 1e-5,
+                              3e-5, 4.2e-5, 5e-5, 2e-4], np.float32), (nblocks, 31))
+    vals = ((k + np.float32(0.5) + off) * d[:, None]).astype(np.float32)
+    vals = np.clip(vals, -amax[:, None], amax[:, None])
+    return np.concatenate([amax[:, None], vals], axis=1).astype(np.float32).ravel()
+
+
+@pytest.mark.parametrize("kind", ["edge", "random", "ragged_large", "near_ties"])
 def test_q8_bit_exact(tpb, kind):
     rng = np.random.default_rng(3)
     if kind == "edge":
         x = _edge_cases()
+    elif kind == "near_ties":
+        x = _near_ties(rng)
     elif kind == "random":
         x = (rng.standard_normal(4096 * 37) * rng.uniform(1e-6, 1e4, 4096 * 37)).astype(np.float32)
     else:  # not a multiple of the grid stride or of a warp's 1024 values
