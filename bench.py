@@ -53,6 +53,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the C4 block and C3 model measurements")
+    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p"], default=None,
+                    help="only run a few eager steps of one extra workload (for profiler launch "
+                         "lists: c4 block, c3 model at batch 1, c2 block on the persistent kernel)")
+    ap.add_argument("--profile-steps", type=int, default=3)
     return ap.parse_args(argv)
 
 
@@ -162,6 +166,12 @@ def barrier(world: int):
         import torch.distributed as dist
 
         dist.barrier()
+
+
+# DRAM bytes (read + write) of one launch of the W1/W3 slice GEMV in the C2 block,
+# from `ncu --set full` of that launch (180.434688 MB read + 3.469056 MB written):
+# the weights once, plus the activations and the SwiGLU output.
+W13_DRAM_BYTES = 180434688 + 3469056
 
 
 def block_bytes(s):
@@ -344,7 +354,10 @@ def bench_block(args, world, rank, local):
         "block_gbs": (wbytes + kvbytes) / step_s / 1e9, "stage_us": {
             n: v * 1e3 for n, v in zip(STAGES, stage_ms_max)},
         "roofline": {"bound": "hbm", "achieved": w13_bytes / w13_s / 1e9, "peak": hbm,
-                     "unit": "GB/s", "frac": w13_bytes / w13_s / 1e9 / hbm, "traffic": None,
+                     "unit": "GB/s", "frac": w13_bytes / w13_s / 1e9 / hbm,
+                     "traffic": W13_DRAM_BYTES,
+                     "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of one "
+                                       "launch, ncu capture of this kernel in this workload",
                      "kernel": "k_gemv<1,EPI_SWIGLU,2> (RMSNorm+Q8, W1/W3, SwiGLU)",
                      "algorithmic_bytes": w13_bytes, "peak_kind": peak_kind},
         "e2e": {"value": world * B * E / e2e_s, "unit": "tokens/s",
@@ -411,6 +424,12 @@ def bench_c4(args):
     nb = tpb.tp_block_workspace_bytes(dims, s.n_slices, 1, 0)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     h = tpb.tp_block_create(dims, s.n_slices, 1, 0, tpb.make_weights(*w), ws, nb)
+    if args.profile == "c4":
+        for _ in range(args.profile_steps):
+            tpb.tp_block_forward(h, x, kc, vc, pos, B)
+        torch.cuda.synchronize()
+        tpb.tp_block_destroy(h)
+        return {"profile": "c4", "steps": args.profile_steps}
     ms = _time_graph(torch, lambda: tpb.tp_block_forward(h, x, kc, vc, pos, B), 10, 5)
     tpb.tp_block_destroy(h)
     wb, kvb = block_bytes(s)
@@ -420,6 +439,65 @@ def bench_c4(args):
             "frac": gbs / hbm, "bytes_per_step": wb + kvb,
             "workload": "C4: 70B-shape GQA block, dim 8192, 64/8 heads, SwiGLU 28672, batch 32, "
                         "context 4096, n=8, float32 sync buffers"}
+
+
+def bench_c2_persistent(args):
+    """The C2 block (Llama-2-7B shapes, n = 4, Q8 sync, KV 1024, batch 1) as one persistent
+    kernel per step (tp_block_set_persistent), for comparison with the headline's
+    kernel-per-step graph."""
+    import torch
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+
+    s = synth.C2
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1001)
+    B, D, F, H, Hkv, hd = s.batch, s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim
+    w = [torch.ones(D, device="cuda"), _randn_bf16(torch, gen, (H * hd, D), s.w_std),
+         _randn_bf16(torch, gen, (Hkv * hd, D), s.w_std), _randn_bf16(torch, gen, (Hkv * hd, D), s.w_std),
+         _randn_bf16(torch, gen, (D, H * hd), s.w_std), torch.ones(D, device="cuda"),
+         _randn_bf16(torch, gen, (F, D), s.w_std), _randn_bf16(torch, gen, (F, D), s.w_std),
+         _randn_bf16(torch, gen, (D, F), s.w_std)]
+    kc = _randn_bf16(torch, gen, (B, Hkv, s.max_seq, hd), 1.0)
+    vc = _randn_bf16(torch, gen, (B, Hkv, s.max_seq, hd), 1.0)
+    x = torch.randn((B, D), generator=gen, device="cuda")
+    pos = torch.full((B,), s.pos, dtype=torch.int32, device="cuda")
+    dims = tpb.make_dims(D, H, Hkv, hd, F, s.vocab, B, s.max_seq, s.norm_eps, s.rope_theta)
+    nb = tpb.tp_block_workspace_bytes(dims, s.n_slices, 1, 1)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    h = tpb.tp_block_create(dims, s.n_slices, 1, 1, tpb.make_weights(*w), ws, nb)
+    tpb.tp_block_set_persistent(h, 1)
+    if args.profile == "c2p":
+        for _ in range(args.profile_steps):
+            tpb.tp_block_forward(h, x, kc, vc, pos, B)
+        torch.cuda.synchronize()
+        tpb.tp_block_destroy(h)
+        return {"profile": "c2p", "steps": args.profile_steps}
+    ms = _time_graph(torch, lambda: tpb.tp_block_forward(h, x, kc, vc, pos, B), 100, 20)
+    err = int(ws[tpb.tp_block_buffer(h, 7)[0]:][:4].view(torch.int32).item())
+    # one traced step: per-phase durations (median over CTAs, from kernel start)
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    tr = torch.zeros(nsm * tpb.TP_BLOCK_TRACE_SLOTS, dtype=torch.int64, device="cuda")
+    tpb.tp_block_set_trace(h, tr, tr.numel() * 8)
+    tpb.tp_block_forward(h, x, kc, vc, pos, B)
+    torch.cuda.synchronize()
+    tpb.tp_block_set_trace(h, None, 0)
+    tpb.tp_block_destroy(h)
+    t = tr.view(nsm, -1).cpu().numpy().astype("float64")
+    t = t[t[:, 0] > 0]
+    base = t[:, 0].min()
+    marks = {"qkv_end": 1, "barrier1": 2, "attention_end": 3, "barrier2": 4, "wo_end": 5,
+             "barrier3": 6, "merge_barrier": 13, "w13_staged": 14, "w13_end": 7, "barrier5": 8,
+             "w2_end": 9, "barrier6": 10, "final_merge_end": 11}
+    phase_us = {k: round(float(statistics.median((t[:, i] - base) / 1e3)), 2) for k, i in marks.items()}
+    phase_us["kernel_end_max"] = round(float(((t[:, 11] - base) / 1e3).max()), 2)
+    wb, kvb = block_bytes(s)
+    hbm, _, _, kind = peaks()
+    gbs = (wb + kvb) / (ms / 1e3) / 1e9
+    return {"us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "hbm_gbs": gbs,
+            "frac": gbs / hbm, "pipeline_error": err, "phase_end_us_median": phase_us,
+            "workload": "C2 block as one persistent kernel per step (same shapes as the headline)"}
 
 
 def bench_c3(args, B):
@@ -451,6 +529,12 @@ def bench_c3(args, B):
     nb = tpb.tp_model_workspace_bytes(dims, L, s.n_slices, 1, 0)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     m = tpb.tp_model_create(dims, L, s.n_slices, 1, 0, layers, emb, ones, wcls, ws, nb)
+    if args.profile == "c3b1":
+        for _ in range(args.profile_steps):
+            tpb.tp_model_forward(m, toks, kc, vc, pos, B, logits)
+        torch.cuda.synchronize()
+        tpb.tp_model_destroy(m)
+        return {"profile": "c3b1", "steps": args.profile_steps}
     ms = _time_graph(torch, lambda: tpb.tp_model_forward(m, toks, kc, vc, pos, B, logits), 3, 5)
     tpb.tp_model_destroy(m)
     wb = L * block_bytes(s)[0] + V * D * 2  # every layer's weights + the classifier
@@ -528,6 +612,10 @@ def main(argv=None):
     if not torch.cuda.is_available():
         print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
         return 1
+    if args.profile:
+        fn = {"c4": bench_c4, "c3b1": lambda a: bench_c3(a, 1), "c2p": bench_c2_persistent}
+        print(json.dumps(fn[args.profile](args)))
+        return 0
     world, rank, local = dist_setup()
     res = bench_block(args, world, rank, local)
     ffn = None if args.no_ffn else bench_ffn(args)
@@ -535,7 +623,12 @@ def main(argv=None):
     if not args.no_extra:
         import torch
 
-        extra = {"c4_block": bench_c4(args)}
+        try:
+            extra = {"c2_block_persistent": bench_c2_persistent(args)}
+        except Exception as e:  # reported, not fatal: the headline does not depend on it
+            extra = {"c2_block_persistent": {"error": str(e)[:200]}}
+        torch.cuda.empty_cache()
+        extra["c4_block"] = bench_c4(args)
         torch.cuda.empty_cache()
         extra["c3_model_b1"] = bench_c3(args, 1)
         torch.cuda.empty_cache()

@@ -3,8 +3,8 @@
 This module only *generates numbers*: it holds none of the decoder-block
 arithmetic. Every tensor is a pure function of (config seed, tensor name,
 element index), so any sub-range of a tensor (one batch row of a KV cache,
-one layer of a 32-layer model) can be regenerated on its own, on the host
-here or on the device by ``synth/fill.cu``, bit for bit the same.
+one layer of a 32-layer model) can be regenerated on its own, bit for bit the
+same; the tensors are made here, on the host, and copied to the device.
 
 Generator (counter based):
   * SplitMix64 (Steele, Lea & Flood, "Fast splittable pseudorandom number

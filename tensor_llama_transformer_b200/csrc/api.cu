@@ -80,7 +80,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // ------------------------------------------------------------------ block layout
 enum Buf {
   BUF_XQ = 0, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H, BUF_ERR, BUF_PO, BUF_PML,
-  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_XMID, BUF_CNT, BUF_COUNT
+  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_XMID, BUF_COUNT
 };
 // BUF_ERR (16 bytes): int error word at byte 0; the persistent kernel's two grid
 // barrier counters at bytes 8 and 12.
@@ -152,7 +152,6 @@ Layout block_layout(const Cfg& c) {
   // per-row sums of squares: merge pieces of 512 values, or (persistent kernel) 128
   L.size[BUF_SSQ] = B * (size_t)(c.d.dim / 128) * 4;
   L.size[BUF_XMID] = B * D * 4;  // x + attention branch (persistent kernel)
-  L.size[BUF_CNT] = B * (size_t)c.d.n_kv_heads * 4;  // finished attention splits (persistent kernel)
   // batched decode (tensor-core path): bf16 operands and the float32 product planes
   if (c.d.max_batch >= kTcMinBatch) {
     const size_t KD = (size_t)c.d.n_kv_heads * c.d.head_dim;
@@ -443,11 +442,9 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
   a.h = at<float>(blk, BUF_H);
   a.err = at<int>(blk, BUF_ERR);
   a.bar = reinterpret_cast<unsigned*>(blk->ws + blk->L.off[BUF_ERR] + 8);
-  a.cnt = at<unsigned>(blk, BUF_CNT);
   a.trace = blk->trace;
   if (!blk->bar_ready) {  // counters start at zero; each launch leaves them so
     if (cudaMemsetAsync(a.bar, 0, 8, s) != cudaSuccess) return TP_ECUDA;
-    if (cudaMemsetAsync(a.cnt, 0, blk->L.size[BUF_CNT], s) != cudaSuccess) return TP_ECUDA;
     blk->bar_ready = true;
   }
   *used = true;
@@ -766,8 +763,6 @@ int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition,
   blk.ws_bytes = ws_bytes;
   blk.events = nullptr;
   if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_ERR], 0, blk.L.size[BUF_ERR], stream) != cudaSuccess)
-    return TP_ECUDA;
-  if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_CNT], 0, blk.L.size[BUF_CNT], stream) != cudaSuccess)
     return TP_ECUDA;
   blk.bar_ready = true;  // the memsets above cover the persistent kernel's counters
   blk.trace = nullptr;

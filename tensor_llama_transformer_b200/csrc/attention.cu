@@ -96,16 +96,17 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   if (warp == kCWarps) {
     // ------------------------------------------------------------ producer warp
     if (lane == 0) {
+      const uint64_t pol = l2_evict_first();  // cache tiles are read once per step
       for (int i = i0; i < i1; ++i) {
         const int k = i - i0, s = k % kStages;
         if (!mbar_wait(&empty[s], ((uint32_t)(k / kStages) & 1u) ^ 1u, a.err)) break;
         mbar_expect_tx(&full[s], kStageBytes);
         uint8_t* st = smem + s * kStageBytes;
         const int y = row_base + i * kTile;
-        tma_load_2d(st, &mK, 0, y, &full[s]);
-        tma_load_2d(st + kBox, &mK, 64, y, &full[s]);
-        tma_load_2d(st + 2 * kBox, &mV, 0, y, &full[s]);
-        tma_load_2d(st + 3 * kBox, &mV, 64, y, &full[s]);
+        tma_load_2d_hint(st, &mK, 0, y, &full[s], pol);
+        tma_load_2d_hint(st + kBox, &mK, 64, y, &full[s], pol);
+        tma_load_2d_hint(st + 2 * kBox, &mV, 0, y, &full[s], pol);
+        tma_load_2d_hint(st + 3 * kBox, &mV, 64, y, &full[s], pol);
       }
     }
   } else {

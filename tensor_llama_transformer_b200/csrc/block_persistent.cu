@@ -12,19 +12,24 @@
 //   -- barrier 2
 //   C  W_O rows        (activation: the context splits of each head combined)
 //   -- barrier 3
-//   D  W1/W3 rows      (activation: RMSNorm(x + sum_s sync(W_O partial_s))*g)
+//   M  x_mid = x + sum_s sync(W_O partial_s), each 128-value chunk by one warp
 //   -- barrier 4
-//   E  W2 rows         (activation: the SwiGLU output h)
+//   D  W1/W3 rows      (activation: RMSNorm(x_mid)*g, +Q8)
 //   -- barrier 5
+//   E  W2 rows         (activation: the SwiGLU output h)
+//   -- barrier 6
 //   F  x = x_mid + sum_s sync(W2 partial_s)
 // Within a CTA, one producer warp streams everything the CTA will read from HBM
-// (its share of every weight matrix, then its attention tiles) through one
-// shared-memory ring of variable-size stages, and never waits for a grid
-// barrier: weights are read-only, and cache rows below pos are not written in
-// this step. Only the attention tiles that hold position pos (written in phase
-// A by another CTA) wait for barrier 1. So while the consumer warps sit at a
-// barrier, the next phase's first ~190 KB per SM is already arriving, and HBM
-// stays busy across the step instead of draining at every kernel boundary.
+// (the RMSNorm inputs, its share of every weight matrix, its attention tiles)
+// through one shared-memory ring of variable-size stages, and never waits for a
+// grid barrier: weights are read-only, x changes only in phase F, and cache rows
+// below pos are not written in this step. Only the attention tiles that hold
+// position pos (written in phase A by another CTA) wait for barrier 1. So while
+// the consumer warps sit at a barrier, the next phase's first ~200 KB per SM is
+// already arriving, and HBM stays busy across the step instead of draining at
+// every kernel boundary. Weights and cache tiles are read with an L2 evict-first
+// policy, which keeps the small activations and partials that the phases pass
+// to one another resident in L2.
 //
 // The eight consumer warps do the arithmetic of each phase:
 //   GEMV phases: as the ring-buffer slice GEMV (rows in pairs, each pair split
@@ -32,10 +37,11 @@
 //   in shared memory, per-row partial sums combined in a fixed order);
 //   attention: as the split flash-decoding kernel (mma.m16n8k16 with hi/lo bf16
 //   Q and P rows, online softmax in registers), four warps per tile, the two
-//   halves of the consumers taking alternate tiles of a head.
-// Activations that several CTAs need (normalised x, the merged residual, the
-// combined attention output) are recomputed by every CTA from the previous
-// phase's outputs in L2, identically, instead of by a separate kernel.
+//   halves of the consumers taking alternate tiles of a head; each CTA writes
+//   one partial (o, m, l) per head group it touched.
+// Activations that several CTAs need (normalised x_mid, the attention output
+// combined from its splits) are recomputed by every CTA that needs them, from
+// the previous phase's outputs in L2, instead of by a separate kernel.
 //
 // Every wait is bounded (2 s): mbarrier waits and grid-barrier spins raise the
 // error word and the kernel walks on without the data, so it always exits.
@@ -56,6 +62,7 @@ constexpr uint32_t kTileBytes = 4 * 8192;   // K and V, two 64-dim boxes each
 constexpr int kQStride = 136;               // staged Q rows (bf16), padded
 constexpr uint32_t kQsBytes = 16 * kQStride * 2;
 constexpr int kMaxSlices = 8;               // slices whose partials a merge holds at once
+constexpr int kMaxSegHeads = 64;            // query heads per W_O segment
 
 enum { PH_QKV = 0, PH_WO = 1, PH_W13 = 2, PH_W2 = 3 };
 
@@ -266,12 +273,14 @@ TP_DEV int attn_cta_of(const AttnWork& w, int u) {
   return (int)(((unsigned)(u + 1) * gridDim.x - 1u) / (unsigned)w.total);
 }
 
-// A head group's context splits are stored at slot = the group's first tile in
-// the CTA that computed the split. Given the split at slot s of the group whose
-// first list index is uf, the next split starts where that CTA's range ends.
-TP_DEV int attn_next_slot(const AttnWork& w, int uf, int s) {
-  const unsigned c = (unsigned)attn_cta_of(w, uf + s);
-  return (int)(((unsigned)w.total * (c + 1u)) / gridDim.x) - uf;
+// Context split of CTA c for the head group whose first list index is uf: the
+// split is stored at slot = the group's first tile in that CTA's range; -1 when
+// the CTA has no tiles at all (fewer tiles than CTAs).
+TP_DEV int split_slot(const AttnWork& w, int uf, int c) {
+  const int start = (int)(((unsigned)w.total * (unsigned)c) / gridDim.x);
+  const int end = (int)(((unsigned)w.total * (unsigned)(c + 1)) / gridDim.x);
+  if (end <= start) return -1;
+  return (start > uf ? start : uf) - uf;
 }
 
 TP_DEV bool produce_attn(Producer& pr, const BpArgs& a, const CUtensorMap* mK,
@@ -333,6 +342,56 @@ struct Consumer {
   }
 };
 
+// One ring stage of a GEMV phase for one consumer warp: PW row pairs (pairs pw
+// and pw + 8 when PW = 2), or 1/Q of one pair (vectors [vb, ve)) when Q > 1.
+template <int NB, int PW>
+TP_DEV void gemv_stage(const Consumer& c, uint32_t off, int cur, int end, const float4* xs,
+                       float* res, int nv, uint32_t rb, int pw, int part, int Q, int vb, int ve,
+                       int lane) {
+  constexpr int R = 2 * PW * NB;  // values: (pair j, row, batch row)
+  int rr[PW];
+  bool valid[PW];
+  const uint4* wr[PW];
+#pragma unroll
+  for (int j = 0; j < PW; ++j) {
+    rr[j] = cur + 2 * (pw + 8 * j);
+    valid[j] = c.ok && rr[j] < end;
+    wr[j] = reinterpret_cast<const uint4*>(c.ring + off + (size_t)(rr[j] - cur) * rb);
+  }
+  if (!valid[0]) return;  // pairs are filled in order: no pair for this warp
+  uint64_t acc[R][2];
+#pragma unroll
+  for (int i = 0; i < R; ++i) acc[i][0] = acc[i][1] = 0ull;
+#pragma unroll 4
+  for (int v = vb + lane; v < ve; v += 32) {
+    float4 lo[NB], hi[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      lo[b] = xs[b * nv + v];
+      hi[b] = xs[(NB + b) * nv + v];
+    }
+#pragma unroll
+    for (int j = 0; j < PW; ++j) {
+      if (!valid[j]) continue;
+      const uint4 u0 = wr[j][v], u1 = wr[j][nv + v];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        fma8_2(acc[(2 * j) * NB + b][0], acc[(2 * j) * NB + b][1], u0, lo[b], hi[b]);
+        fma8_2(acc[(2 * j + 1) * NB + b][0], acc[(2 * j + 1) * NB + b][1], u1, lo[b], hi[b]);
+      }
+    }
+  }
+  float val[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) val[i] = hsum2(acc[i][0]) + hsum2(acc[i][1]);
+  const float tot = warp_sum_multi<R>(val, lane);
+  constexpr int kLanes = 32 / R;  // lanes holding each total
+  if ((lane & (kLanes - 1)) == 0) {
+    const int i = lane / kLanes, j = i / (2 * NB), row = (i / NB) & 1, b = i % NB;
+    if (valid[j]) res[((size_t)(rr[j] + row) * NB + b) * Q + part] = tot;
+  }
+}
+
 // One GEMV phase for the consumer warps. stage(seg, publish) fills xs with the
 // segment's activations (lo halves [NB][nv], then hi halves); res receives the
 // per-row partial sums [row][NB][split].
@@ -360,33 +419,8 @@ TP_DEV void consume_gemv(Consumer& c, const BpGemv& g, float4* xs, float* res, i
     }
     const int end = min(min(nrows, seg_end), cur + 2 * g.pairs);
     const uint32_t off = c.next(round1k((uint32_t)(end - cur) * rb));
-    const int r = cur + 2 * pw;
-    if (c.ok && r < end) {
-      const uint4* w0 = reinterpret_cast<const uint4*>(c.ring + off + (size_t)(2 * pw) * rb);
-      const uint4* w1 = w0 + nv;
-      uint64_t acc0[NB], acc1[NB], acc2[NB], acc3[NB];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) acc0[b] = acc1[b] = acc2[b] = acc3[b] = 0ull;
-#pragma unroll 4
-      for (int v = vb + lane; v < ve; v += 32) {
-        const uint4 u0 = w0[v], u1 = w1[v];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float4 lo = xs[b * nv + v], hi = xs[(NB + b) * nv + v];
-          fma8_2(acc0[b], acc2[b], u0, lo, hi);
-          fma8_2(acc1[b], acc3[b], u1, lo, hi);
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float y0 = warp_sum(hsum2(acc0[b]) + hsum2(acc2[b]));
-        const float y1 = warp_sum(hsum2(acc1[b]) + hsum2(acc3[b]));
-        if (lane == 0) {
-          res[((size_t)r * NB + b) * Q + part] = y0;
-          res[((size_t)(r + 1) * NB + b) * Q + part] = y1;
-        }
-      }
-    }
+    if (g.pw == 2) gemv_stage<NB, 2>(c, off, cur, end, xs, res, nv, rb, pw, part, Q, vb, ve, lane);
+    else gemv_stage<NB, 1>(c, off, cur, end, xs, res, nv, rb, pw, part, Q, vb, ve, lane);
     c.release();
     cur = end;
   }
@@ -438,6 +472,7 @@ TP_DEV void stage_norm(const BpArgs& a, float4* xs, const float* xsrc, bool src_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int b = 0; b < NB; ++b) {
     float ss = 0.f;
+#pragma unroll 4
     for (int v = threadIdx.x; v < nv; v += kNCons) {
       const size_t e0 = (size_t)b * D + 8 * (size_t)v;
       float xm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -455,13 +490,19 @@ TP_DEV void stage_norm(const BpArgs& a, float4* xs, const float* xsrc, bool src_
       if (lane == 0) s_red[warp][b] = ss;
     }
   }
+  if (ssq && warp < NB) {  // warp b sums row b's per-chunk sums of squares
+    const int chunks = D >> 7;
+    float t = 0.f;
+    if (warp < a.nb)
+      for (int k = lane; k < chunks; k += 32) t += __ldcg(ssq + (size_t)warp * chunks + k);
+    t = warp_sum(t);
+    if (lane == 0) s_red[0][warp] = t;
+  }
   consumers_sync(kNCons);
   if (threadIdx.x < NB) {
     float tsum = 0.f;
     if (ssq) {
-      const int chunks = D >> 7;
-      if ((int)threadIdx.x < a.nb)
-        for (int k = 0; k < chunks; ++k) tsum += __ldcg(ssq + (size_t)threadIdx.x * chunks + k);
+      tsum = s_red[0][threadIdx.x];
     } else {
       for (int w = 0; w < kNC; ++w) tsum += s_red[w][threadIdx.x];
     }
@@ -518,7 +559,9 @@ TP_DEV void stage_norm(const BpArgs& a, float4* xs, const float* xsrc, bool src_
 TP_DEV void merge_rows(const BpArgs& a, const float* base, float* out, float* ssq_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int D = a.D, chunks = D >> 7;
-  for (int item = blockIdx.x * kNC + warp; item < a.nb * chunks; item += gridDim.x * kNC) {
+  // item i goes to CTA i % grid, warp i / grid: one warp per SM while there are
+  // fewer items than SMs
+  for (int item = warp * gridDim.x + blockIdx.x; item < a.nb * chunks; item += gridDim.x * kNC) {
     const int b = item / chunks, i4 = (item - b * chunks) * 32 + lane;
     float4 p[kMaxSlices];
 #pragma unroll
@@ -548,6 +591,70 @@ TP_DEV void merge_rows(const BpArgs& a, const float* base, float* out, float* ss
   }
 }
 
+// Activations of phase C for W_O segment seg: the attention output of the
+// segment's heads, each combined from its context splits (the CTAs whose tile
+// ranges cover the head group):
+//   M = max_j m_j,  o = sum_j e^{m_j - M} o_j / sum_j e^{m_j - M} l_j.
+// Each thread combines 8 output values in two rounds of loads: the splits'
+// maxima, then their sums and partial outputs (splits in CTA order). The owner
+// of the segment's first row publishes att.
+template <int NB>
+TP_DEV void stage_att(const BpArgs& a, const AttnWork& w, int seg, int Ks, bool publish,
+                      float4* xs) {
+  const int hs = Ks / kHeadDim, G = a.H / a.Hkv, nv = Ks >> 3;
+  for (int idx = threadIdx.x; idx < NB * nv; idx += kNCons) {
+    const int b = idx / nv, v = idx - b * nv;
+    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (b < a.nb) {
+      const int hl = v >> 4, d0 = (v & 15) * 8;  // 16 vectors of 8 per head
+      const int h = seg * hs + hl, uf = w.off[b] + (h / G) * w.nt[b];
+      const int clo = attn_cta_of(w, uf), chi = attn_cta_of(w, uf + w.nt[b] - 1);
+      const float* ml = a.part_ml + ((size_t)b * a.H + h) * a.nchunk * 2;
+      const float* po = a.part_o + ((size_t)b * a.H + h) * a.nchunk * kHeadDim + d0;
+      float M = -INFINITY;
+      for (int c0 = clo; c0 <= chi; c0 += 8) {  // eight splits' loads in flight
+        float mq[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int slot = c0 + q <= chi ? split_slot(w, uf, c0 + q) : -1;
+          mq[q] = slot >= 0 ? __ldcg(ml + 2 * slot) : -INFINITY;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) M = fmaxf(M, mq[q]);
+      }
+      float L = 0.f;
+      for (int c0 = clo; c0 <= chi; c0 += 4) {  // four splits' loads in flight
+        float mj[4], lj[4], pj[4][8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int slot = c0 + q <= chi ? split_slot(w, uf, c0 + q) : -1;
+          mj[q] = -INFINITY;
+          lj[q] = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pj[q][e] = 0.f;
+          if (slot >= 0) {
+            mj[q] = __ldcg(ml + 2 * slot);
+            lj[q] = __ldcg(ml + 2 * slot + 1);
+            load8cg(po + (size_t)slot * kHeadDim, pj[q]);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float wj = mj[q] == -INFINITY ? 0.f : expf(mj[q] - M);
+          L = fmaf(wj, lj[q], L);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = fmaf(wj, pj[q][e], o[e]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = o[e] / L;
+      if (publish) store8(a.att + (size_t)b * a.QD + (size_t)seg * Ks + 8 * v, o);
+    }
+    xs[b * nv + v] = make_float4(o[0], o[1], o[2], o[3]);
+    xs[(NB + b) * nv + v] = make_float4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 // Activations of phases C and E for segment seg: a float32 row segment that
 // other CTAs wrote earlier in this launch (the attention output, the SwiGLU
 // output h), read through L2.
@@ -563,75 +670,13 @@ TP_DEV void stage_plain(const float* src, int ld, int nb, int seg, int Ks, float
   }
 }
 
-// Splits of the head group (b, kvh): their slots, in order (at most one per CTA).
-TP_DEV int attn_slots(const AttnWork& w, int uf, int nt, int* slots) {
-  int np = 0;
-  for (int j = 0; j < nt; j = attn_next_slot(w, uf, j)) slots[np++] = j;
-  return np;
-}
-
-// Combination of the context splits of head group (b, kvh) into the attention
-// output, run by the CTA that finished the group's last split:
-//   M = max_j m_j,  o = sum_j e^{m_j - M} o_j / sum_j e^{m_j - M} l_j.
-// `area` holds the np split slots (ints), then scratch of 2 G kMaxSplits floats.
-constexpr int kMaxSplits = 160;  // one split per CTA at most, CTAs <= SMs
-TP_DEV void attn_combine(const BpArgs& a, int b, int kvh, int np, float* area) {
-  const int G = a.H / a.Hkv;
-  const int* s_slot = reinterpret_cast<const int*>(area);
-  float* s_m = area + kMaxSplits;       // [G][kMaxSplits], then the weights
-  float* s_l = s_m + G * kMaxSplits;    // [G][kMaxSplits]
-  __shared__ float s_L[8];
-  const size_t hbase = (size_t)b * a.H + (size_t)kvh * G;  // first head of the group
-  for (int idx = threadIdx.x; idx < G * np; idx += kNCons) {
-    const int g = idx / np, j = idx - g * np;
-    const size_t pi = (hbase + g) * a.nchunk + s_slot[j];
-    s_m[g * kMaxSplits + j] = __ldcg(a.part_ml + pi * 2);
-    s_l[g * kMaxSplits + j] = __ldcg(a.part_ml + pi * 2 + 1);
-  }
-  consumers_sync(kNCons);
-  if (threadIdx.x < G) {
-    const int g = threadIdx.x;
-    float M = -INFINITY;
-    for (int j = 0; j < np; ++j) M = fmaxf(M, s_m[g * kMaxSplits + j]);
-    float L = 0.f;
-    for (int j = 0; j < np; ++j) {
-      const float mj = s_m[g * kMaxSplits + j];
-      const float wj = mj == -INFINITY ? 0.f : expf(mj - M);
-      s_m[g * kMaxSplits + j] = wj;
-      L = fmaf(wj, s_l[g * kMaxSplits + j], L);
-    }
-    s_L[g] = L;
-  }
-  consumers_sync(kNCons);
-  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kNCons) {
-    const int g = idx / kHeadDim, d = idx - g * kHeadDim;
-    const float* po = a.part_o + (hbase + g) * a.nchunk * kHeadDim + d;
-    const float* wg = s_m + g * kMaxSplits;
-    float o = 0.f;
-    int j = 0;
-    for (; j + 4 <= np; j += 4) {  // four independent loads in flight
-      const float p0 = __ldcg(po + (size_t)s_slot[j] * kHeadDim);
-      const float p1 = __ldcg(po + (size_t)s_slot[j + 1] * kHeadDim);
-      const float p2 = __ldcg(po + (size_t)s_slot[j + 2] * kHeadDim);
-      const float p3 = __ldcg(po + (size_t)s_slot[j + 3] * kHeadDim);
-      o = fmaf(wg[j], p0, o);
-      o = fmaf(wg[j + 1], p1, o);
-      o = fmaf(wg[j + 2], p2, o);
-      o = fmaf(wg[j + 3], p3, o);
-    }
-    for (; j < np; ++j) o = fmaf(wg[j], __ldcg(po + (size_t)s_slot[j] * kHeadDim), o);
-    a.att[(size_t)b * a.QD + (size_t)(kvh * G + g) * kHeadDim + d] = o / s_L[g];
-  }
-  consumers_sync(kNCons);
-}
-
 // Attention of the CTA's tiles (phase B). Warps 0-3 take the even tiles of a
 // head, warps 4-7 the odd ones; each warp covers 16 positions of a tile. At the
 // end of each head the 8 warps' partials are merged and written as the CTA's
 // split of that head.
 template <int NB>
 TP_DEV void consume_attn(Consumer& c, const BpArgs& a, const AttnWork& w, uint8_t* xsb,
-                         float (*s_m)[8], float (*s_l)[8], int* s_last) {
+                         float (*s_m)[8], float (*s_l)[8]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.H / a.Hkv;
   float* ro = reinterpret_cast<float*>(xsb);  // the warps' partials [8][G][128]
@@ -777,22 +822,6 @@ TP_DEV void consume_attn(Consumer& c, const BpArgs& a, const AttnWork& w, uint8_
         a.part_ml[pi * 2 + 1] = ls;
       }
     }
-    // count the split (the barrier, then one gpu-scope fence, release every
-    // thread's partial); the CTA that completes the group combines its splits
-    consumers_sync(kNCons);
-    if (threadIdx.x == 0) {
-      int* slots = reinterpret_cast<int*>(ro);  // the merge area is free again
-      const int np = attn_slots(w, uf, w.nt[b], slots);
-      __threadfence();
-      const unsigned prev = atomicAdd(a.cnt + b * a.Hkv + kvh, 1u);
-      *s_last = prev + 1 == (unsigned)np ? np : 0;
-      if (*s_last) {
-        __threadfence();
-        atomicExch(a.cnt + b * a.Hkv + kvh, 0u);  // ready for the next launch
-      }
-    }
-    consumers_sync(kNCons);
-    if (*s_last) attn_combine(a, b, kvh, *s_last, ro);
     u = useg;
   }
 }
@@ -810,7 +839,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t full[kMaxQ], empty[kMaxQ], st_start[kMaxQ];
   __shared__ float s_red[kNC][2], s_rstd[2];
   __shared__ float s_m[kNC][8], s_l[kNC][8];
-  __shared__ int s_last;
 
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
@@ -889,7 +917,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- B: attention
   AttnWork w;
   attn_work(a, w);
-  consume_attn<NB>(c, a, w, xsb, s_m, s_l, &s_last);
+  consume_attn<NB>(c, a, w, xsb, s_m, s_l);
   if (tr) stamp(a, 3);
   grid_barrier(a.bar, 2, a.err);
   if (tr) stamp(a, 4);
@@ -897,8 +925,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- C: W_O partials
   {
     const BpGemv& g = a.g[PH_WO];
-    consume_gemv<NB, EPI_PLAIN>(c, g, xs, res, R0, nrows, [&](int seg, bool) {
-      stage_plain<NB>(a.att, a.QD, a.nb, seg, g.Ks, xs);
+    consume_gemv<NB, EPI_PLAIN>(c, g, xs, res, R0, nrows, [&](int seg, bool publish) {
+      stage_att<NB>(a, w, seg, g.Ks, publish, xs);
     });
     for (int tt = threadIdx.x; tt < (nrows >> 1) * NB; tt += kNCons) {
       const int pr = tt / NB, b = tt - pr * NB;
@@ -974,21 +1002,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (atomicAdd(a.bar + 1, 1u) == gridDim.x - 1) {
       atomicExch(a.bar, 0u);
       atomicExch(a.bar + 1, 0u);
-      for (int i = 0; i < a.nb * a.Hkv; ++i) atomicExch(a.cnt + i, 0u);
     }
   }
 }
 
 
-// Rows per stage for a phase: the most row pairs (8, 4, 2, 1) whose stage
+// Rows per stage for a phase: the most row pairs (16, 8, 4, 2, 1) whose stage
 // stays within a third of the ring, so that at least three stages are in
-// flight; each pair is then split over 8 / pairs warps.
+// flight; 16 pairs give each warp two pairs, fewer are split over 8 / pairs
+// warps each.
 bool plan_phase(BpGemv& g, uint32_t max_stage) {
   const uint32_t rb = (uint32_t)g.Ks * 2;
-  for (int P = 8; P >= 1; P >>= 1) {
+  for (int P = 16; P >= 1; P >>= 1) {
     if ((uint32_t)(2 * P) * rb <= max_stage) {
       g.pairs = P;
-      g.split = 8 / P;
+      g.split = P >= 8 ? 1 : 8 / P;
+      g.pw = P == 16 ? 2 : 1;
       return true;
     }
   }
@@ -1013,7 +1042,7 @@ bool persistent_default() {
 
 bool plan_block_persistent(BpArgs& a, int nb_max) {
   if (nb_max < 1 || nb_max > 2 || a.n < 1) return false;
-  if (a.n > kMaxSlices || a.H / a.Hkv > 8) return false;
+  if (a.n > kMaxSlices || a.H / a.Hkv > 8 || a.QD / a.n / kHeadDim > kMaxSegHeads) return false;
   // every CTA gets at least one row pair of every phase (so that the owner of
   // each segment's first row, which publishes its activations, exists)
   int grid = num_sms();
@@ -1029,7 +1058,6 @@ bool plan_block_persistent(BpArgs& a, int nb_max) {
   // reuses the partials' area
   const uint32_t G = (uint32_t)(a.H / a.Hkv);
   const uint32_t merge_bytes = kNC * G * kHeadDim * 4u;
-  if ((1u + 2u * G) * kMaxSplits * 4u > merge_bytes || grid > kMaxSplits) return false;
   uint32_t xs_region = xs_bytes > merge_bytes + kQsBytes ? xs_bytes : merge_bytes + kQsBytes;
   xs_region = (xs_region + 1023u) & ~1023u;
   uint32_t res_bytes = 0;  // per-row partial sums, bounded by the widest split (8)

@@ -13,7 +13,8 @@
 // of row pairs (a RoPE pair of q/k, row f of W1 with row f of W3, or two
 // consecutive rows); every CTA owns a contiguous, equal share of the pairs, so
 // every SM streams the same bytes. A producer warp copies the CTA's rows into a
-// ring of shared-memory stages with bulk asynchronous copies (cp.async.bulk),
+// ring of shared-memory stages with bulk asynchronous copies (cp.async.bulk, L2
+// evict-first: the weights are read once per step, the activations often),
 // completion counted on one mbarrier per stage; a stage holds one row pair for
 // each of the NC consumer warps and never crosses a segment boundary, and the
 // ring keeps 100-200 KB per SM in flight. A consumer warp dots its pair with the
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   if (warp == nc) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
+      const uint64_t pol = l2_evict_first();  // weights are read once per step
       int t = 0;
       for (int cur = 0; cur < nrows; ++t) {
         const int end = stage_end(cur, nrows, R0, rps, P);
@@ -134,8 +136,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
           const uint16_t* p1 = a.w[0] + (size_t)(lr0 >> 1) * a.ldw + col0;
           const uint16_t* p3 = a.w[1] + (size_t)(lr0 >> 1) * a.ldw + col0;
           for (int i = 0; i < n; i += 2) {
-            bulk_g2s(dst + (size_t)i * row_bytes, p1, row_bytes, &full[s]);
-            bulk_g2s(dst + (size_t)(i + 1) * row_bytes, p3, row_bytes, &full[s]);
+            bulk_g2s_hint(dst + (size_t)i * row_bytes, p1, row_bytes, &full[s], pol);
+            bulk_g2s_hint(dst + (size_t)(i + 1) * row_bytes, p3, row_bytes, &full[s], pol);
             p1 += a.ldw;
             p3 += a.ldw;
           }
@@ -148,10 +150,10 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
             if (EPI == EPI_QKV) mat_end = mat == 0 ? a.rows[0] : (mat == 1 ? a.rows[0] + a.rows[1] : rps);
             const int run = min(n - done, mat_end - r);
             if (a.ldw == a.Ks) {
-              bulk_g2s(dst + (size_t)done * row_bytes, src, (uint32_t)run * row_bytes, &full[s]);
+              bulk_g2s_hint(dst + (size_t)done * row_bytes, src, (uint32_t)run * row_bytes, &full[s], pol);
             } else {
               for (int i = 0; i < run; ++i, src += a.ldw)
-                bulk_g2s(dst + (size_t)(done + i) * row_bytes, src, row_bytes, &full[s]);
+                bulk_g2s_hint(dst + (size_t)(done + i) * row_bytes, src, row_bytes, &full[s], pol);
             }
             done += run;
             r += run;
@@ -290,27 +292,28 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       if (ok && r < end) {
         const uint4* w0 = reinterpret_cast<const uint4*>(ring + ((size_t)s * 2 * P + 2 * pw) * row_bytes);
         const uint4* w1 = w0 + nv;
-        uint64_t acc0[NB], acc1[NB];
+        constexpr int R = 2 * NB;  // values: (row of the pair, batch row)
+        uint64_t acc[R][2];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) acc0[b] = acc1[b] = 0ull;
+        for (int i = 0; i < R; ++i) acc[i][0] = acc[i][1] = 0ull;
 #pragma unroll 4
         for (int v = vb + lane; v < ve; v += 32) {
           const uint4 u0 = w0[v], u1 = w1[v];
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
             const float4 lo = xs[b * nv + v], hi = xs[(NB + b) * nv + v];
-            fma8(acc0[b], u0, lo, hi);
-            fma8(acc1[b], u1, lo, hi);
+            fma8_2(acc[b][0], acc[b][1], u0, lo, hi);
+            fma8_2(acc[NB + b][0], acc[NB + b][1], u1, lo, hi);
           }
         }
+        float val[R];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float y0 = warp_sum(hsum2(acc0[b]));
-          const float y1 = warp_sum(hsum2(acc1[b]));
-          if (lane == 0) {
-            res[((size_t)r * NB + b) * Q + part] = y0;
-            res[((size_t)(r + 1) * NB + b) * Q + part] = y1;
-          }
+        for (int i = 0; i < R; ++i) val[i] = hsum2(acc[i][0]) + hsum2(acc[i][1]);
+        const float tot = warp_sum_multi<R>(val, lane);
+        constexpr int kLanes = 32 / R;  // lanes holding each total
+        if ((lane & (kLanes - 1)) == 0) {
+          const int i = lane / kLanes, row = i / NB, b = i - row * NB;
+          res[((size_t)(r + row) * NB + b) * Q + part] = tot;
         }
       }
       __syncwarp();

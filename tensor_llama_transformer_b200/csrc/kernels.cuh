@@ -137,6 +137,7 @@ struct BpGemv {
   int64_t ldw;
   int Ks, nseg, rps;  // rps: virtual rows per segment
   int pairs, split;   // row pairs per ring stage; warps per pair
+  int pw;             // row pairs per warp and stage (1, or 2 with 16 pairs per stage)
 };
 
 struct BpArgs {
@@ -162,7 +163,6 @@ struct BpArgs {
   float* h;             // SwiGLU output [nb, F]
   int* err;             // error word
   unsigned* bar;        // grid barrier counters (two words, zero between launches)
-  unsigned* cnt;        // finished context splits per (batch row, kv head), zero between launches
   unsigned long long* trace;  // optional [grid][kBpTraceSlots] %globaltimer stamps (ns)
   int grid;
   uint32_t ring_bytes, xs_off, res_off, smem_total;

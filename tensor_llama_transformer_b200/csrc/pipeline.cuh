@@ -176,6 +176,29 @@ TP_DEV float hsum2(uint64_t acc) {
   return __uint_as_float((uint32_t)acc) + __uint_as_float((uint32_t)(acc >> 32));
 }
 
+// Sums each of R values (R = 2, 4, 8) over the warp's 32 lanes with
+// log2(R) exchange steps that halve the values a lane holds, then a butterfly
+// over the remaining lanes: 5 + R/2 - 1 shuffles in all instead of 5 R. Lane l
+// returns the total of value l / (32 / R).
+template <int R>
+TP_DEV float warp_sum_multi(float (&v)[R], int lane) {
+#pragma unroll
+  for (int k = 0; (1 << k) < R; ++k) {
+    const int m = 16 >> k, half = R >> (k + 1);
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = up ? v[i] : v[i + half];
+      const float keep = up ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int m = 32 / R / 2; m >= 1; m >>= 1) t += __shfl_xor_sync(0xffffffffu, t, m);
+  return t;
+}
+
 // Shared address of 16-byte chunk c (8 dims, 0..15) of row t of a 64-row K or
 // V tile that TMA wrote as two boxes of 64 rows x 64 dims (8 KB each, the first
 // for dims 0..63) with the 128-byte swizzle; base must be 1024-byte aligned.
