@@ -85,6 +85,9 @@ enum Buf {
 // BUF_ERR (16 bytes): int error word at byte 0; the persistent kernel's two grid
 // barrier counters at bytes 8 and 12.
 
+// Largest contraction splits of the batched-decode GEMMs (the planes are sized for them).
+constexpr int kQkvMaxParts = 8, kW13MaxParts = 4, kW2MaxParts = 2;
+
 struct Layout {
   size_t off[BUF_COUNT];
   size_t size[BUF_COUNT];
@@ -141,7 +144,8 @@ Layout block_layout(const Cfg& c) {
   L.size[BUF_XN] = B * D * 4;
   L.size[BUF_Q] = B * QD * 4;
   L.size[BUF_ATT] = B * QD * 4;
-  L.size[BUF_PART] = (size_t)c.n * B * D * 4;
+  // row-split partials: n slices (x kW2MaxParts contraction parts on the tensor path)
+  L.size[BUF_PART] = (size_t)c.n * (c.d.max_batch >= kTcMinBatch ? kW2MaxParts : 1) * B * D * 4;
   L.size[BUF_H] = B * F * 4;
   L.size[BUF_ERR] = 16;
   L.size[BUF_PO] = B * c.d.n_heads * (size_t)c.nchunk * c.d.head_dim * 4;
@@ -158,8 +162,8 @@ Layout block_layout(const Cfg& c) {
     L.size[BUF_XB] = 2 * B * D * 2;  // hi/lo bf16 pairs
     L.size[BUF_ATTB] = 2 * B * QD * 2;
     L.size[BUF_HB] = 2 * B * F * 2;
-    const size_t qkv = 2 * B * (QD + 2 * KD) * 4;  // up to 2 contraction parts
-    const size_t w13 = B * 2 * F * 4;
+    const size_t qkv = kQkvMaxParts * B * (QD + 2 * KD) * 4;  // contraction parts
+    const size_t w13 = kW13MaxParts * B * 2 * F * 4;
     L.size[BUF_PLANE] = qkv > w13 ? qkv : w13;
   }
   size_t o = 0;
@@ -244,10 +248,29 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
   return e == cudaSuccess ? TP_OK : TP_ECUDA;
 }
 
-int tc_parts_for(int tiles) {
-  // contraction parts so that the q/k/v launch has work for every SM
-  return tiles * 2 <= num_sms() * 3 ? 2 : 1;
+// Contraction parts for a batched-decode GEMM of `tiles` 128-row output tiles
+// (per existing segment) over K: the persistent GEMM gives each SM ceil(tiles *
+// parts / SMs) tiles of K / parts, and every extra part adds a float32 plane
+// [batch, rows] that is written and read back. Picks the power of two <= pmax
+// (with K / parts a multiple of 64) that minimises the busiest SM's weight bytes
+// plus its share of the planes' traffic.
+int tc_split(int64_t tiles, int64_t K, int64_t rows_total, int batch, int pmax) {
+  const int64_t sms = num_sms();
+  int best = 1;
+  double best_cost = -1.0;
+  for (int p = 1; p <= pmax; p *= 2) {
+    if (K % (64 * p) != 0 && p > 1) break;
+    const double main = (double)((tiles * p + sms - 1) / sms) * 128.0 * (double)(K / p) * 2.0;
+    const double planes = 2.0 * p * (double)batch * (double)rows_total * 4.0 / (double)sms;
+    const double cost = main + planes;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = p;
+    }
+  }
+  return best;
 }
+
 
 // The batched form of the block: the same steps, with the slice products on the
 // tcgen05 GEMM (weights = M operand, batch = N) writing float32 planes, small
@@ -306,8 +329,7 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
   if ((rc = stage_mark(blk, 0, s))) return rc;
   if ((rc = norm(blk->w.attn_norm, chained ? at<float>(blk, BUF_SSQ) : nullptr))) return rc;
   const int qkv_tiles = (QD + 127) / 128 + 2 * ((KD + 127) / 128);
-  int parts = tc_parts_for(qkv_tiles);
-  if ((D / parts) % 8 != 0) parts = 1;
+  const int parts = tc_split(qkv_tiles, D, QD + 2 * KD, batch, kQkvMaxParts);
   if ((rc = gemm(blk->w.wq, QD, blk->w.wk, KD, blk->w.wv, KD, 3, D, xb, D / parts, parts, plane,
                  QD + 2 * KD)))
     return rc;
@@ -361,8 +383,10 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
   float* hbuf = at<float>(blk, BUF_H);
   uint16_t* hb = at<uint16_t>(blk, BUF_HB);
   if (c.partition == TP_PART_1D) {
-    if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D, 1, plane, 2 * F))) return rc;
-    if ((rc = launch_swiglu_finalize(plane, F, batch, hbuf, hb, s))) return rc;
+    const int p13 = tc_split(2 * ((F + 127) / 128), D, 2 * F, batch, kW13MaxParts);
+    if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F)))
+      return rc;
+    if ((rc = launch_swiglu_finalize(plane, p13, F, batch, hbuf, hb, s))) return rc;
   } else {
     float* pa = at<float>(blk, BUF_PA);
     float* pb = at<float>(blk, BUF_PB);
@@ -385,17 +409,18 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
   // a9
   if ((rc = stage_mark(blk, 5, s))) return rc;
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
-  if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2, nseg2, part, D))) return rc;
+  const int p2 = tc_split((int64_t)nseg2 * ((D + 127) / 128), F / nseg2, (int64_t)nseg2 * D, batch,
+                          kW2MaxParts);
+  if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2 / p2, nseg2 * p2, part,
+                 D)))
+    return rc;
   // a10
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
+  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, at<float>(blk, BUF_SSQ), s, p2)))
+    return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
-// One block forward (the distributed-llama root-node order for one layer).
-// chained: x was produced by the previous block's final merge of this same
-// launch sequence, which left the row sums of squares in the workspace (inside
-// a model); the final merge here leaves them for the next block.
 // Batch 1-2, 1D partition: the whole block as one persistent kernel (*used set
 // when it ran; otherwise the caller runs the kernel-per-step path).
 int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos,
@@ -451,6 +476,10 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
   return launch_block_persistent(a, batch, s);
 }
 
+// One block forward (the distributed-llama root-node order for one layer).
+// chained: x was produced by the previous block's final merge of this same
+// launch sequence, which left the row sums of squares in the workspace (inside
+// a model); the final merge here leaves them for the next block.
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
                        cudaStream_t s, bool chained = false) {
   if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained);

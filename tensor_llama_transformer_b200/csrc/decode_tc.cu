@@ -123,15 +123,21 @@ __global__ void k_qkv_finalize(QkvFinalizeArgs a) {
   }
 }
 
-// plane [batch][2F]: columns [0, F) are x W1^T, [F, 2F) are x W3^T.
-__global__ void k_swiglu_finalize(const float* __restrict__ plane, int F, int batch,
+// planes [parts][batch][2F]: columns [0, F) are x W1^T, [F, 2F) are x W3^T, each
+// summed over the contraction parts in order.
+__global__ void k_swiglu_finalize(const float* __restrict__ plane, int parts, int F, int batch,
                                   float* __restrict__ h, uint16_t* __restrict__ hb) {
   pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.y;
   const int f = blockIdx.x * blockDim.x + threadIdx.x;
   if (f >= F) return;
-  const float a = plane[(size_t)b * 2 * F + f], g = plane[(size_t)b * 2 * F + F + f];
+  float a = 0.f, g = 0.f;
+  for (int p = 0; p < parts; ++p) {
+    const float* pl = plane + ((size_t)p * batch + b) * 2 * F;
+    a += pl[f];
+    g += pl[F + f];
+  }
   const float v = a / (1.0f + expf(-a)) * g;
   h[(size_t)b * F + f] = v;
   bf16_split(v, hb[(size_t)(2 * b) * F + f], hb[(size_t)(2 * b + 1) * F + f]);
@@ -149,10 +155,10 @@ int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s) {
   return launch_pdl(k_qkv_finalize, dim3((pairs + 255) / 256, a.batch), dim3(256), 0, s, a);
 }
 
-int launch_swiglu_finalize(const float* plane, int F, int batch, float* h, uint16_t* hb,
-                           cudaStream_t s) {
-  return launch_pdl(k_swiglu_finalize, dim3((F + 255) / 256, batch), dim3(256), 0, s, plane, F,
-                    batch, h, hb);
+int launch_swiglu_finalize(const float* plane, int parts, int F, int batch, float* h,
+                           uint16_t* hb, cudaStream_t s) {
+  return launch_pdl(k_swiglu_finalize, dim3((F + 255) / 256, batch), dim3(256), 0, s, plane, parts,
+                    F, batch, h, hb);
 }
 
 }  // namespace tp

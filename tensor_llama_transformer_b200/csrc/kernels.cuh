@@ -6,11 +6,13 @@
 namespace tp {
 
 // ------------------------------------------------------------------ merge / codec
-// x[b] += sum_{s<n} sync(part[s][b]) in slice order; part is [n, B, dim]. With
-// ssq != nullptr each CTA also writes the sum of squares of its piece of the new
-// row: ssq[b][piece], piece = 512-element block index (merge_ssq_parts(dim) of them).
+// x[b] += sum_{s<n} sync(part_s[b]) in slice order, part_s = the sum of planes
+// s*parts .. s*parts+parts-1 of part [n*parts, B, dim] (a slice's contraction
+// split further by the GEMM). With ssq != nullptr each CTA also writes the sum of
+// squares of its piece of the new row: ssq[b][piece], piece = 512-element block
+// index (merge_ssq_parts(dim) of them).
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s);
+                 cudaStream_t s, int parts = 1);
 inline int merge_ssq_parts(int dim) { return (dim / 4 + 127) / 128; }
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s);
 int launch_dequantize(const int8_t* q, const float* d, float* x, int64_t n, cudaStream_t s);
@@ -124,8 +126,10 @@ struct QkvFinalizeArgs {
   int n_kv_heads, max_seq;
 };
 int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s);
-int launch_swiglu_finalize(const float* plane, int F, int batch, float* h, uint16_t* hb,
-                           cudaStream_t s);
+// h = silu(a) * g from planes [parts][batch][2F] (a = columns [0, F), g = [F, 2F),
+// each the sum of the parts in order), with its hi/lo bf16 pair rows.
+int launch_swiglu_finalize(const float* plane, int parts, int F, int batch, float* h,
+                           uint16_t* hb, cudaStream_t s);
 
 // ------------------------------------------------------------------ persistent block
 // One weight-streaming phase of the persistent block kernel: the rows of up to

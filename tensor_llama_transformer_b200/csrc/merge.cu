@@ -2,8 +2,9 @@
 //
 // distributed-llama issue #29: llamaDequantizeAtt + llamaMergeAtt (and the Ffn2
 // twins) sum the slices' partial outputs into the residual. Here one launch
-// does both for every element: each partial passes through the sync buffer's
-// format (the Q8 round trip when quantisation is on), the partials are summed
+// does both for every element: each partial (the sum of its contraction parts
+// when a GEMM split it further) passes through the sync buffer's format (the Q8
+// round trip when quantisation is on), the partials are summed
 // in slice order 0..n-1 in float32, and the sum is added to x. The grid covers
 // the batch rows in 512-element pieces so that the merge of a single token is
 // spread over many SMs instead of waiting on one.
@@ -17,7 +18,7 @@ constexpr int kMergeThreads = 128;  // 4 values per thread: 512 values per CTA
 
 __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
                                                          const float* __restrict__ part, int n,
-                                                         int B, int dim, int quant,
+                                                         int parts, int B, int dim, int quant,
                                                          float* __restrict__ ssq) {
   __shared__ float red[kMergeThreads / 32];
   pdl_launch_dependents();
@@ -29,8 +30,15 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
   const bool in = i4 < n4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < n; ++s) {
-    float4 p = in ? reinterpret_cast<const float4*>(part + ((size_t)s * B + b) * dim)[i4]
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    // slice s's partial: the sum of its contraction parts (planes s*parts .. s*parts+parts-1)
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < parts && in; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(part + ((size_t)(s * parts + k) * B + b) * dim)[i4];
+      p.x += v.x;
+      p.y += v.y;
+      p.z += v.z;
+      p.w += v.w;
+    }
     if (quant) q8_roundtrip4(p);
     acc.x += p.x;
     acc.y += p.y;
@@ -86,9 +94,9 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 }  // namespace
 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s) {
+                 cudaStream_t s, int parts) {
   const dim3 grid(merge_ssq_parts(dim), B);
-  return launch_pdl(k_merge, grid, dim3(kMergeThreads), 0, s, x, part, n, B, dim, quant, ssq);
+  return launch_pdl(k_merge, grid, dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim, quant, ssq);
 }
 
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s) {
