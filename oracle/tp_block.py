@@ -44,7 +44,7 @@ import numpy as np
 __all__ = [
     "bf16_to_f64", "round_to_bf16", "rmsnorm", "q8_quantize", "q8_dequantize", "sync_buffer",
     "rope", "attention_decode", "silu", "swiglu", "relu", "block_forward", "ffn_forward",
-    "model_forward", "grid_2d", "slice_range", "ffn_unsharded_chunked",
+    "model_forward", "grid_2d", "slice_range", "ffn_unsharded_chunked", "q8_weights", "q8_exact",
 ]
 
 
@@ -303,8 +303,27 @@ def ffn_forward(X, W1, W2, act: str = "relu", W3=None, partition: int = 1, n_sli
 # decoder block
 # ---------------------------------------------------------------------------
 
+def q8_exact(v: np.ndarray) -> np.ndarray:
+    """The Q8 round trip of ``v`` with the dequantised values kept exact in float64
+    (``q * d``, 7 + 24 bits): the value an integer block dot product uses."""
+    q, d = q8_quantize(np.asarray(v, dtype=np.float32))
+    return q.astype(np.float64) * np.repeat(d.astype(np.float64), Q8_BLOCK, axis=-1)
+
+
+def q8_weights(w_bits: np.ndarray):
+    """Int8 weights: each row of a bf16 weight matrix ``[out, in]`` in the Q8 block
+    format along ``in`` (``q8_quantize`` of the row's float32 values).
+
+    [POPE] demo4 ("int8 weights" for PaLM decode, which is bound by weight bytes)
+    gives no format; the reading taken is the one the [DL] task list already uses
+    for its sync buffers: 32 consecutive values share one float32 scale
+    ``d = amax / 127``. Returns ``(codes int8 [out, in], scales float32 [out, in/32])``.
+    """
+    return q8_quantize(bf16_to_f64(w_bits).astype(np.float32))
+
+
 def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid=None,
-                  trace: dict | None = None):
+                  trace: dict | None = None, weights_q8: bool = False):
     """One decode step of one decoder block, partitioned into ``n_slices`` slices.
 
     Follows the [DL] root-node task order for one layer:
@@ -326,6 +345,15 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
     ``att`` (all heads), ``x1``, ``xin2`` and, for 1D, ``h``; recording them does
     not change the arithmetic.
 
+    ``weights_q8`` (1D partition, with ``sync_quant``): int8 weights with Q8
+    activations, the form in which every slice product is an integer dot product
+    per 32-value block scaled by ``d_w * d_x``, i.e. exactly
+    ``sum_i (q_w,i d_w)(q_x,i d_x)``. Every weight matrix enters as its Q8 codes
+    times scales (``q8_weights``, exact in float64) and every slice product's
+    input as ``q8_exact`` of it: the normalised inputs, each slice's attention
+    output before W_O and its SwiGLU output before W2. The partials cross the
+    sync as with ``sync_quant``.
+
     ``inp`` is a ``synth.BlockInputs``. Returns ``(x_out float64 [B, dim],
     k_row uint16 [B, Hkv, hd], v_row uint16 [B, Hkv, hd])``: the new block
     output and the bf16 k/v rows written at ``pos`` (the caches are not modified).
@@ -337,11 +365,25 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
     x = np.asarray(inp.x, dtype=np.float64)
     B = x.shape[0]
     pos = np.asarray(inp.pos)
-    wq, wk, wv = bf16_to_f64(inp.wq), bf16_to_f64(inp.wk), bf16_to_f64(inp.wv)
-    wo = bf16_to_f64(inp.wo)
+    if weights_q8:
+        assert partition == 1 and sync_quant
+
+        def wload(bits):
+            q, d = q8_weights(bits)
+            return q.astype(np.float64) * np.repeat(d.astype(np.float64), Q8_BLOCK, axis=-1)
+
+        def act(v):
+            return q8_exact(v)
+    else:
+        wload = bf16_to_f64
+
+        def act(v):
+            return sync_buffer(v, sync_quant)
+    wq, wk, wv = wload(inp.wq), wload(inp.wk), wload(inp.wv)
+    wo = wload(inp.wo)
 
     # a1-a2
-    xin = sync_buffer(rmsnorm(x, inp.attn_norm, s_.norm_eps), sync_quant)
+    xin = act(rmsnorm(x, inp.attn_norm, s_.norm_eps))
 
     # a3-a4, per slice
     kc = bf16_to_f64(inp.k_cache)
@@ -375,16 +417,26 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
         att_s = attention_decode(q_rot, kc, vc, pos, heads, H, Hkv, hd)
         cols = slice_range(H * hd, n, s)
         att_all[:, cols] = att_s
+        if weights_q8:
+            att_s = q8_exact(att_s)
         p_s = att_s @ wo[:, cols].T
         x1 = x1 + sync_buffer(p_s, sync_quant)
 
     # a7-a10
-    xin2 = sync_buffer(rmsnorm(x1, inp.ffn_norm, s_.norm_eps), sync_quant)
-    w1, w3, w2 = bf16_to_f64(inp.w1), bf16_to_f64(inp.w3), bf16_to_f64(inp.w2)
+    xin2 = act(rmsnorm(x1, inp.ffn_norm, s_.norm_eps))
+    w1, w3, w2 = wload(inp.w1), wload(inp.w3), wload(inp.w2)
     if trace is not None:
         trace.update(xin=xin, q=q_rot, att=att_all, x1=x1, xin2=xin2)
         if partition == 1:
             trace["h"] = swiglu(xin2 @ w1.T, xin2 @ w3.T)
+    if weights_q8:  # 1D FFN whose W2 inputs are Q8 too
+        hq = q8_exact(swiglu(xin2 @ w1.T, xin2 @ w3.T))
+        F = w1.shape[0]
+        x2 = x1.copy()
+        for s in range(n):
+            fs = slice_range(F, n, s)
+            x2 = x2 + sync_buffer(hq[:, fs] @ w2[:, fs].T, True)
+        return x2, k_new, v_new
     x2 = ffn_forward(xin2, w1, w2, act="swiglu", W3=w3, partition=partition, n_slices=n,
                      grid=grid, quant=sync_quant, residual=x1)
     return x2, k_new, v_new
