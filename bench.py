@@ -53,9 +53,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the C4 block and C3 model measurements")
-    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p"], default=None,
+    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w"], default=None,
                     help="only run a few eager steps of one extra workload (for profiler launch "
-                         "lists: c4 block, c3 model at batch 1, c2 block on the persistent kernel)")
+                         "lists: c4 block, c3 model at batch 1, c2 block on the persistent kernel, "
+                         "c2 block with int8 weights)")
     ap.add_argument("--profile-steps", type=int, default=3)
     return ap.parse_args(argv)
 
@@ -500,6 +501,60 @@ def bench_c2_persistent(args):
             "workload": "C2 block as one persistent kernel per step (same shapes as the headline)"}
 
 
+def bench_c2_q8w(args):
+    """The C2 block with int8 weights (tp_block_create_q8w): Q8 codes and scales for every
+    matrix, Q8 activations, integer block dot products; same shapes and batch 1."""
+    import torch
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+
+    s = synth.C2
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1001)
+    B, D, F, H, Hkv, hd = s.batch, s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim
+    mats = {k: _randn_bf16(torch, gen, shp, s.w_std) for k, shp in
+            (("wq", (H * hd, D)), ("wk", (Hkv * hd, D)), ("wv", (Hkv * hd, D)), ("wo", (D, H * hd)),
+             ("w1", (F, D)), ("w3", (F, D)), ("w2", (D, F)))}
+    qd = {}
+    for k, t in mats.items():
+        f = t.float()
+        q = torch.empty(f.shape, dtype=torch.int8, device="cuda")
+        d = torch.empty((f.shape[0], f.shape[1] // 32), dtype=torch.float32, device="cuda")
+        tpb.tp_quantize_q8(f, q, d, f.numel())
+        qd[k] = (q, d)
+        del f
+    del mats
+    ones = torch.ones(D, device="cuda")
+    kc = _randn_bf16(torch, gen, (B, Hkv, s.max_seq, hd), 1.0)
+    vc = _randn_bf16(torch, gen, (B, Hkv, s.max_seq, hd), 1.0)
+    x = torch.randn((B, D), generator=gen, device="cuda")
+    pos = torch.full((B,), s.pos, dtype=torch.int32, device="cuda")
+    dims = tpb.make_dims(D, H, Hkv, hd, F, s.vocab, B, s.max_seq, s.norm_eps, s.rope_theta)
+    nb = tpb.tp_block_workspace_bytes(dims, s.n_slices, 1, 1)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    w = tpb.make_weights_q8(ones, *qd["wq"], *qd["wk"], *qd["wv"], *qd["wo"], ones, *qd["w1"],
+                            *qd["w3"], *qd["w2"])
+    h = tpb.tp_block_create_q8w(dims, s.n_slices, 1, 1, w, ws, nb)
+    if args.profile == "c2q8w":
+        for _ in range(args.profile_steps):
+            tpb.tp_block_forward(h, x, kc, vc, pos, B)
+        torch.cuda.synchronize()
+        tpb.tp_block_destroy(h)
+        return {"profile": "c2q8w", "steps": args.profile_steps}
+    ms = _time_graph(torch, lambda: tpb.tp_block_forward(h, x, kc, vc, pos, B), 100, 20)
+    err = int(ws[tpb.tp_block_buffer(h, 7)[0]:][:4].view(torch.int32).item())
+    tpb.tp_block_destroy(h)
+    wb_bf16, kvb = block_bytes(s)
+    wb = wb_bf16 // 2 + wb_bf16 // 2 // 32 * 4  # int8 codes + a float32 scale per 32
+    hbm, _, _, kind = peaks()
+    gbs = (wb + kvb) / (ms / 1e3) / 1e9
+    return {"us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "hbm_gbs": gbs,
+            "frac": gbs / hbm, "bytes_per_step": wb + kvb, "pipeline_error": err,
+            "workload": "C2 block with int8 weights (Q8 codes + float32 scales per 32) and Q8 "
+                        "activations, batch 1, n=4"}
+
+
 def bench_c3(args, B):
     """Full 32-layer Llama-2-7B-shaped decode step (embedding -> logits), context 4096, n = 8."""
     import torch
@@ -613,7 +668,8 @@ def main(argv=None):
         print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
         return 1
     if args.profile:
-        fn = {"c4": bench_c4, "c3b1": lambda a: bench_c3(a, 1), "c2p": bench_c2_persistent}
+        fn = {"c4": bench_c4, "c3b1": lambda a: bench_c3(a, 1), "c2p": bench_c2_persistent,
+              "c2q8w": bench_c2_q8w}
         print(json.dumps(fn[args.profile](args)))
         return 0
     world, rank, local = dist_setup()
@@ -627,6 +683,11 @@ def main(argv=None):
             extra = {"c2_block_persistent": bench_c2_persistent(args)}
         except Exception as e:  # reported, not fatal: the headline does not depend on it
             extra = {"c2_block_persistent": {"error": str(e)[:200]}}
+        torch.cuda.empty_cache()
+        try:
+            extra["c2_block_int8_weights"] = bench_c2_q8w(args)
+        except Exception as e:  # reported, not fatal
+            extra["c2_block_int8_weights"] = {"error": str(e)[:200]}
         torch.cuda.empty_cache()
         extra["c4_block"] = bench_c4(args)
         torch.cuda.empty_cache()

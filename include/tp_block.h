@@ -89,6 +89,24 @@ typedef struct {
   const void* w2;         /* bf16 [dim, F]      row split (columns F_s)       */
 } tp_block_weights;
 
+/* The same parameters with int8 weights (Pope et al. demo4: decode is bound by the
+ * weight bytes, and int8 weights halve them). Each matrix is given as Q8 codes
+ * (int8, the same [out, in] layout and slicing as above) and float32 scales
+ * [out, in/32]: blocks of 32 consecutive elements along `in`, d = amax/127,
+ * codes = x/d rounded half away from zero (the sync-buffer format; tp_quantize_q8
+ * of the float32 weights produces exactly this). All pointers 16-byte aligned. */
+typedef struct {
+  const float* attn_norm;
+  const int8_t* wq; const float* wq_d;
+  const int8_t* wk; const float* wk_d;
+  const int8_t* wv; const float* wv_d;
+  const int8_t* wo; const float* wo_d;
+  const float* ffn_norm;
+  const int8_t* w1; const float* w1_d;
+  const int8_t* w3; const float* w3_d;
+  const int8_t* w2; const float* w2_d;
+} tp_block_weights_q8;
+
 typedef struct tp_block tp_block;
 
 /* Bytes of device workspace a block needs for dims->max_batch rows.
@@ -106,6 +124,18 @@ TP_API int tp_block_workspace_bytes(const tp_dims* dims, int n_slices, int parti
  * Errors: TP_EINVAL, TP_EALIGN, TP_EWORKSPACE, TP_EARCH, TP_ECUDA. */
 TP_API int tp_block_create(const tp_dims* dims, int n_slices, int partition, int sync_quant,
                     const tp_block_weights* w, void* workspace, size_t ws_bytes, tp_block** out);
+
+/* A block handle over int8 weights (tp_block_weights_q8). Every slice product
+ * then takes Q8 activations as well (the normalised inputs, the attention output
+ * before W_O, the SwiGLU output before W2, each quantised in blocks of 32) and
+ * runs as integer dot products per block scaled by d_w * d_x, accumulated in
+ * float32. Requires partition TP_PART_1D, sync_quant = 1 and ffn_dim % 64 == 0.
+ * tp_block_forward on such a handle takes batch <= 5 (the weight-streaming
+ * path); larger batches return TP_ENOTSUP. Workspace as for tp_block_create.
+ * Errors: TP_EINVAL, TP_EALIGN, TP_EWORKSPACE, TP_EARCH, TP_ENOTSUP. */
+TP_API int tp_block_create_q8w(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                               const tp_block_weights_q8* w, void* workspace, size_t ws_bytes,
+                               tp_block** out);
 
 /* One decode step of the block for `batch` rows (1 <= batch <= max_batch):
  *   x       float32 [batch, dim], read as the residual input and overwritten with

@@ -46,6 +46,12 @@ class tp_block_weights(C.Structure):
                                           "w3", "w2")]
 
 
+class tp_block_weights_q8(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("attn_norm", "wq", "wq_d", "wk", "wk_d", "wv", "wv_d", "wo",
+                                          "wo_d", "ffn_norm", "w1", "w1_d", "w3", "w3_d", "w2",
+                                          "w2_d")]
+
+
 class tp_ffn_desc(C.Structure):
     _fields_ = [(n, C.c_int32) for n in ("batch", "E", "F", "dtype", "act", "partition", "n_slices",
                                          "grid_x", "grid_y", "sync_quant", "merge")]
@@ -59,6 +65,9 @@ _sig = {
     "tp_block_workspace_bytes": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int, _SZ]),
     "tp_block_create": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int,
                                   C.POINTER(tp_block_weights), _P, C.c_size_t, C.POINTER(_P)]),
+    "tp_block_create_q8w": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int,
+                                      C.POINTER(tp_block_weights_q8), _P, C.c_size_t,
+                                      C.POINTER(_P)]),
     "tp_block_forward": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _P]),
     "tp_block_buffer": (C.c_int, [_P, C.c_int, _SZ, _SZ]),
     "tp_block_destroy": (None, [_P]),
@@ -142,6 +151,21 @@ def tp_block_create(dims, n_slices, partition, sync_quant, weights, workspace, w
     _check(_lib.tp_block_create(C.byref(dims), n_slices, partition, int(sync_quant),
                                 C.byref(weights), _ptr(workspace), ws_bytes, C.byref(h)),
            "tp_block_create")
+    return h.value
+
+
+def make_weights_q8(attn_norm, wq, wq_d, wk, wk_d, wv, wv_d, wo, wo_d, ffn_norm, w1, w1_d, w3,
+                    w3_d, w2, w2_d) -> tp_block_weights_q8:
+    """Int8 weights: each matrix as Q8 codes (int8) and float32 scales [out, in/32]."""
+    return tp_block_weights_q8(*[_ptr(t) for t in (attn_norm, wq, wq_d, wk, wk_d, wv, wv_d, wo, wo_d,
+                                                   ffn_norm, w1, w1_d, w3, w3_d, w2, w2_d)])
+
+
+def tp_block_create_q8w(dims, n_slices, partition, sync_quant, weights, workspace, ws_bytes) -> int:
+    h = C.c_void_p()
+    _check(_lib.tp_block_create_q8w(C.byref(dims), n_slices, partition, int(sync_quant),
+                                    C.byref(weights), _ptr(workspace), ws_bytes, C.byref(h)),
+           "tp_block_create_q8w")
     return h.value
 
 

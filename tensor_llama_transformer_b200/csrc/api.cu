@@ -198,6 +198,14 @@ struct tp_block {
   bool bar_ready;       // grid barrier counters known to be zero
   unsigned long long* trace;  // optional phase trace of the persistent kernel
   int persistent;       // use the persistent kernel where the shapes allow (batch 1-2, 1D)
+  bool wq8;             // int8 weights: w holds the codes, wd their scales
+  const float* wd_q;
+  const float* wd_k;
+  const float* wd_v;
+  const float* wd_o;
+  const float* wd_1;
+  const float* wd_3;
+  const float* wd_2;
 };
 
 struct tp_model {
@@ -482,6 +490,7 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
 // a model); the final merge here leaves them for the next block.
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
                        cudaStream_t s, bool chained = false) {
+  if (blk->wq8 && batch >= kTcMinBatch) return TP_ENOTSUP;
   if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained);
   if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent) {
     bool used = false;
@@ -504,6 +513,11 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.w[0] = static_cast<const uint16_t*>(blk->w.wq);
     a.w[1] = static_cast<const uint16_t*>(blk->w.wk);
     a.w[2] = static_cast<const uint16_t*>(blk->w.wv);
+    if (blk->wq8) {
+      a.wd[0] = blk->wd_q;
+      a.wd[1] = blk->wd_k;
+      a.wd[2] = blk->wd_v;
+    }
     a.rows[0] = QD;
     a.rows[1] = Hkv * hd;
     a.rows[2] = Hkv * hd;
@@ -551,6 +565,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   {
     GemvArgs a{};
     a.w[0] = static_cast<const uint16_t*>(blk->w.wo);
+    if (blk->wq8) a.wd[0] = blk->wd_o;
     a.rows[0] = D;
     a.ldw = QD;
     a.Ks = QD / c.n;
@@ -573,6 +588,10 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     GemvArgs a{};
     a.w[0] = static_cast<const uint16_t*>(blk->w.w1);
     a.w[1] = static_cast<const uint16_t*>(blk->w.w3);
+    if (blk->wq8) {
+      a.wd[0] = blk->wd_1;
+      a.wd[1] = blk->wd_3;
+    }
     a.rows[0] = F;
     a.ldw = D;
     a.Ks = D;
@@ -624,6 +643,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   {
     GemvArgs a{};
     a.w[0] = static_cast<const uint16_t*>(blk->w.w2);
+    if (blk->wq8) a.wd[0] = blk->wd_2;
     a.rows[0] = D;
     a.ldw = F;
     a.Ks = F / nseg2;
@@ -721,7 +741,36 @@ int tp_block_create(const tp_dims* dims, int n_slices, int partition, int sync_q
   b->bar_ready = false;
   b->trace = nullptr;
   b->persistent = persistent_default() ? 1 : 0;
+  b->wq8 = false;
   *out = b;
+  return TP_OK;
+}
+
+int tp_block_create_q8w(const tp_dims* dims, int n_slices, int partition, int sync_quant,
+                        const tp_block_weights_q8* w, void* workspace, size_t ws_bytes,
+                        tp_block** out) {
+  if (!out || !w || !dims) return TP_EINVAL;
+  *out = nullptr;
+  if (partition != TP_PART_1D || sync_quant != 1 || dims->ffn_dim % 64 != 0) return TP_EINVAL;
+  const void* ptrs[] = {w->attn_norm, w->wq, w->wq_d, w->wk, w->wk_d, w->wv, w->wv_d, w->wo, w->wo_d,
+                        w->ffn_norm, w->w1, w->w1_d, w->w3, w->w3_d, w->w2, w->w2_d};
+  for (const void* p : ptrs) {
+    if (!p) return TP_EINVAL;
+    if (!aligned16(p)) return TP_EALIGN;
+  }
+  tp_block_weights codes{w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->ffn_norm, w->w1, w->w3, w->w2};
+  const int rc = tp_block_create(dims, n_slices, partition, sync_quant, &codes, workspace, ws_bytes, out);
+  if (rc) return rc;
+  tp_block* b = *out;
+  b->wq8 = true;
+  b->persistent = 0;
+  b->wd_q = w->wq_d;
+  b->wd_k = w->wk_d;
+  b->wd_v = w->wv_d;
+  b->wd_o = w->wo_d;
+  b->wd_1 = w->w1_d;
+  b->wd_3 = w->w3_d;
+  b->wd_2 = w->w2_d;
   return TP_OK;
 }
 
@@ -744,6 +793,7 @@ void tp_block_destroy(tp_block* blk) { delete blk; }
 
 int tp_block_set_persistent(tp_block* blk, int enable) {
   if (!blk || (enable != 0 && enable != 1)) return TP_EINVAL;
+  if (enable && blk->wq8) return TP_ENOTSUP;
   blk->persistent = enable;
   return TP_OK;
 }
@@ -796,6 +846,7 @@ int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition,
   blk.bar_ready = true;  // the memsets above cover the persistent kernel's counters
   blk.trace = nullptr;
   blk.persistent = persistent_default() ? 1 : 0;
+  blk.wq8 = false;
   return block_forward_impl(&blk, x, k_cache, v_cache, pos, batch, stream);
 }
 }  // namespace tp

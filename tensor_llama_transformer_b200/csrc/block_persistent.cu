@@ -342,56 +342,6 @@ struct Consumer {
   }
 };
 
-// One ring stage of a GEMV phase for one consumer warp: PW row pairs (pairs pw
-// and pw + 8 when PW = 2), or 1/Q of one pair (vectors [vb, ve)) when Q > 1.
-template <int NB, int PW>
-TP_DEV void gemv_stage(const Consumer& c, uint32_t off, int cur, int end, const float4* xs,
-                       float* res, int nv, uint32_t rb, int pw, int part, int Q, int vb, int ve,
-                       int lane) {
-  constexpr int R = 2 * PW * NB;  // values: (pair j, row, batch row)
-  int rr[PW];
-  bool valid[PW];
-  const uint4* wr[PW];
-#pragma unroll
-  for (int j = 0; j < PW; ++j) {
-    rr[j] = cur + 2 * (pw + 8 * j);
-    valid[j] = c.ok && rr[j] < end;
-    wr[j] = reinterpret_cast<const uint4*>(c.ring + off + (size_t)(rr[j] - cur) * rb);
-  }
-  if (!valid[0]) return;  // pairs are filled in order: no pair for this warp
-  uint64_t acc[R][2];
-#pragma unroll
-  for (int i = 0; i < R; ++i) acc[i][0] = acc[i][1] = 0ull;
-#pragma unroll 4
-  for (int v = vb + lane; v < ve; v += 32) {
-    float4 lo[NB], hi[NB];
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      lo[b] = xs[b * nv + v];
-      hi[b] = xs[(NB + b) * nv + v];
-    }
-#pragma unroll
-    for (int j = 0; j < PW; ++j) {
-      if (!valid[j]) continue;
-      const uint4 u0 = wr[j][v], u1 = wr[j][nv + v];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        fma8_2(acc[(2 * j) * NB + b][0], acc[(2 * j) * NB + b][1], u0, lo[b], hi[b]);
-        fma8_2(acc[(2 * j + 1) * NB + b][0], acc[(2 * j + 1) * NB + b][1], u1, lo[b], hi[b]);
-      }
-    }
-  }
-  float val[R];
-#pragma unroll
-  for (int i = 0; i < R; ++i) val[i] = hsum2(acc[i][0]) + hsum2(acc[i][1]);
-  const float tot = warp_sum_multi<R>(val, lane);
-  constexpr int kLanes = 32 / R;  // lanes holding each total
-  if ((lane & (kLanes - 1)) == 0) {
-    const int i = lane / kLanes, j = i / (2 * NB), row = (i / NB) & 1, b = i % NB;
-    if (valid[j]) res[((size_t)(rr[j] + row) * NB + b) * Q + part] = tot;
-  }
-}
-
 // One GEMV phase for the consumer warps. stage(seg, publish) fills xs with the
 // segment's activations (lo halves [NB][nv], then hi halves); res receives the
 // per-row partial sums [row][NB][split].
@@ -419,8 +369,10 @@ TP_DEV void consume_gemv(Consumer& c, const BpGemv& g, float4* xs, float* res, i
     }
     const int end = min(min(nrows, seg_end), cur + 2 * g.pairs);
     const uint32_t off = c.next(round1k((uint32_t)(end - cur) * rb));
-    if (g.pw == 2) gemv_stage<NB, 2>(c, off, cur, end, xs, res, nv, rb, pw, part, Q, vb, ve, lane);
-    else gemv_stage<NB, 1>(c, off, cur, end, xs, res, nv, rb, pw, part, Q, vb, ve, lane);
+    if (c.ok) {
+      if (g.pw == 2) ring_pairs_dot<NB, 2>(c.ring + off, cur, end, xs, res, nv, rb, pw, part, Q, vb, ve, lane);
+      else ring_pairs_dot<NB, 1>(c.ring + off, cur, end, xs, res, nv, rb, pw, part, Q, vb, ve, lane);
+    }
     c.release();
     cur = end;
   }

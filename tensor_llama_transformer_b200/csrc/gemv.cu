@@ -84,17 +84,33 @@ TP_DEV int stage_end(int cur, int nrows, int R0, int rps, int P) {
   return min(min(nrows, seg_end), cur + 2 * P);
 }
 
-template <int NB, int EPI>
+// Stage bytes of one row of int8 weights beyond its codes: the 16-byte-aligned
+// run of global memory that covers the row's scales (a segment's scales need
+// not start on a 16-byte boundary), with room for the misalignment.
+inline __host__ __device__ uint32_t q8w_scale_slot(int Ks) {
+  return (((uint32_t)Ks / 32u * 4u + 15u) & ~15u) + 16u;
+}
+
+template <int NB, int PW>
+TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pad, int cur, int end,
+                              const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
+                              int part, int Q, int cb, int ce, int lane);
+
+template <int NB, int EPI, bool WQ8>
 __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_rstd[NB];
   __shared__ float s_red[8][NB];
   const int nc = pl.nc, nstage = pl.nstage, P = pl.pairs, Q = pl.split;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nv = a.Ks >> 3;  // 16-byte vectors per row
-  const uint32_t row_bytes = (uint32_t)a.Ks * 2;
+  const int nv = a.Ks >> 3;  // 8-element vectors per row
+  const uint32_t row_bytes = WQ8 ? (uint32_t)a.Ks : (uint32_t)a.Ks * 2;  // weight bytes of a row
+  const uint32_t slot = WQ8 ? row_bytes + q8w_scale_slot(a.Ks) : row_bytes;  // stage bytes of a row
   uint8_t* ring = smem + pl.ring_off;
   float4* xs = reinterpret_cast<float4*>(smem + pl.x_off);  // lo[NB][nv] then hi[NB][nv]
+  // int8 weights: the activations as Q8 codes [NB][Ks] and scales [NB][Ks / 32]
+  int8_t* xsq = reinterpret_cast<int8_t*>(smem + pl.x_off);
+  float* xsd = reinterpret_cast<float*>(smem + pl.x_off + (size_t)NB * a.Ks);
   float* res = reinterpret_cast<float*>(smem + pl.res_off);  // [rows of this CTA][NB]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.bar_off);
   uint64_t* empty = full + kMaxStages;
@@ -117,21 +133,52 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
 
   if (warp == nc) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
+    // (bf16 weights: lane 0 issues the copies; int8 weights, whose rows take two
+    // small copies each, spread them over the warp's lanes)
+    if (WQ8 || lane == 0) {
       const uint64_t pol = l2_evict_first();  // weights are read once per step
       int t = 0;
       for (int cur = 0; cur < nrows; ++t) {
         const int end = stage_end(cur, nrows, R0, rps, P);
         const int s = t % nstage;
         const uint32_t ph = (uint32_t)(t / nstage) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, a.err)) break;
-        mbar_expect_tx(&full[s], (uint32_t)(end - cur) * row_bytes);
-        uint8_t* dst = ring + (size_t)s * 2 * P * row_bytes;
+        bool waited = mbar_wait(&empty[s], ph ^ 1u, a.err);
+        if (WQ8) waited = __all_sync(0xffffffffu, waited);
+        if (!waited) break;
+        uint8_t* dst = ring + (size_t)s * 2 * P * slot;
         // one division per stage; rows are then walked with pointer increments
         const int seg = (R0 + cur) / rps;
         const int lr0 = R0 + cur - seg * rps;
         const int n = end - cur;
         const size_t col0 = (size_t)seg * a.Ks;
+        if constexpr (WQ8) {
+          // per row: its codes, then the aligned run covering its scales
+          const size_t sstride = (size_t)(a.ldw / 32) * 4, sseg = (size_t)seg * (a.Ks / 32) * 4;
+          const uint32_t sbytes = (uint32_t)(a.Ks / 32) * 4;
+          uint32_t tx = 0;
+          for (int i = lane; i < n; i += 32) {
+            int mat, lrow;
+            row_ptr<EPI>(a, seg, lr0 + i, mat, lrow);
+            const size_t s0 = (size_t)lrow * sstride + sseg;
+            tx += row_bytes + (uint32_t)(((s0 + sbytes + 15) & ~(size_t)15) - (s0 & ~(size_t)15));
+          }
+          tx = __reduce_add_sync(0xffffffffu, tx);
+          if (lane == 0) mbar_expect_tx(&full[s], tx);
+          __syncwarp();
+          for (int i = lane; i < n; i += 32) {
+            int mat, lrow;
+            row_ptr<EPI>(a, seg, lr0 + i, mat, lrow);
+            const int8_t* src = reinterpret_cast<const int8_t*>(a.w[mat]) + (size_t)lrow * a.ldw + col0;
+            bulk_g2s_hint(dst + (size_t)i * slot, src, row_bytes, &full[s], pol);
+            const size_t s0 = (size_t)lrow * sstride + sseg, slo = s0 & ~(size_t)15;
+            const uint32_t sl = (uint32_t)(((s0 + sbytes + 15) & ~(size_t)15) - slo);
+            bulk_g2s_hint(dst + (size_t)i * slot + row_bytes,
+                          reinterpret_cast<const uint8_t*>(a.wd[mat]) + slo, sl, &full[s], pol);
+          }
+          cur = end;
+          continue;
+        }
+        mbar_expect_tx(&full[s], (uint32_t)(end - cur) * row_bytes);
         if (EPI == EPI_SWIGLU) {  // rows alternate W1[f], W3[f]
           const uint16_t* p1 = a.w[0] + (size_t)(lr0 >> 1) * a.ldw + col0;
           const uint16_t* p3 = a.w[1] + (size_t)(lr0 >> 1) * a.ldw + col0;
@@ -222,6 +269,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
             const bool in = b < a.nb && v < nv;
             const size_t e0 = (size_t)(a.b0 + b) * a.ldx + col0 + 8 * (size_t)v;
             float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            uint2 qin = make_uint2(0u, 0u);  // codes as read (Q8 input)
+            float din = 0.f;
             if (in) {
               if (a.gain) {
                 const float rstd = s_rstd[b];
@@ -241,6 +290,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
               } else if (a.xq) {
                 const uint2 c = *reinterpret_cast<const uint2*>(a.xq + e0);
                 const float d = a.xd[e0 / kQ8Block];
+                qin = c;
+                din = d;
                 const float4 l = q8_unpack4(c.x, d), h = q8_unpack4(c.y, d);
                 xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
                 xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
@@ -251,7 +302,35 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
                 xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
               }
             }
-            if (a.gain && a.quant) {
+            if (WQ8) {
+              // the integer products need Q8 activations: the codes read, or those of xv
+              uint2 qc = qin;
+              float qd = din;
+              if (!a.xq || a.gain) {
+                float am = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
+                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+                qd = q8_scale(am);
+                qc = make_uint2(0u, 0u);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int c = q8_code(xv[e], qd);
+                  xv[e] = q8_value(c, qd);
+                  if (e < 4) qc.x |= (uint32_t)(c & 0xFF) << (8 * e);
+                  else qc.y |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
+                }
+                if (a.gain && publish && in && a.xq_out) {
+                  *reinterpret_cast<uint2*>(a.xq_out + e0) = qc;
+                  if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = qd;
+                }
+              }
+              if (v < nv) {
+                *reinterpret_cast<uint2*>(xsq + (size_t)b * a.Ks + 8 * (size_t)v) = qc;
+                if ((v & 3) == 0) xsd[(size_t)b * (a.Ks / 32) + (v >> 2)] = qd;
+              }
+            } else if (a.gain && a.quant) {
               float am = 0.f;
 #pragma unroll
               for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
@@ -276,7 +355,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
               *reinterpret_cast<float4*>(a.xn_out + e0 + 4) =
                   make_float4(xv[4], xv[5], xv[6], xv[7]);
             }
-            if (v < nv) {
+            if (!WQ8 && v < nv) {
               xs[b * nv + v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
               xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
             }
@@ -288,32 +367,31 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       // after a wait gives up, keep walking the stages (so that every consumer warp
       // reaches the same named barriers) but skip the work
       if (ok && !mbar_wait(&full[s], ph, a.err)) ok = false;
-      const int r = cur + 2 * pw;  // this warp's row pair in the stage
-      if (ok && r < end) {
-        const uint4* w0 = reinterpret_cast<const uint4*>(ring + ((size_t)s * 2 * P + 2 * pw) * row_bytes);
-        const uint4* w1 = w0 + nv;
-        constexpr int R = 2 * NB;  // values: (row of the pair, batch row)
-        uint64_t acc[R][2];
-#pragma unroll
-        for (int i = 0; i < R; ++i) acc[i][0] = acc[i][1] = 0ull;
-#pragma unroll 4
-        for (int v = vb + lane; v < ve; v += 32) {
-          const uint4 u0 = w0[v], u1 = w1[v];
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const float4 lo = xs[b * nv + v], hi = xs[(NB + b) * nv + v];
-            fma8_2(acc[b][0], acc[b][1], u0, lo, hi);
-            fma8_2(acc[NB + b][0], acc[NB + b][1], u1, lo, hi);
+      if (ok) {
+        const uint8_t* st = ring + (size_t)s * 2 * P * slot;
+        if constexpr (WQ8) {
+          // scale offset (floats) of each of the warp's rows inside its aligned run
+          int pad[2 * 2];
+          for (int i = 0; i < 2 * pl.pw; ++i) {
+            const int r = cur + 2 * (pw + 8 * (i >> 1)) + (i & 1);
+            pad[i] = 0;
+            if (r < end) {
+              const int gr = R0 + r, sg = gr / rps;
+              int mat, lrow;
+              row_ptr<EPI>(a, sg, gr - sg * rps, mat, lrow);
+              pad[i] = (int)(((size_t)lrow * (a.ldw / 32) + (size_t)sg * (a.Ks / 32)) & 3);
+            }
           }
-        }
-        float val[R];
-#pragma unroll
-        for (int i = 0; i < R; ++i) val[i] = hsum2(acc[i][0]) + hsum2(acc[i][1]);
-        const float tot = warp_sum_multi<R>(val, lane);
-        constexpr int kLanes = 32 / R;  // lanes holding each total
-        if ((lane & (kLanes - 1)) == 0) {
-          const int i = lane / kLanes, row = i / NB, b = i - row * NB;
-          res[((size_t)(r + row) * NB + b) * Q + part] = tot;
+          const int nc16 = a.Ks >> 4, cb = (nc16 * part) / Q, ce = (nc16 * (part + 1)) / Q;
+          if (pl.pw == 2)
+            ring_pairs_dot_q8<NB, 2>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+          else
+            ring_pairs_dot_q8<NB, 1>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+        } else {
+          if (pl.pw == 2)
+            ring_pairs_dot<NB, 2>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
+          else
+            ring_pairs_dot<NB, 1>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
         }
       }
       __syncwarp();
@@ -373,18 +451,77 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   }
 }
 
+// The int8-weight consumer step (see ring_pairs_dot): each row's codes are read
+// 16 at a time, 16 consecutive bytes per lane (conflict-free), against the
+// activation codes with four dp4a; the integer sum of a half block is scaled by
+// d_w d_x of its 32-value block and accumulated in float32. pad[i] is the offset
+// (floats) of row i's scales inside its aligned run in the stage.
+template <int NB, int PW>
+TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pad, int cur, int end,
+                              const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
+                              int part, int Q, int cb, int ce, int lane) {
+  constexpr int R = 2 * PW * NB;  // values: (pair j, row, batch row)
+  int rr[PW];
+  bool valid[PW];
+#pragma unroll
+  for (int j = 0; j < PW; ++j) {
+    rr[j] = cur + 2 * (pw + 8 * j);
+    valid[j] = rr[j] < end;
+  }
+  if (!valid[0]) return;
+  const int nblk = Ks >> 5;
+  float acc[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) acc[i] = 0.f;
+#pragma unroll 2
+  for (int c = cb + lane; c < ce; c += 32) {
+    int4 xq[NB];
+    float xd[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      xq[b] = *reinterpret_cast<const int4*>(xsq + (size_t)b * Ks + 16 * c);
+      xd[b] = xsd[b * nblk + (c >> 1)];
+    }
+#pragma unroll
+    for (int j = 0; j < PW; ++j) {
+      if (!valid[j]) continue;
+#pragma unroll
+      for (int row = 0; row < 2; ++row) {
+        const uint8_t* rp = stage + (size_t)(rr[j] + row - cur) * slot;
+        const int4 wq = *reinterpret_cast<const int4*>(rp + 16 * c);
+        const float dw = reinterpret_cast<const float*>(rp + Ks)[pad[2 * j + row] + (c >> 1)];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          int sdot = __dp4a(wq.x, xq[b].x, 0);
+          sdot = __dp4a(wq.y, xq[b].y, sdot);
+          sdot = __dp4a(wq.z, xq[b].z, sdot);
+          sdot = __dp4a(wq.w, xq[b].w, sdot);
+          acc[(2 * j + row) * NB + b] = fmaf((float)sdot, dw * xd[b], acc[(2 * j + row) * NB + b]);
+        }
+      }
+    }
+  }
+  const float tot = warp_sum_multi<R>(acc, lane);
+  constexpr int kLanes = 32 / R;
+  if ((lane & (kLanes - 1)) == 0) {
+    const int i = lane / kLanes, j = i / (2 * NB), row = (i / NB) & 1, b = i % NB;
+    if (valid[j]) res[((size_t)(rr[j] + row) * NB + b) * Q + part] = tot;
+  }
+}
+
 size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
 
-// Shared-memory plan: 8 consumer warps; the most row pairs per stage (8, 4, 2,
-// 1) that still leave a ring of at least 3 stages (2 for the longest rows), each
-// pair split over 8 / pairs warps.
-bool make_plan(int NB, int Ks, int cta_rows, GemvPlan* p) {
-  const size_t row_bytes = (size_t)Ks * 2;
-  const size_t x_bytes = a128((size_t)NB * Ks * 4);
+// Shared-memory plan: 8 consumer warps; the most row pairs per stage (16, 8, 4,
+// 2, 1) that still leave a ring of at least 3 stages (2 for the longest rows):
+// 16 pairs give each warp two pairs, fewer are each split over 8 / pairs warps.
+bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
+  const size_t row_bytes = wq8 ? (size_t)Ks + q8w_scale_slot(Ks) : (size_t)Ks * 2;
+  const size_t x_bytes = wq8 ? a128((size_t)NB * Ks + (size_t)NB * (Ks / 32) * 4)
+                             : a128((size_t)NB * Ks * 4);
   const size_t bar_bytes = 2 * kMaxStages * 8;
   for (int min_stages : {3, 2}) {
-    for (int P = 8; P >= 1; P >>= 1) {
-      const int Q = 8 / P;
+    for (int P = 16; P >= 1; P >>= 1) {
+      const int Q = P >= 8 ? 1 : 8 / P;
       const size_t res_bytes = a128((size_t)cta_rows * NB * Q * 4);
       const size_t fixed = x_bytes + res_bytes + bar_bytes;
       if (fixed >= (size_t)kSmemBudget) continue;
@@ -395,6 +532,7 @@ bool make_plan(int NB, int Ks, int cta_rows, GemvPlan* p) {
         p->nc = 8;
         p->pairs = P;
         p->split = Q;
+        p->pw = P == 16 ? 2 : 1;
         p->nstage = ns;
         p->cta_rows = cta_rows;
         p->ring_off = 0;
@@ -409,7 +547,7 @@ bool make_plan(int NB, int Ks, int cta_rows, GemvPlan* p) {
   return false;
 }
 
-template <int NB, int EPI>
+template <int NB, int EPI, bool WQ8>
 int launch_one(const GemvArgs& a, cudaStream_t s) {
   int rps = a.rows[0];
   if (EPI == EPI_SWIGLU) rps = 2 * a.rows[0];
@@ -419,18 +557,23 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   if (grid > npairs) grid = npairs;
   const int cta_rows = 2 * ((npairs + grid - 1) / grid);
   GemvPlan pl;
-  if (!make_plan(NB, a.Ks, cta_rows, &pl)) return TP_ENOTSUP;
-  if (set_smem_once((const void*)k_gemv<NB, EPI>, (int)pl.total)) return TP_ECUDA;
-  return launch_pdl(k_gemv<NB, EPI>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
+  if (!make_plan(NB, a.Ks, cta_rows, WQ8, &pl)) return TP_ENOTSUP;
+  if (set_smem_once((const void*)k_gemv<NB, EPI, WQ8>, (int)pl.total)) return TP_ECUDA;
+  return launch_pdl(k_gemv<NB, EPI, WQ8>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
+}
+
+template <int NB, bool WQ8>
+int launch_nbw(const GemvArgs& a, int epi, cudaStream_t s) {
+  switch (epi) {
+    case EPI_PLAIN: return launch_one<NB, EPI_PLAIN, WQ8>(a, s);
+    case EPI_SWIGLU: return launch_one<NB, EPI_SWIGLU, WQ8>(a, s);
+    default: return launch_one<NB, EPI_QKV, WQ8>(a, s);
+  }
 }
 
 template <int NB>
 int launch_nb(const GemvArgs& a, int epi, cudaStream_t s) {
-  switch (epi) {
-    case EPI_PLAIN: return launch_one<NB, EPI_PLAIN>(a, s);
-    case EPI_SWIGLU: return launch_one<NB, EPI_SWIGLU>(a, s);
-    default: return launch_one<NB, EPI_QKV>(a, s);
-  }
+  return a.wd[0] ? launch_nbw<NB, true>(a, epi, s) : launch_nbw<NB, false>(a, epi, s);
 }
 
 }  // namespace
@@ -438,6 +581,7 @@ int launch_nb(const GemvArgs& a, int epi, cudaStream_t s) {
 // Batch rows are handled two at a time (each launch streams the weights once).
 int launch_gemv(const GemvArgs& a0, int epi, cudaStream_t s) {
   if (a0.Ks % 32 != 0 || a0.Ks < 32 || a0.nseg < 1) return TP_EINVAL;
+  if (a0.wd[0] && a0.ldw % 64 != 0) return TP_EINVAL;  // whole 16-byte scale runs per matrix
   if (((a0.rows[0] | a0.rows[1] | a0.rows[2]) & 1) != 0) return TP_EINVAL;
   for (int b = 0; b < a0.nb;) {
     GemvArgs a = a0;

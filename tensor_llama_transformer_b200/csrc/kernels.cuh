@@ -26,6 +26,10 @@ struct GemvArgs {
   const uint16_t* w[3];
   int rows[3];
   int64_t ldw;   // row stride in elements (= full input width K)
+  // int8 weights: w[i] then holds Q8 codes (int8, same layout) and wd[i] their
+  // float32 scales [rows_i, ldw / 32]; the activations enter as Q8 codes too and
+  // the products are integer dot products per 32-value block, scaled by d_w d_x.
+  const float* wd[3];
   int Ks;        // contraction length of one segment
   int nseg;      // number of segments: segment s reads columns [s*Ks, (s+1)*Ks)
   // input: float32 x [B, ldx] or Q8 (xq [B, ldx], xd [B, ldx/32]); with `gain`
@@ -69,6 +73,7 @@ struct GemvPlan {
   int nc;
   int pairs;
   int split;
+  int pw;  // row pairs per warp and stage (2 with 16 pairs per stage)
   int nstage;
   int cta_rows;
   size_t ring_off, x_off, res_off, bar_off, total;

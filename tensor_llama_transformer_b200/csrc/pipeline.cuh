@@ -199,6 +199,60 @@ TP_DEV float warp_sum_multi(float (&v)[R], int lane) {
   return t;
 }
 
+// The GEMV consumer step for one warp and one ring stage (rows cur .. end-1 of
+// the CTA's range, stored from `stage`, row_bytes each): with PW = 2, row pairs
+// pw and pw + 8 of the stage; with PW = 1, pair pw, or 1/Q of it (vectors
+// [vb, ve) of 8 elements) when Q > 1. Each row is dotted with the NB staged
+// activation rows (xs: lo halves [NB][nv], then hi halves) with packed FMA, and
+// the warp's 2 PW NB sums are reduced in one butterfly:
+//   res[((r + row) NB + b) Q + part] = sum.
+template <int NB, int PW>
+TP_DEV void ring_pairs_dot(const uint8_t* stage, int cur, int end, const float4* xs, float* res,
+                           int nv, uint32_t rb, int pw, int part, int Q, int vb, int ve, int lane) {
+  constexpr int R = 2 * PW * NB;  // values: (pair j, row, batch row)
+  int rr[PW];
+  bool valid[PW];
+  const uint4* wr[PW];
+#pragma unroll
+  for (int j = 0; j < PW; ++j) {
+    rr[j] = cur + 2 * (pw + 8 * j);
+    valid[j] = rr[j] < end;
+    wr[j] = reinterpret_cast<const uint4*>(stage + (size_t)(rr[j] - cur) * rb);
+  }
+  if (!valid[0]) return;  // pairs are filled in order: no pair for this warp
+  uint64_t acc[R][2];
+#pragma unroll
+  for (int i = 0; i < R; ++i) acc[i][0] = acc[i][1] = 0ull;
+#pragma unroll 4
+  for (int v = vb + lane; v < ve; v += 32) {
+    float4 lo[NB], hi[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      lo[b] = xs[b * nv + v];
+      hi[b] = xs[(NB + b) * nv + v];
+    }
+#pragma unroll
+    for (int j = 0; j < PW; ++j) {
+      if (!valid[j]) continue;
+      const uint4 u0 = wr[j][v], u1 = wr[j][nv + v];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        fma8_2(acc[(2 * j) * NB + b][0], acc[(2 * j) * NB + b][1], u0, lo[b], hi[b]);
+        fma8_2(acc[(2 * j + 1) * NB + b][0], acc[(2 * j + 1) * NB + b][1], u1, lo[b], hi[b]);
+      }
+    }
+  }
+  float val[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) val[i] = hsum2(acc[i][0]) + hsum2(acc[i][1]);
+  const float tot = warp_sum_multi<R>(val, lane);
+  constexpr int kLanes = 32 / R;  // lanes holding each total
+  if ((lane & (kLanes - 1)) == 0) {
+    const int i = lane / kLanes, j = i / (2 * NB), row = (i / NB) & 1, b = i % NB;
+    if (valid[j]) res[((size_t)(rr[j] + row) * NB + b) * Q + part] = tot;
+  }
+}
+
 // Shared address of 16-byte chunk c (8 dims, 0..15) of row t of a 64-row K or
 // V tile that TMA wrote as two boxes of 64 rows x 64 dims (8 KB each, the first
 // for dims 0..63) with the 128-byte swizzle; base must be 1024-byte aligned.
