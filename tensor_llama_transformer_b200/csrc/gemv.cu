@@ -370,17 +370,19 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       if (ok) {
         const uint8_t* st = ring + (size_t)s * 2 * P * slot;
         if constexpr (WQ8) {
-          // scale offset (floats) of each of the warp's rows inside its aligned run
+          // scale offset (floats) of each of the warp's rows inside its aligned run:
+          // (lrow * ldw / 32 + seg * Ks / 32) mod 4. Matrix boundaries inside a
+          // segment's rows are multiples of 4 rows (multiples of 128), so lrow mod 4
+          // follows from the row's place in its segment (halved for W1/W3 pairs).
           int pad[2 * 2];
-          for (int i = 0; i < 2 * pl.pw; ++i) {
+          const int s32 = (int)((a.ldw / 32) & 3), segpad = (int)(((size_t)seg * (a.Ks / 32)) & 3);
+          const int seg_first = seg * rps - R0;  // CTA-local row where this segment starts
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
             const int r = cur + 2 * (pw + 8 * (i >> 1)) + (i & 1);
-            pad[i] = 0;
-            if (r < end) {
-              const int gr = R0 + r, sg = gr / rps;
-              int mat, lrow;
-              row_ptr<EPI>(a, sg, gr - sg * rps, mat, lrow);
-              pad[i] = (int)(((size_t)lrow * (a.ldw / 32) + (size_t)sg * (a.Ks / 32)) & 3);
-            }
+            int lr = r - seg_first;
+            if (EPI == EPI_SWIGLU) lr >>= 1;
+            pad[i] = ((lr & 3) * s32 + segpad) & 3;
           }
           const int nc16 = a.Ks >> 4, cb = (nc16 * part) / Q, ce = (nc16 * (part + 1)) / Q;
           if (pl.pw == 2)
