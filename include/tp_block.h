@@ -68,8 +68,9 @@ enum { TP_F32 = 0, TP_BF16 = 1 };
 enum { TP_MERGE_FAITHFUL = 0, TP_MERGE_FUSED = 1 };
 
 /* Model dimensions (the distributed-llama TransformerSpec, reduced to what one
- * block needs). Requirements checked at create: dim % 32 == 0, head_dim == 128,
- * n_heads % n_kv_heads == 0, H % n == 0, Hkv % n == 0, ffn_dim % (32*n) == 0,
+ * block needs). Requirements checked at create: dim % 128 == 0, head_dim == 128,
+ * n_heads / n_kv_heads (query heads per kv head) in {1, 2, 4} or a multiple of 8
+ * up to 64 (multi-query attention), H % n == 0, Hkv % n == 0, ffn_dim % (32*n) == 0,
  * 1 <= max_batch <= 64, 1 <= max_seq. */
 typedef struct {
   int32_t dim, n_heads, n_kv_heads, head_dim, ffn_dim, vocab, max_batch, max_seq;

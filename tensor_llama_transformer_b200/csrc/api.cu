@@ -114,8 +114,8 @@ int check_cfg(const tp_dims* d, int n, int partition, int quant, Cfg* c) {
   if (d->dim <= 0 || d->dim % 128 != 0) return TP_EINVAL;
   if (d->head_dim != kHeadDim) return TP_ENOTSUP;
   if (d->n_heads <= 0 || d->n_kv_heads <= 0 || d->n_heads % d->n_kv_heads != 0) return TP_EINVAL;
-  const int G = d->n_heads / d->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return TP_ENOTSUP;
+  const int G = d->n_heads / d->n_kv_heads;  // query heads per kv head (GQA / MQA)
+  if (G != 1 && G != 2 && G != 4 && !(G % 8 == 0 && G <= 64)) return TP_ENOTSUP;
   if (d->n_heads % n != 0 || d->n_kv_heads % n != 0) return TP_EINVAL;
   if (d->ffn_dim <= 0 || d->ffn_dim % (32 * n) != 0) return TP_EINVAL;
   if (d->max_batch < 1 || d->max_batch > 64 || d->max_seq < 1) return TP_EINVAL;

@@ -5,7 +5,9 @@
 // attention of its own heads locally; tt-metal's Llama-2 thread separates GQA
 // from MHA. A CTA owns (context split, kv head, batch row) and every query head
 // that reads that kv head (1 for MHA, 8 for the 70B shape), so each K/V byte is
-// read from HBM once per step. The split's 64-position K and V tiles stream
+// read from HBM once per step. With more query heads per kv head (multi-query
+// attention, Pope et al. demo 3: up to 64 on one kv head) the heads go in groups
+// of 8 to CTAs that read the same tiles, concurrently, mostly from L2. The split's 64-position K and V tiles stream
 // through a 3-stage shared-memory ring by TMA (128-byte swizzle, so the
 // ldmatrix reads below are conflict-free), issued by a producer warp. Four
 // consumer warps take 16 positions of each tile:
@@ -56,7 +58,11 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   __shared__ uint64_t full[kStages], empty[kStages];
   __shared__ float s_m[kCWarps][8], s_l[kCWarps][8];
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  // blockIdx.y = kv head x groups of G query heads: with more than 8 query heads
+  // per kv head (multi-query attention), groups of 8 share the kv head's tiles
+  const int hgroups = a.H / a.Hkv / G;
+  const int split = blockIdx.x, kvh = blockIdx.y / hgroups, b = blockIdx.z;
+  const int h0 = kvh * (a.H / a.Hkv) + (blockIdx.y - kvh * hgroups) * G;  // first query head
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
   pdl_wait();  // q and the cache rows at pos come from the q/k/v kernel
@@ -64,7 +70,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   const int ntiles = (P + kTile - 1) / kTile;
   const int tpc = tiles_per_split(P, nsplit);
   const int i0 = split * tpc, i1 = min(ntiles, i0 + tpc);
-  const size_t pbase = ((size_t)b * a.H + (size_t)kvh * G) * nsplit + split;
+  const size_t pbase = ((size_t)b * a.H + (size_t)h0) * nsplit + split;
   if (i0 >= i1) {  // nothing left for this split (the combine does not read it)
     if (threadIdx.x < G) {
       a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 0] = -INFINITY;
@@ -87,7 +93,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
     const int g = i / kHeadDim, d = i - g * kHeadDim;
     uint16_t hi = 0, lo = 0;
     if (g < G)
-      bf16_split(a.q[((size_t)b * a.H + (size_t)kvh * G + g) * kHeadDim + d] * scale, hi, lo);
+      bf16_split(a.q[((size_t)b * a.H + (size_t)h0 + g) * kHeadDim + d] * scale, hi, lo);
     qs[g * kQStride + d] = hi;
     qs[(g + 8) * kQStride + d] = lo;
   }
@@ -280,7 +286,8 @@ template <int G>
 int launch_g(const AttnArgs& a, const CUtensorMap& mK, const CUtensorMap& mV, int nsplit,
              cudaStream_t s) {
   if (set_smem_once((const void*)k_attn_split<G>, kSmemBytes)) return TP_ECUDA;
-  return launch_pdl(k_attn_split<G>, dim3(nsplit, a.Hkv, a.B), dim3(kAThreads), kSmemBytes, s,
+  const int hgroups = a.H / a.Hkv / G;
+  return launch_pdl(k_attn_split<G>, dim3(nsplit, a.Hkv * hgroups, a.B), dim3(kAThreads), kSmemBytes, s,
                     mK, mV, a, nsplit);
 }
 
@@ -311,7 +318,8 @@ int attention_splits(int B, int Hkv, int max_seq) {
 
 int launch_attention(const AttnArgs& a, cudaStream_t s) {
   const int G = a.H / a.Hkv;
-  const int nsplit = attention_splits(a.B, a.Hkv, a.max_seq);
+  const int hgroups = G > 8 ? G / 8 : 1;  // CTAs per kv head
+  const int nsplit = attention_splits(a.B, a.Hkv * hgroups, a.max_seq);
   if (nsplit > a.nchunk) return TP_EINVAL;
   if (!aligned16(a.kc) || !aligned16(a.vc)) return TP_EALIGN;
   CUtensorMap mK, mV;
@@ -325,7 +333,10 @@ int launch_attention(const AttnArgs& a, cudaStream_t s) {
     case 2: rc = launch_g<2>(a, mK, mV, nsplit, s); break;
     case 4: rc = launch_g<4>(a, mK, mV, nsplit, s); break;
     case 8: rc = launch_g<8>(a, mK, mV, nsplit, s); break;
-    default: return TP_ENOTSUP;
+    default:
+      if (G % 8 != 0 || G > 64) return TP_ENOTSUP;
+      rc = launch_g<8>(a, mK, mV, nsplit, s);  // groups of 8 query heads per CTA
+      break;
   }
   if (rc != TP_OK) return rc;
   return launch_pdl(k_attn_combine, dim3(a.H, a.B), dim3(kHeadDim), 0, s, a, nsplit);

@@ -110,9 +110,17 @@ SMALL_GQA8 = synth.BlockShape(dim=1024, n_heads=8, n_kv_heads=1, head_dim=128, f
                               w_std=0.03)
 
 
+MQA16 = synth.BlockShape(dim=512, n_heads=16, n_kv_heads=1, head_dim=128, ffn_dim=1024, vocab=0,
+                         max_seq=200, batch=2, n_slices=1, sync_quant=False, pos=199, w_std=0.03)
+MQA64 = synth.BlockShape(dim=512, n_heads=64, n_kv_heads=1, head_dim=128, ffn_dim=1024, vocab=0,
+                         max_seq=140, batch=3, n_slices=1, sync_quant=False, pos=139, w_std=0.02)
+
+
 @pytest.mark.parametrize("quant", [0, 1])
 @pytest.mark.parametrize("shape,n,pos", [
     (SMALL_MHA, 2, [299, 130, 0]),      # ragged context: 5 tiles of 64, 3 tiles, a single position
+    (MQA16, 1, [199, 64]),              # multi-query: 16 query heads on one kv head (2 CTA groups)
+    (MQA64, 1, [139, 0, 70]),           # multi-query: 64 query heads on one kv head (8 groups)
     (SMALL_GQA, 2, [259, 127]),         # GQA group of 4 per kv head
     (SMALL_GQA8, 1, [128, 1, 64, 127, 5]),  # GQA group of 8, batch 5 (two launches of 4 + 1)
 ])
@@ -173,7 +181,8 @@ SMALL_TC_MHA = synth.BlockShape(dim=1024, n_heads=8, n_kv_heads=8, head_dim=128,
 
 @pytest.mark.parametrize("quant", [0, 1])
 @pytest.mark.parametrize("shape,n,partition", [
-    (SMALL_TC_GQA, 2, 1), (SMALL_TC_GQA, 2, 2), (SMALL_TC_MHA, 8, 1)])
+    (SMALL_TC_GQA, 2, 1), (SMALL_TC_GQA, 2, 2), (SMALL_TC_MHA, 8, 1),
+    (synth.BlockShape(**{**MQA16.__dict__, "batch": 7}), 1, 1)])  # multi-query, batched
 def test_block_batched_tensor_path(tpb, shape, n, partition, quant):
     inp = synth.block_inputs(5252, shape)
     B = shape.batch
