@@ -349,7 +349,9 @@ def bench_block(args, world, rank, local):
     hbm, bf16_tf, bf16_sus, peak_kind = peaks()
     w13_bytes = 2 * s.ffn_dim * s.dim * 2 + B * s.dim * (1 + 4 / 32) + B * s.ffn_dim * 4
     w13_s = stage_ms_max[STAGES.index("norm_w13_swiglu")] / 1e3
-    launches_per_step = 8  # batch <= 4: one launch per stage, attention = chunks + combine
+    # batch 1 (weight-streaming path): q/k/v GEMV, attention splits, W_O GEMV (which also
+    # combines the splits), merge, W1/W3 GEMV, W2 GEMV, merge
+    launches_per_step = 7
     res = {
         "tokens_per_s": world * B * K / (ms_max / 1e3), "ms_per_step": ms_max / K, "K": K,
         "block_gbs": (wbytes + kvbytes) / step_s / 1e9, "stage_us": {

@@ -558,7 +558,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.part_ml = at<float>(blk, BUF_PML);
     a.att = at<float>(blk, BUF_ATT);
     a.err = at<int>(blk, BUF_ERR);
-    if ((rc = launch_attention(a, s))) return rc;
+    if ((rc = launch_attention(a, s, false))) return rc;  // W_O's staging combines the splits
   }
   // a5: W_O row-split partials, one plane per slice
   if ((rc = stage_mark(blk, 2, s))) return rc;
@@ -570,7 +570,12 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     a.ldw = QD;
     a.Ks = QD / c.n;
     a.nseg = c.n;
-    a.x = at<float>(blk, BUF_ATT);
+    a.att_po = at<float>(blk, BUF_PO);
+    a.att_pml = at<float>(blk, BUF_PML);
+    a.att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq);
+    a.att_out = at<float>(blk, BUF_ATT);
+    a.pos = pos;
+    a.n_heads = H;
     a.ldx = QD;
     a.nb = batch;
     a.out = part;

@@ -316,10 +316,15 @@ int attention_splits(int B, int Hkv, int max_seq) {
   return best;
 }
 
-int launch_attention(const AttnArgs& a, cudaStream_t s) {
-  const int G = a.H / a.Hkv;
+int attention_nsplit(int B, int H, int Hkv, int max_seq) {
+  const int G = H / Hkv;
   const int hgroups = G > 8 ? G / 8 : 1;  // CTAs per kv head
-  const int nsplit = attention_splits(a.B, a.Hkv * hgroups, a.max_seq);
+  return attention_splits(B, Hkv * hgroups, max_seq);
+}
+
+int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {
+  const int G = a.H / a.Hkv;
+  const int nsplit = attention_nsplit(a.B, a.H, a.Hkv, a.max_seq);
   if (nsplit > a.nchunk) return TP_EINVAL;
   if (!aligned16(a.kc) || !aligned16(a.vc)) return TP_EALIGN;
   CUtensorMap mK, mV;
@@ -338,7 +343,7 @@ int launch_attention(const AttnArgs& a, cudaStream_t s) {
       rc = launch_g<8>(a, mK, mV, nsplit, s);  // groups of 8 query heads per CTA
       break;
   }
-  if (rc != TP_OK) return rc;
+  if (rc != TP_OK || !combine) return rc;
   return launch_pdl(k_attn_combine, dim3(a.H, a.B), dim3(kHeadDim), 0, s, a, nsplit);
 }
 

@@ -287,6 +287,36 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
                 xv[5] = __fmul_rn(__fmul_rn(x1.y, rstd), g1.y);
                 xv[6] = __fmul_rn(__fmul_rn(x1.z, rstd), g1.z);
                 xv[7] = __fmul_rn(__fmul_rn(x1.w, rstd), g1.w);
+              } else if (a.att_po) {
+                // the attention output of these 8 dims, combined from the context splits:
+                // M = max_c m_c, o = sum_c e^{m_c - M} o_c / sum_c e^{m_c - M} l_c
+                const int gb = a.b0 + b;
+                const int P = a.pos[gb] + 1, ntiles = (P + 63) / 64;
+                const int tpc = (ntiles + a.att_nsplit - 1) / a.att_nsplit;
+                const int ncs = (ntiles + tpc - 1) / tpc;
+                const int col = (int)col0 + 8 * v, h = col / kHeadDim, d0 = col - h * kHeadDim;
+                const size_t base = ((size_t)gb * a.n_heads + h) * a.att_nsplit;
+                float M = -INFINITY;
+                for (int c = 0; c < ncs; ++c) M = fmaxf(M, a.att_pml[(base + c) * 2]);
+                float L = 0.f;
+                for (int c = 0; c < ncs; ++c) {
+                  const float mc = a.att_pml[(base + c) * 2];
+                  const float w = mc == -INFINITY ? 0.f : expf(mc - M);
+                  L = fmaf(w, a.att_pml[(base + c) * 2 + 1], L);
+                  const float4 o0 = *reinterpret_cast<const float4*>(a.att_po + (base + c) * kHeadDim + d0);
+                  const float4 o1 = *reinterpret_cast<const float4*>(a.att_po + (base + c) * kHeadDim + d0 + 4);
+                  xv[0] = fmaf(w, o0.x, xv[0]); xv[1] = fmaf(w, o0.y, xv[1]);
+                  xv[2] = fmaf(w, o0.z, xv[2]); xv[3] = fmaf(w, o0.w, xv[3]);
+                  xv[4] = fmaf(w, o1.x, xv[4]); xv[5] = fmaf(w, o1.y, xv[5]);
+                  xv[6] = fmaf(w, o1.z, xv[6]); xv[7] = fmaf(w, o1.w, xv[7]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xv[e] = xv[e] / L;
+                if (publish && a.att_out) {
+                  float* dst = a.att_out + (size_t)gb * a.ldx + col;
+                  *reinterpret_cast<float4*>(dst) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+                  *reinterpret_cast<float4*>(dst + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
+                }
               } else if (a.xq) {
                 const uint2 c = *reinterpret_cast<const uint2*>(a.xq + e0);
                 const float d = a.xd[e0 / kQ8Block];

@@ -30,6 +30,14 @@ struct GemvArgs {
   // float32 scales [rows_i, ldw / 32]; the activations enter as Q8 codes too and
   // the products are integer dot products per 32-value block, scaled by d_w d_x.
   const float* wd[3];
+  // input taken from the attention's context splits instead of x (W_O on the
+  // weight-streaming path): partial outputs [B, H, att_nsplit, hd] and (m, l)
+  // [B, H, att_nsplit, 2], combined while staging; the CTA that owns a segment's
+  // first row writes the combined row to att_out [B, H*hd].
+  const float* att_po;
+  const float* att_pml;
+  int att_nsplit;
+  float* att_out;
   int Ks;        // contraction length of one segment
   int nseg;      // number of segments: segment s reads columns [s*Ks, (s+1)*Ks)
   // input: float32 x [B, ldx] or Q8 (xq [B, ldx], xd [B, ldx/32]); with `gain`
@@ -96,7 +104,11 @@ struct AttnArgs {
   int* err;             // device error flag (bounded waits)
 };
 
-int launch_attention(const AttnArgs& a, cudaStream_t s);
+// combine = false leaves the splits' partials for the consumer to combine (the
+// W_O GEMV's staging on the weight-streaming path).
+int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine = true);
+// Context splits per (batch row, kv head) the attention uses for these shapes.
+int attention_nsplit(int B, int H, int Hkv, int max_seq);
 // Largest number of context splits any launch over max_seq positions uses.
 int attention_max_splits(int max_seq);
 
