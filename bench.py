@@ -170,9 +170,9 @@ def barrier(world: int):
 
 
 # DRAM bytes (read + write) of one launch of the W1/W3 slice GEMV in the C2 block,
-# from `ncu --set full` of that launch (180.434688 MB read + 3.469056 MB written):
+# from `ncu --set full` of that launch (180.458752 MB read + 3.833088 MB written):
 # the weights once, plus the activations and the SwiGLU output.
-W13_DRAM_BYTES = 180434688 + 3469056
+W13_DRAM_BYTES = 180458752 + 3833088
 
 
 def block_bytes(s):
