@@ -175,14 +175,6 @@ Layout block_layout(const Cfg& c) {
   return L;
 }
 
-int ctas_for(int nseg, int pairs_per_seg) {
-  int target = num_sms() * 3;
-  int per = target / nseg;
-  if (per < 1) per = 1;
-  if (per > pairs_per_seg) per = pairs_per_seg;
-  return per;
-}
-
 }  // namespace
 }  // namespace tp
 

@@ -70,7 +70,6 @@ struct GemvArgs {
   int n_heads, n_kv_heads, max_seq;
   float theta;
   int* err;  // device error flag, set when a bounded wait gives up (nullable)
-  int ctas_per_seg;  // unused by the ring-buffer kernel (one CTA per SM)
 };
 
 // Shared-memory plan of the GEMV (host computes, kernel reads): NC consumer
