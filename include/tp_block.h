@@ -162,6 +162,65 @@ TP_API int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_
 
 TP_API void tp_block_destroy(tp_block* blk);
 
+/* ---------------------------------------------------------------------------
+ * The block spread over processes (one GPU each): the distributed-llama task
+ * list's nodes, where every node computes its slices' partials and the SyncAtt /
+ * SyncFfn2 transfers carry them (quantised when sync_quant is set) to be
+ * dequantised and merged (DequantizeAtt, MergeAtt; DequantizeFfn2, MergeFfn2),
+ * and the aiterms.tw glossary's "how it works": input replicated, column-split
+ * products local, row-split products summed across devices.
+ *
+ * Rank r of `world` holds slices [r*n/world, (r+1)*n/world) of an n-slice block
+ * (requires n % world == 0 and the whole block's rules for n): its weights are
+ * those slices only, packed as for tp_block_create -- wq [H/world*hd, dim], wk and
+ * wv [Hkv/world*hd, dim], wo [dim, H/world*hd] (the columns of its heads), w1 and
+ * w3 [F/world, dim], w2 [dim, F/world], the norm gains whole -- and its KV caches
+ * hold its kv heads only, bf16 [max_batch, Hkv/world, max_seq, hd]. `dims`
+ * describes the whole block. The residual x [batch, dim] is replicated: every
+ * rank passes the same values and all end with the same bits.
+ *
+ * A decode step is three calls of tp_block_rank_step with phase 0, 1, 2 and the
+ * same arguments, with an exchange before phases 1 and 2: the caller gathers the
+ * send buffers of all ranks, in rank order, into every rank's receive buffer (an
+ * all-gather of tp_block_rank_sync_bytes per rank; rank r's bytes at offset r
+ * times that). Phase 0 runs RMSNorm (+Q8), the q/k/v products with RoPE and the
+ * cache write, attention and the W_O partials of this rank's slices, and packs
+ * them into the send buffer; phase 1 merges the received buffer into x (every
+ * slice's partial dequantised and summed in slice order, then added), then runs
+ * RMSNorm (+Q8), W1/W3 with SwiGLU and the W2 partials, and packs them; phase 2
+ * merges again. Each slice's sync format is float32 [batch, dim], or with
+ * sync_quant the int8 codes [batch, dim] followed by the float32 scales
+ * [batch, dim/32]. Because every rank merges all n partials in slice order, the
+ * result equals the single-process block's merge of the same partials. Phases
+ * out of order, or a batch that changes within a step, return TP_EINVAL with
+ * nothing enqueued. 1D partition; batch 1..max_batch (<= 5 on the weight-streaming
+ * kernels, >= 6 on the tensor-core path, as for tp_block_forward). */
+enum { TP_RANK_ATT = 0, TP_RANK_FFN = 1, TP_RANK_OUT = 2 };
+#define TP_BUF_SEND 18 /* tp_block_buffer id: this rank's send buffer */
+#define TP_BUF_RECV 19 /* tp_block_buffer id: the gathered receive buffer (world x send) */
+
+/* Workspace bytes of rank `rank` of `world` (as tp_block_workspace_bytes, plus
+ * the send and receive buffers for max_batch rows). Errors: TP_EINVAL. */
+TP_API int tp_block_rank_workspace_bytes(const tp_dims* dims, int n_slices, int sync_quant,
+                                         int rank, int world, size_t* out_bytes);
+
+/* A handle for rank `rank` of `world` (weights: this rank's slices, see above).
+ * Errors: TP_EINVAL, TP_EALIGN, TP_EWORKSPACE, TP_EARCH, TP_ECUDA. */
+TP_API int tp_block_create_rank(const tp_dims* dims, int n_slices, int sync_quant, int rank,
+                                int world, const tp_block_weights* w, void* workspace,
+                                size_t ws_bytes, tp_block** out);
+
+/* Bytes each rank contributes to an exchange for `batch` rows:
+ * (n/world slices) x the slice format's size. Errors: TP_EINVAL (not a rank
+ * handle, batch out of range). */
+TP_API int tp_block_rank_sync_bytes(const tp_block* blk, int batch, size_t* send_bytes);
+
+/* One phase of a rank's decode step (see above); x, caches and pos as for
+ * tp_block_forward, with this rank's kv heads in the caches. Errors: TP_EINVAL,
+ * TP_EALIGN, TP_ECUDA. tp_block_forward on a rank handle returns TP_EINVAL. */
+TP_API int tp_block_rank_step(tp_block* blk, int phase, float* x, void* k_cache, void* v_cache,
+                              const int32_t* pos, int batch, tp_stream stream);
+
 /* Per-stage timing hook. events: host array of n cudaEvent_t handles created by
  * the caller (timing enabled), or NULL to switch the hook off. While set, each
  * tp_block_forward records events[i] on `stream` just before stage i and

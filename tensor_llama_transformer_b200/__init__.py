@@ -27,6 +27,8 @@ TP_ACT_RELU, TP_ACT_SWIGLU = 0, 1
 TP_F32, TP_BF16 = 0, 1
 TP_MERGE_FAITHFUL, TP_MERGE_FUSED = 0, 1
 BUF_XQ, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H = range(7)
+TP_RANK_ATT, TP_RANK_FFN, TP_RANK_OUT = 0, 1, 2
+TP_BUF_SEND, TP_BUF_RECV = 18, 19
 
 
 class TpError(RuntimeError):
@@ -69,6 +71,13 @@ _sig = {
                                       C.POINTER(tp_block_weights_q8), _P, C.c_size_t,
                                       C.POINTER(_P)]),
     "tp_block_forward": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _P]),
+    "tp_block_rank_workspace_bytes": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int,
+                                                C.c_int, _SZ]),
+    "tp_block_create_rank": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int, C.c_int,
+                                       C.POINTER(tp_block_weights), _P, C.c_size_t,
+                                       C.POINTER(_P)]),
+    "tp_block_rank_sync_bytes": (C.c_int, [_P, C.c_int, _SZ]),
+    "tp_block_rank_step": (C.c_int, [_P, C.c_int, _P, _P, _P, _P, C.c_int, _P]),
     "tp_block_buffer": (C.c_int, [_P, C.c_int, _SZ, _SZ]),
     "tp_block_destroy": (None, [_P]),
     "tp_block_set_events": (C.c_int, [_P, _P, C.c_int]),
@@ -172,6 +181,35 @@ def tp_block_create_q8w(dims, n_slices, partition, sync_quant, weights, workspac
 def tp_block_forward(handle, x, k_cache, v_cache, pos, batch, stream=None):
     _check(_lib.tp_block_forward(handle, _ptr(x), _ptr(k_cache), _ptr(v_cache), _ptr(pos), batch,
                                  _stream(stream)), "tp_block_forward")
+
+
+def tp_block_rank_workspace_bytes(dims, n_slices, sync_quant, rank, world) -> int:
+    out = C.c_size_t()
+    _check(_lib.tp_block_rank_workspace_bytes(C.byref(dims), n_slices, int(sync_quant), rank, world,
+                                              C.byref(out)), "tp_block_rank_workspace_bytes")
+    return out.value
+
+
+def tp_block_create_rank(dims, n_slices, sync_quant, rank, world, weights, workspace,
+                         ws_bytes) -> int:
+    """Handle for rank `rank` of `world` holding slices [rank n/world, (rank+1) n/world);
+    `weights` are that rank's slices (``tensor_parallel.rank_weights``)."""
+    h = C.c_void_p()
+    _check(_lib.tp_block_create_rank(C.byref(dims), n_slices, int(sync_quant), rank, world,
+                                     C.byref(weights), _ptr(workspace), ws_bytes, C.byref(h)),
+           "tp_block_create_rank")
+    return h.value
+
+
+def tp_block_rank_sync_bytes(handle, batch) -> int:
+    out = C.c_size_t()
+    _check(_lib.tp_block_rank_sync_bytes(handle, batch, C.byref(out)), "tp_block_rank_sync_bytes")
+    return out.value
+
+
+def tp_block_rank_step(handle, phase, x, k_cache, v_cache, pos, batch, stream=None):
+    _check(_lib.tp_block_rank_step(handle, phase, _ptr(x), _ptr(k_cache), _ptr(v_cache), _ptr(pos),
+                                   batch, _stream(stream)), "tp_block_rank_step")
 
 
 def tp_block_buffer(handle, which):

@@ -80,8 +80,10 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // ------------------------------------------------------------------ block layout
 enum Buf {
   BUF_XQ = 0, BUF_XD, BUF_XN, BUF_Q, BUF_ATT, BUF_PART, BUF_H, BUF_ERR, BUF_PO, BUF_PML,
-  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_XMID, BUF_COUNT
+  BUF_PA, BUF_PB, BUF_SSQ, BUF_XB, BUF_ATTB, BUF_HB, BUF_PLANE, BUF_XMID, BUF_SEND, BUF_RECV,
+  BUF_COUNT
 };
+static_assert(BUF_SEND == TP_BUF_SEND && BUF_RECV == TP_BUF_RECV, "buffer ids of the C ABI");
 // BUF_ERR (16 bytes): int error word at byte 0; the persistent kernel's two grid
 // barrier counters at bytes 8 and 12.
 
@@ -95,8 +97,9 @@ struct Layout {
 };
 
 struct Cfg {
-  tp_dims d;
+  tp_dims d;  // for a rank block: this rank's share (H, Hkv, ffn_dim divided by world)
   int n, partition, quant, gx, gy, nchunk;
+  int rank, world;  // world 0: the whole block; else this process holds n of n * world slices
 };
 
 void grid2d(int n, int* gx, int* gy) {
@@ -132,6 +135,27 @@ int check_cfg(const tp_dims* d, int n, int partition, int quant, Cfg* c) {
     c->gy = n;
   }
   c->nchunk = attention_max_splits(d->max_seq);
+  c->rank = 0;
+  c->world = 0;
+  return TP_OK;
+}
+
+// A rank's share of an n-slice block spread over `world` processes: slices
+// [rank n/world, (rank+1) n/world) with their q/kv heads and ffn rows, i.e. a
+// block of n/world slices over H/world heads, Hkv/world kv heads and F/world
+// ffn rows; dim and the norms are whole.
+int check_rank_cfg(const tp_dims* d, int n, int quant, int rank, int world, Cfg* c) {
+  if (!d || world < 1 || rank < 0 || rank >= world || n < 1 || n % world != 0) return TP_EINVAL;
+  int rc = check_cfg(d, n, TP_PART_1D, quant, c);  // the whole block's rules
+  if (rc) return rc;
+  tp_dims local = *d;
+  local.n_heads /= world;
+  local.n_kv_heads /= world;
+  local.ffn_dim /= world;
+  rc = check_cfg(&local, n / world, TP_PART_1D, quant, c);
+  if (rc) return rc;
+  c->rank = rank;
+  c->world = world;
   return TP_OK;
 }
 
@@ -156,6 +180,11 @@ Layout block_layout(const Cfg& c) {
   // per-row sums of squares: merge pieces of 512 values, or (persistent kernel) 128
   L.size[BUF_SSQ] = B * (size_t)(c.d.dim / 128) * 4;
   L.size[BUF_XMID] = B * D * 4;  // x + attention branch (persistent kernel)
+  if (c.world > 0) {  // rank block: its slices' sync buffers out, every rank's in
+    const size_t chunk = (size_t)sync_slice_bytes(c.d.max_batch, c.d.dim, c.quant);
+    L.size[BUF_SEND] = (size_t)c.n * chunk;
+    L.size[BUF_RECV] = (size_t)c.n * c.world * chunk;
+  }
   // batched decode (tensor-core path): bf16 operands and the float32 product planes
   if (c.d.max_batch >= kTcMinBatch) {
     const size_t KD = (size_t)c.d.n_kv_heads * c.d.head_dim;
@@ -198,6 +227,8 @@ struct tp_block {
   const float* wd_1;
   const float* wd_3;
   const float* wd_2;
+  int phase_next;   // rank block: the phase tp_block_rank_step expects next
+  int phase_batch;  // rank block: the batch of the step in progress
 };
 
 struct tp_model {
@@ -248,6 +279,24 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
   return e == cudaSuccess ? TP_OK : TP_ECUDA;
 }
 
+// a6 / a10. Whole block: x += the slice partials (planes of `part`), summed in
+// slice order through the sync format. Rank block: the same over the gathered
+// sync buffer, which holds every rank's slices in slice order.
+int merge_step(tp_block* blk, float* x, const float* part, int nseg, int parts, int batch,
+               cudaStream_t s) {
+  const Cfg& c = blk->c;
+  float* ssq = at<float>(blk, BUF_SSQ);
+  if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts);
+  return launch_merge_sync(x, at<uint8_t>(blk, BUF_RECV), c.n * c.world, batch, c.d.dim, c.quant,
+                           ssq, s);
+}
+
+// End of a rank block's phase 0 / 1: this rank's partials into its send buffer.
+int pack_step(tp_block* blk, const float* part, int parts, int batch, cudaStream_t s) {
+  const Cfg& c = blk->c;
+  return launch_sync_pack(part, c.n, parts, batch, c.d.dim, c.quant, at<uint8_t>(blk, BUF_SEND), s);
+}
+
 // Contraction parts for a batched-decode GEMM of `tiles` 128-row output tiles
 // (per existing segment) over K: the persistent GEMM gives each SM ceil(tiles *
 // parts / SMs) tiles of K / parts, and every extra part adds a float32 plane
@@ -275,8 +324,9 @@ int tc_split(int64_t tiles, int64_t K, int64_t rows_total, int batch, int pmax) 
 // The batched form of the block: the same steps, with the slice products on the
 // tcgen05 GEMM (weights = M operand, batch = N) writing float32 planes, small
 // kernels for the norms and epilogues, and the same attention and merges.
+// phase: -1 the whole step; 0 / 1 / 2 a rank block's steps (tp_block_rank_step).
 int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
-                     cudaStream_t s, bool chained) {
+                     cudaStream_t s, bool chained, int phase) {
   const Cfg& c = blk->c;
   const tp_dims& d = c.d;
   const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
@@ -325,99 +375,105 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     return launch_tc_gemm(g, s);
   };
 
-  // a1-a4
-  if ((rc = stage_mark(blk, 0, s))) return rc;
-  if ((rc = norm(blk->w.attn_norm, chained ? at<float>(blk, BUF_SSQ) : nullptr))) return rc;
-  const int qkv_tiles = (QD + 127) / 128 + 2 * ((KD + 127) / 128);
-  const int parts = tc_split(qkv_tiles, D, QD + 2 * KD, batch, kQkvMaxParts);
-  if ((rc = gemm(blk->w.wq, QD, blk->w.wk, KD, blk->w.wv, KD, 3, D, xb, D / parts, parts, plane,
-                 QD + 2 * KD)))
-    return rc;
-  {
-    QkvFinalizeArgs f{};
-    f.plane = plane;
-    f.parts = parts;
-    f.batch = batch;
-    f.qd = QD;
-    f.kd = KD;
-    f.pos = pos;
-    f.theta = d.rope_theta;
-    f.q = at<float>(blk, BUF_Q);
-    f.kc = static_cast<uint16_t*>(kc);
-    f.vc = static_cast<uint16_t*>(vc);
-    f.n_kv_heads = Hkv;
-    f.max_seq = d.max_seq;
-    if ((rc = launch_qkv_finalize(f, s))) return rc;
-  }
-  // a4
-  if ((rc = stage_mark(blk, 1, s))) return rc;
-  {
-    AttnArgs a{};
-    a.q = at<float>(blk, BUF_Q);
-    a.kc = static_cast<const uint16_t*>(kc);
-    a.vc = static_cast<const uint16_t*>(vc);
-    a.pos = pos;
-    a.B = batch;
-    a.H = H;
-    a.Hkv = Hkv;
-    a.max_seq = d.max_seq;
-    a.nchunk = c.nchunk;
-    a.part_o = at<float>(blk, BUF_PO);
-    a.part_ml = at<float>(blk, BUF_PML);
-    a.att = at<float>(blk, BUF_ATT);
-    a.att_bf16 = at<uint16_t>(blk, BUF_ATTB);
-    a.err = err;
-    if ((rc = launch_attention(a, s))) return rc;
-  }
-  // a5: W_O row-split partials (segment s = slice s's head columns)
-  if ((rc = stage_mark(blk, 2, s))) return rc;
-  if ((rc = gemm(blk->w.wo, D, nullptr, 0, nullptr, 0, 1, QD, at<uint16_t>(blk, BUF_ATTB), QD / c.n,
-                 c.n, part, D)))
-    return rc;
-  // a6
-  if ((rc = stage_mark(blk, 3, s))) return rc;
-  if ((rc = launch_merge(x, part, c.n, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
-  // a7-a8
-  if ((rc = stage_mark(blk, 4, s))) return rc;
-  if ((rc = norm(blk->w.ffn_norm, at<float>(blk, BUF_SSQ)))) return rc;
-  float* hbuf = at<float>(blk, BUF_H);
-  uint16_t* hb = at<uint16_t>(blk, BUF_HB);
-  if (c.partition == TP_PART_1D) {
-    const int p13 = tc_split(2 * ((F + 127) / 128), D, 2 * F, batch, kW13MaxParts);
-    if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F)))
-      return rc;
-    if ((rc = launch_swiglu_finalize(plane, p13, F, batch, hbuf, hb, s))) return rc;
-  } else {
-    float* pa = at<float>(blk, BUF_PA);
-    float* pb = at<float>(blk, BUF_PB);
-    if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F))) return rc;
-    if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F))) return rc;
-    FfnMergeArgs m{};
-    m.P1 = pa;
-    m.P3 = pb;
-    m.seg_stride = (int64_t)batch * F;
-    m.nseg = c.gx;
-    m.M = batch;
-    m.N = F;
-    m.quant = c.quant;
-    m.act = ACT_SWIGLU;
-    m.out_f32 = hbuf;
-    m.out_bf16 = hb;
-    m.bf16_split = 1;
-    if ((rc = launch_ffn_merge(m, s))) return rc;
-  }
-  // a9
-  if ((rc = stage_mark(blk, 5, s))) return rc;
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
-  const int p2 = tc_split((int64_t)nseg2 * ((D + 127) / 128), F / nseg2, (int64_t)nseg2 * D, batch,
-                          kW2MaxParts);
-  if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2 / p2, nseg2 * p2, part,
-                 D)))
-    return rc;
+  int p2 = 1;
+  if (phase <= 0) {
+    // a1-a4
+    if ((rc = stage_mark(blk, 0, s))) return rc;
+    if ((rc = norm(blk->w.attn_norm, chained ? at<float>(blk, BUF_SSQ) : nullptr))) return rc;
+    const int qkv_tiles = (QD + 127) / 128 + 2 * ((KD + 127) / 128);
+    const int parts = tc_split(qkv_tiles, D, QD + 2 * KD, batch, kQkvMaxParts);
+    if ((rc = gemm(blk->w.wq, QD, blk->w.wk, KD, blk->w.wv, KD, 3, D, xb, D / parts, parts, plane,
+                   QD + 2 * KD)))
+      return rc;
+    {
+      QkvFinalizeArgs f{};
+      f.plane = plane;
+      f.parts = parts;
+      f.batch = batch;
+      f.qd = QD;
+      f.kd = KD;
+      f.pos = pos;
+      f.theta = d.rope_theta;
+      f.q = at<float>(blk, BUF_Q);
+      f.kc = static_cast<uint16_t*>(kc);
+      f.vc = static_cast<uint16_t*>(vc);
+      f.n_kv_heads = Hkv;
+      f.max_seq = d.max_seq;
+      if ((rc = launch_qkv_finalize(f, s))) return rc;
+    }
+    // a4
+    if ((rc = stage_mark(blk, 1, s))) return rc;
+    {
+      AttnArgs a{};
+      a.q = at<float>(blk, BUF_Q);
+      a.kc = static_cast<const uint16_t*>(kc);
+      a.vc = static_cast<const uint16_t*>(vc);
+      a.pos = pos;
+      a.B = batch;
+      a.H = H;
+      a.Hkv = Hkv;
+      a.max_seq = d.max_seq;
+      a.nchunk = c.nchunk;
+      a.part_o = at<float>(blk, BUF_PO);
+      a.part_ml = at<float>(blk, BUF_PML);
+      a.att = at<float>(blk, BUF_ATT);
+      a.att_bf16 = at<uint16_t>(blk, BUF_ATTB);
+      a.err = err;
+      if ((rc = launch_attention(a, s))) return rc;
+    }
+    // a5: W_O row-split partials (segment s = slice s's head columns)
+    if ((rc = stage_mark(blk, 2, s))) return rc;
+    if ((rc = gemm(blk->w.wo, D, nullptr, 0, nullptr, 0, 1, QD, at<uint16_t>(blk, BUF_ATTB), QD / c.n,
+                   c.n, part, D)))
+      return rc;
+    if (phase == 0) return pack_step(blk, part, 1, batch, s);
+  }
+  if (phase <= 1) {
+    // a6
+    if ((rc = stage_mark(blk, 3, s))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    // a7-a8
+    if ((rc = stage_mark(blk, 4, s))) return rc;
+    if ((rc = norm(blk->w.ffn_norm, at<float>(blk, BUF_SSQ)))) return rc;
+    float* hbuf = at<float>(blk, BUF_H);
+    uint16_t* hb = at<uint16_t>(blk, BUF_HB);
+    if (c.partition == TP_PART_1D) {
+      const int p13 = tc_split(2 * ((F + 127) / 128), D, 2 * F, batch, kW13MaxParts);
+      if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F)))
+        return rc;
+      if ((rc = launch_swiglu_finalize(plane, p13, F, batch, hbuf, hb, s))) return rc;
+    } else {
+      float* pa = at<float>(blk, BUF_PA);
+      float* pb = at<float>(blk, BUF_PB);
+      if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F))) return rc;
+      if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F))) return rc;
+      FfnMergeArgs m{};
+      m.P1 = pa;
+      m.P3 = pb;
+      m.seg_stride = (int64_t)batch * F;
+      m.nseg = c.gx;
+      m.M = batch;
+      m.N = F;
+      m.quant = c.quant;
+      m.act = ACT_SWIGLU;
+      m.out_f32 = hbuf;
+      m.out_bf16 = hb;
+      m.bf16_split = 1;
+      if ((rc = launch_ffn_merge(m, s))) return rc;
+    }
+    // a9
+    if ((rc = stage_mark(blk, 5, s))) return rc;
+    p2 = tc_split((int64_t)nseg2 * ((D + 127) / 128), F / nseg2, (int64_t)nseg2 * D, batch,
+                  kW2MaxParts);
+    if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2 / p2, nseg2 * p2, part,
+                   D)))
+      return rc;
+    if (phase == 1) return pack_step(blk, part, p2, batch, s);
+  }
   // a10
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, at<float>(blk, BUF_SSQ), s, p2)))
-    return rc;
+  if ((rc = merge_step(blk, x, part, nseg2, p2, batch, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -480,11 +536,16 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
 // chained: x was produced by the previous block's final merge of this same
 // launch sequence, which left the row sums of squares in the workspace (inside
 // a model); the final merge here leaves them for the next block.
+// phase: -1 the whole step; 0 / 1 / 2 the three steps of a rank block (a1-a5 and
+// the pack of its W_O partials; the merge of the gathered buffer, a7-a9 and the
+// pack of its W2 partials; the final merge), between which the caller exchanges
+// the sync buffers.
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
-                       cudaStream_t s, bool chained = false) {
+                       cudaStream_t s, bool chained = false, int phase = -1) {
   if (blk->wq8 && batch >= kTcMinBatch) return TP_ENOTSUP;
-  if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained);
-  if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent) {
+  if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained, phase);
+  if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent &&
+      blk->c.world == 0) {
     bool used = false;
     const int rc = block_forward_persistent(blk, x, kc, vc, pos, batch, s, &used);
     if (used || rc) return rc;
@@ -496,167 +557,173 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   int rc;
   float* part = at<float>(blk, BUF_PART);
   float* hbuf = at<float>(blk, BUF_H);
+  const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
 
-  // a1-a4: RMSNorm (+Q8, the buffer every slice reads) fused into the q/k/v slice
-  // products, with RoPE and the cache write in the epilogue
-  if ((rc = stage_mark(blk, 0, s))) return rc;
-  {
-    GemvArgs a{};
-    a.w[0] = static_cast<const uint16_t*>(blk->w.wq);
-    a.w[1] = static_cast<const uint16_t*>(blk->w.wk);
-    a.w[2] = static_cast<const uint16_t*>(blk->w.wv);
-    if (blk->wq8) {
-      a.wd[0] = blk->wd_q;
-      a.wd[1] = blk->wd_k;
-      a.wd[2] = blk->wd_v;
-    }
-    a.rows[0] = QD;
-    a.rows[1] = Hkv * hd;
-    a.rows[2] = Hkv * hd;
-    a.ldw = D;
-    a.Ks = D;
-    a.nseg = 1;
-    set_norm_input(blk, a, x, blk->w.attn_norm);
-    if (chained) {
-      a.ssq = at<float>(blk, BUF_SSQ);
-      a.ssq_parts = merge_ssq_parts(D);
-    }
-    a.nb = batch;
-    a.qout = at<float>(blk, BUF_Q);
-    a.kc = static_cast<uint16_t*>(kc);
-    a.vc = static_cast<uint16_t*>(vc);
-    a.pos = pos;
-    a.n_heads = H;
-    a.n_kv_heads = Hkv;
-    a.max_seq = d.max_seq;
-    a.theta = d.rope_theta;
-    a.err = at<int>(blk, BUF_ERR);
-    if ((rc = launch_gemv(a, EPI_QKV, s))) return rc;
-  }
-  // a4: attention per head slice (context chunks, then their combination)
-  if ((rc = stage_mark(blk, 1, s))) return rc;
-  {
-    AttnArgs a{};
-    a.q = at<float>(blk, BUF_Q);
-    a.kc = static_cast<const uint16_t*>(kc);
-    a.vc = static_cast<const uint16_t*>(vc);
-    a.pos = pos;
-    a.B = batch;
-    a.H = H;
-    a.Hkv = Hkv;
-    a.max_seq = d.max_seq;
-    a.nchunk = c.nchunk;
-    a.part_o = at<float>(blk, BUF_PO);
-    a.part_ml = at<float>(blk, BUF_PML);
-    a.att = at<float>(blk, BUF_ATT);
-    a.err = at<int>(blk, BUF_ERR);
-    if ((rc = launch_attention(a, s, false))) return rc;  // W_O's staging combines the splits
-  }
-  // a5: W_O row-split partials, one plane per slice
-  if ((rc = stage_mark(blk, 2, s))) return rc;
-  {
-    GemvArgs a{};
-    a.w[0] = static_cast<const uint16_t*>(blk->w.wo);
-    if (blk->wq8) a.wd[0] = blk->wd_o;
-    a.rows[0] = D;
-    a.ldw = QD;
-    a.Ks = QD / c.n;
-    a.nseg = c.n;
-    a.att_po = at<float>(blk, BUF_PO);
-    a.att_pml = at<float>(blk, BUF_PML);
-    a.att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq);
-    a.att_out = at<float>(blk, BUF_ATT);
-    a.pos = pos;
-    a.n_heads = H;
-    a.ldx = QD;
-    a.nb = batch;
-    a.out = part;
-    a.out_seg = (int64_t)batch * D;
-    a.ldo = D;
-    a.err = at<int>(blk, BUF_ERR);
-    if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
-  }
-  // a6: sync + dequantise + merge into the residual
-  if ((rc = stage_mark(blk, 3, s))) return rc;
-  if ((rc = launch_merge(x, part, c.n, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
-  // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
-  if ((rc = stage_mark(blk, 4, s))) return rc;
-  if (c.partition == TP_PART_1D) {
-    GemvArgs a{};
-    a.w[0] = static_cast<const uint16_t*>(blk->w.w1);
-    a.w[1] = static_cast<const uint16_t*>(blk->w.w3);
-    if (blk->wq8) {
-      a.wd[0] = blk->wd_1;
-      a.wd[1] = blk->wd_3;
-    }
-    a.rows[0] = F;
-    a.ldw = D;
-    a.Ks = D;
-    a.nseg = 1;
-    set_norm_input(blk, a, x, blk->w.ffn_norm);
-    a.ssq = at<float>(blk, BUF_SSQ);  // written by the merge just above
-    a.ssq_parts = merge_ssq_parts(D);
-    a.nb = batch;
-    a.out = hbuf;
-    a.ldo = F;
-    a.err = at<int>(blk, BUF_ERR);
-    if ((rc = launch_gemv(a, EPI_SWIGLU, s))) return rc;
-  } else {
-    // 2D stage 1: partials over the gx dim-slices for W1 and W3, merged with SwiGLU
-    float* pa = at<float>(blk, BUF_PA);
-    float* pb = at<float>(blk, BUF_PB);
-    for (int m = 0; m < 2; ++m) {
+  if (phase <= 0) {
+    // a1-a4: RMSNorm (+Q8, the buffer every slice reads) fused into the q/k/v slice
+    // products, with RoPE and the cache write in the epilogue
+    if ((rc = stage_mark(blk, 0, s))) return rc;
+    {
       GemvArgs a{};
-      a.w[0] = static_cast<const uint16_t*>(m == 0 ? blk->w.w1 : blk->w.w3);
-      a.rows[0] = F;
+      a.w[0] = static_cast<const uint16_t*>(blk->w.wq);
+      a.w[1] = static_cast<const uint16_t*>(blk->w.wk);
+      a.w[2] = static_cast<const uint16_t*>(blk->w.wv);
+      if (blk->wq8) {
+        a.wd[0] = blk->wd_q;
+        a.wd[1] = blk->wd_k;
+        a.wd[2] = blk->wd_v;
+      }
+      a.rows[0] = QD;
+      a.rows[1] = Hkv * hd;
+      a.rows[2] = Hkv * hd;
       a.ldw = D;
-      a.Ks = D / c.gx;
-      a.nseg = c.gx;
-      set_norm_input(blk, a, x, blk->w.ffn_norm);
-      a.ssq = at<float>(blk, BUF_SSQ);
-      a.ssq_parts = merge_ssq_parts(D);
+      a.Ks = D;
+      a.nseg = 1;
+      set_norm_input(blk, a, x, blk->w.attn_norm);
+      if (chained) {
+        a.ssq = at<float>(blk, BUF_SSQ);
+        a.ssq_parts = merge_ssq_parts(D);
+      }
       a.nb = batch;
-      a.out = m == 0 ? pa : pb;
-      a.out_seg = (int64_t)batch * F;
-      a.ldo = F;
+      a.qout = at<float>(blk, BUF_Q);
+      a.kc = static_cast<uint16_t*>(kc);
+      a.vc = static_cast<uint16_t*>(vc);
+      a.pos = pos;
+      a.n_heads = H;
+      a.n_kv_heads = Hkv;
+      a.max_seq = d.max_seq;
+      a.theta = d.rope_theta;
+      a.err = at<int>(blk, BUF_ERR);
+      if ((rc = launch_gemv(a, EPI_QKV, s))) return rc;
+    }
+    // a4: attention per head slice (context chunks, then their combination)
+    if ((rc = stage_mark(blk, 1, s))) return rc;
+    {
+      AttnArgs a{};
+      a.q = at<float>(blk, BUF_Q);
+      a.kc = static_cast<const uint16_t*>(kc);
+      a.vc = static_cast<const uint16_t*>(vc);
+      a.pos = pos;
+      a.B = batch;
+      a.H = H;
+      a.Hkv = Hkv;
+      a.max_seq = d.max_seq;
+      a.nchunk = c.nchunk;
+      a.part_o = at<float>(blk, BUF_PO);
+      a.part_ml = at<float>(blk, BUF_PML);
+      a.att = at<float>(blk, BUF_ATT);
+      a.err = at<int>(blk, BUF_ERR);
+      if ((rc = launch_attention(a, s, false))) return rc;  // W_O's staging combines the splits
+    }
+    // a5: W_O row-split partials, one plane per slice
+    if ((rc = stage_mark(blk, 2, s))) return rc;
+    {
+      GemvArgs a{};
+      a.w[0] = static_cast<const uint16_t*>(blk->w.wo);
+      if (blk->wq8) a.wd[0] = blk->wd_o;
+      a.rows[0] = D;
+      a.ldw = QD;
+      a.Ks = QD / c.n;
+      a.nseg = c.n;
+      a.att_po = at<float>(blk, BUF_PO);
+      a.att_pml = at<float>(blk, BUF_PML);
+      a.att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq);
+      a.att_out = at<float>(blk, BUF_ATT);
+      a.pos = pos;
+      a.n_heads = H;
+      a.ldx = QD;
+      a.nb = batch;
+      a.out = part;
+      a.out_seg = (int64_t)batch * D;
+      a.ldo = D;
       a.err = at<int>(blk, BUF_ERR);
       if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
-    FfnMergeArgs m{};
-    m.P1 = pa;
-    m.P3 = pb;
-    m.seg_stride = (int64_t)batch * F;
-    m.nseg = c.gx;
-    m.M = batch;
-    m.N = F;
-    m.quant = c.quant;
-    m.act = ACT_SWIGLU;
-    m.out_f32 = hbuf;
-    if ((rc = launch_ffn_merge(m, s))) return rc;
+    if (phase == 0) return pack_step(blk, part, 1, batch, s);
   }
-  // a9: W2 row-split partials
-  if ((rc = stage_mark(blk, 5, s))) return rc;
-  const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
-  {
-    GemvArgs a{};
-    a.w[0] = static_cast<const uint16_t*>(blk->w.w2);
-    if (blk->wq8) a.wd[0] = blk->wd_2;
-    a.rows[0] = D;
-    a.ldw = F;
-    a.Ks = F / nseg2;
-    a.nseg = nseg2;
-    a.x = hbuf;
-    a.ldx = F;
-    a.nb = batch;
-    a.out = part;
-    a.out_seg = (int64_t)batch * D;
-    a.ldo = D;
-    a.err = at<int>(blk, BUF_ERR);
-    if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
+  if (phase <= 1) {
+    // a6: sync + dequantise + merge into the residual
+    if ((rc = stage_mark(blk, 3, s))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
+    if ((rc = stage_mark(blk, 4, s))) return rc;
+    if (c.partition == TP_PART_1D) {
+      GemvArgs a{};
+      a.w[0] = static_cast<const uint16_t*>(blk->w.w1);
+      a.w[1] = static_cast<const uint16_t*>(blk->w.w3);
+      if (blk->wq8) {
+        a.wd[0] = blk->wd_1;
+        a.wd[1] = blk->wd_3;
+      }
+      a.rows[0] = F;
+      a.ldw = D;
+      a.Ks = D;
+      a.nseg = 1;
+      set_norm_input(blk, a, x, blk->w.ffn_norm);
+      a.ssq = at<float>(blk, BUF_SSQ);  // written by the merge just above
+      a.ssq_parts = merge_ssq_parts(D);
+      a.nb = batch;
+      a.out = hbuf;
+      a.ldo = F;
+      a.err = at<int>(blk, BUF_ERR);
+      if ((rc = launch_gemv(a, EPI_SWIGLU, s))) return rc;
+    } else {
+      // 2D stage 1: partials over the gx dim-slices for W1 and W3, merged with SwiGLU
+      float* pa = at<float>(blk, BUF_PA);
+      float* pb = at<float>(blk, BUF_PB);
+      for (int m = 0; m < 2; ++m) {
+        GemvArgs a{};
+        a.w[0] = static_cast<const uint16_t*>(m == 0 ? blk->w.w1 : blk->w.w3);
+        a.rows[0] = F;
+        a.ldw = D;
+        a.Ks = D / c.gx;
+        a.nseg = c.gx;
+        set_norm_input(blk, a, x, blk->w.ffn_norm);
+        a.ssq = at<float>(blk, BUF_SSQ);
+        a.ssq_parts = merge_ssq_parts(D);
+        a.nb = batch;
+        a.out = m == 0 ? pa : pb;
+        a.out_seg = (int64_t)batch * F;
+        a.ldo = F;
+        a.err = at<int>(blk, BUF_ERR);
+        if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
+      }
+      FfnMergeArgs m{};
+      m.P1 = pa;
+      m.P3 = pb;
+      m.seg_stride = (int64_t)batch * F;
+      m.nseg = c.gx;
+      m.M = batch;
+      m.N = F;
+      m.quant = c.quant;
+      m.act = ACT_SWIGLU;
+      m.out_f32 = hbuf;
+      if ((rc = launch_ffn_merge(m, s))) return rc;
+    }
+    // a9: W2 row-split partials
+    if ((rc = stage_mark(blk, 5, s))) return rc;
+    {
+      GemvArgs a{};
+      a.w[0] = static_cast<const uint16_t*>(blk->w.w2);
+      if (blk->wq8) a.wd[0] = blk->wd_2;
+      a.rows[0] = D;
+      a.ldw = F;
+      a.Ks = F / nseg2;
+      a.nseg = nseg2;
+      a.x = hbuf;
+      a.ldx = F;
+      a.nb = batch;
+      a.out = part;
+      a.out_seg = (int64_t)batch * D;
+      a.ldo = D;
+      a.err = at<int>(blk, BUF_ERR);
+      if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
+    }
+    if (phase == 1) return pack_step(blk, part, 1, batch, s);
   }
   // a10: sync + dequantise + merge
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = launch_merge(x, part, nseg2, batch, D, c.quant, at<float>(blk, BUF_SSQ), s))) return rc;
+  if ((rc = merge_step(blk, x, part, nseg2, 1, batch, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -739,8 +806,73 @@ int tp_block_create(const tp_dims* dims, int n_slices, int partition, int sync_q
   b->trace = nullptr;
   b->persistent = persistent_default() ? 1 : 0;
   b->wq8 = false;
+  b->phase_next = 0;
+  b->phase_batch = 0;
   *out = b;
   return TP_OK;
+}
+
+int tp_block_rank_workspace_bytes(const tp_dims* dims, int n_slices, int sync_quant, int rank,
+                                  int world, size_t* out_bytes) {
+  Cfg c;
+  const int rc = check_rank_cfg(dims, n_slices, sync_quant, rank, world, &c);
+  if (rc) return rc;
+  if (!out_bytes) return TP_EINVAL;
+  *out_bytes = block_layout(c).total;
+  return TP_OK;
+}
+
+int tp_block_create_rank(const tp_dims* dims, int n_slices, int sync_quant, int rank, int world,
+                         const tp_block_weights* w, void* workspace, size_t ws_bytes,
+                         tp_block** out) {
+  if (!out) return TP_EINVAL;
+  *out = nullptr;
+  Cfg c;
+  int rc = check_rank_cfg(dims, n_slices, sync_quant, rank, world, &c);
+  if (rc) return rc;
+  if (!weights_present(w)) return TP_EINVAL;
+  if (!weights_aligned(w)) return TP_EALIGN;
+  const Layout L = block_layout(c);
+  if (!workspace || ws_bytes < L.total) return TP_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return TP_EALIGN;
+  rc = device_check();
+  if (rc) return rc;
+  tp_block* b = new (std::nothrow) tp_block;
+  if (!b) return TP_EINVAL;
+  b->c = c;
+  b->L = L;
+  b->w = *w;
+  b->ws = static_cast<uint8_t*>(workspace);
+  b->ws_bytes = ws_bytes;
+  b->events = nullptr;
+  b->bar_ready = false;
+  b->trace = nullptr;
+  b->persistent = 0;
+  b->wq8 = false;
+  b->phase_next = 0;
+  b->phase_batch = 0;
+  *out = b;
+  return TP_OK;
+}
+
+int tp_block_rank_sync_bytes(const tp_block* blk, int batch, size_t* send_bytes) {
+  if (!blk || !send_bytes || blk->c.world == 0) return TP_EINVAL;
+  if (batch < 1 || batch > blk->c.d.max_batch) return TP_EINVAL;
+  *send_bytes = (size_t)blk->c.n * (size_t)sync_slice_bytes(batch, blk->c.d.dim, blk->c.quant);
+  return TP_OK;
+}
+
+int tp_block_rank_step(tp_block* blk, int phase, float* x, void* k_cache, void* v_cache,
+                       const int32_t* pos, int batch, tp_stream stream) {
+  if (!blk || blk->c.world == 0 || !x || !k_cache || !v_cache || !pos) return TP_EINVAL;
+  if (batch < 1 || batch > blk->c.d.max_batch) return TP_EINVAL;
+  if (phase != blk->phase_next || (phase > 0 && batch != blk->phase_batch)) return TP_EINVAL;
+  if (!aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache)) return TP_EALIGN;
+  const int rc =
+      block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream, false, phase);
+  blk->phase_next = rc ? 0 : (phase + 1) % 3;
+  blk->phase_batch = batch;
+  return rc;
 }
 
 int tp_block_create_q8w(const tp_dims* dims, int n_slices, int partition, int sync_quant,
@@ -774,6 +906,7 @@ int tp_block_create_q8w(const tp_dims* dims, int n_slices, int partition, int sy
 int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, const int32_t* pos,
                      int batch, tp_stream stream) {
   if (!blk || !x || !k_cache || !v_cache || !pos) return TP_EINVAL;
+  if (blk->c.world > 0) return TP_EINVAL;  // a rank block runs through tp_block_rank_step
   if (batch < 1 || batch > blk->c.d.max_batch) return TP_EINVAL;
   if (!aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache)) return TP_EALIGN;
   return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream);
@@ -844,6 +977,8 @@ int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition,
   blk.trace = nullptr;
   blk.persistent = persistent_default() ? 1 : 0;
   blk.wq8 = false;
+  blk.phase_next = 0;
+  blk.phase_batch = 0;
   return block_forward_impl(&blk, x, k_cache, v_cache, pos, batch, stream);
 }
 }  // namespace tp

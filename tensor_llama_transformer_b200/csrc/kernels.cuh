@@ -14,6 +14,19 @@ namespace tp {
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts = 1);
 inline int merge_ssq_parts(int dim) { return (dim / 4 + 127) / 128; }
+// One slice's partial in the sync format for B rows: float32 [B, dim], or with Q8
+// the codes int8 [B, dim] followed by the scales float32 [B, dim/32].
+__host__ __device__ inline int64_t sync_slice_bytes(int B, int dim, int quant) {
+  return quant ? (int64_t)B * dim + (int64_t)B * (dim / 32) * 4 : (int64_t)B * dim * 4;
+}
+// Rank side of a block spread over processes: pack the n_local slices' partials
+// (planes as for launch_merge) into their sync format, slice after slice; and
+// merge a gathered buffer of n slices in that format into x (slice order, ssq as
+// launch_merge). dim % 128 == 0.
+int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
+                     uint8_t* out, cudaStream_t s);
+int launch_merge_sync(float* x, const uint8_t* sync, int n, int B, int dim, int quant, float* ssq,
+                      cudaStream_t s);
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s);
 int launch_dequantize(const int8_t* q, const float* d, float* x, int64_t n, cudaStream_t s);
 

@@ -68,6 +68,92 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
   }
 }
 
+// Sync-buffer pack for a rank that holds slices of the block (the send side of
+// distributed-llama's SyncAtt / SyncFfn2): slice s's partial, the sum of its
+// contraction parts, written in the slice's sync format -- float32 [B, dim], or
+// with Q8 the codes int8 [B, dim] followed by the scales float32 [B, dim/32].
+// Grid (pieces of 512 values, B, local slices).
+__global__ void __launch_bounds__(kMergeThreads) k_sync_pack(const float* __restrict__ part,
+                                                             int parts, int B, int dim, int quant,
+                                                             uint8_t* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.y, s = blockIdx.z;
+  const int i4 = blockIdx.x * kMergeThreads + threadIdx.x;
+  const int n4 = dim >> 2;
+  if (blockIdx.x * kMergeThreads + (threadIdx.x & ~31) >= n4) return;  // dim % 128: whole warps
+  float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < parts; ++k) {
+    const float4 v = reinterpret_cast<const float4*>(part + ((size_t)(s * parts + k) * B + b) * dim)[i4];
+    p.x += v.x;
+    p.y += v.y;
+    p.z += v.z;
+    p.w += v.w;
+  }
+  uint8_t* base = out + (size_t)s * sync_slice_bytes(B, dim, quant);
+  if (quant) {
+    float* scales = reinterpret_cast<float*>(base + (size_t)B * dim);
+    const uint32_t codes = q8_quantize4(p, scales + ((size_t)b * dim + 4 * (size_t)i4) / kQ8Block);
+    reinterpret_cast<uint32_t*>(base)[(size_t)b * n4 + i4] = codes;
+  } else {
+    reinterpret_cast<float4*>(base)[(size_t)b * n4 + i4] = p;
+  }
+}
+
+// The receive side: x[b] += sum_{s<n} deq(slice s of the gathered buffer), in
+// slice order, with the same per-piece sums of squares as k_merge. Dequantising a
+// packed slice gives the same bits as k_merge's in-place round trip, so a block
+// whose slices are spread over ranks merges exactly as the whole block does.
+__global__ void __launch_bounds__(kMergeThreads) k_merge_sync(float* __restrict__ x,
+                                                              const uint8_t* __restrict__ sync,
+                                                              int n, int B, int dim, int quant,
+                                                              float* __restrict__ ssq) {
+  __shared__ float red[kMergeThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.y;
+  const int i4 = blockIdx.x * kMergeThreads + threadIdx.x;
+  const int n4 = dim >> 2;
+  const bool in = i4 < n4;
+  const size_t chunk = (size_t)sync_slice_bytes(B, dim, quant);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n && in; ++s) {
+    const uint8_t* base = sync + (size_t)s * chunk;
+    float4 p;
+    if (quant) {
+      const float d = reinterpret_cast<const float*>(base + (size_t)B * dim)[((size_t)b * dim + 4 * (size_t)i4) / kQ8Block];
+      p = q8_unpack4(reinterpret_cast<const uint32_t*>(base)[(size_t)b * n4 + i4], d);
+    } else {
+      p = reinterpret_cast<const float4*>(base)[(size_t)b * n4 + i4];
+    }
+    acc.x += p.x;
+    acc.y += p.y;
+    acc.z += p.z;
+    acc.w += p.w;
+  }
+  float sq = 0.f;
+  if (in) {
+    float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim);
+    float4 v = xr[i4];
+    v.x += acc.x;
+    v.y += acc.y;
+    v.z += acc.z;
+    v.w += acc.w;
+    xr[i4] = v;
+    sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (ssq) {
+    sq = warp_sum(sq);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.f;
+      for (int w = 0; w < kMergeThreads / 32; ++w) t += red[w];
+      ssq[(size_t)b * gridDim.x + blockIdx.x] = t;
+    }
+  }
+}
+
 __global__ void k_quantize(const float* __restrict__ x, int8_t* __restrict__ q,
                            float* __restrict__ d, int64_t n) {
   const int64_t n4 = n >> 2;
@@ -97,6 +183,18 @@ int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, 
                  cudaStream_t s, int parts) {
   const dim3 grid(merge_ssq_parts(dim), B);
   return launch_pdl(k_merge, grid, dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim, quant, ssq);
+}
+
+int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
+                     uint8_t* out, cudaStream_t s) {
+  const dim3 grid(merge_ssq_parts(dim), B, n_local);
+  return launch_pdl(k_sync_pack, grid, dim3(kMergeThreads), 0, s, part, parts, B, dim, quant, out);
+}
+
+int launch_merge_sync(float* x, const uint8_t* sync, int n, int B, int dim, int quant, float* ssq,
+                      cudaStream_t s) {
+  const dim3 grid(merge_ssq_parts(dim), B);
+  return launch_pdl(k_merge_sync, grid, dim3(kMergeThreads), 0, s, x, sync, n, B, dim, quant, ssq);
 }
 
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s) {

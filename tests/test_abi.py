@@ -117,3 +117,28 @@ def test_quantize_rejects_bad_sizes(tpb):
         tpb.tp_quantize_q8(16, 16, 16, 33, stream=0)
     assert e.value.status == tpb.TP_EINVAL
     tpb.tp_quantize_q8(16, 16, 16, 0, stream=0)  # empty input: nothing to do
+
+
+def test_rank_block_sizes_and_validation(tpb):
+    """A block spread over ranks: each rank's workspace covers its share of the
+    heads and ffn rows plus the send / receive buffers; bad rank layouts are
+    rejected before any CUDA call."""
+    d = _dims(tpb)
+    whole = tpb.tp_block_workspace_bytes(d, 8, tpb.TP_PART_1D, 1)
+    sizes = [tpb.tp_block_rank_workspace_bytes(d, 8, 1, r, 4) for r in range(4)]
+    assert len(set(sizes)) == 1 and 0 < sizes[0] < whole and sizes[0] % 256 == 0
+    assert tpb.tp_block_rank_workspace_bytes(d, 8, 0, 0, 4) > sizes[0]  # float32 sync buffers
+    for n, rank, world in ((8, 4, 4), (8, -1, 4), (8, 0, 0), (6, 0, 4), (4, 0, 8)):
+        with pytest.raises(tpb.TpError) as e:
+            tpb.tp_block_rank_workspace_bytes(d, n, 1, rank, world)
+        assert e.value.status == tpb.TP_EINVAL
+    w = tpb.make_weights(*([16] * 9))
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_block_create_rank(d, 8, 1, 0, 4, w, None, 0)
+    assert e.value.status == tpb.TP_EWORKSPACE
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_block_rank_step(None, 0, 16, 16, 16, 16, 1, stream=0)
+    assert e.value.status == tpb.TP_EINVAL
+    with pytest.raises(tpb.TpError) as e:
+        tpb.tp_block_rank_sync_bytes(None, 1)
+    assert e.value.status == tpb.TP_EINVAL
