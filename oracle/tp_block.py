@@ -195,26 +195,31 @@ def rope(v: np.ndarray, pos: np.ndarray, n_heads: int, head_dim: int, theta: flo
 
 
 def attention_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, pos: np.ndarray,
-                     heads: range, n_heads: int, n_kv_heads: int, head_dim: int) -> np.ndarray:
-    """Causal softmax attention of one new token per row over cache positions ``0..pos``.
+                     heads: range, n_heads: int, n_kv_heads: int, head_dim: int,
+                     seq=None) -> np.ndarray:
+    """Causal softmax attention of one token per row over cache positions ``0..pos``.
 
     [DL] llamaMultiheadAtt: each slice computes "a part of multi-head attention
     locally" for its heads; [TT] distinguishes GQA from MHA. For query head h
     the key/value head is ``h // (n_heads // n_kv_heads)``.
         s_t = q_h . k_t / sqrt(head_dim),  p = softmax(s),  o_h = sum_t p_t v_t
     ``q`` is ``[B, n_heads*head_dim]`` (already rotated); caches are float64
-    ``[B, n_kv_heads, T, head_dim]``. Returns ``[B, len(heads)*head_dim]``.
+    ``[S, n_kv_heads, T, head_dim]`` and row b reads sequence ``seq[b]`` (default
+    b). Rows of one sequence at consecutive positions are a prefill chunk: each
+    row attends to its own position and the ones before it, i.e. causal
+    attention. Returns ``[B, len(heads)*head_dim]``.
     """
     group = n_heads // n_kv_heads
     B = q.shape[0]
     out = np.zeros((B, len(heads) * head_dim), dtype=np.float64)
     for b in range(B):
         P = int(pos[b]) + 1
+        sq = b if seq is None else int(seq[b])
         for j, h in enumerate(heads):
             kv = h // group
             qh = q[b, h * head_dim:(h + 1) * head_dim]
-            K = k_cache[b, kv, :P, :]
-            V = v_cache[b, kv, :P, :]
+            K = k_cache[sq, kv, :P, :]
+            V = v_cache[sq, kv, :P, :]
             s = K @ qh / math.sqrt(head_dim)
             s = s - np.max(s)
             p = np.exp(s)
@@ -323,7 +328,7 @@ def q8_weights(w_bits: np.ndarray):
 
 
 def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid=None,
-                  trace: dict | None = None, weights_q8: bool = False):
+                  trace: dict | None = None, weights_q8: bool = False, seq=None):
     """One decode step of one decoder block, partitioned into ``n_slices`` slices.
 
     Follows the [DL] root-node task order for one layer:
@@ -354,6 +359,14 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
     output before W_O and its SwiGLU output before W2. The partials cross the
     sync as with ``sync_quant``.
 
+    ``seq`` (optional, ``[B]``): the cache sequence of each row (default row b
+    uses sequence b). Several rows of one sequence at distinct positions form a
+    prefill chunk (Pope et al. demo 2's prefill, many tokens per step): every
+    row's k/v are written to the cache before any row's attention, so row b
+    attends to positions ``0..pos[b]`` of its sequence, including the rows of
+    this step below it. Reading taken (the pages define no prefill step): a
+    prefill chunk computes exactly what decoding its tokens one at a time does.
+
     ``inp`` is a ``synth.BlockInputs``. Returns ``(x_out float64 [B, dim],
     k_row uint16 [B, Hkv, hd], v_row uint16 [B, Hkv, hd])``: the new block
     output and the bf16 k/v rows written at ``pos`` (the caches are not modified).
@@ -365,6 +378,7 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
     x = np.asarray(inp.x, dtype=np.float64)
     B = x.shape[0]
     pos = np.asarray(inp.pos)
+    sq = np.arange(B) if seq is None else np.asarray(seq)
     if weights_q8:
         assert partition == 1 and sync_quant
 
@@ -405,8 +419,8 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
                 vr = round_to_bf16(v_s[b, j * hd:(j + 1) * hd])
                 k_new[b, kv0 + j] = kr
                 v_new[b, kv0 + j] = vr
-                kc[b, kv0 + j, pos[b], :] = bf16_to_f64(kr)
-                vc[b, kv0 + j, pos[b], :] = bf16_to_f64(vr)
+                kc[sq[b], kv0 + j, pos[b], :] = bf16_to_f64(kr)
+                vc[sq[b], kv0 + j, pos[b], :] = bf16_to_f64(vr)
     q_rot = rope(q_all, pos, H, hd, s_.rope_theta)
 
     # a4-a6
@@ -414,7 +428,7 @@ def block_forward(inp, n_slices: int, sync_quant: bool, partition: int = 1, grid
     att_all = np.zeros((B, H * hd))
     for s in range(n):
         heads = range(s * (H // n), (s + 1) * (H // n))
-        att_s = attention_decode(q_rot, kc, vc, pos, heads, H, Hkv, hd)
+        att_s = attention_decode(q_rot, kc, vc, pos, heads, H, Hkv, hd, seq=sq)
         cols = slice_range(H * hd, n, s)
         att_all[:, cols] = att_s
         if weights_q8:

@@ -268,6 +268,24 @@ def block_inputs(seed: int, s: BlockShape, layer: int = 0, batch: int | None = N
         pos=np.full(B, s.pos, dtype=np.int32), **w)
 
 
+def chunk_inputs(seed: int, s: BlockShape, pos, seq, n_seq: int | None = None,
+                 layer: int = 0) -> BlockInputs:
+    """Rows of one or more sequences in one step (a prefill chunk, or decode rows of
+    several sequences mixed with one): row b is a token of sequence ``seq[b]`` at
+    position ``pos[b]``. The caches hold ``n_seq`` sequences (default max(seq) + 1),
+    each with positions < ``s.pos`` filled; ``extra["seq"]`` holds ``seq``."""
+    seq = np.asarray(seq, dtype=np.int32)
+    pos = np.asarray(pos, dtype=np.int32)
+    S = int(seq.max()) + 1 if n_seq is None else n_seq
+    w = block_weights(seed, s, layer)
+    k = np.stack([kv_row(seed, s, "k", q, layer) for q in range(S)])
+    v = np.stack([kv_row(seed, s, "v", q, layer) for q in range(S)])
+    ones = np.ones(s.dim, dtype=np.float32)
+    return BlockInputs(
+        shape=s, x=normal_f32(seed, f"L{layer}.chunk.x", (len(pos), s.dim)), attn_norm=ones.copy(),
+        ffn_norm=ones.copy(), k_cache=k, v_cache=v, pos=pos.copy(), extra={"seq": seq.copy()}, **w)
+
+
 def ffn_inputs(seed: int, s: FfnShape, rows: np.ndarray | None = None) -> dict:
     """X, W1, W2 (and W3 for SwiGLU). ``rows`` restricts X to those token rows."""
     gen = normal_f32 if s.dtype == "f32" else normal_bf16

@@ -36,12 +36,15 @@ class DeviceBlock:
         self.ffn_norm = f32_tensor(inp.ffn_norm, device)
         for k in ("wq", "wk", "wv", "wo", "w1", "w3", "w2"):
             setattr(self, k, bf16_tensor(getattr(inp, k), device))
-        shape = (mb, s.n_kv_heads, s.max_seq, s.head_dim)
+        S = inp.k_cache.shape[0]  # cache sequences (one per row unless rows share them)
+        shape = (max(mb, S), s.n_kv_heads, s.max_seq, s.head_dim)
         self.k_cache = torch.zeros(shape, dtype=torch.bfloat16, device=device)
         self.v_cache = torch.zeros(shape, dtype=torch.bfloat16, device=device)
-        self.k_cache[:B] = bf16_tensor(inp.k_cache, device)
-        self.v_cache[:B] = bf16_tensor(inp.v_cache, device)
+        self.k_cache[:S] = bf16_tensor(inp.k_cache, device)
+        self.v_cache[:S] = bf16_tensor(inp.v_cache, device)
         self.pos = i32_tensor(inp.pos, device)
+        seq = inp.extra.get("seq") if getattr(inp, "extra", None) else None
+        self.seq = i32_tensor(seq, device) if seq is not None else None
 
     def weights(self):
         return (self.attn_norm, self.wq, self.wk, self.wv, self.wo, self.ffn_norm, self.w1,

@@ -2,7 +2,8 @@
 Inference" (CS349E lecture 4 script ``03_pope_partitioning.py``).
 
 Bandwidth-only estimates for choosing how to split a transformer across chips:
-the FFN's communication under 1D and 2D weight-stationary layouts, the
+the FFN's communication under 1D and 2D weight-stationary layouts and under the
+weight-gathered layout used for prefill (demo 2), the
 per-chip weight-read and compute times that communication competes with, the
 longest context a KV-cache budget holds under the ways of splitting multi-query
 attention, and a roofline lower bound on decode latency. Times follow the
@@ -64,6 +65,27 @@ def ffn_comm_2d(tokens: int, E: int, n_chips: int, link_bw: float,
     8 * tokens * E / sqrt(n) elements per layer, which equals the 1D traffic at
     n = 16 (sqrt(n) = 4)."""
     return 8.0 * tokens * E * dtype_bytes / (math.sqrt(n_chips) * link_bw)
+
+
+def ffn_comm_gathered(tokens: int, E: int, F: int, n_chips: int, link_bw: float,
+                      dtype_bytes: int = BF16) -> tuple[float, float]:
+    """Weight-gathered FFN (Pope et al., the prefill layout of demo 2): the weights
+    are all-gathered over N of the n chips and the activations exchanged over the
+    rest, 2 * tokens * E / N + 2 * N * E * F / n elements per layer, least at
+    N = sqrt(tokens * n / F). Reading taken: this form, which the page does not
+    print but whose statements it meets -- traffic growing as sqrt(tokens), equal
+    to the 2D weight-stationary traffic at tokens = F / 4, and the optimal N the
+    page states. Returns (seconds, N at the optimum, not rounded)."""
+    N = math.sqrt(tokens * n_chips / F)
+    elems = 2.0 * tokens * E / N + 2.0 * N * E * F / n_chips
+    return elems * dtype_bytes / link_bw, N
+
+
+def ffn_layout(tokens: int, E: int, F: int, n_chips: int, link_bw: float) -> str:
+    """'gathered' when moving weights is cheaper than moving activations
+    (prefill-sized token counts), else 'stationary' (2D weight-stationary)."""
+    t_g, _ = ffn_comm_gathered(tokens, E, F, n_chips, link_bw)
+    return "gathered" if t_g < ffn_comm_2d(tokens, E, n_chips, link_bw) else "stationary"
 
 
 def ffn_weight_read(E: int, F: int, layers: int, n_chips: int, mem_bw: float,

@@ -75,3 +75,37 @@ def test_weights_dominate_small_batch_decode():
     """Demo 4's reading: at small batch the weight read is the largest term of the bound."""
     b = pc.decode_bound(M, CHIP, 64, 64, 2048, weight_bytes=2)
     assert b.weights > max(b.kv, b.compute, b.comm)
+
+
+# Demo 2 (the paper's Figure 3 setting): one FFN layer, E 16384, F 65536, 64 chips.
+E2, F2 = 16384, 65536
+
+
+def test_demo2_crossover_at_f_over_4():
+    """Weight-stationary and weight-gathered traffic are equal at BL = F / 4 = 16,384
+    tokens; fewer tokens favour moving activations, more favour moving weights."""
+    bl = F2 // 4
+    t_g, N = pc.ffn_comm_gathered(bl, E2, F2, 64, CHIP.link_bw)
+    assert t_g == pytest.approx(pc.ffn_comm_2d(bl, E2, 64, CHIP.link_bw), rel=1e-12)
+    assert N == pytest.approx(4.0)  # sqrt(BL n / F)
+    assert pc.ffn_layout(2048, E2, F2, 64, CHIP.link_bw) == "stationary"
+    assert pc.ffn_layout(65536, E2, F2, 64, CHIP.link_bw) == "gathered"
+
+
+def test_demo2_traffic_scaling():
+    """Stationary traffic grows as BL, gathered as sqrt(BL)."""
+    a = pc.ffn_comm_gathered(65536, E2, F2, 64, CHIP.link_bw)[0]
+    b = pc.ffn_comm_gathered(262144, E2, F2, 64, CHIP.link_bw)[0]
+    assert b / a == pytest.approx(2.0, rel=1e-12)
+    assert pc.ffn_comm_2d(262144, E2, 64, CHIP.link_bw) / pc.ffn_comm_2d(
+        65536, E2, 64, CHIP.link_bw) == pytest.approx(4.0, rel=1e-12)
+
+
+def test_demo2_compute_share_last_row():
+    """Demo 2's last row (1,048,576 tokens): compute is 94 % of compute + the cheaper
+    communication (the page's printed observation)."""
+    bl = 1048576
+    comp = pc.ffn_compute(bl, E2, F2, 1, 64, CHIP.peak_flops)
+    comm = min(pc.ffn_comm_gathered(bl, E2, F2, 64, CHIP.link_bw)[0],
+               pc.ffn_comm_2d(bl, E2, 64, CHIP.link_bw))
+    assert round(comp / (comp + comm) * 100) == 94
