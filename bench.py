@@ -444,6 +444,46 @@ def bench_c4(args):
                         "context 4096, n=8, float32 sync buffers"}
 
 
+def bench_c2_prefill(args):
+    """A 64-token prefill chunk of one sequence through the C2 block (Llama-2-7B
+    shapes, n = 4, Q8 sync) after a 960-token prefix: tp_block_forward_seq, the
+    slice products on the tensor cores with the 64 tokens as the GEMMs' N."""
+    import torch
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+
+    s = synth.C2
+    L, p0 = 64, 960
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1011)
+    D, F, H, Hkv, hd = s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim
+    w = [torch.ones(D, device="cuda"), _randn_bf16(torch, gen, (H * hd, D), s.w_std),
+         _randn_bf16(torch, gen, (Hkv * hd, D), s.w_std), _randn_bf16(torch, gen, (Hkv * hd, D), s.w_std),
+         _randn_bf16(torch, gen, (D, H * hd), s.w_std), torch.ones(D, device="cuda"),
+         _randn_bf16(torch, gen, (F, D), s.w_std), _randn_bf16(torch, gen, (F, D), s.w_std),
+         _randn_bf16(torch, gen, (D, F), s.w_std)]
+    kc = _randn_bf16(torch, gen, (1, Hkv, s.max_seq, hd), 1.0)
+    vc = _randn_bf16(torch, gen, (1, Hkv, s.max_seq, hd), 1.0)
+    x = torch.randn((L, D), generator=gen, device="cuda")
+    pos = torch.arange(p0, p0 + L, dtype=torch.int32, device="cuda")
+    seq = torch.zeros(L, dtype=torch.int32, device="cuda")
+    dims = tpb.make_dims(D, H, Hkv, hd, F, s.vocab, L, s.max_seq, s.norm_eps, s.rope_theta)
+    nb = tpb.tp_block_workspace_bytes(dims, s.n_slices, 1, 1)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    h = tpb.tp_block_create(dims, s.n_slices, 1, 1, tpb.make_weights(*w), ws, nb)
+    ms = _time_graph(torch, lambda: tpb.tp_block_forward_seq(h, x, kc, vc, pos, seq, 1, L), 10, 5)
+    tpb.tp_block_destroy(h)
+    wb, _ = block_bytes(s)
+    kvb = 2 * Hkv * (p0 + L) * hd * 2  # the sequence's cache, read once from HBM
+    hbm, _, _, kind = peaks()
+    gbs = (wb + kvb) / (ms / 1e3) / 1e9
+    return {"us_per_chunk": ms * 1e3, "tokens_per_s": L / (ms / 1e3), "hbm_gbs": gbs,
+            "frac": gbs / hbm, "bytes_per_chunk": wb + kvb,
+            "workload": "C2 block (Llama-2-7B shapes, n=4, Q8 sync), one sequence: a 64-token "
+                        "prefill chunk at positions 960..1023"}
+
+
 def bench_c2_persistent(args):
     """The C2 block (Llama-2-7B shapes, n = 4, Q8 sync, KV 1024, batch 1) as one persistent
     kernel per step (tp_block_set_persistent), for comparison with the headline's
@@ -690,6 +730,11 @@ def main(argv=None):
             extra["c2_block_int8_weights"] = bench_c2_q8w(args)
         except Exception as e:  # reported, not fatal
             extra["c2_block_int8_weights"] = {"error": str(e)[:200]}
+        torch.cuda.empty_cache()
+        try:
+            extra["c2_prefill_chunk64"] = bench_c2_prefill(args)
+        except Exception as e:  # reported, not fatal
+            extra["c2_prefill_chunk64"] = {"error": str(e)[:200]}
         torch.cuda.empty_cache()
         extra["c4_block"] = bench_c4(args)
         torch.cuda.empty_cache()

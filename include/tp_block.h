@@ -153,6 +153,22 @@ TP_API int tp_block_create_q8w(const tp_dims* dims, int n_slices, int partition,
 TP_API int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, const int32_t* pos,
                      int batch, tp_stream stream);
 
+/* tp_block_forward for rows that need not own a cache sequence each: row b is a
+ * token of sequence seq[b] (device int32 [batch], 0 <= seq[b] < n_seq) at
+ * position pos[b], and the caches are bf16 [n_seq, Hkv, max_seq, hd]. Rows of one
+ * sequence at consecutive positions are a prefill chunk (Pope et al. demo 2: many
+ * tokens of a sequence per step, the regime its weight-gathered layout is for);
+ * rows of different sequences mix decode and prefill in one step. Every row's k
+ * and v are written before any row's attention runs, so row b attends to
+ * positions 0..pos[b] of its sequence including the rows of this step below it:
+ * a chunk gives what decoding its tokens one at a time gives. Rows sharing a
+ * sequence must have distinct positions (not checked on device). Up to
+ * max_batch rows per call (longer prompts run as successive chunks).
+ * Errors: TP_EINVAL (also for a rank handle), TP_EALIGN, TP_ECUDA, TP_ENOTSUP. */
+TP_API int tp_block_forward_seq(tp_block* blk, float* x, void* k_cache, void* v_cache,
+                                const int32_t* pos, const int32_t* seq, int n_seq, int batch,
+                                tp_stream stream);
+
 /* Offsets (bytes from the workspace base) and sizes of intermediate buffers,
  * for inspection by tests after a forward. which: 0 xnorm int8 codes [B,dim],
  * 1 xnorm scales float32 [B,dim/32], 2 xnorm float32 [B,dim], 3 q (rotated)
@@ -333,6 +349,12 @@ TP_API int tp_model_create(const tp_dims* dims, int n_layers, int n_slices, int 
 
 /* tokens device int32 [batch] in [0, vocab); caches bf16
  * [n_layers, max_batch, Hkv, max_seq, hd]; logits float32 [batch, vocab] written. */
+/* tp_model_forward with rows mapped to cache sequences (see tp_block_forward_seq):
+ * caches bf16 [n_layers, n_seq, Hkv, max_seq, hd]; logits of every row written. */
+TP_API int tp_model_forward_seq(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
+                                const int32_t* pos, const int32_t* seq, int n_seq, int batch,
+                                float* logits, tp_stream stream);
+
 TP_API int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
                      const int32_t* pos, int batch, float* logits, tp_stream stream);
 

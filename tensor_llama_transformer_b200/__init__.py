@@ -71,6 +71,8 @@ _sig = {
                                       C.POINTER(tp_block_weights_q8), _P, C.c_size_t,
                                       C.POINTER(_P)]),
     "tp_block_forward": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _P]),
+    "tp_block_forward_seq": (C.c_int, [_P, _P, _P, _P, _P, _P, C.c_int, C.c_int, _P]),
+    "tp_model_forward_seq": (C.c_int, [_P, _P, _P, _P, _P, _P, C.c_int, C.c_int, _P, _P]),
     "tp_block_rank_workspace_bytes": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int,
                                                 C.c_int, _SZ]),
     "tp_block_create_rank": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int, C.c_int,
@@ -181,6 +183,20 @@ def tp_block_create_q8w(dims, n_slices, partition, sync_quant, weights, workspac
 def tp_block_forward(handle, x, k_cache, v_cache, pos, batch, stream=None):
     _check(_lib.tp_block_forward(handle, _ptr(x), _ptr(k_cache), _ptr(v_cache), _ptr(pos), batch,
                                  _stream(stream)), "tp_block_forward")
+
+
+def tp_block_forward_seq(handle, x, k_cache, v_cache, pos, seq, n_seq, batch, stream=None):
+    """Rows mapped to cache sequences (seq [batch] int32): prefill chunks, mixed batches."""
+    _check(_lib.tp_block_forward_seq(handle, _ptr(x), _ptr(k_cache), _ptr(v_cache), _ptr(pos),
+                                     _ptr(seq), n_seq, batch, _stream(stream)),
+           "tp_block_forward_seq")
+
+
+def tp_model_forward_seq(handle, tokens, k_cache, v_cache, pos, seq, n_seq, batch, logits,
+                         stream=None):
+    _check(_lib.tp_model_forward_seq(handle, _ptr(tokens), _ptr(k_cache), _ptr(v_cache), _ptr(pos),
+                                     _ptr(seq), n_seq, batch, _ptr(logits), _stream(stream)),
+           "tp_model_forward_seq")
 
 
 def tp_block_rank_workspace_bytes(dims, n_slices, sync_quant, rank, world) -> int:

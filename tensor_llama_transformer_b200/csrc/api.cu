@@ -326,7 +326,7 @@ int tc_split(int64_t tiles, int64_t K, int64_t rows_total, int batch, int pmax) 
 // kernels for the norms and epilogues, and the same attention and merges.
 // phase: -1 the whole step; 0 / 1 / 2 a rank block's steps (tp_block_rank_step).
 int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
-                     cudaStream_t s, bool chained, int phase) {
+                     cudaStream_t s, bool chained, int phase, const int32_t* seq, int nseq) {
   const Cfg& c = blk->c;
   const tp_dims& d = c.d;
   const int D = d.dim, F = d.ffn_dim, H = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim;
@@ -394,6 +394,7 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
       f.qd = QD;
       f.kd = KD;
       f.pos = pos;
+      f.seq = seq;
       f.theta = d.rope_theta;
       f.q = at<float>(blk, BUF_Q);
       f.kc = static_cast<uint16_t*>(kc);
@@ -410,6 +411,8 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
       a.kc = static_cast<const uint16_t*>(kc);
       a.vc = static_cast<const uint16_t*>(vc);
       a.pos = pos;
+      a.seq = seq;
+      a.nseq = nseq;
       a.B = batch;
       a.H = H;
       a.Hkv = Hkv;
@@ -539,13 +542,16 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
 // phase: -1 the whole step; 0 / 1 / 2 the three steps of a rank block (a1-a5 and
 // the pack of its W_O partials; the merge of the gathered buffer, a7-a9 and the
 // pack of its W2 partials; the final merge), between which the caller exchanges
-// the sync buffers.
+// the sync buffers. seq (nullable): the cache sequence of each row, in caches of
+// nseq sequences (rows of one sequence at consecutive positions: a prefill chunk).
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
-                       cudaStream_t s, bool chained = false, int phase = -1) {
+                       cudaStream_t s, bool chained = false, int phase = -1,
+                       const int32_t* seq = nullptr, int nseq = 0) {
   if (blk->wq8 && batch >= kTcMinBatch) return TP_ENOTSUP;
-  if (batch >= kTcMinBatch) return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained, phase);
+  if (batch >= kTcMinBatch)
+    return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained, phase, seq, nseq);
   if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent &&
-      blk->c.world == 0) {
+      blk->c.world == 0 && !seq) {
     bool used = false;
     const int rc = block_forward_persistent(blk, x, kc, vc, pos, batch, s, &used);
     if (used || rc) return rc;
@@ -589,6 +595,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.kc = static_cast<uint16_t*>(kc);
       a.vc = static_cast<uint16_t*>(vc);
       a.pos = pos;
+      a.seq = seq;
       a.n_heads = H;
       a.n_kv_heads = Hkv;
       a.max_seq = d.max_seq;
@@ -604,6 +611,8 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.kc = static_cast<const uint16_t*>(kc);
       a.vc = static_cast<const uint16_t*>(vc);
       a.pos = pos;
+      a.seq = seq;
+      a.nseq = nseq;
       a.B = batch;
       a.H = H;
       a.Hkv = Hkv;
@@ -912,6 +921,16 @@ int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, cons
   return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream);
 }
 
+int tp_block_forward_seq(tp_block* blk, float* x, void* k_cache, void* v_cache, const int32_t* pos,
+                         const int32_t* seq, int n_seq, int batch, tp_stream stream) {
+  if (!blk || !x || !k_cache || !v_cache || !pos || !seq || blk->c.world > 0) return TP_EINVAL;
+  if (batch < 1 || batch > blk->c.d.max_batch || n_seq < 1) return TP_EINVAL;
+  if ((int64_t)n_seq * blk->c.d.n_kv_heads * blk->c.d.max_seq > INT32_MAX) return TP_EINVAL;
+  if (!aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache)) return TP_EALIGN;
+  return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream, false, -1,
+                            seq, n_seq);
+}
+
 int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* bytes) {
   if (!blk || which < 0 || which >= BUF_COUNT) return TP_EINVAL;
   if (offset) *offset = blk->L.off[which];
@@ -1042,22 +1061,23 @@ int tp_model_create(const tp_dims* dims, int n_layers, int n_slices, int partiti
   return TP_OK;
 }
 
-int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
-                     const int32_t* pos, int batch, float* logits, tp_stream stream) {
-  if (!m || !tokens || !k_cache || !v_cache || !pos || !logits) return TP_EINVAL;
-  if (batch < 1 || batch > m->d.max_batch) return TP_EINVAL;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits)) return TP_EALIGN;
-  cudaStream_t s = (cudaStream_t)stream;
+}  // extern "C"
+
+namespace tp_api {
+// The model step; seq (nullable) maps rows to the caches' nseq sequences.
+int model_forward_impl(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
+                       const int32_t* pos, const int32_t* seq, int nseq, int batch, float* logits,
+                       cudaStream_t s) {
   const tp_dims& d = m->d;
   int rc0 = launch_pdl(k_embed, dim3(batch), dim3(256), 0, s,
                        static_cast<const uint16_t*>(m->embed), tokens, (int)d.dim, m->x);
   if (rc0) return rc0;
   const size_t layer_elems =
-      (size_t)d.max_batch * d.n_kv_heads * (size_t)d.max_seq * d.head_dim;
+      (size_t)(seq ? nseq : d.max_batch) * d.n_kv_heads * (size_t)d.max_seq * d.head_dim;
   for (int l = 0; l < m->n_layers; ++l) {
     uint16_t* kc = static_cast<uint16_t*>(k_cache) + (size_t)l * layer_elems;
     uint16_t* vc = static_cast<uint16_t*>(v_cache) + (size_t)l * layer_elems;
-    int rc = block_forward_impl(&m->blocks[l], m->x, kc, vc, pos, batch, s, l > 0);
+    int rc = block_forward_impl(&m->blocks[l], m->x, kc, vc, pos, batch, s, l > 0, -1, seq, nseq);
     if (rc) return rc;
   }
   // RmsFinal(Norm) fused into the logits GEMV; the vocab column split writes each
@@ -1079,6 +1099,29 @@ int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_
   a.ldo = d.vocab;
   a.err = at<int>(&m->blocks[0], BUF_ERR);
   return launch_gemv(a, EPI_PLAIN, s);
+}
+}  // namespace tp_api
+
+extern "C" {
+
+int tp_model_forward(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
+                     const int32_t* pos, int batch, float* logits, tp_stream stream) {
+  if (!m || !tokens || !k_cache || !v_cache || !pos || !logits) return TP_EINVAL;
+  if (batch < 1 || batch > m->d.max_batch) return TP_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits)) return TP_EALIGN;
+  return model_forward_impl(m, tokens, k_cache, v_cache, pos, nullptr, 0, batch, logits,
+                            (cudaStream_t)stream);
+}
+
+int tp_model_forward_seq(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
+                         const int32_t* pos, const int32_t* seq, int n_seq, int batch,
+                         float* logits, tp_stream stream) {
+  if (!m || !tokens || !k_cache || !v_cache || !pos || !seq || !logits) return TP_EINVAL;
+  if (batch < 1 || batch > m->d.max_batch || n_seq < 1) return TP_EINVAL;
+  if ((int64_t)n_seq * m->d.n_kv_heads * m->d.max_seq > INT32_MAX) return TP_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits)) return TP_EALIGN;
+  return model_forward_impl(m, tokens, k_cache, v_cache, pos, seq, n_seq, batch, logits,
+                            (cudaStream_t)stream);
 }
 
 int tp_model_set_persistent(tp_model* m, int enable) {

@@ -21,7 +21,10 @@
 // head; a second kernel combines the splits with the usual rescaling
 //   M = max_c m_c,  o = sum_c e^{m_c - M} o_c / sum_c e^{m_c - M} l_c.
 // Positions past pos are masked (score -inf, and the V rows zeroed in shared
-// memory), so stale cache contents never reach the output. The MMAs do at most
+// memory), so stale cache contents never reach the output. Rows may share a
+// cache sequence (a prefill chunk): each reads its own positions 0..pos, which
+// the q/k/v kernel before this one has written for every row of the step, so
+// the chunk attends causally. The MMAs do at most
 // 16 FLOP per KV byte, far below the tensor pipe's rate: the kernel is HBM-bound.
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
@@ -78,7 +81,8 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
     }
     return;
   }
-  const int row_base = (b * a.Hkv + kvh) * a.max_seq;
+  const int sq = a.seq ? a.seq[b] : b;  // the row's cache sequence
+  const int row_base = (sq * a.Hkv + kvh) * a.max_seq;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -328,7 +332,7 @@ int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {
   if (nsplit > a.nchunk) return TP_EINVAL;
   if (!aligned16(a.kc) || !aligned16(a.vc)) return TP_EALIGN;
   CUtensorMap mK, mV;
-  const uint64_t rows = (uint64_t)a.B * a.Hkv * a.max_seq;
+  const uint64_t rows = (uint64_t)(a.seq ? a.nseq : a.B) * a.Hkv * a.max_seq;
   if (!make_tensor_map_2d(&mK, a.kc, rows, kHeadDim, kHeadDim, 64, kTile) ||
       !make_tensor_map_2d(&mV, a.vc, rows, kHeadDim, kHeadDim, 64, kTile))
     return TP_ECUDA;

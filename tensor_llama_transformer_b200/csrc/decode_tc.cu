@@ -117,7 +117,8 @@ __global__ void k_qkv_finalize(QkvFinalizeArgs a) {
     *reinterpret_cast<float2*>(a.q + (size_t)b * a.qd + lrow) = make_float2(y0, y1);
   } else {
     uint16_t* cache = mat == 1 ? a.kc : a.vc;
-    const size_t o = (((size_t)b * a.n_kv_heads + head) * a.max_seq + pos) * kHeadDim + d;
+    const size_t sq = a.seq ? (size_t)a.seq[b] : (size_t)b;
+    const size_t o = ((sq * a.n_kv_heads + head) * a.max_seq + pos) * kHeadDim + d;
     *reinterpret_cast<uint32_t*>(cache + o) =
         (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
   }

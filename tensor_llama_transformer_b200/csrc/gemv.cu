@@ -475,7 +475,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
             make_float2(y0, y1);
       } else {
         uint16_t* cache = mat == 1 ? a.kc : a.vc;
-        const size_t o = (((size_t)gb * a.n_kv_heads + head) * a.max_seq + pos) * kHeadDim + d;
+        const size_t sq = a.seq ? (size_t)a.seq[gb] : (size_t)gb;
+        const size_t o = ((sq * a.n_kv_heads + head) * a.max_seq + pos) * kHeadDim + d;
         *reinterpret_cast<uint32_t*>(cache + o) =
             (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
       }

@@ -77,9 +77,10 @@ struct GemvArgs {
   int ldo;
   // EPI_QKV
   float* qout;   // rotated q [B, H*hd]
-  uint16_t* kc;  // caches [maxB, Hkv, max_seq, hd]
+  uint16_t* kc;  // caches [sequences, Hkv, max_seq, hd]
   uint16_t* vc;
   const int32_t* pos;
+  const int32_t* seq;  // cache sequence of each row (nullable: row b uses sequence b)
   int n_heads, n_kv_heads, max_seq;
   float theta;
   int* err;  // device error flag, set when a bounded wait gives up (nullable)
@@ -104,9 +105,11 @@ int launch_gemv(const GemvArgs& a, int epi, cudaStream_t s);
 // ------------------------------------------------------------------ attention
 struct AttnArgs {
   const float* q;       // rotated q [B, H*hd]
-  const uint16_t* kc;   // [maxB, Hkv, max_seq, hd] bf16
+  const uint16_t* kc;   // [nseq, Hkv, max_seq, hd] bf16
   const uint16_t* vc;
   const int32_t* pos;   // [B]
+  const int32_t* seq;   // [B] cache sequence of each row (nullable: row b)
+  int nseq;             // sequences in the caches (with seq; else B)
   int B, H, Hkv, max_seq;
   int nchunk;           // capacity of the partial buffers in context splits
   float* part_o;        // [B, H, nsplit, hd] unnormalised partial outputs (nsplit <= nchunk)
@@ -148,6 +151,7 @@ struct QkvFinalizeArgs {
   const float* plane;  // [parts][batch][qd + 2 kd]
   int parts, batch, qd, kd;
   const int32_t* pos;
+  const int32_t* seq;  // cache sequence of each row (nullable: row b)
   float theta;
   float* q;            // [batch, qd]
   uint16_t* kc;

@@ -142,3 +142,12 @@ def test_rank_block_sizes_and_validation(tpb):
     with pytest.raises(tpb.TpError) as e:
         tpb.tp_block_rank_sync_bytes(None, 1)
     assert e.value.status == tpb.TP_EINVAL
+
+
+def test_sequence_map_entry_points_validate(tpb):
+    """Rows mapped to cache sequences: NULL handles and sequence maps are refused."""
+    for call in (lambda: tpb.tp_block_forward_seq(None, 16, 16, 16, 16, 16, 1, 1, stream=0),
+                 lambda: tpb.tp_model_forward_seq(None, 16, 16, 16, 16, 16, 1, 1, 16, stream=0)):
+        with pytest.raises(tpb.TpError) as e:
+            call()
+        assert e.value.status == tpb.TP_EINVAL
