@@ -166,9 +166,10 @@ def test_model_prefill_chunk(tpb):
                          s.max_seq, s.norm_eps, s.rope_theta)
     nbytes = tpb.tp_model_workspace_bytes(dims, n_layers, s.n_slices, 1, 0)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-    h = tpb.tp_model_create(dims, n_layers, s.n_slices, 1, 0, weights, bf16_tensor(emb),
-                            torch.ones(s.dim, dtype=torch.float32, device="cuda"),
-                            bf16_tensor(wcls), ws, nbytes)
+    # the handle borrows these pointers: keep the tensors alive until it is destroyed
+    emb_d, wcls_d = bf16_tensor(emb), bf16_tensor(wcls)
+    fn = torch.ones(s.dim, dtype=torch.float32, device="cuda")
+    h = tpb.tp_model_create(dims, n_layers, s.n_slices, 1, 0, weights, emb_d, fn, wcls_d, ws, nbytes)
     logits = torch.empty((L, s.vocab), dtype=torch.float32, device="cuda")
     try:
         tpb.tp_model_forward_seq(h, i32_tensor(toks), kc, vc, i32_tensor(pos), i32_tensor(seq), 1, L,
