@@ -50,6 +50,85 @@ TP_DEV int tiles_per_split(int P, int nsplit) {
   return (ntiles + nsplit - 1) / nsplit;
 }
 
+// One K/V tile of a consumer warp (positions t0 + w0 .. t0 + w0 + 15): S = Q K^T,
+// the online softmax of the thread's head row (positions >= P_row masked), and
+// O += P V. V rows at positions >= p_zero (past every context the CTA serves)
+// are zeroed first so that stale cache contents never reach O.
+TP_DEV void attn_tile(uint8_t* smem, uint32_t kb, const uint32_t (&qa)[8][4], float (&o)[16][4],
+                      float& m_run, float& l_run, int lane, int w0, int t0, int P_row,
+                      int p_zero) {
+  const uint32_t vb = kb + 2 * kBox;
+  if (t0 + w0 + 16 > p_zero) {  // V rows past every context -> 0 (a context's last tile)
+    for (int idx = lane; idx < 16 * 16; idx += 32) {
+      const int r = idx >> 4, c = idx & 15;
+      if (t0 + w0 + r >= p_zero)
+        *reinterpret_cast<uint4*>(smem + (kv_tile_addr(vb, w0 + r, c) - s2u(smem))) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+  }
+  // S = Q K^T over the warp's two 8-position column tiles
+  float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  {
+    const int t = w0 + (lane & 7) + 8 * (lane >> 4), ch = (lane >> 3) & 1;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t bf[4];
+      ldsm_x4(kv_tile_addr(kb, t, 2 * ks + ch), bf);
+      mma_bf16(sc[0], qa[ks], bf[0], bf[1]);
+      mma_bf16(sc[1], qa[ks], bf[2], bf[3]);
+    }
+  }
+  // this thread's scores of head g: positions t0 + w0 + 8 nt + 2 (lane & 3) + j
+  float sv[2][2], tmax = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int tp = t0 + w0 + 8 * nt + 2 * (lane & 3) + j;
+      const float v = sc[nt][j] + sc[nt][2 + j];  // hi row + lo row
+      sv[nt][j] = tp < P_row ? v : -INFINITY;
+      tmax = fmaxf(tmax, sv[nt][j]);
+    }
+  tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+  tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+  const float m_new = fmaxf(m_run, tmax);
+  const float resc = m_new == -INFINITY ? 1.f : expf(m_run - m_new);
+  uint16_t ph[2][2], pl[2][2];
+  float psum = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float p = sv[nt][j] == -INFINITY ? 0.f : expf(sv[nt][j] - m_new);
+      psum += p;
+      bf16_split(p, ph[nt][j], pl[nt][j]);
+    }
+  const uint32_t pa[4] = {pack_bf16x2(ph[0][0], ph[0][1]), pack_bf16x2(pl[0][0], pl[0][1]),
+                          pack_bf16x2(ph[1][0], ph[1][1]), pack_bf16x2(pl[1][0], pl[1][1])};
+  l_run = l_run * resc + psum;
+  m_run = m_new;
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) {
+    o[nt][0] *= resc;
+    o[nt][1] *= resc;
+    o[nt][2] *= resc;
+    o[nt][3] *= resc;
+  }
+  // O += P V over the warp's 16 positions, 16 dim tiles of 8
+  {
+    const int t = w0 + (lane & 7) + 8 * ((lane >> 3) & 1), ch = lane >> 4;
+#pragma unroll
+    for (int np = 0; np < 8; ++np) {
+      uint32_t bf[4];
+      ldsm_x4_t(kv_tile_addr(vb, t, 2 * np + ch), bf);
+      mma_bf16(o[2 * np], pa, bf[0], bf[1]);
+      mma_bf16(o[2 * np + 1], pa, bf[2], bf[3]);
+    }
+  }
+}
+
 template <int G>
 __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant__ CUtensorMap mK,
                                                           const __grid_constant__ CUtensorMap mV,
@@ -140,79 +219,8 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
       const int k = i - i0, s = k % kStages;
       const bool got = ok ? mbar_wait(&full[s], (uint32_t)(k / kStages) & 1u, a.err) : false;
       ok = __all_sync(0xffffffffu, got);
-      if (ok) {
-        const uint32_t kb = s2u(smem + s * kStageBytes), vb = kb + 2 * kBox;
-        const int t0 = i * kTile;
-        if (t0 + w0 + 16 > P) {  // V rows past pos -> 0 (only the context's last tile)
-          for (int idx = lane; idx < 16 * 16; idx += 32) {
-            const int r = idx >> 4, c = idx & 15;
-            if (t0 + w0 + r >= P)
-              *reinterpret_cast<uint4*>(smem + (kv_tile_addr(vb, w0 + r, c) - s2u(smem))) =
-                  make_uint4(0u, 0u, 0u, 0u);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-        }
-        // S = Q K^T over the warp's two 8-position column tiles
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        {
-          const int t = w0 + (lane & 7) + 8 * (lane >> 4), ch = (lane >> 3) & 1;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            uint32_t bf[4];
-            ldsm_x4(kv_tile_addr(kb, t, 2 * ks + ch), bf);
-            mma_bf16(sc[0], qa[ks], bf[0], bf[1]);
-            mma_bf16(sc[1], qa[ks], bf[2], bf[3]);
-          }
-        }
-        // this thread's scores of head g: positions t0 + w0 + 8 nt + 2 (lane & 3) + j
-        float sv[2][2], tmax = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int tp = t0 + w0 + 8 * nt + 2 * (lane & 3) + j;
-            const float v = sc[nt][j] + sc[nt][2 + j];  // hi row + lo row
-            sv[nt][j] = tp < P ? v : -INFINITY;
-            tmax = fmaxf(tmax, sv[nt][j]);
-          }
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-        const float m_new = fmaxf(m_run, tmax);
-        const float resc = m_new == -INFINITY ? 1.f : expf(m_run - m_new);
-        uint16_t ph[2][2], pl[2][2];
-        float psum = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const float p = sv[nt][j] == -INFINITY ? 0.f : expf(sv[nt][j] - m_new);
-            psum += p;
-            bf16_split(p, ph[nt][j], pl[nt][j]);
-          }
-        const uint32_t pa[4] = {pack_bf16x2(ph[0][0], ph[0][1]), pack_bf16x2(pl[0][0], pl[0][1]),
-                                pack_bf16x2(ph[1][0], ph[1][1]), pack_bf16x2(pl[1][0], pl[1][1])};
-        l_run = l_run * resc + psum;
-        m_run = m_new;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          o[nt][0] *= resc;
-          o[nt][1] *= resc;
-          o[nt][2] *= resc;
-          o[nt][3] *= resc;
-        }
-        // O += P V over the warp's 16 positions, 16 dim tiles of 8
-        {
-          const int t = w0 + (lane & 7) + 8 * ((lane >> 3) & 1), ch = lane >> 4;
-#pragma unroll
-          for (int np = 0; np < 8; ++np) {
-            uint32_t bf[4];
-            ldsm_x4_t(kv_tile_addr(vb, t, 2 * np + ch), bf);
-            mma_bf16(o[2 * np], pa, bf[0], bf[1]);
-            mma_bf16(o[2 * np + 1], pa, bf[2], bf[3]);
-          }
-        }
-      }
+      if (ok)
+        attn_tile(smem, s2u(smem + s * kStageBytes), qa, o, m_run, l_run, lane, w0, i * kTile, P, P);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
@@ -257,22 +265,187 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   }
 }
 
+// Rows that share a cache sequence (a prefill chunk, given a sequence map on the
+// batched path): a CTA takes R = 8 / G consecutive rows and the G query heads of
+// one kv head, so its 8 head rows are (row, head) pairs that read the same K/V
+// tiles -- each tile crosses into shared memory once for R tokens instead of
+// once per token. Rows of different sequences in one CTA (a step mixing decode
+// rows of several sequences) are taken in passes, one per sequence. A pass's
+// split covers tiles of the longest context among its rows; every row masks the
+// positions past its own, so it attends causally. Each (row, head, split) slot
+// gets a partial, empty ones (m = -inf, l = 0) included, and k_attn_combine reads
+// all splits.
+template <int G>
+__global__ void __launch_bounds__(kAThreads) k_attn_rows(const __grid_constant__ CUtensorMap mK,
+                                                         const __grid_constant__ CUtensorMap mV,
+                                                         AttnArgs a, int nsplit) {
+  constexpr int R = 8 / G;  // rows per CTA
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint16_t* qs = reinterpret_cast<uint16_t*>(smem + kStages * kStageBytes);  // [16][kQStride]
+  __shared__ uint64_t full[kStages], empty[kStages];
+  __shared__ float s_m[kCWarps][8], s_l[kCWarps][8];
+  __shared__ int s_seq[R], s_pmax[R], s_i0[R], s_i1[R];  // per pass
+  __shared__ unsigned s_act[R];  // per pass: bit g set when head row g's token is in it
+  __shared__ int s_npass;
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b0 = blockIdx.z * R;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  pdl_wait();  // q and the cache rows of this step come from the q/k/v kernel
+  if (threadIdx.x == 0) {
+    int np = 0;
+    for (int r = 0; r < R && b0 + r < a.B; ++r) {
+      const int sq = a.seq[b0 + r], P = a.pos[b0 + r] + 1;
+      int p = 0;
+      while (p < np && s_seq[p] != sq) ++p;
+      if (p == np) {
+        s_seq[p] = sq;
+        s_pmax[p] = 0;
+        s_act[p] = 0u;
+        ++np;
+      }
+      s_pmax[p] = max(s_pmax[p], P);
+      s_act[p] |= ((1u << G) - 1u) << (r * G);
+    }
+    for (int p = 0; p < np; ++p) {
+      const int ntiles = (s_pmax[p] + kTile - 1) / kTile;
+      const int tpc = tiles_per_split(s_pmax[p], nsplit);
+      s_i0[p] = split * tpc;
+      s_i1[p] = min(ntiles, split * tpc + tpc);
+    }
+    s_npass = np;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCWarps);
+    }
+    mbar_init_fence();
+  }
+  // head row g = (token b0 + g / G, query head kvh G + g % G), scaled by 1/sqrt(hd):
+  // hi in row g, lo in row g + 8
+  const float scale = 1.0f / sqrtf((float)kHeadDim);
+  for (int i = threadIdx.x; i < 8 * kHeadDim; i += kAThreads) {
+    const int g = i / kHeadDim, d = i - g * kHeadDim, b = b0 + g / G;
+    uint16_t hi = 0, lo = 0;
+    if (b < a.B)
+      bf16_split(a.q[((size_t)b * a.H + (size_t)kvh * G + g % G) * kHeadDim + d] * scale, hi, lo);
+    qs[g * kQStride + d] = hi;
+    qs[(g + 8) * kQStride + d] = lo;
+  }
+  __syncthreads();
+  const int npass = s_npass;
+
+  if (warp == kCWarps) {
+    // ------------------------------------------------------------ producer warp
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first();
+      bool ok = true;
+      int k = 0;
+      for (int p = 0; p < npass && ok; ++p) {
+        const int row_base = (s_seq[p] * a.Hkv + kvh) * a.max_seq;
+        for (int i = s_i0[p]; i < s_i1[p]; ++i, ++k) {
+          const int s = k % kStages;
+          if (!mbar_wait(&empty[s], ((uint32_t)(k / kStages) & 1u) ^ 1u, a.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], kStageBytes);
+          uint8_t* st = smem + s * kStageBytes;
+          const int y = row_base + i * kTile;
+          tma_load_2d_hint(st, &mK, 0, y, &full[s], pol);
+          tma_load_2d_hint(st + kBox, &mK, 64, y, &full[s], pol);
+          tma_load_2d_hint(st + 2 * kBox, &mV, 0, y, &full[s], pol);
+          tma_load_2d_hint(st + 3 * kBox, &mV, 64, y, &full[s], pol);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumer warps
+    const int g = lane >> 2;  // the head row whose scores this thread holds
+    const int bg = b0 + g / G;
+    const int Pg = bg < a.B ? a.pos[bg] + 1 : 0;
+    uint32_t qa[8][4];
+    {
+      const uint32_t qb = s2u(qs);
+      const int r = (lane & 7) + 8 * ((lane >> 3) & 1), ch = lane >> 4;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        ldsm_x4(qb + (uint32_t)((r * kQStride + 16 * ks + 8 * ch) * 2), qa[ks]);
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    bool ok = true;
+    const int w0 = 16 * warp;
+    int k = 0;
+    for (int p = 0; p < npass; ++p) {
+      const int P_row = ((s_act[p] >> g) & 1u) ? Pg : 0;  // 0: not this pass's sequence
+      for (int i = s_i0[p]; i < s_i1[p]; ++i, ++k) {
+        const int s = k % kStages;
+        const bool got = ok ? mbar_wait(&full[s], (uint32_t)(k / kStages) & 1u, a.err) : false;
+        ok = __all_sync(0xffffffffu, got);
+        if (ok)
+          attn_tile(smem, s2u(smem + s * kStageBytes), qa, o, m_run, l_run, lane, w0, i * kTile,
+                    P_row, s_pmax[p]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    if ((lane & 3) == 0) {
+      s_m[warp][g] = m_run;
+      s_l[warp][g] = l_run;
+    }
+    consumers_sync(kCWarps * 32);
+    float* ro = reinterpret_cast<float*>(smem);  // [kCWarps][8][kHeadDim]
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      const int d = 8 * nt + 2 * (lane & 3);
+      ro[(warp * 8 + g) * kHeadDim + d] = o[nt][0] + o[nt][2];
+      ro[(warp * 8 + g) * kHeadDim + d + 1] = o[nt][1] + o[nt][3];
+    }
+  }
+  __syncthreads();
+  const float* ro = reinterpret_cast<const float*>(smem);
+  for (int idx = threadIdx.x; idx < 8 * kHeadDim; idx += kAThreads) {
+    const int gg = idx / kHeadDim, d = idx - gg * kHeadDim, b = b0 + gg / G;
+    if (b >= a.B) continue;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, s_m[w][gg]);
+    float os = 0.f, ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w) {
+      const float f = s_m[w][gg] == -INFINITY ? 0.f : expf(s_m[w][gg] - M);
+      os = fmaf(f, ro[(w * 8 + gg) * kHeadDim + d], os);
+      ls = fmaf(f, s_l[w][gg], ls);
+    }
+    const size_t pi = ((size_t)b * a.H + (size_t)kvh * G + gg % G) * nsplit + split;
+    a.part_o[pi * kHeadDim + d] = os;
+    if (d == 0) {
+      a.part_ml[pi * 2 + 0] = M;
+      a.part_ml[pi * 2 + 1] = ls;
+    }
+  }
+}
+
 // One CTA per (head, batch row); thread d owns output dimension d.
 __global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a, int nsplit) {
   pdl_launch_dependents();
   pdl_wait();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const int P = a.pos[b] + 1;
-  const int ntiles = (P + kTile - 1) / kTile;
-  const int tpc = tiles_per_split(P, nsplit);
-  const int nc = (ntiles + tpc - 1) / tpc;  // splits that hold positions
+  // every split of every (row, head) holds a partial, the empty ones m = -inf, l = 0
   const size_t base = ((size_t)b * a.H + h) * nsplit;
   float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, a.part_ml[(base + c) * 2]);
+  for (int c = 0; c < nsplit; ++c) M = fmaxf(M, a.part_ml[(base + c) * 2]);
   float l = 0.f, o = 0.f;
-  for (int c = 0; c < nc; ++c) {
+  for (int c = 0; c < nsplit; ++c) {
     const float mc = a.part_ml[(base + c) * 2];
-    const float w = mc == -INFINITY ? 0.f : expf(mc - M);
+    if (mc == -INFINITY) continue;  // an empty split: its o may be stale, never read it
+    const float w = expf(mc - M);
     l = fmaf(w, a.part_ml[(base + c) * 2 + 1], l);
     o = fmaf(w, a.part_o[(base + c) * kHeadDim + d], o);
   }
@@ -284,6 +457,14 @@ __global__ void __launch_bounds__(kHeadDim) k_attn_combine(AttnArgs a, int nspli
     const size_t hi = (size_t)(2 * b) * row + (size_t)h * kHeadDim + d;
     bf16_split(r, a.att_bf16[hi], a.att_bf16[hi + row]);
   }
+}
+
+template <int G>
+int launch_rows(const AttnArgs& a, const CUtensorMap& mK, const CUtensorMap& mV, int nsplit,
+                cudaStream_t s) {
+  if (set_smem_once((const void*)k_attn_rows<G>, kSmemBytes)) return TP_ECUDA;
+  return launch_pdl(k_attn_rows<G>, dim3(nsplit, a.Hkv, (a.B + 8 / G - 1) / (8 / G)),
+                    dim3(kAThreads), kSmemBytes, s, mK, mV, a, nsplit);
 }
 
 template <int G>
@@ -328,7 +509,11 @@ int attention_nsplit(int B, int H, int Hkv, int max_seq) {
 
 int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {
   const int G = a.H / a.Hkv;
-  const int nsplit = attention_nsplit(a.B, a.H, a.Hkv, a.max_seq);
+  // rows mapped to cache sequences share tiles (k_attn_rows) when the splits are
+  // combined here and a CTA holds at least two rows
+  const bool shared = a.seq && combine && G <= 4;
+  const int nsplit = shared ? attention_splits((a.B + 8 / G - 1) / (8 / G), a.Hkv, a.max_seq)
+                            : attention_nsplit(a.B, a.H, a.Hkv, a.max_seq);
   if (nsplit > a.nchunk) return TP_EINVAL;
   if (!aligned16(a.kc) || !aligned16(a.vc)) return TP_EALIGN;
   CUtensorMap mK, mV;
@@ -337,6 +522,13 @@ int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {
       !make_tensor_map_2d(&mV, a.vc, rows, kHeadDim, kHeadDim, 64, kTile))
     return TP_ECUDA;
   int rc;
+  if (shared) {
+    rc = G == 1 ? launch_rows<1>(a, mK, mV, nsplit, s)
+       : G == 2 ? launch_rows<2>(a, mK, mV, nsplit, s)
+                : launch_rows<4>(a, mK, mV, nsplit, s);
+    if (rc != TP_OK) return rc;
+    return launch_pdl(k_attn_combine, dim3(a.H, a.B), dim3(kHeadDim), 0, s, a, nsplit);
+  }
   switch (G) {
     case 1: rc = launch_g<1>(a, mK, mV, nsplit, s); break;
     case 2: rc = launch_g<2>(a, mK, mV, nsplit, s); break;
