@@ -53,7 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the C4 block and C3 model measurements")
-    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w"], default=None,
+    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w", "c2prefill"], default=None,
                     help="only run a few eager steps of one extra workload (for profiler launch "
                          "lists: c4 block, c3 model at batch 1, c2 block on the persistent kernel, "
                          "c2 block with int8 weights)")
@@ -472,6 +472,12 @@ def bench_c2_prefill(args):
     nb = tpb.tp_block_workspace_bytes(dims, s.n_slices, 1, 1)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     h = tpb.tp_block_create(dims, s.n_slices, 1, 1, tpb.make_weights(*w), ws, nb)
+    if args.profile == "c2prefill":
+        for _ in range(args.profile_steps):
+            tpb.tp_block_forward_seq(h, x, kc, vc, pos, seq, 1, L)
+        torch.cuda.synchronize()
+        tpb.tp_block_destroy(h)
+        return {"profile": "c2prefill", "steps": args.profile_steps}
     ms = _time_graph(torch, lambda: tpb.tp_block_forward_seq(h, x, kc, vc, pos, seq, 1, L), 10, 5)
     tpb.tp_block_destroy(h)
     wb, _ = block_bytes(s)
@@ -711,7 +717,7 @@ def main(argv=None):
         return 1
     if args.profile:
         fn = {"c4": bench_c4, "c3b1": lambda a: bench_c3(a, 1), "c2p": bench_c2_persistent,
-              "c2q8w": bench_c2_q8w}
+              "c2q8w": bench_c2_q8w, "c2prefill": bench_c2_prefill}
         print(json.dumps(fn[args.profile](args)))
         return 0
     world, rank, local = dist_setup()
