@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   const int tpc = tiles_per_split(P, nsplit);
   const int i0 = split * tpc, i1 = min(ntiles, i0 + tpc);
   const size_t pbase = ((size_t)b * a.H + (size_t)h0) * nsplit + split;
-  if (i0 >= i1) {  // nothing left for this split (the combine does not read it)
+  if (i0 >= i1) {  // nothing left for this split: an empty partial (m = -inf, l = 0)
     if (threadIdx.x < G) {
       a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 0] = -INFINITY;
       a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 1] = 0.f;
