@@ -145,9 +145,10 @@ def _run(world, shape_kw, quant):
     return res
 
 
-@pytest.mark.parametrize("shape_kw", [SHAPE, GQA], ids=["mha", "gqa2"])
+@pytest.mark.parametrize("shape_kw,world", [(SHAPE, 2), (GQA, 2), (SHAPE, 4)],
+                         ids=["mha-2", "gqa2-2", "mha-4"])
 @pytest.mark.parametrize("quant", [0, 1])
-def test_two_ranks_equal_the_whole_block(shape_kw, quant):
+def test_ranks_equal_the_whole_block(shape_kw, world, quant):
     import oracle
     import synth
 
@@ -155,9 +156,10 @@ def test_two_ranks_equal_the_whole_block(shape_kw, quant):
     inp = synth.block_inputs(SEED, s)
     inp.pos[:] = POS
     ref, k_ref, v_ref = oracle.block_forward(inp, s.n_slices, bool(quant))
-    res = _run(2, shape_kw, quant)
+    res = _run(world, shape_kw, quant)
     # every rank ends with the same residual (the same bytes merged the same way)
-    assert np.array_equal(res[0][1], res[1][1])
+    for r in res[1:]:
+        assert np.array_equal(r[1], res[0][1])
     err = np.max(np.abs(res[0][1] - ref)) / np.max(np.abs(ref))
     assert err < 1e-6, err  # float32 transfer of the partials vs the oracle's float64
     # the gathered buffer is the ranks' send buffers in rank order (= slice order)
@@ -165,7 +167,7 @@ def test_two_ranks_equal_the_whole_block(shape_kw, quant):
     for r in res:
         np.testing.assert_array_equal(r[3][1], sends)
     # each rank wrote the k / v rows of its own kv heads
-    Hkvl = s.n_kv_heads // 2
+    Hkvl = s.n_kv_heads // world
     for r, _, rows, _ in res:
         heads = slice(r * Hkvl, (r + 1) * Hkvl)
         np.testing.assert_array_equal(rows[0], k_ref[:, heads])
@@ -195,3 +197,44 @@ def test_rank_split_helpers():
         assert torch.equal(torch.cat([p[k] for p in parts], 1), w[k])
         assert all(p[k].is_contiguous() for p in parts)
     assert parts[1]["wq"].shape == (H // 2 * hd, D) and parts[1]["wo"].shape == (D, H // 2 * hd)
+
+
+def _failing_worker(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    send = torch.zeros(16, dtype=torch.uint8)
+    recv = torch.zeros(16 * world, dtype=torch.uint8)
+
+    def step(phase):
+        if rank == 1 and phase == tp.TP_RANK_ATT:
+            raise RuntimeError("rank 1 failed in phase 0")
+
+    try:
+        tp.run_step(step, tp.all_gather_exchange(), send, recv)
+        out.put((rank, "completed"))
+    except Exception as e:  # reported to the parent, which checks that nobody hangs
+        out.put((rank, f"{type(e).__name__}: {str(e)[:80]}"))
+
+
+def test_failed_rank_ends_the_others_step_with_an_error():
+    """A rank that fails before its first exchange never joins the all-gather: the
+    other rank's exchange ends with an error (process-group timeout or closed
+    connection) instead of waiting for ever. Host-side failure only."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(60)
+        assert p.exitcode is not None
+    assert res[1].startswith("RuntimeError: rank 1 failed")
+    assert res[0] != "completed", res[0]
