@@ -4,6 +4,9 @@
  * One decoder block's decode step, partitioned tensor-parallel into n weight
  * slices that all run as partitions of the same launches on one GPU, plus the
  * 1D / 2D partitioned feed-forward layer and the full multi-layer decode step.
+ * Rows may map to cache sequences (prefill chunks, mixed steps), and a block's
+ * slices may be spread over processes, one GPU each, with the caller moving the
+ * sync buffers between them.
  *
  * Sources for what is computed (pages on the subject, by title and part):
  *   - distributed-llama issue #29, "[Feature Suggest] Tensor Parallellism for

@@ -124,3 +124,9 @@ class RankBlock:
         if self.h:
             self.lib.tp_block_destroy(self.h)
             self.h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
