@@ -15,7 +15,6 @@ all-gather through ``torch.distributed``): it must give exactly the bits of
 tp_block_forward.
 """
 import datetime
-import os
 import socket
 
 import numpy as np

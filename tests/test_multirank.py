@@ -8,7 +8,6 @@ printing (and, for the reference arm, alone running the oracle).
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 
