@@ -60,7 +60,7 @@ enum tp_status {
   TP_EWORKSPACE = 2,  /* workspace pointer NULL or smaller than required */
   TP_EARCH = 3,       /* current device is not compute capability 10.0 (B200) */
   TP_ECUDA = 4,       /* a CUDA runtime call or kernel launch failed */
-  TP_ENOTSUP = 5,     /* a combination this build does not implement */
+  TP_ENOTSUP = 5,     /* a combination this library does not implement */
   TP_EALIGN = 6,      /* a pointer is not 16-byte aligned */
   TP_ESCRATCH = 7     /* the workspace would exceed the no-allocation entry point's fixed scratch */
 };

@@ -770,7 +770,7 @@ const char* tp_status_string(int st) {
     case TP_EWORKSPACE: return "workspace missing or too small";
     case TP_EARCH: return "device is not sm_100 (B200)";
     case TP_ECUDA: return "CUDA runtime error";
-    case TP_ENOTSUP: return "not supported by this build";
+    case TP_ENOTSUP: return "not supported by this library";
     case TP_EALIGN: return "pointer not 16-byte aligned";
     case TP_ESCRATCH: return "workspace exceeds the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
