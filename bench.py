@@ -53,10 +53,14 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the C4 block and C3 model measurements")
-    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w", "c2prefill"], default=None,
+    ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w", "c2prefill", "ffn"],
+                    default=None,
                     help="only run a few eager steps of one extra workload (for profiler launch "
                          "lists: c4 block, c3 model at batch 1, c2 block on the persistent kernel, "
-                         "c2 block with int8 weights)")
+                         "c2 block with int8 weights, c2 prefill chunk, or the fused PaLM-shaped "
+                         "FFN at B 512 with F cut to --profile-ffn-f)")
+    ap.add_argument("--profile-ffn-f", type=int, default=18432,
+                    help="intermediate size of the --profile ffn case (PaLM: 73728)")
     ap.add_argument("--profile-steps", type=int, default=3)
     return ap.parse_args(argv)
 
@@ -715,6 +719,40 @@ def bench_ffn(args):
     return out
 
 
+def profile_ffn(args):
+    """A few fused forwards of the PaLM-shaped FFN (B 512, E 18432, ReLU, 1D over 64
+    slices) with F cut to --profile-ffn-f, so that a full-section capture of one
+    tcgen05 GEMM launch holds a few GB on the device (F 18432: 1.36 GB of weights)."""
+    import torch
+
+    import tensor_llama_transformer_b200 as tpb
+
+    B, E, F = 512, 18432, args.profile_ffn_f
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1004)
+    X = _randn_bf16(torch, gen, (B, E), 1.0)
+    W1 = _randn_bf16(torch, gen, (F, E), 0.01)
+    W2 = _randn_bf16(torch, gen, (E, F), 0.01)
+    Y = torch.empty((B, E), dtype=torch.float32, device="cuda")
+    desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1, 1, 0,
+                           tpb.TP_MERGE_FUSED)
+    nb = tpb.tp_ffn_workspace_bytes(desc)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    for _ in range(args.profile_steps):
+        tpb.tp_ffn_forward(desc, X, W1, None, W2, Y, ws, nb)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    tpb.tp_ffn_forward(desc, X, W1, None, W2, Y, ws, nb)
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b)
+    flops = 2.0 * B * 2 * E * F
+    return {"profile": "ffn", "steps": args.profile_steps + 1, "B": B, "E": E, "F": F,
+            "last_forward_ms": ms, "tflops": flops / (ms / 1e3) / 1e12,
+            "pipeline_error": int(ws[:4].view(torch.int32).item())}
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -726,7 +764,7 @@ def main(argv=None):
         return 1
     if args.profile:
         fn = {"c4": bench_c4, "c3b1": lambda a: bench_c3(a, 1), "c2p": bench_c2_persistent,
-              "c2q8w": bench_c2_q8w, "c2prefill": bench_c2_prefill}
+              "c2q8w": bench_c2_q8w, "c2prefill": bench_c2_prefill, "ffn": profile_ffn}
         print(json.dumps(fn[args.profile](args)))
         return 0
     world, rank, local = dist_setup()

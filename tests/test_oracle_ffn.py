@@ -123,3 +123,133 @@ def test_chunked_unsharded_matches_ffn_forward(act):
                       W3=bf16_to_f64(W3) if W3 is not None else None)
     got = ffn_unsharded_chunked(X, inp["W1"], inp["W2"], act=act, W3_bits=W3, chunk=96)
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# 2D partition with Q8 sync buffers (Pope et al. demo1's 2D weight-stationary
+# layout with the distributed-llama Quantize/Dequantize around every exchange)
+# ---------------------------------------------------------------------------
+
+def _q8_trip(P):
+    """The sync round trip of one partial (q8_quantize / q8_dequantize are pinned in
+    test_oracle_q8.py): float32, codes per 32 values along the last axis, back."""
+    from oracle import q8_dequantize
+
+    q, d = q8_quantize(np.asarray(P, dtype=np.float32))
+    return q8_dequantize(q, d).astype(np.float64)
+
+
+def _loop_ffn_2d_q8(X, W1, W2, gx, gy, act, W3=None):
+    """Plain loops over the gx x gy grid: every stage-1 partial (one per (x, y) cell,
+    summed over x) and every stage-2 partial (one per cell, summed over y) crosses
+    its own quantised sync."""
+    B, E = X.shape
+    F = W1.shape[0]
+    ex, fy = E // gx, F // gy
+    H = np.zeros((B, F))
+    for y in range(gy):
+        a = np.zeros((B, fy))
+        c = np.zeros((B, fy))
+        for x in range(gx):
+            p1 = np.zeros((B, fy))
+            p3 = np.zeros((B, fy))
+            for b in range(B):
+                for f in range(fy):
+                    p1[b, f] = sum(X[b, x * ex + e] * W1[y * fy + f, x * ex + e] for e in range(ex))
+                    if W3 is not None:
+                        p3[b, f] = sum(X[b, x * ex + e] * W3[y * fy + f, x * ex + e]
+                                       for e in range(ex))
+            a = a + _q8_trip(p1)
+            if W3 is not None:
+                c = c + _q8_trip(p3)
+        for b in range(B):
+            for f in range(fy):
+                z = a[b, f]
+                H[b, y * fy + f] = max(z, 0.0) if act == "relu" else z / (1.0 + np.exp(-z)) * c[b, f]
+    Y = np.zeros((B, E))
+    for x in range(gx):
+        acc = np.zeros((B, ex))
+        for y in range(gy):
+            p2 = np.zeros((B, ex))
+            for b in range(B):
+                for e in range(ex):
+                    p2[b, e] = sum(H[b, y * fy + f] * W2[x * ex + e, y * fy + f] for f in range(fy))
+            acc = acc + _q8_trip(p2)
+        Y[:, x * ex:(x + 1) * ex] = acc
+    return Y
+
+
+@pytest.mark.parametrize("act", ["relu", "swiglu"])
+@pytest.mark.parametrize("grid", [(2, 2), (2, 1), (1, 2)])
+def test_quantised_2d_loop_restatement(act, grid):
+    gx, gy = grid
+    B, E, F = 2, 64, 128
+    X, W1, W2 = _rand(31, (B, E)), _rand(32, (F, E), 0.2), _rand(33, (E, F), 0.2)
+    W3 = _rand(34, (F, E), 0.2) if act == "swiglu" else None
+    ref = _loop_ffn_2d_q8(X, W1, W2, gx, gy, act, W3)
+    y = ffn_forward(X, W1, W2, act=act, W3=W3, partition=2, n_slices=gx * gy, grid=grid,
+                    quant=True)
+    scale = np.max(np.abs(ref))
+    assert np.max(np.abs(y - ref)) <= 1e-12 * scale
+
+
+def test_quantised_2d_quantises_every_cell():
+    """The same grid quantising once after each sum over x (stage 1) or y (stage 2),
+    instead of every cell's partial, gives a different layer: the loop restatement
+    above tells the two apart."""
+    B, E, F, gx, gy = 2, 64, 128, 2, 2
+    X, W1, W2 = _rand(35, (B, E)), _rand(36, (F, E), 0.2), _rand(37, (E, F), 0.2)
+    ex, fy = E // gx, F // gy
+    H = np.zeros((B, F))
+    for y in range(gy):
+        fs = slice(y * fy, (y + 1) * fy)
+        H[:, fs] = relu(_q8_trip(X @ W1[fs].T))
+    Y = np.zeros((B, E))
+    for x in range(gx):
+        es = slice(x * ex, (x + 1) * ex)
+        Y[:, es] = _q8_trip(H @ W2[es].T)
+    y = ffn_forward(X, W1, W2, act="relu", partition=2, n_slices=4, grid=(gx, gy), quant=True)
+    assert np.max(np.abs(y - Y)) > 1e-6 * np.max(np.abs(Y))
+    np.testing.assert_allclose(y, _loop_ffn_2d_q8(X, W1, W2, gx, gy, "relu"), rtol=0,
+                               atol=1e-12 * np.max(np.abs(y)))
+
+
+@pytest.mark.parametrize("grid", [(2, 2), (4, 2), (2, 4)])
+def test_quantised_2d_within_bound(grid):
+    """Every quantised sync moves a value by at most half its block's scale d (plus
+    float32 rounding). Stage 1: |A_q - A| <= sum_x d_xy / 2; ReLU is 1-Lipschitz, so
+    H moves by no more; stage 2 carries that through |W2| and adds each cell's own
+    d / 2, whose block scale is at most (block max of |P2| + its carried error) / 127."""
+    gx, gy = grid
+    B, E, F = 4, 128, 256
+    X, W1, W2 = _rand(38, (B, E)), _rand(39, (F, E), 0.15), _rand(40, (E, F), 0.15)
+    ex, fy = E // gx, F // gy
+    exact = ffn_forward(X, W1, W2, act="relu", partition=2, n_slices=gx * gy, grid=grid)
+    yq = ffn_forward(X, W1, W2, act="relu", partition=2, n_slices=gx * gy, grid=grid, quant=True)
+    rnd = 2.0 ** -23
+    eA = np.zeros((B, F))
+    H = np.zeros((B, F))
+    for y in range(gy):
+        fs = slice(y * fy, (y + 1) * fy)
+        A = np.zeros((B, fy))
+        for x in range(gx):
+            P = X[:, x * ex:(x + 1) * ex] @ W1[fs, x * ex:(x + 1) * ex].T
+            _, d = q8_quantize(P.astype(np.float32))
+            dd = np.repeat(d.astype(np.float64), 32, axis=-1)
+            eA[:, fs] += dd * 0.5 + rnd * (np.abs(P) + dd)
+            A += P
+        H[:, fs] = relu(A)
+    bound = np.zeros((B, E))
+    for x in range(gx):
+        es = slice(x * ex, (x + 1) * ex)
+        for y in range(gy):
+            fs = slice(y * fy, (y + 1) * fy)
+            P2 = H[:, fs] @ W2[es, fs].T
+            e2 = eA[:, fs] @ np.abs(W2[es, fs]).T
+            hi = np.abs(P2) + e2
+            dmax = hi.reshape(B, -1, 32).max(axis=-1) / 127.0 * (1 + 4 * rnd)
+            dd = np.repeat(dmax, 32, axis=-1)
+            bound[:, es] += e2 + dd * 0.5 + rnd * (hi + dd)
+    diff = np.abs(yq - exact)
+    assert np.all(diff <= bound)
+    assert np.max(diff) > 0
