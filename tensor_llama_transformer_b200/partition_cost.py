@@ -57,14 +57,14 @@ def ffn_comm_1d(tokens: int, E: int, link_bw: float, dtype_bytes: int = BF16) ->
     return 2.0 * tokens * E * dtype_bytes / link_bw
 
 
-def ffn_comm_2d(tokens: int, E: int, n_chips: int, link_bw: float,
+def ffn_comm_2d(tokens: int, E: int, F: int, n_chips: int, link_bw: float,
                 dtype_bytes: int = BF16) -> float:
     """2D weight-stationary FFN (split along E and F, roughly square blocks per
     chip): activations are gathered along one mesh axis only, so the traffic falls
-    as 1 / sqrt(n). Reading taken: the paper's form for its F = 4 E models,
-    8 * tokens * E / sqrt(n) elements per layer, which equals the 1D traffic at
-    n = 16 (sqrt(n) = 4)."""
-    return 8.0 * tokens * E * dtype_bytes / (math.sqrt(n_chips) * link_bw)
+    as 1 / sqrt(n). Reading taken: 4 * tokens * sqrt(E * F / n) elements per
+    layer, which for the paper's F = 4 E models is 8 * tokens * E / sqrt(n) and
+    equals the 1D traffic at n = 16 (sqrt(n) = 4)."""
+    return 4.0 * tokens * math.sqrt(E * F / n_chips) * dtype_bytes / link_bw
 
 
 def ffn_comm_gathered(tokens: int, E: int, F: int, n_chips: int, link_bw: float,
@@ -85,7 +85,7 @@ def ffn_layout(tokens: int, E: int, F: int, n_chips: int, link_bw: float) -> str
     """'gathered' when moving weights is cheaper than moving activations
     (prefill-sized token counts), else 'stationary' (2D weight-stationary)."""
     t_g, _ = ffn_comm_gathered(tokens, E, F, n_chips, link_bw)
-    return "gathered" if t_g < ffn_comm_2d(tokens, E, n_chips, link_bw) else "stationary"
+    return "gathered" if t_g < ffn_comm_2d(tokens, E, F, n_chips, link_bw) else "stationary"
 
 
 def ffn_weight_read(E: int, F: int, layers: int, n_chips: int, mem_bw: float,
@@ -144,7 +144,7 @@ def decode_bound(m: Model, chip: Chip, n_chips: int, batch: int, context: int,
     t_w = m.params * weight_bytes / (n_chips * chip.mem_bw)
     t_kv = batch * context * kv_bytes_per_token(m, True) / n_chips / chip.mem_bw
     t_fl = 2.0 * m.params * batch / (n_chips * chip.peak_flops)
-    t_comm = ffn_comm_2d(batch, m.E, n_chips, chip.link_bw) * m.layers
+    t_comm = ffn_comm_2d(batch, m.E, m.F, n_chips, chip.link_bw) * m.layers
     return DecodeBound(t_w, t_kv, t_fl, t_comm, max(t_w + t_kv, t_fl) + t_comm)
 
 

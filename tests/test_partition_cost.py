@@ -23,7 +23,7 @@ def test_demo1_1d_comm_independent_of_chips():
 def test_demo1_2d_comm(n, ms):
     """Demo 1: 2D is 8.3 ms at n = 64 and 4.1 ms at n = 256, i.e. 1/2 and 1/4 of the 1D
     16.5 ms (the page's 8.3 is half of its rounded 16.5; the unrounded half is 8.249)."""
-    t = pc.ffn_comm_2d(512, M.E, n, CHIP.link_bw) * M.layers
+    t = pc.ffn_comm_2d(512, M.E, M.F, n, CHIP.link_bw) * M.layers
     assert t == pytest.approx(ms * 1e-3, abs=0.06e-3)
     t1 = pc.ffn_comm_1d(512, M.E, CHIP.link_bw) * M.layers
     assert t == pytest.approx(t1 * 4 / n ** 0.5, rel=1e-12)
@@ -32,9 +32,9 @@ def test_demo1_2d_comm(n, ms):
 def test_demo1_crossover_at_16_chips():
     """Demo 1: 1D and 2D are equal at sqrt(n) = 4 (F = 4E), and 2D is cheaper above 16 chips."""
     t1 = pc.ffn_comm_1d(512, M.E, CHIP.link_bw)
-    assert pc.ffn_comm_2d(512, M.E, 16, CHIP.link_bw) == pytest.approx(t1, rel=1e-12)
-    assert pc.ffn_comm_2d(512, M.E, 8, CHIP.link_bw) > t1
-    assert pc.ffn_comm_2d(512, M.E, 32, CHIP.link_bw) < t1
+    assert pc.ffn_comm_2d(512, M.E, M.F, 16, CHIP.link_bw) == pytest.approx(t1, rel=1e-12)
+    assert pc.ffn_comm_2d(512, M.E, M.F, 8, CHIP.link_bw) > t1
+    assert pc.ffn_comm_2d(512, M.E, M.F, 32, CHIP.link_bw) < t1
     assert M.F == 4 * M.E
 
 
@@ -86,7 +86,7 @@ def test_demo2_crossover_at_f_over_4():
     tokens; fewer tokens favour moving activations, more favour moving weights."""
     bl = F2 // 4
     t_g, N = pc.ffn_comm_gathered(bl, E2, F2, 64, CHIP.link_bw)
-    assert t_g == pytest.approx(pc.ffn_comm_2d(bl, E2, 64, CHIP.link_bw), rel=1e-12)
+    assert t_g == pytest.approx(pc.ffn_comm_2d(bl, E2, F2, 64, CHIP.link_bw), rel=1e-12)
     assert N == pytest.approx(4.0)  # sqrt(BL n / F)
     assert pc.ffn_layout(2048, E2, F2, 64, CHIP.link_bw) == "stationary"
     assert pc.ffn_layout(65536, E2, F2, 64, CHIP.link_bw) == "gathered"
@@ -97,8 +97,8 @@ def test_demo2_traffic_scaling():
     a = pc.ffn_comm_gathered(65536, E2, F2, 64, CHIP.link_bw)[0]
     b = pc.ffn_comm_gathered(262144, E2, F2, 64, CHIP.link_bw)[0]
     assert b / a == pytest.approx(2.0, rel=1e-12)
-    assert pc.ffn_comm_2d(262144, E2, 64, CHIP.link_bw) / pc.ffn_comm_2d(
-        65536, E2, 64, CHIP.link_bw) == pytest.approx(4.0, rel=1e-12)
+    assert pc.ffn_comm_2d(262144, E2, F2, 64, CHIP.link_bw) / pc.ffn_comm_2d(
+        65536, E2, F2, 64, CHIP.link_bw) == pytest.approx(4.0, rel=1e-12)
 
 
 def test_demo2_compute_share_last_row():
@@ -107,5 +107,20 @@ def test_demo2_compute_share_last_row():
     bl = 1048576
     comp = pc.ffn_compute(bl, E2, F2, 1, 64, CHIP.peak_flops)
     comm = min(pc.ffn_comm_gathered(bl, E2, F2, 64, CHIP.link_bw)[0],
-               pc.ffn_comm_2d(bl, E2, 64, CHIP.link_bw))
+               pc.ffn_comm_2d(bl, E2, F2, 64, CHIP.link_bw))
     assert round(comp / (comp + comm) * 100) == 94
+
+
+def test_2d_traffic_general_f():
+    """4 BL sqrt(E F / n): the paper's 8 BL E / sqrt(n) at F = 4 E (the printed values
+    above pin that case); for F = E it is half of that, and at any F the optimum
+    weight-gathered traffic (4 E sqrt(BL F / n)) meets it at BL = E."""
+    bw = CHIP.link_bw
+    E, n, bl = 8192, 64, 1024
+    assert pc.ffn_comm_2d(bl, E, 4 * E, n, bw) == pytest.approx(8.0 * bl * E * 2 / (8 * bw),
+                                                                rel=1e-12)
+    assert pc.ffn_comm_2d(bl, E, E, n, bw) == pytest.approx(
+        0.5 * pc.ffn_comm_2d(bl, E, 4 * E, n, bw), rel=1e-12)
+    for F in (E, 2 * E, 4 * E, 7 * E):
+        t_g, _ = pc.ffn_comm_gathered(E, E, F, n, bw)
+        assert t_g == pytest.approx(pc.ffn_comm_2d(E, E, F, n, bw), rel=1e-12)
