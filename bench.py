@@ -34,6 +34,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode tokens/s & HBM GB/s per TP-sliced block; FFN TFLOP/s at B=512 (1 B200)"
+# the workload of the headline (both arms print this same dict)
+CONFIG = {"workload": "C2: Llama-2-7B-shaped decoder block decode, dim 4096, 32x128 heads, "
+                      "SwiGLU 11008, KV 1024, batch 1, n=4 slices, Q8 sync buffers",
+          "batch": 1, "n_slices": 4, "sync_quant": True, "kv_len": 1024}
 STAGES = ["norm_qkv_rope", "attention", "wo_partials", "merge", "norm_w13_swiglu", "w2_partials",
           "merge2"]
 
@@ -62,6 +66,10 @@ def parse_args(argv=None):
     ap.add_argument("--profile-ffn-f", type=int, default=18432,
                     help="intermediate size of the --profile ffn case (PaLM: 73728)")
     ap.add_argument("--profile-steps", type=int, default=3)
+    ap.add_argument("--rank-exchange", action="store_true",
+                    help="also time the C2 block spread over the ranks (one slice group per GPU, "
+                         "NCCL all-gather of the sync buffers); on by default when N > 1, and with "
+                         "N = 1 it runs a one-rank NCCL group")
     return ap.parse_args(argv)
 
 
@@ -80,15 +88,59 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled while the GPU works.
 
+    Read-only NVML queries from a thread of this process (every 10 ms), so that a
+    short timed region still gets samples; nvidia-smi --query-gpu as the fallback
+    when the NVML bindings cannot load. Nothing here changes a GPU setting."""
+
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
+        import threading
+
+        self.rows = []  # (sm_mhz, sm_max_mhz, reasons)
         self.proc = None
-        self.path = None
+        self.thread = None
+        self.stop_flag = threading.Event()
+        self.source = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            bits = (pynvml.nvmlClocksEventReasonHwSlowdown,
+                    pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    pynvml.nvmlClocksEventReasonSwPowerCap)
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((float(sm), float(smax),
+                                          [n for n, b in zip(self.NAMES, bits) if r & b]))
+                    except Exception:
+                        pass
+                    self.stop_flag.wait(0.01)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml"
+            return
+        except Exception:
+            self.thread = None
+        self._start_smi(device_index)
+
+    def _start_smi(self, device_index: int):
         try:
             import torch
 
@@ -105,33 +157,38 @@ class ClockSampler:
         try:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi"
         except Exception:
             self.proc = None
 
+    def count(self) -> int:
+        return len(self.rows)
+
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+            for ln in open(self.path):
+                r = [p.strip() for p in ln.split(",")]
+                if len(r) >= 9 and r[1].replace(".", "").isdigit():
+                    self.rows.append((float(r[1]), float(r[2]) if r[2].replace(".", "").isdigit()
+                                      else None,
+                                      [self.NAMES[i] for i in range(4) if r[5 + i].lower() == "active"]))
+            os.unlink(self.path)
+        if not self.rows:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.out.close()
-        rows = []
-        for ln in open(self.path):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+        sm = [r[0] for r in self.rows]
+        smax = [r[1] for r in self.rows if r[1]]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted({n for r in self.rows for n in r[2]}),
+                "samples": len(self.rows), "source": self.source}
 
 
 def dist_setup():
@@ -232,9 +289,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": world,
         "steps": n, "warmup": warm, "ms_per_step": el / n * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "C2: Llama-2-7B-shaped decoder block decode, dim 4096, 32x128 heads, "
-                               "SwiGLU 11008, KV 1024, batch 1, n=4 slices, Q8 sync buffers",
-                   "batch": 1, "n_slices": 4, "sync_quant": True, "kv_len": 1024},
+        "config": dict(CONFIG),
         "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -321,8 +376,20 @@ def bench_block(args, world, rank, local):
     end.synchronize()
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
     ms = start.elapsed_time(end)
+    # a timed region of a few ms gives the sampler few or no samples: keep the same
+    # graph running (untimed) until it holds at least 20, at most 2 s more
+    t_extra, extra_replays = time.perf_counter(), 0
+    while clocks.count() < 20 and time.perf_counter() - t_extra < 2.0:
+        g.replay()
+        extra_replays += 1
+        if extra_replays % 20 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if clk is not None:
+        clk["window"] = (f"the timed region ({ms:.1f} ms) and {extra_replays} more untimed replays "
+                         f"of the same graph right after it")
     ms_max = allreduce_max(ms, world)
     # per-stage device time: one replay of the stage graph right after the timed region
     g_ev.replay()
@@ -333,6 +400,31 @@ def bench_block(args, world, rank, local):
             stage_ms[i] += ev[i].elapsed_time(ev[i + 1]) / S
     stage_ms_max = [allreduce_max(v, world) for v in stage_ms]
     del g, g_ev
+
+    # per-CTA timeline of the four slice GEMVs (%globaltimer stamps) in one replay of a
+    # captured step, relative to the first q/k/v CTA's start: the median over CTAs of
+    # start / activations staged / last stage consumed / end, and the latest end
+    nsm = torch.cuda.get_device_properties(local).multi_processor_count
+    tr = torch.zeros(nsm * tpb.TP_BLOCK_TRACE_SLOTS, dtype=torch.int64, device="cuda")
+    tpb.tp_block_set_trace(h, tr, tr.numel() * 8)
+    g_tr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_tr):
+        for _ in range(2):
+            fwd()
+    tpb.tp_block_set_trace(h, None, 0)
+    g_tr.replay()
+    torch.cuda.synchronize()
+    del g_tr
+    t = tr.view(nsm, -1).cpu().numpy().astype("float64")
+    timeline = {}
+    base = t[t[:, 0] > 0, 0].min()
+    for gi, name in enumerate(("qkv", "wo", "w13", "w2")):
+        cols = t[:, 4 * gi:4 * gi + 4]
+        cols = cols[cols[:, 0] > 0]
+        med = [round(float(statistics.median((cols[:, k] - base) / 1e3)), 2) for k in range(4)]
+        timeline[name] = {"start": med[0], "staged": med[1], "consumed": med[2], "end": med[3],
+                          "first_start": round(float((cols[:, 0].min() - base) / 1e3), 2),
+                          "last_end": round(float((cols[:, 3].max() - base) / 1e3), 2)}
 
     # end to end through the public API: host buffers, copies inside the timed region
     xh = torch.empty_like(dev.x, device="cpu").pin_memory()
@@ -363,8 +455,8 @@ def bench_block(args, world, rank, local):
     w13_bytes = 2 * s.ffn_dim * s.dim * 2 + B * s.dim * (1 + 4 / 32) + B * s.ffn_dim * 4
     w13_s = stage_ms_max[STAGES.index("norm_w13_swiglu")] / 1e3
     # batch 1 (weight-streaming path): q/k/v GEMV, attention splits, W_O GEMV (which also
-    # combines the splits), merge, W1/W3 GEMV, W2 GEMV, merge
-    launches_per_step = 7
+    # combines the splits and ends with the fused merge), W1/W3 GEMV, W2 GEMV (+ merge)
+    launches_per_step = 5
     res = {
         "tokens_per_s": world * B * K / (ms_max / 1e3), "ms_per_step": ms_max / K, "K": K,
         "block_gbs": (wbytes + kvbytes) / step_s / 1e9, "stage_us": {
@@ -379,10 +471,94 @@ def bench_block(args, world, rank, local):
         "e2e": {"value": world * B * E / e2e_s, "unit": "tokens/s",
                 "h2d_bytes_per_step": B * s.dim * 4 + B * 4, "d2h_bytes_per_step": B * s.dim * 4},
         "gpu_launches": launches_per_step * K, "clocks": clk, "inp": inp,
+        "gemv_timeline_us": timeline,
         "stage_sum_us": sum(stage_ms_max) * 1e3,
         "block_roofline_frac": (wbytes + kvbytes) / step_s / 1e9 / hbm,
     }
     return res
+
+
+def bench_rank_block(args, world, rank, local):
+    """The C2 block (Llama-2-7B shapes, Q8 sync, KV 1024, batch 1) with its slices
+    spread over the ranks, one GPU each (tp_block_rank_step: three phases per step
+    and two NCCL all-gathers of the sync buffers between them, every rank merging
+    all slices in slice order). n = 4 slices, or one per rank when world > 4.
+    Each rank's weights are its slices, drawn from its own seeded generator (a
+    timing workload: parity of this path is tests/test_gpu_tensor_parallel.py)."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import tensor_llama_transformer_b200 as tpb
+    from tensor_llama_transformer_b200 import tensor_parallel as tp
+
+    s = synth.C2
+    n = s.n_slices if s.n_slices % world == 0 else world
+    B, D, F, H, Hkv, hd = s.batch, s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim
+    if H % n or Hkv % n or n % world:
+        return {"error": f"C2 does not split into {n} slices over {world} ranks"}
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(2000 + rank)
+    Hr, Hkvr, Fr = H // world, Hkv // world, F // world
+    w = {"attn_norm": torch.ones(D, device="cuda"), "ffn_norm": torch.ones(D, device="cuda")}
+    for k, shp in (("wq", (Hr * hd, D)), ("wk", (Hkvr * hd, D)), ("wv", (Hkvr * hd, D)),
+                   ("wo", (D, Hr * hd)), ("w1", (Fr, D)), ("w3", (Fr, D)), ("w2", (D, Fr))):
+        w[k] = _randn_bf16(torch, gen, shp, s.w_std)
+    kc = _randn_bf16(torch, gen, (B, Hkvr, s.max_seq, hd), 1.0)
+    vc = _randn_bf16(torch, gen, (B, Hkvr, s.max_seq, hd), 1.0)
+    gx = torch.Generator(device="cuda")
+    gx.manual_seed(2999)  # the residual is replicated: the same values on every rank
+    x = torch.randn((B, D), generator=gx, device="cuda")
+    pos = torch.full((B,), s.pos, dtype=torch.int32, device="cuda")
+    dims = tpb.make_dims(D, H, Hkv, hd, F, s.vocab, B, s.max_seq, s.norm_eps, s.rope_theta)
+    rb = tp.RankBlock(dims, n, 1, rank, world, w)
+    sync_bytes = tpb.tp_block_rank_sync_bytes(rb.h, B)
+
+    def step():
+        rb.forward(x, kc, vc, pos, B)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    mode, g = "eager", None
+    try:  # NCCL collectives inside a CUDA graph (the communicator exists after the warm-up)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(10):
+                step()
+        g.replay()
+        torch.cuda.synchronize()
+        mode = "graph"
+    except Exception:
+        g = None
+        torch.cuda.synchronize()
+    dist.barrier()
+    reps = max(1, min(args.steps, 2000) // 10)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    dist.barrier()
+    a.record()
+    for _ in range(reps):
+        if g is not None:
+            g.replay()
+        else:
+            for _ in range(10):
+                step()
+    b.record()
+    b.synchronize()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = allreduce_max(a.elapsed_time(b), world) / (10 * reps)
+    err_off, _ = tpb.tp_block_buffer(rb.h, 7)
+    err = int(rb.ws[err_off:err_off + 4].view(torch.int32).item())
+    del g  # a graph holding NCCL calls goes before the process group
+    rb.close()
+    return {"world": world, "n_slices": n, "us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3),
+            "mode": mode, "steps": 10 * reps, "pipeline_error": err,
+            "exchange": "two NCCL all-gathers per step of every rank's Q8 sync buffers "
+                        f"({sync_bytes} bytes per rank each)",
+            "workload": "C2 block, batch 1, KV 1024, Q8 sync, slices spread over the ranks"}
 
 
 def _randn_bf16(torch, gen, shape, std):
@@ -769,6 +945,30 @@ def main(argv=None):
         return 0
     world, rank, local = dist_setup()
     res = bench_block(args, world, rank, local)
+    multi_rank = None
+    if world > 1 or args.rank_exchange:
+        own_group = False
+        try:
+            import torch.distributed as dist
+
+            if not dist.is_initialized():  # one rank: a one-rank NCCL group
+                import datetime
+                import socket
+
+                sk = socket.socket()
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+                sk.close()
+                dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                        world_size=1, timeout=datetime.timedelta(seconds=120),
+                                        device_id=torch.device("cuda", local))
+                own_group = True
+            multi_rank = bench_rank_block(args, world, rank, local)
+        except Exception as e:  # reported, not fatal: the headline does not depend on it
+            multi_rank = {"error": str(e)[:200]}
+        if own_group:
+            dist.destroy_process_group()
+        torch.cuda.empty_cache()
     ffn = None if args.no_ffn else bench_ffn(args)
     extra = None
     if not args.no_extra:
@@ -809,21 +1009,25 @@ def main(argv=None):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "dtype_detail": "bf16 weights, fp32 activations and accumulation, int8 Q8 sync buffers",
             "data": "synthetic",
-            "config": {"workload": "C2: Llama-2-7B-shaped decoder block decode, dim 4096, "
-                                   "32x128 heads, SwiGLU 11008, KV 1024, batch 1, n=4 slices, "
-                                   "Q8 sync buffers",
-                       "batch": 1, "n_slices": 4, "sync_quant": True, "kv_len": 1024,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (404.75 MB of weights per step), no flush"},
+            "config": dict(CONFIG),
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (404.75 MB of weights per step), no flush",
             "hbm_gbs": res["block_gbs"], "block_roofline_frac": res["block_roofline_frac"],
             "stage_us": res["stage_us"], "stage_sum_us": res["stage_sum_us"],
+            "gemv_timeline_us": res["gemv_timeline_us"],
+            "gemv_timeline_note": "one replay of a captured step: per slice GEMV the median over "
+                                  "CTAs of its start, activations staged, last weight stage "
+                                  "consumed and end (us from the first q/k/v CTA's start), and "
+                                  "the earliest start / latest end",
             "stage_note": "per-stage CUDA-event times from a replay of the same steps with an event "
                           "before every stage (serialised, so upper bounds); value and ms_per_step "
-                          "come from the event-free graph",
+                          "come from the event-free graph; the merges run in the W_O and W2 "
+                          "GEMVs' epilogues, so their own stages hold no kernel",
             "pdl": os.environ.get("TP_PDL", "1") != "0",
             "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
             "ffn_b512": ffn,
+            "multi_rank": multi_rank,
             "extra": extra,
         }
         print(json.dumps(line), flush=True)

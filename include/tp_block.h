@@ -113,7 +113,10 @@ typedef struct {
 
 typedef struct tp_block tp_block;
 
-/* Bytes of device workspace a block needs for dims->max_batch rows.
+/* Bytes of device workspace a block needs for dims->max_batch rows: the buffers
+ * the distributed-llama task list's Sync* steps move (the normalised input in
+ * its sync format, the row-split partials) and the kernels' scratch (q, the
+ * attention's context splits, the SwiGLU output, the error word and counters).
  * partition: TP_PART_1D or TP_PART_2D (2D applies to the FFN: a gx x gy grid, gx
  * the largest divisor of n with gx*gx <= n splits dim, gy = n/gx splits ffn_dim;
  * attention stays split by heads). sync_quant: 0 = float32 sync buffers,
@@ -174,9 +177,12 @@ TP_API int tp_block_forward_seq(tp_block* blk, float* x, void* k_cache, void* v_
 
 /* Offsets (bytes from the workspace base) and sizes of intermediate buffers,
  * for inspection by tests after a forward. which: 0 xnorm int8 codes [B,dim],
- * 1 xnorm scales float32 [B,dim/32], 2 xnorm float32 [B,dim], 3 q (rotated)
- * float32 [B,H*hd], 4 attention output float32 [B,H*hd], 5 partials float32
- * [n,B,dim], 6 SwiGLU output h float32 [B,F]. */
+ * 1 xnorm scales float32 [B,dim/32], 2 xnorm float32 [B,dim] (the RMSNorm
+ * output before the Q8 round trip; codes and scales are its Q8 form), 3 q
+ * (rotated) float32 [B,H*hd], 4 attention output float32 [B,H*hd], 5 partials
+ * float32 [n,B,dim], 6 SwiGLU output h float32 [B,F], 7 the kernels' error word
+ * (int32 at offset 0: nonzero when a bounded wait in a kernel gave up). Buffers
+ * 0-2 hold the last norm a call ran (the FFN's after a whole step). */
 TP_API int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* bytes);
 
 TP_API void tp_block_destroy(tp_block* blk);
@@ -273,7 +279,12 @@ TP_API int tp_block_set_persistent(tp_block* blk, int enable);
  * W_O partials (which precedes W1/W3), 14 end of the W1/W3 activation staging
  * (RMSNorm); 15 a duration, not a time: the nanoseconds the CTA's first consumer
  * thread spent waiting for weight stages during W1/W3. While events are set (tp_block_set_events) the
- * block runs as separate kernels and the trace is not written.
+ * block runs as separate kernels and the trace is not written. A forward on the
+ * kernel-per-step weight-streaming path (batch <= 5, persistent kernel off)
+ * writes instead, for each of its four slice GEMVs g (0 q/k/v, 1 W_O, 2 W1/W3,
+ * 3 W2) and CTA c of that launch, trace[c * TP_BLOCK_TRACE_SLOTS + 4g + k]: k = 0
+ * start, 1 activations staged, 2 last weight stage consumed, 3 end (after the
+ * epilogue and the fused merge); for batch > 2 the last launch of each wins.
  * Errors: TP_EINVAL (NULL handle, buffer too small). */
 #define TP_BLOCK_TRACE_SLOTS 16
 TP_API int tp_block_set_trace(tp_block* blk, void* trace, size_t bytes);
@@ -293,7 +304,10 @@ TP_API int tp_block_set_trace(tp_block* blk, void* trace, size_t bytes);
  *
  * - The first call on a device (with that device current) looks up the array's
  *   device address with cudaGetSymbolAddress; make that first call outside any
- *   stream capture. The call never allocates memory and frees none.
+ *   stream capture. Every later call made outside stream capture looks it up
+ *   again (a device reset moves the array); a call under capture uses the
+ *   address of the last call outside it. The call never allocates memory and
+ *   frees none.
  * - Configurations whose tp_block_workspace_bytes exceeds the array are refused
  *   with TP_ESCRATCH before anything is enqueued (the 7B block at batch 1 needs
  *   well under 1 MiB; batch 32 of the 70B shape does not fit).
@@ -306,6 +320,14 @@ TP_API int tp_block_forward_noalloc(const tp_dims* dims, int n_slices, int parti
                                     int sync_quant, const tp_block_weights* w, float* x,
                                     void* k_cache, void* v_cache, const int32_t* pos, int batch,
                                     tp_stream stream);
+
+/* The kernels' error word of the last tp_block_forward_noalloc on the current
+ * device (the array is private to the library, so the caller cannot read it
+ * from a workspace): copies it into *err (host memory) on `stream`; the value is
+ * there once the stream has reached this point. Nonzero means a bounded wait in
+ * a kernel gave up and that call's x and cache rows are not valid. Allocates
+ * nothing. Errors: TP_EINVAL (err NULL), TP_EARCH, TP_ECUDA. */
+TP_API int tp_block_noalloc_error(int* err, tp_stream stream);
 
 /* ------------------------------------------------------------------------- */
 /* Partitioned feed-forward layer  Y = act(X W1^T [, X W3^T]) W2^T.            */
@@ -323,14 +345,29 @@ typedef struct {
                          contraction (bf16 only, sync_quant must be 0) */
 } tp_ffn_desc;
 
-/* Workspace bytes for tp_ffn_forward with this descriptor. */
+/* Workspace bytes for tp_ffn_forward with this descriptor: the error word, the
+ * materialised partials (per slice for TP_MERGE_FAITHFUL; per E-slice of stage 1
+ * for 2D) and the hidden activations H [B,F]. Errors: TP_EINVAL (sizes that do
+ * not divide, see tp_ffn_forward), TP_ENOTSUP. */
 TP_API int tp_ffn_workspace_bytes(const tp_ffn_desc* d, size_t* out_bytes);
 
-/* X [B,E], W1 [F,E], W3 [F,E] (NULL unless SwiGLU), W2 [E,F] in d->dtype;
- * Y float32 [B,E] written. 1D: H_s = act(X W1_s^T) per F-slice (column split),
- * P_s = H_s W2_s^T (row split), Y = sum_s P_s. 2D: stage 1 sums over the E-slices,
- * stage 2 over the F-slices. Requirements: E % (32*grid_x) == 0 and F % (32*n)
- * == 0 (1D) or F % (32*grid_y) == 0 (2D). */
+/* The tensor-parallel FFN Y = act(X W1^T [, X W3^T]) W2^T.
+ * Defined by the aiterms.tw "Tensor Parallelism" glossary, "how it works" (the
+ * input replicated, Linear1 split by columns, the activation applied locally,
+ * Linear2 split by rows, one all-reduce of the partials) and by the Pope et al.
+ * lecture script, demo1_1d_vs_2d (1D splits F over n slices; 2D weight-stationary
+ * splits E over grid_x and F over grid_y); the ggmlR ggml_pp_dp_forward example
+ * fixes the activation after the first stage only.
+ * X [B,E], W1 [F,E], W3 [F,E] (NULL unless SwiGLU), W2 [E,F] in d->dtype, all
+ * device pointers, row-major, borrowed for the call; Y float32 [B,E] (device)
+ * written. 1D: H_s = act(X W1_s^T) per F-slice (column split), P_s = H_s W2_s^T
+ * (row split), Y = sum_s P_s in slice order. 2D: stage 1 sums over the E-slices
+ * before the activation, stage 2 over the F-slices. With sync_quant every
+ * materialised partial passes through the Q8 format before its sum.
+ * Requirements: E % (32*grid_x) == 0 and F % (32*n) == 0 (1D) or
+ * F % (32*grid_y) == 0 (2D); B >= 1. Errors: TP_EINVAL (sizes, flags, NULL),
+ * TP_EALIGN, TP_EWORKSPACE, TP_ENOTSUP (TP_MERGE_FUSED with float32 or with
+ * sync_quant), TP_EARCH, TP_ECUDA; nothing is enqueued on an error. */
 TP_API int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const void* W3,
                    const void* W2, float* Y, void* workspace, size_t ws_bytes, tp_stream stream);
 
@@ -339,6 +376,9 @@ TP_API int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, c
 /* ------------------------------------------------------------------------- */
 typedef struct tp_model tp_model;
 
+/* Workspace bytes of a model (the distributed-llama layer loop, NextBlock, then
+ * RmsFinal, Logits, MergeLogits): one block workspace shared by every layer, the
+ * residual and the final normalised rows. Errors: TP_EINVAL. */
 TP_API int tp_model_workspace_bytes(const tp_dims* dims, int n_layers, int n_slices, int partition,
                              int sync_quant, size_t* out_bytes);
 
@@ -369,9 +409,16 @@ TP_API void tp_model_destroy(tp_model* m);
 /* ------------------------------------------------------------------------- */
 /* Standalone Q8 codec of the sync buffers (same arithmetic as inside the block). */
 /* ------------------------------------------------------------------------- */
-/* x float32 [n] -> q int8 [n], d float32 [n/32]; n % 32 == 0. */
+/* The distributed-llama task list's Quantize* steps (QuantizeRmsAtt, QuantizeAtt,
+ * QuantizeRmfFfn, QuantizeFfn2) as one call: x float32 [n] -> q int8 [n],
+ * d float32 [n/32], device pointers. Per block of 32 consecutive values:
+ * d = amax / 127 (float32, rounded to nearest), q = x / d rounded half away from
+ * zero, clamped to +-127; an all-zero block gives d = 0 and zero codes.
+ * n % 32 == 0, n >= 0. Errors: TP_EINVAL, TP_EALIGN, TP_EARCH, TP_ECUDA. */
 TP_API int tp_quantize_q8(const float* x, int8_t* q, float* d, int64_t n, tp_stream stream);
-/* q int8 [n], d float32 [n/32] -> x float32 [n], x_i = q_i * d_block. */
+/* The Dequantize* steps (DequantizeAtt, DequantizeFfn2): q int8 [n],
+ * d float32 [n/32] -> x float32 [n], x_i = q_i * d_block (one float32 product).
+ * Errors as tp_quantize_q8. */
 TP_API int tp_dequantize_q8(const int8_t* q, const float* d, float* x, int64_t n, tp_stream stream);
 
 /* Human-readable name of a status code (static storage). */

@@ -100,6 +100,7 @@ _sig = {
     "tp_block_forward_noalloc": (C.c_int, [C.POINTER(tp_dims), C.c_int, C.c_int, C.c_int,
                                            C.POINTER(tp_block_weights), _P, _P, _P, _P, C.c_int,
                                            _P]),
+    "tp_block_noalloc_error": (C.c_int, [C.POINTER(C.c_int), _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -238,7 +239,8 @@ def tp_block_destroy(handle):
     _lib.tp_block_destroy(handle)
 
 
-TP_BLOCK_STAGES = 8
+TP_BLOCK_STAGES = 7  # stages of one block step (include/tp_block.h)
+TP_BLOCK_STAGE_EVENTS = TP_BLOCK_STAGES + 1  # events tp_block_set_events takes: one per stage, one after
 
 
 def tp_block_set_events(handle, events, n):
@@ -318,3 +320,14 @@ def tp_block_forward_noalloc(dims, n_slices, partition, sync_quant, weights, x, 
                                          C.byref(weights), _ptr(x), _ptr(k_cache), _ptr(v_cache),
                                          _ptr(pos), batch, _stream(stream)),
            "tp_block_forward_noalloc")
+
+
+def tp_block_noalloc_error(stream=None) -> int:
+    """The kernels' error word of the last tp_block_forward_noalloc on this device
+    (copied on `stream`; this call then synchronises the device; 0 = no wait gave up)."""
+    import torch
+
+    out = C.c_int(-1)
+    _check(_lib.tp_block_noalloc_error(C.byref(out), _stream(stream)), "tp_block_noalloc_error")
+    torch.cuda.synchronize()
+    return out.value

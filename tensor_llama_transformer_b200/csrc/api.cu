@@ -58,6 +58,16 @@ int set_smem_once(const void* kernel, int bytes) {
   return TP_OK;
 }
 
+// The W_O GEMV streams its weights beside the attention (one attention CTA per SM,
+// the GEMV's ring sized to fit next to it) unless TP_ATT_OVERLAP=0.
+bool att_overlap_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("TP_ATT_OVERLAP");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = getenv("TP_PDL");
@@ -84,8 +94,13 @@ enum Buf {
   BUF_COUNT
 };
 static_assert(BUF_SEND == TP_BUF_SEND && BUF_RECV == TP_BUF_RECV, "buffer ids of the C ABI");
-// BUF_ERR (16 bytes): int error word at byte 0; the persistent kernel's two grid
-// barrier counters at bytes 8 and 12.
+// BUF_ERR (placed first: byte 0 of every block workspace): the int error word at
+// byte 0; the persistent kernel's two grid barrier counters at bytes 8 and 12;
+// from byte 16 the fused merges' counters (int [max_batch][dim / 128] at most).
+// Every counter starts at zero and every launch leaves it so.
+constexpr size_t kCountersOff = 8;
+constexpr size_t kMergeCntOff = 16;
+int merge_pieces(int dim) { return (dim + kMergePiece - 1) / kMergePiece; }
 
 // Largest contraction splits of the batched-decode GEMMs (the planes are sized for them).
 constexpr int kQkvMaxParts = 8, kW13MaxParts = 4, kW2MaxParts = 2;
@@ -171,7 +186,15 @@ Layout block_layout(const Cfg& c) {
   // row-split partials: n slices (x kW2MaxParts contraction parts on the tensor path)
   L.size[BUF_PART] = (size_t)c.n * (c.d.max_batch >= kTcMinBatch ? kW2MaxParts : 1) * B * D * 4;
   L.size[BUF_H] = B * F * 4;
-  L.size[BUF_ERR] = 16;
+  // counters: the GEMV's per (batch group, 512-output piece), the GEMM's per 128-row tile
+  {
+    const size_t kd = (size_t)c.d.n_kv_heads * c.d.head_dim;
+    size_t cnt = B * (size_t)(c.d.dim / 128);
+    const size_t tiles_qkv = (QD + 127) / 128 + 2 * ((kd + 127) / 128), tiles_f = (F + 127) / 128;
+    if (tiles_qkv > cnt) cnt = tiles_qkv;
+    if (tiles_f > cnt) cnt = tiles_f;
+    L.size[BUF_ERR] = kMergeCntOff + cnt * 4;
+  }
   L.size[BUF_PO] = B * c.d.n_heads * (size_t)c.nchunk * c.d.head_dim * 4;
   L.size[BUF_PML] = B * c.d.n_heads * (size_t)c.nchunk * 2 * 4;
   const size_t pa = c.partition == TP_PART_2D ? (size_t)c.gx * B * F * 4 : 0;
@@ -195,8 +218,11 @@ Layout block_layout(const Cfg& c) {
     const size_t w13 = kW13MaxParts * B * 2 * F * 4;
     L.size[BUF_PLANE] = qkv > w13 ? qkv : w13;
   }
-  size_t o = 0;
+  // the error word first, at byte 0 of the workspace; then the others in id order
+  size_t o = align256(L.size[BUF_ERR]);
+  L.off[BUF_ERR] = 0;
   for (int i = 0; i < BUF_COUNT; ++i) {
+    if (i == BUF_ERR) continue;
     L.off[i] = o;
     o += align256(L.size[i]);
   }
@@ -216,8 +242,8 @@ struct tp_block {
   uint8_t* ws;
   size_t ws_bytes;
   void* const* events;  // optional per-stage timing events (borrowed)
-  bool bar_ready;       // grid barrier counters known to be zero
-  unsigned long long* trace;  // optional phase trace of the persistent kernel
+  bool bar_ready;       // the counters of BUF_ERR (grid barriers, merge pieces) known to be zero
+  unsigned long long* trace;  // optional phase trace (persistent kernel, or the four slice GEMVs)
   int persistent;       // use the persistent kernel where the shapes allow (batch 1-2, 1D)
   bool wq8;             // int8 weights: w holds the codes, wd their scales
   const float* wd_q;
@@ -260,9 +286,8 @@ void set_norm_input(const tp_block* b, GemvArgs& a, const float* x, const float*
   if (b->c.quant) {
     a.xq_out = at<int8_t>(b, BUF_XQ);
     a.xd_out = at<float>(b, BUF_XD);
-  } else {
-    a.xn_out = at<float>(b, BUF_XN);
   }
+  a.xn_out = at<float>(b, BUF_XN);  // the float32 RMSNorm output (before Q8)
 }
 
 // Records the caller's timing event before `stage`. Inside stream capture the
@@ -289,6 +314,25 @@ int merge_step(tp_block* blk, float* x, const float* part, int nseg, int parts, 
   if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts);
   return launch_merge_sync(x, at<uint8_t>(blk, BUF_RECV), c.n * c.world, batch, c.d.dim, c.quant,
                            ssq, s);
+}
+
+// a6 / a10 fused into the row-split GEMV that produces the partials (whole
+// block on the weight-streaming kernels): the CTA that completes a piece of the
+// output merges it into x and leaves the piece's sum of squares.
+void set_fused_merge(tp_block* blk, GemvArgs& a, float* x) {
+  a.merge_x = x;
+  a.merge_ssq = at<float>(blk, BUF_SSQ);
+  a.merge_cnt = reinterpret_cast<int*>(blk->ws + blk->L.off[BUF_ERR] + kMergeCntOff);
+  a.merge_quant = blk->c.quant;
+  a.merge_pieces = merge_pieces(blk->c.d.dim);
+}
+
+// Trace slots 4g .. 4g+3 of every CTA for the slice GEMV g (0 q/k/v, 1 W_O,
+// 2 W1/W3, 3 W2) when a trace buffer is set.
+void set_gemv_trace(const tp_block* blk, GemvArgs& a, int g) {
+  if (!blk->trace) return;
+  a.trace = blk->trace + 4 * g;
+  a.trace_stride = TP_BLOCK_TRACE_SLOTS;
 }
 
 // End of a rank block's phase 0 / 1: this rank's partials into its send buffer.
@@ -347,12 +391,15 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     n.quant = c.quant;
     n.xq = c.quant ? at<int8_t>(blk, BUF_XQ) : nullptr;
     n.xd = c.quant ? at<float>(blk, BUF_XD) : nullptr;
-    n.xn = c.quant ? nullptr : at<float>(blk, BUF_XN);
+    n.xn = at<float>(blk, BUF_XN);
     n.xb = xb;
     return launch_norm_rows(n, batch, s);
   };
+  // fin: the step fused into the GEMM's epilogue after the last plane of a tile
+  int* fin_cnt = reinterpret_cast<int*>(blk->ws + blk->L.off[BUF_ERR] + kMergeCntOff);
   auto gemm = [&](const void* A0, int m0, const void* A1, int m1, const void* A2, int m2, int nA,
-                  int64_t lda, const uint16_t* Bop, int K, int nseg, float* out, int64_t rows) {
+                  int64_t lda, const uint16_t* Bop, int K, int nseg, float* out, int64_t rows,
+                  TcFinish fin) {
     TcGemm g{};
     g.A[0] = A0;
     g.A[1] = A1;
@@ -372,37 +419,47 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     g.ldo = rows;
     g.out_seg = (int64_t)batch * rows;
     g.err = err;
+    g.indep = TC_INDEP_A;  // the weights
+    g.fin = fin;
+    if (fin.kind != TC_FIN_NONE) g.fin.cnt = fin_cnt;
     return launch_tc_gemm(g, s);
   };
 
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
   int p2 = 1;
+  TcFinish none{};
+  auto merge_fin = [&](int parts) {  // a6 / a10 in the epilogue (whole block)
+    TcFinish f{};
+    if (c.world != 0) return f;
+    f.kind = TC_FIN_MERGE;
+    f.parts = parts;
+    f.x = x;
+    f.ssq = at<float>(blk, BUF_SSQ);
+    f.quant = c.quant;
+    return f;
+  };
   if (phase <= 0) {
     // a1-a4
     if ((rc = stage_mark(blk, 0, s))) return rc;
     if ((rc = norm(blk->w.attn_norm, chained ? at<float>(blk, BUF_SSQ) : nullptr))) return rc;
     const int qkv_tiles = (QD + 127) / 128 + 2 * ((KD + 127) / 128);
     const int parts = tc_split(qkv_tiles, D, QD + 2 * KD, batch, kQkvMaxParts);
+    // the parts' sum, RoPE, q and the cache rows in the epilogue (llamaQkv + the
+    // cache merge of llamaMultiheadAtt)
+    TcFinish fq{};
+    fq.kind = TC_FIN_QKV;
+    fq.parts = parts;
+    fq.q = at<float>(blk, BUF_Q);
+    fq.kc = static_cast<uint16_t*>(kc);
+    fq.vc = static_cast<uint16_t*>(vc);
+    fq.pos = pos;
+    fq.seq = seq;
+    fq.theta = d.rope_theta;
+    fq.n_kv_heads = Hkv;
+    fq.max_seq = d.max_seq;
     if ((rc = gemm(blk->w.wq, QD, blk->w.wk, KD, blk->w.wv, KD, 3, D, xb, D / parts, parts, plane,
-                   QD + 2 * KD)))
+                   QD + 2 * KD, fq)))
       return rc;
-    {
-      QkvFinalizeArgs f{};
-      f.plane = plane;
-      f.parts = parts;
-      f.batch = batch;
-      f.qd = QD;
-      f.kd = KD;
-      f.pos = pos;
-      f.seq = seq;
-      f.theta = d.rope_theta;
-      f.q = at<float>(blk, BUF_Q);
-      f.kc = static_cast<uint16_t*>(kc);
-      f.vc = static_cast<uint16_t*>(vc);
-      f.n_kv_heads = Hkv;
-      f.max_seq = d.max_seq;
-      if ((rc = launch_qkv_finalize(f, s))) return rc;
-    }
     // a4
     if ((rc = stage_mark(blk, 1, s))) return rc;
     {
@@ -427,15 +484,16 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     }
     // a5: W_O row-split partials (segment s = slice s's head columns)
     if ((rc = stage_mark(blk, 2, s))) return rc;
+    // (a6 fused into its epilogue for the whole block)
     if ((rc = gemm(blk->w.wo, D, nullptr, 0, nullptr, 0, 1, QD, at<uint16_t>(blk, BUF_ATTB), QD / c.n,
-                   c.n, part, D)))
+                   c.n, part, D, merge_fin(1))))
       return rc;
     if (phase == 0) return pack_step(blk, part, 1, batch, s);
   }
   if (phase <= 1) {
-    // a6
+    // a6 (a rank block: the merge of the gathered buffer)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    if (c.world != 0 && (rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
     // a7-a8
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if ((rc = norm(blk->w.ffn_norm, at<float>(blk, BUF_SSQ)))) return rc;
@@ -443,14 +501,21 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     uint16_t* hb = at<uint16_t>(blk, BUF_HB);
     if (c.partition == TP_PART_1D) {
       const int p13 = tc_split(2 * ((F + 127) / 128), D, 2 * F, batch, kW13MaxParts);
-      if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F)))
+      TcFinish fs{};  // silu(W1 row) * W3 row in the epilogue (llamaFfn)
+      fs.kind = TC_FIN_SWIGLU;
+      fs.parts = p13;
+      fs.h = hbuf;
+      fs.hb = hb;
+      if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F,
+                     fs)))
         return rc;
-      if ((rc = launch_swiglu_finalize(plane, p13, F, batch, hbuf, hb, s))) return rc;
     } else {
       float* pa = at<float>(blk, BUF_PA);
       float* pb = at<float>(blk, BUF_PB);
-      if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F))) return rc;
-      if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F))) return rc;
+      if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F, none)))
+        return rc;
+      if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F, none)))
+        return rc;
       FfnMergeArgs m{};
       m.P1 = pa;
       m.P3 = pb;
@@ -470,13 +535,13 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     p2 = tc_split((int64_t)nseg2 * ((D + 127) / 128), F / nseg2, (int64_t)nseg2 * D, batch,
                   kW2MaxParts);
     if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2 / p2, nseg2 * p2, part,
-                   D)))
+                   D, merge_fin(p2))))
       return rc;
     if (phase == 1) return pack_step(blk, part, p2, batch, s);
   }
-  // a10
+  // a10 (fused into the W2 GEMM's epilogue for the whole block)
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = merge_step(blk, x, part, nseg2, p2, batch, s))) return rc;
+  if (c.world != 0 && (rc = merge_step(blk, x, part, nseg2, p2, batch, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -525,12 +590,8 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
   a.ssq = at<float>(blk, BUF_SSQ);
   a.h = at<float>(blk, BUF_H);
   a.err = at<int>(blk, BUF_ERR);
-  a.bar = reinterpret_cast<unsigned*>(blk->ws + blk->L.off[BUF_ERR] + 8);
+  a.bar = reinterpret_cast<unsigned*>(blk->ws + blk->L.off[BUF_ERR] + kCountersOff);
   a.trace = blk->trace;
-  if (!blk->bar_ready) {  // counters start at zero; each launch leaves them so
-    if (cudaMemsetAsync(a.bar, 0, 8, s) != cudaSuccess) return TP_ECUDA;
-    blk->bar_ready = true;
-  }
   *used = true;
   return launch_block_persistent(a, batch, s);
 }
@@ -548,6 +609,12 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
                        cudaStream_t s, bool chained = false, int phase = -1,
                        const int32_t* seq = nullptr, int nseq = 0) {
   if (blk->wq8 && batch >= kTcMinBatch) return TP_ENOTSUP;
+  if (!blk->bar_ready) {  // the counters start at zero (first use of this workspace)
+    uint8_t* cnt = blk->ws + blk->L.off[BUF_ERR] + kCountersOff;
+    if (cudaMemsetAsync(cnt, 0, blk->L.size[BUF_ERR] - kCountersOff, s) != cudaSuccess)
+      return TP_ECUDA;
+    blk->bar_ready = true;
+  }
   if (batch >= kTcMinBatch)
     return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained, phase, seq, nseq);
   if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent &&
@@ -564,6 +631,10 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   float* part = at<float>(blk, BUF_PART);
   float* hbuf = at<float>(blk, BUF_H);
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
+  // context splits of the attention, which the W_O GEMV's staging combines; with
+  // the overlap on, one attention CTA per SM leaves room for the W_O GEMV's CTA
+  const bool overlap = att_overlap_enabled() && pdl_enabled();
+  const int att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq, overlap ? 1 : 2);
 
   if (phase <= 0) {
     // a1-a4: RMSNorm (+Q8, the buffer every slice reads) fused into the q/k/v slice
@@ -601,6 +672,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.max_seq = d.max_seq;
       a.theta = d.rope_theta;
       a.err = at<int>(blk, BUF_ERR);
+      set_gemv_trace(blk, a, 0);
       if ((rc = launch_gemv(a, EPI_QKV, s))) return rc;
     }
     // a4: attention per head slice (context chunks, then their combination)
@@ -621,6 +693,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.part_o = at<float>(blk, BUF_PO);
       a.part_ml = at<float>(blk, BUF_PML);
       a.att = at<float>(blk, BUF_ATT);
+      a.nsplit = att_nsplit;
       a.err = at<int>(blk, BUF_ERR);
       if ((rc = launch_attention(a, s, false))) return rc;  // W_O's staging combines the splits
     }
@@ -636,7 +709,8 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.nseg = c.n;
       a.att_po = at<float>(blk, BUF_PO);
       a.att_pml = at<float>(blk, BUF_PML);
-      a.att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq);
+      a.att_nsplit = att_nsplit;
+      if (overlap) a.co_smem = attention_cta_smem();
       a.att_out = at<float>(blk, BUF_ATT);
       a.pos = pos;
       a.n_heads = H;
@@ -646,14 +720,17 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.out_seg = (int64_t)batch * D;
       a.ldo = D;
       a.err = at<int>(blk, BUF_ERR);
+      set_gemv_trace(blk, a, 1);
+      if (c.world == 0) set_fused_merge(blk, a, x);  // a6 in the epilogue
       if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
     if (phase == 0) return pack_step(blk, part, 1, batch, s);
   }
   if (phase <= 1) {
-    // a6: sync + dequantise + merge into the residual
+    // a6: sync + dequantise + merge into the residual (a rank block: of the
+    // gathered buffer; the whole block did it in the W_O GEMV's epilogue)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    if (c.world != 0 && (rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
     // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if (c.partition == TP_PART_1D) {
@@ -675,6 +752,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.out = hbuf;
       a.ldo = F;
       a.err = at<int>(blk, BUF_ERR);
+      set_gemv_trace(blk, a, 2);
       if ((rc = launch_gemv(a, EPI_SWIGLU, s))) return rc;
     } else {
       // 2D stage 1: partials over the gx dim-slices for W1 and W3, merged with SwiGLU
@@ -726,13 +804,15 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.out_seg = (int64_t)batch * D;
       a.ldo = D;
       a.err = at<int>(blk, BUF_ERR);
+      set_gemv_trace(blk, a, 3);
+      if (c.world == 0) set_fused_merge(blk, a, x);  // a10 in the epilogue
       if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
     if (phase == 1) return pack_step(blk, part, 1, batch, s);
   }
-  // a10: sync + dequantise + merge
+  // a10: sync + dequantise + merge (fused into the W2 GEMV for the whole block)
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = merge_step(blk, x, part, nseg2, 1, batch, s))) return rc;
+  if (c.world != 0 && (rc = merge_step(blk, x, part, nseg2, 1, batch, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -992,7 +1072,7 @@ int block_forward_on_workspace(const tp_dims* dims, int n_slices, int partition,
   blk.events = nullptr;
   if (cudaMemsetAsync(blk.ws + blk.L.off[BUF_ERR], 0, blk.L.size[BUF_ERR], stream) != cudaSuccess)
     return TP_ECUDA;
-  blk.bar_ready = true;  // the memsets above cover the persistent kernel's counters
+  blk.bar_ready = true;  // the memset above covers every counter of BUF_ERR
   blk.trace = nullptr;
   blk.persistent = persistent_default() ? 1 : 0;
   blk.wq8 = false;

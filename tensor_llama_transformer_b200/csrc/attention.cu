@@ -147,13 +147,14 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   const int h0 = kvh * (a.H / a.Hkv) + (blockIdx.y - kvh * hgroups) * G;  // first query head
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
-  pdl_wait();  // q and the cache rows at pos come from the q/k/v kernel
+  // pos and seq are the caller's inputs (no kernel of the step writes them)
   const int P = a.pos[b] + 1;
   const int ntiles = (P + kTile - 1) / kTile;
   const int tpc = tiles_per_split(P, nsplit);
   const int i0 = split * tpc, i1 = min(ntiles, i0 + tpc);
   const size_t pbase = ((size_t)b * a.H + (size_t)h0) * nsplit + split;
   if (i0 >= i1) {  // nothing left for this split: an empty partial (m = -inf, l = 0)
+    pdl_wait();
     if (threadIdx.x < G) {
       a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 0] = -INFINITY;
       a.part_ml[(pbase + (size_t)threadIdx.x * nsplit) * 2 + 1] = 0.f;
@@ -162,6 +163,10 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
   }
   const int sq = a.seq ? a.seq[b] : b;  // the row's cache sequence
   const int row_base = (sq * a.Hkv + kvh) * a.max_seq;
+  // The q/k/v kernel before this one writes q and, in the cache, the row's
+  // position pos only (with a sequence map, the positions of every row of the
+  // step): the tiles below pos's tile are streamed before waiting for it.
+  const int first_dep = a.seq ? i0 : ntiles - 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -170,24 +175,19 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
     }
     mbar_init_fence();
   }
-  // Q of the group's heads scaled by 1/sqrt(hd): hi in row g, lo in row g + 8
-  const float scale = 1.0f / sqrtf((float)kHeadDim);
-  for (int i = threadIdx.x; i < 8 * kHeadDim; i += kAThreads) {
-    const int g = i / kHeadDim, d = i - g * kHeadDim;
-    uint16_t hi = 0, lo = 0;
-    if (g < G)
-      bf16_split(a.q[((size_t)b * a.H + (size_t)h0 + g) * kHeadDim + d] * scale, hi, lo);
-    qs[g * kQStride + d] = hi;
-    qs[(g + 8) * kQStride + d] = lo;
-  }
   __syncthreads();
 
   if (warp == kCWarps) {
     // ------------------------------------------------------------ producer warp
     if (lane == 0) {
       const uint64_t pol = l2_evict_first();  // cache tiles are read once per step
+      bool waited = false;
       for (int i = i0; i < i1; ++i) {
         const int k = i - i0, s = k % kStages;
+        if (i >= first_dep && !waited) {
+          pdl_wait();
+          waited = true;
+        }
         if (!mbar_wait(&empty[s], ((uint32_t)(k / kStages) & 1u) ^ 1u, a.err)) break;
         mbar_expect_tx(&full[s], kStageBytes);
         uint8_t* st = smem + s * kStageBytes;
@@ -197,9 +197,24 @@ __global__ void __launch_bounds__(kAThreads) k_attn_split(const __grid_constant_
         tma_load_2d_hint(st + 2 * kBox, &mV, 0, y, &full[s], pol);
         tma_load_2d_hint(st + 3 * kBox, &mV, 64, y, &full[s], pol);
       }
+      if (!waited) pdl_wait();
     }
+    __syncwarp();
+    pdl_wait();  // (every thread: the partials below overwrite a buffer earlier kernels read)
   } else {
     // ------------------------------------------------------------ consumer warps
+    pdl_wait();  // q comes from the q/k/v kernel
+    // Q of the group's heads scaled by 1/sqrt(hd): hi in row g, lo in row g + 8
+    const float scale = 1.0f / sqrtf((float)kHeadDim);
+    for (int i = threadIdx.x; i < 8 * kHeadDim; i += kCWarps * 32) {
+      const int gq = i / kHeadDim, d = i - gq * kHeadDim;
+      uint16_t hi = 0, lo = 0;
+      if (gq < G)
+        bf16_split(a.q[((size_t)b * a.H + (size_t)h0 + gq) * kHeadDim + d] * scale, hi, lo);
+      qs[gq * kQStride + d] = hi;
+      qs[(gq + 8) * kQStride + d] = lo;
+    }
+    consumers_sync(kCWarps * 32);
     const int g = lane >> 2;  // the head row whose scores this thread holds
     uint32_t qa[8][4];        // A fragments of Q, one per 16-dim step
     {
@@ -483,9 +498,9 @@ int attention_max_splits(int max_seq) { return (max_seq + kTile - 1) / kTile; }
 // Splits per (batch row, kv head): the count that minimises waves x (tiles per
 // CTA + 1), two CTAs resident per SM, over a context of max_seq positions. The
 // kernels divide the actual context (pos + 1) over that many splits.
-int attention_splits(int B, int Hkv, int max_seq) {
+int attention_splits(int B, int Hkv, int max_seq, int per_sm = 2) {
   const int T = attention_max_splits(max_seq);
-  const long slots = 2L * num_sms();
+  const long slots = (long)per_sm * num_sms();
   int best = 1;
   long best_cost = -1;
   for (int sp = 1; sp <= T; ++sp) {
@@ -501,10 +516,20 @@ int attention_splits(int B, int Hkv, int max_seq) {
   return best;
 }
 
-int attention_nsplit(int B, int H, int Hkv, int max_seq) {
+int attention_nsplit(int B, int H, int Hkv, int max_seq, int per_sm) {
   const int G = H / Hkv;
   const int hgroups = G > 8 ? G / 8 : 1;  // CTAs per kv head
-  return attention_splits(B, Hkv * hgroups, max_seq);
+  return attention_splits(B, Hkv * hgroups, max_seq, per_sm);
+}
+
+int attention_cta_smem() {
+  static int bytes = [] {
+    cudaFuncAttributes fa{};
+    const int st = cudaFuncGetAttributes(&fa, (const void*)k_attn_split<1>) == cudaSuccess
+                       ? (int)fa.sharedSizeBytes : 1024;
+    return kSmemBytes + st;
+  }();
+  return bytes;
 }
 
 int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {
@@ -512,8 +537,9 @@ int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {
   // rows mapped to cache sequences share tiles (k_attn_rows) when the splits are
   // combined here and a CTA holds at least two rows
   const bool shared = a.seq && combine && G <= 4;
-  const int nsplit = shared ? attention_splits((a.B + 8 / G - 1) / (8 / G), a.Hkv, a.max_seq)
-                            : attention_nsplit(a.B, a.H, a.Hkv, a.max_seq);
+  const int nsplit = a.nsplit > 0 ? a.nsplit
+                     : shared ? attention_splits((a.B + 8 / G - 1) / (8 / G), a.Hkv, a.max_seq)
+                              : attention_nsplit(a.B, a.H, a.Hkv, a.max_seq);
   if (nsplit > a.nchunk) return TP_EINVAL;
   if (!aligned16(a.kc) || !aligned16(a.vc)) return TP_EALIGN;
   CUtensorMap mK, mV;

@@ -474,6 +474,7 @@ TP_DEV void stage_norm(const BpArgs& a, float4* xs, const float* xsrc, bool src_
         load8(gain + 8 * (size_t)v, gg);
 #pragma unroll
         for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(__fmul_rn(xm[e], rstd), gg[e]);
+        if (publish) store8(a.xn + e0, y);  // before any Q8 round trip
       }
       if (a.quant) {
         float am = 0.f;
@@ -496,7 +497,6 @@ TP_DEV void stage_norm(const BpArgs& a, float4* xs, const float* xsrc, bool src_
         }
       }
       if (in) {
-        if (publish) store8(a.xn + e0, y);
         xs[b * nv + v] = make_float4(y[0], y[1], y[2], y[3]);
         xs[(NB + b) * nv + v] = make_float4(y[4], y[5], y[6], y[7]);
       }

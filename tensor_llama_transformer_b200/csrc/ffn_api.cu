@@ -121,6 +121,7 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
     g.out = H;
     g.ldo = F;
     g.err = err;
+    g.indep = TC_INDEP_B;  // the weights
     rc = launch_tc_gemm(g, s);
     if (rc) return rc;
     // stage 2: Y = H W2^T over the full F
@@ -138,6 +139,7 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
     g2.out = Y;
     g2.ldo = E;
     g2.err = err;
+    g2.indep = TC_INDEP_B;
     return launch_tc_gemm(g2, s);
   }
 
@@ -162,6 +164,7 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
     g.ldo = N;
     g.out_seg = (int64_t)M * N;
     g.err = err;
+    g.indep = TC_INDEP_B;  // the weights
     return launch_tc_gemm(g, s);
   };
 

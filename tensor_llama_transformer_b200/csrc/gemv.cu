@@ -36,6 +36,8 @@
 // EPI_SWIGLU stores silu(a)*b (llamaFfn); EPI_QKV applies RoPE to q and k
 // pairs, stores rotated q, and writes k and v into the bf16 cache at pos
 // (llamaMultiheadAtt's "merge kv-cache, add RoPE encoding").
+#include <cstdlib>
+
 #include "kernels.cuh"
 #include "pipeline.cuh"
 
@@ -96,8 +98,78 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
                               const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
                               int part, int Q, int cb, int ce, int lane);
 
+// The merge fused into a row-split product's epilogue (distributed-llama
+// SyncAtt + DequantizeAtt + MergeAtt, and the Ffn2 twins): the CTA counts the
+// partial values it stored per piece of kMergePiece outputs; the CTA whose
+// count completes a piece (all nseg slices' partials of it stored) sums the
+// piece's slices in slice order through the sync format and adds the sum to the
+// residual, as k_merge does, then writes the sums of squares of its 128-value
+// chunks for the next RMSNorm and clears the counter. Every thread of the CTA
+// calls this.
+template <int NB>
+TP_DEV void fused_merge(const GemvArgs& a, int R0, int nrows, int rps) {
+  __shared__ int s_done[kMaxMergePieces];
+  __shared__ int s_ndone;
+  const int t = threadIdx.x;
+  int count = 0, total = 0;
+  if (t < a.merge_pieces) {  // this CTA's outputs inside piece t, over the segments it covers
+    const int f0 = t * kMergePiece, f1 = min(f0 + kMergePiece, rps);
+    total = a.nseg * (f1 - f0);
+    for (int sg = R0 / rps; sg <= (R0 + nrows - 1) / rps; ++sg) {
+      const int lo = max(R0, sg * rps + f0), hi = min(R0 + nrows, sg * rps + f1);
+      count += max(0, hi - lo);
+    }
+  }
+  if (t == 0) s_ndone = 0;
+  __threadfence();  // each thread's partial stores, before the counts that publish them
+  __syncthreads();
+  if (count > 0) {
+    int* c = a.merge_cnt + (size_t)a.b0 * a.merge_pieces + t;
+    if (atomicAdd(c, count) + count == total) s_done[atomicAdd(&s_ndone, 1)] = t;
+  }
+  __syncthreads();
+  const int nd = s_ndone;
+  if (nd == 0) return;
+  __threadfence();  // the other CTAs' partials, after their counts
+  const int b = t >> 7, i4 = t & 127;  // 128 threads (4 warps) per batch row
+  for (int k = 0; k < nd; ++k) {
+    const int p = s_done[k];
+    const int f0 = p * kMergePiece, n4 = (min(f0 + kMergePiece, rps) - f0) >> 2;
+    // whole warps: n4 is a multiple of 32, so an 8-lane Q8 group is always complete
+    const bool in = b < a.nb && i4 < n4;
+    const int gb = a.b0 + b;
+    float sq = 0.f;
+    if (in) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sg = 0; sg < a.nseg; ++sg) {
+        float4 v = __ldcg(reinterpret_cast<const float4*>(a.out + (size_t)sg * a.out_seg +
+                                                          (size_t)gb * a.ldo + f0) + i4);
+        if (a.merge_quant) q8_roundtrip4(v);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      float4* xr = reinterpret_cast<float4*>(a.merge_x + (size_t)gb * rps + f0) + i4;
+      float4 x = __ldcg(xr);
+      x.x += acc.x;
+      x.y += acc.y;
+      x.z += acc.z;
+      x.w += acc.w;
+      *xr = x;
+      sq = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    }
+    if (t < NB * 128) {  // each warp's 128 values: one sum of squares (as k_merge)
+      sq = warp_sum(sq);
+      if ((t & 31) == 0 && in)
+        a.merge_ssq[(size_t)gb * (rps >> 7) + (f0 >> 7) + ((t >> 5) & 3)] = sq;
+    }
+    if (t == 0) a.merge_cnt[(size_t)a.b0 * a.merge_pieces + p] = 0;
+  }
+}
+
 template <int NB, int EPI, bool WQ8>
-__global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
+__global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_rstd[NB];
   __shared__ float s_red[8][NB];
@@ -130,6 +202,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   }
   __syncthreads();
   pdl_launch_dependents();
+  unsigned long long* tr = a.trace ? a.trace + (size_t)blockIdx.x * a.trace_stride : nullptr;
+  if (tr && threadIdx.x == 0) tr[0] = gtimer();
 
   if (warp == nc) {
     // ---------------------------------------------------------------- producer
@@ -332,6 +406,12 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
                 xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
               }
             }
+            // the normalised value before any Q8 round trip (float32 RMSNorm output)
+            if (a.gain && publish && in && a.xn_out) {
+              *reinterpret_cast<float4*>(a.xn_out + e0) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+              *reinterpret_cast<float4*>(a.xn_out + e0 + 4) =
+                  make_float4(xv[4], xv[5], xv[6], xv[7]);
+            }
             if (WQ8) {
               // the integer products need Q8 activations: the codes read, or those of xv
               uint2 qc = qin;
@@ -380,11 +460,6 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
                 if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = d;
               }
             }
-            if (a.gain && publish && in && a.xn_out) {
-              *reinterpret_cast<float4*>(a.xn_out + e0) = make_float4(xv[0], xv[1], xv[2], xv[3]);
-              *reinterpret_cast<float4*>(a.xn_out + e0 + 4) =
-                  make_float4(xv[4], xv[5], xv[6], xv[7]);
-            }
             if (!WQ8 && v < nv) {
               xs[b * nv + v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
               xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
@@ -393,6 +468,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
         }
         consumers_sync(ncons);
         cur_seg = seg;
+        if (tr && t == 0 && threadIdx.x == 0) tr[1] = gtimer();
       }
       // after a wait gives up, keep walking the stages (so that every consumer warp
       // reaches the same named barriers) but skip the work
@@ -430,6 +506,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       if (lane == 0) mbar_arrive(&empty[s]);
       cur = end;
     }
+    if (tr && threadIdx.x == 0) tr[2] = gtimer();
   }
   __syncthreads();
 
@@ -482,6 +559,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       }
     }
   }
+  if (EPI == EPI_PLAIN && a.merge_x) fused_merge<NB>(a, R0, nrows, rps);
+  if (tr && threadIdx.x == 0) tr[3] = gtimer();
 }
 
 // The int8-weight consumer step (see ring_pairs_dot): each row's codes are read
@@ -544,10 +623,22 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
 
 size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
 
+// Shared memory of a GEMV CTA: kSmemBudget (one CTA per SM, the deepest ring),
+// or TP_GEMV_SMEM_KB (a tuning knob: e.g. 110 lets two GEMV CTAs share an SM, so
+// that the next launch's ring fills while this one finishes).
+int gemv_smem_budget() {
+  static const int b = [] {
+    const char* v = getenv("TP_GEMV_SMEM_KB");
+    const int kb = v ? atoi(v) : 0;
+    return kb >= 32 && kb * 1024 <= kSmemBudget ? kb * 1024 : kSmemBudget;
+  }();
+  return b;
+}
+
 // Shared-memory plan: 8 consumer warps; the most row pairs per stage (16, 8, 4,
 // 2, 1) that still leave a ring of at least 3 stages (2 for the longest rows):
 // 16 pairs give each warp two pairs, fewer are each split over 8 / pairs warps.
-bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
+bool make_plan(int NB, int Ks, int cta_rows, bool wq8, int budget, GemvPlan* p) {
   const size_t row_bytes = wq8 ? (size_t)Ks + q8w_scale_slot(Ks) : (size_t)Ks * 2;
   const size_t x_bytes = wq8 ? a128((size_t)NB * Ks + (size_t)NB * (Ks / 32) * 4)
                              : a128((size_t)NB * Ks * 4);
@@ -557,9 +648,9 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
       const int Q = P >= 8 ? 1 : 8 / P;
       const size_t res_bytes = a128((size_t)cta_rows * NB * Q * 4);
       const size_t fixed = x_bytes + res_bytes + bar_bytes;
-      if (fixed >= (size_t)kSmemBudget) continue;
+      if (fixed >= (size_t)budget) continue;
       const size_t stage = 2 * (size_t)P * row_bytes;
-      int ns = (int)(((size_t)kSmemBudget - fixed) / stage);
+      int ns = (int)(((size_t)budget - fixed) / stage);
       if (ns > kMaxStages) ns = kMaxStages;
       if (ns >= min_stages) {
         p->nc = 8;
@@ -589,8 +680,24 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   int grid = num_sms();
   if (grid > npairs) grid = npairs;
   const int cta_rows = 2 * ((npairs + grid - 1) / grid);
+  int budget = gemv_smem_budget();
+  if (a.co_smem > 0) {  // fit beside another kernel's CTA (1 KB reserved per CTA)
+    static int per_sm = 0, st = 0;
+    if (!per_sm) {
+      int dev = 0, v = 0;
+      cudaFuncAttributes fa{};
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, (const void*)k_gemv<NB, EPI, WQ8>) != cudaSuccess)
+        return TP_ECUDA;
+      st = (int)fa.sharedSizeBytes;
+      per_sm = v;
+    }
+    const int room = per_sm - (a.co_smem + 1024) - (st + 1024) - 256;
+    if (room < budget) budget = room;
+  }
   GemvPlan pl;
-  if (!make_plan(NB, a.Ks, cta_rows, WQ8, &pl)) return TP_ENOTSUP;
+  if (!make_plan(NB, a.Ks, cta_rows, WQ8, budget, &pl)) return TP_ENOTSUP;
   if (set_smem_once((const void*)k_gemv<NB, EPI, WQ8>, (int)pl.total)) return TP_ECUDA;
   return launch_pdl(k_gemv<NB, EPI, WQ8>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
 }
@@ -614,6 +721,12 @@ int launch_nb(const GemvArgs& a, int epi, cudaStream_t s) {
 // Batch rows are handled two at a time (each launch streams the weights once).
 int launch_gemv(const GemvArgs& a0, int epi, cudaStream_t s) {
   if (a0.Ks % 32 != 0 || a0.Ks < 32 || a0.nseg < 1) return TP_EINVAL;
+  if (a0.merge_x) {  // fused merge: whole 128-value chunks per piece, counters sized by the caller
+    if (epi != EPI_PLAIN || a0.rows[0] % 128 != 0 || !a0.merge_cnt || !a0.merge_ssq ||
+        a0.merge_pieces != (a0.rows[0] + kMergePiece - 1) / kMergePiece ||
+        a0.merge_pieces > kMaxMergePieces || a0.ldo != a0.rows[0])
+      return TP_EINVAL;
+  }
   if (a0.wd[0] && a0.ldw % 64 != 0) return TP_EINVAL;  // whole 16-byte scale runs per matrix
   if (((a0.rows[0] | a0.rows[1] | a0.rows[2]) & 1) != 0) return TP_EINVAL;
   for (int b = 0; b < a0.nb;) {

@@ -8,12 +8,13 @@ namespace tp {
 // ------------------------------------------------------------------ merge / codec
 // x[b] += sum_{s<n} sync(part_s[b]) in slice order, part_s = the sum of planes
 // s*parts .. s*parts+parts-1 of part [n*parts, B, dim] (a slice's contraction
-// split further by the GEMM). With ssq != nullptr each CTA also writes the sum of
-// squares of its piece of the new row: ssq[b][piece], piece = 512-element block
-// index (merge_ssq_parts(dim) of them).
+// split further by the GEMM). With ssq != nullptr the sum of squares of every
+// 128-value chunk of the new row is written too: ssq[b][chunk] (merge_ssq_parts(dim)
+// of them; one warp's float4 lanes summed by warp_sum, in every merge variant, so
+// that all of them give the next RMSNorm the same bits). dim % 128 == 0.
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts = 1);
-inline int merge_ssq_parts(int dim) { return (dim / 4 + 127) / 128; }
+inline int merge_ssq_parts(int dim) { return dim / 128; }
 // One slice's partial in the sync format for B rows: float32 [B, dim], or with Q8
 // the codes int8 [B, dim] followed by the scales float32 [B, dim/32].
 __host__ __device__ inline int64_t sync_slice_bytes(int B, int dim, int quant) {
@@ -56,7 +57,8 @@ struct GemvArgs {
   // input: float32 x [B, ldx] or Q8 (xq [B, ldx], xd [B, ldx/32]); with `gain`
   // set, x is a residual and the input is RMSNorm(x) * gain (+Q8 when quant),
   // computed in the prologue; the first CTA of each segment then writes the
-  // shared buffer (xq_out/xd_out for Q8, xn_out for float32; each nullable).
+  // shared buffer (xq_out/xd_out: the Q8 codes and scales; xn_out: the float32
+  // RMSNorm output before any Q8 round trip; each nullable).
   const float* x;
   const int8_t* xq;
   const float* xd;
@@ -83,8 +85,33 @@ struct GemvArgs {
   const int32_t* seq;  // cache sequence of each row (nullable: row b uses sequence b)
   int n_heads, n_kv_heads, max_seq;
   float theta;
+  // EPI_PLAIN row-split products with merge_x set: the merge fused into the
+  // epilogue. Each CTA counts the partial values it stored per (batch group b0,
+  // piece of kMergePiece outputs) on merge_cnt[b0 * merge_pieces + piece]; the
+  // CTA whose count completes a piece merges it, x[b] += sum_s sync(out[s][b])
+  // in slice order (the Q8 round trip when merge_quant), writes the sums of
+  // squares of its 128-value chunks to merge_ssq[b][chunk] (as launch_merge) and
+  // sets the counter back to zero (counters start at zero and every launch
+  // leaves them so).
+  float* merge_x;
+  float* merge_ssq;
+  int* merge_cnt;
+  int merge_quant;
+  int merge_pieces;
+  // optional %globaltimer stamps (ns) of CTA c at trace[c * trace_stride + k]:
+  // k = 0 start, 1 activations staged, 2 last ring stage consumed, 3 end
+  unsigned long long* trace;
+  int trace_stride;
+  // shared memory of another kernel's CTA that this launch's CTAs must fit beside
+  // on one SM (0: none, the ring takes the whole SM). The W_O GEMV leaves room
+  // for one attention CTA, so that it becomes resident and streams its weights
+  // while the attention still runs (programmatic dependent launch).
+  int co_smem;
   int* err;  // device error flag, set when a bounded wait gives up (nullable)
 };
+// Outputs per piece (counter) of the fused merge.
+constexpr int kMergePiece = 512;
+constexpr int kMaxMergePieces = 64;
 
 // Shared-memory plan of the GEMV (host computes, kernel reads): NC consumer
 // warps, row pairs per stage (each pair split over `split` warps), ring depth,
@@ -116,14 +143,19 @@ struct AttnArgs {
   float* part_ml;       // [B, H, nsplit, 2] running max and sum
   float* att;           // [B, H*hd] combined output
   uint16_t* att_bf16;   // optional hi/lo bf16 pairs [2B, H*hd] (rows 2b, 2b+1)
+  int nsplit;           // context splits (0: attention_nsplit's choice)
   int* err;             // device error flag (bounded waits)
 };
 
 // combine = false leaves the splits' partials for the consumer to combine (the
 // W_O GEMV's staging on the weight-streaming path).
 int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine = true);
-// Context splits per (batch row, kv head) the attention uses for these shapes.
-int attention_nsplit(int B, int H, int Hkv, int max_seq);
+// Context splits per (batch row, kv head) the attention uses for these shapes,
+// with at most `per_sm` of its CTAs resident per SM (2 fit; 1 leaves room beside
+// each for the next kernel's CTA, see attention_cta_smem).
+int attention_nsplit(int B, int H, int Hkv, int max_seq, int per_sm = 2);
+// Shared memory (dynamic + static) one decode-attention CTA holds.
+int attention_cta_smem();
 // Largest number of context splits any launch over max_seq positions uses.
 int attention_max_splits(int max_seq);
 
@@ -142,27 +174,11 @@ struct NormRowsArgs {
   int quant;
   int8_t* xq;          // Q8 codes [B, dim] (nullable)
   float* xd;           // Q8 scales [B, dim/32] (nullable)
-  float* xn;           // float32 value the slices read (nullable)
-  uint16_t* xb;        // that value as hi/lo bf16 pairs [2B, dim] (tensor-core operand)
+  float* xn;           // float32 RMSNorm output, before any Q8 round trip (nullable)
+  uint16_t* xb;        // the value the slices read (after Q8 when quant) as hi/lo bf16
+                       // pairs [2B, dim] (tensor-core operand)
 };
 int launch_norm_rows(const NormRowsArgs& a, int batch, cudaStream_t s);
-
-struct QkvFinalizeArgs {
-  const float* plane;  // [parts][batch][qd + 2 kd]
-  int parts, batch, qd, kd;
-  const int32_t* pos;
-  const int32_t* seq;  // cache sequence of each row (nullable: row b)
-  float theta;
-  float* q;            // [batch, qd]
-  uint16_t* kc;
-  uint16_t* vc;
-  int n_kv_heads, max_seq;
-};
-int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s);
-// h = silu(a) * g from planes [parts][batch][2F] (a = columns [0, F), g = [F, 2F),
-// each the sum of the parts in order), with its hi/lo bf16 pair rows.
-int launch_swiglu_finalize(const float* plane, int parts, int F, int batch, float* h,
-                           uint16_t* hb, cudaStream_t s);
 
 // ------------------------------------------------------------------ persistent block
 // One weight-streaming phase of the persistent block kernel: the rows of up to

@@ -20,7 +20,6 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
                                                          const float* __restrict__ part, int n,
                                                          int parts, int B, int dim, int quant,
                                                          float* __restrict__ ssq) {
-  __shared__ float red[kMergeThreads / 32];
   pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.y;
@@ -56,15 +55,10 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
     xr[i4] = v;
     sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
-  if (ssq) {  // this piece's sum of squares, for the next RMSNorm (fixed summation order)
+  if (ssq) {  // each warp's 128 values: their sum of squares, for the next RMSNorm
     sq = warp_sum(sq);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = 0.f;
-      for (int w = 0; w < kMergeThreads / 32; ++w) t += red[w];
-      ssq[(size_t)b * gridDim.x + blockIdx.x] = t;
-    }
+    const int chunk = (blockIdx.x * kMergeThreads + (threadIdx.x & ~31)) >> 5;
+    if ((threadIdx.x & 31) == 0 && chunk < (dim >> 7)) ssq[(size_t)b * (dim >> 7) + chunk] = sq;
   }
 }
 
@@ -108,7 +102,6 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge_sync(float* __restrict_
                                                               const uint8_t* __restrict__ sync,
                                                               int n, int B, int dim, int quant,
                                                               float* __restrict__ ssq) {
-  __shared__ float red[kMergeThreads / 32];
   pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.y;
@@ -142,15 +135,10 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge_sync(float* __restrict_
     xr[i4] = v;
     sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
-  if (ssq) {
+  if (ssq) {  // as k_merge: one sum of squares per warp's 128 values
     sq = warp_sum(sq);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = 0.f;
-      for (int w = 0; w < kMergeThreads / 32; ++w) t += red[w];
-      ssq[(size_t)b * gridDim.x + blockIdx.x] = t;
-    }
+    const int chunk = (blockIdx.x * kMergeThreads + (threadIdx.x & ~31)) >> 5;
+    if ((threadIdx.x & 31) == 0 && chunk < (dim >> 7)) ssq[(size_t)b * (dim >> 7) + chunk] = sq;
   }
 }
 
@@ -179,21 +167,24 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 
 }  // namespace
 
+// 512 values (4 warps of float4 lanes) per CTA
+int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; }
+
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts) {
-  const dim3 grid(merge_ssq_parts(dim), B);
+  const dim3 grid(merge_grid(dim), B);
   return launch_pdl(k_merge, grid, dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim, quant, ssq);
 }
 
 int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
                      uint8_t* out, cudaStream_t s) {
-  const dim3 grid(merge_ssq_parts(dim), B, n_local);
+  const dim3 grid(merge_grid(dim), B, n_local);
   return launch_pdl(k_sync_pack, grid, dim3(kMergeThreads), 0, s, part, parts, B, dim, quant, out);
 }
 
 int launch_merge_sync(float* x, const uint8_t* sync, int n, int B, int dim, int quant, float* ssq,
                       cudaStream_t s) {
-  const dim3 grid(merge_ssq_parts(dim), B);
+  const dim3 grid(merge_grid(dim), B);
   return launch_pdl(k_merge_sync, grid, dim3(kMergeThreads), 0, s, x, sync, n, B, dim, quant, ssq);
 }
 

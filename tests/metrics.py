@@ -30,3 +30,19 @@ def report(name, y, ref):
     r, p = max_rel(y, ref), pcc(y, ref)
     print(f"[parity] {name}: max_rel={r:.3e} pcc={p:.8f}")
     return r, p
+
+
+def assert_q8_codes_exact(xn, xq, xd, rows, dim, name="xnorm"):
+    """The Q8 codes and scales a kernel wrote equal, bit for bit, the oracle's Q8 of
+    the kernel's own float32 normalised rows (identical float32 inputs: the
+    distributed-llama Quantize step after RMSNorm, checked on the hot path)."""
+    import oracle
+
+    xn = np.asarray(xn, dtype=np.float32)[:rows * dim].reshape(rows, dim)
+    q_ref, d_ref = oracle.q8_quantize(xn)
+    q = np.asarray(xq)[:rows * dim].reshape(rows, dim)
+    d = np.asarray(xd, dtype=np.float32)[:rows * (dim // 32)].reshape(rows, dim // 32)
+    np.testing.assert_array_equal(q, q_ref, err_msg=f"{name}: Q8 codes")
+    np.testing.assert_array_equal(d.view(np.uint32), np.asarray(d_ref, np.float32).view(np.uint32),
+                                  err_msg=f"{name}: Q8 scales")
+    print(f"[parity] {name}: Q8 codes and scales bit-exact ({rows} x {dim})")

@@ -13,7 +13,7 @@ import torch
 import oracle
 import synth
 from synth.device import DeviceBlock, to_bits
-from tests.metrics import BF16_TOL, report
+from tests.metrics import BF16_TOL, assert_q8_codes_exact, report
 
 pytestmark = pytest.mark.gpu
 
@@ -96,6 +96,15 @@ def check_block(tpb, inp, n, quant, partition=1, tol_out=BF16_TOL, tight=None, n
     if tight is not None:
         assert max(r_q, r_att, r_out, r_dx) <= tight, "regression against the expected error level"
     assert p_out > 0.9999
+    # the last RMSNorm of the step (the FFN's): its float32 output against the oracle's,
+    # and, with the Q8 sync, the codes and scales the fused prologue wrote bit-exact
+    # against the oracle's Q8 of that same float32 row
+    D = s.dim
+    xn_ref = oracle.rmsnorm(tr["x1"], inp.ffn_norm, s.norm_eps)
+    r_xn, _ = report(f"{name} xnorm(ffn)", bufs["xn"][:B * D].reshape(B, D), xn_ref)
+    assert r_xn <= (tight if tight is not None else tol_out)
+    if quant:
+        assert_q8_codes_exact(bufs["xn"], bufs["xq"], bufs["xd"], B, D, f"{name} xnorm(ffn)")
     return r_out
 
 

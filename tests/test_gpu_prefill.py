@@ -16,7 +16,7 @@ import torch
 import oracle
 import synth
 from synth.device import DeviceBlock, bf16_tensor, f32_tensor, i32_tensor, to_bits
-from tests.metrics import BF16_TOL, report
+from tests.metrics import BF16_TOL, assert_q8_codes_exact, report
 from tests.test_gpu_block import TIGHT, TIGHT_Q8, _dims
 
 pytestmark = pytest.mark.gpu
@@ -43,18 +43,24 @@ def run_seq(tpb, inp, n, quant):
         torch.cuda.synchronize()
         off, _ = tpb.tp_block_buffer(h, 7)
         err = int(ws[off:off + 4].view(torch.int32).item())
+        norm = {}
+        for key, which, dt in (("xn", tpb.BUF_XN, torch.float32), ("xq", tpb.BUF_XQ, torch.int8),
+                               ("xd", tpb.BUF_XD, torch.float32)):
+            o, size = tpb.tp_block_buffer(h, which)
+            norm[key] = ws[o:o + size].view(dt).cpu().numpy()
     finally:
         tpb.tp_block_destroy(h)
     seq, pos = inp.extra["seq"], inp.pos
     kb, vb = to_bits(dev.k_cache), to_bits(dev.v_cache)
     k_rows = np.stack([kb[seq[b], :, pos[b], :] for b in range(B)])
     v_rows = np.stack([vb[seq[b], :, pos[b], :] for b in range(B)])
-    return dev.x.cpu().numpy().astype(np.float64), k_rows, v_rows, err
+    return dev.x.cpu().numpy().astype(np.float64), k_rows, v_rows, err, norm
 
 
 def check_seq(tpb, inp, n, quant, tight, name):
-    ref, k_ref, v_ref = oracle.block_forward(inp, n, bool(quant), seq=inp.extra["seq"])
-    y, k_rows, v_rows, err = run_seq(tpb, inp, n, quant)
+    tr = {}
+    ref, k_ref, v_ref = oracle.block_forward(inp, n, bool(quant), seq=inp.extra["seq"], trace=tr)
+    y, k_rows, v_rows, err, norm = run_seq(tpb, inp, n, quant)
     assert err == 0, "a bounded wait in a kernel gave up"
     r_out, p_out = report(f"{name} out", y, ref)
     r_dx, _ = report(f"{name} out-x", y - inp.x, ref - inp.x)
@@ -64,6 +70,14 @@ def check_seq(tpb, inp, n, quant, tight, name):
         assert r <= BF16_TOL
     assert max(r_out, r_dx) <= tight, "regression against the expected error level"
     assert p_out > 0.9999
+    # the FFN RMSNorm (+Q8) of every row: float32 output against the oracle's, codes
+    # bit-exact against the oracle's Q8 of the kernel's own float32 rows
+    B, D = inp.x.shape
+    xn_ref = oracle.rmsnorm(tr["x1"], inp.ffn_norm, inp.shape.norm_eps)
+    r_xn, _ = report(f"{name} xnorm(ffn)", norm["xn"][:B * D].reshape(B, D), xn_ref)
+    assert r_xn <= tight
+    if quant:
+        assert_q8_codes_exact(norm["xn"], norm["xq"], norm["xd"], B, D, f"{name} xnorm(ffn)")
     return y
 
 

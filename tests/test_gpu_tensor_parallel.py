@@ -26,7 +26,7 @@ import oracle
 import synth
 from synth.device import DeviceBlock, to_bits
 from tensor_llama_transformer_b200 import tensor_parallel as tp
-from tests.metrics import BF16_TOL, report
+from tests.metrics import BF16_TOL, assert_q8_codes_exact, report
 from tests.test_gpu_block import SMALL_TC_GQA, SMALL_TC_MHA, TIGHT, TIGHT_Q8, _dims, run_block
 
 pytestmark = pytest.mark.gpu
@@ -62,12 +62,23 @@ def run_ranks(tpb, inp, n, quant, world):
                     rk["rb"].buffers(B)[1].copy_(gathered)
             for rk in ranks:
                 rk["rb"].step(phase, rk["x"], rk["kc"], rk["vc"], dev.pos, B)
+            if phase == tp.TP_RANK_ATT:  # the attention RMSNorm (+Q8) each rank's prologue wrote
+                torch.cuda.synchronize()
+                for rk in ranks:
+                    norm = {}
+                    for key, which, dt in (("xn", tpb.BUF_XN, torch.float32),
+                                           ("xq", tpb.BUF_XQ, torch.int8),
+                                           ("xd", tpb.BUF_XD, torch.float32)):
+                        off, size = tpb.tp_block_buffer(rk["rb"].h, which)
+                        norm[key] = rk["rb"].ws[off:off + size].view(dt).cpu().numpy()
+                    rk["att_norm"] = norm
         torch.cuda.synchronize()
         errs = []
         for rk in ranks:
             off, _ = tpb.tp_block_buffer(rk["rb"].h, 7)
             errs.append(int(rk["rb"].ws[off:off + 4].view(torch.int32).item()))
         xs = [rk["x"].cpu().numpy().astype(np.float64) for rk in ranks]
+        norms = [rk["att_norm"] for rk in ranks]
         kb = np.concatenate([to_bits(rk["kc"]) for rk in ranks], axis=1)
         vb = np.concatenate([to_bits(rk["vc"]) for rk in ranks], axis=1)
     finally:
@@ -75,11 +86,11 @@ def run_ranks(tpb, inp, n, quant, world):
             rk["rb"].close()
     k_rows = np.stack([kb[b, :, inp.pos[b], :] for b in range(B)])
     v_rows = np.stack([vb[b, :, inp.pos[b], :] for b in range(B)])
-    return xs, k_rows, v_rows, errs
+    return xs, k_rows, v_rows, errs, norms
 
 
 def check_ranks(tpb, inp, n, quant, world, tight, name):
-    xs, k_rows, v_rows, errs = run_ranks(tpb, inp, n, quant, world)
+    xs, k_rows, v_rows, errs, norms = run_ranks(tpb, inp, n, quant, world)
     assert errs == [0] * world, "a bounded wait in a kernel gave up"
     for x in xs[1:]:
         assert np.array_equal(x, xs[0]), "ranks ended with different residuals"
@@ -95,6 +106,16 @@ def check_ranks(tpb, inp, n, quant, world, tight, name):
     whole = run_block(tpb, inp, n, quant)[0]
     r_w, _ = report(f"{name} vs whole block", xs[0] - inp.x, whole - inp.x)
     assert r_w <= tight
+    # the attention RMSNorm of phase 0 on every rank: float32 output against the
+    # oracle's, and with the Q8 sync its codes bit-exact from that same float32 row
+    s = inp.shape
+    B, D = inp.x.shape
+    xn_ref = oracle.rmsnorm(inp.x, inp.attn_norm, s.norm_eps)
+    for r, nm in enumerate(norms):
+        r_xn, _ = report(f"{name} rank {r} xnorm(att)", nm["xn"][:B * D].reshape(B, D), xn_ref)
+        assert r_xn <= 1e-5
+        if quant:
+            assert_q8_codes_exact(nm["xn"], nm["xq"], nm["xd"], B, D, f"{name} rank {r} xnorm(att)")
 
 
 MHA4 = synth.BlockShape(dim=256, n_heads=4, n_kv_heads=4, head_dim=128, ffn_dim=512, vocab=0,
