@@ -57,6 +57,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the C4 block and C3 model measurements")
+    ap.add_argument("--extras", default=None,
+                    help="comma list of the extra workloads to time (default: all of them): "
+                         "c2_block_persistent, c2_block_int8_weights, c2_prefill_chunk64, c4_block, "
+                         "c3_model_b1, c3_model_b16")
     ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w", "c2prefill", "ffn"],
                     default=None,
                     help="only run a few eager steps of one extra workload (for profiler launch "
@@ -418,13 +422,13 @@ def bench_block(args, world, rank, local):
     t = tr.view(nsm, -1).cpu().numpy().astype("float64")
     timeline = {}
     base = t[t[:, 0] > 0, 0].min()
+    marks = ("start", "prev_done", "staged", "first_stage", "consumed", "end")
     for gi, name in enumerate(("qkv", "wo", "w13", "w2")):
-        cols = t[:, 4 * gi:4 * gi + 4]
+        cols = t[:, 6 * gi:6 * gi + 6]
         cols = cols[cols[:, 0] > 0]
-        med = [round(float(statistics.median((cols[:, k] - base) / 1e3)), 2) for k in range(4)]
-        timeline[name] = {"start": med[0], "staged": med[1], "consumed": med[2], "end": med[3],
-                          "first_start": round(float((cols[:, 0].min() - base) / 1e3), 2),
-                          "last_end": round(float((cols[:, 3].max() - base) / 1e3), 2)}
+        timeline[name] = {m: [round(float(f((cols[:, k] - base) / 1e3)), 2)
+                              for f in (min, statistics.median, max)]
+                          for k, m in enumerate(marks)}
 
     # end to end through the public API: host buffers, copies inside the timed region
     xh = torch.empty_like(dev.x, device="cpu").pin_memory()
@@ -974,27 +978,19 @@ def main(argv=None):
     if not args.no_extra:
         import torch
 
-        try:
-            extra = {"c2_block_persistent": bench_c2_persistent(args)}
-        except Exception as e:  # reported, not fatal: the headline does not depend on it
-            extra = {"c2_block_persistent": {"error": str(e)[:200]}}
-        torch.cuda.empty_cache()
-        try:
-            extra["c2_block_int8_weights"] = bench_c2_q8w(args)
-        except Exception as e:  # reported, not fatal
-            extra["c2_block_int8_weights"] = {"error": str(e)[:200]}
-        torch.cuda.empty_cache()
-        try:
-            extra["c2_prefill_chunk64"] = bench_c2_prefill(args)
-        except Exception as e:  # reported, not fatal
-            extra["c2_prefill_chunk64"] = {"error": str(e)[:200]}
-        torch.cuda.empty_cache()
-        extra["c4_block"] = bench_c4(args)
-        torch.cuda.empty_cache()
-        extra["c3_model_b1"] = bench_c3(args, 1)
-        torch.cuda.empty_cache()
-        extra["c3_model_b16"] = bench_c3(args, 16)
-        torch.cuda.empty_cache()
+        runs = [("c2_block_persistent", bench_c2_persistent), ("c2_block_int8_weights", bench_c2_q8w),
+                ("c2_prefill_chunk64", bench_c2_prefill), ("c4_block", bench_c4),
+                ("c3_model_b1", lambda a: bench_c3(a, 1)), ("c3_model_b16", lambda a: bench_c3(a, 16))]
+        want = set(args.extras.split(",")) if args.extras else None
+        extra = {}
+        for name, fn in runs:
+            if want is not None and name not in want:
+                continue
+            try:
+                extra[name] = fn(args)
+            except Exception as e:  # reported, not fatal: the headline does not depend on it
+                extra[name] = {"error": str(e)[:200]}
+            torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
@@ -1015,10 +1011,10 @@ def main(argv=None):
             "hbm_gbs": res["block_gbs"], "block_roofline_frac": res["block_roofline_frac"],
             "stage_us": res["stage_us"], "stage_sum_us": res["stage_sum_us"],
             "gemv_timeline_us": res["gemv_timeline_us"],
-            "gemv_timeline_note": "one replay of a captured step: per slice GEMV the median over "
-                                  "CTAs of its start, activations staged, last weight stage "
-                                  "consumed and end (us from the first q/k/v CTA's start), and "
-                                  "the earliest start / latest end",
+            "gemv_timeline_note": "one replay of a captured step: per slice GEMV, [min, median, "
+                                  "max] over CTAs (us from the first q/k/v CTA's start) of its "
+                                  "start, previous kernel complete, activations staged, first "
+                                  "weight stage arrived, last stage consumed, end",
             "stage_note": "per-stage CUDA-event times from a replay of the same steps with an event "
                           "before every stage (serialised, so upper bounds); value and ms_per_step "
                           "come from the event-free graph; the merges run in the W_O and W2 "

@@ -282,11 +282,13 @@ TP_API int tp_block_set_persistent(tp_block* blk, int enable);
  * block runs as separate kernels and the trace is not written. A forward on the
  * kernel-per-step weight-streaming path (batch <= 5, persistent kernel off)
  * writes instead, for each of its four slice GEMVs g (0 q/k/v, 1 W_O, 2 W1/W3,
- * 3 W2) and CTA c of that launch, trace[c * TP_BLOCK_TRACE_SLOTS + 4g + k]: k = 0
- * start, 1 activations staged, 2 last weight stage consumed, 3 end (after the
- * epilogue and the fused merge); for batch > 2 the last launch of each wins.
+ * 3 W2) and CTA c of that launch, trace[c * TP_BLOCK_TRACE_SLOTS + 6g + k]: k = 0
+ * start, 1 the previous kernel complete (its wait returned), 2 activations
+ * staged, 3 the first weight stage arrived, 4 the last stage consumed, 5 end
+ * (after the epilogue and the fused merge); for batch > 2 the last launch of each
+ * wins. The persistent kernel uses slots 0-15.
  * Errors: TP_EINVAL (NULL handle, buffer too small). */
-#define TP_BLOCK_TRACE_SLOTS 16
+#define TP_BLOCK_TRACE_SLOTS 32
 TP_API int tp_block_set_trace(tp_block* blk, void* trace, size_t bytes);
 
 /* One block decode step that allocates nothing (no counterpart in the paper: this

@@ -58,13 +58,18 @@ int set_smem_once(const void* kernel, int bytes) {
   return TP_OK;
 }
 
-// The W_O GEMV streams its weights beside the attention (one attention CTA per SM,
-// the GEMV's ring sized to fit next to it) unless TP_ATT_OVERLAP=0.
+// Tuning switches read once from the environment (for comparison runs):
+//   TP_ATT_OVERLAP=1  the W_O GEMV streams its weights beside the attention (one
+//                     attention CTA per SM, the GEMV's ring sized to fit next to
+//                     it); off by default: the smaller ring streams slower than the
+//                     overlap gains.
+bool env_flag(const char* name, bool dflt) {
+  const char* v = getenv(name);
+  if (!v || !v[0]) return dflt;
+  return v[0] != '0';
+}
 bool att_overlap_enabled() {
-  static const bool on = [] {
-    const char* v = getenv("TP_ATT_OVERLAP");
-    return !(v && v[0] == '0');
-  }();
+  static const bool on = env_flag("TP_ATT_OVERLAP", false);
   return on;
 }
 
@@ -94,13 +99,10 @@ enum Buf {
   BUF_COUNT
 };
 static_assert(BUF_SEND == TP_BUF_SEND && BUF_RECV == TP_BUF_RECV, "buffer ids of the C ABI");
-// BUF_ERR (placed first: byte 0 of every block workspace): the int error word at
-// byte 0; the persistent kernel's two grid barrier counters at bytes 8 and 12;
-// from byte 16 the fused merges' counters (int [max_batch][dim / 128] at most).
-// Every counter starts at zero and every launch leaves it so.
+// BUF_ERR (16 bytes, placed first: byte 0 of every block workspace): the int
+// error word at byte 0; the persistent kernel's two grid barrier counters at
+// bytes 8 and 12 (zero between launches). The handle's first forward zeroes all.
 constexpr size_t kCountersOff = 8;
-constexpr size_t kMergeCntOff = 16;
-int merge_pieces(int dim) { return (dim + kMergePiece - 1) / kMergePiece; }
 
 // Largest contraction splits of the batched-decode GEMMs (the planes are sized for them).
 constexpr int kQkvMaxParts = 8, kW13MaxParts = 4, kW2MaxParts = 2;
@@ -186,15 +188,7 @@ Layout block_layout(const Cfg& c) {
   // row-split partials: n slices (x kW2MaxParts contraction parts on the tensor path)
   L.size[BUF_PART] = (size_t)c.n * (c.d.max_batch >= kTcMinBatch ? kW2MaxParts : 1) * B * D * 4;
   L.size[BUF_H] = B * F * 4;
-  // counters: the GEMV's per (batch group, 512-output piece), the GEMM's per 128-row tile
-  {
-    const size_t kd = (size_t)c.d.n_kv_heads * c.d.head_dim;
-    size_t cnt = B * (size_t)(c.d.dim / 128);
-    const size_t tiles_qkv = (QD + 127) / 128 + 2 * ((kd + 127) / 128), tiles_f = (F + 127) / 128;
-    if (tiles_qkv > cnt) cnt = tiles_qkv;
-    if (tiles_f > cnt) cnt = tiles_f;
-    L.size[BUF_ERR] = kMergeCntOff + cnt * 4;
-  }
+  L.size[BUF_ERR] = 16;
   L.size[BUF_PO] = B * c.d.n_heads * (size_t)c.nchunk * c.d.head_dim * 4;
   L.size[BUF_PML] = B * c.d.n_heads * (size_t)c.nchunk * 2 * 4;
   const size_t pa = c.partition == TP_PART_2D ? (size_t)c.gx * B * F * 4 : 0;
@@ -316,22 +310,11 @@ int merge_step(tp_block* blk, float* x, const float* part, int nseg, int parts, 
                            ssq, s);
 }
 
-// a6 / a10 fused into the row-split GEMV that produces the partials (whole
-// block on the weight-streaming kernels): the CTA that completes a piece of the
-// output merges it into x and leaves the piece's sum of squares.
-void set_fused_merge(tp_block* blk, GemvArgs& a, float* x) {
-  a.merge_x = x;
-  a.merge_ssq = at<float>(blk, BUF_SSQ);
-  a.merge_cnt = reinterpret_cast<int*>(blk->ws + blk->L.off[BUF_ERR] + kMergeCntOff);
-  a.merge_quant = blk->c.quant;
-  a.merge_pieces = merge_pieces(blk->c.d.dim);
-}
-
-// Trace slots 4g .. 4g+3 of every CTA for the slice GEMV g (0 q/k/v, 1 W_O,
+// Trace slots 6g .. 6g+5 of every CTA for the slice GEMV g (0 q/k/v, 1 W_O,
 // 2 W1/W3, 3 W2) when a trace buffer is set.
 void set_gemv_trace(const tp_block* blk, GemvArgs& a, int g) {
   if (!blk->trace) return;
-  a.trace = blk->trace + 4 * g;
+  a.trace = blk->trace + 6 * g;
   a.trace_stride = TP_BLOCK_TRACE_SLOTS;
 }
 
@@ -395,11 +378,8 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     n.xb = xb;
     return launch_norm_rows(n, batch, s);
   };
-  // fin: the step fused into the GEMM's epilogue after the last plane of a tile
-  int* fin_cnt = reinterpret_cast<int*>(blk->ws + blk->L.off[BUF_ERR] + kMergeCntOff);
   auto gemm = [&](const void* A0, int m0, const void* A1, int m1, const void* A2, int m2, int nA,
-                  int64_t lda, const uint16_t* Bop, int K, int nseg, float* out, int64_t rows,
-                  TcFinish fin) {
+                  int64_t lda, const uint16_t* Bop, int K, int nseg, float* out, int64_t rows) {
     TcGemm g{};
     g.A[0] = A0;
     g.A[1] = A1;
@@ -420,46 +400,37 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     g.out_seg = (int64_t)batch * rows;
     g.err = err;
     g.indep = TC_INDEP_A;  // the weights
-    g.fin = fin;
-    if (fin.kind != TC_FIN_NONE) g.fin.cnt = fin_cnt;
     return launch_tc_gemm(g, s);
   };
 
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
   int p2 = 1;
-  TcFinish none{};
-  auto merge_fin = [&](int parts) {  // a6 / a10 in the epilogue (whole block)
-    TcFinish f{};
-    if (c.world != 0) return f;
-    f.kind = TC_FIN_MERGE;
-    f.parts = parts;
-    f.x = x;
-    f.ssq = at<float>(blk, BUF_SSQ);
-    f.quant = c.quant;
-    return f;
-  };
   if (phase <= 0) {
     // a1-a4
     if ((rc = stage_mark(blk, 0, s))) return rc;
     if ((rc = norm(blk->w.attn_norm, chained ? at<float>(blk, BUF_SSQ) : nullptr))) return rc;
     const int qkv_tiles = (QD + 127) / 128 + 2 * ((KD + 127) / 128);
     const int parts = tc_split(qkv_tiles, D, QD + 2 * KD, batch, kQkvMaxParts);
-    // the parts' sum, RoPE, q and the cache rows in the epilogue (llamaQkv + the
-    // cache merge of llamaMultiheadAtt)
-    TcFinish fq{};
-    fq.kind = TC_FIN_QKV;
-    fq.parts = parts;
-    fq.q = at<float>(blk, BUF_Q);
-    fq.kc = static_cast<uint16_t*>(kc);
-    fq.vc = static_cast<uint16_t*>(vc);
-    fq.pos = pos;
-    fq.seq = seq;
-    fq.theta = d.rope_theta;
-    fq.n_kv_heads = Hkv;
-    fq.max_seq = d.max_seq;
     if ((rc = gemm(blk->w.wq, QD, blk->w.wk, KD, blk->w.wv, KD, 3, D, xb, D / parts, parts, plane,
-                   QD + 2 * KD, fq)))
+                   QD + 2 * KD)))
       return rc;
+    {
+      QkvFinalizeArgs f{};
+      f.plane = plane;
+      f.parts = parts;
+      f.batch = batch;
+      f.qd = QD;
+      f.kd = KD;
+      f.pos = pos;
+      f.seq = seq;
+      f.theta = d.rope_theta;
+      f.q = at<float>(blk, BUF_Q);
+      f.kc = static_cast<uint16_t*>(kc);
+      f.vc = static_cast<uint16_t*>(vc);
+      f.n_kv_heads = Hkv;
+      f.max_seq = d.max_seq;
+      if ((rc = launch_qkv_finalize(f, s))) return rc;
+    }
     // a4
     if ((rc = stage_mark(blk, 1, s))) return rc;
     {
@@ -484,16 +455,15 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     }
     // a5: W_O row-split partials (segment s = slice s's head columns)
     if ((rc = stage_mark(blk, 2, s))) return rc;
-    // (a6 fused into its epilogue for the whole block)
     if ((rc = gemm(blk->w.wo, D, nullptr, 0, nullptr, 0, 1, QD, at<uint16_t>(blk, BUF_ATTB), QD / c.n,
-                   c.n, part, D, merge_fin(1))))
+                   c.n, part, D)))
       return rc;
     if (phase == 0) return pack_step(blk, part, 1, batch, s);
   }
   if (phase <= 1) {
     // a6 (a rank block: the merge of the gathered buffer)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if (c.world != 0 && (rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
     // a7-a8
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if ((rc = norm(blk->w.ffn_norm, at<float>(blk, BUF_SSQ)))) return rc;
@@ -501,21 +471,14 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     uint16_t* hb = at<uint16_t>(blk, BUF_HB);
     if (c.partition == TP_PART_1D) {
       const int p13 = tc_split(2 * ((F + 127) / 128), D, 2 * F, batch, kW13MaxParts);
-      TcFinish fs{};  // silu(W1 row) * W3 row in the epilogue (llamaFfn)
-      fs.kind = TC_FIN_SWIGLU;
-      fs.parts = p13;
-      fs.h = hbuf;
-      fs.hb = hb;
-      if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F,
-                     fs)))
+      if ((rc = gemm(blk->w.w1, F, blk->w.w3, F, nullptr, 0, 2, D, xb, D / p13, p13, plane, 2 * F)))
         return rc;
+      if ((rc = launch_swiglu_finalize(plane, p13, F, batch, hbuf, hb, s))) return rc;
     } else {
       float* pa = at<float>(blk, BUF_PA);
       float* pb = at<float>(blk, BUF_PB);
-      if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F, none)))
-        return rc;
-      if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F, none)))
-        return rc;
+      if ((rc = gemm(blk->w.w1, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pa, F))) return rc;
+      if ((rc = gemm(blk->w.w3, F, nullptr, 0, nullptr, 0, 1, D, xb, D / c.gx, c.gx, pb, F))) return rc;
       FfnMergeArgs m{};
       m.P1 = pa;
       m.P3 = pb;
@@ -535,13 +498,13 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
     p2 = tc_split((int64_t)nseg2 * ((D + 127) / 128), F / nseg2, (int64_t)nseg2 * D, batch,
                   kW2MaxParts);
     if ((rc = gemm(blk->w.w2, D, nullptr, 0, nullptr, 0, 1, F, hb, F / nseg2 / p2, nseg2 * p2, part,
-                   D, merge_fin(p2))))
+                   D)))
       return rc;
     if (phase == 1) return pack_step(blk, part, p2, batch, s);
   }
-  // a10 (fused into the W2 GEMM's epilogue for the whole block)
+  // a10
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if (c.world != 0 && (rc = merge_step(blk, x, part, nseg2, p2, batch, s))) return rc;
+  if ((rc = merge_step(blk, x, part, nseg2, p2, batch, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -609,9 +572,8 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
                        cudaStream_t s, bool chained = false, int phase = -1,
                        const int32_t* seq = nullptr, int nseq = 0) {
   if (blk->wq8 && batch >= kTcMinBatch) return TP_ENOTSUP;
-  if (!blk->bar_ready) {  // the counters start at zero (first use of this workspace)
-    uint8_t* cnt = blk->ws + blk->L.off[BUF_ERR] + kCountersOff;
-    if (cudaMemsetAsync(cnt, 0, blk->L.size[BUF_ERR] - kCountersOff, s) != cudaSuccess)
+  if (!blk->bar_ready) {  // error word and counters start at zero (first use of the workspace)
+    if (cudaMemsetAsync(blk->ws + blk->L.off[BUF_ERR], 0, blk->L.size[BUF_ERR], s) != cudaSuccess)
       return TP_ECUDA;
     blk->bar_ready = true;
   }
@@ -721,16 +683,15 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.ldo = D;
       a.err = at<int>(blk, BUF_ERR);
       set_gemv_trace(blk, a, 1);
-      if (c.world == 0) set_fused_merge(blk, a, x);  // a6 in the epilogue
       if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
     if (phase == 0) return pack_step(blk, part, 1, batch, s);
   }
   if (phase <= 1) {
     // a6: sync + dequantise + merge into the residual (a rank block: of the
-    // gathered buffer; the whole block did it in the W_O GEMV's epilogue)
+    // gathered buffer)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if (c.world != 0 && (rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
     // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if (c.partition == TP_PART_1D) {
@@ -805,14 +766,13 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.ldo = D;
       a.err = at<int>(blk, BUF_ERR);
       set_gemv_trace(blk, a, 3);
-      if (c.world == 0) set_fused_merge(blk, a, x);  // a10 in the epilogue
       if ((rc = launch_gemv(a, EPI_PLAIN, s))) return rc;
     }
     if (phase == 1) return pack_step(blk, part, 1, batch, s);
   }
-  // a10: sync + dequantise + merge (fused into the W2 GEMV for the whole block)
+  // a10: sync + dequantise + merge
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if (c.world != 0 && (rc = merge_step(blk, x, part, nseg2, 1, batch, s))) return rc;
+  if ((rc = merge_step(blk, x, part, nseg2, 1, batch, s))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 

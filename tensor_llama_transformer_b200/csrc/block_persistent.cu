@@ -69,7 +69,7 @@ enum { PH_QKV = 0, PH_WO = 1, PH_W13 = 2, PH_W2 = 3 };
 TP_DEV uint32_t round1k(uint32_t v) { return (v + 1023u) & ~1023u; }
 
 TP_DEV void stamp(const BpArgs& a, int slot) {
-  if (a.trace) a.trace[(size_t)blockIdx.x * kBpTraceSlots + slot] = gtimer();
+  if (a.trace) a.trace[(size_t)blockIdx.x * TP_BLOCK_TRACE_SLOTS + slot] = gtimer();
 }
 
 TP_DEV unsigned ld_acquire(const unsigned* p) {
@@ -910,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage_norm<NB>(a, xs, a.xmid, true, gin, a.ssq, publish, s_red, s_rstd);
       if (tr) stamp(a, 14);
     }, true);
-    if (tr) a.trace[(size_t)blockIdx.x * kBpTraceSlots + 15] = c.waited;
+    if (tr) a.trace[(size_t)blockIdx.x * TP_BLOCK_TRACE_SLOTS + 15] = c.waited;
     for (int tt = threadIdx.x; tt < (nrows >> 1) * NB; tt += kNCons) {
       const int pr = tt / NB, b = tt - pr * NB;
       if (b >= a.nb) continue;

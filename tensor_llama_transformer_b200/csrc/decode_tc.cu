@@ -4,8 +4,12 @@
 //   k_norm_rows     RMSNorm(+Q8) of the residual rows -> the shared input (the
 //                   SyncRmsAtt / SyncRmfFfn buffer) and its hi/lo bf16 pair, the
 //                   tensor-core operand.
-// The other steps of that path (the parts' sums, RoPE and the cache write, SwiGLU,
-// the merges) run in the GEMM's epilogue (gemm_tc.cu, TcFinish).
+//   k_qkv_finalize  sums the contraction parts of the q/k/v plane, applies RoPE
+//                   to q and k pairs, stores q and writes k/v into the cache at pos
+//                   (distributed-llama llamaQkv + llamaMultiheadAtt's cache merge);
+//   k_swiglu_finalize  silu(W1 row) * W3 row from the W1/W3 plane (llamaFfn).
+// The same steps (and the merges) can run instead in the GEMM's epilogue
+// (gemm_tc.cu, TcFinish).
 #include "kernels.cuh"
 
 namespace tp {
@@ -75,11 +79,89 @@ __global__ void __launch_bounds__(kRowThreads) k_norm_rows(NormRowsArgs a) {
   }
 }
 
+// One thread per row pair of the concatenated [q | k | v] rows of one batch row.
+__global__ void k_qkv_finalize(QkvFinalizeArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.y;
+  const int pr = blockIdx.x * blockDim.x + threadIdx.x;
+  const int R = a.qd + 2 * a.kd;
+  if (2 * pr >= R) return;
+  const int row = 2 * pr;
+  float y0 = 0.f, y1 = 0.f;
+  for (int p = 0; p < a.parts; ++p) {  // contraction parts in order
+    const float2 v = *reinterpret_cast<const float2*>(a.plane + ((size_t)p * a.batch + b) * R + row);
+    y0 += v.x;
+    y1 += v.y;
+  }
+  int mat = 0, lrow = row;
+  if (lrow >= a.qd) {
+    lrow -= a.qd;
+    mat = 1;
+    if (lrow >= a.kd) {
+      lrow -= a.kd;
+      mat = 2;
+    }
+  }
+  const int pos = a.pos[b];
+  const int d = lrow % kHeadDim;  // even: first element of the RoPE pair
+  const int head = lrow / kHeadDim;
+  if (mat < 2) {
+    const float freq = powf(a.theta, -(float)d / (float)kHeadDim);
+    float sn, cs;
+    sincosf((float)pos * freq, &sn, &cs);
+    const float r0 = y0 * cs - y1 * sn;
+    const float r1 = y0 * sn + y1 * cs;
+    y0 = r0;
+    y1 = r1;
+  }
+  if (mat == 0) {
+    *reinterpret_cast<float2*>(a.q + (size_t)b * a.qd + lrow) = make_float2(y0, y1);
+  } else {
+    uint16_t* cache = mat == 1 ? a.kc : a.vc;
+    const size_t sq = a.seq ? (size_t)a.seq[b] : (size_t)b;
+    const size_t o = ((sq * a.n_kv_heads + head) * a.max_seq + pos) * kHeadDim + d;
+    *reinterpret_cast<uint32_t*>(cache + o) =
+        (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
+  }
+}
+
+// planes [parts][batch][2F]: columns [0, F) are x W1^T, [F, 2F) are x W3^T, each
+// summed over the contraction parts in order.
+__global__ void k_swiglu_finalize(const float* __restrict__ plane, int parts, int F, int batch,
+                                  float* __restrict__ h, uint16_t* __restrict__ hb) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.y;
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= F) return;
+  float a = 0.f, g = 0.f;
+  for (int p = 0; p < parts; ++p) {
+    const float* pl = plane + ((size_t)p * batch + b) * 2 * F;
+    a += pl[f];
+    g += pl[F + f];
+  }
+  const float v = a / (1.0f + expf(-a)) * g;
+  h[(size_t)b * F + f] = v;
+  bf16_split(v, hb[(size_t)(2 * b) * F + f], hb[(size_t)(2 * b + 1) * F + f]);
+}
+
 }  // namespace
 
 int launch_norm_rows(const NormRowsArgs& a, int batch, cudaStream_t s) {
   if (a.dim % 128 != 0) return TP_EINVAL;
   return launch_pdl(k_norm_rows, dim3(batch), dim3(kRowThreads), 0, s, a);
+}
+
+int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s) {
+  const int pairs = (a.qd + 2 * a.kd) / 2;
+  return launch_pdl(k_qkv_finalize, dim3((pairs + 255) / 256, a.batch), dim3(256), 0, s, a);
+}
+
+int launch_swiglu_finalize(const float* plane, int parts, int F, int batch, float* h,
+                           uint16_t* hb, cudaStream_t s) {
+  return launch_pdl(k_swiglu_finalize, dim3((F + 255) / 256, batch), dim3(256), 0, s, plane, parts,
+                    F, batch, h, hb);
 }
 
 }  // namespace tp

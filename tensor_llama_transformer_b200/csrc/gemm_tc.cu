@@ -155,106 +155,6 @@ struct TcTiles {
   int ntiles;
 };
 
-// Named barrier 2 among the four epilogue warps (128 threads).
-TP_DEV void epilogue_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
-
-// The finish step of one 128-row m-tile of the transposed planes [nseg][N/2][ldo]
-// (see TcFinish), by the four epilogue warps (thread e = 0..127 = 32 q + lane).
-// MERGE: warp q takes batch rows q, q + 4, ..., a float4 of 4 consecutive rows
-// per lane (8-lane groups = one Q8 block of 32), as k_merge does. QKV: thread e
-// takes row pair e % 64 of the tile for batch rows e / 64, e / 64 + 2, ...
-// SWIGLU: thread e takes W1/W3 row f = tile row e for every batch row.
-TP_DEV void tile_finish(const TcGemm& g, const TcTiles& tt, int mt, int q, int lane) {
-  const TcFinish& f = g.fin;
-  const int nb = g.N >> 1, e = 32 * q + lane;
-  const float* planes = static_cast<const float*>(g.out);
-  if (f.kind == TC_FIN_MERGE) {
-    const int64_t D = g.ldo;
-    const int nslices = g.nseg / f.parts, orow0 = mt * BM;
-    for (int b = q; b < nb; b += 4) {
-      const size_t o = (size_t)b * D + orow0 + 4 * lane;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sl = 0; sl < nslices; ++sl) {
-        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < f.parts; ++k) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(
-              planes + (size_t)(sl * f.parts + k) * g.out_seg + o));
-          p.x += v.x;
-          p.y += v.y;
-          p.z += v.z;
-          p.w += v.w;
-        }
-        if (f.quant) q8_roundtrip4(p);
-        acc.x += p.x;
-        acc.y += p.y;
-        acc.z += p.z;
-        acc.w += p.w;
-      }
-      float4* xr = reinterpret_cast<float4*>(f.x + o);
-      float4 v = __ldcg(xr);
-      v.x += acc.x;
-      v.y += acc.y;
-      v.z += acc.z;
-      v.w += acc.w;
-      *xr = v;
-      const float sq = warp_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w);
-      if (lane == 0) f.ssq[(size_t)b * (D >> 7) + mt] = sq;
-    }
-  } else if (f.kind == TC_FIN_QKV) {
-    // the tile's matrix and first row: q rows, then k rows, then v rows
-    const int mat = (mt >= tt.mt_off[1]) + (mt >= tt.mt_off[2]);
-    const int lrow = (mt - tt.mt_off[mat]) * BM + 2 * (e & 63);  // even: a RoPE pair
-    if (lrow >= g.Am[mat]) return;
-    int orow = lrow;
-    for (int j = 0; j < mat; ++j) orow += g.Am[j];
-    const int R = g.Am[0] + g.Am[1] + g.Am[2];
-    const int d = lrow % kHeadDim, head = lrow / kHeadDim;
-    const float freq = powf(f.theta, -(float)d / (float)kHeadDim);
-    for (int b = e >> 6; b < nb; b += 2) {
-      float y0 = 0.f, y1 = 0.f;
-      for (int p = 0; p < f.parts; ++p) {  // contraction parts in order
-        const float2 v =
-            __ldcg(reinterpret_cast<const float2*>(planes + ((size_t)p * nb + b) * R + orow));
-        y0 += v.x;
-        y1 += v.y;
-      }
-      const int pos = f.pos[b];
-      if (mat < 2) {
-        float sn, cs;
-        sincosf((float)pos * freq, &sn, &cs);
-        const float r0 = y0 * cs - y1 * sn;
-        const float r1 = y0 * sn + y1 * cs;
-        y0 = r0;
-        y1 = r1;
-      }
-      if (mat == 0) {
-        *reinterpret_cast<float2*>(f.q + (size_t)b * g.Am[0] + lrow) = make_float2(y0, y1);
-      } else {
-        uint16_t* cache = mat == 1 ? f.kc : f.vc;
-        const size_t sq = f.seq ? (size_t)f.seq[b] : (size_t)b;
-        const size_t o = ((sq * f.n_kv_heads + head) * f.max_seq + pos) * kHeadDim + d;
-        *reinterpret_cast<uint32_t*>(cache + o) =
-            (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
-      }
-    }
-  } else if (f.kind == TC_FIN_SWIGLU) {
-    const int F = g.Am[0], row = (mt - tt.mt_off[0]) * BM + e;  // mt: the W1 tile
-    if (row >= F) return;
-    for (int b = 0; b < nb; ++b) {
-      float a = 0.f, gg = 0.f;
-      for (int p = 0; p < f.parts; ++p) {
-        const float* pl = planes + ((size_t)p * nb + b) * 2 * F;
-        a += __ldcg(pl + row);
-        gg += __ldcg(pl + F + row);
-      }
-      const float v = a / (1.0f + expf(-a)) * gg;
-      f.h[(size_t)b * F + row] = v;
-      bf16_split(v, f.hb[(size_t)(2 * b) * F + row], f.hb[(size_t)(2 * b + 1) * F + row]);
-    }
-  }
-}
-
-
 template <int BN, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
@@ -273,13 +173,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  __shared__ int s_last;  // finish step: this CTA stored the last plane of the tile
-  __shared__ int s_fail;  // finish step: an epilogue warp's wait gave up (all four leave)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
-    s_fail = 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -423,15 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-      const bool got = mbar_wait(&tfull[acc], aph, g.err);
-      if (EPI == TC_EPI_STORE_T_PAIRS_F32 && g.fin.kind != TC_FIN_NONE) {
-        // the finish step below syncs the four epilogue warps: they leave together
-        if (!got) s_fail = 1;
-        epilogue_sync();
-        if (s_fail) break;
-      } else if (!got) {
-        break;
-      }
+      if (!mbar_wait(&tfull[acc], aph, g.err)) break;
       tc_fence_after();
       int seg, nb, mat, m0, orow0;
       decode(tile, seg, nb, mat, m0, orow0);
@@ -532,23 +421,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (EPI == TC_EPI_STORE_T_PAIRS_F32 && g.fin.kind != TC_FIN_NONE) {
-        // the finish step of this m-tile, by the CTA that stored its last plane (the
-        // accumulator is already handed back: the next tile's MMAs go on meanwhile).
-        // SwiGLU counts a W1 tile and its W3 tile together.
-        int mt = tt.mt_off[mat] + m0 / BM;
-        if (g.fin.kind == TC_FIN_SWIGLU && mat == 1) mt -= tt.mt_off[1];
-        const int total = g.fin.kind == TC_FIN_SWIGLU ? 2 * g.nseg : g.nseg;
-        __threadfence();  // this thread's plane stores, before the count
-        epilogue_sync();
-        if (threadIdx.x == 64) s_last = atomicAdd(g.fin.cnt + mt, 1) + 1 == total;
-        epilogue_sync();
-        if (s_last) {
-          __threadfence();  // the other CTAs' planes
-          tile_finish(g, tt, mt, q, lane);
-          if (threadIdx.x == 64) g.fin.cnt[mt] = 0;
-        }
-      }
     }
   }
 
@@ -640,25 +512,6 @@ int launch_tc_gemm(const TcGemm& g, cudaStream_t s) {
   if (!trans && (g.N % 32 != 0 || g.ldo % 8 != 0 || g.nA != 1)) return TP_EINVAL;
   if (trans && g.N > 128) return TP_EINVAL;
   if (g.epi == TC_EPI_STORE_T_PAIRS_F32 && (g.N & 1)) return TP_EINVAL;
-  if (g.fin.kind != TC_FIN_NONE) {
-    const TcFinish& f = g.fin;
-    if (g.epi != TC_EPI_STORE_T_PAIRS_F32 || !f.cnt || f.parts < 1 ||
-        g.out_seg < (int64_t)(g.N / 2) * g.ldo)
-      return TP_EINVAL;
-    const bool ok =
-        f.kind == TC_FIN_MERGE
-            ? g.nA == 1 && g.Am[0] % 128 == 0 && g.ldo == g.Am[0] && g.nseg % f.parts == 0 && f.x &&
-                  f.ssq
-        : f.kind == TC_FIN_QKV
-            ? g.nA == 3 && g.nseg == f.parts && g.ldo == (int64_t)g.Am[0] + g.Am[1] + g.Am[2] &&
-                  g.Am[0] % kHeadDim == 0 && g.Am[1] % kHeadDim == 0 && g.Am[1] == g.Am[2] && f.q &&
-                  f.kc && f.vc && f.pos
-        : f.kind == TC_FIN_SWIGLU
-            ? g.nA == 2 && g.nseg == f.parts && g.Am[0] == g.Am[1] && g.ldo == 2 * (int64_t)g.Am[0] &&
-                  f.h && f.hb
-            : false;
-    if (!ok) return TP_EINVAL;
-  }
   const int BN = trans ? (g.N <= 32 ? 32 : (g.N <= 64 ? 64 : 128)) : 256;
   CUtensorMap mA[3], mB, mB2;
   TcTiles tt{};

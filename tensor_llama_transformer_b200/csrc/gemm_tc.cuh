@@ -25,41 +25,6 @@ enum TcEpi {
 // transposed store, so that each partial plane is [batch, rows]; with the
 // activations given as hi/lo bf16 row pairs (N = 2 x batch) the pair-folding
 // store adds the two columns of each batch row.
-// The last step of a batched-decode product, done by the CTA that stores the last
-// contraction-part plane of a 128-row m-tile (every CTA counts the planes it
-// stores on cnt[tile], which starts at zero and is left so), for every batch row:
-//   TC_FIN_MERGE   x[b][rows] += sum_s sync(sum_k plane[s * parts + k][b][rows])
-//                  in slice order (the Q8 round trip when quant), and the sums of
-//                  squares of those 128 values to ssq[b][tile] (launch_merge's
-//                  layout and arithmetic); requires nA == 1;
-//   TC_FIN_QKV     the q/k/v rows summed over the parts in order, RoPE of q and k
-//                  pairs at pos[b], q stored, k and v written to the caches at
-//                  pos[b] (k_qkv_finalize's arithmetic); A = [Wq; Wk; Wv];
-//   TC_FIN_SWIGLU  h = silu(a) * g with a, g the W1 and W3 rows summed over the
-//                  parts (k_swiglu_finalize's arithmetic), h and its hi/lo bf16
-//                  rows stored; A = [W1; W3], counted per W1 tile over both.
-enum { TC_FIN_NONE = 0, TC_FIN_MERGE = 1, TC_FIN_QKV = 2, TC_FIN_SWIGLU = 3 };
-struct TcFinish {
-  int kind;
-  int* cnt;
-  int parts;  // MERGE: contraction parts per slice; QKV, SWIGLU: parts of the whole product
-  // MERGE
-  float* x;
-  float* ssq;
-  int quant;
-  // QKV
-  float* q;
-  uint16_t* kc;
-  uint16_t* vc;
-  const int32_t* pos;
-  const int32_t* seq;
-  float theta;
-  int n_kv_heads, max_seq;
-  // SWIGLU
-  float* h;
-  uint16_t* hb;
-};
-
 struct TcGemm {
   const void* A[3];
   int Am[3];        // rows of each A matrix
@@ -79,9 +44,6 @@ struct TcGemm {
   // weights): under programmatic dependent launch the producer loads their tiles for
   // the first ring stages before waiting for the previous kernel, the others after.
   int indep;
-  // Work fused after the transposed pair store (TC_EPI_STORE_T_PAIRS_F32) by the
-  // CTA that stores the last plane of a 128-row m-tile (counted on fin.cnt).
-  TcFinish fin;
 };
 enum { TC_INDEP_A = 1, TC_INDEP_B = 2 };
 

@@ -98,78 +98,8 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
                               const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
                               int part, int Q, int cb, int ce, int lane);
 
-// The merge fused into a row-split product's epilogue (distributed-llama
-// SyncAtt + DequantizeAtt + MergeAtt, and the Ffn2 twins): the CTA counts the
-// partial values it stored per piece of kMergePiece outputs; the CTA whose
-// count completes a piece (all nseg slices' partials of it stored) sums the
-// piece's slices in slice order through the sync format and adds the sum to the
-// residual, as k_merge does, then writes the sums of squares of its 128-value
-// chunks for the next RMSNorm and clears the counter. Every thread of the CTA
-// calls this.
-template <int NB>
-TP_DEV void fused_merge(const GemvArgs& a, int R0, int nrows, int rps) {
-  __shared__ int s_done[kMaxMergePieces];
-  __shared__ int s_ndone;
-  const int t = threadIdx.x;
-  int count = 0, total = 0;
-  if (t < a.merge_pieces) {  // this CTA's outputs inside piece t, over the segments it covers
-    const int f0 = t * kMergePiece, f1 = min(f0 + kMergePiece, rps);
-    total = a.nseg * (f1 - f0);
-    for (int sg = R0 / rps; sg <= (R0 + nrows - 1) / rps; ++sg) {
-      const int lo = max(R0, sg * rps + f0), hi = min(R0 + nrows, sg * rps + f1);
-      count += max(0, hi - lo);
-    }
-  }
-  if (t == 0) s_ndone = 0;
-  __threadfence();  // each thread's partial stores, before the counts that publish them
-  __syncthreads();
-  if (count > 0) {
-    int* c = a.merge_cnt + (size_t)a.b0 * a.merge_pieces + t;
-    if (atomicAdd(c, count) + count == total) s_done[atomicAdd(&s_ndone, 1)] = t;
-  }
-  __syncthreads();
-  const int nd = s_ndone;
-  if (nd == 0) return;
-  __threadfence();  // the other CTAs' partials, after their counts
-  const int b = t >> 7, i4 = t & 127;  // 128 threads (4 warps) per batch row
-  for (int k = 0; k < nd; ++k) {
-    const int p = s_done[k];
-    const int f0 = p * kMergePiece, n4 = (min(f0 + kMergePiece, rps) - f0) >> 2;
-    // whole warps: n4 is a multiple of 32, so an 8-lane Q8 group is always complete
-    const bool in = b < a.nb && i4 < n4;
-    const int gb = a.b0 + b;
-    float sq = 0.f;
-    if (in) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sg = 0; sg < a.nseg; ++sg) {
-        float4 v = __ldcg(reinterpret_cast<const float4*>(a.out + (size_t)sg * a.out_seg +
-                                                          (size_t)gb * a.ldo + f0) + i4);
-        if (a.merge_quant) q8_roundtrip4(v);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
-      float4* xr = reinterpret_cast<float4*>(a.merge_x + (size_t)gb * rps + f0) + i4;
-      float4 x = __ldcg(xr);
-      x.x += acc.x;
-      x.y += acc.y;
-      x.z += acc.z;
-      x.w += acc.w;
-      *xr = x;
-      sq = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-    }
-    if (t < NB * 128) {  // each warp's 128 values: one sum of squares (as k_merge)
-      sq = warp_sum(sq);
-      if ((t & 31) == 0 && in)
-        a.merge_ssq[(size_t)gb * (rps >> 7) + (f0 >> 7) + ((t >> 5) & 3)] = sq;
-    }
-    if (t == 0) a.merge_cnt[(size_t)a.b0 * a.merge_pieces + p] = 0;
-  }
-}
-
 template <int NB, int EPI, bool WQ8>
-__global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
+__global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_rstd[NB];
   __shared__ float s_red[8][NB];
@@ -186,6 +116,7 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
   float* res = reinterpret_cast<float*>(smem + pl.res_off);  // [rows of this CTA][NB]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.bar_off);
   uint64_t* empty = full + kMaxStages;
+  uint64_t* staged = empty + kMaxStages;  // the consumers have staged their activations
 
   const int rps = rows_per_seg<EPI>(a);
   const int npairs = a.nseg * (rps >> 1);
@@ -198,6 +129,7 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], nc);
     }
+    mbar_init(staged, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -216,6 +148,13 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
         const int end = stage_end(cur, nrows, R0, rps, P);
         const int s = t % nstage;
         const uint32_t ph = (uint32_t)(t / nstage) & 1u;
+        // beyond the first pl.prefill stages, wait for the consumers' staging: their loads
+        // (the previous kernel's output) then do not queue behind the whole ring's copies
+        if (t == pl.prefill && pl.prefill > 0) {
+          bool st = mbar_wait(staged, 0, a.err);
+          if (WQ8) st = __all_sync(0xffffffffu, st);
+          if (!st) break;
+        }
         bool waited = mbar_wait(&empty[s], ph ^ 1u, a.err);
         if (WQ8) waited = __all_sync(0xffffffffu, waited);
         if (!waited) break;
@@ -287,13 +226,38 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
   } else {
     // ---------------------------------------------------------------- consumers
     pdl_wait();  // activations / residual come from the previous kernel
+    if (tr && threadIdx.x == 0) tr[1] = gtimer();
     const int ncons = nc * 32;
+    // RMSNorm input with one segment (q/k/v, W1/W3 in 1D): each consumer thread loads
+    // the x and gain values of its vectors (8 values, v = thread + 256 k) once, up
+    // front, for the scale and the staging both: one round of loads, not two
+    constexpr int kPreV = 2;
+    const bool pre = a.gain && a.nseg == 1 && nc == 8 && nv <= kPreV * 256;
+    float4 px[NB][kPreV][2], pg[kPreV][2];
+    if (pre) {
+#pragma unroll
+      for (int k = 0; k < kPreV; ++k) {
+        const int v = threadIdx.x + 256 * k;
+        const bool vin = v < nv;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        pg[k][0] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v) : z;
+        pg[k][1] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v + 4) : z;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const bool in = vin && b < a.nb;
+          const float* xr = a.x + (size_t)(a.b0 + b) * a.ldx + 8 * (size_t)v;
+          px[b][k][0] = in ? *reinterpret_cast<const float4*>(xr) : z;
+          px[b][k][1] = in ? *reinterpret_cast<const float4*>(xr + 4) : z;
+        }
+      }
+    }
     if (a.gain && a.ssq) {  // sums of squares left by the merge that produced x
-      if (threadIdx.x < NB) {
+      if (warp < NB) {  // warp b: row b's parts, lanes in stride, then the butterfly
         float t = 0.f;
-        if ((int)threadIdx.x < a.nb)
-          for (int c = 0; c < a.ssq_parts; ++c) t += a.ssq[(size_t)(a.b0 + threadIdx.x) * a.ssq_parts + c];
-        s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
+        if (warp < a.nb)
+          for (int c = lane; c < a.ssq_parts; c += 32) t += a.ssq[(size_t)(a.b0 + warp) * a.ssq_parts + c];
+        t = warp_sum(t);
+        if (lane == 0) s_rstd[warp] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
       }
       consumers_sync(ncons);
     } else if (a.gain) {  // RMSNorm scale of each batch row, over the whole row
@@ -301,7 +265,15 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         float ss = 0.f;
-        if (b < a.nb) {
+        if (pre) {
+#pragma unroll
+          for (int k = 0; k < kPreV; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float4 v = px[b][k][h];
+              ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+            }
+        } else if (b < a.nb) {
           const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
           for (int i = threadIdx.x; i < (D >> 2); i += ncons) {
             const float4 v = xrow[i];
@@ -338,8 +310,9 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
         const size_t col0 = (size_t)seg * a.Ks;
         const int nvr = (nv + 31) & ~31;
         consumers_sync(ncons);
-        for (int b = 0; b < NB; ++b) {
-          for (int v = threadIdx.x; v < nvr; v += ncons) {
+        // one 8-value vector v of batch row b (x, g: the preloaded values when have_pre)
+        auto stage = [&](int b, int v, bool have_pre, float4 px0, float4 px1, float4 pg0,
+                         float4 pg1) {
             const bool in = b < a.nb && v < nv;
             const size_t e0 = (size_t)(a.b0 + b) * a.ldx + col0 + 8 * (size_t)v;
             float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -348,11 +321,13 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
             if (in) {
               if (a.gain) {
                 const float rstd = s_rstd[b];
-                const float4 x0 = *reinterpret_cast<const float4*>(a.x + e0);
-                const float4 x1 = *reinterpret_cast<const float4*>(a.x + e0 + 4);
-                const float4 g0 = *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v);
-                const float4 g1 =
-                    *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v + 4);
+                const float4 x0 = have_pre ? px0 : *reinterpret_cast<const float4*>(a.x + e0);
+                const float4 x1 = have_pre ? px1 : *reinterpret_cast<const float4*>(a.x + e0 + 4);
+                const float4 g0 =
+                    have_pre ? pg0 : *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v);
+                const float4 g1 = have_pre ? pg1
+                                           : *reinterpret_cast<const float4*>(a.gain + col0 +
+                                                                              8 * (size_t)v + 4);
                 xv[0] = __fmul_rn(__fmul_rn(x0.x, rstd), g0.x);
                 xv[1] = __fmul_rn(__fmul_rn(x0.y, rstd), g0.y);
                 xv[2] = __fmul_rn(__fmul_rn(x0.z, rstd), g0.z);
@@ -370,19 +345,47 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
                 const int ncs = (ntiles + tpc - 1) / tpc;
                 const int col = (int)col0 + 8 * v, h = col / kHeadDim, d0 = col - h * kHeadDim;
                 const size_t base = ((size_t)gb * a.n_heads + h) * a.att_nsplit;
+                // the splits' (m, l) in one round of loads, then their outputs 4 splits
+                // at a time (the same sums, in split order)
+                constexpr int kCm = 8;
+                float mcs[kCm], lcs[kCm];
+#pragma unroll
+                for (int c = 0; c < kCm; ++c) {
+                  mcs[c] = c < ncs ? a.att_pml[(base + c) * 2] : -INFINITY;
+                  lcs[c] = c < ncs ? a.att_pml[(base + c) * 2 + 1] : 0.f;
+                }
                 float M = -INFINITY;
-                for (int c = 0; c < ncs; ++c) M = fmaxf(M, a.att_pml[(base + c) * 2]);
+                for (int c = kCm; c < ncs; ++c) M = fmaxf(M, a.att_pml[(base + c) * 2]);
+#pragma unroll
+                for (int c = 0; c < kCm; ++c) M = fmaxf(M, mcs[c]);
                 float L = 0.f;
-                for (int c = 0; c < ncs; ++c) {
-                  const float mc = a.att_pml[(base + c) * 2];
+                auto add_split = [&](float mc, float lc, float4 o0, float4 o1) {
                   const float w = mc == -INFINITY ? 0.f : expf(mc - M);
-                  L = fmaf(w, a.att_pml[(base + c) * 2 + 1], L);
-                  const float4 o0 = *reinterpret_cast<const float4*>(a.att_po + (base + c) * kHeadDim + d0);
-                  const float4 o1 = *reinterpret_cast<const float4*>(a.att_po + (base + c) * kHeadDim + d0 + 4);
+                  L = fmaf(w, lc, L);
                   xv[0] = fmaf(w, o0.x, xv[0]); xv[1] = fmaf(w, o0.y, xv[1]);
                   xv[2] = fmaf(w, o0.z, xv[2]); xv[3] = fmaf(w, o0.w, xv[3]);
                   xv[4] = fmaf(w, o1.x, xv[4]); xv[5] = fmaf(w, o1.y, xv[5]);
                   xv[6] = fmaf(w, o1.z, xv[6]); xv[7] = fmaf(w, o1.w, xv[7]);
+                };
+#pragma unroll
+                for (int c0 = 0; c0 < kCm; c0 += 4) {
+                  if (c0 >= ncs) break;
+                  float4 o[4][2];
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const float* op = a.att_po + (base + c0 + j) * kHeadDim + d0;
+                    const bool cin = c0 + j < ncs;
+                    o[j][0] = cin ? *reinterpret_cast<const float4*>(op) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    o[j][1] = cin ? *reinterpret_cast<const float4*>(op + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  }
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    if (c0 + j < ncs) add_split(mcs[c0 + j], lcs[c0 + j], o[j][0], o[j][1]);
+                }
+                for (int c = kCm; c < ncs; ++c) {  // beyond 8 splits: one at a time
+                  const float* op = a.att_po + (base + c) * kHeadDim + d0;
+                  add_split(a.att_pml[(base + c) * 2], a.att_pml[(base + c) * 2 + 1],
+                            *reinterpret_cast<const float4*>(op), *reinterpret_cast<const float4*>(op + 4));
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) xv[e] = xv[e] / L;
@@ -464,15 +467,31 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
               xs[b * nv + v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
               xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
             }
+        };
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (pre) {
+#pragma unroll
+            for (int k = 0; k < kPreV; ++k) {
+              const int v = threadIdx.x + 256 * k;
+              if (v < nvr) stage(b, v, true, px[b][k][0], px[b][k][1], pg[k][0], pg[k][1]);
+            }
+          } else {
+            for (int v = threadIdx.x; v < nvr; v += ncons) stage(b, v, false, z4, z4, z4, z4);
           }
         }
         consumers_sync(ncons);
         cur_seg = seg;
-        if (tr && t == 0 && threadIdx.x == 0) tr[1] = gtimer();
+        if (t == 0 && threadIdx.x == 0) {
+          if (tr) tr[2] = gtimer();
+          mbar_arrive(staged);
+        }
       }
       // after a wait gives up, keep walking the stages (so that every consumer warp
       // reaches the same named barriers) but skip the work
       if (ok && !mbar_wait(&full[s], ph, a.err)) ok = false;
+      if (tr && t == 0 && threadIdx.x == 0) tr[3] = gtimer();
       if (ok) {
         const uint8_t* st = ring + (size_t)s * 2 * P * slot;
         if constexpr (WQ8) {
@@ -506,7 +525,7 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
       if (lane == 0) mbar_arrive(&empty[s]);
       cur = end;
     }
-    if (tr && threadIdx.x == 0) tr[2] = gtimer();
+    if (tr && threadIdx.x == 0) tr[4] = gtimer();
   }
   __syncthreads();
 
@@ -559,8 +578,7 @@ __global__ void __launch_bounds__(288, 2) k_gemv(GemvArgs a, GemvPlan pl) {
       }
     }
   }
-  if (EPI == EPI_PLAIN && a.merge_x) fused_merge<NB>(a, R0, nrows, rps);
-  if (tr && threadIdx.x == 0) tr[3] = gtimer();
+  if (tr && threadIdx.x == 0) tr[5] = gtimer();
 }
 
 // The int8-weight consumer step (see ring_pairs_dot): each row's codes are read
@@ -623,6 +641,16 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
 
 size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
 
+// Ring stages a GEMV fills before its consumers have staged the activations:
+// TP_GEMV_PREFILL (a tuning knob), default 0 = the whole ring.
+int gemv_prefill() {
+  static const int n = [] {
+    const char* v = getenv("TP_GEMV_PREFILL");
+    return v ? atoi(v) : 0;
+  }();
+  return n;
+}
+
 // Shared memory of a GEMV CTA: kSmemBudget (one CTA per SM, the deepest ring),
 // or TP_GEMV_SMEM_KB (a tuning knob: e.g. 110 lets two GEMV CTAs share an SM, so
 // that the next launch's ring fills while this one finishes).
@@ -642,7 +670,7 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, int budget, GemvPlan* p) 
   const size_t row_bytes = wq8 ? (size_t)Ks + q8w_scale_slot(Ks) : (size_t)Ks * 2;
   const size_t x_bytes = wq8 ? a128((size_t)NB * Ks + (size_t)NB * (Ks / 32) * 4)
                              : a128((size_t)NB * Ks * 4);
-  const size_t bar_bytes = 2 * kMaxStages * 8;
+  const size_t bar_bytes = (2 * kMaxStages + 1) * 8;
   for (int min_stages : {3, 2}) {
     for (int P = 16; P >= 1; P >>= 1) {
       const int Q = P >= 8 ? 1 : 8 / P;
@@ -658,6 +686,7 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, int budget, GemvPlan* p) 
         p->split = Q;
         p->pw = P == 16 ? 2 : 1;
         p->nstage = ns;
+        p->prefill = gemv_prefill() < ns ? gemv_prefill() : 0;
         p->cta_rows = cta_rows;
         p->ring_off = 0;
         p->x_off = a128((size_t)ns * stage);
@@ -697,7 +726,10 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
     if (room < budget) budget = room;
   }
   GemvPlan pl;
-  if (!make_plan(NB, a.Ks, cta_rows, WQ8, budget, &pl)) return TP_ENOTSUP;
+  // a ring too small beside the other CTA (long rows): take the whole SM instead
+  if (!make_plan(NB, a.Ks, cta_rows, WQ8, budget, &pl) &&
+      (budget == kSmemBudget || !make_plan(NB, a.Ks, cta_rows, WQ8, kSmemBudget, &pl)))
+    return TP_ENOTSUP;
   if (set_smem_once((const void*)k_gemv<NB, EPI, WQ8>, (int)pl.total)) return TP_ECUDA;
   return launch_pdl(k_gemv<NB, EPI, WQ8>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
 }
@@ -721,12 +753,6 @@ int launch_nb(const GemvArgs& a, int epi, cudaStream_t s) {
 // Batch rows are handled two at a time (each launch streams the weights once).
 int launch_gemv(const GemvArgs& a0, int epi, cudaStream_t s) {
   if (a0.Ks % 32 != 0 || a0.Ks < 32 || a0.nseg < 1) return TP_EINVAL;
-  if (a0.merge_x) {  // fused merge: whole 128-value chunks per piece, counters sized by the caller
-    if (epi != EPI_PLAIN || a0.rows[0] % 128 != 0 || !a0.merge_cnt || !a0.merge_ssq ||
-        a0.merge_pieces != (a0.rows[0] + kMergePiece - 1) / kMergePiece ||
-        a0.merge_pieces > kMaxMergePieces || a0.ldo != a0.rows[0])
-      return TP_EINVAL;
-  }
   if (a0.wd[0] && a0.ldw % 64 != 0) return TP_EINVAL;  // whole 16-byte scale runs per matrix
   if (((a0.rows[0] | a0.rows[1] | a0.rows[2]) & 1) != 0) return TP_EINVAL;
   for (int b = 0; b < a0.nb;) {

@@ -10,8 +10,8 @@ namespace tp {
 // s*parts .. s*parts+parts-1 of part [n*parts, B, dim] (a slice's contraction
 // split further by the GEMM). With ssq != nullptr the sum of squares of every
 // 128-value chunk of the new row is written too: ssq[b][chunk] (merge_ssq_parts(dim)
-// of them; one warp's float4 lanes summed by warp_sum, in every merge variant, so
-// that all of them give the next RMSNorm the same bits). dim % 128 == 0.
+// of them; one warp's float4 lanes summed by warp_sum, in both merge kernels, so
+// that both give the next RMSNorm the same bits). dim % 128 == 0, parts <= 2.
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts = 1);
 inline int merge_ssq_parts(int dim) { return dim / 128; }
@@ -85,21 +85,9 @@ struct GemvArgs {
   const int32_t* seq;  // cache sequence of each row (nullable: row b uses sequence b)
   int n_heads, n_kv_heads, max_seq;
   float theta;
-  // EPI_PLAIN row-split products with merge_x set: the merge fused into the
-  // epilogue. Each CTA counts the partial values it stored per (batch group b0,
-  // piece of kMergePiece outputs) on merge_cnt[b0 * merge_pieces + piece]; the
-  // CTA whose count completes a piece merges it, x[b] += sum_s sync(out[s][b])
-  // in slice order (the Q8 round trip when merge_quant), writes the sums of
-  // squares of its 128-value chunks to merge_ssq[b][chunk] (as launch_merge) and
-  // sets the counter back to zero (counters start at zero and every launch
-  // leaves them so).
-  float* merge_x;
-  float* merge_ssq;
-  int* merge_cnt;
-  int merge_quant;
-  int merge_pieces;
   // optional %globaltimer stamps (ns) of CTA c at trace[c * trace_stride + k]:
-  // k = 0 start, 1 activations staged, 2 last ring stage consumed, 3 end
+  // k = 0 start, 1 previous kernel complete, 2 activations staged, 3 first ring
+  // stage arrived, 4 last ring stage consumed, 5 end
   unsigned long long* trace;
   int trace_stride;
   // shared memory of another kernel's CTA that this launch's CTAs must fit beside
@@ -109,9 +97,7 @@ struct GemvArgs {
   int co_smem;
   int* err;  // device error flag, set when a bounded wait gives up (nullable)
 };
-// Outputs per piece (counter) of the fused merge.
-constexpr int kMergePiece = 512;
-constexpr int kMaxMergePieces = 64;
+
 
 // Shared-memory plan of the GEMV (host computes, kernel reads): NC consumer
 // warps, row pairs per stage (each pair split over `split` warps), ring depth,
@@ -123,6 +109,7 @@ struct GemvPlan {
   int split;
   int pw;  // row pairs per warp and stage (2 with 16 pairs per stage)
   int nstage;
+  int prefill;  // ring stages filled before the activations are staged (0: all of them)
   int cta_rows;
   size_t ring_off, x_off, res_off, bar_off, total;
 };
@@ -180,6 +167,23 @@ struct NormRowsArgs {
 };
 int launch_norm_rows(const NormRowsArgs& a, int batch, cudaStream_t s);
 
+struct QkvFinalizeArgs {
+  const float* plane;  // [parts][batch][qd + 2 kd]
+  int parts, batch, qd, kd;
+  const int32_t* pos;
+  const int32_t* seq;  // cache sequence of each row (nullable: row b)
+  float theta;
+  float* q;            // [batch, qd]
+  uint16_t* kc;
+  uint16_t* vc;
+  int n_kv_heads, max_seq;
+};
+int launch_qkv_finalize(const QkvFinalizeArgs& a, cudaStream_t s);
+// h = silu(a) * g from planes [parts][batch][2F] (a = columns [0, F), g = [F, 2F),
+// each the sum of the parts in order), with its hi/lo bf16 pair rows.
+int launch_swiglu_finalize(const float* plane, int parts, int F, int batch, float* h,
+                           uint16_t* hb, cudaStream_t s);
+
 // ------------------------------------------------------------------ persistent block
 // One weight-streaming phase of the persistent block kernel: the rows of up to
 // three matrices (q/k/v stacked; W1/W3 interleaved row for row), contracted over
@@ -226,7 +230,7 @@ struct BpArgs {
 // the activation staging of phase D; 15 the time (ns) thread 0 waited for ring
 // stages during phase D.
 constexpr int kBpTraceSlots = 16;
-static_assert(kBpTraceSlots == TP_BLOCK_TRACE_SLOTS, "trace layout");
+static_assert(kBpTraceSlots <= TP_BLOCK_TRACE_SLOTS, "trace layout");
 // Fills the launch plan (grid, shared-memory layout, rows per stage); false when
 // the shapes rule the persistent kernel out.
 bool plan_block_persistent(BpArgs& a, int nb_max);

@@ -25,36 +25,13 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
   const int b = blockIdx.y;
   const int i4 = blockIdx.x * kMergeThreads + threadIdx.x;  // float4 index within the row
   const int n4 = dim >> 2;
-  // whole warps stay in the loop so that an 8-lane Q8 group is always complete
-  const bool in = i4 < n4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n; ++s) {
-    // slice s's partial: the sum of its contraction parts (planes s*parts .. s*parts+parts-1)
-    float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < parts && in; ++k) {
-      const float4 v = reinterpret_cast<const float4*>(part + ((size_t)(s * parts + k) * B + b) * dim)[i4];
-      p.x += v.x;
-      p.y += v.y;
-      p.z += v.z;
-      p.w += v.w;
-    }
-    if (quant) q8_roundtrip4(p);
-    acc.x += p.x;
-    acc.y += p.y;
-    acc.z += p.z;
-    acc.w += p.w;
-  }
-  float sq = 0.f;
-  if (in) {
-    float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim);
-    float4 v = xr[i4];
-    v.x += acc.x;
-    v.y += acc.y;
-    v.z += acc.z;
-    v.w += acc.w;
-    xr[i4] = v;
-    sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  }
+  if (blockIdx.x * kMergeThreads + (threadIdx.x & ~31) >= n4) return;  // dim % 128: whole warps
+  // slice s's partial: the sum of its contraction parts (planes s*parts .. s*parts+parts-1)
+  float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim) + i4;
+  const float4 v = merge_lane4(part, (size_t)B * dim, (size_t)b * dim + 4 * (size_t)i4, n, parts,
+                               quant, *xr);
+  *xr = v;
+  float sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   if (ssq) {  // each warp's 128 values: their sum of squares, for the next RMSNorm
     sq = warp_sum(sq);
     const int chunk = (blockIdx.x * kMergeThreads + (threadIdx.x & ~31)) >> 5;
@@ -172,6 +149,7 @@ int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; 
 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts) {
+  if (parts < 1 || parts > 2 || dim % 128 != 0) return TP_EINVAL;
   const dim3 grid(merge_grid(dim), B);
   return launch_pdl(k_merge, grid, dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim, quant, ssq);
 }
