@@ -315,6 +315,37 @@ def make_events(torch, n):
     return evs
 
 
+def gemv_timeline(torch, tpb, h, fwd, local):
+    """Per-CTA timeline of the four slice GEMVs of a block step (%globaltimer stamps)
+    in one replay of two captured steps, relative to the first q/k/v CTA's start of
+    the first: per GEMV and mark, [min, median, max] over CTAs in us, and how many
+    CTAs started more than 2 us after the GEMV's first."""
+    nsm = torch.cuda.get_device_properties(local).multi_processor_count
+    tr = torch.zeros(nsm * tpb.TP_BLOCK_TRACE_SLOTS, dtype=torch.int64, device="cuda")
+    tpb.tp_block_set_trace(h, tr, tr.numel() * 8)
+    g_tr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_tr):
+        for _ in range(2):
+            fwd()
+    tpb.tp_block_set_trace(h, None, 0)
+    g_tr.replay()
+    torch.cuda.synchronize()
+    del g_tr
+    t = tr.view(nsm, -1).cpu().numpy().astype("float64")
+    timeline = {}
+    base = t[t[:, 0] > 0, 0].min()
+    marks = ("start", "prev_done", "norm", "staged", "first_stage", "consumed", "end")
+    for gi, name in enumerate(("qkv", "wo", "w13", "w2")):
+        cols = t[:, 7 * gi:7 * gi + 7]
+        cols = cols[cols[:, 0] > 0]
+        timeline[name] = {m: [round(float(f((cols[:, k] - base) / 1e3)), 2)
+                              for f in (min, statistics.median, max)]
+                          for k, m in enumerate(marks)}
+        st = (cols[:, 0] - cols[:, 0].min()) / 1e3
+        timeline[name]["late_ctas"] = int((st > 2.0).sum())
+    return timeline
+
+
 def bench_block(args, world, rank, local):
     import torch
 
@@ -405,30 +436,7 @@ def bench_block(args, world, rank, local):
     stage_ms_max = [allreduce_max(v, world) for v in stage_ms]
     del g, g_ev
 
-    # per-CTA timeline of the four slice GEMVs (%globaltimer stamps) in one replay of a
-    # captured step, relative to the first q/k/v CTA's start: the median over CTAs of
-    # start / activations staged / last stage consumed / end, and the latest end
-    nsm = torch.cuda.get_device_properties(local).multi_processor_count
-    tr = torch.zeros(nsm * tpb.TP_BLOCK_TRACE_SLOTS, dtype=torch.int64, device="cuda")
-    tpb.tp_block_set_trace(h, tr, tr.numel() * 8)
-    g_tr = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_tr):
-        for _ in range(2):
-            fwd()
-    tpb.tp_block_set_trace(h, None, 0)
-    g_tr.replay()
-    torch.cuda.synchronize()
-    del g_tr
-    t = tr.view(nsm, -1).cpu().numpy().astype("float64")
-    timeline = {}
-    base = t[t[:, 0] > 0, 0].min()
-    marks = ("start", "prev_done", "staged", "first_stage", "consumed", "end")
-    for gi, name in enumerate(("qkv", "wo", "w13", "w2")):
-        cols = t[:, 6 * gi:6 * gi + 6]
-        cols = cols[cols[:, 0] > 0]
-        timeline[name] = {m: [round(float(f((cols[:, k] - base) / 1e3)), 2)
-                              for f in (min, statistics.median, max)]
-                          for k, m in enumerate(marks)}
+    timeline = gemv_timeline(torch, tpb, h, fwd, local)
 
     # end to end through the public API: host buffers, copies inside the timed region
     xh = torch.empty_like(dev.x, device="cpu").pin_memory()
@@ -459,8 +467,8 @@ def bench_block(args, world, rank, local):
     w13_bytes = 2 * s.ffn_dim * s.dim * 2 + B * s.dim * (1 + 4 / 32) + B * s.ffn_dim * 4
     w13_s = stage_ms_max[STAGES.index("norm_w13_swiglu")] / 1e3
     # batch 1 (weight-streaming path): q/k/v GEMV, attention splits, W_O GEMV (which also
-    # combines the splits and ends with the fused merge), W1/W3 GEMV, W2 GEMV (+ merge)
-    launches_per_step = 5
+    # combines the splits), merge, W1/W3 GEMV, W2 GEMV, merge
+    launches_per_step = 7
     res = {
         "tokens_per_s": world * B * K / (ms_max / 1e3), "ms_per_step": ms_max / K, "K": K,
         "block_gbs": (wbytes + kvbytes) / step_s / 1e9, "stage_us": {
@@ -783,7 +791,9 @@ def bench_c2_q8w(args):
         torch.cuda.synchronize()
         tpb.tp_block_destroy(h)
         return {"profile": "c2q8w", "steps": args.profile_steps}
-    ms = _time_graph(torch, lambda: tpb.tp_block_forward(h, x, kc, vc, pos, B), 100, 20)
+    fwd = lambda: tpb.tp_block_forward(h, x, kc, vc, pos, B)  # noqa: E731
+    ms = _time_graph(torch, fwd, 100, 20)
+    timeline = gemv_timeline(torch, tpb, h, fwd, torch.cuda.current_device())
     err = int(ws[tpb.tp_block_buffer(h, 7)[0]:][:4].view(torch.int32).item())
     tpb.tp_block_destroy(h)
     wb_bf16, kvb = block_bytes(s)
@@ -792,6 +802,7 @@ def bench_c2_q8w(args):
     gbs = (wb + kvb) / (ms / 1e3) / 1e9
     return {"us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "hbm_gbs": gbs,
             "frac": gbs / hbm, "bytes_per_step": wb + kvb, "pipeline_error": err,
+            "gemv_timeline_us": timeline,
             "workload": "C2 block with int8 weights (Q8 codes + float32 scales per 32) and Q8 "
                         "activations, batch 1, n=4"}
 
@@ -869,11 +880,15 @@ def bench_ffn(args):
     flops = 2.0 * B * 2 * E * F
     out = {}
     _, bf16_tf, _, peak_kind = peaks()
-    forms = [("fused", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FUSED),
-             ("1d64_faithful", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FAITHFUL),
-             ("2d8x8_faithful", tpb.TP_PART_2D, 64, 8, 8, tpb.TP_MERGE_FAITHFUL)]
-    for name, part, n, gx, gy, merge in forms:
-        desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, part, n, gx, gy, 0, merge)
+    # faithful: every slice's partial formed on its own and summed in slice order (in
+    # the GEMM epilogue), _q8 with the Q8 round trip of every partial
+    forms = [("fused", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FUSED, 0),
+             ("1d64_faithful", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FAITHFUL, 0),
+             ("1d64_faithful_q8", tpb.TP_PART_1D, 64, 1, 1, tpb.TP_MERGE_FAITHFUL, 1),
+             ("2d8x8_faithful", tpb.TP_PART_2D, 64, 8, 8, tpb.TP_MERGE_FAITHFUL, 0),
+             ("2d8x8_faithful_q8", tpb.TP_PART_2D, 64, 8, 8, tpb.TP_MERGE_FAITHFUL, 1)]
+    for name, part, n, gx, gy, merge, quant in forms:
+        desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, part, n, gx, gy, quant, merge)
         nb = tpb.tp_ffn_workspace_bytes(desc)
         ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
         for _ in range(2):
@@ -1013,8 +1028,9 @@ def main(argv=None):
             "gemv_timeline_us": res["gemv_timeline_us"],
             "gemv_timeline_note": "one replay of a captured step: per slice GEMV, [min, median, "
                                   "max] over CTAs (us from the first q/k/v CTA's start) of its "
-                                  "start, previous kernel complete, activations staged, first "
-                                  "weight stage arrived, last stage consumed, end",
+                                  "start, previous kernel complete, RMSNorm scale known, "
+                                  "activations staged, first weight stage arrived, last stage "
+                                  "consumed, end",
             "stage_note": "per-stage CUDA-event times from a replay of the same steps with an event "
                           "before every stage (serialised, so upper bounds); value and ms_per_step "
                           "come from the event-free graph; the merges run in the W_O and W2 "

@@ -282,10 +282,10 @@ TP_API int tp_block_set_persistent(tp_block* blk, int enable);
  * block runs as separate kernels and the trace is not written. A forward on the
  * kernel-per-step weight-streaming path (batch <= 5, persistent kernel off)
  * writes instead, for each of its four slice GEMVs g (0 q/k/v, 1 W_O, 2 W1/W3,
- * 3 W2) and CTA c of that launch, trace[c * TP_BLOCK_TRACE_SLOTS + 6g + k]: k = 0
- * start, 1 the previous kernel complete (its wait returned), 2 activations
- * staged, 3 the first weight stage arrived, 4 the last stage consumed, 5 end
- * (after the epilogue and the fused merge); for batch > 2 the last launch of each
+ * 3 W2) and CTA c of that launch, trace[c * TP_BLOCK_TRACE_SLOTS + 7g + k]: k = 0
+ * start, 1 the previous kernel complete (its wait returned), 2 the RMSNorm scale
+ * known, 3 activations staged, 4 the first weight stage arrived, 5 the last stage
+ * consumed, 6 end (after the epilogue); for batch > 2 the last launch of each
  * wins. The persistent kernel uses slots 0-15.
  * Errors: TP_EINVAL (NULL handle, buffer too small). */
 #define TP_BLOCK_TRACE_SLOTS 32
@@ -342,15 +342,19 @@ typedef struct {
   int32_t partition;  /* TP_PART_1D (n = n_slices over F) or TP_PART_2D (grid_x over E, grid_y over F) */
   int32_t n_slices, grid_x, grid_y;
   int32_t sync_quant; /* 1 = Q8 round trip of every partial before its merge */
-  int32_t merge;      /* TP_MERGE_FAITHFUL: partials materialised and summed in slice order;
-                         TP_MERGE_FUSED: partials accumulated in slice order inside the
-                         contraction (bf16 only, sync_quant must be 0) */
+  int32_t merge;      /* TP_MERGE_FAITHFUL: every slice's partial formed on its own in
+                         float32 (through Q8 with sync_quant) and the partials summed in
+                         slice order; TP_MERGE_FUSED: the slices' contraction ranges
+                         accumulated in slice order inside the contraction, rounded once
+                         (bf16 only, sync_quant must be 0) */
 } tp_ffn_desc;
 
 /* Workspace bytes for tp_ffn_forward with this descriptor: the error word, the
- * materialised partials (per slice for TP_MERGE_FAITHFUL; per E-slice of stage 1
- * for 2D) and the hidden activations H [B,F]. Errors: TP_EINVAL (sizes that do
- * not divide, see tp_ffn_forward), TP_ENOTSUP. */
+ * hidden activations H [B,F] and, where partials are materialised, their float32
+ * planes: TP_F32 with TP_MERGE_FAITHFUL (every stage), and the 2D SwiGLU first
+ * stage in bf16 (per E-slice). bf16 faithful forms otherwise sum the partials in
+ * the tensor-core GEMM's epilogue and need no planes. Errors: TP_EINVAL (sizes
+ * that do not divide, see tp_ffn_forward), TP_ENOTSUP. */
 TP_API int tp_ffn_workspace_bytes(const tp_ffn_desc* d, size_t* out_bytes);
 
 /* The tensor-parallel FFN Y = act(X W1^T [, X W3^T]) W2^T.

@@ -59,18 +59,37 @@ int set_smem_once(const void* kernel, int bytes) {
 }
 
 // Tuning switches read once from the environment (for comparison runs):
-//   TP_ATT_OVERLAP=1  the W_O GEMV streams its weights beside the attention (one
-//                     attention CTA per SM, the GEMV's ring sized to fit next to
-//                     it); off by default: the smaller ring streams slower than the
-//                     overlap gains.
 bool env_flag(const char* name, bool dflt) {
   const char* v = getenv(name);
   if (!v || !v[0]) return dflt;
   return v[0] != '0';
 }
-bool att_overlap_enabled() {
-  static const bool on = env_flag("TP_ATT_OVERLAP", false);
+//   TP_L2_AHEAD=0     the merge kernels do not prefetch the next GEMV's first rows.
+bool l2_ahead_enabled() {
+  static const bool on = env_flag("TP_L2_AHEAD", true);
   return on;
+}
+// Bytes per next-GEMV CTA the merge prefetches (a W1/W3 pair is 2 rows).
+constexpr int64_t kAheadBytes = 192 * 1024;
+
+int prefer_max_shared(const void* kernel) {
+  struct Entry {
+    const void* fn;
+    int dev;
+  };
+  static Entry tab[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TP_ECUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (tab[i].fn == kernel && tab[i].dev == dev) return TP_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return TP_ECUDA;
+  if (used < 256) tab[used++] = Entry{kernel, dev};
+  return TP_OK;
 }
 
 bool pdl_enabled() {
@@ -302,19 +321,19 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
 // slice order through the sync format. Rank block: the same over the gathered
 // sync buffer, which holds every rank's slices in slice order.
 int merge_step(tp_block* blk, float* x, const float* part, int nseg, int parts, int batch,
-               cudaStream_t s) {
+               cudaStream_t s, const L2Ahead* ahead = nullptr) {
   const Cfg& c = blk->c;
   float* ssq = at<float>(blk, BUF_SSQ);
-  if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts);
+  if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts, ahead);
   return launch_merge_sync(x, at<uint8_t>(blk, BUF_RECV), c.n * c.world, batch, c.d.dim, c.quant,
                            ssq, s);
 }
 
-// Trace slots 6g .. 6g+5 of every CTA for the slice GEMV g (0 q/k/v, 1 W_O,
+// Trace slots 7g .. 7g+6 of every CTA for the slice GEMV g (0 q/k/v, 1 W_O,
 // 2 W1/W3, 3 W2) when a trace buffer is set.
 void set_gemv_trace(const tp_block* blk, GemvArgs& a, int g) {
   if (!blk->trace) return;
-  a.trace = blk->trace + 6 * g;
+  a.trace = blk->trace + 7 * g;
   a.trace_stride = TP_BLOCK_TRACE_SLOTS;
 }
 
@@ -593,10 +612,8 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   float* part = at<float>(blk, BUF_PART);
   float* hbuf = at<float>(blk, BUF_H);
   const int nseg2 = c.partition == TP_PART_1D ? c.n : c.gy;
-  // context splits of the attention, which the W_O GEMV's staging combines; with
-  // the overlap on, one attention CTA per SM leaves room for the W_O GEMV's CTA
-  const bool overlap = att_overlap_enabled() && pdl_enabled();
-  const int att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq, overlap ? 1 : 2);
+  // context splits of the attention, which the W_O GEMV's staging combines
+  const int att_nsplit = attention_nsplit(batch, H, Hkv, d.max_seq);
 
   if (phase <= 0) {
     // a1-a4: RMSNorm (+Q8, the buffer every slice reads) fused into the q/k/v slice
@@ -672,7 +689,6 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
       a.att_po = at<float>(blk, BUF_PO);
       a.att_pml = at<float>(blk, BUF_PML);
       a.att_nsplit = att_nsplit;
-      if (overlap) a.co_smem = attention_cta_smem();
       a.att_out = at<float>(blk, BUF_ATT);
       a.pos = pos;
       a.n_heads = H;
@@ -689,9 +705,20 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   }
   if (phase <= 1) {
     // a6: sync + dequantise + merge into the residual (a rank block: of the
-    // gathered buffer)
+    // gathered buffer); while it waits, the merge prefetches into L2 the first
+    // W1/W3 rows each CTA of the next GEMV streams
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    L2Ahead ahead{};
+    if (c.partition == TP_PART_1D && !blk->wq8 && l2_ahead_enabled()) {
+      ahead.w[0] = blk->w.w1;
+      ahead.w[1] = blk->w.w3;
+      ahead.ld_bytes = (int64_t)D * 2;
+      ahead.row_bytes = D * 2;
+      ahead.npairs = F;
+      ahead.grid = num_sms() < F ? num_sms() : F;
+      ahead.pairs = (int)(kAheadBytes / (2 * ahead.row_bytes));
+    }
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s, &ahead))) return rc;
     // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if (c.partition == TP_PART_1D) {

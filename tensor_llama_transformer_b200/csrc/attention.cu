@@ -498,9 +498,9 @@ int attention_max_splits(int max_seq) { return (max_seq + kTile - 1) / kTile; }
 // Splits per (batch row, kv head): the count that minimises waves x (tiles per
 // CTA + 1), two CTAs resident per SM, over a context of max_seq positions. The
 // kernels divide the actual context (pos + 1) over that many splits.
-int attention_splits(int B, int Hkv, int max_seq, int per_sm = 2) {
+int attention_splits(int B, int Hkv, int max_seq) {
   const int T = attention_max_splits(max_seq);
-  const long slots = (long)per_sm * num_sms();
+  const long slots = 2L * num_sms();
   int best = 1;
   long best_cost = -1;
   for (int sp = 1; sp <= T; ++sp) {
@@ -516,20 +516,10 @@ int attention_splits(int B, int Hkv, int max_seq, int per_sm = 2) {
   return best;
 }
 
-int attention_nsplit(int B, int H, int Hkv, int max_seq, int per_sm) {
+int attention_nsplit(int B, int H, int Hkv, int max_seq) {
   const int G = H / Hkv;
   const int hgroups = G > 8 ? G / 8 : 1;  // CTAs per kv head
-  return attention_splits(B, Hkv * hgroups, max_seq, per_sm);
-}
-
-int attention_cta_smem() {
-  static int bytes = [] {
-    cudaFuncAttributes fa{};
-    const int st = cudaFuncGetAttributes(&fa, (const void*)k_attn_split<1>) == cudaSuccess
-                       ? (int)fa.sharedSizeBytes : 1024;
-    return kSmemBytes + st;
-  }();
-  return bytes;
+  return attention_splits(B, Hkv * hgroups, max_seq);
 }
 
 int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine) {

@@ -219,11 +219,18 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // the environment variable TP_PDL=0 turns it off, for comparison runs).
 bool pdl_enabled();
 
+// Every kernel asks for the largest shared-memory carve-out (once per kernel and
+// device): an SM whose L1 / shared split changes between kernels must drain first,
+// so a small kernel run with a smaller carve-out would keep the next big-ring
+// kernel's CTA off its SM until it ends.
+int prefer_max_shared(const void* kernel);
+
 // Launches `kernel` on `s`, allowing it to overlap its predecessor's tail
 // (programmatic dependent launch) when pdl_enabled().
 template <typename... KArgs, typename... Args>
 int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                Args&&... args) {
+  if (prefer_max_shared((const void*)kernel)) return TP_ECUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

@@ -9,11 +9,17 @@
 // partial-sum stage before the activation.
 //
 // On one GPU every slice is a segment of the same launch: a segment is the
-// contraction range one slice owns, and its partial product is written to its
-// own plane of the partial buffer, which the merge kernel sums in slice order
-// (TP_MERGE_FAITHFUL). With TP_MERGE_FUSED the slices' contraction ranges are
+// contraction range one slice owns. TP_MERGE_FAITHFUL forms every slice's
+// partial product on its own (float32) and sums the partials in slice order,
+// each through the Q8 round trip when quantising: for bf16 inside the tensor-core
+// GEMM (the CTA that owns an output tile computes its segments one after another
+// and adds them up in its epilogue; in 1D the first stage has one segment, so its
+// activation is applied to the accumulator directly), for float32 (and the 2D
+// SwiGLU first stage) by writing each partial to its own plane of the workspace
+// and summing the planes in the merge kernel. The sums are the same float32
+// additions either way. With TP_MERGE_FUSED the slices' contraction ranges are
 // accumulated in slice order inside the tensor-core accumulator instead, which
-// is the same sum without materialising the partials.
+// is the sum of the exact partials rounded once.
 #include "ffn.cuh"
 #include "gemm_tc.cuh"
 
@@ -24,6 +30,7 @@ size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct FfnPlan {
   int nseg1, nseg2, Ks1, Ks2, swiglu, esize;
+  bool planes1, planes2;  // stage 1 / stage 2 partials materialised in the workspace
   size_t off_err, off_p1a, off_p1b, off_h, off_p2, total;
 };
 
@@ -54,17 +61,22 @@ int plan_ffn(const tp_ffn_desc* d, FfnPlan* p) {
   if (d->merge == TP_MERGE_FUSED && (d->dtype != TP_BF16 || d->sync_quant)) return TP_ENOTSUP;
   const size_t B = d->batch, E = d->E, F = d->F;
   const bool fused = d->merge == TP_MERGE_FUSED;
+  const bool f32 = d->dtype == TP_F32;
+  // bf16: the tensor-core GEMM sums the segments itself, except for the 2D SwiGLU
+  // first stage (two products per hidden value)
+  p->planes1 = !fused && (f32 || (p->nseg1 > 1 && p->swiglu));
+  p->planes2 = !fused && f32;
   size_t o = 0;
   p->off_err = o;
   o += 256;
   p->off_p1a = o;
-  if (!fused) o += a256((size_t)p->nseg1 * B * F * 4);
+  if (p->planes1) o += a256((size_t)p->nseg1 * B * F * 4);
   p->off_p1b = o;
-  if (!fused && p->swiglu) o += a256((size_t)p->nseg1 * B * F * 4);
+  if (p->planes1 && p->swiglu) o += a256((size_t)p->nseg1 * B * F * 4);
   p->off_h = o;
   o += a256(B * F * p->esize);
   p->off_p2 = o;
-  if (!fused) o += a256((size_t)p->nseg2 * B * E * 4);
+  if (p->planes2) o += a256((size_t)p->nseg2 * B * E * 4);
   p->total = o;
   return TP_OK;
 }
@@ -146,36 +158,53 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
   float* P1a = reinterpret_cast<float*>(ws + p.off_p1a);
   float* P1b = reinterpret_cast<float*>(ws + p.off_p1b);
   float* P2 = reinterpret_cast<float*>(ws + p.off_p2);
-  auto contract = [&](const void* A, int64_t lda, const void* Bm, int64_t ldb, float* P, int M,
-                      int N, int Ks, int nseg) -> int {
-    if (d->dtype == TP_F32) return launch_gemm_simt(TP_F32, A, lda, Bm, ldb, P, M, N, Ks, nseg, s);
+  // one bf16 tensor-core product over nseg segments of Ks with epilogue `epi`
+  auto tc = [&](const void* A, int64_t lda, const void* Bm, const void* Bm2, int64_t ldb, void* out,
+                int M, int N, int Ks, int nseg, int epi, int quant) -> int {
     TcGemm g{};
     g.A[0] = A;
     g.Am[0] = M;
     g.nA = 1;
     g.lda = lda;
     g.B = Bm;
+    g.B2 = Bm2;
     g.ldb = ldb;
     g.N = N;
     g.K = Ks;
     g.nseg = nseg;
-    g.epi = TC_EPI_STORE_F32;
-    g.out = P;
+    g.epi = epi;
+    g.quant = quant;
+    g.out = out;
     g.ldo = N;
     g.out_seg = (int64_t)M * N;
     g.err = err;
     g.indep = TC_INDEP_B;  // the weights
     return launch_tc_gemm(g, s);
   };
+  // the partials of A B^T over nseg segments of Ks, one float32 plane each
+  auto contract = [&](const void* A, int64_t lda, const void* Bm, int64_t ldb, float* P, int M,
+                      int N, int Ks, int nseg) -> int {
+    if (d->dtype == TP_F32) return launch_gemm_simt(TP_F32, A, lda, Bm, ldb, P, M, N, Ks, nseg, s);
+    return tc(A, lda, Bm, nullptr, ldb, P, M, N, Ks, nseg, TC_EPI_STORE_F32, 0);
+  };
+  // in 1D the hidden columns stay local to their slice: no sync buffer there
+  const int quant1 = d->partition == TP_PART_2D ? d->sync_quant : 0;
 
-  // stage 1: partials of X W1^T over the E-segments (one segment in 1D)
-  rc = contract(X, E, W1, E, P1a, B, F, p.Ks1, p.nseg1);
-  if (rc) return rc;
-  if (p.swiglu) {
-    rc = contract(X, E, W3, E, P1b, B, F, p.Ks1, p.nseg1);
+  // stage 1: H = act(sum over the E-segments of X W1^T [, X W3^T]) (one segment in 1D)
+  if (!p.planes1) {
+    if (p.nseg1 == 1)
+      rc = tc(X, E, W1, p.swiglu ? W3 : nullptr, E, H, B, F, p.Ks1, 1,
+              p.swiglu ? TC_EPI_SWIGLU_BF16 : TC_EPI_RELU_BF16, 0);
+    else
+      rc = tc(X, E, W1, nullptr, E, H, B, F, p.Ks1, p.nseg1, TC_EPI_SEGSUM_RELU_BF16, quant1);
     if (rc) return rc;
-  }
-  {
+  } else {
+    rc = contract(X, E, W1, E, P1a, B, F, p.Ks1, p.nseg1);
+    if (rc) return rc;
+    if (p.swiglu) {
+      rc = contract(X, E, W3, E, P1b, B, F, p.Ks1, p.nseg1);
+      if (rc) return rc;
+    }
     FfnMergeArgs m{};
     m.P1 = P1a;
     m.P3 = p.swiglu ? P1b : nullptr;
@@ -183,8 +212,7 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
     m.nseg = p.nseg1;
     m.M = B;
     m.N = F;
-    // in 1D the hidden columns stay local to their slice: no sync buffer there
-    m.quant = d->partition == TP_PART_2D ? d->sync_quant : 0;
+    m.quant = quant1;
     m.act = p.swiglu ? ACT_SWIGLU : ACT_RELU;
     if (d->dtype == TP_F32)
       m.out_f32 = static_cast<float*>(H);
@@ -193,7 +221,9 @@ int tp_ffn_forward(const tp_ffn_desc* d, const void* X, const void* W1, const vo
     rc = launch_ffn_merge(m, s);
     if (rc) return rc;
   }
-  // stage 2: partials of H W2^T over the F-segments
+  // stage 2: Y = sum over the F-segments of H W2^T
+  if (!p.planes2) return tc(H, F, W2, nullptr, F, Y, B, E, p.Ks2, p.nseg2, TC_EPI_SEGSUM_F32,
+                            d->sync_quant);
   rc = contract(H, F, W2, F, P2, B, E, p.Ks2, p.nseg2);
   if (rc) return rc;
   FfnMergeArgs m{};

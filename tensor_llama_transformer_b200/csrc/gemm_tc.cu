@@ -8,9 +8,14 @@
 // partial product goes to its own plane of the output, to be summed by the
 // merge (aiterms.tw "Tensor Parallelism": Linear2 split by rows, then an
 // all-reduce; Pope et al. demo1: 2D weight-stationary adds a partial-sum stage
-// before the activation). The FFN puts tokens on M and features on N (N tile
-// 256); batched decode puts weight rows on M and the batch on N (N tile 32 or
-// 64, transposed store), so the weight stream is the M x K operand.
+// before the activation), or, with the segment-sum epilogue, is summed in
+// slice order by the CTA that owns the output tile: it computes the tile's
+// segments one after another, each into a fresh TMEM accumulator, and adds
+// each partial (through the Q8 round trip when quantising) to a running sum
+// in registers, so the partials never reach HBM. The FFN puts tokens on M and
+// features on N (N tile 256, 128 with the segment sum); batched decode puts
+// weight rows on M and the batch on N (N tile 32 or 64, transposed store), so
+// the weight stream is the M x K operand.
 //
 // Structure (one CTA per SM, 192 threads):
 //   warp 0  : TMA producer — 128x64 A tile and BNx64 B tile per stage, 128-byte
@@ -29,13 +34,13 @@
 #include <cuda.h>
 
 #include "gemm_tc.cuh"
+#include "pipeline.cuh"
 
 namespace tp {
 namespace {
 
 constexpr int BM = 128, BK = 64, THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 template <int BN>
 struct TcCfg {
@@ -46,47 +51,6 @@ struct TcCfg {
   // two accumulators of BN columns, allocated as a power of two >= 32
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
 };
-
-TP_DEV uint32_t s2u(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-TP_DEV uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-TP_DEV void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
-}
-TP_DEV void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
-               : "memory");
-}
-TP_DEV void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
-}
-TP_DEV bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(s2u(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Wait for the phase of `parity` to complete; gives up after kTimeoutNs.
-TP_DEV bool mbar_wait(uint64_t* b, uint32_t parity, int* err) {
-  if (mbar_try(b, parity)) return true;
-  const uint64_t t0 = gtimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try(b, parity)) return true;
-    if ((i & 255) == 0 && gtimer() - t0 > kTimeoutNs) {
-      if (err) atomicExch(err, 1);
-      return false;
-    }
-  }
-}
 
 // 3D tile load: coordinates {k within the segment, segment, row}.
 TP_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int seg, int row, uint64_t* bar) {
@@ -203,6 +167,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int per_seg = num_m * tt.num_n;
   const int ntiles = tt.ntiles;
   constexpr int NOUT = EPI == TC_EPI_SWIGLU_BF16 ? BN / 2 : BN;  // output columns per tile
+  constexpr bool SEGSUM = EPI == TC_EPI_SEGSUM_F32 || EPI == TC_EPI_SEGSUM_RELU_BF16;
+  // The CTA's i-th tile, or -1 past its last: tiles blockIdx.x, + gridDim.x, ...; with
+  // the segment sum, all segments of one output tile in order, then the next output tile.
+  auto tile_of = [&](int i) -> int {
+    if (!SEGSUM) {
+      const int64_t t = blockIdx.x + (int64_t)i * gridDim.x;
+      return t < ntiles ? (int)t : -1;
+    }
+    const int64_t u = blockIdx.x + (int64_t)(i / g.nseg) * gridDim.x;
+    return u < per_seg ? (i % g.nseg) * per_seg + (int)u : -1;
+  };
   // tile -> (segment, n block, matrix, first row in the matrix, first output row)
   auto decode = [&](int tile, int& seg, int& nb, int& mat, int& m0, int& orow0) {
     seg = tile / per_seg;
@@ -247,7 +222,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         npend = 0;
       };
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int i = 0; ok; ++i) {
+        const int tile = tile_of(i);
+        if (tile < 0) break;
         int seg, nb, mat, m0, orow0;
         decode(tile, seg, nb, mat, m0, orow0);
         const int n0 = nb * NOUT;
@@ -285,9 +262,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t IDESC = idesc_bf16(BM, BN);
       int stage = 0;
       uint32_t ph = 0;
-      int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      for (int it = 0; ok && tile_of(it) >= 0; ++it) {
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], aph ^ 1, g.err)) break;
@@ -316,8 +292,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // epilogue warps 2..5: TMEM lanes 32*(warp%4) .. +31
     const int q = warp & 3;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    // TC_EPI_SEGSUM_*: the thread's row of the output tile, summed over the segments so far
+    float run[SEGSUM ? BN : 1];
+    for (int it = 0;; ++it) {
+      const int tile = tile_of(it);
+      if (tile < 0) break;
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       if (!mbar_wait(&tfull[acc], aph, g.err)) break;
@@ -328,7 +307,55 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int n0 = nb * NOUT;
       const bool row_ok = row < g.Am[mat];
       const uint32_t taddr = tmem + (uint32_t)(acc * BN) + ((uint32_t)(32 * q) << 16);
-      if (EPI == TC_EPI_STORE_T_PAIRS_F32) {
+      if constexpr (SEGSUM) {
+        // run[j] += sync(partial of this segment), in segment order from 0.f: the same
+        // float32 additions as summing materialised partials one slice after another
+        if (seg == 0) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) run[j] = 0.f;
+        }
+        const bool last = seg == g.nseg - 1;
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          float p[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p[j] = __uint_as_float(v[j]);
+          if (g.quant) {  // the 32 columns are one Q8 block of the row (n0 + c is a multiple of 32)
+            float am = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(p[j]));
+            const float d = q8_scale(am);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) p[j] = q8_value(q8_code(p[j], d), d);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) run[c + j] += p[j];
+          if (last && row_ok && n0 + c < g.N) {
+            if (EPI == TC_EPI_SEGSUM_F32) {
+              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
+                                                     (size_t)row * g.ldo + n0 + c);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                o4[j] = make_float4(run[c + 4 * j], run[c + 4 * j + 1], run[c + 4 * j + 2],
+                                    run[c + 4 * j + 3]);
+            } else {
+              uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) +
+                                                   (size_t)row * g.ldo + n0 + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = fmaxf(run[c + 8 * j + e], 0.f);
+                o4[j] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                   pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+              }
+            }
+          }
+        }
+      } else if (EPI == TC_EPI_STORE_T_PAIRS_F32) {
         // columns (2j, 2j+1) hold batch row j's hi and lo terms: fold them
         float* o = static_cast<float*>(g.out) + (size_t)seg * g.out_seg + orow0 + 32 * q + lane;
 #pragma unroll 1
@@ -495,7 +522,10 @@ int launch_cfg(const CUtensorMap* mA, const CUtensorMap& mB, const CUtensorMap& 
                const TcGemm& g, const TcTiles& tt, cudaStream_t s) {
   constexpr int smem = TcCfg<BN>::SMEM_BYTES;
   if (set_smem_once((const void*)k_tc_gemm<BN, EPI>, smem)) return TP_ECUDA;
-  int grid = tt.ntiles < num_sms() ? tt.ntiles : num_sms();
+  // with the segment sum a CTA takes every segment of an output tile
+  const int units =
+      EPI == TC_EPI_SEGSUM_F32 || EPI == TC_EPI_SEGSUM_RELU_BF16 ? tt.ntiles / g.nseg : tt.ntiles;
+  const int grid = units < num_sms() ? units : num_sms();
   return launch_pdl(k_tc_gemm<BN, EPI>, dim3(grid), dim3(THREADS), smem, s, mA[0], mA[1], mA[2], mB,
                     mB2, g, tt);
 }
@@ -512,7 +542,9 @@ int launch_tc_gemm(const TcGemm& g, cudaStream_t s) {
   if (!trans && (g.N % 32 != 0 || g.ldo % 8 != 0 || g.nA != 1)) return TP_EINVAL;
   if (trans && g.N > 128) return TP_EINVAL;
   if (g.epi == TC_EPI_STORE_T_PAIRS_F32 && (g.N & 1)) return TP_EINVAL;
-  const int BN = trans ? (g.N <= 32 ? 32 : (g.N <= 64 ? 64 : 128)) : 256;
+  const bool segsum = g.epi == TC_EPI_SEGSUM_F32 || g.epi == TC_EPI_SEGSUM_RELU_BF16;
+  // the segment sum keeps a row's BN running sums in registers: 128 columns per tile
+  const int BN = trans ? (g.N <= 32 ? 32 : (g.N <= 64 ? 64 : 128)) : (segsum ? 128 : 256);
   CUtensorMap mA[3], mB, mB2;
   TcTiles tt{};
   tt.mt_off[0] = 0;
@@ -545,6 +577,9 @@ int launch_tc_gemm(const TcGemm& g, cudaStream_t s) {
     case TC_EPI_STORE_F32: return launch_cfg<256, TC_EPI_STORE_F32>(mA, mB, mB2, g, tt, s);
     case TC_EPI_RELU_BF16: return launch_cfg<256, TC_EPI_RELU_BF16>(mA, mB, mB2, g, tt, s);
     case TC_EPI_SWIGLU_BF16: return launch_cfg<256, TC_EPI_SWIGLU_BF16>(mA, mB, mB2, g, tt, s);
+    case TC_EPI_SEGSUM_F32: return launch_cfg<128, TC_EPI_SEGSUM_F32>(mA, mB, mB2, g, tt, s);
+    case TC_EPI_SEGSUM_RELU_BF16:
+      return launch_cfg<128, TC_EPI_SEGSUM_RELU_BF16>(mA, mB, mB2, g, tt, s);
     default: return TP_EINVAL;
   }
 }

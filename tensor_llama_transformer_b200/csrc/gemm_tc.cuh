@@ -14,6 +14,11 @@ enum TcEpi {
   TC_EPI_SWIGLU_BF16 = 2,  // out[m][n] = bf16(silu(acc_W1) * acc_W3)    (B = W1, B2 = W3)
   TC_EPI_STORE_T_F32 = 3,  // out[seg][n][row_off(matrix) + m] = acc     (transposed float32)
   TC_EPI_STORE_T_PAIRS_F32 = 4,  // as 3 with B rows in hi/lo pairs: out[seg][n/2][..] = acc_2j + acc_2j+1
+  // out[m][n] = sum over seg = 0, 1, ... of sync(acc_seg[m][n]), in segment order, float32:
+  // each segment's partial is formed on its own (a fresh accumulator) and, with g.quant,
+  // passes the Q8 round trip (blocks of 32 columns) before it is added
+  TC_EPI_SEGSUM_F32 = 5,
+  TC_EPI_SEGSUM_RELU_BF16 = 6,  // as 5, then out[m][n] = bf16(max(sum, 0))
 };
 
 // D[seg, m, n] = sum_{k < K} A[m, seg*K + k] * B[n, seg*K + k]
@@ -39,6 +44,7 @@ struct TcGemm {
   void* out;
   int64_t ldo;
   int64_t out_seg;  // elements between segment planes (float32 stores)
+  int quant;        // TC_EPI_SEGSUM_*: Q8 round trip of every segment's partial
   int* err;         // device flag set to 1 when a pipeline wait gives up (nullable: not reported)
   // Operands that no kernel before this one writes (TC_INDEP_A / TC_INDEP_B, e.g. the
   // weights): under programmatic dependent launch the producer loads their tiles for

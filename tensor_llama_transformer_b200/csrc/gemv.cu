@@ -116,7 +116,6 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   float* res = reinterpret_cast<float*>(smem + pl.res_off);  // [rows of this CTA][NB]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + pl.bar_off);
   uint64_t* empty = full + kMaxStages;
-  uint64_t* staged = empty + kMaxStages;  // the consumers have staged their activations
 
   const int rps = rows_per_seg<EPI>(a);
   const int npairs = a.nseg * (rps >> 1);
@@ -129,7 +128,6 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], nc);
     }
-    mbar_init(staged, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -141,6 +139,9 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
     // ---------------------------------------------------------------- producer
     // (bf16 weights: lane 0 issues the copies; int8 weights, whose rows take two
     // small copies each, spread them over the warp's lanes)
+    // the RMSNorm gain (a constant input: no wait) into L2 before the weights, for the
+    // consumers' prologue
+    if (a.gain && lane == 0) bulk_prefetch_l2(a.gain, (uint32_t)a.ldx * 4);
     if (WQ8 || lane == 0) {
       const uint64_t pol = l2_evict_first();  // weights are read once per step
       int t = 0;
@@ -148,13 +149,6 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
         const int end = stage_end(cur, nrows, R0, rps, P);
         const int s = t % nstage;
         const uint32_t ph = (uint32_t)(t / nstage) & 1u;
-        // beyond the first pl.prefill stages, wait for the consumers' staging: their loads
-        // (the previous kernel's output) then do not queue behind the whole ring's copies
-        if (t == pl.prefill && pl.prefill > 0) {
-          bool st = mbar_wait(staged, 0, a.err);
-          if (WQ8) st = __all_sync(0xffffffffu, st);
-          if (!st) break;
-        }
         bool waited = mbar_wait(&empty[s], ph ^ 1u, a.err);
         if (WQ8) waited = __all_sync(0xffffffffu, waited);
         if (!waited) break;
@@ -225,74 +219,270 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
     pdl_wait();  // the epilogue below writes buffers earlier kernels may read
   } else {
     // ---------------------------------------------------------------- consumers
-    pdl_wait();  // activations / residual come from the previous kernel
-    if (tr && threadIdx.x == 0) tr[1] = gtimer();
     const int ncons = nc * 32;
     // RMSNorm input with one segment (q/k/v, W1/W3 in 1D): each consumer thread loads
     // the x and gain values of its vectors (8 values, v = thread + 256 k) once, up
     // front, for the scale and the staging both: one round of loads, not two
     constexpr int kPreV = 2;
-    const bool pre = a.gain && a.nseg == 1 && nc == 8 && nv <= kPreV * 256;
+    const bool pre = pl.pre && a.gain && a.nseg == 1 && nc == 8 && nv <= kPreV * 256;
     float4 px[NB][kPreV][2], pg[kPreV][2];
-    if (pre) {
-#pragma unroll
-      for (int k = 0; k < kPreV; ++k) {
-        const int v = threadIdx.x + 256 * k;
-        const bool vin = v < nv;
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        pg[k][0] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v) : z;
-        pg[k][1] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v + 4) : z;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const bool in = vin && b < a.nb;
-          const float* xr = a.x + (size_t)(a.b0 + b) * a.ldx + 8 * (size_t)v;
-          px[b][k][0] = in ? *reinterpret_cast<const float4*>(xr) : z;
-          px[b][k][1] = in ? *reinterpret_cast<const float4*>(xr + 4) : z;
-        }
-      }
-    }
-    if (a.gain && a.ssq) {  // sums of squares left by the merge that produced x
-      if (warp < NB) {  // warp b: row b's parts, lanes in stride, then the butterfly
-        float t = 0.f;
-        if (warp < a.nb)
-          for (int c = lane; c < a.ssq_parts; c += 32) t += a.ssq[(size_t)(a.b0 + warp) * a.ssq_parts + c];
-        t = warp_sum(t);
-        if (lane == 0) s_rstd[warp] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
-      }
+    // (re)stage the activations of segment `seg`; whole warps per iteration so that 4
+    // consecutive lanes always hold one 32-value Q8 block. publish: this CTA owns the
+    // segment's first row and writes the shared buffers.
+    auto stage_segment = [&](int seg, bool publish) {
+      const size_t col0 = (size_t)seg * a.Ks;
+      const int nvr = (nv + 31) & ~31;
       consumers_sync(ncons);
-    } else if (a.gain) {  // RMSNorm scale of each batch row, over the whole row
-      const int D = a.ldx;
+      // one 8-value vector v of batch row b (x, g: the preloaded values when have_pre)
+      auto stage = [&](int b, int v, bool have_pre, float4 px0, float4 px1, float4 pg0,
+                       float4 pg1) {
+          const bool in = b < a.nb && v < nv;
+          const size_t e0 = (size_t)(a.b0 + b) * a.ldx + col0 + 8 * (size_t)v;
+          float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          uint2 qin = make_uint2(0u, 0u);  // codes as read (Q8 input)
+          float din = 0.f;
+          if (in) {
+            if (a.gain) {
+              const float rstd = s_rstd[b];
+              const float4 x0 = have_pre ? px0 : *reinterpret_cast<const float4*>(a.x + e0);
+              const float4 x1 = have_pre ? px1 : *reinterpret_cast<const float4*>(a.x + e0 + 4);
+              const float4 g0 =
+                  have_pre ? pg0 : *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v);
+              const float4 g1 = have_pre ? pg1
+                                         : *reinterpret_cast<const float4*>(a.gain + col0 +
+                                                                            8 * (size_t)v + 4);
+              xv[0] = __fmul_rn(__fmul_rn(x0.x, rstd), g0.x);
+              xv[1] = __fmul_rn(__fmul_rn(x0.y, rstd), g0.y);
+              xv[2] = __fmul_rn(__fmul_rn(x0.z, rstd), g0.z);
+              xv[3] = __fmul_rn(__fmul_rn(x0.w, rstd), g0.w);
+              xv[4] = __fmul_rn(__fmul_rn(x1.x, rstd), g1.x);
+              xv[5] = __fmul_rn(__fmul_rn(x1.y, rstd), g1.y);
+              xv[6] = __fmul_rn(__fmul_rn(x1.z, rstd), g1.z);
+              xv[7] = __fmul_rn(__fmul_rn(x1.w, rstd), g1.w);
+            } else if (a.att_po) {
+              // the attention output of these 8 dims, combined from the context splits:
+              // M = max_c m_c, o = sum_c e^{m_c - M} o_c / sum_c e^{m_c - M} l_c
+              const int gb = a.b0 + b;
+              const int P = a.pos[gb] + 1, ntiles = (P + 63) / 64;
+              const int tpc = (ntiles + a.att_nsplit - 1) / a.att_nsplit;
+              const int ncs = (ntiles + tpc - 1) / tpc;
+              const int col = (int)col0 + 8 * v, h = col / kHeadDim, d0 = col - h * kHeadDim;
+              const size_t base = ((size_t)gb * a.n_heads + h) * a.att_nsplit;
+              // the splits' (m, l) in one round of loads, then their outputs 4 splits
+              // at a time (the same sums, in split order)
+              constexpr int kCm = 8;
+              float mcs[kCm], lcs[kCm];
+#pragma unroll
+              for (int c = 0; c < kCm; ++c) {
+                mcs[c] = c < ncs ? a.att_pml[(base + c) * 2] : -INFINITY;
+                lcs[c] = c < ncs ? a.att_pml[(base + c) * 2 + 1] : 0.f;
+              }
+              float M = -INFINITY;
+              for (int c = kCm; c < ncs; ++c) M = fmaxf(M, a.att_pml[(base + c) * 2]);
+#pragma unroll
+              for (int c = 0; c < kCm; ++c) M = fmaxf(M, mcs[c]);
+              float L = 0.f;
+              auto add_split = [&](float mc, float lc, float4 o0, float4 o1) {
+                const float w = mc == -INFINITY ? 0.f : expf(mc - M);
+                L = fmaf(w, lc, L);
+                xv[0] = fmaf(w, o0.x, xv[0]); xv[1] = fmaf(w, o0.y, xv[1]);
+                xv[2] = fmaf(w, o0.z, xv[2]); xv[3] = fmaf(w, o0.w, xv[3]);
+                xv[4] = fmaf(w, o1.x, xv[4]); xv[5] = fmaf(w, o1.y, xv[5]);
+                xv[6] = fmaf(w, o1.z, xv[6]); xv[7] = fmaf(w, o1.w, xv[7]);
+              };
+#pragma unroll
+              for (int c0 = 0; c0 < kCm; c0 += 4) {
+                if (c0 >= ncs) break;
+                float4 o[4][2];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float* op = a.att_po + (base + c0 + j) * kHeadDim + d0;
+                  const bool cin = c0 + j < ncs;
+                  o[j][0] = cin ? *reinterpret_cast<const float4*>(op) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  o[j][1] = cin ? *reinterpret_cast<const float4*>(op + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  if (c0 + j < ncs) add_split(mcs[c0 + j], lcs[c0 + j], o[j][0], o[j][1]);
+              }
+              for (int c = kCm; c < ncs; ++c) {  // beyond 8 splits: one at a time
+                const float* op = a.att_po + (base + c) * kHeadDim + d0;
+                add_split(a.att_pml[(base + c) * 2], a.att_pml[(base + c) * 2 + 1],
+                          *reinterpret_cast<const float4*>(op), *reinterpret_cast<const float4*>(op + 4));
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) xv[e] = xv[e] / L;
+              if (publish && a.att_out) {
+                float* dst = a.att_out + (size_t)gb * a.ldx + col;
+                *reinterpret_cast<float4*>(dst) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
+              }
+            } else if (a.xq) {
+              const uint2 c = *reinterpret_cast<const uint2*>(a.xq + e0);
+              const float d = a.xd[e0 / kQ8Block];
+              qin = c;
+              din = d;
+              const float4 l = q8_unpack4(c.x, d), h = q8_unpack4(c.y, d);
+              xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
+              xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
+            } else {
+              const float4 l = *reinterpret_cast<const float4*>(a.x + e0);
+              const float4 h = *reinterpret_cast<const float4*>(a.x + e0 + 4);
+              xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
+              xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
+            }
+          }
+          // the normalised value before any Q8 round trip (float32 RMSNorm output)
+          if (a.gain && publish && in && a.xn_out) {
+            *reinterpret_cast<float4*>(a.xn_out + e0) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+            *reinterpret_cast<float4*>(a.xn_out + e0 + 4) =
+                make_float4(xv[4], xv[5], xv[6], xv[7]);
+          }
+          if (WQ8) {
+            // the integer products need Q8 activations: the codes read, or those of xv
+            uint2 qc = qin;
+            float qd = din;
+            if (!a.xq || a.gain) {
+              float am = 0.f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
+              am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+              am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+              qd = q8_scale(am);
+              qc = make_uint2(0u, 0u);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int c = q8_code(xv[e], qd);
+                xv[e] = q8_value(c, qd);
+                if (e < 4) qc.x |= (uint32_t)(c & 0xFF) << (8 * e);
+                else qc.y |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
+              }
+              if (a.gain && publish && in && a.xq_out) {
+                *reinterpret_cast<uint2*>(a.xq_out + e0) = qc;
+                if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = qd;
+              }
+            }
+            if (v < nv) {
+              *reinterpret_cast<uint2*>(xsq + (size_t)b * a.Ks + 8 * (size_t)v) = qc;
+              if ((v & 3) == 0) xsd[(size_t)b * (a.Ks / 32) + (v >> 2)] = qd;
+            }
+          } else if (a.gain && a.quant) {
+            float am = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+            const float d = q8_scale(am);
+            uint32_t lo = 0, hi = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c = q8_code(xv[e], d);
+              xv[e] = q8_value(c, d);
+              if (e < 4) lo |= (uint32_t)(c & 0xFF) << (8 * e);
+              else hi |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
+            }
+            if (publish && in && a.xq_out) {
+              *reinterpret_cast<uint2*>(a.xq_out + e0) = make_uint2(lo, hi);
+              if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = d;
+            }
+          }
+          if (!WQ8 && v < nv) {
+            xs[b * nv + v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+            xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+          }
+      };
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        float ss = 0.f;
         if (pre) {
 #pragma unroll
-          for (int k = 0; k < kPreV; ++k)
+          for (int k = 0; k < kPreV; ++k) {
+            const int v = threadIdx.x + 256 * k;
+            if (v < nvr) stage(b, v, true, px[b][k][0], px[b][k][1], pg[k][0], pg[k][1]);
+          }
+        } else {
+          for (int v = threadIdx.x; v < nvr; v += ncons) stage(b, v, false, z4, z4, z4, z4);
+        }
+      }
+      consumers_sync(ncons);
+    };
+
+    // The q/k/v and W1/W3 products (RMSNorm input staged from registers) wait for a
+    // merge before their input exists. Their prologue runs first on dummy values,
+    // before that wait, with nothing written outside shared memory: its code is then
+    // in the SM's instruction cache when the input arrives (the first run of this
+    // code was measured about 2 us slower than a second one).
+    const int seg0 = R0 / rps;
+    for (int pass = pre ? 0 : 1; pass < 2; ++pass) {
+      const bool warm = pass == 0;
+      if (!warm) {
+        pdl_wait();  // activations / residual come from the previous kernel
+        if (tr && threadIdx.x == 0) tr[1] = gtimer();
+      }
+      if (pre) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float4 v = px[b][k][h];
-              ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-            }
-        } else if (b < a.nb) {
-          const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
-          for (int i = threadIdx.x; i < (D >> 2); i += ncons) {
-            const float4 v = xrow[i];
-            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        for (int k = 0; k < kPreV; ++k) {
+          const int v = threadIdx.x + 256 * k;
+          const bool vin = v < nv && !warm;
+          const float zf = warm ? 1.f : 0.f;  // dummy values; past the row: zero
+          const float4 z = make_float4(zf, zf, zf, zf);
+          pg[k][0] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v) : z;
+          pg[k][1] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v + 4) : z;
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const bool in = vin && b < a.nb;
+            const float* xr = a.x + (size_t)(a.b0 + b) * a.ldx + 8 * (size_t)v;
+            px[b][k][0] = in ? *reinterpret_cast<const float4*>(xr) : z;
+            px[b][k][1] = in ? *reinterpret_cast<const float4*>(xr + 4) : z;
           }
         }
-        ss = warp_sum(ss);
-        if (lane == 0) s_red[warp][b] = ss;
       }
-      consumers_sync(ncons);
-      if (threadIdx.x < NB) {
-        float t = 0.f;
-        for (int w = 0; w < nc; ++w) t += s_red[w][threadIdx.x];
-        s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)D + a.eps);
+      if (a.gain && a.ssq) {  // sums of squares left by the merge that produced x
+        if (warp < NB) {  // warp b: row b's parts, lanes in stride, then the butterfly
+          float t = warm ? 1.f : 0.f;
+          if (warp < a.nb && !warm)
+            for (int c = lane; c < a.ssq_parts; c += 32) t += a.ssq[(size_t)(a.b0 + warp) * a.ssq_parts + c];
+          t = warp_sum(t);
+          if (lane == 0) s_rstd[warp] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
+        }
+        consumers_sync(ncons);
+      } else if (a.gain) {  // RMSNorm scale of each batch row, over the whole row
+        const int D = a.ldx;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          float ss = 0.f;
+          if (pre) {
+#pragma unroll
+            for (int k = 0; k < kPreV; ++k)
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float4 v = px[b][k][h];
+                ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+              }
+          } else if (b < a.nb) {
+            const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
+            for (int i = threadIdx.x; i < (D >> 2); i += ncons) {
+              const float4 v = xrow[i];
+              ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+            }
+          }
+          ss = warp_sum(ss);
+          if (lane == 0) s_red[warp][b] = ss;
+        }
+        consumers_sync(ncons);
+        if (threadIdx.x < NB) {
+          float t = 0.f;
+          for (int w = 0; w < nc; ++w) t += s_red[w][threadIdx.x];
+          s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)D + a.eps);
+        }
+        consumers_sync(ncons);
       }
-      consumers_sync(ncons);
+      if (!warm && tr && threadIdx.x == 0) tr[2] = gtimer();  // the RMSNorm scale known
+      stage_segment(seg0, !warm && R0 == seg0 * rps);
     }
+    if (tr && threadIdx.x == 0) tr[3] = gtimer();
 
-    int cur_seg = -1;
+    int cur_seg = seg0;
     bool ok = true;
     int t = 0;
     // this warp's share of a stage: row pair `pw` of the stage, vectors [vb, ve)
@@ -304,194 +494,13 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       const uint32_t ph = (uint32_t)(t / nstage) & 1u;
       const int seg = (R0 + cur) / rps;
       if (seg != cur_seg) {
-        // (re)stage the activations of this segment; whole warps per iteration so
-        // that 4 consecutive lanes always hold one 32-value Q8 block
-        const bool publish = (R0 + cur) == seg * rps;  // this CTA owns the segment's first row
-        const size_t col0 = (size_t)seg * a.Ks;
-        const int nvr = (nv + 31) & ~31;
-        consumers_sync(ncons);
-        // one 8-value vector v of batch row b (x, g: the preloaded values when have_pre)
-        auto stage = [&](int b, int v, bool have_pre, float4 px0, float4 px1, float4 pg0,
-                         float4 pg1) {
-            const bool in = b < a.nb && v < nv;
-            const size_t e0 = (size_t)(a.b0 + b) * a.ldx + col0 + 8 * (size_t)v;
-            float xv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint2 qin = make_uint2(0u, 0u);  // codes as read (Q8 input)
-            float din = 0.f;
-            if (in) {
-              if (a.gain) {
-                const float rstd = s_rstd[b];
-                const float4 x0 = have_pre ? px0 : *reinterpret_cast<const float4*>(a.x + e0);
-                const float4 x1 = have_pre ? px1 : *reinterpret_cast<const float4*>(a.x + e0 + 4);
-                const float4 g0 =
-                    have_pre ? pg0 : *reinterpret_cast<const float4*>(a.gain + col0 + 8 * (size_t)v);
-                const float4 g1 = have_pre ? pg1
-                                           : *reinterpret_cast<const float4*>(a.gain + col0 +
-                                                                              8 * (size_t)v + 4);
-                xv[0] = __fmul_rn(__fmul_rn(x0.x, rstd), g0.x);
-                xv[1] = __fmul_rn(__fmul_rn(x0.y, rstd), g0.y);
-                xv[2] = __fmul_rn(__fmul_rn(x0.z, rstd), g0.z);
-                xv[3] = __fmul_rn(__fmul_rn(x0.w, rstd), g0.w);
-                xv[4] = __fmul_rn(__fmul_rn(x1.x, rstd), g1.x);
-                xv[5] = __fmul_rn(__fmul_rn(x1.y, rstd), g1.y);
-                xv[6] = __fmul_rn(__fmul_rn(x1.z, rstd), g1.z);
-                xv[7] = __fmul_rn(__fmul_rn(x1.w, rstd), g1.w);
-              } else if (a.att_po) {
-                // the attention output of these 8 dims, combined from the context splits:
-                // M = max_c m_c, o = sum_c e^{m_c - M} o_c / sum_c e^{m_c - M} l_c
-                const int gb = a.b0 + b;
-                const int P = a.pos[gb] + 1, ntiles = (P + 63) / 64;
-                const int tpc = (ntiles + a.att_nsplit - 1) / a.att_nsplit;
-                const int ncs = (ntiles + tpc - 1) / tpc;
-                const int col = (int)col0 + 8 * v, h = col / kHeadDim, d0 = col - h * kHeadDim;
-                const size_t base = ((size_t)gb * a.n_heads + h) * a.att_nsplit;
-                // the splits' (m, l) in one round of loads, then their outputs 4 splits
-                // at a time (the same sums, in split order)
-                constexpr int kCm = 8;
-                float mcs[kCm], lcs[kCm];
-#pragma unroll
-                for (int c = 0; c < kCm; ++c) {
-                  mcs[c] = c < ncs ? a.att_pml[(base + c) * 2] : -INFINITY;
-                  lcs[c] = c < ncs ? a.att_pml[(base + c) * 2 + 1] : 0.f;
-                }
-                float M = -INFINITY;
-                for (int c = kCm; c < ncs; ++c) M = fmaxf(M, a.att_pml[(base + c) * 2]);
-#pragma unroll
-                for (int c = 0; c < kCm; ++c) M = fmaxf(M, mcs[c]);
-                float L = 0.f;
-                auto add_split = [&](float mc, float lc, float4 o0, float4 o1) {
-                  const float w = mc == -INFINITY ? 0.f : expf(mc - M);
-                  L = fmaf(w, lc, L);
-                  xv[0] = fmaf(w, o0.x, xv[0]); xv[1] = fmaf(w, o0.y, xv[1]);
-                  xv[2] = fmaf(w, o0.z, xv[2]); xv[3] = fmaf(w, o0.w, xv[3]);
-                  xv[4] = fmaf(w, o1.x, xv[4]); xv[5] = fmaf(w, o1.y, xv[5]);
-                  xv[6] = fmaf(w, o1.z, xv[6]); xv[7] = fmaf(w, o1.w, xv[7]);
-                };
-#pragma unroll
-                for (int c0 = 0; c0 < kCm; c0 += 4) {
-                  if (c0 >= ncs) break;
-                  float4 o[4][2];
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const float* op = a.att_po + (base + c0 + j) * kHeadDim + d0;
-                    const bool cin = c0 + j < ncs;
-                    o[j][0] = cin ? *reinterpret_cast<const float4*>(op) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    o[j][1] = cin ? *reinterpret_cast<const float4*>(op + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-                  }
-#pragma unroll
-                  for (int j = 0; j < 4; ++j)
-                    if (c0 + j < ncs) add_split(mcs[c0 + j], lcs[c0 + j], o[j][0], o[j][1]);
-                }
-                for (int c = kCm; c < ncs; ++c) {  // beyond 8 splits: one at a time
-                  const float* op = a.att_po + (base + c) * kHeadDim + d0;
-                  add_split(a.att_pml[(base + c) * 2], a.att_pml[(base + c) * 2 + 1],
-                            *reinterpret_cast<const float4*>(op), *reinterpret_cast<const float4*>(op + 4));
-                }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xv[e] = xv[e] / L;
-                if (publish && a.att_out) {
-                  float* dst = a.att_out + (size_t)gb * a.ldx + col;
-                  *reinterpret_cast<float4*>(dst) = make_float4(xv[0], xv[1], xv[2], xv[3]);
-                  *reinterpret_cast<float4*>(dst + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
-                }
-              } else if (a.xq) {
-                const uint2 c = *reinterpret_cast<const uint2*>(a.xq + e0);
-                const float d = a.xd[e0 / kQ8Block];
-                qin = c;
-                din = d;
-                const float4 l = q8_unpack4(c.x, d), h = q8_unpack4(c.y, d);
-                xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
-                xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
-              } else {
-                const float4 l = *reinterpret_cast<const float4*>(a.x + e0);
-                const float4 h = *reinterpret_cast<const float4*>(a.x + e0 + 4);
-                xv[0] = l.x; xv[1] = l.y; xv[2] = l.z; xv[3] = l.w;
-                xv[4] = h.x; xv[5] = h.y; xv[6] = h.z; xv[7] = h.w;
-              }
-            }
-            // the normalised value before any Q8 round trip (float32 RMSNorm output)
-            if (a.gain && publish && in && a.xn_out) {
-              *reinterpret_cast<float4*>(a.xn_out + e0) = make_float4(xv[0], xv[1], xv[2], xv[3]);
-              *reinterpret_cast<float4*>(a.xn_out + e0 + 4) =
-                  make_float4(xv[4], xv[5], xv[6], xv[7]);
-            }
-            if (WQ8) {
-              // the integer products need Q8 activations: the codes read, or those of xv
-              uint2 qc = qin;
-              float qd = din;
-              if (!a.xq || a.gain) {
-                float am = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
-                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-                qd = q8_scale(am);
-                qc = make_uint2(0u, 0u);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const int c = q8_code(xv[e], qd);
-                  xv[e] = q8_value(c, qd);
-                  if (e < 4) qc.x |= (uint32_t)(c & 0xFF) << (8 * e);
-                  else qc.y |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
-                }
-                if (a.gain && publish && in && a.xq_out) {
-                  *reinterpret_cast<uint2*>(a.xq_out + e0) = qc;
-                  if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = qd;
-                }
-              }
-              if (v < nv) {
-                *reinterpret_cast<uint2*>(xsq + (size_t)b * a.Ks + 8 * (size_t)v) = qc;
-                if ((v & 3) == 0) xsd[(size_t)b * (a.Ks / 32) + (v >> 2)] = qd;
-              }
-            } else if (a.gain && a.quant) {
-              float am = 0.f;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(xv[e]));
-              am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-              am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-              const float d = q8_scale(am);
-              uint32_t lo = 0, hi = 0;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int c = q8_code(xv[e], d);
-                xv[e] = q8_value(c, d);
-                if (e < 4) lo |= (uint32_t)(c & 0xFF) << (8 * e);
-                else hi |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
-              }
-              if (publish && in && a.xq_out) {
-                *reinterpret_cast<uint2*>(a.xq_out + e0) = make_uint2(lo, hi);
-                if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = d;
-              }
-            }
-            if (!WQ8 && v < nv) {
-              xs[b * nv + v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
-              xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
-            }
-        };
-        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          if (pre) {
-#pragma unroll
-            for (int k = 0; k < kPreV; ++k) {
-              const int v = threadIdx.x + 256 * k;
-              if (v < nvr) stage(b, v, true, px[b][k][0], px[b][k][1], pg[k][0], pg[k][1]);
-            }
-          } else {
-            for (int v = threadIdx.x; v < nvr; v += ncons) stage(b, v, false, z4, z4, z4, z4);
-          }
-        }
-        consumers_sync(ncons);
+        stage_segment(seg, (R0 + cur) == seg * rps);
         cur_seg = seg;
-        if (t == 0 && threadIdx.x == 0) {
-          if (tr) tr[2] = gtimer();
-          mbar_arrive(staged);
-        }
       }
       // after a wait gives up, keep walking the stages (so that every consumer warp
       // reaches the same named barriers) but skip the work
       if (ok && !mbar_wait(&full[s], ph, a.err)) ok = false;
-      if (tr && t == 0 && threadIdx.x == 0) tr[3] = gtimer();
+      if (tr && t == 0 && threadIdx.x == 0) tr[4] = gtimer();
       if (ok) {
         const uint8_t* st = ring + (size_t)s * 2 * P * slot;
         if constexpr (WQ8) {
@@ -525,7 +534,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       if (lane == 0) mbar_arrive(&empty[s]);
       cur = end;
     }
-    if (tr && threadIdx.x == 0) tr[4] = gtimer();
+    if (tr && threadIdx.x == 0) tr[5] = gtimer();
   }
   __syncthreads();
 
@@ -578,7 +587,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       }
     }
   }
-  if (tr && threadIdx.x == 0) tr[5] = gtimer();
+  if (tr && threadIdx.x == 0) tr[6] = gtimer();
 }
 
 // The int8-weight consumer step (see ring_pairs_dot): each row's codes are read
@@ -641,44 +650,30 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
 
 size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
 
-// Ring stages a GEMV fills before its consumers have staged the activations:
-// TP_GEMV_PREFILL (a tuning knob), default 0 = the whole ring.
-int gemv_prefill() {
-  static const int n = [] {
-    const char* v = getenv("TP_GEMV_PREFILL");
-    return v ? atoi(v) : 0;
+int gemv_pre() {
+  static const int on = [] {
+    const char* v = getenv("TP_GEMV_PRE");
+    return v && v[0] == '0' ? 0 : 1;
   }();
-  return n;
-}
-
-// Shared memory of a GEMV CTA: kSmemBudget (one CTA per SM, the deepest ring),
-// or TP_GEMV_SMEM_KB (a tuning knob: e.g. 110 lets two GEMV CTAs share an SM, so
-// that the next launch's ring fills while this one finishes).
-int gemv_smem_budget() {
-  static const int b = [] {
-    const char* v = getenv("TP_GEMV_SMEM_KB");
-    const int kb = v ? atoi(v) : 0;
-    return kb >= 32 && kb * 1024 <= kSmemBudget ? kb * 1024 : kSmemBudget;
-  }();
-  return b;
+  return on;
 }
 
 // Shared-memory plan: 8 consumer warps; the most row pairs per stage (16, 8, 4,
 // 2, 1) that still leave a ring of at least 3 stages (2 for the longest rows):
 // 16 pairs give each warp two pairs, fewer are each split over 8 / pairs warps.
-bool make_plan(int NB, int Ks, int cta_rows, bool wq8, int budget, GemvPlan* p) {
+bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
   const size_t row_bytes = wq8 ? (size_t)Ks + q8w_scale_slot(Ks) : (size_t)Ks * 2;
   const size_t x_bytes = wq8 ? a128((size_t)NB * Ks + (size_t)NB * (Ks / 32) * 4)
                              : a128((size_t)NB * Ks * 4);
-  const size_t bar_bytes = (2 * kMaxStages + 1) * 8;
+  const size_t bar_bytes = 2 * kMaxStages * 8;
   for (int min_stages : {3, 2}) {
     for (int P = 16; P >= 1; P >>= 1) {
       const int Q = P >= 8 ? 1 : 8 / P;
       const size_t res_bytes = a128((size_t)cta_rows * NB * Q * 4);
       const size_t fixed = x_bytes + res_bytes + bar_bytes;
-      if (fixed >= (size_t)budget) continue;
+      if (fixed >= (size_t)kSmemBudget) continue;
       const size_t stage = 2 * (size_t)P * row_bytes;
-      int ns = (int)(((size_t)budget - fixed) / stage);
+      int ns = (int)(((size_t)kSmemBudget - fixed) / stage);
       if (ns > kMaxStages) ns = kMaxStages;
       if (ns >= min_stages) {
         p->nc = 8;
@@ -686,8 +681,8 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, int budget, GemvPlan* p) 
         p->split = Q;
         p->pw = P == 16 ? 2 : 1;
         p->nstage = ns;
-        p->prefill = gemv_prefill() < ns ? gemv_prefill() : 0;
         p->cta_rows = cta_rows;
+        p->pre = gemv_pre() ? 1 : 0;
         p->ring_off = 0;
         p->x_off = a128((size_t)ns * stage);
         p->res_off = p->x_off + x_bytes;
@@ -709,27 +704,8 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   int grid = num_sms();
   if (grid > npairs) grid = npairs;
   const int cta_rows = 2 * ((npairs + grid - 1) / grid);
-  int budget = gemv_smem_budget();
-  if (a.co_smem > 0) {  // fit beside another kernel's CTA (1 KB reserved per CTA)
-    static int per_sm = 0, st = 0;
-    if (!per_sm) {
-      int dev = 0, v = 0;
-      cudaFuncAttributes fa{};
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
-          cudaFuncGetAttributes(&fa, (const void*)k_gemv<NB, EPI, WQ8>) != cudaSuccess)
-        return TP_ECUDA;
-      st = (int)fa.sharedSizeBytes;
-      per_sm = v;
-    }
-    const int room = per_sm - (a.co_smem + 1024) - (st + 1024) - 256;
-    if (room < budget) budget = room;
-  }
   GemvPlan pl;
-  // a ring too small beside the other CTA (long rows): take the whole SM instead
-  if (!make_plan(NB, a.Ks, cta_rows, WQ8, budget, &pl) &&
-      (budget == kSmemBudget || !make_plan(NB, a.Ks, cta_rows, WQ8, kSmemBudget, &pl)))
-    return TP_ENOTSUP;
+  if (!make_plan(NB, a.Ks, cta_rows, WQ8, &pl)) return TP_ENOTSUP;
   if (set_smem_once((const void*)k_gemv<NB, EPI, WQ8>, (int)pl.total)) return TP_ECUDA;
   return launch_pdl(k_gemv<NB, EPI, WQ8>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
 }

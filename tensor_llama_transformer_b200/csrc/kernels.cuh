@@ -12,8 +12,18 @@ namespace tp {
 // 128-value chunk of the new row is written too: ssq[b][chunk] (merge_ssq_parts(dim)
 // of them; one warp's float4 lanes summed by warp_sum, in both merge kernels, so
 // that both give the next RMSNorm the same bits). dim % 128 == 0, parts <= 2.
+// The first rows each CTA of the next slice GEMV streams, for a small kernel that
+// runs in the gap before it to prefetch into L2 (while it waits for its own
+// input): for pair-interleaved W1/W3 (SwiGLU), next-GEMV CTA c of `grid` starts at
+// pair P0(c) = npairs c / grid; `pairs` pairs of each are prefetched (rows of
+// row_bytes bytes, ld_bytes apart, in w[0] and w[1]). w[0] null: nothing.
+struct L2Ahead {
+  const void* w[2];
+  int64_t ld_bytes;
+  int row_bytes, npairs, grid, pairs;
+};
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts = 1);
+                 cudaStream_t s, int parts = 1, const L2Ahead* ahead = nullptr);
 inline int merge_ssq_parts(int dim) { return dim / 128; }
 // One slice's partial in the sync format for B rows: float32 [B, dim], or with Q8
 // the codes int8 [B, dim] followed by the scales float32 [B, dim/32].
@@ -86,15 +96,10 @@ struct GemvArgs {
   int n_heads, n_kv_heads, max_seq;
   float theta;
   // optional %globaltimer stamps (ns) of CTA c at trace[c * trace_stride + k]:
-  // k = 0 start, 1 previous kernel complete, 2 activations staged, 3 first ring
-  // stage arrived, 4 last ring stage consumed, 5 end
+  // k = 0 start, 1 previous kernel complete, 2 RMSNorm scale known, 3 activations
+  // staged, 4 first ring stage arrived, 5 last ring stage consumed, 6 end
   unsigned long long* trace;
   int trace_stride;
-  // shared memory of another kernel's CTA that this launch's CTAs must fit beside
-  // on one SM (0: none, the ring takes the whole SM). The W_O GEMV leaves room
-  // for one attention CTA, so that it becomes resident and streams its weights
-  // while the attention still runs (programmatic dependent launch).
-  int co_smem;
   int* err;  // device error flag, set when a bounded wait gives up (nullable)
 };
 
@@ -109,8 +114,8 @@ struct GemvPlan {
   int split;
   int pw;  // row pairs per warp and stage (2 with 16 pairs per stage)
   int nstage;
-  int prefill;  // ring stages filled before the activations are staged (0: all of them)
   int cta_rows;
+  int pre;  // RMSNorm input preloaded into registers, prologue warmed before the wait
   size_t ring_off, x_off, res_off, bar_off, total;
 };
 
@@ -137,12 +142,8 @@ struct AttnArgs {
 // combine = false leaves the splits' partials for the consumer to combine (the
 // W_O GEMV's staging on the weight-streaming path).
 int launch_attention(const AttnArgs& a, cudaStream_t s, bool combine = true);
-// Context splits per (batch row, kv head) the attention uses for these shapes,
-// with at most `per_sm` of its CTAs resident per SM (2 fit; 1 leaves room beside
-// each for the next kernel's CTA, see attention_cta_smem).
-int attention_nsplit(int B, int H, int Hkv, int max_seq, int per_sm = 2);
-// Shared memory (dynamic + static) one decode-attention CTA holds.
-int attention_cta_smem();
+// Context splits per (batch row, kv head) the attention uses for these shapes.
+int attention_nsplit(int B, int H, int Hkv, int max_seq);
 // Largest number of context splits any launch over max_seq positions uses.
 int attention_max_splits(int max_seq);
 

@@ -86,6 +86,12 @@ TP_DEV void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* 
       : "memory");
 }
 
+// Prefetch of a contiguous global range into L2 (16-byte aligned, size a
+// multiple of 16); no completion to wait for.
+TP_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // One box of a 2D tensor map at element coordinates (x, y) -> shared memory.
 TP_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(

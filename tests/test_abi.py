@@ -94,14 +94,25 @@ def test_create_rejects_missing_workspace_before_cuda(tpb):
 def test_ffn_plan_validation(tpb):
     desc = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1, 1,
                            0, tpb.TP_MERGE_FAITHFUL)
+    h_bytes = 512 * 73728 * 2  # the hidden activations H, bf16
+    # bf16 faithful: the partials are summed in the GEMM epilogue, no planes
     ws1d = tpb.tp_ffn_workspace_bytes(desc)
-    assert ws1d >= 64 * 512 * 18432 * 4  # the 64 materialised partials of the row split
+    assert h_bytes <= ws1d < h_bytes + 4096
     desc2 = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_2D, 64, 8,
                             8, 0, tpb.TP_MERGE_FAITHFUL)
-    assert tpb.tp_ffn_workspace_bytes(desc2) < ws1d
+    assert tpb.tp_ffn_workspace_bytes(desc2) == ws1d
+    # ... except the 2D SwiGLU first stage: two products per hidden value, one plane
+    # per E-slice each
+    sw2 = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_SWIGLU, tpb.TP_PART_2D, 64, 8,
+                          8, 0, tpb.TP_MERGE_FAITHFUL)
+    assert tpb.tp_ffn_workspace_bytes(sw2) >= h_bytes + 2 * 8 * 512 * 73728 * 4
+    # float32: every stage's partials materialised (64 planes of the row split)
+    f32 = tpb.tp_ffn_desc(64, 256, 4096, tpb.TP_F32, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1, 1, 0,
+                          tpb.TP_MERGE_FAITHFUL)
+    assert tpb.tp_ffn_workspace_bytes(f32) >= 64 * 64 * 256 * 4 + 64 * 4096 * 4 * 2
     fused = tpb.tp_ffn_desc(512, 18432, 73728, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1,
                             1, 0, tpb.TP_MERGE_FUSED)
-    assert tpb.tp_ffn_workspace_bytes(fused) < 512 * 73728 * 2 + 4096
+    assert tpb.tp_ffn_workspace_bytes(fused) < h_bytes + 4096
     bad = tpb.tp_ffn_desc(8, 64, 250, tpb.TP_F32, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 2, 1, 1, 0, 0)
     with pytest.raises(tpb.TpError):
         tpb.tp_ffn_workspace_bytes(bad)

@@ -1,9 +1,11 @@
 """Partitioned FFN on the GPU through the C ABI versus the float64 oracle.
 
 float32 (the ggmlR-shaped two-stage ReLU FFN, 1e-5) on CUDA cores; bf16 on the
-tcgen05 tensor-core contraction (2e-2), in 1D and 2D partitions, with the
-partials materialised (faithful merge) or accumulated in the contraction
-(fused merge), ReLU and SwiGLU, with and without Q8 sync of the partials.
+tcgen05 tensor-core contraction (2e-2), in 1D and 2D partitions, with every
+slice's partial formed on its own and summed in slice order (faithful merge:
+in the GEMM's epilogue, or through partial planes for the 2D SwiGLU first
+stage) or accumulated in the contraction (fused merge), ReLU and SwiGLU, with
+and without Q8 sync of the partials; bit-exact on integer-valued inputs.
 """
 import numpy as np
 import pytest
@@ -94,6 +96,71 @@ def test_bf16_m_tails(tpb, M):
         y = run_ffn(tpb, s, inputs, 1, merge)
         r, _ = report(f"bf16 M={M} merge{merge}", y, _ref(s, inputs, 1, False))
         assert r <= BF16_TOL
+
+
+def _int_bf16(a):
+    """bf16 bits of small integers (exact: they need at most 8 significant bits)."""
+    a = np.asarray(a, dtype=np.float32)
+    assert np.all(np.abs(a) <= 256)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("partition,quant", [(1, False), (1, True), (2, False)])
+def test_bf16_faithful_bit_exact_on_integers(tpb, partition, quant):
+    """Integer-valued X, W1, W2 make every partial an exact integer in float32, so the
+    faithful form's output is fixed bit for bit: the float32 sum, in slice order, of
+    each slice's partial after the sync (oracle.sync_buffer: the Q8 round trip when
+    quantising). The quantised 1D case checks the order and the per-partial rounding:
+    a sum in another order, or a Q8 round trip of the sum instead of each partial,
+    changes low bits. B = 130 and E = 320, F = 480 leave partial M and N tiles."""
+    rng = np.random.default_rng(2024 + partition + 10 * quant)
+    B, E, F = 130, 320, 480
+    n, (gx, gy) = 3, (2, 3)
+    X = rng.integers(-1, 2, (B, E)).astype(np.float64)
+    W1 = rng.integers(-1, 2, (F, E)).astype(np.float64)
+    W2 = rng.integers(-1, 2, (E, F)).astype(np.float64)
+    H = np.maximum(X @ W1.T, 0.0)
+    assert H.max() <= 256  # every hidden value an exact bf16
+    Y32 = np.zeros((B, E), dtype=np.float32)
+    if partition == 1:
+        for s in range(n):
+            fs = oracle.slice_range(F, n, s)
+            P = H[:, fs] @ W2[:, fs].T
+            Y32 = (Y32 + oracle.sync_buffer(P, quant).astype(np.float32)).astype(np.float32)
+    else:  # integer partials without quantisation: every sum exact
+        Y32 = (H @ W2.T).astype(np.float32)
+        assert np.all(np.abs(H @ W2.T) < 2 ** 24)
+    desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, partition, n, gx, gy, int(quant),
+                           tpb.TP_MERGE_FAITHFUL)
+    nbytes = tpb.tp_ffn_workspace_bytes(desc)
+    ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+    Y = torch.full((B, E), float("nan"), dtype=torch.float32, device="cuda")
+    tpb.tp_ffn_forward(desc, bf16_tensor(_int_bf16(X)), bf16_tensor(_int_bf16(W1)), None,
+                       bf16_tensor(_int_bf16(W2)), Y, ws, nbytes)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    got = Y.cpu().numpy()
+    bad = np.argwhere(got.view(np.uint32) != Y32.view(np.uint32))
+    assert bad.size == 0, f"{len(bad)} values differ, first at {bad[0]}: {got[tuple(bad[0])]!r} " \
+                          f"vs {Y32[tuple(bad[0])]!r}"
+    if quant:  # the quantised sum must differ from the exact one somewhere (the test has teeth)
+        assert np.any(Y32 != (H @ W2.T).astype(np.float32))
+    print(f"[parity] faithful FFN part{partition} q{int(quant)} on integers: bit-exact")
+
+
+@pytest.mark.parametrize("partition", [1, 2])
+def test_bf16_faithful_n_tails(tpb, partition):
+    """Feature and model dims that leave partial 128-column tiles (E 320, F 480) in
+    both stages, with Q8, SwiGLU and ReLU, against the oracle."""
+    for act in ("relu", "swiglu"):
+        s = synth.FfnShape(batch=130, E=320, F=480, dtype="bf16", act=act, n_slices=3, grid_x=2,
+                           grid_y=3, x_std=1.0, w_std=0.06)
+        inputs = synth.ffn_inputs(7272 + partition, s)
+        for quant in (False, True):
+            y = run_ffn(tpb, s, inputs, partition, tpb.TP_MERGE_FAITHFUL, quant)
+            r, p = report(f"bf16 {act} part{partition} q{int(quant)} E320 F480", y,
+                          _ref(s, inputs, partition, quant))
+            assert r <= BF16_TOL and p > 0.9999
 
 
 @pytest.fixture(scope="module")
