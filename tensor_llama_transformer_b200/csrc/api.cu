@@ -58,40 +58,6 @@ int set_smem_once(const void* kernel, int bytes) {
   return TP_OK;
 }
 
-// Tuning switches read once from the environment (for comparison runs):
-bool env_flag(const char* name, bool dflt) {
-  const char* v = getenv(name);
-  if (!v || !v[0]) return dflt;
-  return v[0] != '0';
-}
-//   TP_L2_AHEAD=0     the merge kernels do not prefetch the next GEMV's first rows.
-bool l2_ahead_enabled() {
-  static const bool on = env_flag("TP_L2_AHEAD", true);
-  return on;
-}
-// Bytes per next-GEMV CTA the merge prefetches (a W1/W3 pair is 2 rows).
-constexpr int64_t kAheadBytes = 192 * 1024;
-
-int prefer_max_shared(const void* kernel) {
-  struct Entry {
-    const void* fn;
-    int dev;
-  };
-  static Entry tab[256];
-  static int used = 0;
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return TP_ECUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < used; ++i)
-    if (tab[i].fn == kernel && tab[i].dev == dev) return TP_OK;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-    return TP_ECUDA;
-  if (used < 256) tab[used++] = Entry{kernel, dev};
-  return TP_OK;
-}
-
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = getenv("TP_PDL");
@@ -321,10 +287,10 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
 // slice order through the sync format. Rank block: the same over the gathered
 // sync buffer, which holds every rank's slices in slice order.
 int merge_step(tp_block* blk, float* x, const float* part, int nseg, int parts, int batch,
-               cudaStream_t s, const L2Ahead* ahead = nullptr) {
+               cudaStream_t s) {
   const Cfg& c = blk->c;
   float* ssq = at<float>(blk, BUF_SSQ);
-  if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts, ahead);
+  if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts);
   return launch_merge_sync(x, at<uint8_t>(blk, BUF_RECV), c.n * c.world, batch, c.d.dim, c.quant,
                            ssq, s);
 }
@@ -705,20 +671,9 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   }
   if (phase <= 1) {
     // a6: sync + dequantise + merge into the residual (a rank block: of the
-    // gathered buffer); while it waits, the merge prefetches into L2 the first
-    // W1/W3 rows each CTA of the next GEMV streams
+    // gathered buffer)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    L2Ahead ahead{};
-    if (c.partition == TP_PART_1D && !blk->wq8 && l2_ahead_enabled()) {
-      ahead.w[0] = blk->w.w1;
-      ahead.w[1] = blk->w.w3;
-      ahead.ld_bytes = (int64_t)D * 2;
-      ahead.row_bytes = D * 2;
-      ahead.npairs = F;
-      ahead.grid = num_sms() < F ? num_sms() : F;
-      ahead.pairs = (int)(kAheadBytes / (2 * ahead.row_bytes));
-    }
-    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s, &ahead))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
     // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if (c.partition == TP_PART_1D) {

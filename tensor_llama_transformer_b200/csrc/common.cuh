@@ -107,6 +107,31 @@ TP_DEV int q8_code(float x, float d) {
 
 TP_DEV float q8_value(int q, float d) { return __fmul_rn((float)q, d); }
 
+// For many values of one block: the block's reciprocal r = 1/d, correctly rounded
+// (__frcp_rn), or 0 when d is outside [2^-120, 2^120] (every value of the block then
+// takes the division).
+TP_DEV float q8_recip(float d) { return d > 0x1p-120f && d < 0x1p120f ? __frcp_rn(d) : 0.f; }
+
+// q8_code(x, d) as an integral float (+0 for a zero code), from q = x * r with
+// r = q8_recip(d): two correctly rounded steps put q within 2^-23 relative of the exact
+// x / d, and |x / d| <= 127.0001, so q is within 1.6e-5 of x / d and within 2e-5 of
+// fl(x / d) (half an ulp below 128 is 3.8e-6). Rounding q and fl(x / d) to an integer
+// can then differ only when one of them lies within 2e-5 of a tie k + 1/2, and there
+// the correctly rounded division is taken instead (window 4e-5, as in q8_code).
+TP_DEV float q8_code_rf(float x, float d, float r) {
+  if (d == 0.0f) return 0.f;
+  float q;
+  if (r != 0.f) {
+    q = __fmul_rn(x, r);
+    const float a = fabsf(q);
+    if (fabsf(a - truncf(a) - 0.5f) < 4e-5f) q = __fdiv_rn(x, d);
+  } else {
+    q = __fdiv_rn(x, d);
+  }
+  // roundf: halfway cases away from zero; + 0 turns a -0 code into +0
+  return fminf(fmaxf(roundf(q), -127.0f), 127.0f) + 0.0f;
+}
+
 // Quantise-dequantise of 4 consecutive values held by each of 8 consecutive
 // lanes (one 32-value block per 8-lane group). All 32 lanes must call it.
 TP_DEV void q8_roundtrip4(float4& v) {
@@ -128,10 +153,12 @@ TP_DEV uint32_t q8_quantize4(float4 v, float* scale_out /* nullable */) {
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-  const float d = q8_scale(a);
+  const float d = q8_scale(a), r = q8_recip(d);
   if (scale_out && (threadIdx.x & 7) == 0) *scale_out = d;
-  const uint32_t c0 = (uint32_t)(q8_code(v.x, d) & 0xFF), c1 = (uint32_t)(q8_code(v.y, d) & 0xFF);
-  const uint32_t c2 = (uint32_t)(q8_code(v.z, d) & 0xFF), c3 = (uint32_t)(q8_code(v.w, d) & 0xFF);
+  const uint32_t c0 = (uint32_t)((int)q8_code_rf(v.x, d, r) & 0xFF);
+  const uint32_t c1 = (uint32_t)((int)q8_code_rf(v.y, d, r) & 0xFF);
+  const uint32_t c2 = (uint32_t)((int)q8_code_rf(v.z, d, r) & 0xFF);
+  const uint32_t c3 = (uint32_t)((int)q8_code_rf(v.w, d, r) & 0xFF);
   return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
 }
 
@@ -154,16 +181,17 @@ TP_DEV float4 q8_unpack4(uint32_t codes, float d) {
 // x4 + sum_{s < nslices} sync(sum_{k < parts} plane[(s parts + k) stride + off]),
 // slices in order, each partial passed through the Q8 round trip when quant (8
 // consecutive lanes hold a 32-value block: all 32 lanes call it, with the same
-// nslices). parts <= 2. The loads of 8 slices at a time are issued together
-// (L2 reads of partials other CTAs just stored: one latency per 8 slices, not
+// nslices). parts <= 2. The loads of 4 slices at a time are issued together
+// (L2 reads of partials other CTAs just stored: one latency per 4 slices, not
 // per slice). Reads through L2 (ld.cg); returns the new x4, not stored.
 TP_DEV float4 merge_lane4(const float* planes, size_t stride, size_t off, int nslices, int parts,
                           int quant, float4 x4) {
+  constexpr int kBatch = 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < nslices; s0 += 8) {
-    float4 p[8];
+  for (int s0 = 0; s0 < nslices; s0 += kBatch) {
+    float4 p[kBatch];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kBatch; ++j) {
       p[j] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
@@ -178,7 +206,7 @@ TP_DEV float4 merge_lane4(const float* planes, size_t stride, size_t off, int ns
       }
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kBatch; ++j) {
       if (s0 + j < nslices) {
         if (quant) q8_roundtrip4(p[j]);
         acc.x += p[j].x;
@@ -219,18 +247,11 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // the environment variable TP_PDL=0 turns it off, for comparison runs).
 bool pdl_enabled();
 
-// Every kernel asks for the largest shared-memory carve-out (once per kernel and
-// device): an SM whose L1 / shared split changes between kernels must drain first,
-// so a small kernel run with a smaller carve-out would keep the next big-ring
-// kernel's CTA off its SM until it ends.
-int prefer_max_shared(const void* kernel);
-
 // Launches `kernel` on `s`, allowing it to overlap its predecessor's tail
 // (programmatic dependent launch) when pdl_enabled().
 template <typename... KArgs, typename... Args>
 int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                Args&&... args) {
-  if (prefer_max_shared((const void*)kernel)) return TP_ECUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

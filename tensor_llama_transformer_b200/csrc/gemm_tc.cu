@@ -327,9 +327,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             float am = 0.f;
 #pragma unroll
             for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(p[j]));
-            const float d = q8_scale(am);
+            const float d = q8_scale(am), r = q8_recip(d);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) p[j] = q8_value(q8_code(p[j], d), d);
+            for (int j = 0; j < 32; ++j) p[j] = __fmul_rn(q8_code_rf(p[j], d, r), d);
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) run[c + j] += p[j];

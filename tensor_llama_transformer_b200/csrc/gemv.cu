@@ -220,11 +220,12 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   } else {
     // ---------------------------------------------------------------- consumers
     const int ncons = nc * 32;
-    // RMSNorm input with one segment (q/k/v, W1/W3 in 1D): each consumer thread loads
-    // the x and gain values of its vectors (8 values, v = thread + 256 k) once, up
-    // front, for the scale and the staging both: one round of loads, not two
+    // RMSNorm input with one segment (q/k/v, W1/W3 in 1D), one batch row per launch:
+    // each consumer thread loads the x and gain values of its vectors (8 values,
+    // v = thread + 256 k) once, up front, for the scale and the staging both: one
+    // round of loads, not two (two rows would spill registers)
     constexpr int kPreV = 2;
-    const bool pre = pl.pre && a.gain && a.nseg == 1 && nc == 8 && nv <= kPreV * 256;
+    const bool pre = NB == 1 && a.gain && a.nseg == 1 && nc == 8 && nv <= kPreV * 256;
     float4 px[NB][kPreV][2], pg[kPreV][2];
     // (re)stage the activations of segment `seg`; whole warps per iteration so that 4
     // consecutive lanes always hold one 32-value Q8 block. publish: this CTA owns the
@@ -413,7 +414,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
     // in the SM's instruction cache when the input arrives (the first run of this
     // code was measured about 2 us slower than a second one).
     const int seg0 = R0 / rps;
-    for (int pass = pre ? 0 : 1; pass < 2; ++pass) {
+    for (int pass = pre && pl.warm ? 0 : 1; pass < 2; ++pass) {
       const bool warm = pass == 0;
       if (!warm) {
         pdl_wait();  // activations / residual come from the previous kernel
@@ -650,9 +651,9 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
 
 size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
 
-int gemv_pre() {
+int gemv_warm() {
   static const int on = [] {
-    const char* v = getenv("TP_GEMV_PRE");
+    const char* v = getenv("TP_GEMV_WARM");
     return v && v[0] == '0' ? 0 : 1;
   }();
   return on;
@@ -682,7 +683,7 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
         p->pw = P == 16 ? 2 : 1;
         p->nstage = ns;
         p->cta_rows = cta_rows;
-        p->pre = gemv_pre() ? 1 : 0;
+        p->warm = gemv_warm();
         p->ring_off = 0;
         p->x_off = a128((size_t)ns * stage);
         p->res_off = p->x_off + x_bytes;

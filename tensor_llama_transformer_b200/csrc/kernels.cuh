@@ -12,18 +12,8 @@ namespace tp {
 // 128-value chunk of the new row is written too: ssq[b][chunk] (merge_ssq_parts(dim)
 // of them; one warp's float4 lanes summed by warp_sum, in both merge kernels, so
 // that both give the next RMSNorm the same bits). dim % 128 == 0, parts <= 2.
-// The first rows each CTA of the next slice GEMV streams, for a small kernel that
-// runs in the gap before it to prefetch into L2 (while it waits for its own
-// input): for pair-interleaved W1/W3 (SwiGLU), next-GEMV CTA c of `grid` starts at
-// pair P0(c) = npairs c / grid; `pairs` pairs of each are prefetched (rows of
-// row_bytes bytes, ld_bytes apart, in w[0] and w[1]). w[0] null: nothing.
-struct L2Ahead {
-  const void* w[2];
-  int64_t ld_bytes;
-  int row_bytes, npairs, grid, pairs;
-};
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts = 1, const L2Ahead* ahead = nullptr);
+                 cudaStream_t s, int parts = 1);
 inline int merge_ssq_parts(int dim) { return dim / 128; }
 // One slice's partial in the sync format for B rows: float32 [B, dim], or with Q8
 // the codes int8 [B, dim] followed by the scales float32 [B, dim/32].
@@ -115,7 +105,7 @@ struct GemvPlan {
   int pw;  // row pairs per warp and stage (2 with 16 pairs per stage)
   int nstage;
   int cta_rows;
-  int pre;  // RMSNorm input preloaded into registers, prologue warmed before the wait
+  int warm;  // run the preloading prologue once on dummy values before the wait
   size_t ring_off, x_off, res_off, bar_off, total;
 };
 

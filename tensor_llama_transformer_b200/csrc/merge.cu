@@ -16,38 +16,14 @@ namespace {
 
 constexpr int kMergeThreads = 128;  // 4 values per thread: 512 values per CTA
 
-// L2 prefetch of the next GEMV's first rows (L2Ahead): CTA c issues next-GEMV CTA
-// c's two ranges (an SM's bulk unit moves ~60 GB/s, so the prefetch needs as many
-// SMs as the GEMV has CTAs).
-TP_DEV void prefetch_ahead(const L2Ahead& h) {
-  if (!h.w[0] || threadIdx.x >= 2) return;
-  for (int i = 2 * blockIdx.x + threadIdx.x; i < 2 * h.grid; i += 2 * gridDim.x) {
-    const int c = i >> 1, m = i & 1;
-    const int p0 = (int)(((int64_t)h.npairs * c) / h.grid);
-    const int p1 = (int)(((int64_t)h.npairs * (c + 1)) / h.grid);
-    const int k = min(p1 - p0, h.pairs);
-    const uint8_t* src = static_cast<const uint8_t*>(h.w[m]) + (int64_t)p0 * h.ld_bytes;
-    if (h.ld_bytes == h.row_bytes) {
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src),
-                   "r"((uint32_t)k * h.row_bytes) : "memory");
-    } else {
-      for (int r = 0; r < k; ++r, src += h.ld_bytes)
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src),
-                     "r"((uint32_t)h.row_bytes) : "memory");
-    }
-  }
-}
-
 __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
-                                                         const float* __restrict__ part, int n,
-                                                         int parts, int B, int dim, int quant,
-                                                         float* __restrict__ ssq, L2Ahead ahead) {
+                                                      const float* __restrict__ part, int n,
+                                                      int parts, int B, int dim, int quant,
+                                                      float* __restrict__ ssq) {
   pdl_launch_dependents();
-  prefetch_ahead(ahead);  // the next GEMV's weights: no wait needed
-  // merge pieces: CTAs [0, pieces * B) (the grid may be larger, for the prefetch)
-  const int pieces = (dim / 4 + kMergeThreads - 1) / kMergeThreads;
-  if ((int)blockIdx.x >= pieces * B) return;
   pdl_wait();
+  // CTA = (batch row, 512-value piece)
+  const int pieces = (dim / 4 + kMergeThreads - 1) / kMergeThreads;
   const int b = blockIdx.x / pieces, piece = blockIdx.x - b * pieces;
   const int i4 = piece * kMergeThreads + threadIdx.x;  // float4 index within the row
   const int n4 = dim >> 2;
@@ -174,14 +150,10 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; }
 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts, const L2Ahead* ahead) {
+                 cudaStream_t s, int parts) {
   if (parts < 1 || parts > 2 || dim % 128 != 0) return TP_EINVAL;
-  L2Ahead h{};
-  if (ahead) h = *ahead;
-  int grid = merge_grid(dim) * B;
-  if (h.w[0] && grid < h.grid) grid = h.grid;
-  return launch_pdl(k_merge, dim3(grid), dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim, quant,
-                    ssq, h);
+  return launch_pdl(k_merge, dim3(merge_grid(dim) * B), dim3(kMergeThreads), 0, s, x, part, n, parts,
+                    B, dim, quant, ssq);
 }
 
 int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
