@@ -60,6 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--extras", default=None,
                     help="comma list of the extra workloads to time (default: all of them): "
                          "c2_block_persistent, c2_block_int8_weights, c2_prefill_chunk64, c4_block, "
+                         "c4_block_mqa, "
                          "c3_model_b1, c3_model_b16")
     ap.add_argument("--profile", choices=["c4", "c3b1", "c2p", "c2q8w", "c2prefill", "ffn"],
                     default=None,
@@ -604,14 +605,21 @@ def _time_graph(torch, fn, steps_per_graph, replays, warm=2):
     return ms
 
 
-def bench_c4(args):
-    """70B-shape GQA block (dim 8192, 64/8 heads, F 28672), batch 32, context 4096, n = 8."""
+def bench_c4(args, kv_heads=None):
+    """70B-shape GQA block (dim 8192, 64/8 heads, F 28672), batch 32, context 4096, n = 8;
+    with kv_heads = 1 the multi-query form of the same block as one slice (64 query heads
+    on one kv head: every group of 8 query heads streams the kv head's tiles; Pope et al.
+    demo 3)."""
+    import dataclasses
+
     import torch
 
     import synth
     import tensor_llama_transformer_b200 as tpb
 
-    s = synth.C4
+    # one kv head cannot be split over slices by heads: the multi-query block is one slice
+    s = synth.C4 if kv_heads is None else dataclasses.replace(synth.C4, n_kv_heads=kv_heads,
+                                                              n_slices=1)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(1003)
     B, D, F, H, Hkv, hd = s.batch, s.dim, s.ffn_dim, s.n_heads, s.n_kv_heads, s.head_dim
@@ -641,8 +649,9 @@ def bench_c4(args):
     gbs = (wb + kvb) / (ms / 1e3) / 1e9
     return {"us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "hbm_gbs": gbs,
             "frac": gbs / hbm, "bytes_per_step": wb + kvb,
-            "workload": "C4: 70B-shape GQA block, dim 8192, 64/8 heads, SwiGLU 28672, batch 32, "
-                        "context 4096, n=8, float32 sync buffers"}
+            "workload": f"C4{'' if kv_heads is None else ' multi-query'}: 70B-shape block, dim 8192, "
+                        f"{s.n_heads}/{s.n_kv_heads} heads, SwiGLU 28672, batch 32, context 4096, "
+                        f"n={s.n_slices}, float32 sync buffers"}
 
 
 def bench_c2_prefill(args):
@@ -995,6 +1004,7 @@ def main(argv=None):
 
         runs = [("c2_block_persistent", bench_c2_persistent), ("c2_block_int8_weights", bench_c2_q8w),
                 ("c2_prefill_chunk64", bench_c2_prefill), ("c4_block", bench_c4),
+                ("c4_block_mqa", lambda a: bench_c4(a, kv_heads=1)),
                 ("c3_model_b1", lambda a: bench_c3(a, 1)), ("c3_model_b16", lambda a: bench_c3(a, 16))]
         want = set(args.extras.split(",")) if args.extras else None
         extra = {}

@@ -392,148 +392,135 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
             xs[(NB + b) * nv + v] = make_float4(xv[4], xv[5], xv[6], xv[7]);
           }
       };
-      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+      // one call site of `stage` (its code is large): the preloaded registers of vector
+      // k = 0, 1 are picked by selects, not by a second, unrolled copy of the loop
       for (int b = 0; b < NB; ++b) {
-        if (pre) {
-#pragma unroll
-          for (int k = 0; k < kPreV; ++k) {
-            const int v = threadIdx.x + 256 * k;
-            if (v < nvr) stage(b, v, true, px[b][k][0], px[b][k][1], pg[k][0], pg[k][1]);
-          }
-        } else {
-          for (int v = threadIdx.x; v < nvr; v += ncons) stage(b, v, false, z4, z4, z4, z4);
+        int k = 0;
+#pragma unroll 1
+        for (int v = threadIdx.x; v < nvr; v += ncons, ++k) {
+          const bool hp = pre && k < kPreV;
+          const int b1 = NB == 1 ? 0 : b;
+          stage(b, v, hp, k == 0 ? px[b1][0][0] : px[b1][1][0], k == 0 ? px[b1][0][1] : px[b1][1][1],
+                k == 0 ? pg[0][0] : pg[1][0], k == 0 ? pg[0][1] : pg[1][1]);
         }
       }
       consumers_sync(ncons);
     };
 
-    // The q/k/v and W1/W3 products (RMSNorm input staged from registers) wait for a
-    // merge before their input exists. Their prologue runs first on dummy values,
-    // before that wait, with nothing written outside shared memory: its code is then
-    // in the SM's instruction cache when the input arrives (the first run of this
-    // code was measured about 2 us slower than a second one).
-    const int seg0 = R0 / rps;
-    for (int pass = pre && pl.warm ? 0 : 1; pass < 2; ++pass) {
-      const bool warm = pass == 0;
-      if (!warm) {
-        pdl_wait();  // activations / residual come from the previous kernel
-        if (tr && threadIdx.x == 0) tr[1] = gtimer();
-      }
-      if (pre) {
+    pdl_wait();  // activations / residual come from the previous kernel
+    if (tr && threadIdx.x == 0) tr[1] = gtimer();
+    if (pre) {
 #pragma unroll
-        for (int k = 0; k < kPreV; ++k) {
-          const int v = threadIdx.x + 256 * k;
-          const bool vin = v < nv && !warm;
-          const float zf = warm ? 1.f : 0.f;  // dummy values; past the row: zero
-          const float4 z = make_float4(zf, zf, zf, zf);
-          pg[k][0] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v) : z;
-          pg[k][1] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v + 4) : z;
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const bool in = vin && b < a.nb;
-            const float* xr = a.x + (size_t)(a.b0 + b) * a.ldx + 8 * (size_t)v;
-            px[b][k][0] = in ? *reinterpret_cast<const float4*>(xr) : z;
-            px[b][k][1] = in ? *reinterpret_cast<const float4*>(xr + 4) : z;
-          }
-        }
-      }
-      if (a.gain && a.ssq) {  // sums of squares left by the merge that produced x
-        if (warp < NB) {  // warp b: row b's parts, lanes in stride, then the butterfly
-          float t = warm ? 1.f : 0.f;
-          if (warp < a.nb && !warm)
-            for (int c = lane; c < a.ssq_parts; c += 32) t += a.ssq[(size_t)(a.b0 + warp) * a.ssq_parts + c];
-          t = warp_sum(t);
-          if (lane == 0) s_rstd[warp] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
-        }
-        consumers_sync(ncons);
-      } else if (a.gain) {  // RMSNorm scale of each batch row, over the whole row
-        const int D = a.ldx;
+      for (int k = 0; k < kPreV; ++k) {
+        const int v = threadIdx.x + 256 * k;
+        const bool vin = v < nv;  // past the row: zero
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        pg[k][0] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v) : z;
+        pg[k][1] = vin ? *reinterpret_cast<const float4*>(a.gain + 8 * (size_t)v + 4) : z;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          float ss = 0.f;
-          if (pre) {
+          const bool in = vin && b < a.nb;
+          const float* xr = a.x + (size_t)(a.b0 + b) * a.ldx + 8 * (size_t)v;
+          px[b][k][0] = in ? *reinterpret_cast<const float4*>(xr) : z;
+          px[b][k][1] = in ? *reinterpret_cast<const float4*>(xr + 4) : z;
+        }
+      }
+    }
+    if (a.gain && a.ssq) {  // sums of squares left by the merge that produced x
+      if (warp < NB) {  // warp b: row b's parts, lanes in stride, then the butterfly
+        float t = 0.f;
+        if (warp < a.nb)
+          for (int c = lane; c < a.ssq_parts; c += 32) t += a.ssq[(size_t)(a.b0 + warp) * a.ssq_parts + c];
+        t = warp_sum(t);
+        if (lane == 0) s_rstd[warp] = 1.0f / sqrtf(t / (float)a.ldx + a.eps);
+      }
+      consumers_sync(ncons);
+    } else if (a.gain) {  // RMSNorm scale of each batch row, over the whole row
+      const int D = a.ldx;
 #pragma unroll
-            for (int k = 0; k < kPreV; ++k)
+      for (int b = 0; b < NB; ++b) {
+        float ss = 0.f;
+        if (pre) {
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const float4 v = px[b][k][h];
-                ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-              }
-          } else if (b < a.nb) {
-            const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
-            for (int i = threadIdx.x; i < (D >> 2); i += ncons) {
-              const float4 v = xrow[i];
+          for (int k = 0; k < kPreV; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float4 v = px[b][k][h];
               ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
             }
+        } else if (b < a.nb) {
+          const float4* xrow = reinterpret_cast<const float4*>(a.x + (size_t)(a.b0 + b) * D);
+          for (int i = threadIdx.x; i < (D >> 2); i += ncons) {
+            const float4 v = xrow[i];
+            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
           }
-          ss = warp_sum(ss);
-          if (lane == 0) s_red[warp][b] = ss;
         }
-        consumers_sync(ncons);
-        if (threadIdx.x < NB) {
-          float t = 0.f;
-          for (int w = 0; w < nc; ++w) t += s_red[w][threadIdx.x];
-          s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)D + a.eps);
-        }
-        consumers_sync(ncons);
+        ss = warp_sum(ss);
+        if (lane == 0) s_red[warp][b] = ss;
       }
-      if (!warm && tr && threadIdx.x == 0) tr[2] = gtimer();  // the RMSNorm scale known
-      stage_segment(seg0, !warm && R0 == seg0 * rps);
+      consumers_sync(ncons);
+      if (threadIdx.x < NB) {
+        float t = 0.f;
+        for (int w = 0; w < nc; ++w) t += s_red[w][threadIdx.x];
+        s_rstd[threadIdx.x] = 1.0f / sqrtf(t / (float)D + a.eps);
+      }
+      consumers_sync(ncons);
     }
-    if (tr && threadIdx.x == 0) tr[3] = gtimer();
-
-    int cur_seg = seg0;
+    if (tr && threadIdx.x == 0) tr[2] = gtimer();  // the RMSNorm scale known
     bool ok = true;
     int t = 0;
     // this warp's share of a stage: row pair `pw` of the stage, vectors [vb, ve)
     const int pw = warp / Q, part = warp - pw * Q;
     const int vb = (nv * part) / Q, ve = (nv * (part + 1)) / Q;
-    for (int cur = 0; cur < nrows; ++t) {
-      const int end = stage_end(cur, nrows, R0, rps, P);
-      const int s = t % nstage;
-      const uint32_t ph = (uint32_t)(t / nstage) & 1u;
+    // one pass per segment of the CTA's rows: stage that segment's activations, then
+    // consume its ring stages (a stage never crosses a segment boundary); the staging
+    // code has this one call site, outside the streaming loop
+    for (int cur = 0; cur < nrows;) {
       const int seg = (R0 + cur) / rps;
-      if (seg != cur_seg) {
-        stage_segment(seg, (R0 + cur) == seg * rps);
-        cur_seg = seg;
-      }
-      // after a wait gives up, keep walking the stages (so that every consumer warp
-      // reaches the same named barriers) but skip the work
-      if (ok && !mbar_wait(&full[s], ph, a.err)) ok = false;
-      if (tr && t == 0 && threadIdx.x == 0) tr[4] = gtimer();
-      if (ok) {
-        const uint8_t* st = ring + (size_t)s * 2 * P * slot;
-        if constexpr (WQ8) {
-          // scale offset (floats) of each of the warp's rows inside its aligned run:
-          // (lrow * ldw / 32 + seg * Ks / 32) mod 4. Matrix boundaries inside a
-          // segment's rows are multiples of 4 rows (multiples of 128), so lrow mod 4
-          // follows from the row's place in its segment (halved for W1/W3 pairs).
-          int pad[2 * 2];
-          const int s32 = (int)((a.ldw / 32) & 3), segpad = (int)(((size_t)seg * (a.Ks / 32)) & 3);
-          const int seg_first = seg * rps - R0;  // CTA-local row where this segment starts
+      stage_segment(seg, (R0 + cur) == seg * rps);
+      if (tr && cur == 0 && threadIdx.x == 0) tr[3] = gtimer();
+      const int seg_end = min(nrows, (seg + 1) * rps - R0);
+      for (; cur < seg_end; ++t) {
+        const int end = stage_end(cur, nrows, R0, rps, P);
+        const int s = t % nstage;
+        const uint32_t ph = (uint32_t)(t / nstage) & 1u;
+        // after a wait gives up, keep walking the stages (so that every consumer warp
+        // reaches the same named barriers) but skip the work
+        if (ok && !mbar_wait(&full[s], ph, a.err)) ok = false;
+        if (tr && t == 0 && threadIdx.x == 0) tr[4] = gtimer();
+        if (ok) {
+          const uint8_t* st = ring + (size_t)s * 2 * P * slot;
+          if constexpr (WQ8) {
+            // scale offset (floats) of each of the warp's rows inside its aligned run:
+            // (lrow * ldw / 32 + seg * Ks / 32) mod 4. Matrix boundaries inside a
+            // segment's rows are multiples of 4 rows (multiples of 128), so lrow mod 4
+            // follows from the row's place in its segment (halved for W1/W3 pairs).
+            int pad[2 * 2];
+            const int s32 = (int)((a.ldw / 32) & 3), segpad = (int)(((size_t)seg * (a.Ks / 32)) & 3);
+            const int seg_first = seg * rps - R0;  // CTA-local row where this segment starts
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = cur + 2 * (pw + 8 * (i >> 1)) + (i & 1);
-            int lr = r - seg_first;
-            if (EPI == EPI_SWIGLU) lr >>= 1;
-            pad[i] = ((lr & 3) * s32 + segpad) & 3;
+            for (int i = 0; i < 4; ++i) {
+              const int r = cur + 2 * (pw + 8 * (i >> 1)) + (i & 1);
+              int lr = r - seg_first;
+              if (EPI == EPI_SWIGLU) lr >>= 1;
+              pad[i] = ((lr & 3) * s32 + segpad) & 3;
+            }
+            const int nc16 = a.Ks >> 4, cb = (nc16 * part) / Q, ce = (nc16 * (part + 1)) / Q;
+            if (pl.pw == 2)
+              ring_pairs_dot_q8<NB, 2>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+            else
+              ring_pairs_dot_q8<NB, 1>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+          } else {
+            if (pl.pw == 2)
+              ring_pairs_dot<NB, 2>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
+            else
+              ring_pairs_dot<NB, 1>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
           }
-          const int nc16 = a.Ks >> 4, cb = (nc16 * part) / Q, ce = (nc16 * (part + 1)) / Q;
-          if (pl.pw == 2)
-            ring_pairs_dot_q8<NB, 2>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
-          else
-            ring_pairs_dot_q8<NB, 1>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
-        } else {
-          if (pl.pw == 2)
-            ring_pairs_dot<NB, 2>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
-          else
-            ring_pairs_dot<NB, 1>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        cur = end;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      cur = end;
     }
     if (tr && threadIdx.x == 0) tr[5] = gtimer();
   }
@@ -651,14 +638,6 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
 
 size_t a128(size_t v) { return (v + 127) & ~(size_t)127; }
 
-int gemv_warm() {
-  static const int on = [] {
-    const char* v = getenv("TP_GEMV_WARM");
-    return v && v[0] == '0' ? 0 : 1;
-  }();
-  return on;
-}
-
 // Shared-memory plan: 8 consumer warps; the most row pairs per stage (16, 8, 4,
 // 2, 1) that still leave a ring of at least 3 stages (2 for the longest rows):
 // 16 pairs give each warp two pairs, fewer are each split over 8 / pairs warps.
@@ -683,7 +662,6 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
         p->pw = P == 16 ? 2 : 1;
         p->nstage = ns;
         p->cta_rows = cta_rows;
-        p->warm = gemv_warm();
         p->ring_off = 0;
         p->x_off = a128((size_t)ns * stage);
         p->res_off = p->x_off + x_bytes;

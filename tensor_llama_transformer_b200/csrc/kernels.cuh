@@ -105,7 +105,6 @@ struct GemvPlan {
   int pw;  // row pairs per warp and stage (2 with 16 pairs per stage)
   int nstage;
   int cta_rows;
-  int warm;  // run the preloading prologue once on dummy values before the wait
   size_t ring_off, x_off, res_off, bar_off, total;
 };
 
