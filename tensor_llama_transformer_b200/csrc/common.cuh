@@ -177,52 +177,6 @@ TP_DEV float4 q8_unpack4(uint32_t codes, float d) {
 // kernel waits for its predecessor's completion and memory (wait) only where it
 // first touches data the predecessor produced. Work before the wait may only
 // read inputs no earlier kernel writes (weights, pos, cache rows before pos).
-// The merge of one float4 of a row (distributed-llama DequantizeAtt + MergeAtt):
-// x4 + sum_{s < nslices} sync(sum_{k < parts} plane[(s parts + k) stride + off]),
-// slices in order, each partial passed through the Q8 round trip when quant (8
-// consecutive lanes hold a 32-value block: all 32 lanes call it, with the same
-// nslices). parts <= 2. The loads of 4 slices at a time are issued together
-// (L2 reads of partials other CTAs just stored: one latency per 4 slices, not
-// per slice). Reads through L2 (ld.cg); returns the new x4, not stored.
-TP_DEV float4 merge_lane4(const float* planes, size_t stride, size_t off, int nslices, int parts,
-                          int quant, float4 x4) {
-  constexpr int kBatch = 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < nslices; s0 += kBatch) {
-    float4 p[kBatch];
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      p[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        if (s0 + j < nslices && k < parts) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(
-              planes + (size_t)((s0 + j) * parts + k) * stride + off));
-          p[j].x += v.x;
-          p[j].y += v.y;
-          p[j].z += v.z;
-          p[j].w += v.w;
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      if (s0 + j < nslices) {
-        if (quant) q8_roundtrip4(p[j]);
-        acc.x += p[j].x;
-        acc.y += p[j].y;
-        acc.z += p[j].z;
-        acc.w += p[j].w;
-      }
-    }
-  }
-  x4.x += acc.x;
-  x4.y += acc.y;
-  x4.z += acc.z;
-  x4.w += acc.w;
-  return x4;
-}
-
 TP_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 TP_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

@@ -98,7 +98,9 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
                               const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
                               int part, int Q, int cb, int ce, int lane);
 
-template <int NB, int EPI, bool WQ8>
+// PW: row pairs per consumer warp and stage (GemvPlan::pw), a template parameter so
+// that each kernel's streaming loop holds only the dot-product variant it runs
+template <int NB, int EPI, bool WQ8, int PW>
 __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_rstd[NB];
@@ -506,15 +508,9 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
               pad[i] = ((lr & 3) * s32 + segpad) & 3;
             }
             const int nc16 = a.Ks >> 4, cb = (nc16 * part) / Q, ce = (nc16 * (part + 1)) / Q;
-            if (pl.pw == 2)
-              ring_pairs_dot_q8<NB, 2>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
-            else
-              ring_pairs_dot_q8<NB, 1>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+            ring_pairs_dot_q8<NB, PW>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
           } else {
-            if (pl.pw == 2)
-              ring_pairs_dot<NB, 2>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
-            else
-              ring_pairs_dot<NB, 1>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
+            ring_pairs_dot<NB, PW>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
           }
         }
         __syncwarp();
@@ -685,8 +681,9 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   const int cta_rows = 2 * ((npairs + grid - 1) / grid);
   GemvPlan pl;
   if (!make_plan(NB, a.Ks, cta_rows, WQ8, &pl)) return TP_ENOTSUP;
-  if (set_smem_once((const void*)k_gemv<NB, EPI, WQ8>, (int)pl.total)) return TP_ECUDA;
-  return launch_pdl(k_gemv<NB, EPI, WQ8>, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
+  auto kernel = pl.pw == 2 ? k_gemv<NB, EPI, WQ8, 2> : k_gemv<NB, EPI, WQ8, 1>;
+  if (set_smem_once((const void*)kernel, (int)pl.total)) return TP_ECUDA;
+  return launch_pdl(kernel, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
 }
 
 template <int NB, bool WQ8>

@@ -10,8 +10,9 @@ namespace tp {
 // s*parts .. s*parts+parts-1 of part [n*parts, B, dim] (a slice's contraction
 // split further by the GEMM). With ssq != nullptr the sum of squares of every
 // 128-value chunk of the new row is written too: ssq[b][chunk] (merge_ssq_parts(dim)
-// of them; one warp's float4 lanes summed by warp_sum, in both merge kernels, so
-// that both give the next RMSNorm the same bits). dim % 128 == 0, parts <= 2.
+// of them; each warp's squares summed by warp_sum and the chunk's four warp sums in
+// order, in both merge kernels, so that both give the next RMSNorm the same bits).
+// dim % 128 == 0, parts <= 2.
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts = 1);
 inline int merge_ssq_parts(int dim) { return dim / 128; }

@@ -5,16 +5,39 @@
 // does both for every element: each partial (the sum of its contraction parts
 // when a GEMM split it further) passes through the sync buffer's format (the Q8
 // round trip when quantisation is on), the partials are summed
-// in slice order 0..n-1 in float32, and the sum is added to x. The grid covers
-// the batch rows in 512-element pieces so that the merge of a single token is
-// spread over many SMs instead of waiting on one.
+// in slice order 0..n-1 in float32, and the sum is added to x. One value per
+// thread, one 128-value chunk of a row per CTA: the merge of a single token is
+// spread over dim/128 SMs, and each thread's chain of dependent steps (loads,
+// Q8 round trips, sum) is as short as it can be; a Q8 block is one warp.
 #include "kernels.cuh"
 
 namespace tp {
 
 namespace {
 
-constexpr int kMergeThreads = 128;  // 4 values per thread: 512 values per CTA
+constexpr int kMergeThreads = 128;  // one value per thread: a CTA is one 128-value chunk
+
+// The chunk's sum of squares from every thread's v*v: each warp's butterfly sum,
+// then the four warps' sums in order, written by thread 0 (the same bits in both
+// merge kernels, so the next RMSNorm sees the same scale either way).
+TP_DEV void chunk_ssq(float v, float* ssq_out) {
+  __shared__ float w[kMergeThreads / 32];
+  const float sq = warp_sum(v * v);
+  if ((threadIdx.x & 31) == 0) w[threadIdx.x >> 5] = sq;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = w[0];
+#pragma unroll
+    for (int i = 1; i < kMergeThreads / 32; ++i) t += w[i];
+    *ssq_out = t;
+  }
+}
+
+// The Q8 round trip of one value per lane, the 32 lanes of the warp being one block.
+TP_DEV float q8_roundtrip1(float p) {
+  const float d = q8_scale(warp_max(fabsf(p)));
+  return __fmul_rn(q8_code_rf(p, d, q8_recip(d)), d);
+}
 
 __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
                                                       const float* __restrict__ part, int n,
@@ -22,30 +45,34 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
                                                       float* __restrict__ ssq) {
   pdl_launch_dependents();
   pdl_wait();
-  // CTA = (batch row, 512-value piece)
-  const int pieces = (dim / 4 + kMergeThreads - 1) / kMergeThreads;
-  const int b = blockIdx.x / pieces, piece = blockIdx.x - b * pieces;
-  const int i4 = piece * kMergeThreads + threadIdx.x;  // float4 index within the row
-  const int n4 = dim >> 2;
-  if (piece * kMergeThreads + (threadIdx.x & ~31) >= n4) return;  // dim % 128: whole warps
-  // slice s's partial: the sum of its contraction parts (planes s*parts .. s*parts+parts-1)
-  float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim) + i4;
-  const float4 v = merge_lane4(part, (size_t)B * dim, (size_t)b * dim + 4 * (size_t)i4, n, parts,
-                               quant, *xr);
-  *xr = v;
-  float sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  if (ssq) {  // each warp's 128 values: their sum of squares, for the next RMSNorm
-    sq = warp_sum(sq);
-    const int chunk = (piece * kMergeThreads + (threadIdx.x & ~31)) >> 5;
-    if ((threadIdx.x & 31) == 0 && chunk < (dim >> 7)) ssq[(size_t)b * (dim >> 7) + chunk] = sq;
+  // CTA = (batch row, 128-value chunk), grid (dim / 128) x B
+  const int nch = dim >> 7;
+  const int b = blockIdx.x / nch, ch = blockIdx.x - b * nch;
+  const size_t i = (size_t)b * dim + (size_t)ch * kMergeThreads + threadIdx.x;
+  const size_t stride = (size_t)B * dim;
+  const float x0 = x[i];
+  // slice s's partial: the sum of its contraction parts (planes s*parts .. s*parts+parts-1);
+  // the loads of 4 slices at a time are issued together (L2 reads of partials other
+  // CTAs just stored: one latency per 4 slices)
+  float acc = 0.f;
+  for (int s0 = 0; s0 < n; s0 += 4) {
+    float p[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      p[j] = 0.f;
+      for (int k = 0; k < parts && s0 + j < n; ++k)
+        p[j] += __ldcg(part + (size_t)((s0 + j) * parts + k) * stride + i);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (s0 + j < n) acc += quant ? q8_roundtrip1(p[j]) : p[j];
+    }
   }
+  const float v = x0 + acc;
+  x[i] = v;
+  if (ssq) chunk_ssq(v, ssq + (size_t)b * nch + ch);
 }
 
-// Sync-buffer pack for a rank that holds slices of the block (the send side of
-// distributed-llama's SyncAtt / SyncFfn2): slice s's partial, the sum of its
-// contraction parts, written in the slice's sync format -- float32 [B, dim], or
-// with Q8 the codes int8 [B, dim] followed by the scales float32 [B, dim/32].
-// Grid (pieces of 512 values, B, local slices).
 __global__ void __launch_bounds__(kMergeThreads) k_sync_pack(const float* __restrict__ part,
                                                              int parts, int B, int dim, int quant,
                                                              uint8_t* __restrict__ out) {
@@ -74,7 +101,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_sync_pack(const float* __rest
 }
 
 // The receive side: x[b] += sum_{s<n} deq(slice s of the gathered buffer), in
-// slice order, with the same per-piece sums of squares as k_merge. Dequantising a
+// slice order, with the same chunk sums of squares as k_merge. Dequantising a
 // packed slice gives the same bits as k_merge's in-place round trip, so a block
 // whose slices are spread over ranks merges exactly as the whole block does.
 __global__ void __launch_bounds__(kMergeThreads) k_merge_sync(float* __restrict__ x,
@@ -83,42 +110,25 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge_sync(float* __restrict_
                                                               float* __restrict__ ssq) {
   pdl_launch_dependents();
   pdl_wait();
-  const int b = blockIdx.y;
-  const int i4 = blockIdx.x * kMergeThreads + threadIdx.x;
-  const int n4 = dim >> 2;
-  const bool in = i4 < n4;
-  const size_t chunk = (size_t)sync_slice_bytes(B, dim, quant);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n && in; ++s) {
-    const uint8_t* base = sync + (size_t)s * chunk;
-    float4 p;
+  const int nch = dim >> 7;
+  const int b = blockIdx.x / nch, ch = blockIdx.x - b * nch;
+  const size_t e = (size_t)b * dim + (size_t)ch * kMergeThreads + threadIdx.x;  // [B, dim] index
+  const size_t bytes = (size_t)sync_slice_bytes(B, dim, quant);
+  float acc = 0.f;
+  for (int s = 0; s < n; ++s) {
+    const uint8_t* base = sync + (size_t)s * bytes;
+    float p;
     if (quant) {
-      const float d = reinterpret_cast<const float*>(base + (size_t)B * dim)[((size_t)b * dim + 4 * (size_t)i4) / kQ8Block];
-      p = q8_unpack4(reinterpret_cast<const uint32_t*>(base)[(size_t)b * n4 + i4], d);
+      const float d = reinterpret_cast<const float*>(base + (size_t)B * dim)[e / kQ8Block];
+      p = q8_value((int)reinterpret_cast<const int8_t*>(base)[e], d);
     } else {
-      p = reinterpret_cast<const float4*>(base)[(size_t)b * n4 + i4];
+      p = reinterpret_cast<const float*>(base)[e];
     }
-    acc.x += p.x;
-    acc.y += p.y;
-    acc.z += p.z;
-    acc.w += p.w;
+    acc += p;
   }
-  float sq = 0.f;
-  if (in) {
-    float4* xr = reinterpret_cast<float4*>(x + (size_t)b * dim);
-    float4 v = xr[i4];
-    v.x += acc.x;
-    v.y += acc.y;
-    v.z += acc.z;
-    v.w += acc.w;
-    xr[i4] = v;
-    sq = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  }
-  if (ssq) {  // as k_merge: one sum of squares per warp's 128 values
-    sq = warp_sum(sq);
-    const int chunk = (blockIdx.x * kMergeThreads + (threadIdx.x & ~31)) >> 5;
-    if ((threadIdx.x & 31) == 0 && chunk < (dim >> 7)) ssq[(size_t)b * (dim >> 7) + chunk] = sq;
-  }
+  const float v = x[e] + acc;
+  x[e] = v;
+  if (ssq) chunk_ssq(v, ssq + (size_t)b * nch + ch);
 }
 
 __global__ void k_quantize(const float* __restrict__ x, int8_t* __restrict__ q,
@@ -146,14 +156,14 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 
 }  // namespace
 
-// 512 values (4 warps of float4 lanes) per CTA
+// 512 values (4 warps of float4 lanes) per CTA of the sync pack
 int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; }
 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts) {
   if (parts < 1 || parts > 2 || dim % 128 != 0) return TP_EINVAL;
-  return launch_pdl(k_merge, dim3(merge_grid(dim) * B), dim3(kMergeThreads), 0, s, x, part, n, parts,
-                    B, dim, quant, ssq);
+  return launch_pdl(k_merge, dim3((dim >> 7) * B), dim3(kMergeThreads), 0, s, x, part, n, parts, B,
+                    dim, quant, ssq);
 }
 
 int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
@@ -164,8 +174,9 @@ int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, 
 
 int launch_merge_sync(float* x, const uint8_t* sync, int n, int B, int dim, int quant, float* ssq,
                       cudaStream_t s) {
-  const dim3 grid(merge_grid(dim), B);
-  return launch_pdl(k_merge_sync, grid, dim3(kMergeThreads), 0, s, x, sync, n, B, dim, quant, ssq);
+  if (dim % 128 != 0) return TP_EINVAL;
+  return launch_pdl(k_merge_sync, dim3((dim >> 7) * B), dim3(kMergeThreads), 0, s, x, sync, n, B, dim,
+                    quant, ssq);
 }
 
 int launch_quantize(const float* x, int8_t* q, float* d, int64_t n, cudaStream_t s) {
