@@ -336,12 +336,16 @@ def gemv_timeline(torch, tpb, h, fwd, local):
     timeline = {}
     base = t[t[:, 0] > 0, 0].min()
     marks = ("start", "prev_done", "norm", "staged", "first_stage", "consumed", "end")
-    for gi, name in enumerate(("qkv", "wo", "w13", "w2")):
-        cols = t[:, 7 * gi:7 * gi + 7]
+    merge_marks = ("start", "prev_done", "end")
+    for name, c0, mk in (("qkv", 0, marks), ("wo", 7, marks), ("merge_wo", 28, merge_marks),
+                         ("w13", 14, marks), ("w2", 21, marks), ("merge_w2", 31, merge_marks)):
+        cols = t[:, c0:c0 + len(mk)]
         cols = cols[cols[:, 0] > 0]
+        if not len(cols):
+            continue
         timeline[name] = {m: [round(float(f((cols[:, k] - base) / 1e3)), 2)
                               for f in (min, statistics.median, max)]
-                          for k, m in enumerate(marks)}
+                          for k, m in enumerate(mk)}
         st = (cols[:, 0] - cols[:, 0].min()) / 1e3
         timeline[name]["late_ctas"] = int((st > 2.0).sum())
     return timeline

@@ -286,9 +286,11 @@ TP_API int tp_block_set_persistent(tp_block* blk, int enable);
  * start, 1 the previous kernel complete (its wait returned), 2 the RMSNorm scale
  * known, 3 activations staged, 4 the first weight stage arrived, 5 the last stage
  * consumed, 6 end (after the epilogue); for batch > 2 the last launch of each
- * wins. The persistent kernel uses slots 0-15.
+ * wins; and for its two merges m (0 after W_O, 1 after W2) and merge CTA c < SM
+ * count, trace[c * TP_BLOCK_TRACE_SLOTS + 28 + 3m + k]: k = 0 start, 1 the previous
+ * kernel complete, 2 end. The persistent kernel uses slots 0-15.
  * Errors: TP_EINVAL (NULL handle, buffer too small). */
-#define TP_BLOCK_TRACE_SLOTS 32
+#define TP_BLOCK_TRACE_SLOTS 40
 TP_API int tp_block_set_trace(tp_block* blk, void* trace, size_t bytes);
 
 /* One block decode step that allocates nothing (no counterpart in the paper: this

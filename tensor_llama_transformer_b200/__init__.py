@@ -264,7 +264,7 @@ def tp_block_set_trace(handle, buf, nbytes):
     _check(_lib.tp_block_set_trace(handle, _ptr(buf), nbytes), "tp_block_set_trace")
 
 
-TP_BLOCK_TRACE_SLOTS = 32
+TP_BLOCK_TRACE_SLOTS = 40
 
 
 def tp_ffn_workspace_bytes(desc: tp_ffn_desc) -> int:

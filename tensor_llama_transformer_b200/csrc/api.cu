@@ -286,11 +286,20 @@ int stage_mark(const tp_block* blk, int stage, cudaStream_t s) {
 // a6 / a10. Whole block: x += the slice partials (planes of `part`), summed in
 // slice order through the sync format. Rank block: the same over the gathered
 // sync buffer, which holds every rank's slices in slice order.
+// m: 0 the merge after W_O, 1 the merge after W2 (trace slots 28 + 3m .. 30 + 3m).
 int merge_step(tp_block* blk, float* x, const float* part, int nseg, int parts, int batch,
-               cudaStream_t s) {
+               cudaStream_t s, int m) {
   const Cfg& c = blk->c;
   float* ssq = at<float>(blk, BUF_SSQ);
-  if (c.world == 0) return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts);
+  if (c.world == 0) {
+    MergeTrace t{};
+    if (blk->trace) {
+      t.stamps = blk->trace + 28 + 3 * m;
+      t.stride = TP_BLOCK_TRACE_SLOTS;
+      t.rows = num_sms();
+    }
+    return launch_merge(x, part, nseg, batch, c.d.dim, c.quant, ssq, s, parts, t);
+  }
   return launch_merge_sync(x, at<uint8_t>(blk, BUF_RECV), c.n * c.world, batch, c.d.dim, c.quant,
                            ssq, s);
 }
@@ -448,7 +457,7 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
   if (phase <= 1) {
     // a6 (a rank block: the merge of the gathered buffer)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s, 0))) return rc;
     // a7-a8
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if ((rc = norm(blk->w.ffn_norm, at<float>(blk, BUF_SSQ)))) return rc;
@@ -489,7 +498,7 @@ int block_forward_tc(tp_block* blk, float* x, void* kc, void* vc, const int32_t*
   }
   // a10
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = merge_step(blk, x, part, nseg2, p2, batch, s))) return rc;
+  if ((rc = merge_step(blk, x, part, nseg2, p2, batch, s, 1))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 
@@ -673,7 +682,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
     // a6: sync + dequantise + merge into the residual (a rank block: of the
     // gathered buffer)
     if ((rc = stage_mark(blk, 3, s))) return rc;
-    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s))) return rc;
+    if ((rc = merge_step(blk, x, part, c.n, 1, batch, s, 0))) return rc;
     // a7-a8: RMSNorm (+Q8) fused into the W1/W3 slice products, SwiGLU epilogue
     if ((rc = stage_mark(blk, 4, s))) return rc;
     if (c.partition == TP_PART_1D) {
@@ -754,7 +763,7 @@ int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_
   }
   // a10: sync + dequantise + merge
   if ((rc = stage_mark(blk, 6, s))) return rc;
-  if ((rc = merge_step(blk, x, part, nseg2, 1, batch, s))) return rc;
+  if ((rc = merge_step(blk, x, part, nseg2, 1, batch, s, 1))) return rc;
   return stage_mark(blk, TP_BLOCK_STAGES, s);
 }
 

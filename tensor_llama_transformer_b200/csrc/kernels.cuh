@@ -13,8 +13,14 @@ namespace tp {
 // of them; each warp's squares summed by warp_sum and the chunk's four warp sums in
 // order, in both merge kernels, so that both give the next RMSNorm the same bits).
 // dim % 128 == 0, parts <= 2.
+// Optional %globaltimer stamps of merge CTA c < rows: stamps[c * stride + k], k = 0
+// start, 1 the previous kernel complete, 2 end.
+struct MergeTrace {
+  unsigned long long* stamps;
+  int stride, rows;
+};
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts = 1);
+                 cudaStream_t s, int parts = 1, MergeTrace trace = MergeTrace{});
 inline int merge_ssq_parts(int dim) { return dim / 128; }
 // One slice's partial in the sync format for B rows: float32 [B, dim], or with Q8
 // the codes int8 [B, dim] followed by the scales float32 [B, dim/32].

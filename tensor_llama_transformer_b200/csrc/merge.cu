@@ -10,6 +10,7 @@
 // spread over dim/128 SMs, and each thread's chain of dependent steps (loads,
 // Q8 round trips, sum) is as short as it can be; a Q8 block is one warp.
 #include "kernels.cuh"
+#include "pipeline.cuh"
 
 namespace tp {
 
@@ -42,9 +43,14 @@ TP_DEV float q8_roundtrip1(float p) {
 __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
                                                       const float* __restrict__ part, int n,
                                                       int parts, int B, int dim, int quant,
-                                                      float* __restrict__ ssq) {
+                                                      float* __restrict__ ssq, MergeTrace tr) {
   pdl_launch_dependents();
+  unsigned long long* st =
+      tr.stamps && threadIdx.x == 0 && (int)blockIdx.x < tr.rows ? tr.stamps + (size_t)blockIdx.x * tr.stride
+                                                                 : nullptr;
+  if (st) st[0] = gtimer();
   pdl_wait();
+  if (st) st[1] = gtimer();
   // CTA = (batch row, 128-value chunk), grid (dim / 128) x B
   const int nch = dim >> 7;
   const int b = blockIdx.x / nch, ch = blockIdx.x - b * nch;
@@ -71,6 +77,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
   const float v = x0 + acc;
   x[i] = v;
   if (ssq) chunk_ssq(v, ssq + (size_t)b * nch + ch);
+  if (st) st[2] = gtimer();
 }
 
 __global__ void __launch_bounds__(kMergeThreads) k_sync_pack(const float* __restrict__ part,
@@ -160,10 +167,10 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; }
 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts) {
+                 cudaStream_t s, int parts, MergeTrace trace) {
   if (parts < 1 || parts > 2 || dim % 128 != 0) return TP_EINVAL;
   return launch_pdl(k_merge, dim3((dim >> 7) * B), dim3(kMergeThreads), 0, s, x, part, n, parts, B,
-                    dim, quant, ssq);
+                    dim, quant, ssq, trace);
 }
 
 int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
