@@ -68,6 +68,10 @@ def parse_args(argv=None):
                          "lists: c4 block, c3 model at batch 1, c2 block on the persistent kernel, "
                          "c2 block with int8 weights, c2 prefill chunk, or the fused PaLM-shaped "
                          "FFN at B 512 with F cut to --profile-ffn-f)")
+    ap.add_argument("--profile-ffn-form", choices=["fused", "faithful", "faithful_q8"],
+                    default="fused",
+                    help="--profile ffn: the merge form (faithful: 1D over F / 1152 slices, so every "
+                         "slice has the 1152-wide contraction of the full-size 1D-64 form)")
     ap.add_argument("--profile-ffn-f", type=int, default=18432,
                     help="intermediate size of the --profile ffn case (PaLM: 73728)")
     ap.add_argument("--profile-steps", type=int, default=3)
@@ -928,9 +932,12 @@ def bench_ffn(args):
 
 
 def profile_ffn(args):
-    """A few fused forwards of the PaLM-shaped FFN (B 512, E 18432, ReLU, 1D over 64
-    slices) with F cut to --profile-ffn-f, so that a full-section capture of one
-    tcgen05 GEMM launch holds a few GB on the device (F 18432: 1.36 GB of weights)."""
+    """A few forwards of the PaLM-shaped FFN (B 512, E 18432, ReLU, 1D) with F cut to
+    --profile-ffn-f, so that a full-section capture of one tcgen05 GEMM launch holds a
+    few GB on the device (F 18432: 1.36 GB of weights). --profile-ffn-form: fused (64
+    slices), or faithful / faithful_q8 over F / 1152 slices (16 at F 18432), the slice
+    width of the full-size 1D-64 form, so the segment-sum GEMM does the same work per
+    segment as at full size."""
     import torch
 
     import tensor_llama_transformer_b200 as tpb
@@ -942,8 +949,11 @@ def profile_ffn(args):
     W1 = _randn_bf16(torch, gen, (F, E), 0.01)
     W2 = _randn_bf16(torch, gen, (E, F), 0.01)
     Y = torch.empty((B, E), dtype=torch.float32, device="cuda")
-    desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, 64, 1, 1, 0,
-                           tpb.TP_MERGE_FUSED)
+    form = args.profile_ffn_form
+    n = 64 if form == "fused" else max(1, F // 1152)
+    merge = tpb.TP_MERGE_FUSED if form == "fused" else tpb.TP_MERGE_FAITHFUL
+    desc = tpb.tp_ffn_desc(B, E, F, tpb.TP_BF16, tpb.TP_ACT_RELU, tpb.TP_PART_1D, n, 1, 1,
+                           int(form == "faithful_q8"), merge)
     nb = tpb.tp_ffn_workspace_bytes(desc)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     for _ in range(args.profile_steps):
@@ -956,7 +966,8 @@ def profile_ffn(args):
     b.synchronize()
     ms = a.elapsed_time(b)
     flops = 2.0 * B * 2 * E * F
-    return {"profile": "ffn", "steps": args.profile_steps + 1, "B": B, "E": E, "F": F,
+    return {"profile": "ffn", "form": form, "n_slices": n, "steps": args.profile_steps + 1, "B": B,
+            "E": E, "F": F,
             "last_forward_ms": ms, "tflops": flops / (ms / 1e3) / 1e12,
             "pipeline_error": int(ws[:4].view(torch.int32).item())}
 
