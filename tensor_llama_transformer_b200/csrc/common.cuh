@@ -83,6 +83,11 @@ TP_DEV float block_max(float v, float* red) {
 // the codes are reproducible bit for bit on any IEEE machine.
 TP_DEV float q8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
 
+// The correctly rounded quotient, out of line: the codecs below take it only for the
+// rare values near a rounding tie (and for scales outside [2^-120, 2^120]), so one copy
+// of its code serves every caller instead of one inlined per value of an unrolled loop.
+static __device__ __noinline__ float q8_div_rn(float x, float d) { return __fdiv_rn(x, d); }
+
 // The code is round(fl(x / d)) with fl the correctly rounded quotient. The
 // quotient is first taken with the fast division __fdividef (at most 2 ulp from
 // x / d for d in the normal range, so at most 2.5 ulp from fl(x / d)); since
@@ -96,9 +101,9 @@ TP_DEV int q8_code(float x, float d) {
   if (d > 0x1p-120f && d < 0x1p120f) {
     q = __fdividef(x, d);
     const float a = fabsf(q);
-    if (fabsf(a - truncf(a) - 0.5f) < 4e-5f) q = __fdiv_rn(x, d);
+    if (fabsf(a - truncf(a) - 0.5f) < 4e-5f) q = q8_div_rn(x, d);
   } else {
-    q = __fdiv_rn(x, d);
+    q = q8_div_rn(x, d);
   }
   float v = roundf(q);  // roundf: halfway cases away from zero
   v = fminf(fmaxf(v, -127.0f), 127.0f);
@@ -124,9 +129,9 @@ TP_DEV float q8_code_rf(float x, float d, float r) {
   if (r != 0.f) {
     q = __fmul_rn(x, r);
     const float a = fabsf(q);
-    if (fabsf(a - truncf(a) - 0.5f) < 4e-5f) q = __fdiv_rn(x, d);
+    if (fabsf(a - truncf(a) - 0.5f) < 4e-5f) q = q8_div_rn(x, d);
   } else {
-    q = __fdiv_rn(x, d);
+    q = q8_div_rn(x, d);
   }
   // roundf: halfway cases away from zero; + 0 turns a -0 code into +0
   return fminf(fmaxf(roundf(q), -127.0f), 127.0f) + 0.0f;

@@ -17,7 +17,7 @@
 // weight rows on M and the batch on N (N tile 32 or 64, transposed store), so
 // the weight stream is the M x K operand.
 //
-// Structure (one CTA per SM, 192 threads):
+// Structure (one CTA per SM, 192 threads; 320 with the quantised segment sum):
 //   warp 0  : TMA producer — 128x64 A tile and BNx64 B tile per stage, 128-byte
 //             swizzle, a ring of 4 (BN 256) to 10 (BN 32) stages of shared
 //             memory, completion on mbarriers.
@@ -26,7 +26,9 @@
 //             tcgen05.commit releases each smem stage and publishes each tile.
 //   warps 2-5: epilogue — tcgen05.ld of the accumulator (each warp its 32 TMEM
 //             lanes = 32 output rows), activation, stores to global memory,
-//             overlapped with the next tile's mainloop (double-buffered TMEM).
+//             overlapped with the next tile's mainloop (double-buffered TMEM);
+//             warps 2-9 with the quantised segment sum, two per lane quarter,
+//             each owning half of the tile's columns.
 // Tiles are visited m-fastest so that the CTAs working at the same time share
 // the weight tile through L2. No TMA multicast is used. Every wait on an
 // mbarrier is bounded by a 2 s timer; on expiry the kernel sets *err and the
@@ -39,7 +41,16 @@
 namespace tp {
 namespace {
 
-constexpr int BM = 128, BK = 64, THREADS = 192;
+constexpr int BM = 128, BK = 64;
+
+// EW epilogue warps: 4 (one per 32-lane quarter of TMEM), or 8 for the segment sum with
+// the Q8 round trip (the only 8-warp form, so EW == 8 also selects the round trip at
+// compile time), where two warps share a lane quarter and each owns half of the
+// tile's columns: each then waits for two column loads per segment instead of four,
+// keeps half the running sums and quantises half the values, and every SM
+// sub-partition has two epilogue warps to hide the latencies (measured: Q8 faithful
+// 1D-64 FFN 5.8 -> 3.6 ms; without Q8 the 4-warp form is 4 % faster).
+constexpr int tc_threads(int ew) { return 64 + 32 * ew; }
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 
 template <int BN>
@@ -119,8 +130,8 @@ struct TcTiles {
   int ntiles;
 };
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int BN, int EPI, int EW>
+__global__ void __launch_bounds__(tc_threads(EW), 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
               const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB,
               const __grid_constant__ CUtensorMap mB2, TcGemm g, TcTiles tt) {
@@ -147,7 +158,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(&tfull[j], 1);
-      mbar_init(&tempty[j], 4);
+      mbar_init(&tempty[j], EW);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -291,9 +302,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // epilogue warps 2..5: TMEM lanes 32*(warp%4) .. +31
-    const int q = warp & 3;
+    const int q = warp & 3;  // TMEM lane quarter (hardware: warp w reads lanes 32 (w % 4) ..)
+    // segment sum: the warp's half of the tile's columns, [cw * cpart, cw * (cpart + 1))
+    constexpr int CW = BN * 4 / EW;
+    const int cpart = (warp - 2) >> 2;
     // TC_EPI_SEGSUM_*: the thread's row of the output tile, summed over the segments so far
-    float run[SEGSUM ? BN : 1];
+    float run[SEGSUM ? CW : 1];
     for (int it = 0;; ++it) {
       const int tile = tile_of(it);
       if (tile < 0) break;
@@ -312,18 +326,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         // float32 additions as summing materialised partials one slice after another
         if (seg == 0) {
 #pragma unroll
-          for (int j = 0; j < BN; ++j) run[j] = 0.f;
+          for (int j = 0; j < CW; ++j) run[j] = 0.f;
         }
         const bool last = seg == g.nseg - 1;
+        const int cb = cpart * CW;  // the warp's first column within the tile
 #pragma unroll
-        for (int c = 0; c < BN; c += 32) {
+        for (int h = 0; h < CW / 32; ++h) {
+          const int c = cb + 32 * h;  // tile column of this 32-column block
           uint32_t v[32];
           tmem_ld32(taddr + c, v);
           tmem_wait_ld();
           float p[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) p[j] = __uint_as_float(v[j]);
-          if (g.quant) {  // the 32 columns are one Q8 block of the row (n0 + c is a multiple of 32)
+          if constexpr (EW == 8) {  // quantised (the host runs the Q8 segment sum with 8 warps):
+            // the 32 columns are one Q8 block of the row (n0 + c is a multiple of 32)
             float am = 0.f;
 #pragma unroll
             for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(p[j]));
@@ -332,15 +349,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j) p[j] = __fmul_rn(q8_code_rf(p[j], d, r), d);
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) run[c + j] += p[j];
+          for (int j = 0; j < 32; ++j) run[32 * h + j] += p[j];
           if (last && row_ok && n0 + c < g.N) {
             if (EPI == TC_EPI_SEGSUM_F32) {
               float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
                                                      (size_t)row * g.ldo + n0 + c);
 #pragma unroll
               for (int j = 0; j < 8; ++j)
-                o4[j] = make_float4(run[c + 4 * j], run[c + 4 * j + 1], run[c + 4 * j + 2],
-                                    run[c + 4 * j + 3]);
+                o4[j] = make_float4(run[32 * h + 4 * j], run[32 * h + 4 * j + 1],
+                                    run[32 * h + 4 * j + 2], run[32 * h + 4 * j + 3]);
             } else {
               uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) +
                                                    (size_t)row * g.ldo + n0 + c);
@@ -348,7 +365,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int j = 0; j < 4; ++j) {
                 float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = fmaxf(run[c + 8 * j + e], 0.f);
+                for (int e = 0; e < 8; ++e) f[e] = fmaxf(run[32 * h + 8 * j + e], 0.f);
                 o4[j] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                    pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
               }
@@ -517,16 +534,16 @@ bool make_tensor_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_
 
 namespace {
 
-template <int BN, int EPI>
+template <int BN, int EPI, int EW = 4>
 int launch_cfg(const CUtensorMap* mA, const CUtensorMap& mB, const CUtensorMap& mB2,
                const TcGemm& g, const TcTiles& tt, cudaStream_t s) {
   constexpr int smem = TcCfg<BN>::SMEM_BYTES;
-  if (set_smem_once((const void*)k_tc_gemm<BN, EPI>, smem)) return TP_ECUDA;
+  if (set_smem_once((const void*)k_tc_gemm<BN, EPI, EW>, smem)) return TP_ECUDA;
   // with the segment sum a CTA takes every segment of an output tile
   const int units =
       EPI == TC_EPI_SEGSUM_F32 || EPI == TC_EPI_SEGSUM_RELU_BF16 ? tt.ntiles / g.nseg : tt.ntiles;
   const int grid = units < num_sms() ? units : num_sms();
-  return launch_pdl(k_tc_gemm<BN, EPI>, dim3(grid), dim3(THREADS), smem, s, mA[0], mA[1], mA[2], mB,
+  return launch_pdl(k_tc_gemm<BN, EPI, EW>, dim3(grid), dim3(tc_threads(EW)), smem, s, mA[0], mA[1], mA[2], mB,
                     mB2, g, tt);
 }
 
@@ -577,9 +594,12 @@ int launch_tc_gemm(const TcGemm& g, cudaStream_t s) {
     case TC_EPI_STORE_F32: return launch_cfg<256, TC_EPI_STORE_F32>(mA, mB, mB2, g, tt, s);
     case TC_EPI_RELU_BF16: return launch_cfg<256, TC_EPI_RELU_BF16>(mA, mB, mB2, g, tt, s);
     case TC_EPI_SWIGLU_BF16: return launch_cfg<256, TC_EPI_SWIGLU_BF16>(mA, mB, mB2, g, tt, s);
-    case TC_EPI_SEGSUM_F32: return launch_cfg<128, TC_EPI_SEGSUM_F32>(mA, mB, mB2, g, tt, s);
+    case TC_EPI_SEGSUM_F32:
+      return g.quant ? launch_cfg<128, TC_EPI_SEGSUM_F32, 8>(mA, mB, mB2, g, tt, s)
+                     : launch_cfg<128, TC_EPI_SEGSUM_F32>(mA, mB, mB2, g, tt, s);
     case TC_EPI_SEGSUM_RELU_BF16:
-      return launch_cfg<128, TC_EPI_SEGSUM_RELU_BF16>(mA, mB, mB2, g, tt, s);
+      return g.quant ? launch_cfg<128, TC_EPI_SEGSUM_RELU_BF16, 8>(mA, mB, mB2, g, tt, s)
+                     : launch_cfg<128, TC_EPI_SEGSUM_RELU_BF16>(mA, mB, mB2, g, tt, s);
     default: return TP_EINVAL;
   }
 }
