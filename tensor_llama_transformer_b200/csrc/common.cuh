@@ -137,6 +137,60 @@ TP_DEV float q8_code_rf(float x, float d, float r) {
   return fminf(fmaxf(roundf(q), -127.0f), 127.0f) + 0.0f;
 }
 
+// The Q8 round trip of N values of N different blocks, value i with its block's scale
+// d[i] (a merge's slices): one branch for all of them, as in q8_codes below; the result
+// is q8_value(q8_code(p[i], d[i]), d[i]) bit for bit.
+template <int N>
+TP_DEV void q8_roundtrip_each(float* p, const float* d);
+
+// The codes of N values of one block (q8_code_rf of each, bit for bit) without a branch
+// per value: every quotient q = x * r is formed first, with one flag for "some q lies
+// within 4e-5 of a tie, or the scale is outside [2^-120, 2^120]". Without it (nearly
+// always), round half away from zero is trunc(q + copysign(1/2, q)): for |q| < 128 the
+// sum is off by at most 3.8e-6, so it cannot cross an integer when q is at least 4e-5
+// from a tie. With it, every value takes q8_code_rf. c may be x (codes in place).
+template <int N>
+TP_DEV void q8_codes(const float* x, float* c, float d, float r) {
+  bool near = !(r != 0.f);
+  float q[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    q[i] = __fmul_rn(x[i], r);
+    const float a = fabsf(q[i]);
+    near |= fabsf(a - truncf(a) - 0.5f) < 4e-5f;
+  }
+  if (!near) {
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      c[i] = fminf(fmaxf(truncf(__fadd_rn(q[i], copysignf(0.5f, q[i]))), -127.0f), 127.0f) + 0.0f;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) c[i] = q8_code_rf(x[i], d, r);
+  }
+}
+
+template <int N>
+TP_DEV void q8_roundtrip_each(float* p, const float* d) {
+  bool near = false;
+  float r[N], q[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    r[i] = q8_recip(d[i]);
+    q[i] = __fmul_rn(p[i], r[i]);
+    const float a = fabsf(q[i]);
+    near |= !(r[i] != 0.f) || fabsf(a - truncf(a) - 0.5f) < 4e-5f;
+  }
+  if (!near) {
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      p[i] = __fmul_rn(
+          fminf(fmaxf(truncf(__fadd_rn(q[i], copysignf(0.5f, q[i]))), -127.0f), 127.0f) + 0.0f, d[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) p[i] = __fmul_rn(q8_code_rf(p[i], d[i], r[i]), d[i]);
+  }
+}
+
 // Quantise-dequantise of 4 consecutive values held by each of 8 consecutive
 // lanes (one 32-value block per 8-lane group). All 32 lanes must call it.
 TP_DEV void q8_roundtrip4(float4& v) {
@@ -160,10 +214,11 @@ TP_DEV uint32_t q8_quantize4(float4 v, float* scale_out /* nullable */) {
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
   const float d = q8_scale(a), r = q8_recip(d);
   if (scale_out && (threadIdx.x & 7) == 0) *scale_out = d;
-  const uint32_t c0 = (uint32_t)((int)q8_code_rf(v.x, d, r) & 0xFF);
-  const uint32_t c1 = (uint32_t)((int)q8_code_rf(v.y, d, r) & 0xFF);
-  const uint32_t c2 = (uint32_t)((int)q8_code_rf(v.z, d, r) & 0xFF);
-  const uint32_t c3 = (uint32_t)((int)q8_code_rf(v.w, d, r) & 0xFF);
+  const float xs[4] = {v.x, v.y, v.z, v.w};
+  float cf[4];
+  q8_codes<4>(xs, cf, d, r);
+  const uint32_t c0 = (uint32_t)((int)cf[0] & 0xFF), c1 = (uint32_t)((int)cf[1] & 0xFF);
+  const uint32_t c2 = (uint32_t)((int)cf[2] & 0xFF), c3 = (uint32_t)((int)cf[3] & 0xFF);
   return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
 }
 

@@ -55,7 +55,10 @@ __global__ void __launch_bounds__(kRowThreads) k_norm_rows(NormRowsArgs a) {
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
       const float d = q8_scale(am);
-      const int c0 = q8_code(y.x, d), c1 = q8_code(y.y, d), c2 = q8_code(y.z, d), c3 = q8_code(y.w, d);
+      const float yv[4] = {y.x, y.y, y.z, y.w};
+      float cf[4];
+      q8_codes<4>(yv, cf, d, q8_recip(d));
+      const int c0 = (int)cf[0], c1 = (int)cf[1], c2 = (int)cf[2], c3 = (int)cf[3];
       if (in) {
         if (a.xq)
           *reinterpret_cast<uint32_t*>(a.xq + e) = (uint32_t)(c0 & 0xFF) | ((uint32_t)(c1 & 0xFF) << 8) |

@@ -345,8 +345,10 @@ __global__ void __launch_bounds__(tc_threads(EW), 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(p[j]));
             const float d = q8_scale(am), r = q8_recip(d);
+            q8_codes<16>(p, p, d, r);  // the block's codes in place, 16 at a time
+            q8_codes<16>(p + 16, p + 16, d, r);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) p[j] = __fmul_rn(q8_code_rf(p[j], d, r), d);
+            for (int j = 0; j < 32; ++j) p[j] = __fmul_rn(p[j], d);
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) run[32 * h + j] += p[j];

@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       const size_t col0 = (size_t)seg * a.Ks;
       const int nvr = (nv + 31) & ~31;
       consumers_sync(ncons);
+      if (a.probe && threadIdx.x == 0) a.probe[(size_t)blockIdx.x * a.trace_stride + 0] = gtimer();
       // one 8-value vector v of batch row b (x, g: the preloaded values when have_pre)
       auto stage = [&](int b, int v, bool have_pre, float4 px0, float4 px1, float4 pg0,
                        float4 pg1) {
@@ -352,13 +353,15 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
               am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
               am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
               qd = q8_scale(am);
+              float cf[8];
+              q8_codes<8>(xv, cf, qd, q8_recip(qd));
               qc = make_uint2(0u, 0u);
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const int c = q8_code(xv[e], qd);
-                xv[e] = q8_value(c, qd);
-                if (e < 4) qc.x |= (uint32_t)(c & 0xFF) << (8 * e);
-                else qc.y |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
+                xv[e] = __fmul_rn(cf[e], qd);
+                const uint32_t c = (uint32_t)((int)cf[e] & 0xFF);
+                if (e < 4) qc.x |= c << (8 * e);
+                else qc.y |= c << (8 * (e - 4));
               }
               if (a.gain && publish && in && a.xq_out) {
                 *reinterpret_cast<uint2*>(a.xq_out + e0) = qc;
@@ -376,15 +379,18 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
             const float d = q8_scale(am);
-            uint32_t lo = 0, hi = 0;
+            float cf[8];  // the codes as integral floats; integers only where they are stored
+            q8_codes<8>(xv, cf, d, q8_recip(d));
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int c = q8_code(xv[e], d);
-              xv[e] = q8_value(c, d);
-              if (e < 4) lo |= (uint32_t)(c & 0xFF) << (8 * e);
-              else hi |= (uint32_t)(c & 0xFF) << (8 * (e - 4));
-            }
+            for (int e = 0; e < 8; ++e) xv[e] = __fmul_rn(cf[e], d);
             if (publish && in && a.xq_out) {
+              uint32_t lo = 0, hi = 0;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const uint32_t c = (uint32_t)((int)cf[e] & 0xFF);
+                if (e < 4) lo |= c << (8 * e);
+                else hi |= c << (8 * (e - 4));
+              }
               *reinterpret_cast<uint2*>(a.xq_out + e0) = make_uint2(lo, hi);
               if ((lane & 3) == 0) a.xd_out[e0 / kQ8Block] = d;
             }
@@ -406,6 +412,8 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
                 k == 0 ? pg[0][0] : pg[1][0], k == 0 ? pg[0][1] : pg[1][1]);
         }
       }
+      if (a.probe && threadIdx.x == 0) a.probe[(size_t)blockIdx.x * a.trace_stride + 1] = gtimer();
+      if (a.probe && threadIdx.x == 32 * 7) a.probe[(size_t)blockIdx.x * a.trace_stride + 2] = gtimer();
       consumers_sync(ncons);
     };
 

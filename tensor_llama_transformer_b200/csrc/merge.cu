@@ -34,13 +34,12 @@ TP_DEV void chunk_ssq(float v, float* ssq_out) {
   }
 }
 
-// The Q8 round trip of one value per lane, the 32 lanes of the warp being one block.
-TP_DEV float q8_roundtrip1(float p) {
-  const float d = q8_scale(warp_max(fabsf(p)));
-  return __fmul_rn(q8_code_rf(p, d, q8_recip(d)), d);
-}
-
-__global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
+// CAP: at most 32 registers a thread (16 CTAs per SM), for grids too large to be resident
+// in one wave at the uncapped count (40 registers, 12 CTAs per SM): the 2048 CTAs of a
+// 70B-shaped batch-32 merge (dim 8192) took two waves and the step 12 us more; the capped
+// form costs the 32-CTA single-token merge about 0.6 us (spilled state of the Q8 path).
+template <bool CAP>
+__global__ void __launch_bounds__(kMergeThreads, CAP ? 16 : 1) k_merge(float* __restrict__ x,
                                                       const float* __restrict__ part, int n,
                                                       int parts, int B, int dim, int quant,
                                                       float* __restrict__ ssq, MergeTrace tr) {
@@ -69,9 +68,18 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(float* __restrict__ x,
       for (int k = 0; k < parts && s0 + j < n; ++k)
         p[j] += __ldcg(part + (size_t)((s0 + j) * parts + k) * stride + i);
     }
+    if (quant) {  // each slice's value through the Q8 round trip of its block (a warp)
+#pragma unroll
+      for (int h = 0; h < 4; h += 2) {  // two slices per branch (register pressure)
+        float d[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) d[j] = s0 + h + j < n ? q8_scale(warp_max(fabsf(p[h + j]))) : 1.f;
+        q8_roundtrip_each<2>(p + h, d);
+      }
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      if (s0 + j < n) acc += quant ? q8_roundtrip1(p[j]) : p[j];
+      if (s0 + j < n) acc += p[j];
     }
   }
   const float v = x0 + acc;
@@ -169,8 +177,12 @@ int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
                  cudaStream_t s, int parts, MergeTrace trace) {
   if (parts < 1 || parts > 2 || dim % 128 != 0) return TP_EINVAL;
-  return launch_pdl(k_merge, dim3((dim >> 7) * B), dim3(kMergeThreads), 0, s, x, part, n, parts, B,
-                    dim, quant, ssq, trace);
+  const int grid = (dim >> 7) * B;
+  if (grid > 12 * num_sms())
+    return launch_pdl(k_merge<true>, dim3(grid), dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim,
+                      quant, ssq, trace);
+  return launch_pdl(k_merge<false>, dim3(grid), dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim,
+                    quant, ssq, trace);
 }
 
 int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
