@@ -342,9 +342,7 @@ def gemv_timeline(torch, tpb, h, fwd, local):
     marks = ("start", "prev_done", "norm", "staged", "first_stage", "consumed", "end")
     merge_marks = ("start", "prev_done", "end")
     for name, c0, mk in (("qkv", 0, marks), ("wo", 7, marks), ("merge_wo", 28, merge_marks),
-                         ("w13", 14, marks), ("w2", 21, marks), ("merge_w2", 31, merge_marks),
-                         ("probe_qkv", 34, ("loop_start", "loop_end_w0", "loop_end_w7")),
-                         ("probe_w13", 37, ("loop_start", "loop_end_w0", "loop_end_w7"))):
+                         ("w13", 14, marks), ("w2", 21, marks), ("merge_w2", 31, merge_marks)):
         cols = t[:, c0:c0 + len(mk)]
         cols = cols[cols[:, 0] > 0]
         if not len(cols):

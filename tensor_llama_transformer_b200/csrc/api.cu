@@ -310,7 +310,6 @@ void set_gemv_trace(const tp_block* blk, GemvArgs& a, int g) {
   if (!blk->trace) return;
   a.trace = blk->trace + 7 * g;
   a.trace_stride = TP_BLOCK_TRACE_SLOTS;
-  if (g == 0 || g == 2) a.probe = blk->trace + 34 + 3 * (g / 2);
 }
 
 // End of a rank block's phase 0 / 1: this rank's partials into its send buffer.

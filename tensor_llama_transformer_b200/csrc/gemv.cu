@@ -236,7 +236,6 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
       const size_t col0 = (size_t)seg * a.Ks;
       const int nvr = (nv + 31) & ~31;
       consumers_sync(ncons);
-      if (a.probe && threadIdx.x == 0) a.probe[(size_t)blockIdx.x * a.trace_stride + 0] = gtimer();
       // one 8-value vector v of batch row b (x, g: the preloaded values when have_pre)
       auto stage = [&](int b, int v, bool have_pre, float4 px0, float4 px1, float4 pg0,
                        float4 pg1) {
@@ -412,8 +411,6 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
                 k == 0 ? pg[0][0] : pg[1][0], k == 0 ? pg[0][1] : pg[1][1]);
         }
       }
-      if (a.probe && threadIdx.x == 0) a.probe[(size_t)blockIdx.x * a.trace_stride + 1] = gtimer();
-      if (a.probe && threadIdx.x == 32 * 7) a.probe[(size_t)blockIdx.x * a.trace_stride + 2] = gtimer();
       consumers_sync(ncons);
     };
 

@@ -97,7 +97,6 @@ struct GemvArgs {
   // staged, 4 first ring stage arrived, 5 last ring stage consumed, 6 end
   unsigned long long* trace;
   int trace_stride;
-  unsigned long long* probe;  // (temporary) CTA 0's staging stamps
   int* err;  // device error flag, set when a bounded wait gives up (nullable)
 };
 
