@@ -240,9 +240,9 @@ def barrier(world: int):
 
 
 # DRAM bytes (read + write) of one launch of the W1/W3 slice GEMV in the C2 block,
-# from an ncu capture of that launch (180.450048 MB read + 3.141632 MB written):
+# from an ncu capture of that launch (180.448768 MB read + 3.624192 MB written):
 # the weights once, plus the activations and the SwiGLU output.
-W13_DRAM_BYTES = 180450048 + 3141632
+W13_DRAM_BYTES = 180448768 + 3624192
 
 
 def block_bytes(s):
@@ -467,7 +467,27 @@ def bench_block(args, world, rank, local):
         fwd()
         outh.copy_(dev.x, non_blocking=True)
         stream.synchronize()
+    e2e_eager_s = allreduce_max(time.perf_counter() - t0, world)
+    # the same step as a serving loop runs it: one CUDA graph per step holding the copy of
+    # the step's inputs from the pinned host buffers, the block forward (the same entry
+    # point, captured) and the copy of the result back to pinned host memory; the host
+    # waits for each step's result before the next replay
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e):
+        dev.x.copy_(xh, non_blocking=True)
+        dev.pos.copy_(posh, non_blocking=True)
+        fwd()
+        outh.copy_(dev.x, non_blocking=True)
+    for _ in range(3):
+        g_e2e.replay()
+        stream.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(E):
+        g_e2e.replay()
+        torch.cuda.current_stream().synchronize()
     e2e_s = allreduce_max(time.perf_counter() - t0, world)
+    del g_e2e
     tpb.tp_block_destroy(h)
 
     wbytes, kvbytes = block_bytes(s)
@@ -490,7 +510,12 @@ def bench_block(args, world, rank, local):
                      "kernel": "k_gemv<1, EPI_SWIGLU, false, 1> (RMSNorm+Q8, W1/W3, SwiGLU)",
                      "algorithmic_bytes": w13_bytes, "peak_kind": peak_kind},
         "e2e": {"value": world * B * E / e2e_s, "unit": "tokens/s",
-                "h2d_bytes_per_step": B * s.dim * 4 + B * 4, "d2h_bytes_per_step": B * s.dim * 4},
+                "h2d_bytes_per_step": B * s.dim * 4 + B * 4, "d2h_bytes_per_step": B * s.dim * 4,
+                "how": "per step one CUDA graph replay: copy of x and pos from pinned host memory, "
+                       "tp_block_forward, copy of x back to pinned host memory; host waits for "
+                       "every step's result",
+                "eager_value": world * B * E / e2e_eager_s,
+                "eager_how": "the same copies and tp_block_forward called from Python every step"},
         "gpu_launches": launches_per_step * K, "clocks": clk, "inp": inp,
         "gemv_timeline_us": timeline,
         "stage_sum_us": sum(stage_ms_max) * 1e3,
