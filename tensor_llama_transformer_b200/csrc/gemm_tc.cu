@@ -63,15 +63,6 @@ struct TcCfg {
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
 };
 
-// 3D tile load: coordinates {k within the segment, segment, row}.
-TP_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int seg, int row, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4}], [%5];" ::"r"(s2u(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(seg), "r"(row), "r"(s2u(bar))
-      : "memory");
-}
-
 TP_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 TP_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -518,6 +509,23 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int nseg, int64_t 
 }
 
 }  // namespace
+
+// A bf16 row-major matrix [rows, ld] as a 3D tensor {chunk, ld / chunk, rows} (its own
+// memory order, no swizzle), box {chunk, nchunk, box_rows}: one box is box_rows
+// consecutive rows of nchunk * chunk columns, landing in shared memory row-major
+// (rows of nchunk * chunk elements, nothing between them). Zero fill outside.
+bool make_tensor_map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t ld, int chunk,
+                          int nchunk, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || ld % chunk != 0) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)chunk, (cuuint64_t)(ld / chunk), (cuuint64_t)rows};
+  cuuint64_t gstride[2] = {(cuuint64_t)chunk * 2, (cuuint64_t)ld * 2};
+  cuuint32_t box[3] = {(cuuint32_t)chunk, (cuuint32_t)nchunk, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 // 2D map over a bf16 row-major matrix [rows, cols] (row stride ld elements),
 // box = box_cols x box_rows with the 128-byte swizzle, zero fill outside.

@@ -38,6 +38,7 @@
 // (llamaMultiheadAtt's "merge kv-cache, add RoPE encoding").
 #include <cstdlib>
 
+#include "gemm_tc.cuh"
 #include "kernels.cuh"
 #include "pipeline.cuh"
 
@@ -98,10 +99,20 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
                               const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
                               int part, int Q, int cb, int ce, int lane);
 
+// The weight tensor map of the row-split kernels that read through one (MAP); the
+// other kernels take an empty parameter, so their launches carry no descriptor.
+template <bool MAP>
+struct WeightMap {
+  CUtensorMap m;
+};
+template <>
+struct WeightMap<false> {};
+
 // PW: row pairs per consumer warp and stage (GemvPlan::pw), a template parameter so
 // that each kernel's streaming loop holds only the dot-product variant it runs
-template <int NB, int EPI, bool WQ8, int PW>
-__global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
+template <int NB, int EPI, bool WQ8, int PW, bool MAP = false>
+__global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl,
+                                                  const __grid_constant__ WeightMap<MAP> wmap) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_rstd[NB];
   __shared__ float s_red[8][NB];
@@ -144,6 +155,10 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
     // the RMSNorm gain (a constant input: no wait) into L2 before the weights, for the
     // consumers' prologue
     if (a.gain && lane == 0) bulk_prefetch_l2(a.gain, (uint32_t)a.ldx * 4);
+    if constexpr (MAP) {  // the weight map's descriptor, early
+      if (lane == 0)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap.m)) : "memory");
+    }
     if (WQ8 || lane == 0) {
       const uint64_t pol = l2_evict_first();  // weights are read once per step
       int t = 0;
@@ -184,6 +199,17 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl) {
             bulk_g2s_hint(dst + (size_t)i * slot + row_bytes,
                           reinterpret_cast<const uint8_t*>(a.wd[mat]) + slo, sl, &full[s], pol);
           }
+          cur = end;
+          continue;
+        }
+        if constexpr (MAP) {
+          // whole boxes of map_box rows (a short last box reads a few rows past the
+          // CTA's range, or zeros past the matrix; the stage holds them)
+          const int nbox = (n + pl.map_box - 1) / pl.map_box;
+          mbar_expect_tx(&full[s], (uint32_t)(nbox * pl.map_box) * row_bytes);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_3d_hint(dst + (size_t)i * pl.map_box * row_bytes, &wmap.m, 0,
+                             seg * pl.map_nchunk, lr0 + i * pl.map_box, &full[s], pol);
           cur = end;
           continue;
         }
@@ -686,9 +712,39 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   const int cta_rows = 2 * ((npairs + grid - 1) / grid);
   GemvPlan pl;
   if (!make_plan(NB, a.Ks, cta_rows, WQ8, &pl)) return TP_ENOTSUP;
+  // Row-split bf16 weights (W_O, W2) with segments under 2 KB a row: one bulk copy per
+  // row is bound by the copy unit's request rate (about 22 M copies/s per SM: 1 KB rows
+  // streamed at 3.2 TB/s, 2 KB rows at 6.5); a 3D tensor map moves 8 rows per request
+  // (W_O of the 7B block over 8 slices: 10.5 -> 5.9 us). From 2 KB on, bulk copies keep
+  // up and the map only delays the first stage (measured +1.5 us per step at 2 KB).
+  WeightMap<true> wmap{};
+  pl.map_box = 0;
+  pl.map_nchunk = 0;
+  if (EPI == EPI_PLAIN && !WQ8 && a.nseg > 1 && a.ldw != a.Ks && a.Ks * 2 < 2048 &&
+      2 * pl.pairs >= 8) {
+    int chunk = 0;
+    for (int c : {256, 128, 64, 32, 16, 8})
+      if (a.Ks % c == 0 && a.ldw % c == 0 && a.Ks / c <= 256) {
+        chunk = c;
+        break;
+      }
+    if (chunk && make_tensor_map_rows(&wmap.m, a.w[0], (uint64_t)a.rows[0], (uint64_t)a.ldw, chunk,
+                                      a.Ks / chunk, 8)) {
+      pl.map_box = 8;
+      pl.map_nchunk = a.Ks / chunk;
+    }
+  }
+  const dim3 block(32 * (pl.nc + 1));
+  if constexpr (EPI == EPI_PLAIN && !WQ8) {
+    if (pl.map_box) {
+      auto kernel = pl.pw == 2 ? k_gemv<NB, EPI, WQ8, 2, true> : k_gemv<NB, EPI, WQ8, 1, true>;
+      if (set_smem_once((const void*)kernel, (int)pl.total)) return TP_ECUDA;
+      return launch_pdl(kernel, dim3(grid), block, pl.total, s, a, pl, wmap);
+    }
+  }
   auto kernel = pl.pw == 2 ? k_gemv<NB, EPI, WQ8, 2> : k_gemv<NB, EPI, WQ8, 1>;
   if (set_smem_once((const void*)kernel, (int)pl.total)) return TP_ECUDA;
-  return launch_pdl(kernel, dim3(grid), dim3(32 * (pl.nc + 1)), pl.total, s, a, pl);
+  return launch_pdl(kernel, dim3(grid), block, pl.total, s, a, pl, WeightMap<false>{});
 }
 
 template <int NB, bool WQ8>

@@ -112,6 +112,10 @@ struct GemvPlan {
   int pw;  // row pairs per warp and stage (2 with 16 pairs per stage)
   int nstage;
   int cta_rows;
+  // row-split bf16 weights read through a 3D tensor map (the kernel's wmap): boxes of
+  // map_box consecutive rows of one segment (map_nchunk chunks of the map's inner
+  // width), one TMA per box instead of one bulk copy per row; 0: bulk copies
+  int map_box, map_nchunk;
   size_t ring_off, x_off, res_off, bar_off, total;
 };
 

@@ -111,6 +111,25 @@ TP_DEV void tma_load_2d_hint(void* dst, const CUtensorMap* map, int x, int y, ui
       : "memory");
 }
 
+// One box of a 3D tensor map at element coordinates (x, y, z) -> shared memory.
+TP_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4}], [%5];" ::"r"(s2u(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(s2u(bar))
+      : "memory");
+}
+
+// tma_load_3d with an L2 cache policy.
+TP_DEV void tma_load_3d_hint(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar,
+                             uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(s2u(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(s2u(bar)), "l"(pol)
+      : "memory");
+}
+
 // Named barrier 1 among the consumer warps of a warp-specialised CTA.
 TP_DEV void consumers_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
