@@ -510,19 +510,21 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int nseg, int64_t 
 
 }  // namespace
 
-// A bf16 row-major matrix [rows, ld] as a 3D tensor {chunk, ld / chunk, rows} (its own
+// A row-major matrix [rows, ld] of esize-byte elements (bf16, or int8 codes) as a 3D
+// tensor {chunk, ld / chunk, rows} (its own
 // memory order, no swizzle), box {chunk, nchunk, box_rows}: one box is box_rows
 // consecutive rows of nchunk * chunk columns, landing in shared memory row-major
 // (rows of nchunk * chunk elements, nothing between them). Zero fill outside.
 bool make_tensor_map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t ld, int chunk,
-                          int nchunk, int box_rows) {
+                          int nchunk, int box_rows, int esize) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc || ld % chunk != 0) return false;
+  if (!enc || ld % chunk != 0 || (esize != 1 && esize != 2)) return false;
   cuuint64_t gdim[3] = {(cuuint64_t)chunk, (cuuint64_t)(ld / chunk), (cuuint64_t)rows};
-  cuuint64_t gstride[2] = {(cuuint64_t)chunk * 2, (cuuint64_t)ld * 2};
+  cuuint64_t gstride[2] = {(cuuint64_t)chunk * esize, (cuuint64_t)ld * esize};
   cuuint32_t box[3] = {(cuuint32_t)chunk, (cuuint32_t)nchunk, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box,
+  return enc(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(base), gdim, gstride, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -59,10 +59,11 @@ int launch_tc_gemm(const TcGemm& g, cudaStream_t s);
 // elements: box box_cols x box_rows, 128-byte swizzle, zero fill past the edges.
 bool make_tensor_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                         uint64_t ld, int box_cols, int box_rows);
-// 3D map over a bf16 row-major matrix [rows, ld] viewed as {chunk, ld / chunk, rows}
-// (no swizzle): a box of box_rows consecutive rows of nchunk * chunk columns lands in
-// shared memory row-major. ld % chunk == 0; chunk, nchunk, box_rows <= 256.
+// 3D map over a row-major matrix [rows, ld] of esize-byte elements (2: bf16, 1: int8)
+// viewed as {chunk, ld / chunk, rows} (no swizzle): a box of box_rows consecutive rows
+// of nchunk * chunk columns lands in shared memory row-major. ld % chunk == 0; chunk,
+// nchunk, box_rows <= 256; chunk * esize a multiple of 16.
 bool make_tensor_map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t ld, int chunk,
-                          int nchunk, int box_rows);
+                          int nchunk, int box_rows, int esize);
 
 }  // namespace tp

@@ -95,9 +95,9 @@ inline __host__ __device__ uint32_t q8w_scale_slot(int Ks) {
 }
 
 template <int NB, int PW>
-TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pad, int cur, int end,
-                              const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
-                              int part, int Q, int cb, int ce, int lane);
+TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t cstride, uint32_t soff, uint32_t sstride,
+                              const int* pad, int cur, int end, const int8_t* xsq, const float* xsd,
+                              float* res, int Ks, int pw, int part, int Q, int cb, int ce, int lane);
 
 // The weight tensor map of the row-split kernels that read through one (MAP); the
 // other kernels take an empty parameter, so their launches carry no descriptor.
@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl,
         const int n = end - cur;
         const size_t col0 = (size_t)seg * a.Ks;
         if constexpr (WQ8) {
-          // per row: its codes, then the aligned run covering its scales
+          // per row: its codes, then the aligned run covering its scales; with the weight
+          // map, the stage's codes in boxes of map_box rows (first, dense) and the rows'
+          // scale runs after them
           const size_t sstride = (size_t)(a.ldw / 32) * 4, sseg = (size_t)seg * (a.Ks / 32) * 4;
           const uint32_t sbytes = (uint32_t)(a.Ks / 32) * 4;
           uint32_t tx = 0;
@@ -184,20 +186,32 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl,
             int mat, lrow;
             row_ptr<EPI>(a, seg, lr0 + i, mat, lrow);
             const size_t s0 = (size_t)lrow * sstride + sseg;
-            tx += row_bytes + (uint32_t)(((s0 + sbytes + 15) & ~(size_t)15) - (s0 & ~(size_t)15));
+            tx += (MAP ? 0u : row_bytes) +
+                  (uint32_t)(((s0 + sbytes + 15) & ~(size_t)15) - (s0 & ~(size_t)15));
           }
           tx = __reduce_add_sync(0xffffffffu, tx);
-          if (lane == 0) mbar_expect_tx(&full[s], tx);
+          const int nbox = MAP ? (n + pl.map_box - 1) / pl.map_box : 0;
+          if (lane == 0) mbar_expect_tx(&full[s], tx + (uint32_t)(nbox * pl.map_box) * row_bytes);
           __syncwarp();
+          if constexpr (MAP) {
+            if (lane == 0)
+              for (int k = 0; k < nbox; ++k)
+                tma_load_3d_hint(dst + (size_t)k * pl.map_box * row_bytes, &wmap.m, 0,
+                                 seg * pl.map_nchunk, lr0 + k * pl.map_box, &full[s], pol);
+          }
+          uint8_t* sdst = MAP ? dst + (size_t)2 * P * row_bytes : dst + row_bytes;
+          const uint32_t sstep = MAP ? slot - row_bytes : slot;
           for (int i = lane; i < n; i += 32) {
             int mat, lrow;
             row_ptr<EPI>(a, seg, lr0 + i, mat, lrow);
-            const int8_t* src = reinterpret_cast<const int8_t*>(a.w[mat]) + (size_t)lrow * a.ldw + col0;
-            bulk_g2s_hint(dst + (size_t)i * slot, src, row_bytes, &full[s], pol);
+            if (!MAP) {
+              const int8_t* src = reinterpret_cast<const int8_t*>(a.w[mat]) + (size_t)lrow * a.ldw + col0;
+              bulk_g2s_hint(dst + (size_t)i * slot, src, row_bytes, &full[s], pol);
+            }
             const size_t s0 = (size_t)lrow * sstride + sseg, slo = s0 & ~(size_t)15;
             const uint32_t sl = (uint32_t)(((s0 + sbytes + 15) & ~(size_t)15) - slo);
-            bulk_g2s_hint(dst + (size_t)i * slot + row_bytes,
-                          reinterpret_cast<const uint8_t*>(a.wd[mat]) + slo, sl, &full[s], pol);
+            bulk_g2s_hint(sdst + (size_t)i * sstep, reinterpret_cast<const uint8_t*>(a.wd[mat]) + slo, sl,
+                          &full[s], pol);
           }
           cur = end;
           continue;
@@ -539,7 +553,14 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl,
               pad[i] = ((lr & 3) * s32 + segpad) & 3;
             }
             const int nc16 = a.Ks >> 4, cb = (nc16 * part) / Q, ce = (nc16 * (part + 1)) / Q;
-            ring_pairs_dot_q8<NB, PW>(st, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+            // rows as [codes | scale run] slots, or with the weight map all codes of the
+            // stage first (dense rows of Ks), then the scale runs
+            if constexpr (MAP)
+              ring_pairs_dot_q8<NB, PW>(st, (uint32_t)a.Ks, (uint32_t)(2 * P * a.Ks), slot - (uint32_t)a.Ks,
+                                        pad, cur, end, xsq, xsd, res, a.Ks, pw, part, Q, cb, ce, lane);
+            else
+              ring_pairs_dot_q8<NB, PW>(st, slot, row_bytes, slot, pad, cur, end, xsq, xsd, res, a.Ks, pw,
+                                        part, Q, cb, ce, lane);
           } else {
             ring_pairs_dot<NB, PW>(st, cur, end, xs, res, nv, row_bytes, pw, part, Q, vb, ve, lane);
           }
@@ -611,9 +632,9 @@ __global__ void __launch_bounds__(288, 1) k_gemv(GemvArgs a, GemvPlan pl,
 // d_w d_x of its 32-value block and accumulated in float32. pad[i] is the offset
 // (floats) of row i's scales inside its aligned run in the stage.
 template <int NB, int PW>
-TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pad, int cur, int end,
-                              const int8_t* xsq, const float* xsd, float* res, int Ks, int pw,
-                              int part, int Q, int cb, int ce, int lane) {
+TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t cstride, uint32_t soff, uint32_t sstride,
+                              const int* pad, int cur, int end, const int8_t* xsq, const float* xsd,
+                              float* res, int Ks, int pw, int part, int Q, int cb, int ce, int lane) {
   constexpr int R = 2 * PW * NB;  // values: (pair j, row, batch row)
   int rr[PW];
   bool valid[PW];
@@ -641,9 +662,10 @@ TP_DEV void ring_pairs_dot_q8(const uint8_t* stage, uint32_t slot, const int* pa
       if (!valid[j]) continue;
 #pragma unroll
       for (int row = 0; row < 2; ++row) {
-        const uint8_t* rp = stage + (size_t)(rr[j] + row - cur) * slot;
-        const int4 wq = *reinterpret_cast<const int4*>(rp + 16 * c);
-        const float dw = reinterpret_cast<const float*>(rp + Ks)[pad[2 * j + row] + (c >> 1)];
+        const int lr = rr[j] + row - cur;  // row within the stage
+        const int4 wq = *reinterpret_cast<const int4*>(stage + (size_t)lr * cstride + 16 * c);
+        const float dw = reinterpret_cast<const float*>(stage + soff + (size_t)lr * sstride)
+            [pad[2 * j + row] + (c >> 1)];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           int sdot = __dp4a(wq.x, xq[b].x, 0);
@@ -720,22 +742,25 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   WeightMap<true> wmap{};
   pl.map_box = 0;
   pl.map_nchunk = 0;
-  if (EPI == EPI_PLAIN && !WQ8 && a.nseg > 1 && a.ldw != a.Ks && a.Ks * 2 < 2048 &&
+  // int8 rows take two bulk copies each (codes, scale run): the map carries the codes
+  // when those are under 4 KB a row (W_O and W2 of the 7B block over 4 slices)
+  const int esize = WQ8 ? 1 : 2;
+  if (EPI == EPI_PLAIN && a.nseg > 1 && a.ldw != a.Ks && a.Ks * esize < (WQ8 ? 4096 : 2048) &&
       2 * pl.pairs >= 8) {
     int chunk = 0;
     for (int c : {256, 128, 64, 32, 16, 8})
-      if (a.Ks % c == 0 && a.ldw % c == 0 && a.Ks / c <= 256) {
+      if (a.Ks % c == 0 && a.ldw % c == 0 && a.Ks / c <= 256 && c * esize >= 16) {
         chunk = c;
         break;
       }
     if (chunk && make_tensor_map_rows(&wmap.m, a.w[0], (uint64_t)a.rows[0], (uint64_t)a.ldw, chunk,
-                                      a.Ks / chunk, 8)) {
+                                      a.Ks / chunk, 8, esize)) {
       pl.map_box = 8;
       pl.map_nchunk = a.Ks / chunk;
     }
   }
   const dim3 block(32 * (pl.nc + 1));
-  if constexpr (EPI == EPI_PLAIN && !WQ8) {
+  if constexpr (EPI == EPI_PLAIN) {
     if (pl.map_box) {
       auto kernel = pl.pw == 2 ? k_gemv<NB, EPI, WQ8, 2, true> : k_gemv<NB, EPI, WQ8, 1, true>;
       if (set_smem_once((const void*)kernel, (int)pl.total)) return TP_ECUDA;
