@@ -1083,8 +1083,8 @@ def main(argv=None):
                                   "consumed, end",
             "stage_note": "per-stage CUDA-event times from a replay of the same steps with an event "
                           "before every stage (serialised, so upper bounds); value and ms_per_step "
-                          "come from the event-free graph; the merges run in the W_O and W2 "
-                          "GEMVs' epilogues, so their own stages hold no kernel",
+                          "come from the event-free graph; each merge stage is one k_merge "
+                          "launch (the slices' partials into the residual)",
             "pdl": os.environ.get("TP_PDL", "1") != "0",
             "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
