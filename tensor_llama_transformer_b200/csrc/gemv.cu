@@ -47,7 +47,14 @@ namespace tp {
 namespace {
 
 constexpr int kMaxStages = 16;
+// Dynamic shared memory of a GEMV CTA. bf16: 222 KB, which leaves room on the SM for a
+// merge CTA beside the row-split GEMVs (152 registers). int8 weights: 223 KB, which fits
+// 3 stages of 8 row pairs for the 7B W1/W3 rows (4 KB of codes + their scales; 5,504
+// bytes of activations, partial sums and barriers): 8 pairs per stage instead of 4,
+// one consumer warp per pair. Its kernels take 158 registers or more, so a merge CTA
+// never fits beside them anyway.
 constexpr int kSmemBudget = 222 * 1024;
+constexpr int kSmemBudgetQ8 = 223 * 1024;
 
 template <int EPI>
 TP_DEV int rows_per_seg(const GemvArgs& a) {
@@ -700,9 +707,10 @@ bool make_plan(int NB, int Ks, int cta_rows, bool wq8, GemvPlan* p) {
       const int Q = P >= 8 ? 1 : 8 / P;
       const size_t res_bytes = a128((size_t)cta_rows * NB * Q * 4);
       const size_t fixed = x_bytes + res_bytes + bar_bytes;
-      if (fixed >= (size_t)kSmemBudget) continue;
+      const size_t budget = wq8 ? kSmemBudgetQ8 : kSmemBudget;
+      if (fixed >= budget) continue;
       const size_t stage = 2 * (size_t)P * row_bytes;
-      int ns = (int)(((size_t)kSmemBudget - fixed) / stage);
+      int ns = (int)((budget - fixed) / stage);
       if (ns > kMaxStages) ns = kMaxStages;
       if (ns >= min_stages) {
         p->nc = 8;
