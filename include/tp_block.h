@@ -168,8 +168,11 @@ TP_API int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cach
  * and v are written before any row's attention runs, so row b attends to
  * positions 0..pos[b] of its sequence including the rows of this step below it:
  * a chunk gives what decoding its tokens one at a time gives. Rows sharing a
- * sequence must have distinct positions (not checked on device). Up to
- * max_batch rows per call (longer prompts run as successive chunks).
+ * sequence must have distinct positions (not checked on device). More than
+ * max_batch rows run as successive passes of max_batch rows, in row order: a row
+ * then also sees the k/v of its sequence's rows in earlier passes, so the rows of
+ * a sequence that spans passes must come in increasing position order (a prompt
+ * of any length in one call; not checked on device).
  * Errors: TP_EINVAL (also for a rank handle), TP_EALIGN, TP_ECUDA, TP_ENOTSUP. */
 TP_API int tp_block_forward_seq(tp_block* blk, float* x, void* k_cache, void* v_cache,
                                 const int32_t* pos, const int32_t* seq, int n_seq, int batch,
@@ -401,7 +404,10 @@ TP_API int tp_model_create(const tp_dims* dims, int n_layers, int n_slices, int 
 /* tokens device int32 [batch] in [0, vocab); caches bf16
  * [n_layers, max_batch, Hkv, max_seq, hd]; logits float32 [batch, vocab] written. */
 /* tp_model_forward with rows mapped to cache sequences (see tp_block_forward_seq):
- * caches bf16 [n_layers, n_seq, Hkv, max_seq, hd]; logits of every row written. */
+ * caches bf16 [n_layers, n_seq, Hkv, max_seq, hd]; logits of every row written.
+ * More than max_batch rows: successive passes of max_batch rows through every
+ * layer, in row order (as tp_block_forward_seq); TP_EALIGN unless max_batch *
+ * vocab is a multiple of 4 (each pass's logits rows start 16-byte aligned). */
 TP_API int tp_model_forward_seq(tp_model* m, const int32_t* tokens, void* k_cache, void* v_cache,
                                 const int32_t* pos, const int32_t* seq, int n_seq, int batch,
                                 float* logits, tp_stream stream);

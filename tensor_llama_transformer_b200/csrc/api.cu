@@ -955,11 +955,19 @@ int tp_block_forward(tp_block* blk, float* x, void* k_cache, void* v_cache, cons
 int tp_block_forward_seq(tp_block* blk, float* x, void* k_cache, void* v_cache, const int32_t* pos,
                          const int32_t* seq, int n_seq, int batch, tp_stream stream) {
   if (!blk || !x || !k_cache || !v_cache || !pos || !seq || blk->c.world > 0) return TP_EINVAL;
-  if (batch < 1 || batch > blk->c.d.max_batch || n_seq < 1) return TP_EINVAL;
+  if (batch < 1 || n_seq < 1) return TP_EINVAL;
   if ((int64_t)n_seq * blk->c.d.n_kv_heads * blk->c.d.max_seq > INT32_MAX) return TP_EINVAL;
   if (!aligned16(x) || !aligned16(k_cache) || !aligned16(v_cache)) return TP_EALIGN;
-  return block_forward_impl(blk, x, k_cache, v_cache, pos, batch, (cudaStream_t)stream, false, -1,
-                            seq, n_seq);
+  // more rows than max_batch: successive passes of max_batch rows in row order (each
+  // pass's k/v are in the caches before the next pass's attention reads them)
+  const int mb = blk->c.d.max_batch;
+  for (int r0 = 0; r0 < batch; r0 += mb) {
+    const int nb = batch - r0 < mb ? batch - r0 : mb;
+    const int rc = block_forward_impl(blk, x + (size_t)r0 * blk->c.d.dim, k_cache, v_cache, pos + r0, nb,
+                                      (cudaStream_t)stream, false, -1, seq + r0, n_seq);
+    if (rc) return rc;
+  }
+  return TP_OK;
 }
 
 int tp_block_buffer(const tp_block* blk, int which, size_t* offset, size_t* bytes) {
@@ -1148,11 +1156,20 @@ int tp_model_forward_seq(tp_model* m, const int32_t* tokens, void* k_cache, void
                          const int32_t* pos, const int32_t* seq, int n_seq, int batch,
                          float* logits, tp_stream stream) {
   if (!m || !tokens || !k_cache || !v_cache || !pos || !seq || !logits) return TP_EINVAL;
-  if (batch < 1 || batch > m->d.max_batch || n_seq < 1) return TP_EINVAL;
+  if (batch < 1 || n_seq < 1) return TP_EINVAL;
   if ((int64_t)n_seq * m->d.n_kv_heads * m->d.max_seq > INT32_MAX) return TP_EINVAL;
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits)) return TP_EALIGN;
-  return model_forward_impl(m, tokens, k_cache, v_cache, pos, seq, n_seq, batch, logits,
-                            (cudaStream_t)stream);
+  // more rows than max_batch: successive passes of max_batch rows through every layer,
+  // in row order; each pass's logits rows start 16-byte aligned
+  const int mb = m->d.max_batch;
+  if (batch > mb && ((int64_t)mb * m->d.vocab) % 4 != 0) return TP_EALIGN;
+  for (int r0 = 0; r0 < batch; r0 += mb) {
+    const int nb = batch - r0 < mb ? batch - r0 : mb;
+    const int rc = model_forward_impl(m, tokens + r0, k_cache, v_cache, pos + r0, seq + r0, n_seq, nb,
+                                      logits + (size_t)r0 * m->d.vocab, (cudaStream_t)stream);
+    if (rc) return rc;
+  }
+  return TP_OK;
 }
 
 int tp_model_set_persistent(tp_model* m, int enable) {

@@ -7,7 +7,8 @@ attention, so each row attends causally. Checked against
 ``oracle.block_forward(seq=...)`` (itself pinned to token-by-token decode and to
 the masked-softmax form of causal attention), on the weight-streaming path
 (up to 5 rows) and the tensor-core path (6 or more), at the 7B block's shapes for
-a 64-token chunk, and through the model entry point.
+a 64-token chunk, and through the model entry point; prompts longer than the
+handle's max_batch run as successive passes inside one call.
 """
 import numpy as np
 import pytest
@@ -29,11 +30,12 @@ def tpb(cuda_ok):
     return t
 
 
-def run_seq(tpb, inp, n, quant):
+def run_seq(tpb, inp, n, quant, max_batch=None):
     s = inp.shape
     B = inp.x.shape[0]
-    dev = DeviceBlock(inp, max_batch=B)
-    dims = _dims(tpb, s, B)
+    mb = max_batch or B
+    dev = DeviceBlock(inp, max_batch=mb)
+    dims = _dims(tpb, s, mb)
     nbytes = tpb.tp_block_workspace_bytes(dims, n, 1, quant)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     h = tpb.tp_block_create(dims, n, 1, quant, tpb.make_weights(*dev.weights()), ws, nbytes)
@@ -114,6 +116,27 @@ def test_mixed_decode_and_prefill(tpb, seq, pos, quant):
     check_seq(tpb, inp, 2, quant, tight, f"mixed B{len(pos)} q{quant}")
 
 
+@pytest.mark.parametrize("quant", [0, 1])
+def test_prompt_longer_than_max_batch(tpb, quant):
+    """37 tokens of one sequence through a block built for 16 rows: passes of 16, 16 and 5
+    rows (tensor-core path, then the weight-streaming path), each attending to the cache
+    rows the earlier passes wrote."""
+    s = synth.BlockShape(**{**GQA.__dict__, "pos": 40})
+    L, mb = 37, 16
+    inp = synth.chunk_inputs(8585, s, 40 + np.arange(L), np.zeros(L, dtype=np.int32))
+    ref, k_ref, v_ref = oracle.block_forward(inp, 2, bool(quant), seq=inp.extra["seq"])
+    y, k_rows, v_rows, err, _ = run_seq(tpb, inp, 2, quant, max_batch=mb)
+    assert err == 0, "a bounded wait in a kernel gave up"
+    name = f"prompt L{L} in passes of {mb} q{quant}"
+    r_out, p_out = report(f"{name} out", y, ref)
+    r_dx, _ = report(f"{name} out-x", y - inp.x, ref - inp.x)
+    r_k, _ = report(f"{name} k@pos", oracle.bf16_to_f64(k_rows), oracle.bf16_to_f64(k_ref))
+    r_v, _ = report(f"{name} v@pos", oracle.bf16_to_f64(v_rows), oracle.bf16_to_f64(v_ref))
+    for r in (r_out, r_dx, r_k, r_v):
+        assert r <= BF16_TOL
+    assert max(r_out, r_dx) <= 1e-2 and p_out > 0.9999
+
+
 def test_prefill_chunk_equals_token_by_token(tpb):
     """The GPU's chunk against the GPU decoding the same tokens one per call."""
     s = synth.BlockShape(**{**GQA.__dict__, "pos": 30})
@@ -145,8 +168,10 @@ def test_prefill_chunk_c2_shapes(tpb):
     check_seq(tpb, inp, s.n_slices, 1, 1e-2, "prefill C2 L64")
 
 
-def test_model_prefill_chunk(tpb):
-    """tp_model_forward_seq: a 12-token chunk through 2 layers, embedding to logits."""
+@pytest.mark.parametrize("mb", [12, 5])
+def test_model_prefill_chunk(tpb, mb):
+    """tp_model_forward_seq: a 12-token chunk through 2 layers, embedding to logits; with
+    max_batch 5 the call runs as passes of 5, 5 and 2 rows through every layer."""
     s = synth.BlockShape(dim=512, n_heads=4, n_kv_heads=2, head_dim=128, ffn_dim=1024, vocab=1000,
                          max_seq=100, batch=1, n_slices=2, sync_quant=False, pos=40, w_std=0.05)
     L, n_layers, seed = 12, 2, 8484
@@ -176,7 +201,7 @@ def test_model_prefill_chunk(tpb):
 
     ref = oracle.model_forward(toks, emb, [make_layer(i) for i in range(n_layers)], np.ones(s.dim),
                                wcls, s.n_slices, False, s.norm_eps)
-    dims = tpb.make_dims(s.dim, s.n_heads, s.n_kv_heads, s.head_dim, s.ffn_dim, s.vocab, L,
+    dims = tpb.make_dims(s.dim, s.n_heads, s.n_kv_heads, s.head_dim, s.ffn_dim, s.vocab, mb,
                          s.max_seq, s.norm_eps, s.rope_theta)
     nbytes = tpb.tp_model_workspace_bytes(dims, n_layers, s.n_slices, 1, 0)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
