@@ -137,8 +137,10 @@ TP_API int tp_block_create(const tp_dims* dims, int n_slices, int partition, int
  * before W_O, the SwiGLU output before W2, each quantised in blocks of 32) and
  * runs as integer dot products per block scaled by d_w * d_x, accumulated in
  * float32. Requires partition TP_PART_1D, sync_quant = 1 and ffn_dim % 64 == 0.
- * tp_block_forward on such a handle takes batch <= 5 (the weight-streaming
- * path); larger batches return TP_ENOTSUP. Workspace as for tp_block_create.
+ * tp_block_forward on such a handle runs the weight-streaming kernels at every
+ * batch, 2 rows per launch: from 6 rows on (where bf16 handles switch to the
+ * tensor cores) the weights are read once per 2 rows. Workspace as for
+ * tp_block_create.
  * Errors: TP_EINVAL, TP_EALIGN, TP_EWORKSPACE, TP_EARCH, TP_ENOTSUP. */
 TP_API int tp_block_create_q8w(const tp_dims* dims, int n_slices, int partition, int sync_quant,
                                const tp_block_weights_q8* w, void* workspace, size_t ws_bytes,

@@ -565,13 +565,14 @@ int block_forward_persistent(tp_block* blk, float* x, void* kc, void* vc, const 
 int block_forward_impl(tp_block* blk, float* x, void* kc, void* vc, const int32_t* pos, int batch,
                        cudaStream_t s, bool chained = false, int phase = -1,
                        const int32_t* seq = nullptr, int nseq = 0) {
-  if (blk->wq8 && batch >= kTcMinBatch) return TP_ENOTSUP;
   if (!blk->bar_ready) {  // error word and counters start at zero (first use of the workspace)
     if (cudaMemsetAsync(blk->ws + blk->L.off[BUF_ERR], 0, blk->L.size[BUF_ERR], s) != cudaSuccess)
       return TP_ECUDA;
     blk->bar_ready = true;
   }
-  if (batch >= kTcMinBatch)
+  // batched decode on the tensor cores (bf16 weights); int8 weights stay on the
+  // weight-streaming kernels at every batch (2 rows per launch)
+  if (batch >= kTcMinBatch && !blk->wq8)
     return block_forward_tc(blk, x, kc, vc, pos, batch, s, chained, phase, seq, nseq);
   if (batch <= 2 && blk->c.partition == TP_PART_1D && !blk->events && blk->persistent &&
       blk->c.world == 0 && !seq) {

@@ -127,8 +127,14 @@ def test_q8w_c2_full_size(tpb):
     check_q8w(tpb, inp, synth.C2.n_slices, "q8w C2")
 
 
-def test_q8w_refuses_batched_path(tpb):
-    s = synth.BlockShape(**{**GQA.__dict__, "batch": 6})
-    inp = synth.block_inputs(3, s)
-    with pytest.raises(tpb.TpError):
-        run_block_q8w(tpb, inp, 2)
+@pytest.mark.parametrize("shape,n,pos", [
+    (GQA, 2, [259, 127, 0, 64, 63, 200]),              # batch 6: three launches of 2 rows
+    (MHA, 2, [299, 130, 0, 1, 2, 64, 65, 250, 128]),   # batch 9: four of 2 and one of 1
+])
+def test_q8w_batched(tpb, shape, n, pos):
+    """Batches from 6 rows on, where bf16 handles take the tensor cores: int8 weights stay on
+    the weight-streaming kernels, 2 rows per launch."""
+    s = synth.BlockShape(**{**shape.__dict__, "batch": len(pos)})
+    inp = synth.block_inputs(6262, s)
+    inp.pos[:] = pos
+    check_q8w(tpb, inp, n, f"q8w d{s.dim} n{n} B{len(pos)}", check_codes=True)
