@@ -69,12 +69,19 @@ __global__ void __launch_bounds__(kMergeThreads, CAP ? 16 : 1) k_merge(float* __
         p[j] += __ldcg(part + (size_t)((s0 + j) * parts + k) * stride + i);
     }
     if (quant) {  // each slice's value through the Q8 round trip of its block (a warp)
+      if constexpr (CAP) {
 #pragma unroll
-      for (int h = 0; h < 4; h += 2) {  // two slices per branch (register pressure)
-        float d[2];
+        for (int h = 0; h < 4; h += 2) {  // two slices per branch (32 registers)
+          float d[2];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) d[j] = s0 + h + j < n ? q8_scale(warp_max(fabsf(p[h + j]))) : 1.f;
-        q8_roundtrip_each<2>(p + h, d);
+          for (int j = 0; j < 2; ++j) d[j] = s0 + h + j < n ? q8_scale(warp_max(fabsf(p[h + j]))) : 1.f;
+          q8_roundtrip_each<2>(p + h, d);
+        }
+      } else {  // the four slices' chains side by side
+        float d[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d[j] = s0 + j < n ? q8_scale(warp_max(fabsf(p[j]))) : 1.f;
+        q8_roundtrip_each<4>(p, d);
       }
     }
 #pragma unroll
