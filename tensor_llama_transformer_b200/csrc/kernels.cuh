@@ -19,8 +19,10 @@ struct MergeTrace {
   unsigned long long* stamps;
   int stride, rows;
 };
+// late: the next kernel may launch only once every CTA's partials have been loaded
+// (its weight stream then does not compete with those loads); else at the start.
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts = 1, MergeTrace trace = MergeTrace{});
+                 cudaStream_t s, int parts = 1, MergeTrace trace = MergeTrace{}, int late = 0);
 inline int merge_ssq_parts(int dim) { return dim / 128; }
 // One slice's partial in the sync format for B rows: float32 [B, dim], or with Q8
 // the codes int8 [B, dim] followed by the scales float32 [B, dim/32].

@@ -42,8 +42,9 @@ template <bool CAP>
 __global__ void __launch_bounds__(kMergeThreads, CAP ? 16 : 1) k_merge(float* __restrict__ x,
                                                       const float* __restrict__ part, int n,
                                                       int parts, int B, int dim, int quant,
-                                                      float* __restrict__ ssq, MergeTrace tr) {
-  pdl_launch_dependents();
+                                                      float* __restrict__ ssq, MergeTrace tr,
+                                                      int late) {
+  if (!late) pdl_launch_dependents();
   unsigned long long* st =
       tr.stamps && threadIdx.x == 0 && (int)blockIdx.x < tr.rows ? tr.stamps + (size_t)blockIdx.x * tr.stride
                                                                  : nullptr;
@@ -67,6 +68,11 @@ __global__ void __launch_bounds__(kMergeThreads, CAP ? 16 : 1) k_merge(float* __
       p[j] = 0.f;
       for (int k = 0; k < parts && s0 + j < n; ++k)
         p[j] += __ldcg(part + (size_t)((s0 + j) * parts + k) * stride + i);
+    }
+    if (late && s0 == 0) {  // the next kernel launches once this CTA's partials are in
+      const float dep = x0 + p[0] + p[1] + p[2] + p[3];
+      asm volatile("" ::"f"(dep));
+      pdl_launch_dependents();
     }
     if (quant) {  // each slice's value through the Q8 round trip of its block (a warp)
       if constexpr (CAP) {
@@ -182,14 +188,14 @@ __global__ void k_dequantize(const int8_t* __restrict__ q, const float* __restri
 int merge_grid(int dim) { return (dim / 4 + kMergeThreads - 1) / kMergeThreads; }
 
 int launch_merge(float* x, const float* part, int n, int B, int dim, int quant, float* ssq,
-                 cudaStream_t s, int parts, MergeTrace trace) {
+                 cudaStream_t s, int parts, MergeTrace trace, int late) {
   if (parts < 1 || parts > 2 || dim % 128 != 0) return TP_EINVAL;
   const int grid = (dim >> 7) * B;
   if (grid > 12 * num_sms())
     return launch_pdl(k_merge<true>, dim3(grid), dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim,
-                      quant, ssq, trace);
+                      quant, ssq, trace, late);
   return launch_pdl(k_merge<false>, dim3(grid), dim3(kMergeThreads), 0, s, x, part, n, parts, B, dim,
-                    quant, ssq, trace);
+                    quant, ssq, trace, late);
 }
 
 int launch_sync_pack(const float* part, int n_local, int parts, int B, int dim, int quant,
