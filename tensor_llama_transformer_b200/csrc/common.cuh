@@ -169,6 +169,35 @@ TP_DEV void q8_codes(const float* x, float* c, float d, float r) {
   }
 }
 
+// q8_codes for G blocks at once (block g: x[g N .. g N + N - 1] with scale d[g] and
+// reciprocal r[g]), with one near flag over all of them, so that their chains can run
+// side by side; the codes are q8_code_rf's, bit for bit, as for q8_codes.
+template <int N, int G>
+TP_DEV void q8_codes_g(const float* x, float* c, const float* d, const float* r) {
+  bool near = false;
+  float q[G * N];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    near |= !(r[g] != 0.f);
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      q[g * N + i] = __fmul_rn(x[g * N + i], r[g]);
+      const float a = fabsf(q[g * N + i]);
+      near |= fabsf(a - truncf(a) - 0.5f) < 4e-5f;
+    }
+  }
+  if (!near) {
+#pragma unroll
+    for (int i = 0; i < G * N; ++i)
+      c[i] = fminf(fmaxf(truncf(__fadd_rn(q[i], copysignf(0.5f, q[i]))), -127.0f), 127.0f) + 0.0f;
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int i = 0; i < N; ++i) c[g * N + i] = q8_code_rf(x[g * N + i], d[g], r[g]);
+  }
+}
+
 template <int N>
 TP_DEV void q8_roundtrip_each(float* p, const float* d) {
   bool near = false;
