@@ -830,19 +830,27 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
   const int cta_rows = 2 * ((npairs + grid - 1) / grid);
   GemvPlan pl;
   if (!make_plan(NB, a.Ks, cta_rows, WQ8, &pl)) return TP_ENOTSUP;
-  // Row-split bf16 weights (W_O, W2) with segments under 2 KB a row: one bulk copy per
+  // Row-split bf16 weights (W_O, W2) with segments of up to 2 KB a row: one bulk copy per
   // row is bound by the copy unit's request rate (about 22 M copies/s per SM: 1 KB rows
-  // streamed at 3.2 TB/s, 2 KB rows at 6.5); a 3D tensor map moves 8 rows per request
-  // (W_O of the 7B block over 8 slices: 10.5 -> 5.9 us). From 2 KB on, bulk copies keep
-  // up and the map only delays the first stage (measured +1.5 us per step at 2 KB).
+  // streamed at 3.2 TB/s, 2 KB rows at 6.5, and W_O's 2 KB rows of the 7B block over 4
+  // slices at 3.7 in the step); a 3D tensor map moves several rows per request (W_O of the
+  // 7B block over 8 slices: 10.5 -> 5.9 us). Its boxes are 2 rows high: with 8, a
+  // stage's few large requests held back the W_O staging's loads of the attention splits
+  // (staging 3.1 -> 5.4 us, the 7B step over 4 slices +0.7 us), while 2-row boxes took
+  // 0.3 us off that step and 0.5 % off the 32-layer one against bulk copies and 8-row boxes.
   WeightMap<true> wmap{};
   pl.map_box = 0;
   pl.map_nchunk = 0;
   // int8 rows take two bulk copies each (codes, scale run): the map carries the codes
-  // when those are under 4 KB a row (W_O and W2 of the 7B block over 4 slices)
+  // when those are under 4 KB a row (W_O and W2 of the 7B block over 4 slices), in boxes
+  // of 8 rows (2 or 4 measured slower for the int8 block: 68.8 and 66.6 against 65.8 us).
+  // A box's shared-memory destination is box x row bytes into the stage, which a TMA
+  // load needs 128-byte aligned: 8 int8 rows and 2 bf16 rows always are (rows are
+  // multiples of 32 elements).
   const int esize = WQ8 ? 1 : 2;
-  if (EPI == EPI_PLAIN && a.nseg > 1 && a.ldw != a.Ks && a.Ks * esize < (WQ8 ? 4096 : 2048) &&
-      2 * pl.pairs >= 8) {
+  const int box = WQ8 ? 8 : 2;
+  if (EPI == EPI_PLAIN && a.nseg > 1 && a.ldw != a.Ks && a.Ks * esize <= (WQ8 ? 4095 : 2048) &&
+      ((size_t)box * a.Ks * esize) % 128 == 0 && 2 * pl.pairs >= 8) {
     int chunk = 0;
     for (int c : {256, 128, 64, 32, 16, 8})
       if (a.Ks % c == 0 && a.ldw % c == 0 && a.Ks / c <= 256 && c * esize >= 16) {
@@ -850,8 +858,8 @@ int launch_one(const GemvArgs& a, cudaStream_t s) {
         break;
       }
     if (chunk && make_tensor_map_rows(&wmap.m, a.w[0], (uint64_t)a.rows[0], (uint64_t)a.ldw, chunk,
-                                      a.Ks / chunk, 8, esize)) {
-      pl.map_box = 8;
+                                      a.Ks / chunk, box, esize)) {
+      pl.map_box = box;
       pl.map_nchunk = a.Ks / chunk;
     }
   }
