@@ -140,6 +140,40 @@ def test_block_small(tpb, shape, n, pos, quant):
                 name=f"d{shape.dim} H{shape.n_heads}/{shape.n_kv_heads} n{n} q{quant}")
 
 
+def test_block_q8_staging_near_ties(tpb):
+    """The FFN RMSNorm's Q8 codes where its values sit next to rounding ties (the codec's
+    exact-division fallback, in the staging of one preloaded row). With W_O zero the
+    attention branch adds nothing, so the FFN norm sees x itself. With x = 1, each 32-value
+    block has gain 1 (its maximum) and gains (k + 1/2) / 127, so the quotients by the block
+    scale land within a few ulp of k + 1/2. The codes and scales must match the oracle's Q8
+    of the kernel's own float32 row bit for bit. (The whole block is not held to the tight
+    bound here: the float64 oracle's own normalised row rounds many of these ties the other
+    way, so its FFN branch differs by a code step in many places; bf16 level is asserted.)"""
+    s = synth.BlockShape(**{**SMALL_MHA.__dict__, "batch": 1, "sync_quant": True})
+    inp = synth.block_inputs(4343, s)
+    inp.pos[:] = [150]
+    inp.wo = np.zeros_like(inp.wo)
+    inp.x = np.ones_like(inp.x)
+    g = np.empty(s.dim, dtype=np.float32)
+    for b0 in range(0, s.dim, 32):
+        g[b0] = 1.0
+        g[b0 + 1:b0 + 32] = (np.arange(31) % 20 + 0.5) / 127.0
+    inp.ffn_norm = g
+    tr = {}
+    ref = oracle.block_forward(inp, 2, True, trace=tr)[0]
+    y, _, _, bufs, err = run_block(tpb, inp, 2, 1)
+    assert err == 0, "a bounded wait in a kernel gave up"
+    D = s.dim
+    xn = np.asarray(bufs["xn"], dtype=np.float32)[:D].reshape(1, D)
+    q = xn / (np.abs(xn.reshape(-1, 32)).max(1) / np.float32(127)).repeat(32).reshape(1, D)
+    assert (np.abs(np.abs(q) - np.trunc(np.abs(q)) - 0.5) < 4e-5).sum() >= 200, "ties not reached"
+    r_xn, _ = report("ffn norm near ties xnorm(ffn)", xn, oracle.rmsnorm(tr["x1"], g, s.norm_eps))
+    assert r_xn <= TIGHT_Q8
+    assert_q8_codes_exact(bufs["xn"], bufs["xq"], bufs["xd"], 1, D, "ffn norm near ties xnorm(ffn)")
+    r_out, p_out = report("ffn norm near ties out", y, ref)
+    assert r_out <= BF16_TOL and p_out > 0.999
+
+
 @pytest.mark.parametrize("quant", [0, 1])
 def test_block_2d_ffn(tpb, quant):
     shape = synth.BlockShape(dim=512, n_heads=4, n_kv_heads=4, head_dim=128, ffn_dim=1024, vocab=0,
